@@ -1,0 +1,320 @@
+"""Plain, slow, obviously-correct CPU oracle for the QLoRA-adapted linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module.  The product library never calls it and shares no code, table or
+constant with it.
+
+What it computes, and where each step is defined:
+
+* NF4 level table -- "Low-Rank Adaptation (LoRA) and QLoRA: Mathematical
+  Foundations, Intrinsic Rank Dynamics, NF4 Quantization, and
+  Parameter-Efficient Fine-Tuning" (llms.blog), section "QLoRA: 4-Bit
+  NormalFloat and Memory Optimization", subsection "1. 4-bit NormalFloat (NF4)
+  Quantization", the q_i equation and the sentence on normalising to [-1, 1].
+* Block-wise absmax quantization (block 64) -- same subsection, steps 1-3;
+  block size from "Large Language Model Fine-tuning and LoRA"
+  (aicomputerinstitute.com), section "Quantizing the frozen weights: NF4 and
+  double quantization".
+* Double quantization (8-bit absmax, groups of 256, fp32 second level) --
+  Mathematical Foundations page, subsection "2. Double Quantization (DQ)",
+  the c1^{8bit} = round(c1/c2 * 127) equation; same section of the
+  Fine-tuning-and-LoRA page for the group size.
+* Forward h = W0 x + (alpha/r) B A x -- Mathematical Foundations page,
+  section "Intrinsic Dimensionality and Low-Rank Parameter Dynamics".
+* Gradients dB, dA, dx -- Mathematical Foundations page, section "Gradient
+  Dynamics and Backpropagation Mechanics" (all three equations, alpha/r kept).
+* Merge W_final = W0 + (alpha/r) B A -- Mathematical Foundations page,
+  section "Production Serving and Multi-Tenant Routing", "1. Static Weight
+  Merging"; "Large Language Model Fine-tuning and LoRA", section "Merging
+  adapters vs keeping them separate".
+* Multi-adapter forward (shared x W0, per-request B_i A_i) -- "Large Language
+  Model Fine-tuning and LoRA", section "Serving many adapters at once: the
+  multi-tenant problem".
+
+Where the pages are silent or garbled the oracle takes the readings listed as
+R1..R19 in the design notes; each is named where it is applied.
+
+Parity unpinned: the absolute NF4 code values and the double-quantization
+rounding order are conventions (R1, R5, R8, R10, R11) -- no page prints a
+worked NF4 example, so the tests pin their properties, not their bits.
+
+Row-major throughout: X[T, d_in], H[T, d_out], W0[d_out, d_in], A[r, d_in],
+B[d_out, r].  Floating-point arithmetic is fp64 except where the storage format
+fixes an fp32 decision (quantization codes, scale rebuild, decoded weight), in
+which case the IEEE fp32 operations are written out with numpy float32.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+BLOCK = 64          # weights per absmax block
+GROUP = 256         # absmax constants per second-level group
+Q8_MAX = 127        # 8-bit code range of the first-level constants
+
+# ----------------------------------------------------------------------------
+# NF4 level table (reading R1)
+# ----------------------------------------------------------------------------
+
+
+def normal_cdf(x: float) -> float:
+    """Standard normal CDF, Phi(x) = erfc(-x/sqrt 2)/2, from libm's erfc."""
+    return 0.5 * math.erfc(-x / math.sqrt(2.0))
+
+
+def normal_quantile(p: float) -> float:
+    """Q(p) = Phi^{-1}(p) by Newton's method on Phi(x) - p (fp64).
+
+    Newton from x = 0 converges monotonically on each side because Phi is
+    convex left of 0 and concave right of it; 200 steps is far more than the
+    handful needed for p in [1/18, 17/18].
+    """
+    if not 0.0 < p < 1.0:
+        raise ValueError("p must lie in (0, 1)")
+    x = 0.0
+    for _ in range(200):
+        pdf = math.exp(-0.5 * x * x) / math.sqrt(2.0 * math.pi)
+        step = (normal_cdf(x) - p) / pdf
+        x -= step
+        if abs(step) < 1e-17 * max(1.0, abs(x)):
+            break
+    return x
+
+
+def nf4_unnormalised_levels() -> np.ndarray:
+    """The 16 quantile midpoints before normalisation (fp64), reading R1.
+
+    The pages' q_i = (Q(i/2^k) + Q((i+1)/2^k)) / 2 is infinite for the two end
+    bins.  Reading R1 keeps the same construction on interior plotting
+    positions: edges p_j = j/18, j = 1..17, and q_i = (Q(p_{i+1}) + Q(p_{i+2}))/2
+    for i = 0..15 -- 16 equal-probability bins' quantile midpoints.
+    """
+    edges = [normal_quantile(j / 18.0) for j in range(1, 18)]
+    return np.array([0.5 * (edges[i] + edges[i + 1]) for i in range(16)],
+                    dtype=np.float64)
+
+
+def nf4_levels() -> np.ndarray:
+    """NF4 levels L[0..15] (fp32), normalised by max |q| to span [-1, 1]."""
+    q = nf4_unnormalised_levels()
+    return (q / np.max(np.abs(q))).astype(np.float32)
+
+
+def nf4_midpoints(levels: np.ndarray) -> np.ndarray:
+    """Decision thresholds m_i = fl32((L_i + L_{i+1}) / 2), computed in fp64 (R5)."""
+    L = levels.astype(np.float64)
+    return ((L[:-1] + L[1:]) / 2.0).astype(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# Sizes of the stored format
+# ----------------------------------------------------------------------------
+
+
+def nf4_sizes(d_out: int, d_in: int) -> tuple[int, int, int]:
+    """Byte sizes (codes, absmax_q, c2) for a [d_out, d_in] weight.
+
+    Two 4-bit codes per byte, one uint8 per 64-block, one fp32 per group of
+    256 blocks (the last group may be partial, reading R2).
+    """
+    if d_in % BLOCK:
+        raise ValueError("d_in must be a multiple of 64")
+    n = d_out * d_in
+    nblocks = n // BLOCK
+    ngroups = -(-nblocks // GROUP)
+    return n // 2, nblocks, 4 * ngroups
+
+
+# ----------------------------------------------------------------------------
+# Quantize / double-quantize / pack   (readings R2-R9)
+# ----------------------------------------------------------------------------
+
+
+def nf4_codes_of_normalised(xn: np.ndarray, mids: np.ndarray) -> np.ndarray:
+    """Nearest-level code of normalised values: #{i : x >= m_i} (R5, ties up)."""
+    return np.searchsorted(mids, xn, side="right").astype(np.uint8)
+
+
+def nf4_quantize(W: np.ndarray, levels: np.ndarray | None = None):
+    """Quantize fp32 W[d_out, d_in] -> (codes u8, absmax_q u8, c2 f32, c1 f32).
+
+    Steps, in the pages' order:
+      1. c1 = max |w| over each block of 64 consecutive row-major elements.
+      2. x~ = fl32(w / c1) (IEEE fp32 division; x~ = 0 when c1 = 0, R4).
+      3. code = nearest NF4 level (R5).
+      4. c2 = max of each group of 256 consecutive c1 (R7).
+      5. q8 = rint(fl32(fl32(c1 / c2) * 127)), clamped to [0, 127]; 0 if c2 = 0 (R6, R8).
+      6. Pack: element 2j in the low nibble of byte j, 2j+1 in the high nibble (R3).
+    c1 is returned too (it is not stored; tests use it for bounds).
+    """
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    d_out, d_in = W.shape
+    if d_in % BLOCK:
+        raise ValueError("d_in must be a multiple of 64")
+    L = nf4_levels() if levels is None else levels
+    mids = nf4_midpoints(L)
+
+    blocks = W.reshape(-1, BLOCK)                                   # R2
+    c1 = np.max(np.abs(blocks), axis=1).astype(np.float32)          # step 1
+    safe = np.where(c1 > 0, c1, np.float32(1.0)).astype(np.float32)
+    xn = (blocks / safe[:, None]).astype(np.float32)                # step 2 (fp32 /)
+    xn = np.where(c1[:, None] > 0, xn, np.float32(0.0)).astype(np.float32)
+    codes = nf4_codes_of_normalised(xn, mids).reshape(-1)          # step 3
+
+    nblocks = c1.shape[0]
+    ngroups = -(-nblocks // GROUP)
+    pad = ngroups * GROUP - nblocks
+    c1p = np.concatenate([c1, np.zeros(pad, np.float32)])
+    c2 = np.max(c1p.reshape(ngroups, GROUP), axis=1).astype(np.float32)  # step 4
+    c2_of_block = np.repeat(c2, GROUP)[:nblocks]
+    c2safe = np.where(c2_of_block > 0, c2_of_block, np.float32(1.0)).astype(np.float32)
+    ratio = (c1 / c2safe).astype(np.float32)                         # fl32(c1/c2)
+    scaled = (ratio * np.float32(Q8_MAX)).astype(np.float32)          # fl32(. * 127)
+    q8 = np.clip(np.rint(scaled), 0, Q8_MAX)                          # rint = half-even
+    q8 = np.where(c2_of_block > 0, q8, 0).astype(np.uint8)            # step 5
+
+    packed = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)     # step 6 (R3)
+    return packed.reshape(d_out, d_in // 2), q8, c2, c1
+
+
+def nf4_unpack(codes: np.ndarray) -> np.ndarray:
+    """Inverse of the packing: flat array of 4-bit codes in element order."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8).reshape(-1)
+    out = np.empty(c.size * 2, dtype=np.uint8)
+    out[0::2] = c & 0x0F
+    out[1::2] = c >> 4
+    return out
+
+
+def nf4_block_scales(absmax_q: np.ndarray, c2: np.ndarray) -> np.ndarray:
+    """Rebuilt block scale s_b = fl32(fl32(q8 * c2) / 127) (R10)."""
+    q8 = np.asarray(absmax_q, dtype=np.uint8).astype(np.float32)
+    c2b = np.repeat(np.asarray(c2, np.float32), GROUP)[: q8.size]
+    prod = (q8 * c2b).astype(np.float32)
+    return (prod / np.float32(Q8_MAX)).astype(np.float32)
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round fp32 values to bf16 (round-to-nearest-even), returned as fp32.
+
+    The plain definition on the bit pattern: add 0x7FFF plus the lowest kept
+    bit, then truncate the low 16 bits.  (No NaN/Inf ever reaches it here.)
+    """
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32)
+
+
+def nf4_dequantize(codes, absmax_q, c2, d_out: int, d_in: int,
+                   out: str = "f32", levels: np.ndarray | None = None) -> np.ndarray:
+    """Decoded weight W^[d_out, d_in] (R11).
+
+    w32 = fl32(L[code] * s_b); out="bf16" returns RN-even bf16 of w32 (as fp32
+    values), out="f32" returns w32.
+    """
+    L = nf4_levels() if levels is None else levels
+    cf = nf4_unpack(codes)[: d_out * d_in]
+    s = nf4_block_scales(absmax_q, c2)
+    w32 = (L[cf].reshape(-1, BLOCK) * s[:, None]).astype(np.float32).reshape(d_out, d_in)
+    if out == "f32":
+        return w32
+    if out == "bf16":
+        return bf16_round(w32)
+    raise ValueError(out)
+
+
+# ----------------------------------------------------------------------------
+# LoRA forward / backward / merge in fp64
+# ----------------------------------------------------------------------------
+
+
+def lora_scale(alpha: float, r: int) -> float:
+    """s = alpha / r (fp64)."""
+    return float(alpha) / float(r)
+
+
+def lora_forward(W_hat, X, A, B, alpha, r):
+    """H = X W^T + s (X A^T) B^T: the batched row form of h = W0 x + (alpha/r) B A x."""
+    W_hat, X, A, B = (np.asarray(t, np.float64) for t in (W_hat, X, A, B))
+    s = lora_scale(alpha, r)
+    U = X @ A.T
+    return X @ W_hat.T + s * (U @ B.T)
+
+
+def lora_backward(W_hat, X, dH, A, B, alpha, r):
+    """(dX, dA, dB) for upstream gradient dH[T, d_out].
+
+    Row form of the page's three equations, summed over the T tokens:
+      dB = s dH^T (X A^T),   dA = s B^T dH^T X = s (dH B)^T X,
+      dX = dH (W0 + s B A)  = dH W^ + s (dH B) A            (R12, R13).
+    """
+    W_hat, X, dH, A, B = (np.asarray(t, np.float64) for t in (W_hat, X, dH, A, B))
+    s = lora_scale(alpha, r)
+    U = X @ A.T
+    G = dH @ B
+    dX = dH @ W_hat + s * (G @ A)
+    dA = s * (G.T @ X)
+    dB = s * (dH.T @ U)
+    return dX, dA, dB
+
+
+def lora_merge(W_hat, A, B, alpha, r):
+    """W_final = W^ + s B A (dense; not re-quantized, R17)."""
+    W_hat, A, B = (np.asarray(t, np.float64) for t in (W_hat, A, B))
+    return W_hat + lora_scale(alpha, r) * (B @ A)
+
+
+def lora_forward_batched(W_hat, X, adapter_id, As, Bs, alphas, ranks):
+    """Multi-adapter forward over one shared base (R18).
+
+    The shared base term X W^T is computed once for the whole batch; each token
+    t then adds its own adapter's correction s_i (x_t A_i^T) B_i^T.  An id
+    outside [0, n) is an error.
+    """
+    W_hat = np.asarray(W_hat, np.float64)
+    X = np.asarray(X, np.float64)
+    ids = np.asarray(adapter_id).reshape(-1)
+    n = len(As)
+    if ids.size and (ids.min() < 0 or ids.max() >= n):
+        raise ValueError("adapter id out of range")
+    H = X @ W_hat.T
+    for t in range(X.shape[0]):
+        i = int(ids[t])
+        A = np.asarray(As[i], np.float64)
+        B = np.asarray(Bs[i], np.float64)
+        H[t] += lora_scale(alphas[i], ranks[i]) * ((X[t] @ A.T) @ B.T)
+    return H
+
+
+# ----------------------------------------------------------------------------
+# Counting formulas printed on the pages
+# ----------------------------------------------------------------------------
+
+
+def trainable_params(d_out: int, d_in: int, r: int) -> int:
+    """r (d_in + d_out): r d_out for B plus r d_in for A ("Choosing what to adapt")."""
+    return r * (d_in + d_out)
+
+
+def merge_flops(d_out: int, d_in: int, r: int) -> int:
+    """2 d_out r d_in: cost of B @ A ("Merging adapters vs keeping them separate")."""
+    return 2 * d_out * r * d_in
+
+
+def storage_bits_per_param(d_out: int, d_in: int) -> float:
+    """Stored bits per weight of the double-quantized format."""
+    a, b, c = nf4_sizes(d_out, d_in)
+    return 8.0 * (a + b + c) / (d_out * d_in)
+
+
+def fwd_flops(T, d_out, d_in, r):
+    """Algorithmic forward FLOPs: 2 T d k + 2 T r (d + k)."""
+    return 2 * T * d_out * d_in + 2 * T * r * (d_out + d_in)
+
+
+def bwd_flops(T, d_out, d_in, r):
+    """Algorithmic backward FLOPs: 2 T d k + 4 T r (d + k) (U reused)."""
+    return 2 * T * d_out * d_in + 4 * T * r * (d_out + d_in)

@@ -1,0 +1,340 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+None of these calls the CUDA path.  Each pin is chosen so that a plausible
+mistake in the oracle (a dropped alpha/r, a transposed operand, a wrong sign,
+swapped nibbles, the wrong rounding rule, 255 for 127) fails at least one of
+them; ``test_pins_catch_planted_mistakes`` plants such mistakes in copies of
+the oracle functions and checks that the pins reject them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special as sp
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_numbers.json")
+
+
+def rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+# ---------------------------------------------------------------- NF4 table
+
+
+def test_levels_shape_symmetry_range():
+    L = O.nf4_levels()
+    assert L.dtype == np.float32 and L.shape == (16,)
+    assert np.all(np.diff(L) > 0)                      # strictly increasing
+    assert L[0] == -1.0 and L[15] == 1.0               # normalised to [-1, 1]
+    assert np.array_equal(L, -L[::-1])                 # symmetric quantiles
+
+
+def test_levels_against_independent_quantile():
+    # Re-derive every level with scipy's ndtri (an independent inverse CDF).
+    edges = [sp.ndtri(j / 18.0) for j in range(1, 18)]
+    q = np.array([0.5 * (edges[i] + edges[i + 1]) for i in range(16)])
+    assert np.max(np.abs(O.nf4_unnormalised_levels() - q)) < 1e-12
+    assert np.array_equal(O.nf4_levels(), (q / np.max(np.abs(q))).astype(np.float32))
+
+
+def test_levels_equal_probability_bins():
+    # The bins whose quantile midpoints give the levels each hold 1/18 of N(0,1).
+    edges = [O.normal_quantile(j / 18.0) for j in range(1, 18)]
+    for j, e in enumerate(edges, start=1):
+        assert abs(sp.ndtr(e) - j / 18.0) < 1e-14
+    probs = np.diff([sp.ndtr(e) for e in edges])
+    assert np.allclose(probs, 1.0 / 18.0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- quantize
+
+
+def brute_force_codes(xn, L):
+    """Nearest level by exhaustive fp64 search; ties to the upper level."""
+    d = np.abs(xn.astype(np.float64)[:, None] - L.astype(np.float64)[None, :])
+    best = d.min(axis=1, keepdims=True)
+    cand = np.where(d == best, np.arange(16)[None, :], -1)
+    return cand.max(axis=1), np.sort(d, axis=1)
+
+
+def test_codes_are_nearest_level():
+    rng = np.random.default_rng(1)
+    W = (rng.standard_normal((32, 256)) * 0.141).astype(np.float32)
+    codes, q8, c2, c1 = O.nf4_quantize(W)
+    L = O.nf4_levels()
+    xn = (W.reshape(-1, 64) / c1[:, None]).astype(np.float32).reshape(-1)
+    bf, dsorted = brute_force_codes(xn, L)
+    got = O.nf4_unpack(codes)
+    # Only values within rounding of a midpoint may legitimately differ.
+    clear = (dsorted[:, 1] - dsorted[:, 0]) > 1e-6
+    assert clear.mean() > 0.999
+    assert np.array_equal(got[clear], bf[clear])
+
+
+def test_zero_ties_up_and_zero_block():
+    W = np.zeros((1, 128), np.float32)
+    W[0, 0] = 1.0                         # block 0: max 1, zeros elsewhere
+    W[0, 1] = -0.0
+    codes, q8, c2, c1 = O.nf4_quantize(W)
+    c = O.nf4_unpack(codes)
+    assert c[1] == 8 and c[2] == 8        # 0 and -0 tie between L7, L8 -> upper
+    assert c[0] == 15
+    assert np.all(c[64:] == 8)            # all-zero block (c1 = 0) -> x~ = 0
+    assert c1[1] == 0 and q8[1] == 0
+
+
+def test_round_trip_of_levels_and_nibble_order():
+    # A block holding c * L_j plus one +-c entry quantizes to codes j and, with
+    # c a power of two (so every product is exact), decodes to c * L_j.
+    L = O.nf4_levels()
+    rng = np.random.default_rng(2)
+    c = np.float32(0.25)
+    j = rng.integers(0, 16, size=(8, 64))
+    j[:, 0] = 15                          # guarantees max |w| = c
+    W = (L[j] * c).astype(np.float32)
+    codes, q8, c2, c1 = O.nf4_quantize(W.reshape(8, 64))
+    assert np.array_equal(O.nf4_unpack(codes).reshape(8, 64), j)
+    # element 2i is the low nibble of byte i
+    assert np.array_equal(codes.reshape(-1) & 0xF, j.reshape(-1)[0::2])
+    assert np.all(q8 == 127) and np.all(c2 == c)
+    w = O.nf4_dequantize(codes, q8, c2, 8, 64)
+    assert np.array_equal(w, W)
+
+
+def test_double_quant_range_and_scale_error():
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((64, 1024)) * 0.141).astype(np.float32)
+    W[5] *= 40.0                          # a few large blocks
+    codes, q8, c2, c1 = O.nf4_quantize(W)
+    assert q8.dtype == np.uint8 and q8.max() <= 127
+    nb = c1.size
+    for g in range(c2.size):
+        blk = c1[g * 256:(g + 1) * 256]
+        assert c2[g] == blk.max()
+        assert q8[g * 256 + int(np.argmax(blk))] == 127
+    s = O.nf4_block_scales(q8, c2).astype(np.float64)
+    c2b = np.repeat(c2, 256)[:nb].astype(np.float64)
+    # 8-bit linear code of c1/c2: error at most half a step (c2/254) + fp32 rounding.
+    assert np.all(np.abs(s - c1) <= c2b / 254.0 * (1 + 1e-5) + 1e-12)
+
+
+def test_elementwise_error_bound():
+    rng = np.random.default_rng(4)
+    W = (rng.standard_normal((16, 512)) * 0.141).astype(np.float32)
+    codes, q8, c2, c1 = O.nf4_quantize(W)
+    w = O.nf4_dequantize(codes, q8, c2, 16, 512).astype(np.float64)
+    L = O.nf4_levels().astype(np.float64)
+    half_gap = np.max(np.diff(L)) / 2.0
+    s = O.nf4_block_scales(q8, c2).astype(np.float64)
+    c1b = np.repeat(c1.astype(np.float64), 64)
+    sb = np.repeat(s, 64)
+    bound = c1b * (half_gap + 2.0 ** -22) + np.abs(c1b - sb) + 2.0 ** -23 * np.abs(w.reshape(-1))
+    assert np.all(np.abs(W.reshape(-1) - w.reshape(-1)) <= bound)
+
+
+def test_bf16_rounding_definition():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -1.0 - 2 ** -8,
+                  3.0e-3, 65504.0], np.float32)
+    import torch
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
+    assert np.array_equal(O.bf16_round(x), ref)
+    # halfway cases go to even
+    assert O.bf16_round(np.array([1.0 + 2 ** -8], np.float32))[0] == 1.0
+    assert O.bf16_round(np.array([1.0 + 3 * 2 ** -8], np.float32))[0] == 1.0 + 2 ** -6
+
+
+# ---------------------------------------------------------------- storage rate
+
+
+def test_storage_rate_matches_pages():
+    g = json.load(open(GOLDEN))["storage"]
+    a, b, c = O.nf4_sizes(4096, 4096)
+    assert (a, b, c) == (4096 * 4096 // 2, 4096 * 4096 // 64, 4 * 1024)
+    bits = O.storage_bits_per_param(4096, 4096)
+    assert abs(bits - 4.126953125) < 1e-12
+    assert round(bits, 3) == g["double_quant_bits"]
+    assert round(4 + 32 / 64, 3) == g["single_level_bits"]
+    assert round(g["single_level_bits"] - bits, 3) == g["saving_bits"]
+    assert round(bits / 8, 4) == g["bytes_per_param"]
+    assert round(bits - 4, 3) == g["dq_overhead_bits"]
+    assert round(7e9 * bits / 8 / 1e9, 2) == g["gb_7b_base"]
+    # a partial last group still costs one fp32 constant
+    assert O.nf4_sizes(3, 128)[2] == 4
+
+
+# ---------------------------------------------------------------- counting
+
+
+def test_parameter_counts_and_calculator():
+    g = json.load(open(GOLDEN))
+    for e in g["trainable_params"]:
+        assert O.trainable_params(e["d_out"], e["d_in"], e["r"]) == e["value"]
+    c = g["calculator_output"]
+    base = sum(O.trainable_params(d, k, c["baseline_rank"]) for d, k in c["baseline_targets"]) * c["layers"]
+    exp = sum(O.trainable_params(d, k, c["expanded_rank"]) for d, k in c["expanded_targets"]) * c["layers"]
+    assert (base, exp, exp / base) == (c["baseline"], c["expanded"], c["ratio"])
+    v = g["v_proj_only"]
+    assert O.trainable_params(4096, 4096, v["r"]) * v["layers"] == v["value"]
+
+
+def test_merge_flops():
+    g = json.load(open(GOLDEN))["merge_flops"]
+    assert O.merge_flops(4096, 4096, 8) == g[0]["value"]
+    base = 2 * O.merge_flops(4096, 4096, 8) * 32
+    exp = (3 * O.merge_flops(4096, 4096, 16) + O.merge_flops(4096, 11008, 16)) * 32
+    assert round(base / 1e9, 2) == g[1]["total_gflop_baseline"]
+    assert round(exp / 1e9, 2) == g[1]["total_gflop_expanded"]
+
+
+# ---------------------------------------------------------------- LoRA algebra
+
+
+def small_layer(d=8, k=8, r=2, T=3, seed=5):
+    rng = np.random.default_rng(seed)
+    W = rng.standard_normal((d, k))
+    X = rng.standard_normal((T, k))
+    A = rng.standard_normal((r, k))
+    B = rng.standard_normal((d, r))
+    dH = rng.standard_normal((T, d))
+    return W, X, A, B, dH
+
+
+def check_init_invariant(fwd):
+    W, X, A, B, dH = small_layer(d=12, k=10, r=3, T=4)
+    H0 = fwd(W, X, A, np.zeros_like(B), 6.0, 3)
+    return np.array_equal(H0, X @ W.T)
+
+
+def check_forward_brute(fwd):
+    W, X, A, B, dH = small_layer(d=6, k=5, r=2, T=3)
+    alpha, r = 3.0, 2
+    H = fwd(W, X, A, B, alpha, r)
+    ref = np.zeros((3, 6))
+    for t in range(3):
+        for i in range(6):
+            acc = 0.0
+            for j in range(5):
+                acc += W[i, j] * X[t, j]
+            for q in range(r):
+                ax = 0.0
+                for j in range(5):
+                    ax += A[q, j] * X[t, j]
+                acc += (alpha / r) * B[i, q] * ax
+            ref[t, i] = acc
+    return rel(H, ref)
+
+
+def check_gradients_fd(fwd, bwd):
+    """Central differences of L = <dH, H>; exact up to rounding (L is linear
+    in each single entry of X, A and B)."""
+    W, X, A, B, dH = small_layer()
+    alpha, r = 5.0, 2
+    dX, dA, dB = bwd(W, X, dH, A, B, alpha, r)
+    worst = 0.0
+    for name, P, G in (("X", X, dX), ("A", A, dA), ("B", B, dB)):
+        num = np.zeros_like(P)
+        for idx in np.ndindex(P.shape):
+            h = 0.5
+            orig = P[idx]
+            P[idx] = orig + h
+            lp = np.sum(dH * fwd(W, X, A, B, alpha, r))
+            P[idx] = orig - h
+            lm = np.sum(dH * fwd(W, X, A, B, alpha, r))
+            P[idx] = orig
+            num[idx] = (lp - lm) / (2 * h)
+        worst = max(worst, rel(G, num))
+    return worst
+
+
+def check_merge(fwd, merge):
+    W, X, A, B, dH = small_layer(d=9, k=7, r=3, T=5)
+    Wf = merge(W, A, B, 6.0, 3)
+    return rel(X @ Wf.T, fwd(W, X, A, B, 6.0, 3))
+
+
+def test_init_invariant_B_zero():
+    assert check_init_invariant(O.lora_forward)
+
+
+def test_forward_against_loops():
+    assert check_forward_brute(O.lora_forward) < 1e-13
+
+
+def test_gradients_finite_differences():
+    assert check_gradients_fd(O.lora_forward, O.lora_backward) < 1e-11
+
+
+def test_merge_reproduces_unmerged_output():
+    assert check_merge(O.lora_forward, O.lora_merge) < 1e-12
+
+
+def test_batched_matches_per_adapter():
+    rng = np.random.default_rng(6)
+    d, k, T = 10, 12, 9
+    ranks = [1, 2, 4]
+    W = rng.standard_normal((d, k))
+    X = rng.standard_normal((T, k))
+    As = [rng.standard_normal((r, k)) for r in ranks]
+    Bs = [rng.standard_normal((d, r)) for r in ranks]
+    alphas = [2.0 * r for r in ranks]
+    ids = rng.integers(0, 3, size=T)
+    H = O.lora_forward_batched(W, X, ids, As, Bs, alphas, ranks)
+    for i in range(3):
+        sel = ids == i
+        if sel.any():
+            ref = O.lora_forward(W, X[sel], As[i], Bs[i], alphas[i], ranks[i])
+            assert rel(H[sel], ref) < 1e-13
+    with pytest.raises(ValueError):
+        O.lora_forward_batched(W, X, np.full(T, 3), As, Bs, alphas, ranks)
+
+
+# ---------------------------------------------------------------- mutants
+
+
+def test_pins_catch_planted_mistakes():
+    s = O.lora_scale
+
+    def fwd_sign(W, X, A, B, a, r):
+        return np.asarray(X) @ np.asarray(W).T - s(a, r) * ((X @ A.T) @ B.T)
+
+    def fwd_noscale(W, X, A, B, a, r):
+        return X @ W.T + (X @ A.T) @ B.T
+
+    def bwd_no_scale_dA(W, X, dH, A, B, a, r):
+        dX, dA, dB = O.lora_backward(W, X, dH, A, B, a, r)
+        return dX, dA / s(a, r), dB
+
+    def bwd_dx_no_adapter(W, X, dH, A, B, a, r):
+        dX, dA, dB = O.lora_backward(W, X, dH, A, B, a, r)
+        return dH @ W, dA, dB
+
+    def bwd_transposed_W(W, X, dH, A, B, a, r):
+        dX, dA, dB = O.lora_backward(W, X, dH, A, B, a, r)
+        return dX - dH @ W + dH @ W.T, dA, dB        # square case: W vs W^T
+
+    def merge_noscale(W, A, B, a, r):
+        return W + B @ A
+
+    assert check_forward_brute(fwd_sign) > 1e-3
+    assert check_forward_brute(fwd_noscale) > 1e-3
+    assert check_gradients_fd(O.lora_forward, bwd_no_scale_dA) > 1e-3
+    assert check_gradients_fd(O.lora_forward, bwd_dx_no_adapter) > 1e-3
+    assert check_gradients_fd(O.lora_forward, bwd_transposed_W) > 1e-3
+    assert check_merge(O.lora_forward, merge_noscale) > 1e-3
+
+    # quantizer mutants: swapped nibbles and a 255-level second stage
+    L = O.nf4_levels()
+    j = np.arange(64) % 16
+    j[0] = 15
+    W = (L[j] * np.float32(0.5)).astype(np.float32).reshape(1, 64)
+    codes, q8, c2, c1 = O.nf4_quantize(W)
+    swapped = ((codes >> 4) | (codes << 4)).astype(np.uint8)
+    assert not np.array_equal(O.nf4_unpack(swapped).reshape(1, 64), j.reshape(1, 64))
+    assert int(np.rint(np.float32(1.0) * np.float32(255))) != int(q8.max())
