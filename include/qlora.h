@@ -1,0 +1,176 @@
+/*
+ * qlora.h -- C ABI of libqlora: the QLoRA-adapted linear layer on NVIDIA B200 (sm_100a).
+ *
+ * The frozen base weight W0[d_out, d_in] is stored as 4-bit NormalFloat codes in blocks of
+ * 64 weights, each block's absmax double-quantized to uint8 in groups of 256 blocks with one
+ * fp32 second-level constant per group.  The layer computes
+ *     h = W0 x + (alpha/r) B (A x)
+ * with W0 dequantized on the fly to bf16 inside the tensor-core GEMM, its backward pass, the
+ * adapter merge, and a multi-adapter forward over one shared base.
+ *
+ * Sources of each definition (page title, then section):
+ *  [MF]  "Low-Rank Adaptation (LoRA) and QLoRA: Mathematical Foundations, Intrinsic Rank
+ *        Dynamics, NF4 Quantization, and Parameter-Efficient Fine-Tuning" (llms.blog)
+ *  [CH]  "Large Language Model Fine-tuning and LoRA" (aicomputerinstitute.com)
+ *  [UH]  "LoRA and QLoRA Fine-Tuning Under the Hood" (codingpancake.com)
+ *  [L26] "Lesson 26: LoRA/QLoRA Theory" (teology.holyping.network)
+ *
+ * Conventions for every entry point
+ *  - Layout: row-major, contiguous.  X[T, d_in], H[T, d_out], dH[T, d_out], dX[T, d_in],
+ *    A[r, d_in], B[d_out, r], dA[r, d_in], dB[d_out, r].
+ *  - Memory: every tensor argument is caller-allocated DEVICE memory unless marked "host";
+ *    the library never allocates or frees device memory and never synchronises the host,
+ *    except qlora_get_device_error().  All work is enqueued on the given stream.
+ *  - Alignment: device pointers must be 16-byte aligned, else QLORA_ERR_INVALID_ARG.
+ *  - Shapes: d_in % 64 == 0 (a block never straddles rows), d_out % 8 == 0, T >= 1,
+ *    1 <= r <= 128; otherwise QLORA_ERR_UNSUPPORTED.  Ragged tiles in T, d_out, d_in are handled.
+ *  - dtype: QLORA_BF16 or QLORA_F32 sets X, H, dH, dX, A and B.  dA and dB are always fp32 and
+ *    are overwritten (not accumulated).  The fp32 path is exact fp32 arithmetic (no TF32).
+ *  - Errors found on the host return at once and nothing is launched.  Errors found on the
+ *    device (an adapter id out of range, a pipeline wait that ran past its time limit) set a
+ *    device error word that the next qlora_get_device_error() returns and clears.
+ *  - Workspace: calls that take (ws, ws_bytes) need at least qlora_workspace_bytes(...) bytes
+ *    of device scratch, 256-byte aligned; contents need not be initialised and are clobbered.
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QLORA_OK = 0,
+    QLORA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad dtype, short workspace */
+    QLORA_ERR_UNSUPPORTED = 2,   /* shape outside the supported set (see conventions)    */
+    QLORA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed                    */
+    QLORA_ERR_TIMEOUT = 4,       /* a device pipeline wait exceeded its time limit       */
+    QLORA_ERR_DEVICE = 5         /* device-detected bad input (adapter id out of range)  */
+} qlora_status;
+
+typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
+
+typedef enum {
+    QLORA_OP_FWD = 0, QLORA_OP_BWD = 1, QLORA_OP_FWD_BATCHED = 2, QLORA_OP_MERGE = 3
+} qlora_op;
+
+/* Stored NF4 weight.  Block size 64 and group size 256 are fixed.
+ *   codes    [d_out, d_in/2] bytes: element 2j in the low nibble of byte j, 2j+1 in the high.
+ *   absmax_q [d_out*d_in/64] uint8: q8 = rint(fl32(fl32(c1/c2)*127)), c1 = block absmax.
+ *   c2       [ceil(d_out*d_in/64/256)] fp32: max of each group of 256 consecutive c1.
+ * Blocks are 64 consecutive row-major elements; groups are 256 consecutive blocks.
+ * [MF] "QLoRA: 4-Bit NormalFloat and Memory Optimization", "1. 4-bit NormalFloat (NF4)
+ * Quantization" and "2. Double Quantization (DQ)"; [CH] "Quantizing the frozen weights: NF4
+ * and double quantization" (block 64, 256 constants per second-level block).                */
+typedef struct {
+    const uint8_t* codes;
+    const uint8_t* absmax_q;
+    const float*   c2;
+    int64_t        d_out;
+    int64_t        d_in;
+} qlora_nf4;
+
+/* Byte sizes of the three NF4 buffers for a [d_out, d_in] weight (host-only, no GPU call).
+ * d_out*d_in/2, d_out*d_in/64 and 4*ceil(d_out*d_in/16384): 4.127 bits per weight as in
+ * [CH] "Quantizing the frozen weights".  UNSUPPORTED if d_in % 64 != 0.                       */
+qlora_status qlora_nf4_sizes(int64_t d_out, int64_t d_in,
+                             size_t* codes_bytes, size_t* absmax_bytes, size_t* c2_bytes);
+
+/* The 16 NF4 levels L[0..15] the kernels decode with (host copy, no GPU call): quantile
+ * midpoints of 16 equal-probability bins of N(0,1), normalised to [-1, 1]
+ * ([MF] "1. 4-bit NormalFloat (NF4) Quantization", q_i equation).  out: host float[16].   */
+qlora_status qlora_nf4_levels(float* out);
+
+/* Quantize W[d_out, d_in] (fp32 or bf16, device) into the NF4 + double-quant format.
+ * Per block: c1 = max|w|, x = fl32(w/c1), code = nearest level (ties to the upper level);
+ * per group: c2 = max c1, q8 as above.  Bit-exact, deterministic.
+ * [MF] "1. 4-bit NormalFloat (NF4) Quantization" steps 1-3 and "2. Double Quantization (DQ)".
+ * Outputs are device buffers of the sizes from qlora_nf4_sizes().                            */
+qlora_status nf4_quantize(const void* W, qlora_dtype w_dtype, int64_t d_out, int64_t d_in,
+                          uint8_t* codes, uint8_t* absmax_q, float* c2, cudaStream_t stream);
+
+/* Decode the stored weight to W_out[d_out, d_in] (device): fp32 w = fl32(L[code] * s_b) with
+ * s_b = fl32(fl32(q8*c2)/127); bf16 output is the round-to-nearest-even of that fp32 value.
+ * Bit-exact.  [MF] "1. 4-bit NormalFloat (NF4) Quantization" (dequantized to BF16 before the
+ * matrix multiplication); [CH] "Quantizing the frozen weights" (compute in bf16).           */
+qlora_status nf4_dequantize(const qlora_nf4* w, void* W_out, qlora_dtype out_dtype,
+                            cudaStream_t stream);
+
+/* Scratch bytes needed by an operation (host-only).  op is a qlora_op, dtype the call's dtype;
+ * r_total is r for the single-adapter calls and the sum of ranks for QLORA_OP_FWD_BATCHED.
+ * Returns 0 for an unsupported combination.                                                  */
+size_t qlora_workspace_bytes(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in,
+                             int32_t r_total);
+
+/* Forward: H = X W^T + (alpha/r) (X A^T) B^T, with W = the decoded weight (bf16 when dtype is
+ * QLORA_BF16, fp32 when QLORA_F32).  [MF] "Intrinsic Dimensionality and Low-Rank Parameter
+ * Dynamics" (h = W0 x + (alpha/r) B A x); [L26] "2. LoRA", "The Decomposition".
+ *   X [T, d_in], A [r, d_in], B [d_out, r] in dtype; H [T, d_out] out in dtype.
+ *   U_save (nullable) [T, r] in dtype receives U = X A^T (unscaled) for the backward call.   */
+qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T,
+                              const void* A, const void* B, int32_t r, float alpha,
+                              qlora_dtype dtype, void* H, void* U_save,
+                              void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Backward for upstream dH[T, d_out]:
+ *   dX = dH W + s (dH B) A,   dA = s (dH B)^T X,   dB = s dH^T (X A^T),   s = alpha/r.
+ * [MF] "Gradient Dynamics and Backpropagation Mechanics" (all three equations, alpha/r kept);
+ * W0 is read only by the dX GEMM and no dW0 is formed ([MF], same section; [CH] "Correcting a
+ * common misconception").  U_saved (nullable) is the U from the forward call, else it is
+ * recomputed.  dX (nullable: skipped) in dtype; dA [r, d_in], dB [d_out, r] fp32.            */
+qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                              const void* A, const void* B, int32_t r, float alpha,
+                              const void* U_saved, qlora_dtype dtype, void* dX,
+                              float* dA, float* dB, void* ws, size_t ws_bytes,
+                              cudaStream_t stream);
+
+/* Merge: W_final = W + (alpha/r) B A, dense (not re-quantized), out_dtype fp32 or bf16;
+ * W is the decoded weight in out_dtype's decode.  A, B are given in adapter_dtype.
+ * [MF] "Production Serving and Multi-Tenant Routing", "1. Static Weight Merging";
+ * [CH] "Merging adapters vs keeping them separate".                                          */
+qlora_status lora_merge(const qlora_nf4* w, const void* A, const void* B, int32_t r,
+                        float alpha, qlora_dtype adapter_dtype, qlora_dtype out_dtype,
+                        void* W_final, cudaStream_t stream);
+
+/* Multi-adapter forward over one shared base:
+ *   H[t] = X[t] W^T + s_i (X[t] A_i^T) B_i^T,  i = adapter_id[t],  s_i = alpha[i]/r[i].
+ * The base GEMM is shared by all tokens.  [CH] "Serving many adapters at once: the
+ * multi-tenant problem"; [MF] "2. Multi-Tenant Dynamic Multiplexing"; [UH] "6.2 Multi-Adapter
+ * Serving at Scale".  adapter_id: device int32[T]; A, B: HOST arrays of n_adapters device
+ * pointers (A_i [r_i, d_in], B_i [d_out, r_i]); r, alpha: HOST arrays.  sum(r) <= 128,
+ * n_adapters <= 32.  An id outside [0, n_adapters) contributes no adapter term for that token
+ * and sets QLORA_ERR_DEVICE in the device error word.                                         */
+qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t T,
+                                      const int32_t* adapter_id, int32_t n_adapters,
+                                      const void* const* A, const void* const* B,
+                                      const int32_t* r, const float* alpha, qlora_dtype dtype,
+                                      void* H, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Synchronise `stream`, then read and clear the device error word of the current device.
+ * Returns QLORA_OK, QLORA_ERR_TIMEOUT, QLORA_ERR_DEVICE or QLORA_ERR_CUDA.                   */
+qlora_status qlora_get_device_error(cudaStream_t stream);
+
+/* Self-test of the bounded pipeline wait: launches one block that waits on a shared-memory
+ * barrier nothing ever arrives on, for at most limit_ns nanoseconds, then gives up and sets
+ * QLORA_ERR_TIMEOUT in the device error word.  The context stays usable.                     */
+qlora_status qlora_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
+/* Benchmark instrumentation: while both events are non-NULL, every launch of the fused NF4
+ * GEMM kernel (forward or dX) records `start` right before and `stop` right after itself on
+ * the call's stream.  Pass NULL, NULL to stop.  Not thread-safe.                             */
+qlora_status qlora_set_gemm_events(cudaEvent_t start, cudaEvent_t stop);
+
+/* Number of kernels this library has launched since it was loaded (all entry points). */
+uint64_t qlora_launch_count(void);
+
+/* Human-readable name of a status code (static string). */
+const char* qlora_status_string(qlora_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_H_ */

@@ -253,12 +253,19 @@ def lora_backward(W_hat, X, dH, A, B, alpha, r):
     """
     W_hat, X, dH, A, B = (np.asarray(t, np.float64) for t in (W_hat, X, dH, A, B))
     s = lora_scale(alpha, r)
-    U = X @ A.T
     G = dH @ B
     dX = dH @ W_hat + s * (G @ A)
-    dA = s * (G.T @ X)
-    dB = s * (dH.T @ U)
+    dA, dB = lora_adapter_grads(X, dH, A, B, alpha, r)
     return dX, dA, dB
+
+
+def lora_adapter_grads(X, dH, A, B, alpha, r):
+    """(dA, dB) alone: dA = s (dH B)^T X, dB = s dH^T (X A^T) (same section as above)."""
+    X, dH, A, B = (np.asarray(t, np.float64) for t in (X, dH, A, B))
+    s = lora_scale(alpha, r)
+    U = X @ A.T
+    G = dH @ B
+    return s * (G.T @ X), s * (dH.T @ U)
 
 
 def lora_merge(W_hat, A, B, alpha, r):

@@ -1,0 +1,277 @@
+"""Python binding of libqlora, the B200 (sm_100a) QLoRA-adapted linear layer.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels of
+``libqlora.so`` behind the C ABI declared in ``include/qlora.h``.  PyTorch
+provides device memory and streams.  There is no CPU fallback: if the library
+is missing or a call fails, an exception is raised.
+
+Names follow the C ABI: ``nf4_quantize``, ``nf4_dequantize``,
+``qlora_linear_fwd``, ``qlora_linear_bwd``, ``lora_merge``,
+``qlora_linear_fwd_batched``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libqlora.so")
+
+QLORA_OK = 0
+STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",
+          3: "QLORA_ERR_CUDA", 4: "QLORA_ERR_TIMEOUT", 5: "QLORA_ERR_DEVICE"}
+F32, BF16 = 0, 1
+OP_FWD, OP_BWD, OP_FWD_BATCHED, OP_MERGE = 0, 1, 2, 3
+
+# Every symbol include/qlora.h declares.
+EXPORTS = ["qlora_nf4_sizes", "qlora_nf4_levels", "nf4_quantize", "nf4_dequantize",
+           "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "lora_merge",
+           "qlora_linear_fwd_batched", "qlora_get_device_error",
+           "qlora_selftest_wait_timeout", "qlora_set_gemm_events", "qlora_launch_count",
+           "qlora_status_string"]
+
+
+class QloraError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class _NF4(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("absmax_q", ctypes.c_void_p),
+                ("c2", ctypes.c_void_p), ("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libqlora.so (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m qlora_parameter_efficient_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    pnf4 = ctypes.POINTER(_NF4)
+    sig = {
+        "qlora_nf4_sizes": ([i64, i64, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)], ctypes.c_int),
+        "qlora_nf4_levels": ([ctypes.POINTER(ctypes.c_float)], ctypes.c_int),
+        "nf4_quantize": ([vp, ctypes.c_int, i64, i64, vp, vp, vp, vp], ctypes.c_int),
+        "nf4_dequantize": ([pnf4, vp, ctypes.c_int, vp], ctypes.c_int),
+        "qlora_workspace_bytes": ([ctypes.c_int, ctypes.c_int, i64, i64, i64, i32], sz),
+        "qlora_linear_fwd": ([pnf4, vp, i64, vp, vp, i32, f32, ctypes.c_int, vp, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_linear_bwd": ([pnf4, vp, vp, i64, vp, vp, i32, f32, vp, ctypes.c_int, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "lora_merge": ([pnf4, vp, vp, i32, f32, ctypes.c_int, ctypes.c_int, vp, vp], ctypes.c_int),
+        "qlora_linear_fwd_batched": ([pnf4, vp, i64, vp, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                      ctypes.POINTER(i32), ctypes.POINTER(f32), ctypes.c_int, vp, vp, sz, vp],
+                                     ctypes.c_int),
+        "qlora_get_device_error": ([vp], ctypes.c_int),
+        "qlora_selftest_wait_timeout": ([ctypes.c_uint64, vp], ctypes.c_int),
+        "qlora_set_gemm_events": ([vp, vp], ctypes.c_int),
+        "qlora_launch_count": ([], ctypes.c_uint64),
+        "qlora_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def _check(fn, code):
+    if code != QLORA_OK:
+        raise QloraError(fn, code)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(dt):
+    torch = _torch()
+    if dt == torch.bfloat16:
+        return BF16
+    if dt == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+@dataclass
+class NF4Weight:
+    """Device buffers of a quantized weight (NF4 codes + double-quantized absmax)."""
+    codes: object      # uint8 [d_out, d_in/2]
+    absmax_q: object   # uint8 [d_out*d_in/64]
+    c2: object         # float32 [ceil(d_out*d_in/16384)]
+    d_out: int
+    d_in: int
+
+    def _c(self):
+        return _NF4(self.codes.data_ptr(), self.absmax_q.data_ptr(), self.c2.data_ptr(),
+                    self.d_out, self.d_in)
+
+
+def nf4_sizes(d_out, d_in):
+    L = load()
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check("qlora_nf4_sizes", L.qlora_nf4_sizes(d_out, d_in, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def nf4_levels():
+    L = load()
+    buf = (ctypes.c_float * 16)()
+    _check("qlora_nf4_levels", L.qlora_nf4_levels(buf))
+    return list(buf)
+
+
+def workspace_bytes(op, dtype, T, d_out, d_in, r_total):
+    return int(load().qlora_workspace_bytes(op, dtype, T, d_out, d_in, r_total))
+
+
+def nf4_quantize(W, stream=None) -> NF4Weight:
+    """Quantize a device fp32/bf16 weight W[d_out, d_in] to NF4 + double quant."""
+    torch = _torch()
+    _contig(W)
+    d_out, d_in = W.shape
+    nc, na, n2 = nf4_sizes(d_out, d_in)
+    codes = torch.empty((d_out, d_in // 2), dtype=torch.uint8, device=W.device)
+    absmax = torch.empty(na, dtype=torch.uint8, device=W.device)
+    c2 = torch.empty(n2 // 4, dtype=torch.float32, device=W.device)
+    _check("nf4_quantize", load().nf4_quantize(_ptr(W), _dtype_code(W.dtype), d_out, d_in,
+                                               _ptr(codes), _ptr(absmax), _ptr(c2), _stream(stream)))
+    return NF4Weight(codes, absmax, c2, d_out, d_in)
+
+
+def nf4_dequantize(w: NF4Weight, dtype, out=None, stream=None):
+    torch = _torch()
+    if out is None:
+        out = torch.empty((w.d_out, w.d_in), dtype=dtype, device=w.codes.device)
+    c = w._c()
+    _check("nf4_dequantize", load().nf4_dequantize(ctypes.byref(c), _ptr(out), _dtype_code(dtype), _stream(stream)))
+    return out
+
+
+def _ws(op, dtype_code, T, d_out, d_in, r, device, ws):
+    torch = _torch()
+    need = workspace_bytes(op, dtype_code, T, d_out, d_in, r)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    return ws
+
+
+def qlora_linear_fwd(w: NF4Weight, X, A, B, alpha, H=None, U_save=None, ws=None, stream=None,
+                     save_u=True):
+    """H = X W^T + (alpha/r) (X A^T) B^T.  Returns (H, U_save)."""
+    torch = _torch()
+    _contig(X, A, B, H, U_save)
+    T = X.shape[0]
+    r = A.shape[0]
+    dt = _dtype_code(X.dtype)
+    if H is None:
+        H = torch.empty((T, w.d_out), dtype=X.dtype, device=X.device)
+    if U_save is None and save_u:
+        U_save = torch.empty((T, r), dtype=X.dtype, device=X.device)
+    ws = _ws(OP_FWD, dt, T, w.d_out, w.d_in, r, X.device, ws)
+    c = w._c()
+    _check("qlora_linear_fwd", load().qlora_linear_fwd(
+        ctypes.byref(c), _ptr(X), T, _ptr(A), _ptr(B), r, float(alpha), dt, _ptr(H), _ptr(U_save),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return H, U_save
+
+
+def qlora_linear_bwd(w: NF4Weight, X, dH, A, B, alpha, U_saved=None, dX=None, dA=None, dB=None,
+                     ws=None, stream=None, want_dx=True):
+    """Returns (dX, dA, dB); dA, dB fp32."""
+    torch = _torch()
+    _contig(X, dH, A, B, U_saved, dX, dA, dB)
+    T = X.shape[0]
+    r = A.shape[0]
+    dt = _dtype_code(X.dtype)
+    if dX is None and want_dx:
+        dX = torch.empty((T, w.d_in), dtype=X.dtype, device=X.device)
+    if dA is None:
+        dA = torch.empty((r, w.d_in), dtype=torch.float32, device=X.device)
+    if dB is None:
+        dB = torch.empty((w.d_out, r), dtype=torch.float32, device=X.device)
+    ws = _ws(OP_BWD, dt, T, w.d_out, w.d_in, r, X.device, ws)
+    c = w._c()
+    _check("qlora_linear_bwd", load().qlora_linear_bwd(
+        ctypes.byref(c), _ptr(X), _ptr(dH), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(U_saved), dt,
+        _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream(stream)))
+    return dX, dA, dB
+
+
+def lora_merge(w: NF4Weight, A, B, alpha, out_dtype, out=None, stream=None):
+    torch = _torch()
+    _contig(A, B, out)
+    r = A.shape[0]
+    if out is None:
+        out = torch.empty((w.d_out, w.d_in), dtype=out_dtype, device=A.device)
+    c = w._c()
+    _check("lora_merge", load().lora_merge(ctypes.byref(c), _ptr(A), _ptr(B), r, float(alpha),
+                                           _dtype_code(A.dtype), _dtype_code(out_dtype), _ptr(out),
+                                           _stream(stream)))
+    return out
+
+
+def qlora_linear_fwd_batched(w: NF4Weight, X, adapter_id, As, Bs, alphas, H=None, ws=None,
+                             stream=None):
+    torch = _torch()
+    _contig(X, adapter_id, H, *As, *Bs)
+    T = X.shape[0]
+    n = len(As)
+    ranks = [a.shape[0] for a in As]
+    dt = _dtype_code(X.dtype)
+    if H is None:
+        H = torch.empty((T, w.d_out), dtype=X.dtype, device=X.device)
+    ws = _ws(OP_FWD_BATCHED, dt, T, w.d_out, w.d_in, sum(ranks), X.device, ws)
+    Ap = (ctypes.c_void_p * n)(*[a.data_ptr() for a in As])
+    Bp = (ctypes.c_void_p * n)(*[b.data_ptr() for b in Bs])
+    rp = (ctypes.c_int32 * n)(*ranks)
+    ap = (ctypes.c_float * n)(*[float(a) for a in alphas])
+    c = w._c()
+    _check("qlora_linear_fwd_batched", load().qlora_linear_fwd_batched(
+        ctypes.byref(c), _ptr(X), T, _ptr(adapter_id), n, Ap, Bp, rp, ap, dt, _ptr(H), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return H
+
+
+def get_device_error(stream=None) -> int:
+    return int(load().qlora_get_device_error(_stream(stream)))
+
+
+def selftest_wait_timeout(limit_ns, stream=None):
+    _check("qlora_selftest_wait_timeout", load().qlora_selftest_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def set_gemm_events(start=None, stop=None):
+    """Make the fused NF4 GEMM record torch.cuda.Event objects around itself."""
+    s = ctypes.c_void_p(start.cuda_event) if start is not None else None
+    e = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
+    _check("qlora_set_gemm_events", load().qlora_set_gemm_events(s, e))
+
+
+def launch_count() -> int:
+    return int(load().qlora_launch_count())

@@ -1,0 +1,702 @@
+// qlora_api.cu -- the C ABI of libqlora (see include/qlora.h): argument validation, workspace
+// planning, TMA descriptor construction and the launch sequence of each entry point.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qlora.h"
+#include "common.cuh"
+#include "nf4.cuh"
+#include "simt.cuh"
+#include "tc_gemm.cuh"
+
+using namespace qlora;
+
+// ======================================================================= globals
+
+__device__ int g_qlora_error;   // the device error word (one per device context)
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kSmsForSplit = 148;         // split-K is sized for a B200's 148 SMs
+constexpr uint64_t kWaitNs = 4000000000ull;
+constexpr int kNf4Stages = 4;
+constexpr int kTmaStages = 4;
+
+std::atomic<uint64_t> g_launches{0};
+int* g_err_ptr[kMaxDevices] = {};
+std::mutex g_mu;
+cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+
+#define QL_TRY(expr)                         \
+    do {                                     \
+        qlora_status _s = (expr);            \
+        if (_s != QLORA_OK) return _s;       \
+    } while (0)
+
+#define QL_LAUNCH_CHECK()                                              \
+    do {                                                               \
+        count_launch();                                                \
+        if (cudaPeekAtLastError() != cudaSuccess) return QLORA_ERR_CUDA; \
+    } while (0)
+
+qlora_status err_word(int** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
+    if (!g_err_ptr[dev]) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_err_ptr[dev]) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_qlora_error) != cudaSuccess) return QLORA_ERR_CUDA;
+            g_err_ptr[dev] = static_cast<int*>(p);
+        }
+    }
+    *out = g_err_ptr[dev];
+    return QLORA_OK;
+}
+
+qlora_status get_encoder() {
+    if (g_encode) return QLORA_OK;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode) return QLORA_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return QLORA_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return QLORA_OK;
+}
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned16_or_null(const void* p) { return !p || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// ======================================================================= TMA descriptors
+
+// bf16 matrix [rows, cols] (cols contiguous, row stride ld elements), 128-byte swizzle,
+// box = 64 columns x box_rows rows.
+qlora_status tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                       uint32_t box_rows) {
+    QL_TRY(get_encoder());
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// byte matrix [rows, cols_bytes], no swizzle, box = box_x bytes x box_y rows.
+qlora_status tmap_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                     uint32_t box_x, uint32_t box_y) {
+    QL_TRY(get_encoder());
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
+    cuuint32_t box[2] = {box_x, box_y};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// ======================================================================= planning
+
+int choose_split(int64_t tiles, int64_t k_steps) {
+    int64_t s = cdiv(2 * kSmsForSplit, std::max<int64_t>(tiles, 1));
+    s = std::min<int64_t>(s, std::max<int64_t>(1, k_steps / 4));
+    s = std::max<int64_t>(1, std::min<int64_t>(s, 32));
+    const int64_t per = cdiv(k_steps, s);
+    return static_cast<int>(cdiv(k_steps, per));   // no empty splits
+}
+
+int pad_rank(int r) { return r <= 64 ? 64 : 128; }
+
+struct Plan {
+    int RP = 0;
+    int split_u = 1, split_g = 1, split_da = 1, split_db = 1;
+    size_t a_pad = 0, b_pad = 0, u_spad = 0, u_pad = 0, g_spad = 0, part = 0;
+    size_t w32 = 0, uf = 0, gf = 0;
+    size_t total = 0;
+};
+
+Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in, int r) {
+    Plan p;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    if (op == QLORA_OP_MERGE) return p;
+    if (dtype == QLORA_BF16) {
+        p.RP = pad_rank(r);
+        const int64_t RP = p.RP;
+        const int64_t mt = cdiv(T, kBM);
+        p.a_pad = take(RP * d_in * 2);
+        p.b_pad = take(d_out * RP * 2);
+        p.split_u = choose_split(mt, cdiv(d_in, kBK));
+        size_t part = static_cast<size_t>(p.split_u) * T * RP * 4;
+        if (op == QLORA_OP_FWD || op == QLORA_OP_FWD_BATCHED) {
+            p.u_spad = take(T * RP * 2);
+        } else {
+            p.u_pad = take(T * RP * 2);
+            p.g_spad = take(T * RP * 2);
+            p.split_g = choose_split(mt, cdiv(d_out, kBK));
+            p.split_da = choose_split(cdiv(d_in, kBM), cdiv(T, kBK));
+            p.split_db = choose_split(cdiv(d_out, kBM), cdiv(T, kBK));
+            part = std::max(part, static_cast<size_t>(p.split_g) * T * RP * 4);
+            part = std::max(part, static_cast<size_t>(p.split_da) * d_in * RP * 4);
+            part = std::max(part, static_cast<size_t>(p.split_db) * d_out * RP * 4);
+        }
+        p.part = take(part);
+    } else {
+        p.w32 = take(static_cast<size_t>(d_out) * d_in * 4);
+        if (op == QLORA_OP_FWD_BATCHED) {
+            p.a_pad = take(static_cast<size_t>(r) * d_in * 4);
+            p.b_pad = take(static_cast<size_t>(d_out) * r * 4);
+            p.uf = take(static_cast<size_t>(T) * r * 4);
+        } else {
+            p.uf = take(static_cast<size_t>(T) * r * 4);
+            if (op == QLORA_OP_BWD) p.gf = take(static_cast<size_t>(T) * r * 4);
+        }
+    }
+    p.total = off;
+    return p;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) {
+    return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+dim3 grid1d(int64_t n) {
+    return dim3(static_cast<unsigned>(std::min<int64_t>(std::max<int64_t>(cdiv(n, 256), 1), 148 * 16)));
+}
+
+// ======================================================================= validation
+
+qlora_status check_nf4(const qlora_nf4* w) {
+    if (!w || !aligned16(w->codes) || !aligned16(w->absmax_q) || !aligned16(w->c2))
+        return QLORA_ERR_INVALID_ARG;
+    if (w->d_out < 1 || w->d_in < 64 || w->d_in % 64 || w->d_out % 8) return QLORA_ERR_UNSUPPORTED;
+    if (w->d_out > (1 << 30) || w->d_in > (1 << 30)) return QLORA_ERR_UNSUPPORTED;
+    return QLORA_OK;
+}
+
+qlora_status check_layer(const qlora_nf4* w, int64_t T, int r, qlora_dtype dtype) {
+    QL_TRY(check_nf4(w));
+    if (dtype != QLORA_BF16 && dtype != QLORA_F32) return QLORA_ERR_INVALID_ARG;
+    if (T < 1 || T > (1LL << 30) || r < 1 || r > 128) return QLORA_ERR_UNSUPPORTED;
+    return QLORA_OK;
+}
+
+qlora_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
+    if (need == 0) return QLORA_OK;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < need) return QLORA_ERR_INVALID_ARG;
+    return QLORA_OK;
+}
+
+// ======================================================================= GEMM launchers
+
+template <bool A_MN, bool B_MN, int BMODE, int BN, int STAGES, bool OUT_F32>
+qlora_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& ax,
+                         const CUtensorMap& bx, const GemmArgs& args, dim3 grid,
+                         cudaStream_t st, bool timed) {
+    auto kern = k_tc_gemm<A_MN, B_MN, BMODE, BN, STAGES, OUT_F32>;
+    constexpr int smem = GemmSmem<BN, BMODE, STAGES>::kTotal;
+    static std::atomic<uint64_t> configured{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured.load() & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            return QLORA_ERR_CUDA;
+        configured.fetch_or(bit);
+    }
+    const bool ev = timed && g_ev_start && g_ev_stop;
+    if (ev) cudaEventRecord(g_ev_start, st);
+    kern<<<grid, kGemmThreads, smem, st>>>(a, b, ax, bx, args);
+    QL_LAUNCH_CHECK();
+    if (ev) cudaEventRecord(g_ev_stop, st);
+    return QLORA_OK;
+}
+
+GemmArgs base_args(int M, int N, int k_steps, int* err) {
+    GemmArgs g{};
+    g.M = M;
+    g.N = N;
+    g.k_steps = k_steps;
+    g.ext_steps = 0;
+    g.ext_k16_last = 4;
+    g.split = 1;
+    g.err = err;
+    g.wait_ns = kWaitNs;
+    return g;
+}
+
+// Skinny tensor-core contraction D[M, RP] = sum_K A[M,K] B[RP,K] written as fp32 split-K
+// partials.  a_mn / b_mn give the operand majorness of the two TMA maps.
+qlora_status skinny_gemm(bool a_mn, bool b_mn, int RP, const CUtensorMap& ta,
+                         const CUtensorMap& tb, int64_t M, int64_t k_steps, int split,
+                         float* part, int* err, cudaStream_t st) {
+    GemmArgs g = base_args(static_cast<int>(M), RP, static_cast<int>(k_steps), err);
+    g.split = split;
+    g.out = part;
+    g.ld_out = RP;
+    g.split_stride = M * RP;
+    dim3 grid(1, static_cast<unsigned>(cdiv(M, kBM)), static_cast<unsigned>(split));
+    if (RP == 64) {
+        if (!a_mn && !b_mn) return launch_gemm<false, false, kBTma, 64, kTmaStages, true>(ta, tb, ta, tb, g, grid, st, false);
+        if (!a_mn && b_mn) return launch_gemm<false, true, kBTma, 64, kTmaStages, true>(ta, tb, ta, tb, g, grid, st, false);
+        if (a_mn && b_mn) return launch_gemm<true, true, kBTma, 64, kTmaStages, true>(ta, tb, ta, tb, g, grid, st, false);
+    } else {
+        if (!a_mn && !b_mn) return launch_gemm<false, false, kBTma, 128, kTmaStages, true>(ta, tb, ta, tb, g, grid, st, false);
+        if (!a_mn && b_mn) return launch_gemm<false, true, kBTma, 128, kTmaStages, true>(ta, tb, ta, tb, g, grid, st, false);
+        if (a_mn && b_mn) return launch_gemm<true, true, kBTma, 128, kTmaStages, true>(ta, tb, ta, tb, g, grid, st, false);
+    }
+    return QLORA_ERR_UNSUPPORTED;
+}
+
+// Fused NF4-decode GEMM with the adapter K-extension.
+//   forward (dx = false): out[T, d_out]  = act[T, d_in]  W^T + ext_a[T, RP] ext_b[d_out, RP]^T
+//   dX      (dx = true):  out[T, d_in]   = act[T, d_out] W   + ext_a[T, RP] ext_b[RP, d_in]
+qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, const void* ext_a,
+                      const void* ext_b, int RP, int r_used, void* out, int* err,
+                      cudaStream_t st) {
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    CUtensorMap ta, tc, tax, tbx;
+    const int64_t K = dx ? d_out : d_in;
+    const int64_t N = dx ? d_in : d_out;
+    QL_TRY(tmap_bf16(&ta, act, T, K, K, kBM));
+    if (dx) QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 128, 64));
+    else QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 32, 256));
+    QL_TRY(tmap_bf16(&tax, ext_a, T, RP, RP, kBM));
+    if (dx) QL_TRY(tmap_bf16(&tbx, ext_b, RP, d_in, d_in, 64));
+    else QL_TRY(tmap_bf16(&tbx, ext_b, d_out, RP, RP, 256));
+    GemmArgs g = base_args(static_cast<int>(T), static_cast<int>(N), static_cast<int>(cdiv(K, kBK)), err);
+    g.ext_steps = RP / 64;
+    g.ext_k16_last = static_cast<int>(std::min<int64_t>(4, cdiv(r_used - 64 * (g.ext_steps - 1), 16)));
+    g.absmax_q = w->absmax_q;
+    g.c2 = w->c2;
+    g.nf4_rows = static_cast<int>(d_out);
+    g.nf4_bpr = static_cast<int>(d_in / 64);
+    g.out = out;
+    g.ld_out = N;
+    dim3 grid(static_cast<unsigned>(cdiv(N, 256)), static_cast<unsigned>(cdiv(T, kBM)), 1);
+    if (dx) return launch_gemm<false, true, kBNf4, 256, kNf4Stages, false>(ta, tc, tax, tbx, g, grid, st, true);
+    return launch_gemm<false, false, kBNf4, 256, kNf4Stages, false>(ta, tc, tax, tbx, g, grid, st, true);
+}
+
+// ======================================================================= fp32 helpers
+
+qlora_status sgemm(cudaStream_t st, int64_t M, int64_t N, int64_t K, float alpha, const float* A,
+                   int64_t lda, bool ta, const float* B, int64_t ldb, bool tb, float beta,
+                   float* C, int64_t ldc) {
+    dim3 grid(static_cast<unsigned>(cdiv(N, 64)), static_cast<unsigned>(cdiv(M, 64)));
+    k_sgemm<<<grid, 256, 0, st>>>(static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+                                  alpha, A, lda, ta ? 1 : 0, B, ldb, tb ? 1 : 0, beta, C, ldc);
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+qlora_status dequant_f32(const qlora_nf4* w, float* out, cudaStream_t st) {
+    const int64_t nbytes = w->d_out * w->d_in / 2;
+    k_nf4_dequant_f32<<<static_cast<unsigned>(cdiv(nbytes, 256)), 256, 0, st>>>(
+        w->codes, w->absmax_q, w->c2, nbytes, out);
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+template <typename T>
+qlora_status pad_bf16(const T* src, int64_t rows, int64_t cols, int64_t ld, __nv_bfloat16* dst,
+                      int64_t rows_pad, int64_t ld_dst, int64_t col_off, int64_t col_span,
+                      cudaStream_t st) {
+    k_pad_copy_bf16<T><<<grid1d(rows_pad * col_span), 256, 0, st>>>(src, rows, cols, ld, dst,
+                                                                  rows_pad, ld_dst, col_off,
+                                                                  col_span);
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+// U = X A^T on the tensor cores (split-K), finalized into the requested outputs.
+qlora_status compute_u_bf16(const void* X, int64_t T, int64_t d_in, const __nv_bfloat16* a_pad,
+                            int RP, int r, float s, int split, float* part, __nv_bfloat16* u_save,
+                            __nv_bfloat16* u_pad, __nv_bfloat16* u_spad, int* err,
+                            cudaStream_t st) {
+    CUtensorMap tx, tap;
+    QL_TRY(tmap_bf16(&tx, X, T, d_in, d_in, kBM));
+    QL_TRY(tmap_bf16(&tap, a_pad, RP, d_in, d_in, RP));
+    QL_TRY(skinny_gemm(false, false, RP, tx, tap, T, cdiv(d_in, kBK), split, part, err, st));
+    k_finalize_rows<__nv_bfloat16><<<grid1d(T * RP), 256, 0, st>>>(
+        part, split, T * RP, T, r, RP, s, u_save, u_pad, u_spad);
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+}  // namespace
+
+// ======================================================================= C ABI
+
+extern "C" {
+
+const char* qlora_status_string(qlora_status s) {
+    switch (s) {
+        case QLORA_OK: return "QLORA_OK";
+        case QLORA_ERR_INVALID_ARG: return "QLORA_ERR_INVALID_ARG";
+        case QLORA_ERR_UNSUPPORTED: return "QLORA_ERR_UNSUPPORTED";
+        case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA";
+        case QLORA_ERR_TIMEOUT: return "QLORA_ERR_TIMEOUT";
+        case QLORA_ERR_DEVICE: return "QLORA_ERR_DEVICE";
+    }
+    return "QLORA_ERR_UNKNOWN";
+}
+
+uint64_t qlora_launch_count(void) { return g_launches.load(); }
+
+qlora_status qlora_nf4_sizes(int64_t d_out, int64_t d_in, size_t* codes_bytes,
+                             size_t* absmax_bytes, size_t* c2_bytes) {
+    if (!codes_bytes || !absmax_bytes || !c2_bytes) return QLORA_ERR_INVALID_ARG;
+    if (d_out < 1 || d_in < 64 || d_in % 64) return QLORA_ERR_UNSUPPORTED;
+    const int64_t n = d_out * d_in;
+    *codes_bytes = static_cast<size_t>(n / 2);
+    *absmax_bytes = static_cast<size_t>(n / 64);
+    *c2_bytes = static_cast<size_t>(4 * cdiv(n / 64, 256));
+    return QLORA_OK;
+}
+
+qlora_status qlora_nf4_levels(float* out) {
+    if (!out) return QLORA_ERR_INVALID_ARG;
+    static const float levels[16] = QLORA_NF4_LEVELS;
+    std::memcpy(out, levels, sizeof(levels));
+    return QLORA_OK;
+}
+
+size_t qlora_workspace_bytes(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in,
+                             int32_t r_total) {
+    if (op < QLORA_OP_FWD || op > QLORA_OP_MERGE) return 0;
+    if ((dtype != QLORA_BF16 && dtype != QLORA_F32) || T < 1 || d_out < 1 || d_in < 64 ||
+        r_total < 1 || r_total > 128)
+        return 0;
+    return make_plan(op, dtype, T, d_out, d_in, r_total).total;
+}
+
+qlora_status nf4_quantize(const void* W, qlora_dtype w_dtype, int64_t d_out, int64_t d_in,
+                          uint8_t* codes, uint8_t* absmax_q, float* c2, cudaStream_t stream) {
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(absmax_q) || !aligned16(c2))
+        return QLORA_ERR_INVALID_ARG;
+    if (d_out < 1 || d_in < 64 || d_in % 64) return QLORA_ERR_UNSUPPORTED;
+    const int64_t nblocks = d_out * d_in / 64;
+    const unsigned groups = static_cast<unsigned>(cdiv(nblocks, 256));
+    if (w_dtype == QLORA_F32) {
+        k_nf4_quantize<float><<<groups, 256, 0, stream>>>(static_cast<const float*>(W), nblocks,
+                                                          codes, absmax_q, c2);
+    } else if (w_dtype == QLORA_BF16) {
+        k_nf4_quantize<__nv_bfloat16><<<groups, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(W), nblocks, codes, absmax_q, c2);
+    } else {
+        return QLORA_ERR_INVALID_ARG;
+    }
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+qlora_status nf4_dequantize(const qlora_nf4* w, void* W_out, qlora_dtype out_dtype,
+                            cudaStream_t stream) {
+    if (!w || !aligned16(w->codes) || !aligned16(w->absmax_q) || !aligned16(w->c2) ||
+        !aligned16(W_out))
+        return QLORA_ERR_INVALID_ARG;
+    if (w->d_out < 1 || w->d_in < 64 || w->d_in % 64) return QLORA_ERR_UNSUPPORTED;
+    const int64_t nblocks = w->d_out * w->d_in / 64;
+    if (out_dtype == QLORA_BF16) {
+        k_nf4_dequant_bf16<<<static_cast<unsigned>(cdiv(nblocks, 256)), 256, 0, stream>>>(
+            w->codes, w->absmax_q, w->c2, nblocks, static_cast<__nv_bfloat16*>(W_out));
+        QL_LAUNCH_CHECK();
+        return QLORA_OK;
+    }
+    if (out_dtype == QLORA_F32) return dequant_f32(w, static_cast<float*>(W_out), stream);
+    return QLORA_ERR_INVALID_ARG;
+}
+
+qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T, const void* A,
+                              const void* B, int32_t r, float alpha, qlora_dtype dtype, void* H,
+                              void* U_save, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    QL_TRY(check_layer(w, T, r, dtype));
+    if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) ||
+        !aligned16_or_null(U_save))
+        return QLORA_ERR_INVALID_ARG;
+    const Plan p = make_plan(QLORA_OP_FWD, dtype, T, w->d_out, w->d_in, r);
+    QL_TRY(check_ws(ws, ws_bytes, p.total));
+    int* err = nullptr;
+    QL_TRY(err_word(&err));
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    const float s = alpha / static_cast<float>(r);
+    if (dtype == QLORA_BF16) {
+        const int RP = p.RP;
+        auto* a_pad = at<__nv_bfloat16>(ws, p.a_pad);
+        auto* b_pad = at<__nv_bfloat16>(ws, p.b_pad);
+        auto* u_spad = at<__nv_bfloat16>(ws, p.u_spad);
+        auto* part = at<float>(ws, p.part);
+        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A), r, d_in, d_in, a_pad, RP, d_in, 0, d_in, stream));
+        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
+        QL_TRY(compute_u_bf16(X, T, d_in, a_pad, RP, r, s, p.split_u, part,
+                              static_cast<__nv_bfloat16*>(U_save), nullptr, u_spad, err, stream));
+        return nf4_gemm(false, w, X, T, u_spad, b_pad, RP, r, H, err, stream);
+    }
+    // exact fp32 path
+    float* w32 = at<float>(ws, p.w32);
+    float* U = U_save ? static_cast<float*>(U_save) : at<float>(ws, p.uf);
+    const float* Xf = static_cast<const float*>(X);
+    QL_TRY(dequant_f32(w, w32, stream));
+    QL_TRY(sgemm(stream, T, r, d_in, 1.f, Xf, d_in, false, static_cast<const float*>(A), d_in, true, 0.f, U, r));
+    QL_TRY(sgemm(stream, T, d_out, d_in, 1.f, Xf, d_in, false, w32, d_in, true, 0.f, static_cast<float*>(H), d_out));
+    return sgemm(stream, T, d_out, r, s, U, r, false, static_cast<const float*>(B), r, true, 1.f,
+                 static_cast<float*>(H), d_out);
+}
+
+qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                              const void* A, const void* B, int32_t r, float alpha,
+                              const void* U_saved, qlora_dtype dtype, void* dX, float* dA,
+                              float* dB, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    QL_TRY(check_layer(w, T, r, dtype));
+    if (!aligned16(X) || !aligned16(dH) || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
+        !aligned16(dB) || !aligned16_or_null(dX) || !aligned16_or_null(U_saved))
+        return QLORA_ERR_INVALID_ARG;
+    const Plan p = make_plan(QLORA_OP_BWD, dtype, T, w->d_out, w->d_in, r);
+    QL_TRY(check_ws(ws, ws_bytes, p.total));
+    int* err = nullptr;
+    QL_TRY(err_word(&err));
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    const float s = alpha / static_cast<float>(r);
+    if (dtype == QLORA_BF16) {
+        const int RP = p.RP;
+        auto* a_pad = at<__nv_bfloat16>(ws, p.a_pad);
+        auto* b_pad = at<__nv_bfloat16>(ws, p.b_pad);
+        auto* u_pad = at<__nv_bfloat16>(ws, p.u_pad);
+        auto* g_spad = at<__nv_bfloat16>(ws, p.g_spad);
+        auto* part = at<float>(ws, p.part);
+        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A), r, d_in, d_in, a_pad, RP, d_in, 0, d_in, stream));
+        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
+        if (U_saved) {
+            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(U_saved), T, r, r, u_pad, T, RP, 0, RP, stream));
+        } else {
+            QL_TRY(compute_u_bf16(X, T, d_in, a_pad, RP, r, s, p.split_u, part, nullptr, u_pad,
+                                  nullptr, err, stream));
+        }
+        // G = dH B  ->  g_spad = bf16(s G)
+        {
+            CUtensorMap tdh, tbp;
+            QL_TRY(tmap_bf16(&tdh, dH, T, d_out, d_out, kBM));
+            QL_TRY(tmap_bf16(&tbp, b_pad, d_out, RP, RP, 64));
+            QL_TRY(skinny_gemm(false, true, RP, tdh, tbp, T, cdiv(d_out, kBK), p.split_g, part, err, stream));
+            k_finalize_rows<__nv_bfloat16><<<grid1d(T * RP), 256, 0, stream>>>(
+                part, p.split_g, T * RP, T, r, RP, s, nullptr, nullptr, g_spad);
+            QL_LAUNCH_CHECK();
+        }
+        // dX = dH W^ + (sG) A
+        if (dX) QL_TRY(nf4_gemm(true, w, dH, T, g_spad, a_pad, RP, r, dX, err, stream));
+        // dA^T[d_in, RP] = X^T (sG)
+        {
+            CUtensorMap txm, tgm;
+            QL_TRY(tmap_bf16(&txm, X, T, d_in, d_in, 64));
+            QL_TRY(tmap_bf16(&tgm, g_spad, T, RP, RP, 64));
+            QL_TRY(skinny_gemm(true, true, RP, txm, tgm, d_in, cdiv(T, kBK), p.split_da, part, err, stream));
+            k_finalize_dA<<<grid1d(static_cast<int64_t>(r) * d_in), 256, 0, stream>>>(
+                part, p.split_da, d_in * RP, d_in, r, RP, dA);
+            QL_LAUNCH_CHECK();
+        }
+        // dB[d_out, RP] = s dH^T U
+        {
+            CUtensorMap thm, tum;
+            QL_TRY(tmap_bf16(&thm, dH, T, d_out, d_out, 64));
+            QL_TRY(tmap_bf16(&tum, u_pad, T, RP, RP, 64));
+            QL_TRY(skinny_gemm(true, true, RP, thm, tum, d_out, cdiv(T, kBK), p.split_db, part, err, stream));
+            k_finalize_dB<<<grid1d(d_out * r), 256, 0, stream>>>(part, p.split_db, d_out * RP,
+                                                                 d_out, r, RP, s, dB);
+            QL_LAUNCH_CHECK();
+        }
+        return QLORA_OK;
+    }
+    // exact fp32 path
+    const float* Xf = static_cast<const float*>(X);
+    const float* dHf = static_cast<const float*>(dH);
+    const float* Af = static_cast<const float*>(A);
+    const float* Bf = static_cast<const float*>(B);
+    float* w32 = at<float>(ws, p.w32);
+    float* U = at<float>(ws, p.uf);
+    float* G = at<float>(ws, p.gf);
+    QL_TRY(dequant_f32(w, w32, stream));
+    const float* Uc = static_cast<const float*>(U_saved);
+    if (!Uc) {
+        QL_TRY(sgemm(stream, T, r, d_in, 1.f, Xf, d_in, false, Af, d_in, true, 0.f, U, r));
+        Uc = U;
+    }
+    QL_TRY(sgemm(stream, T, r, d_out, 1.f, dHf, d_out, false, Bf, r, false, 0.f, G, r));
+    if (dX) {
+        float* dXf = static_cast<float*>(dX);
+        QL_TRY(sgemm(stream, T, d_in, d_out, 1.f, dHf, d_out, false, w32, d_in, false, 0.f, dXf, d_in));
+        QL_TRY(sgemm(stream, T, d_in, r, s, G, r, false, Af, d_in, false, 1.f, dXf, d_in));
+    }
+    QL_TRY(sgemm(stream, r, d_in, T, s, G, r, true, Xf, d_in, false, 0.f, dA, d_in));
+    return sgemm(stream, d_out, r, T, s, dHf, d_out, true, Uc, r, false, 0.f, dB, r);
+}
+
+qlora_status lora_merge(const qlora_nf4* w, const void* A, const void* B, int32_t r, float alpha,
+                        qlora_dtype adapter_dtype, qlora_dtype out_dtype, void* W_final,
+                        cudaStream_t stream) {
+    QL_TRY(check_nf4(w));
+    if (!aligned16(A) || !aligned16(B) || !aligned16(W_final)) return QLORA_ERR_INVALID_ARG;
+    if (r < 1 || r > 128) return QLORA_ERR_UNSUPPORTED;
+    const float s = alpha / static_cast<float>(r);
+    dim3 grid(static_cast<unsigned>(cdiv(w->d_in, 256)), static_cast<unsigned>(cdiv(w->d_out, 32)));
+    const size_t smem = static_cast<size_t>(r) * 256 * 4 + 32 * static_cast<size_t>(r) * 4;
+    auto run = [&](auto kern, auto a, auto b, auto o) -> qlora_status {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        kern<<<grid, 256, smem, stream>>>(w->codes, w->absmax_q, w->c2, w->d_out, w->d_in, a, b, r, s, o);
+        QL_LAUNCH_CHECK();
+        return QLORA_OK;
+    };
+    using bf = __nv_bfloat16;
+    if (adapter_dtype == QLORA_BF16 && out_dtype == QLORA_BF16)
+        return run(k_merge<bf, bf>, static_cast<const bf*>(A), static_cast<const bf*>(B), static_cast<bf*>(W_final));
+    if (adapter_dtype == QLORA_BF16 && out_dtype == QLORA_F32)
+        return run(k_merge<bf, float>, static_cast<const bf*>(A), static_cast<const bf*>(B), static_cast<float*>(W_final));
+    if (adapter_dtype == QLORA_F32 && out_dtype == QLORA_BF16)
+        return run(k_merge<float, bf>, static_cast<const float*>(A), static_cast<const float*>(B), static_cast<bf*>(W_final));
+    if (adapter_dtype == QLORA_F32 && out_dtype == QLORA_F32)
+        return run(k_merge<float, float>, static_cast<const float*>(A), static_cast<const float*>(B), static_cast<float*>(W_final));
+    return QLORA_ERR_INVALID_ARG;
+}
+
+qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t T,
+                                      const int32_t* adapter_id, int32_t n_adapters,
+                                      const void* const* A, const void* const* B,
+                                      const int32_t* r, const float* alpha, qlora_dtype dtype,
+                                      void* H, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!A || !B || !r || !alpha || n_adapters < 1 || n_adapters > 32) return QLORA_ERR_INVALID_ARG;
+    int R = 0;
+    for (int i = 0; i < n_adapters; ++i) {
+        if (r[i] < 1 || r[i] > 128) return QLORA_ERR_UNSUPPORTED;
+        if (!aligned16(A[i]) || !aligned16(B[i])) return QLORA_ERR_INVALID_ARG;
+        R += r[i];
+    }
+    if (R > 128) return QLORA_ERR_UNSUPPORTED;
+    QL_TRY(check_layer(w, T, R, dtype));
+    if (!aligned16(X) || !aligned16(H) || !aligned16(adapter_id)) return QLORA_ERR_INVALID_ARG;
+    const Plan p = make_plan(QLORA_OP_FWD_BATCHED, dtype, T, w->d_out, w->d_in, R);
+    QL_TRY(check_ws(ws, ws_bytes, p.total));
+    int* err = nullptr;
+    QL_TRY(err_word(&err));
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    SegTable seg;
+    for (int j = 0; j < 128; ++j) seg.seg_of[j] = -1;
+    for (int i = 0; i < 32; ++i) seg.scale[i] = 0.f;
+    {
+        int off = 0;
+        for (int i = 0; i < n_adapters; ++i) {
+            for (int j = 0; j < r[i]; ++j) seg.seg_of[off + j] = i;
+            seg.scale[i] = alpha[i] / static_cast<float>(r[i]);
+            off += r[i];
+        }
+    }
+    if (dtype == QLORA_BF16) {
+        const int RP = p.RP;
+        auto* a_cat = at<__nv_bfloat16>(ws, p.a_pad);
+        auto* b_cat = at<__nv_bfloat16>(ws, p.b_pad);
+        auto* u_all = at<__nv_bfloat16>(ws, p.u_spad);
+        auto* part = at<float>(ws, p.part);
+        if (cudaMemsetAsync(a_cat, 0, static_cast<size_t>(RP) * d_in * 2, stream) != cudaSuccess ||
+            cudaMemsetAsync(b_cat, 0, static_cast<size_t>(d_out) * RP * 2, stream) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        int off = 0;
+        for (int i = 0; i < n_adapters; ++i) {
+            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A[i]), r[i], d_in, d_in,
+                            a_cat + static_cast<int64_t>(off) * d_in, r[i], d_in, 0, d_in, stream));
+            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B[i]), d_out, r[i], r[i], b_cat,
+                            d_out, RP, off, r[i], stream));
+            off += r[i];
+        }
+        CUtensorMap tx, tap;
+        QL_TRY(tmap_bf16(&tx, X, T, d_in, d_in, kBM));
+        QL_TRY(tmap_bf16(&tap, a_cat, RP, d_in, d_in, RP));
+        QL_TRY(skinny_gemm(false, false, RP, tx, tap, T, cdiv(d_in, kBK), p.split_u, part, err, stream));
+        k_finalize_multi<<<grid1d(T * RP), 256, 0, stream>>>(part, p.split_u, T * RP, T, RP,
+                                                             n_adapters, adapter_id, seg, u_all,
+                                                             nullptr, err);
+        QL_LAUNCH_CHECK();
+        return nf4_gemm(false, w, X, T, u_all, b_cat, RP, R, H, err, stream);
+    }
+    // exact fp32 path
+    float* w32 = at<float>(ws, p.w32);
+    float* a_cat = at<float>(ws, p.a_pad);
+    float* b_cat = at<float>(ws, p.b_pad);
+    float* U = at<float>(ws, p.uf);
+    int off = 0;
+    for (int i = 0; i < n_adapters; ++i) {
+        k_pad_copy_f32<<<grid1d(static_cast<int64_t>(r[i]) * d_in), 256, 0, stream>>>(
+            static_cast<const float*>(A[i]), r[i], d_in, d_in, a_cat + static_cast<int64_t>(off) * d_in,
+            r[i], d_in, 0, d_in);
+        QL_LAUNCH_CHECK();
+        k_pad_copy_f32<<<grid1d(d_out * r[i]), 256, 0, stream>>>(
+            static_cast<const float*>(B[i]), d_out, r[i], r[i], b_cat, d_out, R, off, r[i]);
+        QL_LAUNCH_CHECK();
+        off += r[i];
+    }
+    const float* Xf = static_cast<const float*>(X);
+    QL_TRY(dequant_f32(w, w32, stream));
+    QL_TRY(sgemm(stream, T, R, d_in, 1.f, Xf, d_in, false, a_cat, d_in, true, 0.f, U, R));
+    k_mask_multi_f32<<<grid1d(T * R), 256, 0, stream>>>(U, T, R, n_adapters, adapter_id, seg, err);
+    QL_LAUNCH_CHECK();
+    QL_TRY(sgemm(stream, T, d_out, d_in, 1.f, Xf, d_in, false, w32, d_in, true, 0.f, static_cast<float*>(H), d_out));
+    return sgemm(stream, T, d_out, R, 1.f, U, R, false, b_cat, R, true, 1.f, static_cast<float*>(H), d_out);
+}
+
+qlora_status qlora_get_device_error(cudaStream_t stream) {
+    int* err = nullptr;
+    QL_TRY(err_word(&err));
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return QLORA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+    }
+    return static_cast<qlora_status>(v);
+}
+
+qlora_status qlora_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
+    int* err = nullptr;
+    QL_TRY(err_word(&err));
+    k_wait_timeout_selftest<<<1, 32, 0, stream>>>(err, limit_ns);
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+qlora_status qlora_set_gemm_events(cudaEvent_t start, cudaEvent_t stop) {
+    g_ev_start = start;
+    g_ev_stop = stop;
+    return QLORA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,79 @@
+"""The C-ABI library loads, exports every declared symbol, and its host-only calls agree
+with the oracle.  No GPU needed: nothing here launches a kernel."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+import qlora_parameter_efficient_b200 as q
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "qlora.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from qlora_parameter_efficient_b200 import build
+    build.build_library()
+    return q.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 14
+    assert sorted(names) == sorted(q.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_levels_match_oracle_bitwise(L):
+    lib = np.array(q.nf4_levels(), np.float32)
+    assert np.array_equal(lib.view(np.uint32), O.nf4_levels().view(np.uint32))
+
+
+def test_sizes_match_oracle(L):
+    for d, k in [(4096, 4096), (11008, 4096), (3, 128), (256, 256)]:
+        assert q.nf4_sizes(d, k) == O.nf4_sizes(d, k)
+    with pytest.raises(q.QloraError):
+        q.nf4_sizes(10, 100)
+
+
+def test_workspace_sizes(L):
+    for op in (q.OP_FWD, q.OP_BWD, q.OP_FWD_BATCHED):
+        for dt in (q.BF16, q.F32):
+            assert q.workspace_bytes(op, dt, 4096, 4096, 4096, 16) > 0
+    assert q.workspace_bytes(q.OP_MERGE, q.BF16, 1, 64, 64, 8) == 0
+    assert q.workspace_bytes(q.OP_FWD, q.BF16, 1, 64, 64, 129) == 0
+    assert q.workspace_bytes(9, q.BF16, 1, 64, 64, 8) == 0
+
+
+def test_status_strings(L):
+    for code, name in q.STATUS.items():
+        assert L.qlora_status_string(code).decode() == name
+
+
+def test_host_validation_rejects_before_launch(L):
+    # Invalid arguments are refused on the host, before any CUDA call.
+    nf4 = q._NF4(16, 16, 16, 64, 100)            # d_in not a multiple of 64
+    r = L.qlora_linear_fwd(ctypes.byref(nf4), 16, 1, 16, 16, 8, 16.0, q.BF16, 16, None, 256, 1 << 20, None)
+    assert r == 2
+    nf4 = q._NF4(16, 16, 16, 64, 64)
+    r = L.qlora_linear_fwd(ctypes.byref(nf4), 16, 1, 16, 16, 200, 16.0, q.BF16, 16, None, 256, 1 << 20, None)
+    assert r == 2                                # r > 128
+    r = L.qlora_linear_fwd(ctypes.byref(nf4), 17, 1, 16, 16, 8, 16.0, q.BF16, 16, None, 256, 1 << 20, None)
+    assert r == 1                                # misaligned X
+    r = L.nf4_quantize(None, q.F32, 64, 64, 16, 16, 16, None)
+    assert r == 1
+    r = L.qlora_linear_fwd(ctypes.byref(nf4), 16, 1, 16, 16, 8, 16.0, 7, 16, None, 256, 1 << 20, None)
+    assert r == 1                                # bad dtype
+    r = L.qlora_linear_fwd(ctypes.byref(nf4), 16, 1, 16, 16, 8, 16.0, q.BF16, 16, None, 256, 10, None)
+    assert r == 1                                # workspace too small

@@ -1,0 +1,253 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Integer / byte outputs (NF4 codes, absmax bytes, c2, decoded weights) must be bit-exact;
+H, dX, dA, dB must be within a relative Frobenius error of 5e-3 (bf16) or 1e-5 (fp32).
+Small cases span several 128x256 tiles with ragged tails in T, d_out, d_in and r; the
+full-size Llama-2-7B q_proj case is checked on sampled token rows (H, dX) and in full
+(dA, dB, decode).
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from qlora_parameter_efficient_b200 import synthetic as S
+
+from parity import TOL, dev, host, oracle_weight, quantize_both, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from qlora_parameter_efficient_b200 import build
+    build.build_library()
+    import qlora_parameter_efficient_b200 as lib
+    lib.load()
+    return lib
+
+
+# ------------------------------------------------------------------ NF4 storage
+
+
+@pytest.mark.parametrize("d_out,d_in", [(8, 64), (3, 128), (64, 256), (256, 4096), (100, 1088)])
+def test_quantize_bit_exact(q, d_out, d_in):
+    rng = np.random.default_rng(d_out * 7 + d_in)
+    W = (rng.standard_normal((d_out, d_in)) * 0.141).astype(np.float32)
+    W[0, :64] = 0.0                      # an all-zero block
+    W[-1, -1] = -3.0                      # one large block
+    w = q.nf4_quantize(dev(W))
+    codes, q8, c2, _ = O.nf4_quantize(W)
+    assert np.array_equal(w.codes.cpu().numpy(), codes)
+    assert np.array_equal(w.absmax_q.cpu().numpy(), q8)
+    assert np.array_equal(w.c2.cpu().numpy().view(np.uint32), c2.view(np.uint32))
+
+
+def test_quantize_bf16_input_bit_exact(q):
+    import torch
+    rng = np.random.default_rng(11)
+    W = S.round_to_bf16((rng.standard_normal((96, 512)) * 0.141).astype(np.float32))
+    w = q.nf4_quantize(dev(W, "bf16"))
+    codes, q8, c2, _ = O.nf4_quantize(W)
+    assert w.codes.dtype == torch.uint8
+    assert np.array_equal(w.codes.cpu().numpy(), codes)
+    assert np.array_equal(w.absmax_q.cpu().numpy(), q8)
+    assert np.array_equal(w.c2.cpu().numpy(), c2)
+
+
+@pytest.mark.parametrize("d_out,d_in", [(16, 64), (200, 192), (4096, 4096)])
+def test_dequantize_bit_exact(q, d_out, d_in):
+    import torch
+    rng = np.random.default_rng(d_out + d_in)
+    W = (rng.standard_normal((d_out, d_in)) * 0.141).astype(np.float32)
+    W[1, :64] = 0.0
+    w, oc = quantize_both(q, W)
+    for dt, tdt in (("bf16", torch.bfloat16), ("f32", torch.float32)):
+        got = host(q.nf4_dequantize(w, tdt))
+        ref = O.nf4_dequantize(*oc[:3], d_out, d_in, out=dt)
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), dt
+
+
+# ------------------------------------------------------------------ single-adapter layer
+
+
+def run_layer(q, case, rows=None):
+    """Run fwd + bwd on the GPU and compare with the oracle.  rows: sampled token rows for
+    H and dX (None: all)."""
+    import torch
+    d_out, d_in, r, T, dt = case.d_out, case.d_in, case.r, case.T, case.dtype
+    w, oc = quantize_both(q, case.W0)
+    Wh = oracle_weight(oc, d_out, d_in, dt)
+    X, A, B, dH = dev(case.X, dt), dev(case.A, dt), dev(case.B, dt), dev(case.dH, dt)
+    H, U = q.qlora_linear_fwd(w, X, A, B, case.alpha)
+    dX, dA, dB = q.qlora_linear_bwd(w, X, dH, A, B, case.alpha, U_saved=U)
+    _, dA2, dB2 = q.qlora_linear_bwd(w, X, dH, A, B, case.alpha, U_saved=None, want_dx=False)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    sel = slice(None) if rows is None else rows
+    Href = O.lora_forward(Wh, case.X[sel], case.A, case.B, case.alpha, r)
+    err = {"H": rel_fro(host(H)[sel], Href)}
+    Uref = case.X.astype(np.float64) @ case.A.astype(np.float64).T
+    err["U"] = rel_fro(host(U)[sel], Uref[sel])
+    dXref, _, _ = O.lora_backward(Wh, case.X[sel], case.dH[sel], case.A, case.B, case.alpha, r)
+    err["dX"] = rel_fro(host(dX)[sel], dXref)
+    dAref, dBref = O.lora_adapter_grads(case.X, case.dH, case.A, case.B, case.alpha, r)
+    err["dA"] = rel_fro(host(dA), dAref)
+    err["dB"] = rel_fro(host(dB), dBref)
+    err["dA_recomputedU"] = rel_fro(host(dA2), dAref)
+    err["dB_recomputedU"] = rel_fro(host(dB2), dBref)
+    tol = TOL[dt]
+    bad = {k: v for k, v in err.items() if not v <= tol}
+    assert not bad, f"{err} (tol {tol})"
+    return err
+
+
+SMALL = [
+    # d_out, d_in, r, T   (several 128x256 tiles and ragged tails in every dimension)
+    (256, 256, 8, 64),
+    (200, 192, 5, 77),
+    (64, 64, 1, 1),
+    (520, 320, 16, 300),
+    (256, 512, 64, 129),
+    (136, 256, 100, 50),
+    (1024, 1024, 128, 256),
+    (768, 640, 33, 1000),
+]
+
+
+@pytest.mark.parametrize("d_out,d_in,r,T", SMALL)
+def test_layer_bf16_small(q, d_out, d_in, r, T):
+    case = S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_out + T)
+    run_layer(q, case)
+
+
+@pytest.mark.parametrize("d_out,d_in,r,T", [(256, 256, 8, 64), (200, 192, 5, 77), (64, 128, 3, 1)])
+def test_layer_f32(q, d_out, d_in, r, T):
+    case = S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="f32", seed=3)
+    run_layer(q, case)
+
+
+def test_small_fp32_config(q):
+    case = S.make_layer(**S.CONFIGS["small_256_r8_T64_f32"], seed=0)
+    run_layer(q, case)
+
+
+def test_q_proj_full_size_sampled_rows(q):
+    case = S.make_layer(**S.CONFIGS["q_proj_4096x4096_r16_T4096"], seed=0)
+    rows = np.sort(np.random.default_rng(0).choice(case.T, 256, replace=False))
+    run_layer(q, case, rows=rows)
+
+
+# ------------------------------------------------------------------ invariants on the GPU
+
+
+def test_zero_B_gives_base_output_bitwise(q):
+    # With B = 0 the adapter K-steps add exact zeros, so H(B=0, A) == H(A=0, B') bit for bit.
+    import torch
+    case = S.make_layer(384, 512, 16, 32.0, 200, dtype="bf16", seed=5)
+    w = q.nf4_quantize(dev(case.W0))
+    X, A, B = dev(case.X, "bf16"), dev(case.A, "bf16"), dev(case.B, "bf16")
+    H1, _ = q.qlora_linear_fwd(w, X, A, torch.zeros_like(B), 32.0)
+    H2, _ = q.qlora_linear_fwd(w, X, torch.zeros_like(A), B, 32.0)
+    assert torch.equal(H1, H2)
+    Wh = oracle_weight(O.nf4_quantize(case.W0), 384, 512, "bf16")
+    assert rel_fro(host(H1), case.X.astype(np.float64) @ Wh.T) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_merge(q, out):
+    import torch
+    case = S.make_layer(520, 384, 16, 32.0, 64, dtype="bf16", seed=9)
+    w, oc = quantize_both(q, case.W0)
+    A, B = dev(case.A, "bf16"), dev(case.B, "bf16")
+    Wf = q.lora_merge(w, A, B, 32.0, torch.bfloat16 if out == "bf16" else torch.float32)
+    Wh = oracle_weight(oc, 520, 384, out)
+    ref = O.lora_merge(Wh, case.A, case.B, 32.0, 16)
+    assert rel_fro(host(Wf), ref) <= TOL[out]
+    # the merged weight reproduces the unmerged layer output
+    H, _ = q.qlora_linear_fwd(w, dev(case.X, "bf16"), A, B, 32.0)
+    Hm = case.X.astype(np.float64) @ host(Wf).astype(np.float64).T
+    assert rel_fro(host(H), Hm) <= TOL["bf16"]
+
+
+def test_merge_f32_adapters(q):
+    import torch
+    case = S.make_layer(256, 256, 8, 16.0, 16, dtype="f32", seed=2)
+    w, oc = quantize_both(q, case.W0)
+    Wf = q.lora_merge(w, dev(case.A), dev(case.B), 16.0, torch.float32)
+    ref = O.lora_merge(oracle_weight(oc, 256, 256, "f32"), case.A, case.B, 16.0, 8)
+    assert rel_fro(host(Wf), ref) <= TOL["f32"]
+
+
+# ------------------------------------------------------------------ multi-adapter
+
+
+def run_batched(q, mc, rows=None):
+    import torch
+    w, oc = quantize_both(q, mc.W0)
+    Wh = oracle_weight(oc, mc.d_out, mc.d_in, mc.dtype)
+    X = dev(mc.X, mc.dtype)
+    ids = torch.from_numpy(mc.ids).to("cuda")
+    As = [dev(a, mc.dtype) for a in mc.As]
+    Bs = [dev(b, mc.dtype) for b in mc.Bs]
+    H = q.qlora_linear_fwd_batched(w, X, ids, As, Bs, mc.alphas)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    sel = slice(None) if rows is None else rows
+    ref = O.lora_forward_batched(Wh, mc.X[sel], mc.ids[sel], mc.As, mc.Bs, mc.alphas, mc.ranks)
+    e = rel_fro(host(H)[sel], ref)
+    assert e <= TOL[mc.dtype], e
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_batched_small(q, dtype):
+    mc = S.make_multi_adapter(264, 320, 150, [3, 8, 20], dtype=dtype, seed=4)
+    run_batched(q, mc)
+
+
+def test_batched_full_uniform_and_skewed(q):
+    for split in (None, [0.7, 0.1, 0.1, 0.1]):
+        mc = S.make_multi_adapter(4096, 4096, 4096, [8, 16, 16, 64], split=split, seed=0)
+        rows = np.sort(np.random.default_rng(1).choice(4096, 256, replace=False))
+        run_batched(q, mc, rows=rows)
+
+
+def test_batched_bad_id_reports_device_error(q):
+    import torch
+    mc = S.make_multi_adapter(128, 128, 40, [4, 4], seed=6)
+    mc.ids[7] = 5
+    w = q.nf4_quantize(dev(mc.W0))
+    H = q.qlora_linear_fwd_batched(w, dev(mc.X, "bf16"), torch.from_numpy(mc.ids).cuda(),
+                                   [dev(a, "bf16") for a in mc.As], [dev(b, "bf16") for b in mc.Bs],
+                                   mc.alphas)
+    assert q.get_device_error() == 5
+    assert q.get_device_error() == 0          # read-and-clear
+    # the other tokens are still right
+    Wh = oracle_weight(O.nf4_quantize(mc.W0), 128, 128, "bf16")
+    keep = np.arange(40) != 7
+    ref = O.lora_forward_batched(Wh, mc.X[keep], mc.ids[keep], mc.As, mc.Bs, mc.alphas, mc.ranks)
+    assert rel_fro(host(H)[keep], ref) <= TOL["bf16"]
+
+
+# ------------------------------------------------------------------ failure detection
+
+
+def test_bounded_wait_times_out_and_context_survives(q):
+    import torch
+    q.selftest_wait_timeout(20_000_000)       # 20 ms
+    assert q.get_device_error() == 4
+    assert q.get_device_error() == 0
+    x = torch.ones(4, device="cuda")
+    assert float((x * 2).sum()) == 8.0        # the context is still usable
+
+
+def test_launch_counter_moves(q):
+    import torch
+    n0 = q.launch_count()
+    case = S.make_layer(128, 128, 4, 8.0, 16, dtype="bf16", seed=1)
+    w = q.nf4_quantize(dev(case.W0))
+    q.qlora_linear_fwd(w, dev(case.X, "bf16"), dev(case.A, "bf16"), dev(case.B, "bf16"), 8.0)
+    torch.cuda.synchronize()
+    assert q.launch_count() - n0 >= 5
