@@ -1,0 +1,399 @@
+"""Benchmark of the QLoRA-adapted linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--extra]
+
+A step is one forward + backward pass of the layer (NF4 W0 decoded on the fly inside the
+tensor-core GEMM, LoRA branch fused; dX, dA, dB) over one batch of synthetic tokens shaped
+like Llama-2-7B q_proj: W0 4096x4096 NF4 + double quant, r = 16, alpha = 32, 4096 bf16
+tokens.  With N > 1 (one process per GPU under torchrun) every rank runs its own batch
+(weak scaling, data parallel) and the adapter gradients dA, dB are all-reduced over NCCL
+inside the step.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the plain fp64 implementation the tests check
+against) on this host's cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "q_proj_4096x4096_r16_T4096"
+METRIC = "QLoRA linear fwd+bwd tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def cfg():
+    from qlora_parameter_efficient_b200 import synthetic as S
+    return dict(S.CONFIGS[WORKLOAD])
+
+
+def flops_fwd(T, d, k, r):
+    return 2 * T * d * k + 2 * T * r * (d + k)
+
+
+def flops_bwd(T, d, k, r):
+    return 2 * T * d * k + 4 * T * r * (d + k)
+
+
+# ---------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                       "-i", str(self.index), "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.p:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+
+    def summary(self):
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------- oracle timing
+
+
+def oracle_sample(n_tokens, seed=0):
+    """One bounded-sample step of the oracle: decode W^ and fwd + bwd over n_tokens tokens."""
+    import numpy as np
+    import oracle as O
+    from qlora_parameter_efficient_b200 import synthetic as S
+    c = cfg()
+    case = S.make_layer(c["d_out"], c["d_in"], c["r"], c["alpha"], n_tokens, dtype="bf16", seed=seed)
+    codes, q8, c2, _ = O.nf4_quantize(case.W0)         # storage prepared outside the timing
+    t0 = time.perf_counter()
+    Wh = O.nf4_dequantize(codes, q8, c2, c["d_out"], c["d_in"], out="bf16")
+    O.lora_forward(Wh, case.X, case.A, case.B, case.alpha, case.r)
+    O.lora_backward(Wh, case.X, case.dH, case.A, case.B, case.alpha, case.r)
+    return time.perf_counter() - t0
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(target_s=10.0):
+    t_small = oracle_sample(256)
+    n = int(min(cfg()["T"], max(256, 256 * target_s / max(t_small, 1e-3))))
+    n = max(256, (n // 256) * 256)
+    t = oracle_sample(n, seed=1)
+    return {"value": n / t, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{n} of {cfg()['T']} tokens of {WORKLOAD}: NF4 decode + fp64 fwd + bwd "
+                      f"({t:.1f} s)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    c = cfg()
+    n = 512
+    oracle_sample(256)                                   # warm import / caches
+    for _ in range(args.warmup):
+        oracle_sample(n)
+    times = [oracle_sample(n, seed=i + 1) for i in range(args.steps)]
+    total = sum(times)
+    value = n * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD + " fwd+bwd", "d_out": c["d_out"], "d_in": c["d_in"],
+                   "r": c["r"], "alpha": c["alpha"], "tokens_per_step": n,
+                   "note": "each step is a bounded sample of the workload"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle",
+                         "cores": oracle_threads(),
+                         "sample": f"{n} of {c['T']} tokens per step: NF4 decode + fp64 fwd + bwd"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- GPU arm
+
+
+def run_gpu(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import qlora_parameter_efficient_b200 as q
+    from qlora_parameter_efficient_b200 import build as qb
+    from qlora_parameter_efficient_b200 import synthetic as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    if rank == 0:
+        qb.build_library()
+    if world > 1:
+        dist.barrier()
+    q.load()
+    peaks, peak_src = load_peaks()
+    c = cfg()
+    d, k, r, T, alpha = c["d_out"], c["d_in"], c["r"], c["T"], c["alpha"]
+    bf = torch.bfloat16
+
+    # Rotating input sets so the working set (about 4 x 75 MB) exceeds 2 x the 126 MB L2.
+    NSETS = 4
+    sets = []
+    for i in range(NSETS):
+        case = S.make_layer(d, k, r, alpha, T, dtype="bf16", seed=1000 * rank + i)
+        w = q.nf4_quantize(torch.from_numpy(case.W0).to(dev))
+        sets.append(dict(
+            w=w, X=torch.from_numpy(case.X).to(dev).to(bf), dH=torch.from_numpy(case.dH).to(dev).to(bf),
+            A=torch.from_numpy(case.A).to(dev).to(bf), B=torch.from_numpy(case.B).to(dev).to(bf)))
+        del case
+    H = torch.empty((T, d), dtype=bf, device=dev)
+    U = torch.empty((T, r), dtype=bf, device=dev)
+    dX = torch.empty((T, k), dtype=bf, device=dev)
+    dA = torch.empty((r, k), dtype=torch.float32, device=dev)
+    dB = torch.empty((d, r), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(q.workspace_bytes(q.OP_FWD, q.BF16, T, d, k, r),
+                         q.workspace_bytes(q.OP_BWD, q.BF16, T, d, k, r)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = sets[i % NSETS]
+        q.qlora_linear_fwd(s["w"], s["X"], s["A"], s["B"], alpha, H=H, U_save=U, ws=ws)
+        q.qlora_linear_bwd(s["w"], s["X"], s["dH"], s["A"], s["B"], alpha, U_saved=U, dX=dX, dA=dA,
+                           dB=dB, ws=ws)
+        if world > 1:
+            dist.all_reduce(dA)
+            dist.all_reduce(dB)
+
+    def timed(fn, K, W, with_gemm_events=False):
+        for i in range(W):
+            fn(i)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        gev = []
+        n0 = q.launch_count()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K):
+            if with_gemm_events:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                b.record(stream)      # materialise the events before handing them over
+                q.set_gemm_events(a, b)
+                gev.append((a, b))
+            fn(i)
+            if with_gemm_events:
+                q.set_gemm_events(None, None)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        launches = q.launch_count() - n0
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        g_ms = [a.elapsed_time(b) for a, b in gev]
+        return ms, launches, g_ms
+
+    W = max(3, args.warmup)
+    with ClockSampler(local) as clk:
+        ms, launches, _ = timed(step, args.steps, W)
+    clocks = clk.summary()
+    # Dominant kernel: the fused NF4-decode GEMM of the forward (its last launch in each
+    # step is the dX GEMM, the first the forward one; the hook records the latest launch,
+    # so time the forward alone with the hook on).
+    _, _, g_ms = timed(lambda i: q.qlora_linear_fwd(sets[i % NSETS]["w"], sets[i % NSETS]["X"],
+                                                    sets[i % NSETS]["A"], sets[i % NSETS]["B"], alpha,
+                                                    H=H, U_save=U, ws=ws),
+                       args.steps, W, with_gemm_events=True)
+    # forward alone and backward alone (device time)
+    fwd_ms, _, _ = timed(lambda i: q.qlora_linear_fwd(sets[i % NSETS]["w"], sets[i % NSETS]["X"],
+                                                      sets[i % NSETS]["A"], sets[i % NSETS]["B"], alpha,
+                                                      H=H, U_save=U, ws=ws), args.steps, W)
+    bwd_ms, _, _ = timed(lambda i: q.qlora_linear_bwd(sets[i % NSETS]["w"], sets[i % NSETS]["X"],
+                                                      sets[i % NSETS]["dH"], sets[i % NSETS]["A"],
+                                                      sets[i % NSETS]["B"], alpha, U_saved=U, dX=dX,
+                                                      dA=dA, dB=dB, ws=ws), args.steps, W)
+
+    # ------------------------------------------------------------------ end to end
+    # Each step: pinned host X, dH -> device, fwd + bwd through the C ABI, dA, dB -> host.
+    hX = [sets[i]["X"].cpu().pin_memory() for i in range(2)]
+    hdH = [sets[i]["dH"].cpu().pin_memory() for i in range(2)]
+    hdA = torch.empty_like(dA, device="cpu").pin_memory()
+    hdB = torch.empty_like(dB, device="cpu").pin_memory()
+    Xd = torch.empty_like(sets[0]["X"])
+    dHd = torch.empty_like(sets[0]["dH"])
+
+    def e2e_step(i):
+        s = sets[i % NSETS]
+        Xd.copy_(hX[i % 2], non_blocking=True)
+        dHd.copy_(hdH[i % 2], non_blocking=True)
+        q.qlora_linear_fwd(s["w"], Xd, s["A"], s["B"], alpha, H=H, U_save=U, ws=ws)
+        q.qlora_linear_bwd(s["w"], Xd, dHd, s["A"], s["B"], alpha, U_saved=U, dX=dX, dA=dA, dB=dB, ws=ws)
+        if world > 1:
+            dist.all_reduce(dA)
+            dist.all_reduce(dB)
+        hdA.copy_(dA, non_blocking=True)
+        hdB.copy_(dB, non_blocking=True)
+
+    e2e_ms, _, _ = timed(e2e_step, args.steps, W)
+
+    extra = {}
+    if args.extra and rank == 0:
+        extra = extra_rows(q, torch, S, dev, peaks, args)
+
+    toks = T * args.steps * world
+    value = toks / (ms / 1e3)
+    gemm_flops = 2 * T * d * k + 2 * T * r * d           # base GEMM + adapter K-extension
+    g_avg = statistics.mean(g_ms) if g_ms else None
+    achieved = gemm_flops / (g_avg / 1e3) / 1e12 if g_avg else None
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": (achieved / peak) if achieved else None, "traffic": None,
+                "kernel": "k_tc_gemm<NF4 fwd> (fused decode + adapter K-extension)",
+                "peak_source": f"{peak_src} bf16_tflops_sustained",
+                "kernel_ms": g_avg}
+    step_flops = flops_fwd(T, d, k, r) + flops_bwd(T, d, k, r)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": W, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD + " fwd+bwd", "d_out": d, "d_in": k, "r": r, "alpha": alpha,
+                   "tokens_per_rank": T, "parallelism": f"dp{world}",
+                   "l2": "4 rotating input sets (~300 MB) > 2x L2"},
+        "tflops": step_flops * args.steps * world / (ms / 1e3) / 1e12,
+        "fwd_ms": fwd_ms / args.steps, "bwd_ms": bwd_ms / args.steps,
+        "roofline": roofline,
+        "e2e": {"value": toks / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(Xd.numel() * 2 + dHd.numel() * 2),
+                "d2h_bytes_per_step": int(dA.numel() * 4 + dB.numel() * 4)},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if extra:
+        line["rows"] = extra
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def extra_rows(q, torch, S, dev, peaks, args):
+    """Other rows of the hot path, each timed on the device (not part of the headline)."""
+    out = {}
+    bf = torch.bfloat16
+    hbm = peaks["hbm_gbs"]
+    # decode-size forward on the 11008x4096 MLP shape, r = 64
+    c3 = S.CONFIGS["mlp_up_11008x4096_r64_T8192"]
+    d, k, r = c3["d_out"], c3["d_in"], c3["r"]
+    NW = 8  # rotate 8 weights (8 x 23 MB) so the stream comes from HBM, not L2
+    base = S.make_layer(d, k, r, c3["alpha"], 16, dtype="bf16", seed=7)
+    ws_list = [q.nf4_quantize(torch.from_numpy(base.W0).to(dev) * (1 + 0.01 * i)) for i in range(NW)]
+    A = torch.from_numpy(base.A).to(dev).to(bf)
+    B = torch.from_numpy(base.B).to(dev).to(bf)
+    for T in (1, 4, 16):
+        X = torch.from_numpy(base.X[:T]).to(dev).to(bf)
+        H = torch.empty((T, d), dtype=bf, device=dev)
+        ws = torch.empty(q.workspace_bytes(q.OP_FWD, q.BF16, T, d, k, r), dtype=torch.uint8, device=dev)
+        for i in range(5):
+            q.qlora_linear_fwd(ws_list[i % NW], X, A, B, c3["alpha"], H=H, ws=ws, save_u=False)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = 50
+        e0.record()
+        for i in range(n):
+            q.qlora_linear_fwd(ws_list[i % NW], X, A, B, c3["alpha"], H=H, ws=ws, save_u=False)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / n
+        byts = d * k * (0.5 + 1 / 64) + 4 * ((d * k // 64 + 255) // 256) + 2 * T * (k + d) + 2 * r * (d + k)
+        out[f"decode_T{T}_us"] = us
+        out[f"decode_T{T}_hbm_frac"] = byts / (us * 1e-6) / 1e9 / hbm
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--extra", action="store_true", help="also time the other hot-path rows")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
