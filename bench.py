@@ -108,7 +108,6 @@ class ClockSampler:
 
 def oracle_sample(n_tokens, seed=0):
     """One bounded-sample step of the oracle: decode W^ and fwd + bwd over n_tokens tokens."""
-    import numpy as np
     import oracle as O
     from qlora_parameter_efficient_b200 import synthetic as S
     c = cfg()
@@ -179,6 +178,7 @@ def run_gpu(args):
 
     import qlora_parameter_efficient_b200 as q
     from qlora_parameter_efficient_b200 import build as qb
+    from qlora_parameter_efficient_b200 import dp
     from qlora_parameter_efficient_b200 import synthetic as S
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -224,9 +224,7 @@ def run_gpu(args):
         q.qlora_linear_fwd(s["w"], s["X"], s["A"], s["B"], alpha, H=H, U_save=U, ws=ws)
         q.qlora_linear_bwd(s["w"], s["X"], s["dH"], s["A"], s["B"], alpha, U_saved=U, dX=dX, dA=dA,
                            dB=dB, ws=ws)
-        if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+        dp.allreduce_adapter_grads(dA, dB)
 
     def timed(fn, K, W, with_gemm_events=False):
         for i in range(W):
@@ -252,15 +250,27 @@ def run_gpu(args):
         e1.record(stream)
         torch.cuda.synchronize()
         launches = q.launch_count() - n0
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
+        ms = dp.max_over_ranks(e0.elapsed_time(e1), device=dev)
         g_ms = [a.elapsed_time(b) for a, b in gev]
         return ms, launches, g_ms
 
     W = max(3, args.warmup)
+    if args.only != "step":
+        # One part of the step alone (for profiling a single kernel on the same workload).
+        fn_fwd = lambda i: q.qlora_linear_fwd(sets[i % NSETS]["w"], sets[i % NSETS]["X"],  # noqa: E731
+                                              sets[i % NSETS]["A"], sets[i % NSETS]["B"], alpha,
+                                              H=H, U_save=U, ws=ws)
+        fn_bwd = lambda i: q.qlora_linear_bwd(sets[i % NSETS]["w"], sets[i % NSETS]["X"],  # noqa: E731
+                                              sets[i % NSETS]["dH"], sets[i % NSETS]["A"],
+                                              sets[i % NSETS]["B"], alpha, U_saved=U, dX=dX,
+                                              dA=dA, dB=dB, ws=ws)
+        ms, launches, _ = timed(fn_fwd if args.only == "fwd" else fn_bwd, args.steps, W)
+        if rank == 0:
+            print(json.dumps({"only": args.only, "ms_per_call": ms / args.steps,
+                              "launches": launches, "workload": WORKLOAD}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
     with ClockSampler(local) as clk:
         ms, launches, _ = timed(step, args.steps, W)
     clocks = clk.summary()
@@ -295,9 +305,7 @@ def run_gpu(args):
         dHd.copy_(hdH[i % 2], non_blocking=True)
         q.qlora_linear_fwd(s["w"], Xd, s["A"], s["B"], alpha, H=H, U_save=U, ws=ws)
         q.qlora_linear_bwd(s["w"], Xd, dHd, s["A"], s["B"], alpha, U_saved=U, dX=dX, dA=dA, dB=dB, ws=ws)
-        if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+        dp.allreduce_adapter_grads(dA, dB)
         hdA.copy_(dA, non_blocking=True)
         hdB.copy_(dB, non_blocking=True)
 
@@ -389,6 +397,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--extra", action="store_true", help="also time the other hot-path rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--only", default="step", choices=["step", "fwd", "bwd"],
+                    help="time only the forward or only the backward call")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
