@@ -150,6 +150,25 @@ qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t
                                       const int32_t* r, const float* alpha, qlora_dtype dtype,
                                       void* H, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Size of the device scratch array behind qlora_linear_fwd_noalloc (bytes per GPU). */
+#define QLORA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* qlora_linear_fwd without a workspace argument, for callers that cannot allocate device
+ * memory (an engine that owns all device memory through its own pool, or a hot path that
+ * must not take the allocator's locks) and have none to lend.  It allocates nothing: its
+ * scratch is a fixed QLORA_NOALLOC_SCRATCH_BYTES device array inside the library, held by
+ * every GPU that loads the library until the process exits.  The pages have no counterpart;
+ * the computation and the other arguments are exactly those of qlora_linear_fwd.
+ *   - QLORA_ERR_UNSUPPORTED, with nothing launched, when qlora_workspace_bytes(QLORA_OP_FWD,
+ *     dtype, T, d_out, d_in, r) exceeds QLORA_NOALLOC_SCRATCH_BYTES.
+ *   - All calls share the array; calls whose work overlaps on the GPU race on it.
+ *   - The first call on a device looks up the array's device address; make it before any
+ *     stream capture.                                                                        */
+qlora_status qlora_linear_fwd_noalloc(const qlora_nf4* w, const void* X, int64_t T,
+                                      const void* A, const void* B, int32_t r, float alpha,
+                                      qlora_dtype dtype, void* H, void* U_save,
+                                      cudaStream_t stream);
+
 /* Synchronise `stream`, then read and clear the device error word of the current device.
  * Returns QLORA_OK, QLORA_ERR_TIMEOUT, QLORA_ERR_DEVICE or QLORA_ERR_CUDA.                   */
 qlora_status qlora_get_device_error(cudaStream_t stream);

@@ -27,7 +27,7 @@ OP_FWD, OP_BWD, OP_FWD_BATCHED, OP_MERGE = 0, 1, 2, 3
 # Every symbol include/qlora.h declares.
 EXPORTS = ["qlora_nf4_sizes", "qlora_nf4_levels", "nf4_quantize", "nf4_dequantize",
            "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "lora_merge",
-           "qlora_linear_fwd_batched", "qlora_get_device_error",
+           "qlora_linear_fwd_batched", "qlora_linear_fwd_noalloc", "qlora_get_device_error",
            "qlora_selftest_wait_timeout", "qlora_set_gemm_events", "qlora_launch_count",
            "qlora_status_string"]
 
@@ -69,6 +69,7 @@ def load() -> ctypes.CDLL:
         "qlora_linear_fwd_batched": ([pnf4, vp, i64, vp, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                       ctypes.POINTER(i32), ctypes.POINTER(f32), ctypes.c_int, vp, vp, sz, vp],
                                      ctypes.c_int),
+        "qlora_linear_fwd_noalloc": ([pnf4, vp, i64, vp, vp, i32, f32, ctypes.c_int, vp, vp, vp], ctypes.c_int),
         "qlora_get_device_error": ([vp], ctypes.c_int),
         "qlora_selftest_wait_timeout": ([ctypes.c_uint64, vp], ctypes.c_int),
         "qlora_set_gemm_events": ([vp, vp], ctypes.c_int),
