@@ -52,32 +52,45 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
+// Longest time one try_wait may park the thread before returning "not yet" (ns); the phase
+// completing wakes it earlier.
+constexpr uint32_t kSuspendHintNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
-        : "r"(addr), "r"(parity)
+        : "r"(addr), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
 
 // Wait for the phase with the given parity to complete.  Gives up (returns false) when
-// *abort becomes non-zero or after limit_ns nanoseconds; never spins without bound.
+// *abort becomes non-zero or after limit_ns nanoseconds; never spins without bound.  Each
+// try_wait parks the thread in hardware until the phase completes or the hint expires.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns) {
     const uint32_t addr = smem_u32(bar);
     if (mbar_try_wait(addr, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(addr, parity)) return true;
+        if (mbar_try_wait(addr, parity)) return true;
         if (abort != nullptr && *abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }
+}
+
+// Warp-wide wait: lane 0 polls, the other lanes are released by __syncwarp (which orders
+// memory among the warp's threads) once it has seen the phase complete.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort, uint64_t limit_ns) {
+    uint32_t ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, limit_ns) ? 1u : 0u;
+    __syncwarp();
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 // ------------------------------------------------------------------ proxies and fences

@@ -1,0 +1,528 @@
+// nf4_gemm2.cuh -- persistent 2-SM (tcgen05 cta_group::2) fused NF4-decode GEMM.
+//
+//   forward (B_MN = false):  H[T, d_out]  = X[T, d_in]  W^T + sU[T, RP] B_pad[d_out, RP]^T
+//   dX      (B_MN = true):   dX[T, d_in]  = dH[T, d_out] W  + sG[T, RP] A_pad[RP, d_in]
+//
+// A cluster of two CTAs (a "pair") computes 256 x 256 output tiles with 256x256x16 UMMA
+// instructions issued by the leader CTA.  Each CTA holds half of the A tile (128 token rows)
+// and half of the B tile (128 of the 256 weight columns), so each SM decodes only its half of
+// the weight tile and every decoded weight feeds 256 tokens; each CTA's tensor memory holds
+// its 128 accumulator rows x 256 columns, double-buffered (512 columns) so the epilogue of one
+// tile overlaps the main loop of the next.  The grid is persistent: pair p handles tiles
+// p, p + npairs, ...
+//
+// Warp roles per CTA (6 + 4 x decoder groups warps):
+//   warp 0       TMA producer: this CTA's A half and NF4 code tile (or the K-extension
+//                adapter tiles) into an 8-stage ring, completing on the local full[s]; the
+//                decoded B halves live in a separate, shallower 3-slot ring (the adapter K
+//                step's B tile is loaded straight into its slot).
+//   warp 1       leader CTA only: issues the MMAs, commits stage release (empty[s]) and
+//                accumulator-ready (accf[b]) to both CTAs.
+//   warps 2..5   epilogue: TMEM -> bf16 -> global, then release the accumulator buffer to the
+//                leader (acc_empty[b]).
+//   warps 6..    NF4 decoders in groups of four warps that take K steps in turn: wait
+//                for the stage's code tile, decode 128 blocks of 64 weights into the stage's
+//                B half (one block per thread, written in the 128-byte-swizzled UMMA layout),
+//                then arrive on a local barrier: the leader's ready[s] directly, the peer's
+//                dec_done[s], which the peer's warp 1 forwards to the leader's ready[s] with
+//                one cluster-scope release.  For the adapter K steps the group only reports
+//                "landed".  ready[s] thus certifies, for both CTAs, that the A half has
+//                landed and the B half is in place.
+// Every wait is bounded (QLORA_ERR_TIMEOUT on expiry); all TMA loads are plain local loads.
+#pragma once
+
+#include "common.cuh"
+#include "nf4.cuh"
+
+namespace qlora {
+
+// ------------------------------------------------------------------ cluster / 2-SM PTX
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire (for barriers that remote CTAs arrive on).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort, uint64_t limit_ns) {
+    const uint32_t addr = smem_u32(bar);
+    if (mbar_try_wait_acq_cluster(addr, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_acq_cluster(addr, parity)) return true;
+        if (abort != nullptr && *abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+__device__ __forceinline__ void cluster_barrier() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_2sm(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_2sm() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_2sm(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_ss_2sm(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on the barrier at this offset in both CTAs of the pair when all previously
+// issued tcgen05 operations of this thread have completed.
+__device__ __forceinline__ void umma_commit_2sm_both(uint64_t* bar) {
+    const uint16_t mask = 0x3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(mask)
+        : "memory");
+}
+
+// ------------------------------------------------------------------ kernel
+
+#ifndef QLORA_G2_DEC_GROUPS
+#define QLORA_G2_DEC_GROUPS 4
+#endif
+constexpr int kG2DecGroups = QLORA_G2_DEC_GROUPS;   // groups of 4 decoder warps
+#ifndef QLORA_G2_STAGES_A
+#define QLORA_G2_STAGES_A 8
+#endif
+#ifndef QLORA_G2_STAGES_B
+#define QLORA_G2_STAGES_B 4
+#endif
+constexpr int kG2StagesA = QLORA_G2_STAGES_A;   // A half + NF4 codes: covers the TMA latency
+constexpr int kG2StagesB = QLORA_G2_STAGES_B;   // decoded B half: covers the signalling latency
+static_assert(kG2StagesA >= kG2StagesB, "B-slot reuse is gated through the A ring");
+// Each decoder group waits on full[] of the steps it handles; with the ring depth a multiple
+// of the group count, the previous phase of every such barrier belongs to a step the same
+// group has already observed, so no parity wait can alias.
+static_assert(kG2StagesA % kG2DecGroups == 0, "A-ring depth must be a multiple of the groups");
+constexpr int kG2Threads = 32 * (6 + 4 * kG2DecGroups);
+
+struct G2Smem {
+    static constexpr int kA = 128 * 64 * 2;       // this CTA's A half, one K step
+    static constexpr int kC = 128 * 64 / 2;       // NF4 codes of the B half
+    static constexpr int kB = 128 * 64 * 2;       // this CTA's decoded B half
+    static constexpr int kStageA = kA + kC;
+    static constexpr int kBars = 512;
+    static constexpr int kTotal = 1024 + kG2StagesA * kStageA + kG2StagesB * kB + kBars;
+    static_assert(kTotal <= 232448, "shared memory budget");
+};
+
+struct Gemm2Args {
+    int M, N;              // output rows (tokens) and columns
+    int k_steps;           // main K steps of 64
+    int ext_steps;         // adapter K-extension steps of 64
+    int ext_k16_last;      // K=16 MMAs in the last extension step
+    int m_tiles, n_tiles;  // 256 x 256 tiles
+    const uint8_t* absmax_q;
+    const float* c2;
+    int nf4_rows;          // d_out of the stored weight
+    int nf4_bpr;           // d_in / 64
+    __nv_bfloat16* out;
+    int64_t ld_out;
+    int* err;
+    uint64_t wait_ns;
+};
+
+template <bool B_MN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
+    k_nf4_gemm2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmC,
+                const __grid_constant__ CUtensorMap tmAx, const __grid_constant__ CUtensorMap tmBx,
+                const Gemm2Args args) {
+    using L = G2Smem;
+    constexpr int SA = kG2StagesA;
+    constexpr int SB = kG2StagesB;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;                          // [SA][kA]
+    uint8_t* sB = smem + SA * L::kA;             // [SB][kB]
+    uint8_t* sC = sB + SB * L::kB;               // [SA][kC]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sC + SA * L::kC);
+    uint64_t* full = bars;                  // [SA] local: A half + codes (or ext tiles) landed
+    uint64_t* empty = full + SA;            // [SA] both: A stage consumed by the MMAs
+    uint64_t* ready = empty + SA;           // [SA] leader: both halves ready for this K step
+    uint64_t* dec_done = ready + SA;        // [SA] peer: its decoder warps finished the step
+    uint64_t* accf = dec_done + SA;         // [2]  both: accumulator buffer complete
+    uint64_t* acc_empty = accf + 2;         // [2]  leader: buffer drained (8 warp arrivals)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();          // 0 = leader, 1 = peer
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int n_tiles_total = args.m_tiles * args.n_tiles;
+    const int iters_per_tile = args.k_steps + args.ext_steps;
+    const int my_tiles = (n_tiles_total - pair + npairs - 1) / npairs;
+    const int total_iters = max(0, my_tiles) * iters_per_tile;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&ready[s], 5);      // 4 leader decoder warps + the peer's forwarder
+            mbar_init(&dec_done[s], 4);   // 4 peer decoder warps
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acc_empty[b], 8);
+        }
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmC);
+        if (args.ext_steps > 0) {
+            tma_prefetch_desc(&tmAx);
+            tma_prefetch_desc(&tmBx);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc_2sm(tmem_slot, 512);
+        tmem_relinquish_2sm();
+    }
+    tc_fence_before();
+    cluster_barrier();          // barriers of both CTAs initialised; TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    auto fail = [&]() {
+        set_error(args.err, kErrTimeout);
+        *abort = 1;
+    };
+    // Decoded-B slot git % SB is free once the MMAs of step git - SB (its previous user) have
+    // completed, i.e. once empty[] of that step's A stage has fired.  Every waiter here is
+    // already past full[] of step git, so the MMAs of step git - SA are done and this barrier
+    // is at most one phase behind the awaited one: the parity test cannot alias.
+    auto wait_slot_free = [&](int git) -> bool {
+        if (git < SB) return true;
+        const int g = git - SB;
+        return mbar_wait(&empty[g % SA], (g / SA) & 1, abort, args.wait_ns);
+    };
+    auto wait_slot_free_warp = [&](int git) -> bool {
+        if (git < SB) return true;
+        const int g = git - SB;
+        return mbar_wait_warp(&empty[g % SA], (g / SA) & 1, abort, args.wait_ns);
+    };
+
+    if (warp == 0) {
+        // -------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int git = 0; git < total_iters; ++git) {
+                const int it = git % iters_per_tile;
+                const int tile = pair + (git / iters_per_tile) * npairs;
+                const int m0 = (tile % args.m_tiles) * 256 + static_cast<int>(rank) * 128;
+                const int n0 = (tile / args.m_tiles) * 256 + static_cast<int>(rank) * 128;
+                const int s = git % SA;
+                const uint32_t ph = (git / SA) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort, args.wait_ns)) {
+                    fail();
+                    break;
+                }
+                uint8_t* a = sA + s * L::kA;
+                uint8_t* c = sC + s * L::kC;
+                if (it < args.k_steps) {
+                    const int kx = it * 64;
+                    mbar_arrive_expect_tx(&full[s], L::kA + L::kC);
+                    tma_load_2d(a, &tmA, &full[s], kx, m0);
+                    if (B_MN) tma_load_2d(c, &tmC, &full[s], n0 / 2, kx);
+                    else tma_load_2d(c, &tmC, &full[s], kx / 2, n0);
+                } else {
+                    // adapter K step: the B tile goes straight into its decoded-B slot, once
+                    // the slot's previous user (step git - SB) has been consumed
+                    if (!wait_slot_free(git)) {
+                        fail();
+                        break;
+                    }
+                    uint8_t* b = sB + (git % SB) * L::kB;
+                    const int kx = (it - args.k_steps) * 64;
+                    mbar_arrive_expect_tx(&full[s], L::kA + L::kB);
+                    tma_load_2d(a, &tmAx, &full[s], kx, m0);
+                    if (B_MN) {
+                        tma_load_2d(b, &tmBx, &full[s], n0, kx);
+                        tma_load_2d(b + 8192, &tmBx, &full[s], n0 + 64, kx);
+                    } else {
+                        tma_load_2d(b, &tmBx, &full[s], kx, n0);
+                    }
+                }
+                issued = git + 1;
+            }
+            if (*abort) {
+                for (int g = max(0, issued - SA); g < issued; ++g)
+                    mbar_wait(&full[g % SA], (g / SA) & 1, nullptr, args.wait_ns);
+            }
+        }
+    } else if (warp == 1) {
+        if (rank == 0 && lane == 0) {
+            // ---------------------------------------------------------- MMA issuer (leader)
+            const uint32_t idesc = make_idesc_bf16(256, 256, false, B_MN);
+            int git = 0;
+            bool ok = true;
+            for (int tc = 0; ok && tc < my_tiles; ++tc) {
+                const int buf = tc & 1;
+                const uint32_t aph = (tc >> 1) & 1;
+                if (!mbar_wait_cluster(&acc_empty[buf], aph ^ 1, abort, args.wait_ns)) {
+                    fail();
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * 256);
+                for (int it = 0; it < iters_per_tile; ++it, ++git) {
+                    const int s = git % SA;
+                    const int sb = git % SB;
+                    if (!mbar_wait_cluster(&ready[s], (git / SA) & 1, abort, args.wait_ns)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a = smem_u32(sA + s * L::kA);
+                    const uint32_t b = smem_u32(sB + sb * L::kB);
+                    const int nk = (it == iters_per_tile - 1 && it >= args.k_steps) ? args.ext_k16_last : 4;
+                    for (int k = 0; k < nk; ++k) {
+                        const uint64_t ad = make_sw128_desc(a + k * 32, 16, 1024);
+                        const uint64_t bd = B_MN ? make_sw128_desc(b + k * 2048, 8192, 1024)
+                                                 : make_sw128_desc(b + k * 32, 16, 1024);
+                        umma_bf16_ss_2sm(d_tmem, ad, bd, idesc, (it > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit_2sm_both(&empty[s]);
+                }
+                umma_commit_2sm_both(&accf[buf]);
+            }
+        }
+        if (rank == 1 && lane == 0) {
+            // ---------------------------------------------------------- peer forwarder
+            // One cluster-scope release per K step on the leader's ready[s].
+            const uint32_t ready_leader = mapa_shared(smem_u32(&ready[0]), 0);
+            for (int git = 0; git < total_iters; ++git) {
+                const int s = git % SA;
+                if (!mbar_wait(&dec_done[s], (git / SA) & 1, abort, args.wait_ns)) {
+                    fail();
+                    break;
+                }
+                mbar_arrive_remote(ready_leader + static_cast<uint32_t>(s * 8));
+            }
+        }
+    } else if (warp < 6) {
+        // -------------------------------------------------------------- epilogue
+        const int q = warp & 3;                    // TMEM lane quarter of this warp
+        const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
+        for (int tc = 0; tc < my_tiles; ++tc) {
+            const int tile = pair + tc * npairs;
+            const int buf = tc & 1;
+            const uint32_t aph = (tc >> 1) & 1;
+            if (!mbar_wait_warp(&accf[buf], aph, abort, args.wait_ns)) {
+                fail();
+                break;
+            }
+            tc_fence_after();
+            const int mt = tile % args.m_tiles, nt = tile / args.m_tiles;
+            const int64_t grow = static_cast<int64_t>(mt) * 256 + rank * 128 + q * 32 + lane;
+            const int gc0 = nt * 256;
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(buf * 256);
+#pragma unroll 1
+            for (int c0 = 0; c0 < 256; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tbase + c0, r);
+                tmem_ld_wait();
+                if (grow < args.M) {
+                    const int gc = gc0 + c0;
+                    __nv_bfloat16* o = args.out + grow * args.ld_out + gc;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        if (gc + 8 * g < args.N) {
+                            uint4 v;
+                            v.x = pack_bf16x2(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
+                            v.y = pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
+                            v.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
+                            v.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
+                            *reinterpret_cast<uint4*>(o + 8 * g) = v;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acc_empty_leader + static_cast<uint32_t>(buf * 8));
+        }
+    } else {
+        // -------------------------------------------------------------- NF4 decoders
+        const int grp = (warp - 6) >> 2;
+        const int j = ((warp - 6) & 3) * 32 + lane;      // 0..127: block of this thread
+        int row_in_tile, blk_col_off;
+        if (B_MN) {
+            row_in_tile = j >> 1;           // weight row (K) within the step
+            blk_col_off = j & 1;            // which 64-wide chunk of this CTA's 128 columns
+        } else {
+            row_in_tile = j;                // weight row within this CTA's 128
+            blk_col_off = 0;
+        }
+        auto block_at = [&](int git) -> int64_t {
+            const int it = git % iters_per_tile;
+            if (it >= args.k_steps) return -1;
+            const int tile = pair + (git / iters_per_tile) * npairs;
+            const int n0 = (tile / args.m_tiles) * 256 + static_cast<int>(rank) * 128;
+            int64_t wrow, wblk;
+            if (B_MN) {
+                wrow = static_cast<int64_t>(it) * 64 + row_in_tile;
+                wblk = n0 / 64 + blk_col_off;
+            } else {
+                wrow = n0 + row_in_tile;
+                wblk = it;
+            }
+            if (wrow >= args.nf4_rows || wblk >= args.nf4_bpr) return -1;
+            return wrow * args.nf4_bpr + wblk;
+        };
+        uint64_t* arrive_bar = rank == 0 ? ready : dec_done;   // local arrive either way
+        // Software pipeline per handled step: the step's 64 weights are decoded into registers
+        // as soon as its code tile has landed -- before its decoded-B slot is free -- so the
+        // slot is held only for the stores; the next block's tables are built after that.
+        uint4 dec[8];
+        auto decode_into_regs = [&](int git, int64_t blk, const Nf4Planes& p) {
+            const int s = git % SA;
+            const uint8_t* c = sC + s * L::kC;
+            const uint8_t* src = B_MN ? c + row_in_tile * 64 + blk_col_off * 32 : c + row_in_tile * 32;
+            if (blk >= 0) {
+                const uint4 q0 = *reinterpret_cast<const uint4*>(src);
+                const uint4 q1 = *reinterpret_cast<const uint4*>(src + 16);
+                dec[0] = nf4_decode8(q0.x, p);
+                dec[1] = nf4_decode8(q0.y, p);
+                dec[2] = nf4_decode8(q0.z, p);
+                dec[3] = nf4_decode8(q0.w, p);
+                dec[4] = nf4_decode8(q1.x, p);
+                dec[5] = nf4_decode8(q1.y, p);
+                dec[6] = nf4_decode8(q1.z, p);
+                dec[7] = nf4_decode8(q1.w, p);
+            } else {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) dec[ch] = make_uint4(0, 0, 0, 0);
+            }
+        };
+        int64_t blk_nxt = grp < total_iters ? block_at(grp) : -1;
+        uint32_t q8_nxt = 0;
+        float c2_nxt = 0.f;
+        if (blk_nxt >= 0) {
+            q8_nxt = __ldg(args.absmax_q + blk_nxt);
+            c2_nxt = __ldg(args.c2 + (blk_nxt >> 8));
+        }
+        bool have = false;          // dec[] holds step `git` (decoded ahead)
+        for (int git = grp; git < total_iters; git += kG2DecGroups) {
+            const int s = git % SA;
+            const int it = git % iters_per_tile;
+            const bool main_step = it < args.k_steps;
+            if (!have) {
+                // (first step, or after an adapter step) decode now
+                const int64_t blk = blk_nxt;
+                Nf4Planes p{};
+                if (blk >= 0) p = nf4_make_planes(nf4_block_scale(q8_nxt, c2_nxt));
+                const int gn = git + kG2DecGroups;
+                blk_nxt = gn < total_iters ? block_at(gn) : -1;
+                if (blk_nxt >= 0) {
+                    q8_nxt = __ldg(args.absmax_q + blk_nxt);
+                    c2_nxt = __ldg(args.c2 + (blk_nxt >> 8));
+                }
+                if (!mbar_wait_warp(&full[s], (git / SA) & 1, abort, args.wait_ns)) {
+                    fail();
+                    break;
+                }
+                if (main_step) decode_into_regs(git, blk, p);
+            }
+            if (main_step) {
+                if (!wait_slot_free_warp(git)) {
+                    fail();
+                    break;
+                }
+                uint8_t* dst_row = sB + (git % SB) * L::kB +
+                                   (B_MN ? blk_col_off * 8192 + row_in_tile * 128 : row_in_tile * 128);
+                const uint32_t sw = row_in_tile & 7;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(dst_row + ((ch ^ sw) << 4)) = dec[ch];
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&arrive_bar[s]);
+            // decode the next handled step ahead, as soon as its codes have landed
+            have = false;
+            const int gn = git + kG2DecGroups;
+            if (gn < total_iters && (gn % iters_per_tile) < args.k_steps) {
+                const int64_t blk = blk_nxt;
+                Nf4Planes p{};
+                if (blk >= 0) p = nf4_make_planes(nf4_block_scale(q8_nxt, c2_nxt));
+                const int g2 = gn + kG2DecGroups;
+                blk_nxt = g2 < total_iters ? block_at(g2) : -1;
+                if (blk_nxt >= 0) {
+                    q8_nxt = __ldg(args.absmax_q + blk_nxt);
+                    c2_nxt = __ldg(args.c2 + (blk_nxt >> 8));
+                }
+                if (!mbar_wait_warp(&full[gn % SA], (gn / SA) & 1, abort, args.wait_ns)) {
+                    fail();
+                    break;
+                }
+                decode_into_regs(gn, blk, p);
+                have = true;
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    if (*abort) {
+        // give in-flight copies of the pair time to land before shared memory is released
+        __nanosleep(100000);
+    }
+    tc_fence_before();
+    cluster_barrier();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_2sm(tmem_base, 512);
+    }
+}
+
+}  // namespace qlora

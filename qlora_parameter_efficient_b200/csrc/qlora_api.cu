@@ -13,6 +13,7 @@
 #include "nf4.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
+#include "nf4_gemm2.cuh"
 
 using namespace qlora;
 
@@ -25,7 +26,6 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kSmsForSplit = 148;         // split-K is sized for a B200's 148 SMs
 constexpr uint64_t kWaitNs = 4000000000ull;
-constexpr int kNf4Stages = 4;
 constexpr int kTmaStages = 4;
 
 std::atomic<uint64_t> g_launches{0};
@@ -276,7 +276,7 @@ qlora_status skinny_gemm(bool a_mn, bool b_mn, int RP, const CUtensorMap& ta,
     return QLORA_ERR_UNSUPPORTED;
 }
 
-// Fused NF4-decode GEMM with the adapter K-extension.
+// Fused NF4-decode GEMM with the adapter K-extension (persistent 2-SM kernel).
 //   forward (dx = false): out[T, d_out]  = act[T, d_in]  W^T + ext_a[T, RP] ext_b[d_out, RP]^T
 //   dX      (dx = true):  out[T, d_in]   = act[T, d_out] W   + ext_a[T, RP] ext_b[RP, d_in]
 qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, const void* ext_a,
@@ -286,24 +286,47 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
     CUtensorMap ta, tc, tax, tbx;
     const int64_t K = dx ? d_out : d_in;
     const int64_t N = dx ? d_in : d_out;
-    QL_TRY(tmap_bf16(&ta, act, T, K, K, kBM));
-    if (dx) QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 128, 64));
-    else QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 32, 256));
-    QL_TRY(tmap_bf16(&tax, ext_a, T, RP, RP, kBM));
+    QL_TRY(tmap_bf16(&ta, act, T, K, K, 128));
+    if (dx) QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 64, 64));
+    else QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 32, 128));
+    QL_TRY(tmap_bf16(&tax, ext_a, T, RP, RP, 128));
     if (dx) QL_TRY(tmap_bf16(&tbx, ext_b, RP, d_in, d_in, 64));
-    else QL_TRY(tmap_bf16(&tbx, ext_b, d_out, RP, RP, 256));
-    GemmArgs g = base_args(static_cast<int>(T), static_cast<int>(N), static_cast<int>(cdiv(K, kBK)), err);
+    else QL_TRY(tmap_bf16(&tbx, ext_b, d_out, RP, RP, 128));
+    Gemm2Args g{};
+    g.M = static_cast<int>(T);
+    g.N = static_cast<int>(N);
+    g.k_steps = static_cast<int>(cdiv(K, 64));
     g.ext_steps = RP / 64;
     g.ext_k16_last = static_cast<int>(std::min<int64_t>(4, cdiv(r_used - 64 * (g.ext_steps - 1), 16)));
+    g.m_tiles = static_cast<int>(cdiv(T, 256));
+    g.n_tiles = static_cast<int>(cdiv(N, 256));
     g.absmax_q = w->absmax_q;
     g.c2 = w->c2;
     g.nf4_rows = static_cast<int>(d_out);
     g.nf4_bpr = static_cast<int>(d_in / 64);
-    g.out = out;
+    g.out = static_cast<__nv_bfloat16*>(out);
     g.ld_out = N;
-    dim3 grid(static_cast<unsigned>(cdiv(N, 256)), static_cast<unsigned>(cdiv(T, kBM)), 1);
-    if (dx) return launch_gemm<false, true, kBNf4, 256, kNf4Stages, false>(ta, tc, tax, tbx, g, grid, st, true);
-    return launch_gemm<false, false, kBNf4, 256, kNf4Stages, false>(ta, tc, tax, tbx, g, grid, st, true);
+    g.err = err;
+    g.wait_ns = kWaitNs;
+    const int tiles = g.m_tiles * g.n_tiles;
+    const int pairs = std::max(1, std::min(tiles, kSmsForSplit / 2));
+    auto kern = dx ? k_nf4_gemm2<true> : k_nf4_gemm2<false>;
+    static std::atomic<uint64_t> configured[2] = {0, 0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured[dx].load() & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G2Smem::kTotal) !=
+            cudaSuccess)
+            return QLORA_ERR_CUDA;
+        configured[dx].fetch_or(bit);
+    }
+    const bool ev = g_ev_start && g_ev_stop;
+    if (ev) cudaEventRecord(g_ev_start, st);
+    kern<<<2 * pairs, kG2Threads, G2Smem::kTotal, st>>>(ta, tc, tax, tbx, g);
+    QL_LAUNCH_CHECK();
+    if (ev) cudaEventRecord(g_ev_stop, st);
+    return QLORA_OK;
 }
 
 // ======================================================================= fp32 helpers
