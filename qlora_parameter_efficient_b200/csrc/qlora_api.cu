@@ -14,6 +14,7 @@
 #include "simt.cuh"
 #include "tc_gemm.cuh"
 #include "nf4_gemm2.cuh"
+#include "qgemv.cuh"
 
 using namespace qlora;
 
@@ -117,6 +118,21 @@ qlora_status tmap_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t col
     return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// byte matrix [rows, cols_bytes] with the 128-byte swizzle, box = 128 bytes x box_y rows.
+qlora_status tmap_u8_sw128(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                           uint32_t box_y) {
+    QL_TRY(get_encoder());
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
+    cuuint32_t box[2] = {128, box_y};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 // ======================================================================= planning
 
 int choose_split(int64_t tiles, int64_t k_steps) {
@@ -129,8 +145,27 @@ int choose_split(int64_t tiles, int64_t k_steps) {
 
 int pad_rank(int r) { return r <= 64 ? 64 : 128; }
 
+// Decode-size forward (bf16, T <= 32): stream-K split of (128-row tile x 64-K) units.
+constexpr int kSmallT = 32;
+struct SmallPlan {
+    int nt = 16, kt = 0, kt4 = 0, rt = 0, units = 0, grid = 0, tiles_per_cta = 0;
+};
+SmallPlan make_small_plan(int64_t T, int64_t d_out, int64_t d_in) {
+    SmallPlan sp;
+    sp.nt = T <= 16 ? 16 : 32;
+    sp.kt = static_cast<int>(d_in / 64);
+    sp.kt4 = static_cast<int>(cdiv(sp.kt, 4));
+    sp.rt = static_cast<int>(cdiv(d_out, 128));
+    sp.units = sp.kt4 * sp.rt;
+    sp.grid = std::max(1, std::min(sp.units, kSmsForSplit));
+    sp.tiles_per_cta = static_cast<int>(cdiv(sp.units, sp.grid) / sp.kt4) + 2;
+    return sp;
+}
+
 struct Plan {
     int RP = 0;
+    bool small = false;
+    size_t s_us = 0, s_cnt = 0, s_part = 0;
     int split_u = 1, split_g = 1, split_da = 1, split_db = 1;
     size_t a_pad = 0, b_pad = 0, u_spad = 0, u_pad = 0, g_spad = 0, part = 0;
     size_t w32 = 0, uf = 0, gf = 0;
@@ -146,6 +181,15 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
         return o;
     };
     if (op == QLORA_OP_MERGE) return p;
+    if (op == QLORA_OP_FWD && dtype == QLORA_BF16 && T <= kSmallT) {
+        const SmallPlan sp = make_small_plan(T, d_out, d_in);
+        p.small = true;
+        p.s_us = take(static_cast<size_t>(T) * r * 4);
+        p.s_cnt = take(static_cast<size_t>(sp.rt) * 4);
+        p.s_part = take(static_cast<size_t>(sp.grid) * sp.tiles_per_cta * 128 * sp.nt * 4);
+        p.total = off;
+        return p;
+    }
     if (dtype == QLORA_BF16) {
         p.RP = pad_rank(r);
         const int64_t RP = p.RP;
@@ -329,6 +373,73 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
     return QLORA_OK;
 }
 
+// Decode-size forward: U pre-pass (also zeroes the tile counters) overlapped with the
+// weight stream through programmatic dependent launch.
+qlora_status small_fwd(const qlora_nf4* w, const void* X, int64_t T, const void* A, const void* B,
+                       int r, float s, void* H, void* U_save, const Plan& p, void* ws, int* err,
+                       cudaStream_t st) {
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    const SmallPlan sp = make_small_plan(T, d_out, d_in);
+    float* us = at<float>(ws, p.s_us);
+    int* counters = at<int>(ws, p.s_cnt);
+    float* part = at<float>(ws, p.s_part);
+    k_small_u<<<dim3(static_cast<unsigned>(r), static_cast<unsigned>(cdiv(T, 4))), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(X), static_cast<int>(T),
+                                 static_cast<int>(d_in), static_cast<const __nv_bfloat16*>(A), r, s,
+                                 us, static_cast<__nv_bfloat16*>(U_save), counters, sp.rt);
+    QL_LAUNCH_CHECK();
+    CUtensorMap tc, tx;
+    QL_TRY(tmap_u8_sw128(&tc, w->codes, d_out, d_in / 2, d_in / 2, 128));
+    QL_TRY(tmap_bf16(&tx, X, T, d_in, d_in, static_cast<uint32_t>(sp.nt)));
+    GvArgs g{};
+    g.T = static_cast<int>(T);
+    g.d_out = static_cast<int>(d_out);
+    g.d_in = static_cast<int>(d_in);
+    g.kt = sp.kt;
+    g.kt4 = sp.kt4;
+    g.rt = sp.rt;
+    g.units = sp.units;
+    g.tiles_per_cta = sp.tiles_per_cta;
+    g.absmax_q = w->absmax_q;
+    g.c2 = w->c2;
+    g.part = part;
+    g.counters = counters;
+    g.us = us;
+    g.B = static_cast<const __nv_bfloat16*>(B);
+    g.r = r;
+    g.H = static_cast<__nv_bfloat16*>(H);
+    g.err = err;
+    g.wait_ns = kWaitNs;
+    // one CTA per SM: each holds all 512 tensor-memory columns
+    const int smem = std::max(1024 + kGvLut + kGvStagesC * kGvBlk * (sp.nt * 128 + 128 * 32) + kGvUsMax * 4 + 512, 120 * 1024);
+    auto kern = sp.nt == 16 ? k_qgemv<16> : k_qgemv<32>;
+    static std::atomic<uint64_t> configured[2] = {0, 0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    const int which = sp.nt == 16 ? 0 : 1;
+    if (!(configured[which].load() & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        configured[which].fetch_or(bit);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sp.grid));
+    cfg.blockDim = dim3(kGvThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const bool ev = g_ev_start && g_ev_stop;
+    if (ev) cudaEventRecord(g_ev_start, st);
+    if (cudaLaunchKernelEx(&cfg, kern, tc, tx, g) != cudaSuccess) return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    if (ev) cudaEventRecord(g_ev_stop, st);
+    return QLORA_OK;
+}
+
 // ======================================================================= fp32 helpers
 
 qlora_status sgemm(cudaStream_t st, int64_t M, int64_t N, int64_t K, float alpha, const float* A,
@@ -472,6 +583,8 @@ qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T, cons
     QL_TRY(err_word(&err));
     const int64_t d_out = w->d_out, d_in = w->d_in;
     const float s = alpha / static_cast<float>(r);
+    if (p.small)
+        return small_fwd(w, X, T, A, B, r, s, H, U_save, p, ws, err, stream);
     if (dtype == QLORA_BF16) {
         const int RP = p.RP;
         auto* a_pad = at<__nv_bfloat16>(ws, p.a_pad);
