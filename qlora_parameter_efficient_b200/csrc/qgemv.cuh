@@ -1,35 +1,43 @@
 // qgemv.cuh -- decode-size forward (T <= 32 tokens): an HBM-bound stream over the NF4 codes.
 //
-//   H[t, n] = sum_b s_b(n) * sum_{k in b} L16(code(n, k)) x[t, k]  +  (s U[t, :]) . B[n, :]
+//   H[t, n] = (1/127) sum_b q8_b(n) c2_b(n) sum_{k in b} L16(code(n, k)) x[t, k]
+//             + (s U[t, :]) . B[n, :]
 //
 // With a handful of tokens every weight is used T times, so the layer is a weight stream
-// (0.516 B per weight) and the decode must keep up with HBM: about 44 weights per SM cycle.
-// The exact per-block table of the large-T kernels (a bf16 product per level and block) costs
-// ~2 integer ops per weight, too many here.  This kernel factors the block scale out of the
-// block's dot product instead -- dequantize = LUT(code) x s_b ("Low-Rank Adaptation (LoRA) and
+// (0.516 B per weight) and the decode has to keep pace with HBM.  The block scale is factored
+// out of the block's dot product -- dequantize = L(code) x s_b ("Low-Rank Adaptation (LoRA) and
 // QLoRA: Mathematical Foundations...", section "1. 4-bit NormalFloat (NF4) Quantization";
-// the block scale is that of "2. Double Quantization (DQ)") evaluated as
-// s_b * sum(LUT(code) x): a fixed 256-entry table maps a code byte to its two levels as a
-// bf16 pair (one shared-memory load per two weights, replicated per lane so a warp's loads
-// never conflict), the tensor cores form the block's partial dot products, and s_b multiplies
-// the fp32 partial.  Identical in exact arithmetic; the levels are rounded to bf16 before the
-// scale instead of after (relative 2^-9 per weight, averaging out in the sum).
+// s_b = q8_b c2_b / 127 is the block constant of "2. Double Quantization (DQ)"): each weight
+// decodes to its unscaled level rounded to bf16, the tensor cores form the block's partial dot
+// product in fp32, q8_b c2_b multiplies the fp32 partial and the common 1/127 is applied once to
+// the output.  Identical in exact arithmetic; the level is rounded to bf16 before the scale
+// instead of after (relative 2^-9 per weight, averaging out in the sum).
 //
-// Work: units of (128 weight rows) x (256 K) = four NF4 blocks per row, i.e. 128 contiguous code
-// bytes per row (whole cache lines; the code stream is read once, straight from HBM), with one
-// accumulator per block so each block's scale applies to its own partial; a persistent grid splits
-// the unit sequence (row tile major) into equal contiguous ranges.  Per CTA (448 threads):
-//   warp 0       TMA: the unit's code tile (128 x 128 B, 128-byte swizzle) and X tiles
-//                (4 x N x 64 bf16, rows past T zero-filled) into a 4-stage ring.
-//   warp 1       issues tcgen05.mma (M = 128, N = 16/32, K = 16, A from tensor memory) into a
-//                per-unit accumulator (a ring of four in tensor memory).
-//   warps 2..9   decoders in two groups of four warps taking units in turn: one row per
-//                thread; 32 table loads per block give the row's 64 bf16, written to tensor
-//                memory with one tcgen05.st per block (A operand, 2 stages of 4 x 32 columns).
-//   warps 10..13 accumulate: read the unit's partial from tensor memory, add s_b * partial in
-//                fp32.  At the end of a row tile's range they write a partial row; the last CTA
-//                to finish a tile (semaphore) sums the partials in CTA order, adds the adapter
-//                term and writes H -- deterministic.
+// Why warp-level mma.sync and not tcgen05 here: one tcgen05.mma of M = 128, K = 16 occupies
+// the SM's tensor core for ~130-190 cycles whatever N is (measured on B200 with N = 16..256),
+// i.e. at most ~16 weights per cycle when the weights are the M x K operand -- well below the
+// stream rate.  mma.sync m16n8k16 (~900 MAC per SM cycle measured) takes its operands from
+// registers, so the codes decode (byte-permute arithmetic on the symmetric level table) straight
+// into A fragments.
+//
+// K order inside a block.  The dot product over a block's 64 K is order-free, so K is permuted
+// consistently in A and X: in k16 step j, mma K positions {2c, 2c+1, 2c+8, 2c+9} (thread c of
+// a quad) are block elements 16c + 4j + {0, 1, 2, 3}.  A thread's 8 code bytes 8c..8c+7 of a row
+// then supply its A registers of all four steps, and its X fragment is the 16 consecutive
+// elements 16c..16c+15 of the token's row.
+//
+// Work split.  The rows are cut into tiles of M rows (a multiple of 16, chosen per shape so
+// that the tiles fill the SMs); a cluster of C CTAs (C = 1, 2, 4 or 8) owns a contiguous range
+// of tiles and CTA rank p owns K blocks [kb_lo, kb_hi) of every row.  Warp w owns the blocks
+// kb_lo + w + 8j: their X fragments are loaded once into registers and stay there.  A stage is
+// 16 consecutive rows x the rank's K range -- 16 contiguous runs, one 3-D TMA box (pieces of 128
+// bytes, 128-byte swizzle, so the fragment reads are bank-conflict free); the warps take turns
+// issuing the refills.  Across the M/16 stages of a tile each warp accumulates q8 c2 x partial
+// in fp32 registers; the tile's absmax bytes and c2 values come in once per tile by cp.async.
+// At the end of a tile the 8 warps combine by a fixed tree in shared memory, the ranks' sums
+// meet in rank 0's shared memory over DSMEM, and rank 0 sums them in rank order, applies 1/127,
+// adds the adapter term (a few mma steps) and writes H.  No global partials, atomics or
+// semaphores: the sums are deterministic and the tail is on-chip.
 #pragma once
 
 #include "common.cuh"
@@ -37,461 +45,486 @@
 
 namespace qlora {
 
-constexpr int kGvBlk = 4;       // NF4 blocks per row per unit: 128 contiguous code bytes
-constexpr int kGvStagesC = 4;   // code + X tiles
-constexpr int kGvStagesA = 2;   // decoded A tiles in tensor memory (4 x 32 columns each)
-constexpr int kGvDecGroups = 2; // groups of 4 decoder warps taking units in turn
-constexpr int kGvDBufs = 2;     // per-unit accumulators in tensor memory (4 x NT columns)
-constexpr int kGvEpiWarp = 2 + 4 * kGvDecGroups;     // first accumulate warp
-constexpr int kGvThreads = 32 * (kGvEpiWarp + 4);
-// Decoder group g handles units g, g + groups, ...; with both ring depths multiples of the
-// group count the previous phase of every barrier a group waits on is one it has seen.
-static_assert(kGvStagesC % kGvDecGroups == 0 && kGvStagesA % kGvDecGroups == 0, "ring depths");
-constexpr int kGvLut = 256 * 32 * 4;   // 256 entries x 32 lanes x 4 bytes
-constexpr int kGvUsMax = 32 * 128;     // s*U staging: T <= 32 tokens x r <= 128
+constexpr int kGvWarps = 8;
+constexpr int kGvThreads = 32 * kGvWarps;
+constexpr int kGvUsMax = 32 * 128; // s*U staging (bf16): T <= 32 tokens x r <= 128
+constexpr int kGvTabAbs = 16384;   // a tile's absmax bytes: M x (kb_hi - kb_lo) <= this
+constexpr int kGvTabC2 = 320;      // a tile's c2 groups: M x kt / 256 + 2 <= this
 
-__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-        "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-// D[tmem] (+)= A[tmem] * B[smem desc]^T, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                             uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
+template <int NT8>
+struct GvCfg {
+    static constexpr int NT = 8 * NT8;                 // token tile
+    static constexpr int NBW = 8 / NT8;                // blocks per warp (X fragments in registers)
+    static constexpr int kMaxBlk = 8 * NBW;            // blocks of a CTA's K range
+    static constexpr int MW = NT8 == 1 ? 8 : (NT8 == 2 ? 6 : 3);   // max 16-row groups per tile
+    static constexpr int kStage = 16 * kMaxBlk * 32;   // 16 rows x the K range (<= 32 KB)
+    static constexpr int S = NT8 == 1 ? 5 : (NT8 == 2 ? 7 : 8);
+    static constexpr int kMaxRanks = NT8 == 1 ? 4 : 8;  // cluster size limit
+    static constexpr int kSlot = 32 * MW * NT8 * 16;   // one warp's accumulators
+    static constexpr int kTree = 4 * kSlot;            // tree slots
+    static constexpr int kRing = kMaxRanks * kSlot;    // rank 0: one CTA sum per rank
+    static constexpr int kStageOff = 0;
+    static constexpr int kTreeOff = kStageOff + S * kStage;
+    static constexpr int kRingOff = kTreeOff + kTree;
+    static constexpr int kUsOff = kRingOff + kRing;
+    static constexpr int kTabOff = kUsOff + kGvUsMax * 2;   // the tile's absmax [M][nbk] bytes
+    static constexpr int kC2Off = kTabOff + kGvTabAbs;      // the tile's c2 groups
+    static constexpr int kBarOff = kC2Off + kGvTabC2 * 4;
+    static constexpr int kSmem = kBarOff + 256 + 1024;   // barriers + alignment slack
+    static_assert(kSmem <= 227 * 1024, "shared memory budget");
+};
+
 __device__ __forceinline__ void griddep_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// 4-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros without reading.
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x),
+                 "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1, bool acc) {
+    if (acc) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+            "{%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+            "{%8,%9}, {%10,%10,%10,%10};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+    }
+}
 
 struct GvArgs {
-    int T;                  // tokens (1..NT)
-    int d_out, d_in, kt;    // kt = d_in / 64 blocks per row
-    int kt4;                // units per row tile: ceil(kt / kGvBlk)
-    int rt;                 // row tiles of 128
-    int units;              // rt * kt4
-    int tiles_per_cta;      // partial slots per CTA
+    int T;                   // tokens (1..NT)
+    int d_out, d_in, kt;     // kt = d_in / 64 blocks per row (a multiple of 4)
+    int M;                   // rows per tile (multiple of 16, <= MMAX)
+    int tiles;               // ceil(d_out / M)
+    int C;                   // CTAs per cluster (K ranks)
+    int clusters;            // grid / C
+    int pieces;              // 128-byte pieces per row in a stage box: ceil(kt / 4 / C)
+    const __nv_bfloat16* X;  // [T][d_in]
     const uint8_t* absmax_q;
     const float* c2;
-    float* part;            // [grid][tiles_per_cta][128][NT]
-    int* counters;          // [rt], zeroed by the pre-pass
-    const float* us;        // [T][r]  s * U in fp32, from the pre-pass
-    const __nv_bfloat16* B; // [d_out][r]
+    const float* us;         // [T][r]  s * U in fp32, from the pre-pass
+    const __nv_bfloat16* B;  // [d_out][r]
     int r;
-    __nv_bfloat16* H;       // [T][d_out]
+    int b_vec;               // r % 8 == 0 (B rows are 16-byte aligned)
+    __nv_bfloat16* H;        // [T][d_out]
     int* err;
     uint64_t wait_ns;
 };
 
-__device__ __forceinline__ int gv_start(int c, int units, int grid) {
-    return static_cast<int>((static_cast<int64_t>(c) * units) / grid);
-}
-
-template <int NT>
+template <int NT8>
 __global__ void __launch_bounds__(kGvThreads, 1)
-    k_qgemv(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
-            const GvArgs args) {
-    static_assert(NT == 16 || NT == 32, "token tile");
-    constexpr int SC = kGvStagesC, SA = kGvStagesA, ND = kGvDBufs;
-    constexpr int kCodes = 128 * 32 * kGvBlk;     // bytes per unit (128 rows x 128 B)
-    constexpr int kXb = NT * 128;                 // bytes per block (NT rows x 64 bf16)
-    constexpr int kX = kXb * kGvBlk;              // bytes per unit
-    constexpr uint32_t kTmemCols = 512;
-    constexpr uint32_t kACols = 32 * kGvBlk;      // tensor-memory columns per A stage
-    constexpr uint32_t kDCols = NT * kGvBlk;      // tensor-memory columns per accumulator set
-    constexpr uint32_t kDCol = kACols * kGvStagesA;   // accumulators after the A stages
-    static_assert(kDCol + kDCols * kGvDBufs <= kTmemCols, "tensor memory budget");
+    k_qgemv(const __grid_constant__ CUtensorMap tmC, const GvArgs args) {
+    using Cf = GvCfg<NT8>;
+    constexpr int S = Cf::S, MW = Cf::MW, NT = Cf::NT, NBW = Cf::NBW;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem);          // [256][32]
-    uint8_t* sX = smem + kGvLut;                                 // [SC][kX]
-    uint8_t* sC = sX + SC * kX;                                  // [SC][kCodes]
-    float* s_us = reinterpret_cast<float*>(sC + SC * kCodes);   // [T][r] s*U (reduction only)
-    uint64_t* bars = reinterpret_cast<uint64_t*>(s_us + kGvUsMax);
-    uint64_t* full = bars;                 // [SC] codes + X landed
-    uint64_t* empty = full + SC;           // [SC] decoders (4) + MMA (1) done with the stage
-    uint64_t* a_full = empty + SC;         // [SA] decoded rows in tensor memory (4 warps)
-    uint64_t* a_free = a_full + SA;        // [SA] MMA done with the stage
-    uint64_t* d_full = a_free + SA;        // [ND] unit accumulator ready
-    uint64_t* d_free = d_full + ND;        // [ND] accumulator read (4 warps)
-    uint64_t* seg_bar = d_free + ND;       // [2]  accumulate warps meet at a row-tile end
-    uint64_t* us_bar = seg_bar + 2;        // [1]  s*U staged (used once)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(us_bar + 1);
-    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* last_flag = abort + 1;
+    uint8_t* stages = smem + Cf::kStageOff;
+    float4* tree = reinterpret_cast<float4*>(smem + Cf::kTreeOff);           // [4][MW][NT8][32]
+    float4* ring = reinterpret_cast<float4*>(smem + Cf::kRingOff);           // [ranks][MW][NT8][32]
+    __nv_bfloat16* s_us = reinterpret_cast<__nv_bfloat16*>(smem + Cf::kUsOff);   // [NT][rp]
+    uint8_t* tab_abs = smem + Cf::kTabOff;                                   // [M][nbk]
+    float* tab_c2 = reinterpret_cast<float*>(smem + Cf::kC2Off);             // [groups]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::kBarOff);
+    uint64_t* full = bars;                     // [S] the stage's code box landed
+    uint64_t* empty = full + S;                // [S] all warps done with the stage
+    uint64_t* csync_bar = empty + S;           // the 8 warps meet
+    uint64_t* ring_full = csync_bar + 1;       // rank 0: every rank's sum of the tile is in
+    uint64_t* ring_free = ring_full + 1;       // every rank: rank 0 has consumed the ring
+    volatile int* abort = reinterpret_cast<volatile int*>(ring_free + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int u0 = gv_start(blockIdx.x, args.units, gridDim.x);
-    const int u1 = gv_start(blockIdx.x + 1, args.units, gridDim.x);
-    const int n_units = u1 - u0;
+    const int g = lane >> 2, c = lane & 3;          // mma fragment coordinates
+    const int C = args.C;
+    const int rank = static_cast<int>(blockIdx.x) % C;      // cluster dims (C, 1, 1)
+    const int cl = static_cast<int>(blockIdx.x) / C;
+    const int t_lo = static_cast<int>((static_cast<int64_t>(cl) * args.tiles) / args.clusters);
+    const int t_hi = static_cast<int>((static_cast<int64_t>(cl + 1) * args.tiles) / args.clusters);
+    const int q4 = args.kt / 4;
+    const int kb_lo = 4 * ((rank * q4) / C), kb_hi = 4 * (((rank + 1) * q4) / C);
+    const int nbk = kb_hi - kb_lo;
+    const int M = args.M, mw = M / 16;
+    const int n_units = (t_hi - t_lo) * mw;          // (tile, 16-row group) sequence
 
-    // level-pair table: entry b = (bf16(L[b & 15]), bf16(L[b >> 4])), one copy per lane
-    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-        const int b = i >> 5;
-        lut[i] = pack_bf16x2(c_nf4_levels[b & 15], c_nf4_levels[b >> 4]);
-    }
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < SC; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 5);
-        }
-        for (int s = 0; s < SA; ++s) {
-            mbar_init(&a_full[s], 4);
-            mbar_init(&a_free[s], 1);
-        }
-        for (int b = 0; b < ND; ++b) {
-            mbar_init(&d_full[b], 1);
-            mbar_init(&d_free[b], 4);
-        }
-        for (int b = 0; b < 2; ++b) mbar_init(&seg_bar[b], 4);
-        mbar_init(us_bar, 4);
-        *abort = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmC);
-        tma_prefetch_desc(&tmX);
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
     auto fail = [&]() {
         set_error(args.err, kErrTimeout);
         *abort = 1;
     };
+    // ---- stage issue (one warp in turn, lane 0): 16 full rows of the rank's K range as one box
+    auto issue = [&](int u) {
+        if (lane != 0) return;
+        const int s = u % S;
+        const int row0 = (t_lo + u / mw) * M + (u % mw) * 16;
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(16 * 128 * args.pieces));
+        tma_load_3d(stages + s * Cf::kStage, &tmC, &full[s], 0, row0, kb_lo / 4);
+    };
 
-    if (warp == 0) {
-        // ------------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int i = 0; i < n_units; ++i) {
-                const int u = u0 + i;
-                const int tile = u / args.kt4, ks = u % args.kt4;
-                const int s = i % SC;
-                if (!mbar_wait(&empty[s], ((i / SC) & 1) ^ 1, abort, args.wait_ns)) {
-                    fail();
-                    break;
-                }
-                mbar_arrive_expect_tx(&full[s], kCodes + kX);
-                tma_load_2d(sC + s * kCodes, &tmC, &full[s], ks * 32 * kGvBlk, tile * 128);
-#pragma unroll
-                for (int b = 0; b < kGvBlk; ++b)
-                    tma_load_2d(sX + s * kX + b * kXb, &tmX, &full[s], (ks * kGvBlk + b) * 64, 0);
-                issued = i + 1;
-            }
-            if (*abort)
-                for (int g = max(0, issued - SC); g < issued; ++g)
-                    mbar_wait(&full[g % SC], (g / SC) & 1, nullptr, args.wait_ns);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kGvWarps);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc_bf16(128, NT, false, false);
-            for (int i = 0; i < n_units; ++i) {
-                const int s = i % SC, sa = i % SA, db = i % ND;
-                bool ok = mbar_wait(&full[s], (i / SC) & 1, abort, args.wait_ns);
-                ok = ok && mbar_wait(&a_full[sa], (i / SA) & 1, abort, args.wait_ns);
-                ok = ok && mbar_wait(&d_free[db], ((i / ND) & 1) ^ 1, abort, args.wait_ns);
-                if (!ok) {
-                    fail();
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t xs = smem_u32(sX + s * kX);
-                for (int b = 0; b < kGvBlk; ++b)
-                    for (int k = 0; k < 4; ++k)
-                        umma_bf16_ts(tmem + kDCol + db * kDCols + static_cast<uint32_t>(b * NT),
-                                     tmem + sa * kACols + static_cast<uint32_t>(b * 32 + k * 8),
-                                     make_sw128_desc(xs + b * kXb + k * 32, 16, 1024), idesc,
-                                     k > 0 ? 1u : 0u);
-                umma_commit(&empty[s]);
-                umma_commit(&a_free[sa]);
-                umma_commit(&d_full[db]);
-            }
-        }
-    } else if (warp < kGvEpiWarp) {
-        // ------------------------------------------------------------------ decoders
-        const int q = warp & 3;
-        const int grp = (warp - 2) >> 2;
-        const int row = q * 32 + lane;
-        const uint32_t tlane = static_cast<uint32_t>(q * 32) << 16;
-        const uint32_t* mylut = lut + lane;
-        for (int i = grp; i < n_units; i += kGvDecGroups) {
-            const int s = i % SC, sa = i % SA;
-            if (!mbar_wait_warp(&full[s], (i / SC) & 1, abort, args.wait_ns)) {
-                fail();
-                break;
-            }
-            if (!mbar_wait_warp(&a_free[sa], ((i / SA) & 1) ^ 1, abort, args.wait_ns)) {
-                fail();
-                break;
-            }
-            // row's 128 code bytes (4 blocks): one 32-column tensor-memory store per block
-            // (the code tile is stored with the 128-byte swizzle: chunk j of row r sits at
-            //  chunk j ^ (r & 7), so a warp's reads spread over all banks)
-            const uint8_t* crow = sC + s * kCodes + row * 32 * kGvBlk;
-            const uint32_t sw = static_cast<uint32_t>(row & 7);
-#pragma unroll
-            for (int b = 0; b < kGvBlk; ++b) {
-                const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (((2 * b) ^ sw) << 4));
-                const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2 * b + 1) ^ sw) << 4));
-                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint32_t v[32];
-#pragma unroll
-                for (int w = 0; w < 8; ++w) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) v[4 * w + e] = mylut[((cw[w] >> (8 * e)) & 0xFFu) * 32];
-                }
-                tmem_st_32x32b_x32(tmem + tlane + sa * kACols + static_cast<uint32_t>(b * 32), v);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);         // codes consumed
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[sa]);
-        }
-    } else {
-        // ------------------------------------------------------------------ accumulate
-        const int q = warp & 3;
-        const int row = q * 32 + lane;
-        const int et = threadIdx.x - 32 * kGvEpiWarp;     // 0..127 within the 4 warps
-        const uint32_t tlane = static_cast<uint32_t>(q * 32) << 16;
-        float acc[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-        bool waited_primary = false;
-        bool us_staged = false;
-        int tile_slot = 0;
-        // bounded meeting point of the four accumulate warps (no hardware barrier that a warp
-        // leaving on a timeout could strand the others at)
-        auto epi_sync = [&](int which, int seg) -> bool {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&seg_bar[which]);
-            return mbar_wait_warp(&seg_bar[which], static_cast<uint32_t>(seg & 1), abort, args.wait_ns);
-        };
-        // Block-scale inputs of a unit (kGvBlk consecutive blocks of this row), loaded two
-        // units ahead (an L2 round trip is longer than a unit) and rotated through registers.
-        struct ScaleIn {
-            uint32_t q8[kGvBlk];
-            float c2[kGvBlk];
-        };
-        auto load_scale = [&](int i) -> ScaleIn {
-            ScaleIn v;
-#pragma unroll
-            for (int b = 0; b < kGvBlk; ++b) {
-                v.q8[b] = 0u;
-                v.c2[b] = 0.f;
-            }
-            if (i < n_units) {
-                const int u = u0 + i;
-                const int64_t grow = static_cast<int64_t>(u / args.kt4) * 128 + row;
-                const int kb0 = (u % args.kt4) * kGvBlk;
-                if (grow < args.d_out) {
-#pragma unroll
-                    for (int b = 0; b < kGvBlk; ++b) {
-                        if (kb0 + b < args.kt) {
-                            const int64_t blk = grow * args.kt + kb0 + b;
-                            v.q8[b] = __ldg(args.absmax_q + blk);
-                            v.c2[b] = __ldg(args.c2 + (blk >> 8));
-                        }
-                    }
-                }
-            }
-            return v;
-        };
-        ScaleIn p0 = load_scale(0), p1 = load_scale(1);
-        for (int i = 0; i < n_units; ++i) {
-            const int u = u0 + i;
-            const int db = i % ND;
-            float sc[kGvBlk];
-#pragma unroll
-            for (int b = 0; b < kGvBlk; ++b) sc[b] = nf4_block_scale(p0.q8[b], p0.c2[b]);
-            p0 = p1;
-            p1 = load_scale(i + 2);
-            if (!mbar_wait_warp(&d_full[db], (i / ND) & 1, abort, args.wait_ns)) {
-                fail();
-                break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int b = 0; b < kGvBlk; ++b) {
-                const uint32_t dcol = kDCol + db * kDCols + static_cast<uint32_t>(b * NT);
-                uint32_t r0[16], r1[16];
-                tmem_ld_32x32b_x16(tmem + tlane + dcol, r0);
-                if constexpr (NT == 32) tmem_ld_32x32b_x16(tmem + tlane + dcol + 16, r1);
-                tmem_ld_wait();
-#pragma unroll
-                for (int t = 0; t < 16; ++t) acc[t] = fmaf(sc[b], __uint_as_float(r0[t]), acc[t]);
-                if constexpr (NT == 32) {
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) acc[16 + t] = fmaf(sc[b], __uint_as_float(r1[t]), acc[16 + t]);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&d_free[db]);
-            // end of this CTA's range inside the row tile?
-            const int tile = u / args.kt4;
-            const bool seg_end = (u + 1 == u1) || ((u + 1) % args.kt4 == 0);
-            if (!seg_end) continue;
-            float* pp = args.part + ((static_cast<int64_t>(blockIdx.x) * args.tiles_per_cta + tile_slot) * 128 + row) * NT;
-#pragma unroll
-            for (int t = 0; t < NT; t += 4)
-                *reinterpret_cast<float4*>(pp + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
-#pragma unroll
-            for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-            const int seg = tile_slot++;
-            __threadfence();
-            if (!epi_sync(0, seg)) {
-                fail();
-                break;
-            }
-            if (et == 0) {
-                if (!waited_primary) griddep_wait();     // counters / s*U from the pre-pass
-                // CTAs whose ranges touch this tile
-                const int first_u = tile * args.kt4, last_u = min(args.units, (tile + 1) * args.kt4) - 1;
-                int c_first = static_cast<int>((static_cast<int64_t>(first_u) * gridDim.x) / args.units);
-                while (c_first + 1 < static_cast<int>(gridDim.x) && gv_start(c_first + 1, args.units, gridDim.x) <= first_u) ++c_first;
-                while (gv_start(c_first, args.units, gridDim.x) > first_u) --c_first;
-                int c_last = static_cast<int>((static_cast<int64_t>(last_u) * gridDim.x) / args.units);
-                while (c_last + 1 < static_cast<int>(gridDim.x) && gv_start(c_last + 1, args.units, gridDim.x) <= last_u) ++c_last;
-                while (gv_start(c_last, args.units, gridDim.x) > last_u) --c_last;
-                const int need = c_last - c_first + 1;
-                const int done = atomicAdd(args.counters + tile, 1) + 1;
-                *last_flag = (done == need) ? (c_first + 1) : 0;    // 0: not last
-                if (done == need) *(last_flag + 1) = c_last;
-            }
-            waited_primary = true;
-            if (!epi_sync(1, seg)) {
-                fail();
-                break;
-            }
-            const int lf = *last_flag;
-            if (lf == 0) continue;
-            __threadfence();
-            griddep_wait();
-            if (!us_staged) {      // s*U of all tokens into shared memory, once per CTA
-                for (int e = et; e < args.T * args.r; e += 128) s_us[e] = args.us[e];
-                us_staged = true;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(us_bar);
-                if (!mbar_wait_warp(us_bar, 0, abort, args.wait_ns)) {
-                    fail();
-                    break;
-                }
-            }
-            const int c_first = lf - 1, c_last = *(last_flag + 1);
-            const int64_t grow = static_cast<int64_t>(tile) * 128 + row;
-            if (grow < args.d_out) {
-                float out[NT];
-#pragma unroll
-                for (int t = 0; t < NT; ++t) out[t] = 0.f;
-                for (int c = c_first; c <= c_last; ++c) {
-                    const int slot = tile - gv_start(c, args.units, gridDim.x) / args.kt4;
-                    const float* src = args.part + ((static_cast<int64_t>(c) * args.tiles_per_cta + slot) * 128 + row) * NT;
-#pragma unroll
-                    for (int t = 0; t < NT; t += 4) {
-                        const float4 p4 = __ldcg(reinterpret_cast<const float4*>(src + t));
-                        out[t] += p4.x;
-                        out[t + 1] += p4.y;
-                        out[t + 2] += p4.z;
-                        out[t + 3] += p4.w;
-                    }
-                }
-                // adapter term: (s U[t, :]) . B[row, :], the B row in chunks of 8 from registers
-                const __nv_bfloat16* brow = args.B + grow * args.r;
-                for (int j0 = 0; j0 < args.r; j0 += 8) {
-                    float b8[8];
-                    if (j0 + 8 <= args.r && (args.r & 7) == 0) {
-                        const uint4 bv = __ldg(reinterpret_cast<const uint4*>(brow + j0));
-                        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bv);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(b2[e]);
-                            b8[2 * e] = f.x;
-                            b8[2 * e + 1] = f.y;
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) b8[e] = j0 + e < args.r ? __bfloat162float(brow[j0 + e]) : 0.f;
-                    }
-                    const int jn = min(8, args.r - j0);
-#pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        if (t < args.T) {
-                            const float* ust = s_us + t * args.r + j0;
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                if (e < jn) out[t] = fmaf(ust[e], b8[e], out[t]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int t = 0; t < NT; ++t)
-                    if (t < args.T)
-                        args.H[static_cast<int64_t>(t) * args.d_out + grow] = __float2bfloat16_rn(out[t]);
-            }
-        }
-        if (!waited_primary) griddep_wait();
+        mbar_init(csync_bar, kGvWarps);
+        mbar_init(ring_full, 32 * C);
+        mbar_init(ring_free, 1);
+        *abort = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmC);
+        for (int u = 0; u < S - 1 && u < n_units; ++u) issue(u);
     }
+    const Nf4Planes planes = nf4_make_planes(1.0f);
+    // X fragments of this warp's blocks, held for the whole kernel: token 8n + g, elements
+    // 16c .. 16c + 15 of block kb_lo + warp + 8j
+    uint32_t xw[NBW][NT8][8];
+#pragma unroll
+    for (int j = 0; j < NBW; ++j) {
+        const int L = warp + 8 * j;
+#pragma unroll
+        for (int n = 0; n < NT8; ++n) {
+            const int t = 8 * n + g;
+            uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
+            if (L < nbk && t < args.T) {
+                const uint4* src = reinterpret_cast<const uint4*>(args.X + static_cast<int64_t>(t) * args.d_in + (kb_lo + L) * 64 + 16 * c);
+                x0 = __ldg(src);
+                x1 = __ldg(src + 1);
+            }
+            xw[j][n][0] = x0.x; xw[j][n][1] = x0.y; xw[j][n][2] = x0.z; xw[j][n][3] = x0.w;
+            xw[j][n][4] = x1.x; xw[j][n][5] = x1.y; xw[j][n][6] = x1.z; xw[j][n][7] = x1.w;
+        }
+    }
+    // barriers initialised (and visible cluster-wide) before any remote arrive or store
+    if (C > 1) cluster_barrier();
+    else __syncthreads();
 
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+    uint32_t phase = 0;
+    // bounded meeting point of the 8 warps (no hardware barrier that a warp leaving on a timeout
+    // could strand the others at)
+    auto csync = [&]() -> bool {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(csync_bar);
+        const bool ok = mbar_spin(csync_bar, phase & 1, abort, args.wait_ns);
+        ++phase;
+        return ok;
+    };
+
+    float acc[MW][NT8][4];
+    int last_issued = -1;       // latest stage this warp issued (beyond the initial ones)
+    bool us_ready = false, ok_all = true;
+    int tiles_done = 0;
+
+    for (int tile = t_lo; tile < t_hi && ok_all; ++tile) {
+        const int row0 = tile * M;
+        // ---- the tile's absmax bytes [M][nbk] and c2 groups, by all threads (the previous
+        // tile's readers are past its end-of-tile meetings)
+        {
+            const int wpr = nbk / 4;
+            for (int wi = threadIdx.x; wi < M * wpr; wi += kGvThreads) {
+                const int rr = wi / wpr, q = wi % wpr;
+                const bool ok = row0 + rr < args.d_out;
+                cp_async_4(tab_abs + rr * nbk + 4 * q,
+                           args.absmax_q + (ok ? static_cast<int64_t>(row0 + rr) * args.kt + kb_lo + 4 * q : 0),
+                           ok ? 4u : 0u);
+            }
+        }
+        const int64_t rlast = min(row0 + M, args.d_out) - 1;
+        const int64_t g_first = (static_cast<int64_t>(row0) * args.kt + kb_lo) >> 8;
+        {
+            const int n_c2 = static_cast<int>(((rlast * args.kt + kb_hi - 1) >> 8) - g_first + 1);
+            for (int e = threadIdx.x; e < n_c2; e += kGvThreads) cp_async_4(tab_c2 + e, args.c2 + g_first + e, 4u);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if (!csync()) {
+            fail();
+            break;
+        }
+        if (rank == 0 && warp == 1 && lane == 0 && args.b_vec) {     // adapter rows, to L2
+            const int rows = min(M, args.d_out - row0);
+            bulk_prefetch_l2(args.B + static_cast<int64_t>(row0) * args.r, static_cast<uint32_t>(rows * args.r * 2));
+        }
+#pragma unroll
+        for (int m = 0; m < MW; ++m)
+#pragma unroll
+            for (int n = 0; n < NT8; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[m][n][e] = 0.f;
+
+        // ---- the tile's 16-row groups, one stage each
+#pragma unroll
+        for (int m = 0; m < MW; ++m) {
+            if (m >= mw) break;
+            const int u = (tile - t_lo) * mw + m;
+            const int s = u % S;
+            if (warp == u % kGvWarps && u + S - 1 < n_units) {
+                // refill the slot of stage u - 1 with stage u + S - 1 once every warp has left it
+                // (the warps take this duty in turn)
+                const int nxt = u + S - 1;
+                if (!mbar_wait_warp(&empty[nxt % S], ((nxt / S) & 1) ^ 1, abort, args.wait_ns)) {
+                    ok_all = false;
+                    break;
+                }
+                issue(nxt);
+                last_issued = nxt;
+            }
+            if (!mbar_wait_warp(&full[s], (u / S) & 1, abort, args.wait_ns)) {
+                ok_all = false;
+                break;
+            }
+            const uint8_t* st = stages + s * Cf::kStage;
+            const int ra_ = 16 * m + g, rb_ = ra_ + 8;          // rows within the tile
+            const int64_t base_a = static_cast<int64_t>(row0 + ra_) * args.kt;
+            const int64_t base_b = base_a + 8 * static_cast<int64_t>(args.kt);
+#pragma unroll
+            for (int j = 0; j < NBW; ++j) {
+                const int L = warp + 8 * j;
+                if (L >= nbk) break;
+                // stage layout [piece L/4][16 rows][128 B], 128-byte swizzle: block L of a row is
+                // 16-byte chunks 2(L%4), 2(L%4)+1, stored at chunk ^ (row & 7)
+                const uint8_t* piece = st + (L >> 2) * 2048;
+                const int chunk = ((((L & 3) * 2 + (c >> 1)) ^ g) << 4) + (c & 1) * 8;
+                const uint2 ca = *reinterpret_cast<const uint2*>(piece + g * 128 + chunk);
+                const uint2 cb = *reinterpret_cast<const uint2*>(piece + (g + 8) * 128 + chunk);
+                const uint4 a0 = nf4_decode8(ca.x, planes), a1 = nf4_decode8(ca.y, planes);
+                const uint4 b0 = nf4_decode8(cb.x, planes), b1 = nf4_decode8(cb.y, planes);
+                // A registers per k16 step: {row g: byte 2k, row g+8: byte 2k, row g: byte 2k+1,
+                // row g+8: byte 2k+1} of the thread's 8 bytes
+                const uint32_t A[4][4] = {{a0.x, b0.x, a0.y, b0.y}, {a0.z, b0.z, a0.w, b0.w},
+                                          {a1.x, b1.x, a1.y, b1.y}, {a1.z, b1.z, a1.w, b1.w}};
+                float tmp[NT8][4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int n = 0; n < NT8; ++n)
+                        mma_bf16_16816(tmp[n], A[k], xw[j][n][2 * k], xw[j][n][2 * k + 1], k > 0);
+                // q8 * c2 of rows ra_, rb_ from the tile's tables
+                const int kb = kb_lo + L;
+                const float sa = static_cast<float>(tab_abs[ra_ * nbk + L]) * tab_c2[((base_a + kb) >> 8) - g_first];
+                const float sb = static_cast<float>(tab_abs[rb_ * nbk + L]) * tab_c2[((base_b + kb) >> 8) - g_first];
+#pragma unroll
+                for (int n = 0; n < NT8; ++n) {
+                    acc[m][n][0] = fmaf(sa, tmp[n][0], acc[m][n][0]);
+                    acc[m][n][1] = fmaf(sa, tmp[n][1], acc[m][n][1]);
+                    acc[m][n][2] = fmaf(sb, tmp[n][2], acc[m][n][2]);
+                    acc[m][n][3] = fmaf(sb, tmp[n][3], acc[m][n][3]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        if (!ok_all) {
+            fail();
+            break;
+        }
+
+        // ---- end of the tile: the 8 warps' sums by a fixed tree.  Round with stride h: warps
+        // [h, 2h) hand their sums to warps [0, h).  The first round writes to tree slot
+        // (idx - h); later rounds write to the writer's own slot, which it read (and finished
+        // with) in the round before, so one meeting per round suffices.
+        bool first = true;
+        for (int h = kGvWarps / 2; h >= 1; h >>= 1) {
+            if (warp >= h && warp < 2 * h) {
+                float4* dst = tree + (first ? warp - h : warp) * (Cf::kSlot / 16);
+#pragma unroll
+                for (int m = 0; m < MW; ++m)
+#pragma unroll
+                    for (int n = 0; n < NT8; ++n)
+                        if (m < mw) dst[(m * NT8 + n) * 32 + lane] = make_float4(acc[m][n][0], acc[m][n][1], acc[m][n][2], acc[m][n][3]);
+            }
+            if (!csync()) {
+                ok_all = false;
+                break;
+            }
+            if (warp < h) {
+                const float4* src = tree + (first ? warp : warp + h) * (Cf::kSlot / 16);
+#pragma unroll
+                for (int m = 0; m < MW; ++m)
+#pragma unroll
+                    for (int n = 0; n < NT8; ++n)
+                        if (m < mw) {
+                            const float4 p = src[(m * NT8 + n) * 32 + lane];
+                            acc[m][n][0] += p.x;
+                            acc[m][n][1] += p.y;
+                            acc[m][n][2] += p.z;
+                            acc[m][n][3] += p.w;
+                        }
+            }
+            first = false;
+        }
+        if (!ok_all) {
+            fail();
+            break;
+        }
+        // ---- warp 0 sends the CTA's sum to rank 0 (its own ring slot when C == 1)
+        if (warp == 0) {
+            if (tiles_done > 0 && !mbar_wait_warp(ring_free, (tiles_done - 1) & 1, abort, args.wait_ns)) {
+                fail();
+                break;
+            }
+            const uint32_t dst = mapa_shared(smem_u32(ring + rank * (Cf::kSlot / 16) + lane), 0);
+#pragma unroll
+            for (int m = 0; m < MW; ++m)
+#pragma unroll
+                for (int n = 0; n < NT8; ++n)
+                    if (m < mw) st_cluster_v4(dst + ((m * NT8 + n) * 32) * 16, make_float4(acc[m][n][0], acc[m][n][1], acc[m][n][2], acc[m][n][3]));
+            mbar_arrive_remote(mapa_shared(smem_u32(ring_full), 0));   // release.cluster
+        }
+        ++tiles_done;
+        if (rank != 0) continue;
+
+        // ---- rank 0: finalize the tile -- ranks in order, 1/127, adapter term, H.  Warp w
+        // takes m16 tiles w, w + 8, ...
+        if (!mbar_wait_cluster(ring_full, (tiles_done - 1) & 1, abort, args.wait_ns)) {
+            fail();
+            break;
+        }
+        const int rp = (args.r + 15) & ~15;          // adapter rank padded to the mma K
+        if (!us_ready) {
+            // s*U from the pre-pass as bf16 [NT][rp] (zero beyond T and r), once per CTA
+            griddep_wait();
+            for (int e = threadIdx.x; e < NT * rp; e += kGvThreads) {
+                const int t = e / rp, j = e % rp;
+                s_us[e] = __float2bfloat16_rn(t < args.T && j < args.r ? args.us[t * args.r + j] : 0.f);
+            }
+            us_ready = true;
+            if (!csync()) {
+                fail();
+                break;
+            }
+        }
+        for (int m = warp; m < mw; m += kGvWarps) {
+            float4 tot[NT8];
+#pragma unroll
+            for (int n = 0; n < NT8; ++n) tot[n] = ring[(m * NT8 + n) * 32 + lane];
+            for (int rr = 1; rr < C; ++rr) {
+#pragma unroll
+                for (int n = 0; n < NT8; ++n) {
+                    const float4 v = ring[rr * (Cf::kSlot / 16) + (m * NT8 + n) * 32 + lane];
+                    tot[n].x += v.x;
+                    tot[n].y += v.y;
+                    tot[n].z += v.z;
+                    tot[n].w += v.w;
+                }
+            }
+            const int rbase = row0 + 16 * m;
+            // this thread's outputs: rows rbase + g, rbase + g + 8; tokens 8n + 2c, 8n + 2c + 1
+            float out[2][NT8][2];
+#pragma unroll
+            for (int n = 0; n < NT8; ++n) {
+                out[0][n][0] = __fdiv_rn(tot[n].x, 127.0f);
+                out[0][n][1] = __fdiv_rn(tot[n].y, 127.0f);
+                out[1][n][0] = __fdiv_rn(tot[n].z, 127.0f);
+                out[1][n][1] = __fdiv_rn(tot[n].w, 127.0f);
+            }
+            if (args.b_vec) {
+                // adapter term on the tensor cores: [16 rows x rp] B rows times [rp x NT]
+                // (s U)^T, fp32 accumulation
+                float adp[NT8][4];
+                for (int k0 = 0; k0 < rp; k0 += 16) {
+                    uint32_t a[4];
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const int row = rbase + g + 8 * (q2 & 1);
+                        const int col = k0 + 2 * c + 8 * (q2 >> 1);
+                        a[q2] = (row < args.d_out && col < args.r)
+                            ? __ldg(reinterpret_cast<const unsigned int*>(args.B + static_cast<int64_t>(row) * args.r + col)) : 0u;
+                    }
+#pragma unroll
+                    for (int n = 0; n < NT8; ++n) {
+                        const __nv_bfloat16* ub = s_us + (8 * n + g) * rp + k0 + 2 * c;
+                        mma_bf16_16816(adp[n], a, *reinterpret_cast<const uint32_t*>(ub),
+                                       *reinterpret_cast<const uint32_t*>(ub + 8), k0 > 0);
+                    }
+                }
+#pragma unroll
+                for (int n = 0; n < NT8; ++n) {
+                    out[0][n][0] += adp[n][0];
+                    out[0][n][1] += adp[n][1];
+                    out[1][n][0] += adp[n][2];
+                    out[1][n][1] += adp[n][3];
+                }
+            } else {
+                // r % 8 != 0: scalar adapter term
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int64_t grow = rbase + g + 8 * h;
+                    if (grow >= args.d_out) continue;
+                    const __nv_bfloat16* brow = args.B + grow * args.r;
+                    for (int j = 0; j < args.r; ++j) {
+                        const float bj = __bfloat162float(brow[j]);
+#pragma unroll
+                        for (int n = 0; n < NT8; ++n)
+#pragma unroll
+                            for (int e2 = 0; e2 < 2; ++e2)
+                                out[h][n][e2] = fmaf(__bfloat162float(s_us[(8 * n + 2 * c + e2) * rp + j]), bj, out[h][n][e2]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int64_t grow = rbase + g + 8 * h;
+                if (grow >= args.d_out) continue;
+#pragma unroll
+                for (int n = 0; n < NT8; ++n)
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int t = 8 * n + 2 * c + e2;
+                        if (t < args.T) args.H[static_cast<int64_t>(t) * args.d_out + grow] = __float2bfloat16_rn(out[h][n][e2]);
+                    }
+            }
+        }
+        // everyone is done with the ring: release it to every rank (the last tile needs none)
+        if (!csync()) {
+            fail();
+            break;
+        }
+        if (warp == 0 && lane < C && tile + 1 < t_hi)
+            mbar_arrive_remote(mapa_shared(smem_u32(ring_free), static_cast<uint32_t>(lane)));
+    }
+    if (lane == 0 && *abort) {
+        // leave no copy in flight into shared memory of an exiting CTA: the stages this warp
+        // issued (thread 0 also the initial ones) are waited for, each bounded
+        if (warp == 0)
+            for (int i = 0; i < min(S - 1, n_units); ++i)
+                mbar_wait(&full[i % S], (i / S) & 1, nullptr, args.wait_ns);
+        if (last_issued >= 0)
+            mbar_wait(&full[last_issued % S], (last_issued / S) & 1, nullptr, args.wait_ns);
     }
 }
 
 // Pre-pass for the decode-size forward: U = X A^T (fp32 accumulation), s U in fp32 for the
-// adapter term, U in the call dtype for the backward, and zeroed tile counters.  Grid
-// (r, ceil(T / 4)): each warp computes one (token, adapter row) dot product with all of its
-// loads in flight at once.  Lets the dependent stream kernel start immediately.
+// adapter term and U in the call dtype for the backward.  Grid (r, ceil(T / 4)): each warp
+// computes one (token, adapter row) dot product with all of its loads in flight at once.
+// Lets the dependent stream kernel start immediately.
 __global__ void __launch_bounds__(128) k_small_u(const __nv_bfloat16* __restrict__ X, int T,
                                                  int d_in, const __nv_bfloat16* __restrict__ A,
                                                  int r, float s, float* __restrict__ us,
-                                                 __nv_bfloat16* __restrict__ u_save,
-                                                 int* __restrict__ counters, int n_counters) {
+                                                 __nv_bfloat16* __restrict__ u_save) {
     griddep_launch_dependents();
     const int j = blockIdx.x;
     const int t = blockIdx.y * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (j == 0 && blockIdx.y == 0)
-        for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
     if (t >= T) return;
     const __nv_bfloat16* a = A + static_cast<int64_t>(j) * d_in;
     const __nv_bfloat16* x = X + static_cast<int64_t>(t) * d_in;

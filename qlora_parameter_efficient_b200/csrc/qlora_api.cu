@@ -87,6 +87,24 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 // ======================================================================= TMA descriptors
 
+// 3-D tensor map over a row-major matrix viewed as [dim2 = column blocks][dim1 = rows]
+// [dim0 = inner bytes of a block]: one box brings box2 consecutive column blocks of box1 rows,
+// laid out block-major in shared memory.  elem = element size, inner = elements per block.
+qlora_status tmap_blocks(CUtensorMap* m, CUtensorMapDataType dt, uint32_t elem, const void* base,
+                         int64_t rows, int64_t row_bytes, uint32_t inner, uint32_t box1,
+                         uint32_t box2, CUtensorMapSwizzle sw) {
+    QL_TRY(get_encoder());
+    const int64_t blocks = row_bytes / (static_cast<int64_t>(inner) * elem);
+    cuuint64_t dims[3] = {inner, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(blocks)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(inner) * elem};
+    cuuint32_t box[3] = {inner, box1, box2};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 // bf16 matrix [rows, cols] (cols contiguous, row stride ld elements), 128-byte swizzle,
 // box = 64 columns x box_rows rows.
 qlora_status tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
@@ -118,21 +136,6 @@ qlora_status tmap_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t col
     return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-// byte matrix [rows, cols_bytes] with the 128-byte swizzle, box = 128 bytes x box_y rows.
-qlora_status tmap_u8_sw128(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
-                           uint32_t box_y) {
-    QL_TRY(get_encoder());
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
-    cuuint32_t box[2] = {128, box_y};
-    cuuint32_t es[2] = {1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
-                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
-}
-
 // ======================================================================= planning
 
 int choose_split(int64_t tiles, int64_t k_steps) {
@@ -145,27 +148,27 @@ int choose_split(int64_t tiles, int64_t k_steps) {
 
 int pad_rank(int r) { return r <= 64 ? 64 : 128; }
 
-// Decode-size forward (bf16, T <= 32): stream-K split of (128-row tile x 64-K) units.
+// Decode-size forward (bf16, T <= 32, d_in a multiple of 256): clusters of C CTAs own tiles of
+// M rows, the C ranks split K.  (C, M) is picked at launch by balanced cost.
 constexpr int kSmallT = 32;
 struct SmallPlan {
-    int nt = 16, kt = 0, kt4 = 0, rt = 0, units = 0, grid = 0, tiles_per_cta = 0;
+    bool ok = false;
+    int nt8 = 1, kt = 0;
 };
 SmallPlan make_small_plan(int64_t T, int64_t d_out, int64_t d_in) {
     SmallPlan sp;
-    sp.nt = T <= 16 ? 16 : 32;
+    (void)d_out;
+    if (T < 1 || T > kSmallT) return sp;
+    sp.nt8 = T <= 8 ? 1 : (T <= 16 ? 2 : 4);
     sp.kt = static_cast<int>(d_in / 64);
-    sp.kt4 = static_cast<int>(cdiv(sp.kt, 4));
-    sp.rt = static_cast<int>(cdiv(d_out, 128));
-    sp.units = sp.kt4 * sp.rt;
-    sp.grid = std::max(1, std::min(sp.units, kSmsForSplit));
-    sp.tiles_per_cta = static_cast<int>(cdiv(sp.units, sp.grid) / sp.kt4) + 2;
+    sp.ok = sp.kt % 4 == 0;
     return sp;
 }
 
 struct Plan {
     int RP = 0;
     bool small = false;
-    size_t s_us = 0, s_cnt = 0, s_part = 0;
+    size_t s_us = 0;
     int split_u = 1, split_g = 1, split_da = 1, split_db = 1;
     size_t a_pad = 0, b_pad = 0, u_spad = 0, u_pad = 0, g_spad = 0, part = 0;
     size_t w32 = 0, uf = 0, gf = 0;
@@ -181,12 +184,9 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
         return o;
     };
     if (op == QLORA_OP_MERGE) return p;
-    if (op == QLORA_OP_FWD && dtype == QLORA_BF16 && T <= kSmallT) {
-        const SmallPlan sp = make_small_plan(T, d_out, d_in);
+    if (op == QLORA_OP_FWD && dtype == QLORA_BF16 && make_small_plan(T, d_out, d_in).ok) {
         p.small = true;
         p.s_us = take(static_cast<size_t>(T) * r * 4);
-        p.s_cnt = take(static_cast<size_t>(sp.rt) * 4);
-        p.s_part = take(static_cast<size_t>(sp.grid) * sp.tiles_per_cta * 128 * sp.nt * 4);
         p.total = off;
         return p;
     }
@@ -373,74 +373,131 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
     return QLORA_OK;
 }
 
-// Decode-size forward: U pre-pass (also zeroes the tile counters) overlapped with the
-// weight stream through programmatic dependent launch.
-qlora_status small_fwd(const qlora_nf4* w, const void* X, int64_t T, const void* A, const void* B,
-                       int r, float s, void* H, void* U_save, const Plan& p, void* ws, int* err,
-                       cudaStream_t st) {
-    const int64_t d_out = w->d_out, d_in = w->d_in;
-    const SmallPlan sp = make_small_plan(T, d_out, d_in);
-    float* us = at<float>(ws, p.s_us);
-    int* counters = at<int>(ws, p.s_cnt);
-    float* part = at<float>(ws, p.s_part);
-    k_small_u<<<dim3(static_cast<unsigned>(r), static_cast<unsigned>(cdiv(T, 4))), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(X), static_cast<int>(T),
-                                 static_cast<int>(d_in), static_cast<const __nv_bfloat16*>(A), r, s,
-                                 us, static_cast<__nv_bfloat16*>(U_save), counters, sp.rt);
-    QL_LAUNCH_CHECK();
-    CUtensorMap tc, tx;
-    QL_TRY(tmap_u8_sw128(&tc, w->codes, d_out, d_in / 2, d_in / 2, 128));
-    QL_TRY(tmap_bf16(&tx, X, T, d_in, d_in, static_cast<uint32_t>(sp.nt)));
-    GvArgs g{};
-    g.T = static_cast<int>(T);
-    g.d_out = static_cast<int>(d_out);
-    g.d_in = static_cast<int>(d_in);
-    g.kt = sp.kt;
-    g.kt4 = sp.kt4;
-    g.rt = sp.rt;
-    g.units = sp.units;
-    g.tiles_per_cta = sp.tiles_per_cta;
-    g.absmax_q = w->absmax_q;
-    g.c2 = w->c2;
-    g.part = part;
-    g.counters = counters;
-    g.us = us;
-    g.B = static_cast<const __nv_bfloat16*>(B);
-    g.r = r;
-    g.H = static_cast<__nv_bfloat16*>(H);
-    g.err = err;
-    g.wait_ns = kWaitNs;
-    // one CTA per SM: each holds all 512 tensor-memory columns
-    const int smem = std::max(1024 + kGvLut + kGvStagesC * kGvBlk * (sp.nt * 128 + 128 * 32) + kGvUsMax * 4 + 512, 120 * 1024);
-    auto kern = sp.nt == 16 ? k_qgemv<16> : k_qgemv<32>;
-    static std::atomic<uint64_t> configured[2] = {0, 0};
+// Decode-size forward: the U pre-pass overlapped with the weight stream through programmatic
+// dependent launch; the stream kernel runs as clusters of C CTAs over tiles of M rows.
+template <int NT8>
+qlora_status launch_qgemv(const qlora_nf4* w, const void* X, int64_t T, GvArgs g, cudaStream_t st) {
+    (void)X;
+    (void)T;
+    auto kern = k_qgemv<NT8>;
+    constexpr int smem = GvCfg<NT8>::kSmem;
     int dev = 0;
     cudaGetDevice(&dev);
+    // per device and cluster size 1, 2, 4, 8: clusters that fit at once (0 = not queried,
+    // -1 = none)
+    static std::atomic<int> fit[64][4];
+    static std::atomic<uint64_t> configured{0};
     const uint64_t bit = 1ull << (dev & 63);
-    const int which = sp.nt == 16 ? 0 : 1;
-    if (!(configured[which].load() & bit)) {
+    if (!(configured.load() & bit)) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return QLORA_ERR_CUDA;
-        configured[which].fetch_or(bit);
+        configured.fetch_or(bit);
     }
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(sp.grid));
     cfg.blockDim = dim3(kGvThreads);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
+    const int64_t d_out = g.d_out, q4 = g.kt / 4;
+    int64_t best_cost = -1;
+    int best_C = 0, best_M = 0, best_clusters = 0;
+    for (int e = 0; e < 4; ++e) {
+        const int C = 1 << e;
+        if (C > q4 || C > GvCfg<NT8>::kMaxRanks) break;
+        if (4 * cdiv(q4, C) > GvCfg<NT8>::kMaxBlk) continue;
+        int n = fit[dev & 63][e].load();
+        if (n == 0) {
+            if (C == 1) {
+                n = kSmsForSplit;
+            } else {
+                attr[1].val.clusterDim.x = static_cast<unsigned>(C);
+                cfg.gridDim = dim3(static_cast<unsigned>(C * (kSmsForSplit / C)));
+                cfg.numAttrs = 2;
+                int m = 0;
+                if (cudaOccupancyMaxActiveClusters(&m, kern, &cfg) != cudaSuccess) {
+                    cudaGetLastError();
+                    m = 0;
+                }
+                n = std::min(m, kSmsForSplit / C);
+            }
+            if (n <= 0) n = -1;
+            fit[dev & 63][e].store(n);
+        }
+        if (n < 0) continue;
+        const int64_t nbk = 4 * cdiv(q4, C);
+        for (int M = 16; M <= 16 * GvCfg<NT8>::MW && M * nbk <= kGvTabAbs && M * g.kt / 256 + 2 <= kGvTabC2; M += 16) {
+            const int64_t tiles = cdiv(d_out, M);
+            const int64_t clusters = std::min<int64_t>(n, tiles);
+            const int64_t tpc = cdiv(tiles, clusters);
+            // busiest cluster: its rows x its K range, plus a fixed cost per tile end
+            const int64_t cost = tpc * (M * nbk + 1024) + (C > 1 ? 512 : 0);
+            if (best_cost < 0 || cost < best_cost) {
+                best_cost = cost;
+                best_C = C;
+                best_M = M;
+                best_clusters = static_cast<int>(clusters);
+            }
+        }
+    }
+    if (best_C == 0) return QLORA_ERR_UNSUPPORTED;
+    g.C = best_C;
+    g.M = best_M;
+    g.tiles = static_cast<int>(cdiv(d_out, best_M));
+    g.clusters = best_clusters;
+    g.pieces = static_cast<int>(cdiv(q4, best_C));
+    CUtensorMap tc;
+    QL_TRY(tmap_blocks(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, w->d_out, w->d_in / 2, 128, 16,
+                       static_cast<uint32_t>(g.pieces), CU_TENSOR_MAP_SWIZZLE_128B));
+    cfg.gridDim = dim3(static_cast<unsigned>(best_C * best_clusters));
     cfg.numAttrs = 1;
+    if (best_C > 1) {
+        attr[1].val.clusterDim.x = static_cast<unsigned>(best_C);
+        cfg.numAttrs = 2;
+    }
     const bool ev = g_ev_start && g_ev_stop;
     if (ev) cudaEventRecord(g_ev_start, st);
-    if (cudaLaunchKernelEx(&cfg, kern, tc, tx, g) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, tc, g) != cudaSuccess) return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     if (ev) cudaEventRecord(g_ev_stop, st);
     return QLORA_OK;
 }
 
-// ======================================================================= fp32 helpers
+qlora_status small_fwd(const qlora_nf4* w, const void* X, int64_t T, const void* A, const void* B,
+                       int r, float s, void* H, void* U_save, const Plan& p, void* ws, int* err,
+                       cudaStream_t st) {
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    const SmallPlan sp = make_small_plan(T, d_out, d_in);
+    if (!sp.ok) return QLORA_ERR_UNSUPPORTED;
+    float* us = at<float>(ws, p.s_us);
+    k_small_u<<<dim3(static_cast<unsigned>(r), static_cast<unsigned>(cdiv(T, 4))), 128, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(X), static_cast<int>(T), static_cast<int>(d_in),
+        static_cast<const __nv_bfloat16*>(A), r, s, us, static_cast<__nv_bfloat16*>(U_save));
+    QL_LAUNCH_CHECK();
+    GvArgs g{};
+    g.T = static_cast<int>(T);
+    g.d_out = static_cast<int>(d_out);
+    g.d_in = static_cast<int>(d_in);
+    g.kt = sp.kt;
+    g.X = static_cast<const __nv_bfloat16*>(X);
+    g.absmax_q = w->absmax_q;
+    g.c2 = w->c2;
+    g.us = us;
+    g.B = static_cast<const __nv_bfloat16*>(B);
+    g.r = r;
+    g.b_vec = (r % 8 == 0) ? 1 : 0;    // B is 16-byte aligned (checked by the caller)
+    g.H = static_cast<__nv_bfloat16*>(H);
+    g.err = err;
+    g.wait_ns = kWaitNs;
+    if (sp.nt8 == 1) return launch_qgemv<1>(w, X, T, g, st);
+    if (sp.nt8 == 2) return launch_qgemv<2>(w, X, T, g, st);
+    return launch_qgemv<4>(w, X, T, g, st);
+}
 
 qlora_status sgemm(cudaStream_t st, int64_t M, int64_t N, int64_t K, float alpha, const float* A,
                    int64_t lda, bool ta, const float* B, int64_t ldb, bool tb, float beta,

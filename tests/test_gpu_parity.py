@@ -144,11 +144,15 @@ def test_q_proj_full_size_sampled_rows(q):
 
 
 @pytest.mark.parametrize("d_out,d_in,r,T", [
-    (136, 192, 5, 1),        # ragged row tile, 3 K steps
+    (136, 192, 5, 1),        # d_in/64 not a multiple of 4: the large-T path
     (520, 320, 16, 4),
-    (1000, 512, 64, 16),
-    (264, 640, 33, 17),      # 32-token tile, ragged
-    (2048, 1024, 128, 32),
+    (1000, 512, 64, 16),     # ragged last 16-row tile
+    (264, 640, 33, 17),
+    (2048, 1024, 128, 32),   # 32-token tile
+    (264, 4352, 33, 3),      # 68 blocks per row: K split over a cluster, uneven ranks; r % 8 != 0
+    (2056, 1024, 16, 24),    # 32-token tile, ragged rows
+    (4096, 4096, 16, 1),     # q_proj shape: K split over a cluster
+    (4096, 4096, 16, 8),
 ])
 def test_decode_size_forward(q, d_out, d_in, r, T):
     import torch
