@@ -355,37 +355,138 @@ def run_gpu(args):
     return 0
 
 
+def _graph_time(torch, calls, reps=20):
+    """Per-call device time of `calls` (a list of zero-argument launches) captured in one CUDA
+    graph and replayed `reps` times: (median, min) microseconds per call over 5 measurements."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for fn in calls:       # warm-up (and one-time host setup) outside the capture
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for fn in calls:
+                fn()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        g.replay()
+    samples = []
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        samples.append(a.elapsed_time(b) * 1e3 / (reps * len(calls)))
+    del g
+    return statistics.median(samples), min(samples)
+
+
 def extra_rows(q, torch, S, dev, peaks, args):
-    """Other rows of the hot path, each timed on the device (not part of the headline)."""
+    """The other rows of the hot path, each timed on the device by CUDA-graph replay over
+    rotating weight copies whose working set exceeds the 126 MB L2 (not part of the headline)."""
     out = {}
     bf = torch.bfloat16
     hbm = peaks["hbm_gbs"]
-    # decode-size forward on the 11008x4096 MLP shape, r = 64
+    tc = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+
+    def w_bytes(d, k):
+        return d * k * (0.5 + 1 / 64) + 4 * ((d * k // 64 + 255) // 256)
+
+    # ---- decode-size forward (T = 1, 4, 16) on the 11008 x 4096 MLP shape, r = 64
     c3 = S.CONFIGS["mlp_up_11008x4096_r64_T8192"]
-    d, k, r = c3["d_out"], c3["d_in"], c3["r"]
-    NW = 8  # rotate 8 weights (8 x 23 MB) so the stream comes from HBM, not L2
-    base = S.make_layer(d, k, r, c3["alpha"], 16, dtype="bf16", seed=7)
-    ws_list = [q.nf4_quantize(torch.from_numpy(base.W0).to(dev) * (1 + 0.01 * i)) for i in range(NW)]
+    d, k, r, alpha = c3["d_out"], c3["d_in"], c3["r"], c3["alpha"]
+    NW = 8      # 8 x 23 MB of NF4 weights
+    base = S.make_layer(d, k, r, alpha, 16, dtype="bf16", seed=7, with_grad=False)
+    W0 = torch.from_numpy(base.W0).to(dev)
+    wl = [q.nf4_quantize(W0) for _ in range(NW)]
+    del W0
     A = torch.from_numpy(base.A).to(dev).to(bf)
     B = torch.from_numpy(base.B).to(dev).to(bf)
     for T in (1, 4, 16):
         X = torch.from_numpy(base.X[:T]).to(dev).to(bf)
         H = torch.empty((T, d), dtype=bf, device=dev)
         ws = torch.empty(q.workspace_bytes(q.OP_FWD, q.BF16, T, d, k, r), dtype=torch.uint8, device=dev)
-        for i in range(5):
-            q.qlora_linear_fwd(ws_list[i % NW], X, A, B, c3["alpha"], H=H, ws=ws, save_u=False)
+        calls = [(lambda w=w: q.qlora_linear_fwd(w, X, A, B, alpha, H=H, ws=ws, save_u=False)) for w in wl]
+        med, mn = _graph_time(torch, calls)
+        # the stream kernel alone (events around it; eager calls)
+        kev = []
+        for i in range(3 * NW):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            e1.record()
+            q.set_gemm_events(e0, e1)
+            q.qlora_linear_fwd(wl[i % NW], X, A, B, alpha, H=H, ws=ws, save_u=False)
+            q.set_gemm_events(None, None)
+            kev.append((e0, e1))
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n = 50
-        e0.record()
-        for i in range(n):
-            q.qlora_linear_fwd(ws_list[i % NW], X, A, B, c3["alpha"], H=H, ws=ws, save_u=False)
-        e1.record()
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / n
-        byts = d * k * (0.5 + 1 / 64) + 4 * ((d * k // 64 + 255) // 256) + 2 * T * (k + d) + 2 * r * (d + k)
-        out[f"decode_T{T}_us"] = us
-        out[f"decode_T{T}_hbm_frac"] = byts / (us * 1e-6) / 1e9 / hbm
+        kus = statistics.median(a.elapsed_time(b) * 1e3 for a, b in kev[NW:])
+        byts = w_bytes(d, k) + 2 * T * (k + d) + 2 * r * (d + k)
+        out[f"decode_T{T}"] = {"call_us": med, "call_us_min": mn, "kernel_us": kus,
+                               "GB/s": byts / (med * 1e-6) / 1e9, "hbm_frac": byts / (med * 1e-6) / 1e9 / hbm,
+                               "kernel_hbm_frac": byts / (kus * 1e-6) / 1e9 / hbm,
+                               "bytes": byts, "hbm_peak_gbs": hbm}
+    del wl
+
+    # ---- large-T forward and backward on the same shape, T = 8192
+    T = c3["T"]
+    case = S.make_layer(d, k, r, alpha, T, dtype="bf16", seed=11)
+    wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(2)]
+    X = torch.from_numpy(case.X).to(dev).to(bf)
+    dH = torch.from_numpy(case.dH).to(dev).to(bf)
+    del case
+    H = torch.empty((T, d), dtype=bf, device=dev)
+    U = torch.empty((T, r), dtype=bf, device=dev)
+    dX = torch.empty((T, k), dtype=bf, device=dev)
+    dA = torch.empty((r, k), dtype=torch.float32, device=dev)
+    dB = torch.empty((d, r), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(q.workspace_bytes(q.OP_FWD, q.BF16, T, d, k, r),
+                         q.workspace_bytes(q.OP_BWD, q.BF16, T, d, k, r)), dtype=torch.uint8, device=dev)
+    fwd = [(lambda w=w: q.qlora_linear_fwd(w, X, A, B, alpha, H=H, U_save=U, ws=ws)) for w in wl]
+    bwd = [(lambda w=w: q.qlora_linear_bwd(w, X, dH, A, B, alpha, U_saved=U, dX=dX, dA=dA, dB=dB, ws=ws))
+           for w in wl]
+    fmed, _ = _graph_time(torch, fwd, reps=5)
+    bmed, _ = _graph_time(torch, bwd, reps=5)
+    out["mlp_11008x4096_T8192"] = {"fwd_us": fmed, "bwd_us": bmed,
+                                   "fwd_tflops": flops_fwd(T, d, k, r) / (fmed * 1e-6) / 1e12,
+                                   "bwd_tflops": flops_bwd(T, d, k, r) / (bmed * 1e-6) / 1e12,
+                                   "fwd_tc_frac": flops_fwd(T, d, k, r) / (fmed * 1e-6) / 1e12 / tc,
+                                   "bwd_tc_frac": flops_bwd(T, d, k, r) / (bmed * 1e-6) / 1e12 / tc}
+    del wl, X, dH, H, U, dX, dA, dB, ws
+
+    # ---- multi-adapter forward: 4096^2 base, 4 adapters r = 8, 16, 16, 64, T = 4096
+    for split_name, split in (("uniform", None), ("skewed", [0.7, 0.1, 0.1, 0.1])):
+        mc = S.make_multi_adapter(4096, 4096, 4096, [8, 16, 16, 64], split=split, dtype="bf16", seed=5)
+        wl = [q.nf4_quantize(torch.from_numpy(mc.W0).to(dev)) for _ in range(4)]
+        X = torch.from_numpy(mc.X).to(dev).to(bf)
+        ids = torch.from_numpy(mc.ids).to(dev)
+        As = [torch.from_numpy(a).to(dev).to(bf) for a in mc.As]
+        Bs = [torch.from_numpy(b).to(dev).to(bf) for b in mc.Bs]
+        H = torch.empty((4096, 4096), dtype=bf, device=dev)
+        ws = torch.empty(q.workspace_bytes(q.OP_FWD_BATCHED, q.BF16, 4096, 4096, 4096, sum(mc.ranks)),
+                         dtype=torch.uint8, device=dev)
+        calls = [(lambda w=w: q.qlora_linear_fwd_batched(w, X, ids, As, Bs, mc.alphas, H=H, ws=ws)) for w in wl]
+        med, _ = _graph_time(torch, calls, reps=10)
+        fl = 2 * 4096 * 4096 * 4096 + sum(2 * 4096 * rr * (4096 + 4096) for rr in mc.ranks) // len(mc.ranks)
+        out[f"batched_4x_{split_name}"] = {"fwd_us": med, "tflops": fl / (med * 1e-6) / 1e12,
+                                          "tc_frac": fl / (med * 1e-6) / 1e12 / tc}
+        del wl, X, ids, As, Bs, H, ws
+
+    # ---- merge W_final = W^ + s B A on the 4096^2 shape, bf16 out
+    c2_ = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
+    d, k, r, alpha = c2_["d_out"], c2_["d_in"], c2_["r"], c2_["alpha"]
+    case = S.make_layer(d, k, r, alpha, 1, dtype="bf16", seed=13, with_grad=False)
+    wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(8)]
+    A = torch.from_numpy(case.A).to(dev).to(bf)
+    B = torch.from_numpy(case.B).to(dev).to(bf)
+    outs = [torch.empty((d, k), dtype=bf, device=dev) for _ in range(8)]
+    calls = [(lambda w=w, o=o: q.lora_merge(w, A, B, alpha, bf, out=o)) for w, o in zip(wl, outs)]
+    med, _ = _graph_time(torch, calls, reps=10)
+    byts = w_bytes(d, k) + 2 * d * k + 2 * r * (d + k)
+    out["merge_4096x4096_bf16"] = {"us": med, "GB/s": byts / (med * 1e-6) / 1e9,
+                                   "hbm_frac": byts / (med * 1e-6) / 1e9 / hbm}
     return out
 
 

@@ -1,4 +1,4 @@
-// qgemv.cuh -- decode-size forward (T <= 32 tokens): an HBM-bound stream over the NF4 codes.
+// qgemv.cuh -- decode-size forward (T <= 16 tokens): an HBM-bound stream over the NF4 codes.
 //
 //   H[t, n] = (1/127) sum_b q8_b(n) c2_b(n) sum_{k in b} L16(code(n, k)) x[t, k]
 //             + (s U[t, :]) . B[n, :]
@@ -34,7 +34,7 @@
 // bytes, 128-byte swizzle, so the fragment reads are bank-conflict free); the warps take turns
 // issuing the refills.  Across the M/16 stages of a tile each warp accumulates q8 c2 x partial
 // in fp32 registers; the tile's absmax bytes and c2 values come in once per tile by cp.async.
-// At the end of a tile the 8 warps combine by a fixed tree in shared memory, the ranks' sums
+// At the end of a tile warp w sums 16-row group w over the 8 warps in warp order, the ranks' sums
 // meet in rank 0's shared memory over DSMEM, and rank 0 sums them in rank order, applies 1/127,
 // adds the adapter term (a few mma steps) and writes H.  No global partials, atomics or
 // semaphores: the sums are deterministic and the tail is on-chip.
@@ -47,29 +47,32 @@ namespace qlora {
 
 constexpr int kGvWarps = 8;
 constexpr int kGvThreads = 32 * kGvWarps;
-constexpr int kGvUsMax = 32 * 128; // s*U staging (bf16): T <= 32 tokens x r <= 128
-constexpr int kGvTabAbs = 16384;   // a tile's absmax bytes: M x (kb_hi - kb_lo) <= this
-constexpr int kGvTabC2 = 320;      // a tile's c2 groups: M x kt / 256 + 2 <= this
+constexpr int kGvUsMax = 16 * 128; // s*U staging (bf16): T <= 16 tokens x r <= 128
+constexpr int kGvTabS = 6144;      // a tile's block scales: M x (kb_hi - kb_lo + 1) <= this
+constexpr int kGvRawC2 = 320;      // a tile's c2 groups: M x kt / 256 + 2 <= this
+constexpr int kGvBrowMax = 8192;  // a tile's adapter rows: M x (r + 8) bf16 <= this
 
 template <int NT8>
 struct GvCfg {
     static constexpr int NT = 8 * NT8;                 // token tile
     static constexpr int NBW = 8 / NT8;                // blocks per warp (X fragments in registers)
     static constexpr int kMaxBlk = 8 * NBW;            // blocks of a CTA's K range
-    static constexpr int MW = NT8 == 1 ? 8 : (NT8 == 2 ? 6 : 3);   // max 16-row groups per tile
+    static constexpr int MW = NT8 == 1 ? 8 : 6;        // max 16-row groups per tile
     static constexpr int kStage = 16 * kMaxBlk * 32;   // 16 rows x the K range (<= 32 KB)
-    static constexpr int S = NT8 == 1 ? 5 : (NT8 == 2 ? 7 : 8);
+    static constexpr int S = NT8 == 1 ? 3 : 4;
     static constexpr int kMaxRanks = NT8 == 1 ? 4 : 8;  // cluster size limit
-    static constexpr int kSlot = 32 * MW * NT8 * 16;   // one warp's accumulators
-    static constexpr int kTree = 4 * kSlot;            // tree slots
+    static constexpr int kSlot = 32 * MW * NT8 * 16;   // one warp's partials of a tile
+    static constexpr int kTree = 8 * kSlot;            // every warp's partials
     static constexpr int kRing = kMaxRanks * kSlot;    // rank 0: one CTA sum per rank
     static constexpr int kStageOff = 0;
     static constexpr int kTreeOff = kStageOff + S * kStage;
     static constexpr int kRingOff = kTreeOff + kTree;
     static constexpr int kUsOff = kRingOff + kRing;
-    static constexpr int kTabOff = kUsOff + kGvUsMax * 2;   // the tile's absmax [M][nbk] bytes
-    static constexpr int kC2Off = kTabOff + kGvTabAbs;      // the tile's c2 groups
-    static constexpr int kBarOff = kC2Off + kGvTabC2 * 4;
+    static constexpr int kTabOff = kUsOff + kGvUsMax * 2;   // the tile's scales [M][nbk + 1] fp32
+    static constexpr int kBrowOff = kTabOff + kGvTabS * 4;  // the tile's B rows [M][r + 8] bf16
+    static constexpr int kRawOff = kBrowOff + kGvBrowMax * 2;   // [2] absmax bytes, then c2
+    static constexpr int kRawBuf = kGvTabS + kGvRawC2 * 4;
+    static constexpr int kBarOff = kRawOff + 2 * kRawBuf;
     static constexpr int kSmem = kBarOff + 256 + 1024;   // barriers + alignment slack
     static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -83,6 +86,12 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 // 4-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros without reading.
 __device__ __forceinline__ void cp_async_4(void* dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes)
+                 : "memory");
+}
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros without reading.
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),
                  "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes)
                  : "memory");
 }
@@ -143,11 +152,12 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* stages = smem + Cf::kStageOff;
-    float4* tree = reinterpret_cast<float4*>(smem + Cf::kTreeOff);           // [4][MW][NT8][32]
+    float4* part = reinterpret_cast<float4*>(smem + Cf::kTreeOff);           // [8 warps][MW][NT8][32]
     float4* ring = reinterpret_cast<float4*>(smem + Cf::kRingOff);           // [ranks][MW][NT8][32]
     __nv_bfloat16* s_us = reinterpret_cast<__nv_bfloat16*>(smem + Cf::kUsOff);   // [NT][rp]
-    uint8_t* tab_abs = smem + Cf::kTabOff;                                   // [M][nbk]
-    float* tab_c2 = reinterpret_cast<float*>(smem + Cf::kC2Off);             // [groups]
+    float* tab_s = reinterpret_cast<float*>(smem + Cf::kTabOff);             // [M][nbk + 1]
+    __nv_bfloat16* s_b = reinterpret_cast<__nv_bfloat16*>(smem + Cf::kBrowOff);  // [M][r + 8]
+    uint8_t* raw = smem + Cf::kRawOff;        // [2][absmax bytes [M][nbk] | c2 groups], by tile parity
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::kBarOff);
     uint64_t* full = bars;                     // [S] the stage's code box landed
     uint64_t* empty = full + S;                // [S] all warps done with the stage
@@ -188,7 +198,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
             mbar_init(&empty[s], kGvWarps);
         }
         mbar_init(csync_bar, kGvWarps);
-        mbar_init(ring_full, 32 * C);
+        mbar_init(ring_full, 32 * mw * C);
         mbar_init(ring_free, 1);
         *abort = 0;
         fence_mbar_init();
@@ -230,51 +240,69 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         return ok;
     };
 
-    float acc[MW][NT8][4];
+    // the raw tables of a tile: absmax bytes [M][nbk] and its c2 groups, by all threads, into the
+    // buffer of the tile's parity
+    auto prefetch_tables = [&](int tile) {
+        const int row0 = tile * M;
+        uint8_t* rabs = raw + ((tile - t_lo) & 1) * Cf::kRawBuf;
+        float* rc2 = reinterpret_cast<float*>(rabs + kGvTabS);
+        const int wpr = nbk / 4;
+        for (int wi = threadIdx.x; wi < M * wpr; wi += kGvThreads) {
+            const int rr = wi / wpr, q = wi % wpr;
+            const bool ok = row0 + rr < args.d_out;
+            cp_async_4(rabs + rr * nbk + 4 * q,
+                       args.absmax_q + (ok ? static_cast<int64_t>(row0 + rr) * args.kt + kb_lo + 4 * q : 0),
+                       ok ? 4u : 0u);
+        }
+        const int64_t rlast = min(row0 + M, args.d_out) - 1;
+        const int64_t g_first = (static_cast<int64_t>(row0) * args.kt + kb_lo) >> 8;
+        const int n_c2 = static_cast<int>(((rlast * args.kt + kb_hi - 1) >> 8) - g_first + 1);
+        for (int e = threadIdx.x; e < n_c2; e += kGvThreads) cp_async_4(rc2 + e, args.c2 + g_first + e, 4u);
+    };
+    if (t_lo < t_hi) prefetch_tables(t_lo);
     int last_issued = -1;       // latest stage this warp issued (beyond the initial ones)
-    bool us_ready = false, ok_all = true;
+    bool ok_all = true;
     int tiles_done = 0;
 
     for (int tile = t_lo; tile < t_hi && ok_all; ++tile) {
         const int row0 = tile * M;
-        // ---- the tile's absmax bytes [M][nbk] and c2 groups, by all threads (the previous
-        // tile's readers are past its end-of-tile meetings)
-        {
-            const int wpr = nbk / 4;
-            for (int wi = threadIdx.x; wi < M * wpr; wi += kGvThreads) {
-                const int rr = wi / wpr, q = wi % wpr;
-                const bool ok = row0 + rr < args.d_out;
-                cp_async_4(tab_abs + rr * nbk + 4 * q,
-                           args.absmax_q + (ok ? static_cast<int64_t>(row0 + rr) * args.kt + kb_lo + 4 * q : 0),
-                           ok ? 4u : 0u);
-            }
-        }
-        const int64_t rlast = min(row0 + M, args.d_out) - 1;
-        const int64_t g_first = (static_cast<int64_t>(row0) * args.kt + kb_lo) >> 8;
-        {
-            const int n_c2 = static_cast<int>(((rlast * args.kt + kb_hi - 1) >> 8) - g_first + 1);
-            for (int e = threadIdx.x; e < n_c2; e += kGvThreads) cp_async_4(tab_c2 + e, args.c2 + g_first + e, 4u);
-        }
+        // ---- the tile's block scales q8 * c2 [M][nbk + 1] from its raw tables (prefetched during
+        // the previous tile), then the next tile's raw tables and (rank 0) this tile's adapter
+        // rows go out; the previous tile's readers are past its end-of-tile meetings
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (!csync()) {
             fail();
             break;
         }
-        if (rank == 0 && warp == 1 && lane == 0 && args.b_vec) {     // adapter rows, to L2
-            const int rows = min(M, args.d_out - row0);
-            bulk_prefetch_l2(args.B + static_cast<int64_t>(row0) * args.r, static_cast<uint32_t>(rows * args.r * 2));
+        const int sld = nbk + 1;                  // padded row: the 8 rows a warp reads hit 8 banks
+        {
+            const uint8_t* rabs = raw + ((tile - t_lo) & 1) * Cf::kRawBuf;
+            const float* rc2 = reinterpret_cast<const float*>(rabs + kGvTabS);
+            const int64_t g_first = (static_cast<int64_t>(row0) * args.kt + kb_lo) >> 8;
+            for (int e = threadIdx.x; e < M * nbk; e += kGvThreads) {
+                const int rr = e / nbk, L = e % nbk;
+                const int64_t blk = static_cast<int64_t>(row0 + rr) * args.kt + kb_lo + L;
+                tab_s[rr * sld + L] = row0 + rr < args.d_out
+                    ? static_cast<float>(rabs[e]) * rc2[(blk >> 8) - g_first] : 0.f;
+            }
         }
-#pragma unroll
-        for (int m = 0; m < MW; ++m)
-#pragma unroll
-            for (int n = 0; n < NT8; ++n)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[m][n][e] = 0.f;
-
-        // ---- the tile's 16-row groups, one stage each
-#pragma unroll
-        for (int m = 0; m < MW; ++m) {
-            if (m >= mw) break;
+        if (!csync()) {
+            fail();
+            break;
+        }
+        if (rank == 0 && args.b_vec) {
+            const int cpr = args.r / 8;           // 16-byte pieces per row
+            for (int e = threadIdx.x; e < M * cpr; e += kGvThreads) {
+                const int rr = e / cpr, q = e % cpr;
+                const bool ok = row0 + rr < args.d_out;
+                cp_async_16(s_b + rr * (args.r + 8) + 8 * q,
+                            args.B + (ok ? static_cast<int64_t>(row0 + rr) * args.r + 8 * q : 0), ok ? 16u : 0u);
+            }
+        }
+        if (tile + 1 < t_hi) prefetch_tables(tile + 1);
+        // ---- the tile's 16-row groups, one stage each (a runtime loop: its body is emitted once)
+#pragma unroll 1
+        for (int m = 0; m < mw; ++m) {
             const int u = (tile - t_lo) * mw + m;
             const int s = u % S;
             if (warp == u % kGvWarps && u + S - 1 < n_units) {
@@ -294,8 +322,11 @@ __global__ void __launch_bounds__(kGvThreads, 1)
             }
             const uint8_t* st = stages + s * Cf::kStage;
             const int ra_ = 16 * m + g, rb_ = ra_ + 8;          // rows within the tile
-            const int64_t base_a = static_cast<int64_t>(row0 + ra_) * args.kt;
-            const int64_t base_b = base_a + 8 * static_cast<int64_t>(args.kt);
+            float acc[NT8][4];
+#pragma unroll
+            for (int n = 0; n < NT8; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
 #pragma unroll
             for (int j = 0; j < NBW; ++j) {
                 const int L = warp + 8 * j;
@@ -318,76 +349,66 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 #pragma unroll
                     for (int n = 0; n < NT8; ++n)
                         mma_bf16_16816(tmp[n], A[k], xw[j][n][2 * k], xw[j][n][2 * k + 1], k > 0);
-                // q8 * c2 of rows ra_, rb_ from the tile's tables
-                const int kb = kb_lo + L;
-                const float sa = static_cast<float>(tab_abs[ra_ * nbk + L]) * tab_c2[((base_a + kb) >> 8) - g_first];
-                const float sb = static_cast<float>(tab_abs[rb_ * nbk + L]) * tab_c2[((base_b + kb) >> 8) - g_first];
+                // q8 * c2 of rows ra_, rb_ from the tile's scale table
+                const float sa = tab_s[ra_ * sld + L], sb = tab_s[rb_ * sld + L];
 #pragma unroll
                 for (int n = 0; n < NT8; ++n) {
-                    acc[m][n][0] = fmaf(sa, tmp[n][0], acc[m][n][0]);
-                    acc[m][n][1] = fmaf(sa, tmp[n][1], acc[m][n][1]);
-                    acc[m][n][2] = fmaf(sb, tmp[n][2], acc[m][n][2]);
-                    acc[m][n][3] = fmaf(sb, tmp[n][3], acc[m][n][3]);
+                    acc[n][0] = fmaf(sa, tmp[n][0], acc[n][0]);
+                    acc[n][1] = fmaf(sa, tmp[n][1], acc[n][1]);
+                    acc[n][2] = fmaf(sb, tmp[n][2], acc[n][2]);
+                    acc[n][3] = fmaf(sb, tmp[n][3], acc[n][3]);
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
+            // the warp's partial of this 16-row group
+#pragma unroll
+            for (int n = 0; n < NT8; ++n)
+                part[((warp * MW + m) * NT8 + n) * 32 + lane] = make_float4(acc[n][0], acc[n][1], acc[n][2], acc[n][3]);
         }
         if (!ok_all) {
             fail();
             break;
         }
 
-        // ---- end of the tile: the 8 warps' sums by a fixed tree.  Round with stride h: warps
-        // [h, 2h) hand their sums to warps [0, h).  The first round writes to tree slot
-        // (idx - h); later rounds write to the writer's own slot, which it read (and finished
-        // with) in the round before, so one meeting per round suffices.
-        bool first = true;
-        for (int h = kGvWarps / 2; h >= 1; h >>= 1) {
-            if (warp >= h && warp < 2 * h) {
-                float4* dst = tree + (first ? warp - h : warp) * (Cf::kSlot / 16);
-#pragma unroll
-                for (int m = 0; m < MW; ++m)
-#pragma unroll
-                    for (int n = 0; n < NT8; ++n)
-                        if (m < mw) dst[(m * NT8 + n) * 32 + lane] = make_float4(acc[m][n][0], acc[m][n][1], acc[m][n][2], acc[m][n][3]);
+        asm volatile("cp.async.wait_all;" ::: "memory");   // this tile's adapter rows
+        if (tiles_done == 0 && rank == 0) {
+            // s*U from the pre-pass as bf16 [NT][rp] (zero beyond T and r), once per CTA; the
+            // pre-pass has long finished by the end of the first tile
+            const int rp = (args.r + 15) & ~15;
+            griddep_wait();
+            for (int e = threadIdx.x; e < NT * rp; e += kGvThreads) {
+                const int t = e / rp, jj = e % rp;
+                s_us[e] = __float2bfloat16_rn(t < args.T && jj < args.r ? args.us[t * args.r + jj] : 0.f);
             }
-            if (!csync()) {
-                ok_all = false;
-                break;
-            }
-            if (warp < h) {
-                const float4* src = tree + (first ? warp : warp + h) * (Cf::kSlot / 16);
-#pragma unroll
-                for (int m = 0; m < MW; ++m)
-#pragma unroll
-                    for (int n = 0; n < NT8; ++n)
-                        if (m < mw) {
-                            const float4 p = src[(m * NT8 + n) * 32 + lane];
-                            acc[m][n][0] += p.x;
-                            acc[m][n][1] += p.y;
-                            acc[m][n][2] += p.z;
-                            acc[m][n][3] += p.w;
-                        }
-            }
-            first = false;
         }
-        if (!ok_all) {
+        // ---- end of the tile: warp w sums group w over the 8 warps in warp order and sends it to
+        // rank 0 (its own ring when C == 1)
+        if (!csync()) {
             fail();
             break;
         }
-        // ---- warp 0 sends the CTA's sum to rank 0 (its own ring slot when C == 1)
-        if (warp == 0) {
+        if (warp < mw) {
+            float4 sum[NT8];
+#pragma unroll
+            for (int n = 0; n < NT8; ++n) {
+                sum[n] = part[(warp * NT8 + n) * 32 + lane];
+#pragma unroll
+                for (int w = 1; w < kGvWarps; ++w) {
+                    const float4 v = part[((w * MW + warp) * NT8 + n) * 32 + lane];
+                    sum[n].x += v.x;
+                    sum[n].y += v.y;
+                    sum[n].z += v.z;
+                    sum[n].w += v.w;
+                }
+            }
             if (tiles_done > 0 && !mbar_wait_warp(ring_free, (tiles_done - 1) & 1, abort, args.wait_ns)) {
                 fail();
                 break;
             }
-            const uint32_t dst = mapa_shared(smem_u32(ring + rank * (Cf::kSlot / 16) + lane), 0);
+            const uint32_t dst = mapa_shared(smem_u32(ring + rank * (Cf::kSlot / 16) + (warp * NT8) * 32 + lane), 0);
 #pragma unroll
-            for (int m = 0; m < MW; ++m)
-#pragma unroll
-                for (int n = 0; n < NT8; ++n)
-                    if (m < mw) st_cluster_v4(dst + ((m * NT8 + n) * 32) * 16, make_float4(acc[m][n][0], acc[m][n][1], acc[m][n][2], acc[m][n][3]));
+            for (int n = 0; n < NT8; ++n) st_cluster_v4(dst + n * 32 * 16, sum[n]);
             mbar_arrive_remote(mapa_shared(smem_u32(ring_full), 0));   // release.cluster
         }
         ++tiles_done;
@@ -400,19 +421,6 @@ __global__ void __launch_bounds__(kGvThreads, 1)
             break;
         }
         const int rp = (args.r + 15) & ~15;          // adapter rank padded to the mma K
-        if (!us_ready) {
-            // s*U from the pre-pass as bf16 [NT][rp] (zero beyond T and r), once per CTA
-            griddep_wait();
-            for (int e = threadIdx.x; e < NT * rp; e += kGvThreads) {
-                const int t = e / rp, j = e % rp;
-                s_us[e] = __float2bfloat16_rn(t < args.T && j < args.r ? args.us[t * args.r + j] : 0.f);
-            }
-            us_ready = true;
-            if (!csync()) {
-                fail();
-                break;
-            }
-        }
         for (int m = warp; m < mw; m += kGvWarps) {
             float4 tot[NT8];
 #pragma unroll
@@ -445,10 +453,9 @@ __global__ void __launch_bounds__(kGvThreads, 1)
                     uint32_t a[4];
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2) {
-                        const int row = rbase + g + 8 * (q2 & 1);
+                        const int rr = 16 * m + g + 8 * (q2 & 1);     // row within the tile
                         const int col = k0 + 2 * c + 8 * (q2 >> 1);
-                        a[q2] = (row < args.d_out && col < args.r)
-                            ? __ldg(reinterpret_cast<const unsigned int*>(args.B + static_cast<int64_t>(row) * args.r + col)) : 0u;
+                        a[q2] = col < args.r ? *reinterpret_cast<const uint32_t*>(s_b + rr * (args.r + 8) + col) : 0u;
                     }
 #pragma unroll
                     for (int n = 0; n < NT8; ++n) {
@@ -514,47 +521,65 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 }
 
 // Pre-pass for the decode-size forward: U = X A^T (fp32 accumulation), s U in fp32 for the
-// adapter term and U in the call dtype for the backward.  Grid (r, ceil(T / 4)): each warp
-// computes one (token, adapter row) dot product with all of its loads in flight at once.
-// Lets the dependent stream kernel start immediately.
-__global__ void __launch_bounds__(128) k_small_u(const __nv_bfloat16* __restrict__ X, int T,
+// adapter term and U in the call dtype for the backward.  Few CTAs (ceil(r / 8), 8 warps each)
+// so that they fit beside the stream kernel, which it overlaps through programmatic dependent
+// launch: warp w of CTA b computes adapter row j = 8b + w for the tokens two at a time, each
+// pass over a 4096-element chunk of K with all of its loads in flight at once.
+__global__ void __launch_bounds__(256) k_small_u(const __nv_bfloat16* __restrict__ X, int T,
                                                  int d_in, const __nv_bfloat16* __restrict__ A,
                                                  int r, float s, float* __restrict__ us,
                                                  __nv_bfloat16* __restrict__ u_save) {
     griddep_launch_dependents();
-    const int j = blockIdx.x;
-    const int t = blockIdx.y * 4 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (t >= T) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j = blockIdx.x * 8 + warp;
+    if (j >= r) return;
     const __nv_bfloat16* a = A + static_cast<int64_t>(j) * d_in;
-    const __nv_bfloat16* x = X + static_cast<int64_t>(t) * d_in;
-    float acc = 0.f;
-    for (int k0 = lane * 8; k0 < d_in; k0 += 32 * 8 * 4) {
-        uint4 av[4], xv[4];
+    auto dot8 = [](const uint4& p, const uint4& q, float acc) {
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&p);
+        const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&q);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int k = k0 + u * 256;
-            av[u] = k < d_in ? __ldg(reinterpret_cast<const uint4*>(a + k)) : make_uint4(0, 0, 0, 0);
-            xv[u] = k < d_in ? __ldg(reinterpret_cast<const uint4*>(x + k)) : make_uint4(0, 0, 0, 0);
+        for (int e = 0; e < 4; ++e) {
+            const float2 pf = __bfloat1622float2(p2[e]);
+            const float2 qf = __bfloat1622float2(q2[e]);
+            acc = fmaf(pf.x, qf.x, acc);
+            acc = fmaf(pf.y, qf.y, acc);
         }
+        return acc;
+    };
+    for (int t0 = 0; t0 < T; t0 += 2) {
+        const bool two = t0 + 1 < T;
+        const __nv_bfloat16* x0p = X + static_cast<int64_t>(t0) * d_in;
+        const __nv_bfloat16* x1p = X + static_cast<int64_t>(two ? t0 + 1 : t0) * d_in;
+        float acc0 = 0.f, acc1 = 0.f;
+        for (int kc = 0; kc < d_in; kc += 4096) {
+            uint4 av[16], xv0[16], xv1[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&av[u]);
-            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv[u]);
+            for (int i = 0; i < 16; ++i) {
+                const int k = kc + 256 * i + 8 * lane;
+                const bool ok = k < d_in;
+                av[i] = ok ? __ldg(reinterpret_cast<const uint4*>(a + k)) : make_uint4(0, 0, 0, 0);
+                xv0[i] = ok ? __ldg(reinterpret_cast<const uint4*>(x0p + k)) : make_uint4(0, 0, 0, 0);
+                xv1[i] = (ok && two) ? __ldg(reinterpret_cast<const uint4*>(x1p + k)) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 af = __bfloat1622float2(a2[e]);
-                const float2 xf = __bfloat1622float2(x2[e]);
-                acc = fmaf(af.x, xf.x, acc);
-                acc = fmaf(af.y, xf.y, acc);
+            for (int i = 0; i < 16; ++i) {
+                acc0 = dot8(av[i], xv0[i], acc0);
+                acc1 = dot8(av[i], xv1[i], acc1);
             }
         }
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
-        us[static_cast<int64_t>(t) * r + j] = s * acc;
-        if (u_save) u_save[static_cast<int64_t>(t) * r + j] = __float2bfloat16_rn(acc);
+        for (int o = 16; o > 0; o >>= 1) {
+            acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
+            acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+        }
+        if (lane == 0) {
+            us[static_cast<int64_t>(t0) * r + j] = s * acc0;
+            if (u_save) u_save[static_cast<int64_t>(t0) * r + j] = __float2bfloat16_rn(acc0);
+            if (two) {
+                us[static_cast<int64_t>(t0 + 1) * r + j] = s * acc1;
+                if (u_save) u_save[static_cast<int64_t>(t0 + 1) * r + j] = __float2bfloat16_rn(acc1);
+            }
+        }
     }
 }
 

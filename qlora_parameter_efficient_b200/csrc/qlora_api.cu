@@ -148,9 +148,9 @@ int choose_split(int64_t tiles, int64_t k_steps) {
 
 int pad_rank(int r) { return r <= 64 ? 64 : 128; }
 
-// Decode-size forward (bf16, T <= 32, d_in a multiple of 256): clusters of C CTAs own tiles of
+// Decode-size forward (bf16, T <= 16, d_in a multiple of 256): clusters of C CTAs own tiles of
 // M rows, the C ranks split K.  (C, M) is picked at launch by balanced cost.
-constexpr int kSmallT = 32;
+constexpr int kSmallT = 16;   // above this the large-T path is faster (measured)
 struct SmallPlan {
     bool ok = false;
     int nt8 = 1, kt = 0;
@@ -159,7 +159,7 @@ SmallPlan make_small_plan(int64_t T, int64_t d_out, int64_t d_in) {
     SmallPlan sp;
     (void)d_out;
     if (T < 1 || T > kSmallT) return sp;
-    sp.nt8 = T <= 8 ? 1 : (T <= 16 ? 2 : 4);
+    sp.nt8 = T <= 8 ? 1 : 2;
     sp.kt = static_cast<int>(d_in / 64);
     sp.ok = sp.kt % 4 == 0;
     return sp;
@@ -373,6 +373,10 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
     return QLORA_OK;
 }
 
+// The stream kernel leaves 8 SMs to the U pre-pass (which takes ceil(r / 8) <= 16 CTAs), so the
+// two run side by side.
+constexpr int kGvStreamSms = kSmsForSplit - 8;
+
 // Decode-size forward: the U pre-pass overlapped with the weight stream through programmatic
 // dependent launch; the stream kernel runs as clusters of C CTAs over tiles of M rows.
 template <int NT8>
@@ -414,7 +418,7 @@ qlora_status launch_qgemv(const qlora_nf4* w, const void* X, int64_t T, GvArgs g
         int n = fit[dev & 63][e].load();
         if (n == 0) {
             if (C == 1) {
-                n = kSmsForSplit;
+                n = kGvStreamSms;
             } else {
                 attr[1].val.clusterDim.x = static_cast<unsigned>(C);
                 cfg.gridDim = dim3(static_cast<unsigned>(C * (kSmsForSplit / C)));
@@ -424,14 +428,16 @@ qlora_status launch_qgemv(const qlora_nf4* w, const void* X, int64_t T, GvArgs g
                     cudaGetLastError();
                     m = 0;
                 }
-                n = std::min(m, kSmsForSplit / C);
+                n = std::min(m, kGvStreamSms / C);
             }
             if (n <= 0) n = -1;
             fit[dev & 63][e].store(n);
         }
         if (n < 0) continue;
         const int64_t nbk = 4 * cdiv(q4, C);
-        for (int M = 16; M <= 16 * GvCfg<NT8>::MW && M * nbk <= kGvTabAbs && M * g.kt / 256 + 2 <= kGvTabC2; M += 16) {
+        for (int M = 16; M <= 16 * GvCfg<NT8>::MW && M * (nbk + 1) <= kGvTabS &&
+                        M * g.kt / 256 + 2 <= kGvRawC2 &&
+                        (!g.b_vec || M * (g.r + 8) <= kGvBrowMax); M += 16) {
             const int64_t tiles = cdiv(d_out, M);
             const int64_t clusters = std::min<int64_t>(n, tiles);
             const int64_t tpc = cdiv(tiles, clusters);
@@ -475,7 +481,7 @@ qlora_status small_fwd(const qlora_nf4* w, const void* X, int64_t T, const void*
     const SmallPlan sp = make_small_plan(T, d_out, d_in);
     if (!sp.ok) return QLORA_ERR_UNSUPPORTED;
     float* us = at<float>(ws, p.s_us);
-    k_small_u<<<dim3(static_cast<unsigned>(r), static_cast<unsigned>(cdiv(T, 4))), 128, 0, st>>>(
+    k_small_u<<<static_cast<unsigned>(cdiv(r, 8)), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(X), static_cast<int>(T), static_cast<int>(d_in),
         static_cast<const __nv_bfloat16*>(A), r, s, us, static_cast<__nv_bfloat16*>(U_save));
     QL_LAUNCH_CHECK();
@@ -495,8 +501,7 @@ qlora_status small_fwd(const qlora_nf4* w, const void* X, int64_t T, const void*
     g.err = err;
     g.wait_ns = kWaitNs;
     if (sp.nt8 == 1) return launch_qgemv<1>(w, X, T, g, st);
-    if (sp.nt8 == 2) return launch_qgemv<2>(w, X, T, g, st);
-    return launch_qgemv<4>(w, X, T, g, st);
+    return launch_qgemv<2>(w, X, T, g, st);
 }
 
 qlora_status sgemm(cudaStream_t st, int64_t M, int64_t N, int64_t K, float alpha, const float* A,
