@@ -186,6 +186,8 @@ def run_gpu(args):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.only == "decode":
+        return run_decode_only(args, q, qb, S, torch, dev)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -355,6 +357,40 @@ def run_gpu(args):
     return 0
 
 
+def run_decode_only(args, q, qb, S, torch, dev):
+    """The decode-size forward alone on the 11008 x 4096 MLP shape (r = 64): W warm-up and K
+    timed eager calls over 8 rotating NF4 weights (> L2), for profiling its kernels."""
+    qb.build_library()
+    q.load()
+    bf = torch.bfloat16
+    c3 = S.CONFIGS["mlp_up_11008x4096_r64_T8192"]
+    d, k, r, alpha, T = c3["d_out"], c3["d_in"], c3["r"], c3["alpha"], args.tokens
+    base = S.make_layer(d, k, r, alpha, T, dtype="bf16", seed=7, with_grad=False)
+    W0 = torch.from_numpy(base.W0).to(dev)
+    wl = [q.nf4_quantize(W0) for _ in range(8)]
+    del W0
+    X = torch.from_numpy(base.X).to(dev).to(bf)
+    A = torch.from_numpy(base.A).to(dev).to(bf)
+    B = torch.from_numpy(base.B).to(dev).to(bf)
+    H = torch.empty((T, d), dtype=bf, device=dev)
+    ws = torch.empty(q.workspace_bytes(q.OP_FWD, q.BF16, T, d, k, r), dtype=torch.uint8, device=dev)
+    W = max(3, args.warmup)
+    for i in range(W):
+        q.qlora_linear_fwd(wl[i % 8], X, A, B, alpha, H=H, ws=ws, save_u=False)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        q.qlora_linear_fwd(wl[i % 8], X, A, B, alpha, H=H, ws=ws, save_u=False)
+    e1.record()
+    torch.cuda.synchronize()
+    err = q.get_device_error()
+    print(json.dumps({"only": "decode", "tokens": T, "ms_per_call": e0.elapsed_time(e1) / args.steps,
+                      "device_error": err, "workload": "mlp_up_11008x4096_r64 decode-size forward"}),
+          flush=True)
+    return 0 if err == 0 else 1
+
+
 def _graph_time(torch, calls, reps=20):
     """Per-call device time of `calls` (a list of zero-argument launches) captured in one CUDA
     graph and replayed `reps` times: (median, min) microseconds per call over 5 measurements."""
@@ -498,8 +534,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--extra", action="store_true", help="also time the other hot-path rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--only", default="step", choices=["step", "fwd", "bwd"],
-                    help="time only the forward or only the backward call")
+    ap.add_argument("--only", default="step", choices=["step", "fwd", "bwd", "decode"],
+                    help="time only the forward, only the backward, or the decode-size forward "
+                         "(11008x4096, r = 64, --tokens T) alone, for profiling one kernel")
+    ap.add_argument("--tokens", type=int, default=1, help="tokens of the --only decode run")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

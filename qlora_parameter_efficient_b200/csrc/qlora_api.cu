@@ -764,8 +764,9 @@ qlora_status lora_merge(const qlora_nf4* w, const void* A, const void* B, int32_
     if (!aligned16(A) || !aligned16(B) || !aligned16(W_final)) return QLORA_ERR_INVALID_ARG;
     if (r < 1 || r > 128) return QLORA_ERR_UNSUPPORTED;
     const float s = alpha / static_cast<float>(r);
-    dim3 grid(static_cast<unsigned>(cdiv(w->d_in, 256)), static_cast<unsigned>(cdiv(w->d_out, 32)));
-    const size_t smem = static_cast<size_t>(r) * 256 * 4 + 32 * static_cast<size_t>(r) * 4;
+    dim3 grid(static_cast<unsigned>(cdiv(w->d_in, 128)), static_cast<unsigned>(cdiv(w->d_out, 64)));
+    const size_t rp = static_cast<size_t>((r + 15) & ~15);
+    const size_t smem = rp * 128 * 4 + 64 * rp * 4;
     auto run = [&](auto kern, auto a, auto b, auto o) -> qlora_status {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)

@@ -204,8 +204,12 @@ __global__ void k_mask_multi_f32(float* __restrict__ U, int64_t T, int R, int n_
 // ------------------------------------------------------------------ merge
 
 // W_final[n, kk] = W^[n, kk] + s * sum_j B[n, j] A[j, kk]; W^ is the decoded weight in the
-// output dtype's decode (bf16 decode for bf16 output).  Tile: 32 rows x 256 columns; each
-// thread owns one column.  A tile and B rows staged in shared memory in fp32.
+// output dtype's decode (bf16 decode for bf16 output).  Tile: 64 rows x 128 columns, 256
+// threads; thread (tx, ty) owns columns 2tx, 2tx+1 (one code byte per row) of rows
+// 16ty .. 16ty+15.  The A tile is staged in shared memory in fp32 and read 16 adapter rows
+// at a time into registers, the B rows are read as 4-wide broadcasts, so the products run at
+// FMA rate; each element's sum over j is formed in j order (fp32 FMA), as before.  The level
+// table sits in shared memory (a lookup by code would serialise in the constant cache).
 template <typename TA, typename TOut>
 __global__ void __launch_bounds__(256) k_merge(const uint8_t* __restrict__ codes,
                                                const uint8_t* __restrict__ absmax_q,
@@ -214,24 +218,27 @@ __global__ void __launch_bounds__(256) k_merge(const uint8_t* __restrict__ codes
                                                const TA* __restrict__ B, int r, float s,
                                                TOut* __restrict__ out) {
     extern __shared__ float msm[];
-    float* sA = msm;                 // [r][256]
-    float* sB = msm + r * 256;       // [32][r]
-    __shared__ float sscale[32][4];
-    const int64_t row0 = static_cast<int64_t>(blockIdx.y) * 32;
-    const int64_t col0 = static_cast<int64_t>(blockIdx.x) * 256;
+    const int rp = (r + 15) & ~15;   // adapter rank padded to 16
+    float* sA = msm;                 // [rp][128]
+    float* sB = msm + rp * 128;      // [64][rp]
+    __shared__ float sscale[64][2];
+    __shared__ float s_lv[16];
+    const int64_t row0 = static_cast<int64_t>(blockIdx.y) * 64;
+    const int64_t col0 = static_cast<int64_t>(blockIdx.x) * 128;
     const int tid = threadIdx.x;
-    for (int i = tid; i < r * 256; i += 256) {
-        const int j = i / 256, c = i % 256;
+    if (tid < 16) s_lv[tid] = c_nf4_levels[tid];
+    for (int i = tid; i < rp * 128; i += 256) {
+        const int jj = i / 128, c = i % 128;
         const int64_t gc = col0 + c;
-        sA[i] = gc < d_in ? to_f(A[j * d_in + gc]) : 0.f;
+        sA[i] = (jj < r && gc < d_in) ? to_f(A[jj * d_in + gc]) : 0.f;
     }
-    for (int i = tid; i < 32 * r; i += 256) {
-        const int rr = i / r, j = i % r;
+    for (int i = tid; i < 64 * rp; i += 256) {
+        const int rr = i / rp, jj = i % rp;
         const int64_t gr = row0 + rr;
-        sB[i] = gr < d_out ? to_f(B[gr * r + j]) : 0.f;
+        sB[i] = (jj < r && gr < d_out) ? to_f(B[gr * r + jj]) : 0.f;
     }
     if (tid < 128) {
-        const int rr = tid >> 2, cb = tid & 3;
+        const int rr = tid >> 1, cb = tid & 1;
         const int64_t gr = row0 + rr, gcb = col0 / 64 + cb;
         float sc = 0.f;
         if (gr < d_out && gcb < d_in / 64) {
@@ -241,21 +248,50 @@ __global__ void __launch_bounds__(256) k_merge(const uint8_t* __restrict__ codes
         sscale[rr][cb] = sc;
     }
     __syncthreads();
-    const int64_t gc = col0 + tid;
+    const int tx = tid & 63, ty = tid >> 6;
+    const int64_t gc = col0 + 2 * tx;
     if (gc >= d_in) return;
-    for (int rr = 0; rr < 32; ++rr) {
+    float acc[16][2];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = 0.f;
+    for (int j0 = 0; j0 < rp; j0 += 16) {
+        float2 a[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) a[jj] = *reinterpret_cast<const float2*>(sA + (j0 + jj) * 128 + 2 * tx);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float* brow = sB + (16 * ty + i) * rp + j0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 b4 = *reinterpret_cast<const float4*>(brow + 4 * q);
+                const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    acc[i][0] = fmaf(bv[e], a[4 * q + e].x, acc[i][0]);
+                    acc[i][1] = fmaf(bv[e], a[4 * q + e].y, acc[i][1]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int rr = 16 * ty + i;
         const int64_t gr = row0 + rr;
-        if (gr >= d_out) break;
+        if (gr >= d_out) continue;
         const int64_t e = gr * d_in + gc;
         const uint32_t byte = codes[e >> 1];
-        const uint32_t code = (e & 1) ? (byte >> 4) : (byte & 15u);
-        float w = __fmul_rn(c_nf4_levels[code], sscale[rr][tid >> 6]);
-        if constexpr (sizeof(TOut) == 2) w = __bfloat162float(__float2bfloat16_rn(w));
-        float acc = 0.f;
-        for (int j = 0; j < r; ++j) acc = fmaf(sB[rr * r + j], sA[j * 256 + tid], acc);
-        const float v = w + s * acc;
-        if constexpr (sizeof(TOut) == 2) out[e] = __float2bfloat16_rn(v);
-        else out[e] = v;
+        const float sc = sscale[rr][tx >> 5];
+        float w0 = __fmul_rn(s_lv[byte & 15u], sc), w1 = __fmul_rn(s_lv[byte >> 4], sc);
+        if constexpr (sizeof(TOut) == 2) {
+            w0 = __bfloat162float(__float2bfloat16_rn(w0));
+            w1 = __bfloat162float(__float2bfloat16_rn(w1));
+        }
+        const float v0 = w0 + s * acc[i][0], v1 = w1 + s * acc[i][1];
+        if constexpr (sizeof(TOut) == 2) {
+            *reinterpret_cast<__nv_bfloat162*>(out + e) = __floats2bfloat162_rn(v0, v1);
+        } else {
+            *reinterpret_cast<float2*>(out + e) = make_float2(v0, v1);
+        }
     }
 }
 
