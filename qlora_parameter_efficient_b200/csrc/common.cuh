@@ -108,9 +108,22 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
     return r;
 }
 
+// Arrive on a barrier in another CTA of the cluster with cluster-scope release: the arriving
+// thread's earlier generic-proxy writes (e.g. st.shared::cluster into the target CTA) are
+// visible to a thread that acquires the completed phase.  Measured at ~0.5 us per call on
+// sm_100a, so it is kept off per-K-step paths.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
+}
+
+// Remote arrive with the default (CTA-scope) release, the form CUTLASS's 2-SM pipelines use
+// for hand-offs whose payload is consumed by the tensor core: shared-memory tiles already
+// handed to the async proxy (fence.proxy.async before the arrive), or tensor-memory reads
+// retired with tcgen05.wait::ld + tcgen05.fence::before_thread_sync.  Not for generic-proxy
+// data that a thread of the target CTA reads with ordinary loads (use mbar_arrive_remote).
+__device__ __forceinline__ void mbar_arrive_remote_async_payload(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t addr, uint32_t parity) {

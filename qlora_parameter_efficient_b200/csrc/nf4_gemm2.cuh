@@ -9,7 +9,13 @@
 // the weight tile and every decoded weight feeds 256 tokens; each CTA's tensor memory holds
 // its 128 accumulator rows x 256 columns, double-buffered (512 columns) so the epilogue of one
 // tile overlaps the main loop of the next.  The grid is persistent: pair p handles tiles
-// p, p + npairs, ...
+// p, p + npairs, ...  When the last wave would leave most pairs idle (its tile count is at most
+// half the pairs), its tiles are each split in two along K and run on two pairs: the first half
+// takes main K steps [0, k/2), the second the rest plus the adapter steps.  Each epilogue warp
+// of a split tile writes its fp32 partial (32 rows x 256 columns) to a workspace slot and takes
+// a ticket from a per-warp counter; the second finisher adds the other half's partial to its
+// own and writes the bf16 output.  fp32 addition of two terms is commutative, so the result does
+// not depend on which half finishes first, and no CTA ever waits for another.
 //
 // Warp roles per CTA (6 + 4 x decoder groups warps):
 //   warp 0       TMA producer: this CTA's A half and NF4 code tile (or the K-extension
@@ -25,9 +31,14 @@
 //                B half (one block per thread, written in the 128-byte-swizzled UMMA layout),
 //                then arrive on a local barrier: the leader's ready[s] directly, the peer's
 //                dec_done[s], which the peer's warp 1 forwards to the leader's ready[s] with
-//                one cluster-scope release.  For the adapter K steps the group only reports
+//                one remote arrive.  For the adapter K steps the group only reports
 //                "landed".  ready[s] thus certifies, for both CTAs, that the A half has
 //                landed and the B half is in place.
+// The peer's remote arrives (ready, acc_empty) carry no generic-proxy payload: the decoded
+// tile was handed to the async proxy by fence.proxy.async in every writing thread, and TMEM
+// reads are retired by tcgen05.wait::ld before tcgen05.fence::before_thread_sync; so they use
+// the default CTA-scope release (a cluster-scope release costs ~0.5 us per arrive and, made
+// once per K step by one thread, set the step period).
 // Every wait is bounded (QLORA_ERR_TIMEOUT on expiry); all TMA loads are plain local loads.
 #pragma once
 
@@ -116,9 +127,16 @@ struct Gemm2Args {
     int nf4_bpr;           // d_in / 64
     __nv_bfloat16* out;
     int64_t ld_out;
+    int split_tiles;       // trailing tiles split in two along K (0 = none)
+    float* part;           // [split_tiles][2 ranks][4 warps][2 halves][2048 float4] fp32 partials
+    int* cnt;              // [split_tiles][2 ranks][4 warps] tickets, zero at launch
     int* err;
     uint64_t wait_ns;
 };
+
+// Float4 index of (row = lane, columns 32c + 4g .. +3) in a warp's 32 x 256 partial slot:
+// consecutive lanes of one store are consecutive 16-byte words.
+__device__ __forceinline__ int g2_part_idx(int c, int g, int lane) { return (c * 8 + g) * 32 + lane; }
 
 template <bool B_MN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
@@ -150,8 +168,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
     const int npairs = gridDim.x >> 1;
     const int n_tiles_total = args.m_tiles * args.n_tiles;
     const int iters_per_tile = args.k_steps + args.ext_steps;
-    const int my_tiles = (n_tiles_total - pair + npairs - 1) / npairs;
-    const int total_iters = max(0, my_tiles) * iters_per_tile;
+    // Schedule of this pair: n_full whole tiles pair, pair + npairs, ..., then (split only)
+    // one half tile, K steps [hb, he) of tile half_tile.
+    const int split_base = n_tiles_total - args.split_tiles;   // a multiple of npairs when split
+    int n_full, half = -1, half_tile = 0, hb = 0, he = 0;
+    if (args.split_tiles > 0) {
+        n_full = split_base / npairs;
+        if (pair < 2 * args.split_tiles) {
+            half = pair & 1;
+            half_tile = split_base + (pair >> 1);
+            const int h0 = args.k_steps / 2;
+            hb = half ? h0 : 0;
+            he = half ? iters_per_tile : h0;
+        }
+    } else {
+        n_full = max(0, (n_tiles_total - pair + npairs - 1) / npairs);
+    }
+    const int n_units = n_full + (half >= 0 ? 1 : 0);
+    const int full_iters = n_full * iters_per_tile;
+    const int total_iters = full_iters + (half >= 0 ? he - hb : 0);
+    // (tile, K step within the tile) of this pair's git-th step
+    auto step_of = [&](int git, int& tile, int& ks) {
+        if (git < full_iters) {
+            tile = pair + (git / iters_per_tile) * npairs;
+            ks = git % iters_per_tile;
+        } else {
+            tile = half_tile;
+            ks = hb + (git - full_iters);
+        }
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SA; ++s) {
@@ -208,8 +253,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
         if (lane == 0) {
             int issued = 0;
             for (int git = 0; git < total_iters; ++git) {
-                const int it = git % iters_per_tile;
-                const int tile = pair + (git / iters_per_tile) * npairs;
+                int tile, it;
+                step_of(git, tile, it);
                 const int m0 = (tile % args.m_tiles) * 256 + static_cast<int>(rank) * 128;
                 const int n0 = (tile / args.m_tiles) * 256 + static_cast<int>(rank) * 128;
                 const int s = git % SA;
@@ -257,16 +302,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             const uint32_t idesc = make_idesc_bf16(256, 256, false, B_MN);
             int git = 0;
             bool ok = true;
-            for (int tc = 0; ok && tc < my_tiles; ++tc) {
+            for (int tc = 0; ok && tc < n_units; ++tc) {
                 const int buf = tc & 1;
                 const uint32_t aph = (tc >> 1) & 1;
+                const int it0 = tc < n_full ? 0 : hb;
+                const int it1 = tc < n_full ? iters_per_tile : he;
                 if (!mbar_wait_cluster(&acc_empty[buf], aph ^ 1, abort, args.wait_ns)) {
                     fail();
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * 256);
-                for (int it = 0; it < iters_per_tile; ++it, ++git) {
+                for (int it = it0; it < it1; ++it, ++git) {
                     const int s = git % SA;
                     const int sb = git % SB;
                     if (!mbar_wait_cluster(&ready[s], (git / SA) & 1, abort, args.wait_ns)) {
@@ -282,7 +329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
                         const uint64_t ad = make_sw128_desc(a + k * 32, 16, 1024);
                         const uint64_t bd = B_MN ? make_sw128_desc(b + k * 2048, 8192, 1024)
                                                  : make_sw128_desc(b + k * 32, 16, 1024);
-                        umma_bf16_ss_2sm(d_tmem, ad, bd, idesc, (it > 0 || k > 0) ? 1u : 0u);
+                        umma_bf16_ss_2sm(d_tmem, ad, bd, idesc, (it > it0 || k > 0) ? 1u : 0u);
                     }
                     umma_commit_2sm_both(&empty[s]);
                 }
@@ -299,15 +346,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
                     fail();
                     break;
                 }
-                mbar_arrive_remote(ready_leader + static_cast<uint32_t>(s * 8));
+                mbar_arrive_remote_async_payload(ready_leader + static_cast<uint32_t>(s * 8));
             }
         }
     } else if (warp < 6) {
         // -------------------------------------------------------------- epilogue
         const int q = warp & 3;                    // TMEM lane quarter of this warp
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
-        for (int tc = 0; tc < my_tiles; ++tc) {
-            const int tile = pair + tc * npairs;
+        for (int tc = 0; tc < n_units; ++tc) {
+            const bool is_half = tc >= n_full;
+            const int tile = is_half ? half_tile : pair + tc * npairs;
             const int buf = tc & 1;
             const uint32_t aph = (tc >> 1) & 1;
             if (!mbar_wait_warp(&accf[buf], aph, abort, args.wait_ns)) {
@@ -320,11 +368,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             const int gc0 = nt * 256;
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(buf * 256);
+            const float4* other = nullptr;
+            if (is_half) {
+                // publish this half's partial, then take a ticket: the second finisher adds
+                const int64_t slot = (static_cast<int64_t>(half_tile - split_base) * 2 + rank) * 4 + q;
+                float4* mine = reinterpret_cast<float4*>(args.part) + ((slot * 2 + half) << 11);
 #pragma unroll 1
-            for (int c0 = 0; c0 < 256; c0 += 32) {
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tbase + c * 32, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        mine[g2_part_idx(c, g, lane)] =
+                            make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                        __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
+                }
+                __threadfence();
+                __syncwarp();
+                int ticket = 0;
+                if (lane == 0) ticket = atomicAdd(args.cnt + slot, 1);
+                ticket = __shfl_sync(0xffffffffu, ticket, 0);
+                if (ticket == 1) {
+                    __threadfence();
+                    other = reinterpret_cast<const float4*>(args.part) + ((slot * 2 + (half ^ 1)) << 11);
+                }
+            }
+#pragma unroll 1
+            for (int c0 = 0; c0 < 256 && (!is_half || other != nullptr); c0 += 32) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + c0, r);
                 tmem_ld_wait();
+                if (other != nullptr) {
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        const float4 o = __ldcg(other + g2_part_idx(c0 >> 5, g, lane));
+                        r[4 * g + 0] = __float_as_uint(__uint_as_float(r[4 * g + 0]) + o.x);
+                        r[4 * g + 1] = __float_as_uint(__uint_as_float(r[4 * g + 1]) + o.y);
+                        r[4 * g + 2] = __float_as_uint(__uint_as_float(r[4 * g + 2]) + o.z);
+                        r[4 * g + 3] = __float_as_uint(__uint_as_float(r[4 * g + 3]) + o.w);
+                    }
+                }
                 if (grow < args.M) {
                     const int gc = gc0 + c0;
                     __nv_bfloat16* o = args.out + grow * args.ld_out + gc;
@@ -343,7 +427,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(acc_empty_leader + static_cast<uint32_t>(buf * 8));
+            if (lane == 0) mbar_arrive_remote_async_payload(acc_empty_leader + static_cast<uint32_t>(buf * 8));
         }
     } else {
         // -------------------------------------------------------------- NF4 decoders
@@ -358,9 +442,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             blk_col_off = 0;
         }
         auto block_at = [&](int git) -> int64_t {
-            const int it = git % iters_per_tile;
+            int tile, it;
+            step_of(git, tile, it);
             if (it >= args.k_steps) return -1;
-            const int tile = pair + (git / iters_per_tile) * npairs;
             const int n0 = (tile / args.m_tiles) * 256 + static_cast<int>(rank) * 128;
             int64_t wrow, wblk;
             if (B_MN) {
@@ -408,7 +492,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
         bool have = false;          // dec[] holds step `git` (decoded ahead)
         for (int git = grp; git < total_iters; git += kG2DecGroups) {
             const int s = git % SA;
-            const int it = git % iters_per_tile;
+            int tile_unused, it;
+            step_of(git, tile_unused, it);
             const bool main_step = it < args.k_steps;
             if (!have) {
                 // (first step, or after an adapter step) decode now
@@ -445,7 +530,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             // decode the next handled step ahead, as soon as its codes have landed
             have = false;
             const int gn = git + kG2DecGroups;
-            if (gn < total_iters && (gn % iters_per_tile) < args.k_steps) {
+            int tile_gn = 0, it_gn = 0;
+            if (gn < total_iters) step_of(gn, tile_gn, it_gn);
+            if (gn < total_iters && it_gn < args.k_steps) {
                 const int64_t blk = blk_nxt;
                 Nf4Planes p{};
                 if (blk >= 0) p = nf4_make_planes(nf4_block_scale(q8_nxt, c2_nxt));

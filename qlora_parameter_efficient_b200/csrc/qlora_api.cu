@@ -165,6 +165,26 @@ SmallPlan make_small_plan(int64_t T, int64_t d_out, int64_t d_in) {
     return sp;
 }
 
+// Persistent schedule of the fused NF4 GEMM: pairs of SMs, and how many trailing tiles are
+// split in two along K (only when the last wave has at most half the pairs' worth of tiles).
+struct G2Sched {
+    int pairs = 1, split_tiles = 0;
+    size_t part_bytes = 0, cnt_bytes = 0;
+    size_t bytes() const { return part_bytes + cnt_bytes; }
+};
+G2Sched g2_schedule(int64_t T, int64_t N, int64_t K) {
+    G2Sched g;
+    const int64_t tiles = cdiv(T, 256) * cdiv(N, 256);
+    g.pairs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, kSmsForSplit / 2)));
+    const int64_t rem = tiles % g.pairs;
+    if (tiles > g.pairs && rem > 0 && 2 * rem <= g.pairs && cdiv(K, 64) >= 2) {
+        g.split_tiles = static_cast<int>(rem);
+        g.part_bytes = align256(static_cast<size_t>(rem) * 2 * 4 * 2 * 2048 * 16);
+        g.cnt_bytes = align256(static_cast<size_t>(rem) * 2 * 4 * sizeof(int));
+    }
+    return g;
+}
+
 struct Plan {
     int RP = 0;
     bool small = false;
@@ -172,6 +192,7 @@ struct Plan {
     int split_u = 1, split_g = 1, split_da = 1, split_db = 1;
     size_t a_pad = 0, b_pad = 0, u_spad = 0, u_pad = 0, g_spad = 0, part = 0;
     size_t w32 = 0, uf = 0, gf = 0;
+    size_t g2 = 0;         // fused-GEMM split-tail partials and tickets
     size_t total = 0;
 };
 
@@ -211,6 +232,9 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
             part = std::max(part, static_cast<size_t>(p.split_db) * d_out * RP * 4);
         }
         p.part = take(part);
+        const size_t g2 = op == QLORA_OP_BWD ? g2_schedule(T, d_in, d_out).bytes()
+                                             : g2_schedule(T, d_out, d_in).bytes();
+        p.g2 = take(g2);
     } else {
         p.w32 = take(static_cast<size_t>(d_out) * d_in * 4);
         if (op == QLORA_OP_FWD_BATCHED) {
@@ -324,7 +348,7 @@ qlora_status skinny_gemm(bool a_mn, bool b_mn, int RP, const CUtensorMap& ta,
 //   forward (dx = false): out[T, d_out]  = act[T, d_in]  W^T + ext_a[T, RP] ext_b[d_out, RP]^T
 //   dX      (dx = true):  out[T, d_in]   = act[T, d_out] W   + ext_a[T, RP] ext_b[RP, d_in]
 qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, const void* ext_a,
-                      const void* ext_b, int RP, int r_used, void* out, int* err,
+                      const void* ext_b, int RP, int r_used, void* out, void* g2ws, int* err,
                       cudaStream_t st) {
     const int64_t d_out = w->d_out, d_in = w->d_in;
     CUtensorMap ta, tc, tax, tbx;
@@ -352,8 +376,14 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
     g.ld_out = N;
     g.err = err;
     g.wait_ns = kWaitNs;
-    const int tiles = g.m_tiles * g.n_tiles;
-    const int pairs = std::max(1, std::min(tiles, kSmsForSplit / 2));
+    const G2Sched sch = g2_schedule(T, N, K);
+    const int pairs = sch.pairs;
+    g.split_tiles = sch.split_tiles;
+    if (sch.split_tiles > 0) {
+        if (!g2ws || (reinterpret_cast<uintptr_t>(g2ws) & 255u)) return QLORA_ERR_INVALID_ARG;
+        g.part = static_cast<float*>(g2ws);
+        g.cnt = reinterpret_cast<int*>(static_cast<uint8_t*>(g2ws) + sch.part_bytes);
+    }
     auto kern = dx ? k_nf4_gemm2<true> : k_nf4_gemm2<false>;
     static std::atomic<uint64_t> configured[2] = {0, 0};
     int dev = 0;
@@ -365,6 +395,8 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
             return QLORA_ERR_CUDA;
         configured[dx].fetch_or(bit);
     }
+    if (sch.split_tiles > 0 && cudaMemsetAsync(g.cnt, 0, sch.cnt_bytes, st) != cudaSuccess)
+        return QLORA_ERR_CUDA;
     const bool ev = g_ev_start && g_ev_stop;
     if (ev) cudaEventRecord(g_ev_start, st);
     kern<<<2 * pairs, kG2Threads, G2Smem::kTotal, st>>>(ta, tc, tax, tbx, g);
@@ -657,7 +689,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T, cons
         QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
         QL_TRY(compute_u_bf16(X, T, d_in, a_pad, RP, r, s, p.split_u, part,
                               static_cast<__nv_bfloat16*>(U_save), nullptr, u_spad, err, stream));
-        return nf4_gemm(false, w, X, T, u_spad, b_pad, RP, r, H, err, stream);
+        return nf4_gemm(false, w, X, T, u_spad, b_pad, RP, r, H, at<void>(ws, p.g2), err, stream);
     }
     // exact fp32 path
     float* w32 = at<float>(ws, p.w32);
@@ -710,7 +742,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
             QL_LAUNCH_CHECK();
         }
         // dX = dH W^ + (sG) A
-        if (dX) QL_TRY(nf4_gemm(true, w, dH, T, g_spad, a_pad, RP, r, dX, err, stream));
+        if (dX) QL_TRY(nf4_gemm(true, w, dH, T, g_spad, a_pad, RP, r, dX, at<void>(ws, p.g2), err, stream));
         // dA^T[d_in, RP] = X^T (sG)
         {
             CUtensorMap txm, tgm;
@@ -843,7 +875,7 @@ qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t
                                                              n_adapters, adapter_id, seg, u_all,
                                                              nullptr, err);
         QL_LAUNCH_CHECK();
-        return nf4_gemm(false, w, X, T, u_all, b_cat, RP, R, H, err, stream);
+        return nf4_gemm(false, w, X, T, u_all, b_cat, RP, R, H, at<void>(ws, p.g2), err, stream);
     }
     // exact fp32 path
     float* w32 = at<float>(ws, p.w32);

@@ -123,6 +123,18 @@ def test_layer_bf16_small(q, d_out, d_in, r, T):
     run_layer(q, case)
 
 
+# Shapes whose fused-GEMM tile count leaves a short last wave on 74 SM pairs, so that wave's
+# tiles are split in two along K and reduced through the fp32 partial workspace:
+#   (2048, 2048, 16, 2560): 80 tiles in forward and dX (6 split);
+#   (3272, 640, 7, 1500): forward 78 tiles (4 split, ragged columns and rows);
+#   (1000, 3264, 9, 1500): dX 78 tiles (4 split, ragged columns), ragged K = 1000.
+@pytest.mark.parametrize("d_out,d_in,r,T", [(2048, 2048, 16, 2560), (3272, 640, 7, 1500),
+                                            (1000, 3264, 9, 1500)])
+def test_layer_bf16_split_tail(q, d_out, d_in, r, T):
+    case = S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_in + r)
+    run_layer(q, case)
+
+
 @pytest.mark.parametrize("d_out,d_in,r,T", [(256, 256, 8, 64), (200, 192, 5, 77), (64, 128, 3, 1)])
 def test_layer_f32(q, d_out, d_in, r, T):
     case = S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="f32", seed=3)
