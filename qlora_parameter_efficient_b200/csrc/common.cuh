@@ -83,13 +83,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// Warp-wide wait: lane 0 polls, the other lanes are released by __syncwarp (which orders
-// memory among the warp's threads) once it has seen the phase complete.
+// Warp-wide wait: every lane polls the barrier itself (the warp stays converged; lanes parked
+// at a __syncwarp behind one polling lane measured markedly slower on sm_100a, and they slow
+// the other warps of their scheduler), and lane 0's verdict is broadcast so that the warp
+// leaves the wait together even when a time limit expires in some lanes only.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
                                                volatile int* abort, uint64_t limit_ns) {
-    uint32_t ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, limit_ns) ? 1u : 0u;
-    __syncwarp();
+    const uint32_t ok = mbar_wait(bar, parity, abort, limit_ns) ? 1u : 0u;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 

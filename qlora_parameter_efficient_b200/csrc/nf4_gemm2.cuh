@@ -20,7 +20,7 @@
 // Warp roles per CTA (6 + 4 x decoder groups warps):
 //   warp 0       TMA producer: this CTA's A half and NF4 code tile (or the K-extension
 //                adapter tiles) into an 8-stage ring, completing on the local full[s]; the
-//                decoded B halves live in a separate, shallower 3-slot ring (the adapter K
+//                decoded B halves live in a separate, shallower 4-slot ring (the adapter K
 //                step's B tile is loaded straight into its slot).
 //   warp 1       leader CTA only: issues the MMAs, commits stage release (empty[s]) and
 //                accumulator-ready (accf[b]) to both CTAs.
@@ -338,7 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
         }
         if (rank == 1 && lane == 0) {
             // ---------------------------------------------------------- peer forwarder
-            // One cluster-scope release per K step on the leader's ready[s].
+            // One remote arrive per K step on the leader's ready[s].
             const uint32_t ready_leader = mapa_shared(smem_u32(&ready[0]), 0);
             for (int git = 0; git < total_iters; ++git) {
                 const int s = git % SA;
