@@ -139,7 +139,8 @@ qlora_status tmap_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t col
 // ======================================================================= planning
 
 int choose_split(int64_t tiles, int64_t k_steps) {
-    int64_t s = cdiv(2 * kSmsForSplit, std::max<int64_t>(tiles, 1));
+    // the skinny kernel fits two CTAs per SM: fill one wave of 2 x 148 slots, never more
+    int64_t s = std::max<int64_t>(1, (2 * kSmsForSplit) / std::max<int64_t>(tiles, 1));
     s = std::min<int64_t>(s, std::max<int64_t>(1, k_steps / 4));
     s = std::max<int64_t>(1, std::min<int64_t>(s, 32));
     const int64_t per = cdiv(k_steps, s);
@@ -323,10 +324,11 @@ GemmArgs base_args(int M, int N, int k_steps, int* err) {
 
 // Skinny tensor-core contraction D[M, RP] = sum_K A[M,K] B[RP,K] written as fp32 split-K
 // partials.  a_mn / b_mn give the operand majorness of the two TMA maps.
-qlora_status skinny_gemm(bool a_mn, bool b_mn, int RP, const CUtensorMap& ta,
+qlora_status skinny_gemm(bool a_mn, bool b_mn, int RP, int n_valid, const CUtensorMap& ta,
                          const CUtensorMap& tb, int64_t M, int64_t k_steps, int split,
                          float* part, int* err, cudaStream_t st) {
-    GemmArgs g = base_args(static_cast<int>(M), RP, static_cast<int>(k_steps), err);
+    // partial columns >= n_valid are never read: only the first n_valid are stored
+    GemmArgs g = base_args(static_cast<int>(M), n_valid, static_cast<int>(k_steps), err);
     g.split = split;
     g.out = part;
     g.ld_out = RP;
@@ -347,9 +349,11 @@ qlora_status skinny_gemm(bool a_mn, bool b_mn, int RP, const CUtensorMap& ta,
 // Fused NF4-decode GEMM with the adapter K-extension (persistent 2-SM kernel).
 //   forward (dx = false): out[T, d_out]  = act[T, d_in]  W^T + ext_a[T, RP] ext_b[d_out, RP]^T
 //   dX      (dx = true):  out[T, d_in]   = act[T, d_out] W   + ext_a[T, RP] ext_b[RP, d_in]
+// ext_b_rank: the rank extent stored in ext_b (RP for a zero-padded copy, or the caller's r
+// when the TMA zero-fills the rank padding out of bounds).
 qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, const void* ext_a,
-                      const void* ext_b, int RP, int r_used, void* out, void* g2ws, int* err,
-                      cudaStream_t st) {
+                      const void* ext_b, int RP, int r_used, int ext_b_rank, void* out,
+                      void* g2ws, int* err, cudaStream_t st) {
     const int64_t d_out = w->d_out, d_in = w->d_in;
     CUtensorMap ta, tc, tax, tbx;
     const int64_t K = dx ? d_out : d_in;
@@ -358,8 +362,8 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
     if (dx) QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 64, 64));
     else QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 32, 128));
     QL_TRY(tmap_bf16(&tax, ext_a, T, RP, RP, 128));
-    if (dx) QL_TRY(tmap_bf16(&tbx, ext_b, RP, d_in, d_in, 64));
-    else QL_TRY(tmap_bf16(&tbx, ext_b, d_out, RP, RP, 128));
+    if (dx) QL_TRY(tmap_bf16(&tbx, ext_b, ext_b_rank, d_in, d_in, 64));
+    else QL_TRY(tmap_bf16(&tbx, ext_b, d_out, ext_b_rank, ext_b_rank, 128));
     Gemm2Args g{};
     g.M = static_cast<int>(T);
     g.N = static_cast<int>(N);
@@ -566,14 +570,15 @@ qlora_status pad_bf16(const T* src, int64_t rows, int64_t cols, int64_t ld, __nv
 }
 
 // U = X A^T on the tensor cores (split-K), finalized into the requested outputs.
-qlora_status compute_u_bf16(const void* X, int64_t T, int64_t d_in, const __nv_bfloat16* a_pad,
+// a_src holds a_rows rows of d_in (a_rows = RP for a padded copy, r for the caller's A).
+qlora_status compute_u_bf16(const void* X, int64_t T, int64_t d_in, const void* a_src, int a_rows,
                             int RP, int r, float s, int split, float* part, __nv_bfloat16* u_save,
                             __nv_bfloat16* u_pad, __nv_bfloat16* u_spad, int* err,
                             cudaStream_t st) {
     CUtensorMap tx, tap;
     QL_TRY(tmap_bf16(&tx, X, T, d_in, d_in, kBM));
-    QL_TRY(tmap_bf16(&tap, a_pad, RP, d_in, d_in, RP));
-    QL_TRY(skinny_gemm(false, false, RP, tx, tap, T, cdiv(d_in, kBK), split, part, err, st));
+    QL_TRY(tmap_bf16(&tap, a_src, a_rows, d_in, d_in, RP));
+    QL_TRY(skinny_gemm(false, false, RP, r, tx, tap, T, cdiv(d_in, kBK), split, part, err, st));
     k_finalize_rows<__nv_bfloat16><<<grid1d(T * RP), 256, 0, st>>>(
         part, split, T * RP, T, r, RP, s, u_save, u_pad, u_spad);
     QL_LAUNCH_CHECK();
@@ -685,11 +690,23 @@ qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T, cons
         auto* b_pad = at<__nv_bfloat16>(ws, p.b_pad);
         auto* u_spad = at<__nv_bfloat16>(ws, p.u_spad);
         auto* part = at<float>(ws, p.part);
-        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A), r, d_in, d_in, a_pad, RP, d_in, 0, d_in, stream));
-        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
-        QL_TRY(compute_u_bf16(X, T, d_in, a_pad, RP, r, s, p.split_u, part,
+        // With r a multiple of 8 every row of A, B is a whole number of 16-byte units, so the
+        // tensor maps address the caller's tensors and zero-fill the rank padding out of
+        // bounds; otherwise zero-padded copies are made.
+        const bool direct = r % 8 == 0;
+        const void* a_src = A;
+        const void* b_src = B;
+        int a_rows = r, b_ld = r;
+        if (!direct) {
+            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A), r, d_in, d_in, a_pad, RP, d_in, 0, d_in, stream));
+            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
+            a_src = a_pad;
+            b_src = b_pad;
+            a_rows = b_ld = RP;
+        }
+        QL_TRY(compute_u_bf16(X, T, d_in, a_src, a_rows, RP, r, s, p.split_u, part,
                               static_cast<__nv_bfloat16*>(U_save), nullptr, u_spad, err, stream));
-        return nf4_gemm(false, w, X, T, u_spad, b_pad, RP, r, H, at<void>(ws, p.g2), err, stream);
+        return nf4_gemm(false, w, X, T, u_spad, b_src, RP, r, b_ld, H, at<void>(ws, p.g2), err, stream);
     }
     // exact fp32 path
     float* w32 = at<float>(ws, p.w32);
@@ -723,32 +740,46 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
         auto* u_pad = at<__nv_bfloat16>(ws, p.u_pad);
         auto* g_spad = at<__nv_bfloat16>(ws, p.g_spad);
         auto* part = at<float>(ws, p.part);
-        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A), r, d_in, d_in, a_pad, RP, d_in, 0, d_in, stream));
-        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
-        if (U_saved) {
+        // pad-free operands when r is a multiple of 8 (see the forward)
+        const bool direct = r % 8 == 0;
+        const void* a_src = A;
+        const void* b_src = B;
+        const void* u_src = u_pad;
+        int a_rows = r, b_ld = r, u_ld = RP;
+        if (!direct) {
+            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A), r, d_in, d_in, a_pad, RP, d_in, 0, d_in, stream));
+            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
+            a_src = a_pad;
+            b_src = b_pad;
+            a_rows = b_ld = RP;
+        }
+        if (U_saved && direct) {
+            u_src = U_saved;
+            u_ld = r;
+        } else if (U_saved) {
             QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(U_saved), T, r, r, u_pad, T, RP, 0, RP, stream));
         } else {
-            QL_TRY(compute_u_bf16(X, T, d_in, a_pad, RP, r, s, p.split_u, part, nullptr, u_pad,
-                                  nullptr, err, stream));
+            QL_TRY(compute_u_bf16(X, T, d_in, a_src, a_rows, RP, r, s, p.split_u, part, nullptr,
+                                  u_pad, nullptr, err, stream));
         }
         // G = dH B  ->  g_spad = bf16(s G)
         {
             CUtensorMap tdh, tbp;
             QL_TRY(tmap_bf16(&tdh, dH, T, d_out, d_out, kBM));
-            QL_TRY(tmap_bf16(&tbp, b_pad, d_out, RP, RP, 64));
-            QL_TRY(skinny_gemm(false, true, RP, tdh, tbp, T, cdiv(d_out, kBK), p.split_g, part, err, stream));
+            QL_TRY(tmap_bf16(&tbp, b_src, d_out, b_ld, b_ld, 64));
+            QL_TRY(skinny_gemm(false, true, RP, r, tdh, tbp, T, cdiv(d_out, kBK), p.split_g, part, err, stream));
             k_finalize_rows<__nv_bfloat16><<<grid1d(T * RP), 256, 0, stream>>>(
                 part, p.split_g, T * RP, T, r, RP, s, nullptr, nullptr, g_spad);
             QL_LAUNCH_CHECK();
         }
         // dX = dH W^ + (sG) A
-        if (dX) QL_TRY(nf4_gemm(true, w, dH, T, g_spad, a_pad, RP, r, dX, at<void>(ws, p.g2), err, stream));
+        if (dX) QL_TRY(nf4_gemm(true, w, dH, T, g_spad, a_src, RP, r, a_rows, dX, at<void>(ws, p.g2), err, stream));
         // dA^T[d_in, RP] = X^T (sG)
         {
             CUtensorMap txm, tgm;
             QL_TRY(tmap_bf16(&txm, X, T, d_in, d_in, 64));
             QL_TRY(tmap_bf16(&tgm, g_spad, T, RP, RP, 64));
-            QL_TRY(skinny_gemm(true, true, RP, txm, tgm, d_in, cdiv(T, kBK), p.split_da, part, err, stream));
+            QL_TRY(skinny_gemm(true, true, RP, r, txm, tgm, d_in, cdiv(T, kBK), p.split_da, part, err, stream));
             k_finalize_dA<<<grid1d(static_cast<int64_t>(r) * d_in), 256, 0, stream>>>(
                 part, p.split_da, d_in * RP, d_in, r, RP, dA);
             QL_LAUNCH_CHECK();
@@ -757,8 +788,8 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
         {
             CUtensorMap thm, tum;
             QL_TRY(tmap_bf16(&thm, dH, T, d_out, d_out, 64));
-            QL_TRY(tmap_bf16(&tum, u_pad, T, RP, RP, 64));
-            QL_TRY(skinny_gemm(true, true, RP, thm, tum, d_out, cdiv(T, kBK), p.split_db, part, err, stream));
+            QL_TRY(tmap_bf16(&tum, u_src, T, u_ld, u_ld, 64));
+            QL_TRY(skinny_gemm(true, true, RP, r, thm, tum, d_out, cdiv(T, kBK), p.split_db, part, err, stream));
             k_finalize_dB<<<grid1d(d_out * r), 256, 0, stream>>>(part, p.split_db, d_out * RP,
                                                                  d_out, r, RP, s, dB);
             QL_LAUNCH_CHECK();
@@ -870,12 +901,12 @@ qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t
         CUtensorMap tx, tap;
         QL_TRY(tmap_bf16(&tx, X, T, d_in, d_in, kBM));
         QL_TRY(tmap_bf16(&tap, a_cat, RP, d_in, d_in, RP));
-        QL_TRY(skinny_gemm(false, false, RP, tx, tap, T, cdiv(d_in, kBK), p.split_u, part, err, stream));
+        QL_TRY(skinny_gemm(false, false, RP, R, tx, tap, T, cdiv(d_in, kBK), p.split_u, part, err, stream));
         k_finalize_multi<<<grid1d(T * RP), 256, 0, stream>>>(part, p.split_u, T * RP, T, RP,
                                                              n_adapters, adapter_id, seg, u_all,
                                                              nullptr, err);
         QL_LAUNCH_CHECK();
-        return nf4_gemm(false, w, X, T, u_all, b_cat, RP, R, H, at<void>(ws, p.g2), err, stream);
+        return nf4_gemm(false, w, X, T, u_all, b_cat, RP, R, RP, H, at<void>(ws, p.g2), err, stream);
     }
     // exact fp32 path
     float* w32 = at<float>(ws, p.w32);
