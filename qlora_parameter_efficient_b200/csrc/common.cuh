@@ -181,6 +181,25 @@ __device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the previous
+// kernel on the stream is finishing: it runs its prologue (barriers, tensor memory,
+// descriptor prefetch), then griddep_wait() blocks until the previous grid has completed and
+// its memory is visible.  Every global access of such a kernel comes after the wait, so
+// read-after-write and write-after-read order with the previous kernel is kept.  In a kernel
+// launched without the attribute both calls return at once.
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Let the next kernel launch, then wait for the previous one.
+__device__ __forceinline__ void griddep_enter() {
+    griddep_launch_dependents();
+    griddep_wait();
+}
+
 // ------------------------------------------------------------------ proxies and fences
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

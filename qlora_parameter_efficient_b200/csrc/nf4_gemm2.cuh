@@ -228,6 +228,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
     cluster_barrier();          // barriers of both CTAs initialised; TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    griddep_enter();
 
     auto fail = [&]() {
         set_error(args.err, kErrTimeout);

@@ -77,12 +77,6 @@ struct GvCfg {
     static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
-__device__ __forceinline__ void griddep_wait() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void griddep_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 // 4-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros without reading.
 __device__ __forceinline__ void cp_async_4(void* dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)),

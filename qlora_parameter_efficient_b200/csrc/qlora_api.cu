@@ -50,6 +50,24 @@ inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed);
         if (cudaPeekAtLastError() != cudaSuccess) return QLORA_ERR_CUDA; \
     } while (0)
 
+// Launch a kernel that begins with griddep_enter() with programmatic stream serialization, so
+// that its launch and prologue overlap the end of the previous kernel on the stream.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 qlora_status err_word(int** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
@@ -303,7 +321,8 @@ qlora_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUten
     }
     const bool ev = timed && g_ev_start && g_ev_stop;
     if (ev) cudaEventRecord(g_ev_start, st);
-    kern<<<grid, kGemmThreads, smem, st>>>(a, b, ax, bx, args);
+    if (launch_pdl(kern, grid, dim3(kGemmThreads), smem, st, a, b, ax, bx, args) != cudaSuccess)
+        return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     if (ev) cudaEventRecord(g_ev_stop, st);
     return QLORA_OK;
@@ -403,7 +422,9 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
         return QLORA_ERR_CUDA;
     const bool ev = g_ev_start && g_ev_stop;
     if (ev) cudaEventRecord(g_ev_start, st);
-    kern<<<2 * pairs, kG2Threads, G2Smem::kTotal, st>>>(ta, tc, tax, tbx, g);
+    if (launch_pdl(kern, dim3(2 * pairs), dim3(kG2Threads), G2Smem::kTotal, st, ta, tc, tax, tbx, g) !=
+        cudaSuccess)
+        return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     if (ev) cudaEventRecord(g_ev_stop, st);
     return QLORA_OK;
@@ -562,9 +583,9 @@ template <typename T>
 qlora_status pad_bf16(const T* src, int64_t rows, int64_t cols, int64_t ld, __nv_bfloat16* dst,
                       int64_t rows_pad, int64_t ld_dst, int64_t col_off, int64_t col_span,
                       cudaStream_t st) {
-    k_pad_copy_bf16<T><<<grid1d(rows_pad * col_span), 256, 0, st>>>(src, rows, cols, ld, dst,
-                                                                  rows_pad, ld_dst, col_off,
-                                                                  col_span);
+    if (launch_pdl(k_pad_copy_bf16<T>, grid1d(rows_pad * col_span), dim3(256), 0, st, src, rows,
+                   cols, ld, dst, rows_pad, ld_dst, col_off, col_span) != cudaSuccess)
+        return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     return QLORA_OK;
 }
@@ -579,8 +600,9 @@ qlora_status compute_u_bf16(const void* X, int64_t T, int64_t d_in, const void* 
     QL_TRY(tmap_bf16(&tx, X, T, d_in, d_in, kBM));
     QL_TRY(tmap_bf16(&tap, a_src, a_rows, d_in, d_in, RP));
     QL_TRY(skinny_gemm(false, false, RP, r, tx, tap, T, cdiv(d_in, kBK), split, part, err, st));
-    k_finalize_rows<__nv_bfloat16><<<grid1d(T * RP), 256, 0, st>>>(
-        part, split, T * RP, T, r, RP, s, u_save, u_pad, u_spad);
+    if (launch_pdl(k_finalize_rows<__nv_bfloat16>, grid1d(T * RP), dim3(256), 0, st, part, split,
+                   T * RP, T, r, RP, s, u_save, u_pad, u_spad) != cudaSuccess)
+        return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     return QLORA_OK;
 }
@@ -768,8 +790,10 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
             QL_TRY(tmap_bf16(&tdh, dH, T, d_out, d_out, kBM));
             QL_TRY(tmap_bf16(&tbp, b_src, d_out, b_ld, b_ld, 64));
             QL_TRY(skinny_gemm(false, true, RP, r, tdh, tbp, T, cdiv(d_out, kBK), p.split_g, part, err, stream));
-            k_finalize_rows<__nv_bfloat16><<<grid1d(T * RP), 256, 0, stream>>>(
-                part, p.split_g, T * RP, T, r, RP, s, nullptr, nullptr, g_spad);
+            if (launch_pdl(k_finalize_rows<__nv_bfloat16>, grid1d(T * RP), dim3(256), 0, stream,
+                           part, p.split_g, T * RP, T, r, RP, s, nullptr, nullptr, g_spad) !=
+                cudaSuccess)
+                return QLORA_ERR_CUDA;
             QL_LAUNCH_CHECK();
         }
         // dX = dH W^ + (sG) A
@@ -780,8 +804,9 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
             QL_TRY(tmap_bf16(&txm, X, T, d_in, d_in, 64));
             QL_TRY(tmap_bf16(&tgm, g_spad, T, RP, RP, 64));
             QL_TRY(skinny_gemm(true, true, RP, r, txm, tgm, d_in, cdiv(T, kBK), p.split_da, part, err, stream));
-            k_finalize_dA<<<grid1d(static_cast<int64_t>(r) * d_in), 256, 0, stream>>>(
-                part, p.split_da, d_in * RP, d_in, r, RP, dA);
+            if (launch_pdl(k_finalize_dA, grid1d(static_cast<int64_t>(r) * d_in), dim3(256), 0,
+                           stream, part, p.split_da, d_in * RP, d_in, r, RP, dA) != cudaSuccess)
+                return QLORA_ERR_CUDA;
             QL_LAUNCH_CHECK();
         }
         // dB[d_out, RP] = s dH^T U
@@ -790,8 +815,9 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
             QL_TRY(tmap_bf16(&thm, dH, T, d_out, d_out, 64));
             QL_TRY(tmap_bf16(&tum, u_src, T, u_ld, u_ld, 64));
             QL_TRY(skinny_gemm(true, true, RP, r, thm, tum, d_out, cdiv(T, kBK), p.split_db, part, err, stream));
-            k_finalize_dB<<<grid1d(d_out * r), 256, 0, stream>>>(part, p.split_db, d_out * RP,
-                                                                 d_out, r, RP, s, dB);
+            if (launch_pdl(k_finalize_dB, grid1d(d_out * r), dim3(256), 0, stream, part, p.split_db,
+                           d_out * RP, d_out, r, RP, s, dB) != cudaSuccess)
+                return QLORA_ERR_CUDA;
             QL_LAUNCH_CHECK();
         }
         return QLORA_OK;
@@ -902,9 +928,10 @@ qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t
         QL_TRY(tmap_bf16(&tx, X, T, d_in, d_in, kBM));
         QL_TRY(tmap_bf16(&tap, a_cat, RP, d_in, d_in, RP));
         QL_TRY(skinny_gemm(false, false, RP, R, tx, tap, T, cdiv(d_in, kBK), p.split_u, part, err, stream));
-        k_finalize_multi<<<grid1d(T * RP), 256, 0, stream>>>(part, p.split_u, T * RP, T, RP,
-                                                             n_adapters, adapter_id, seg, u_all,
-                                                             nullptr, err);
+        if (launch_pdl(k_finalize_multi, grid1d(T * RP), dim3(256), 0, stream, part, p.split_u,
+                       T * RP, T, RP, n_adapters, adapter_id, seg, u_all,
+                       static_cast<float*>(nullptr), err) != cudaSuccess)
+            return QLORA_ERR_CUDA;
         QL_LAUNCH_CHECK();
         return nf4_gemm(false, w, X, T, u_all, b_cat, RP, R, RP, H, at<void>(ws, p.g2), err, stream);
     }

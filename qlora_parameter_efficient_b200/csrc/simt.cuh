@@ -77,6 +77,7 @@ template <typename T>
 __global__ void k_pad_copy_bf16(const T* __restrict__ src, int64_t rows, int64_t cols, int64_t ld,
                                 __nv_bfloat16* __restrict__ dst, int64_t rows_pad, int64_t ld_dst,
                                 int64_t col_off, int64_t col_span) {
+    griddep_enter();
     const int64_t n = rows_pad * col_span;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -111,6 +112,7 @@ __global__ void k_finalize_rows(const float* __restrict__ P, int split, int64_t 
                                 int64_t T, int r, int RP, float scale, To* __restrict__ out_raw,
                                 __nv_bfloat16* __restrict__ out_pad,
                                 __nv_bfloat16* __restrict__ out_spad) {
+    griddep_enter();
     const int64_t n = T * RP;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -139,6 +141,7 @@ __global__ void k_finalize_multi(const float* __restrict__ P, int split, int64_t
                                  int64_t T, int RP, int n_adapters, const int32_t* __restrict__ ids,
                                  SegTable seg, __nv_bfloat16* __restrict__ out_bf,
                                  float* __restrict__ out_f32, int* err) {
+    griddep_enter();
     const int64_t n = T * RP;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -161,6 +164,7 @@ __global__ void k_finalize_multi(const float* __restrict__ P, int split, int64_t
 // dA[j, n] = sum_z P[z][n][j]  (the dA GEMM computes dA^T tiles), j < r.
 __global__ void k_finalize_dA(const float* __restrict__ P, int split, int64_t split_stride,
                               int64_t d_in, int r, int RP, float* __restrict__ dA) {
+    griddep_enter();
     const int64_t n = static_cast<int64_t>(r) * d_in;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -174,6 +178,7 @@ __global__ void k_finalize_dA(const float* __restrict__ P, int split, int64_t sp
 // dB[i, j] = scale * sum_z P[z][i][j], j < r.
 __global__ void k_finalize_dB(const float* __restrict__ P, int split, int64_t split_stride,
                               int64_t d_out, int r, int RP, float scale, float* __restrict__ dB) {
+    griddep_enter();
     const int64_t n = d_out * r;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {

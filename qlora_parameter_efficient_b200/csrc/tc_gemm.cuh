@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_acc = *tmem_slot;
+    griddep_enter();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
