@@ -324,8 +324,9 @@ def run_gpu(args):
     achieved = gemm_flops / (g_avg / 1e3) / 1e12 if g_avg else None
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": (achieved / peak) if achieved else None, "traffic": None,
-                "kernel": "k_tc_gemm<NF4 fwd> (fused decode + adapter K-extension)",
+                "frac": (achieved / peak) if achieved else None,
+                "traffic": GEMM_FWD_DRAM_BYTES, "traffic_unit": "bytes per launch",
+                "kernel": "k_nf4_gemm2<0> (fused NF4 decode + adapter K-extension, 2-SM tcgen05)",
                 "peak_source": f"{peak_src} bf16_tflops_sustained",
                 "kernel_ms": g_avg}
     step_flops = flops_fwd(T, d, k, r) + flops_bwd(T, d, k, r)
@@ -524,6 +525,13 @@ def extra_rows(q, torch, S, dev, peaks, args):
     out["merge_4096x4096_bf16"] = {"us": med, "GB/s": byts / (med * 1e-6) / 1e9,
                                    "hbm_frac": byts / (med * 1e-6) / 1e9 / hbm}
     return out
+
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one k_nf4_gemm2<0> launch at this workload,
+# from the ncu capture summarised in profiles/nf4_fused_gemm_q_proj_4096x4096_T4096.md
+# (43.73 MB read + 15.49 MB written; H is still partly in L2 when the kernel ends).  Set to
+# None whenever the kernel changes until it is captured again.
+GEMM_FWD_DRAM_BYTES = 43731968 + 15493376
 
 
 def main():
