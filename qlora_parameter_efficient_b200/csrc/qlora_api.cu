@@ -14,6 +14,7 @@
 #include "simt.cuh"
 #include "tc_gemm.cuh"
 #include "nf4_gemm2.cuh"
+#include "merge.cuh"
 #include "qgemv.cuh"
 
 using namespace qlora;
@@ -865,10 +866,22 @@ qlora_status lora_merge(const qlora_nf4* w, const void* A, const void* B, int32_
         return QLORA_OK;
     };
     using bf = __nv_bfloat16;
+    // bf16 adapters: B A on the tensor cores (exact products, fp32 accumulation)
+    auto run_tc = [&](auto kern, auto o) -> qlora_status {
+        const int tsmem = MergeSmem::bytes(static_cast<int>(rp), static_cast<int>(sizeof(*o)));
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tsmem) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        dim3 tgrid(static_cast<unsigned>(w->d_in / 64), static_cast<unsigned>(cdiv(w->d_out, 128)));
+        kern<<<tgrid, kMergeThreads, tsmem, stream>>>(w->codes, w->absmax_q, w->c2, w->d_out, w->d_in,
+                                                       static_cast<const bf*>(A), static_cast<const bf*>(B),
+                                                       r, s, o);
+        QL_LAUNCH_CHECK();
+        return QLORA_OK;
+    };
     if (adapter_dtype == QLORA_BF16 && out_dtype == QLORA_BF16)
-        return run(k_merge<bf, bf>, static_cast<const bf*>(A), static_cast<const bf*>(B), static_cast<bf*>(W_final));
+        return run_tc(k_merge_tc<bf>, static_cast<bf*>(W_final));
     if (adapter_dtype == QLORA_BF16 && out_dtype == QLORA_F32)
-        return run(k_merge<bf, float>, static_cast<const bf*>(A), static_cast<const bf*>(B), static_cast<float*>(W_final));
+        return run_tc(k_merge_tc<float>, static_cast<float*>(W_final));
     if (adapter_dtype == QLORA_F32 && out_dtype == QLORA_BF16)
         return run(k_merge<float, bf>, static_cast<const float*>(A), static_cast<const float*>(B), static_cast<bf*>(W_final));
     if (adapter_dtype == QLORA_F32 && out_dtype == QLORA_F32)

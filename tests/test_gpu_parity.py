@@ -230,6 +230,21 @@ def test_merge(q, out):
     assert rel_fro(host(H), Hm) <= TOL["bf16"]
 
 
+# Tensor-core merge (bf16 adapters): ragged rows, d_in not a multiple of the 128-column tile,
+# ranks that are not multiples of 16 (zero-padded K), the largest rank, and the full q_proj size.
+@pytest.mark.parametrize("d_out,d_in,r", [(200, 192, 5), (136, 320, 33), (72, 64, 1),
+                                          (256, 1088, 128), (4096, 4096, 16)])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_merge_shapes(q, d_out, d_in, r, out):
+    import torch
+    case = S.make_layer(d_out, d_in, r, 2.0 * r, 1, dtype="bf16", seed=d_out + r, with_grad=False)
+    w, oc = quantize_both(q, case.W0)
+    Wf = q.lora_merge(w, dev(case.A, "bf16"), dev(case.B, "bf16"), 2.0 * r,
+                      torch.bfloat16 if out == "bf16" else torch.float32)
+    ref = O.lora_merge(oracle_weight(oc, d_out, d_in, out), case.A, case.B, 2.0 * r, r)
+    assert rel_fro(host(Wf), ref) <= TOL[out]
+
+
 def test_merge_f32_adapters(q):
     import torch
     case = S.make_layer(256, 256, 8, 16.0, 16, dtype="f32", seed=2)
