@@ -293,25 +293,57 @@ def run_gpu(args):
                                                       dA=dA, dB=dB, ws=ws), args.steps, W)
 
     # ------------------------------------------------------------------ end to end
-    # Each step: pinned host X, dH -> device, fwd + bwd through the C ABI, dA, dB -> host.
+    # Each step: pinned host X, dH -> device, fwd + bwd through the C ABI, dA, dB -> host.  The
+    # next step's inputs are copied on a second stream into the other of two device buffers
+    # while this step computes (a data loader's prefetch); every copy of every step lies inside
+    # the timed region, and a buffer is refilled only after the step that read it has finished.
     hX = [sets[i]["X"].cpu().pin_memory() for i in range(2)]
     hdH = [sets[i]["dH"].cpu().pin_memory() for i in range(2)]
     hdA = torch.empty_like(dA, device="cpu").pin_memory()
     hdB = torch.empty_like(dB, device="cpu").pin_memory()
-    Xd = torch.empty_like(sets[0]["X"])
-    dHd = torch.empty_like(sets[0]["dH"])
+    Xd = [torch.empty_like(sets[0]["X"]) for _ in range(2)]
+    dHd = [torch.empty_like(sets[0]["dH"]) for _ in range(2)]
+    copy_stream = torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_free = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step(i):
-        s = sets[i % NSETS]
-        Xd.copy_(hX[i % 2], non_blocking=True)
-        dHd.copy_(hdH[i % 2], non_blocking=True)
-        q.qlora_linear_fwd(s["w"], Xd, s["A"], s["B"], alpha, H=H, U_save=U, ws=ws)
-        q.qlora_linear_bwd(s["w"], Xd, dHd, s["A"], s["B"], alpha, U_saved=U, dX=dX, dA=dA, dB=dB, ws=ws)
-        dp.allreduce_adapter_grads(dA, dB)
-        hdA.copy_(dA, non_blocking=True)
-        hdB.copy_(dB, non_blocking=True)
+    def copy_in(i):
+        bi = i % 2
+        with torch.cuda.stream(copy_stream):
+            if i >= 2:
+                copy_stream.wait_event(ev_free[bi])
+            Xd[bi].copy_(hX[i % 2], non_blocking=True)
+            dHd[bi].copy_(hdH[i % 2], non_blocking=True)
+            ev_in[bi].record(copy_stream)
 
-    e2e_ms, _, _ = timed(e2e_step, args.steps, W)
+    def e2e_run(K):
+        copy_stream.wait_stream(stream)
+        copy_in(0)
+        for i in range(K):
+            bi = i % 2
+            if i + 1 < K:
+                copy_in(i + 1)
+            stream.wait_event(ev_in[bi])
+            s = sets[i % NSETS]
+            q.qlora_linear_fwd(s["w"], Xd[bi], s["A"], s["B"], alpha, H=H, U_save=U, ws=ws)
+            q.qlora_linear_bwd(s["w"], Xd[bi], dHd[bi], s["A"], s["B"], alpha, U_saved=U, dX=dX,
+                               dA=dA, dB=dB, ws=ws)
+            ev_free[bi].record(stream)
+            dp.allreduce_adapter_grads(dA, dB)
+            hdA.copy_(dA, non_blocking=True)
+            hdB.copy_(dB, non_blocking=True)
+
+    e2e_run(W)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ee0.record(stream)
+    e2e_run(args.steps)
+    ee1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dp.max_over_ranks(ee0.elapsed_time(ee1), device=dev)
 
     extra = {}
     if args.extra and rank == 0:
@@ -341,7 +373,7 @@ def run_gpu(args):
         "fwd_ms": fwd_ms / args.steps, "bwd_ms": bwd_ms / args.steps,
         "roofline": roofline,
         "e2e": {"value": toks / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(Xd.numel() * 2 + dHd.numel() * 2),
+                "h2d_bytes_per_step": int(Xd[0].numel() * 2 + dHd[0].numel() * 2),
                 "d2h_bytes_per_step": int(dA.numel() * 4 + dB.numel() * 4)},
         "gpu_launches": int(launches),
         "clocks": clocks,
