@@ -926,17 +926,21 @@ qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t
         auto* b_cat = at<__nv_bfloat16>(ws, p.b_pad);
         auto* u_all = at<__nv_bfloat16>(ws, p.u_spad);
         auto* part = at<float>(ws, p.part);
-        if (cudaMemsetAsync(a_cat, 0, static_cast<size_t>(RP) * d_in * 2, stream) != cudaSuccess ||
-            cudaMemsetAsync(b_cat, 0, static_cast<size_t>(d_out) * RP * 2, stream) != cudaSuccess)
-            return QLORA_ERR_CUDA;
-        int off = 0;
-        for (int i = 0; i < n_adapters; ++i) {
-            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A[i]), r[i], d_in, d_in,
-                            a_cat + static_cast<int64_t>(off) * d_in, r[i], d_in, 0, d_in, stream));
-            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B[i]), d_out, r[i], r[i], b_cat,
-                            d_out, RP, off, r[i], stream));
-            off += r[i];
+        // all adapters concatenated (and zero-padded to RP) in one launch
+        CatTable cat;
+        for (int j = 0; j < 128; ++j) cat.seg_of[j] = static_cast<int8_t>(seg.seg_of[j]);
+        for (int i = 0, off = 0; i < 32; ++i) {
+            const bool used = i < n_adapters;
+            cat.A[i] = used ? static_cast<const __nv_bfloat16*>(A[i]) : nullptr;
+            cat.B[i] = used ? static_cast<const __nv_bfloat16*>(B[i]) : nullptr;
+            cat.r[i] = used ? r[i] : 0;
+            cat.off[i] = off;
+            if (used) off += r[i];
         }
+        if (launch_pdl(k_concat_adapters, grid1d(static_cast<int64_t>(RP) * (d_in / 8) + d_out * RP),
+                       dim3(256), 0, stream, cat, d_out, d_in, RP, a_cat, b_cat) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        QL_LAUNCH_CHECK();
         CUtensorMap tx, tap;
         QL_TRY(tmap_bf16(&tx, X, T, d_in, d_in, kBM));
         QL_TRY(tmap_bf16(&tap, a_cat, RP, d_in, d_in, RP));

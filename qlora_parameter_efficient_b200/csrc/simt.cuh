@@ -190,6 +190,43 @@ __global__ void k_finalize_dB(const float* __restrict__ P, int split, int64_t sp
     }
 }
 
+// Concatenated adapters of the multi-adapter forward, built in one pass:
+//   a_cat [RP, d_in]:  row j = row (j - off_i) of A_i for the adapter i holding column j, 0 for j >= R
+//   b_cat [d_out, RP]: column j = column (j - off_i) of B_i, 0 for j >= R
+struct CatTable {
+    const __nv_bfloat16* A[32];
+    const __nv_bfloat16* B[32];
+    int32_t r[32];
+    int32_t off[32];
+    int8_t seg_of[128];      // adapter of concatenated column j, -1 beyond R
+};
+
+__global__ void k_concat_adapters(CatTable tab, int64_t d_out, int64_t d_in, int RP,
+                                  __nv_bfloat16* __restrict__ a_cat,
+                                  __nv_bfloat16* __restrict__ b_cat) {
+    griddep_enter();
+    const int64_t na = static_cast<int64_t>(RP) * (d_in / 8);      // 16-byte vectors of a_cat
+    const int64_t nb = d_out * RP;                                  // elements of b_cat
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < na + nb;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        if (i < na) {
+            const int j = static_cast<int>(i / (d_in / 8));
+            const int64_t c = (i % (d_in / 8)) * 8;
+            const int a = tab.seg_of[j];
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (a >= 0)
+                v = *reinterpret_cast<const uint4*>(tab.A[a] + static_cast<int64_t>(j - tab.off[a]) * d_in + c);
+            *reinterpret_cast<uint4*>(a_cat + static_cast<int64_t>(j) * d_in + c) = v;
+        } else {
+            const int64_t e = i - na;
+            const int64_t n = e / RP;
+            const int j = static_cast<int>(e % RP);
+            const int a = tab.seg_of[j];
+            b_cat[e] = a >= 0 ? tab.B[a][n * tab.r[a] + (j - tab.off[a])] : __float2bfloat16_rn(0.f);
+        }
+    }
+}
+
 // Zero columns of U_all[t, :] that do not belong to token t's adapter and scale the rest
 // (fp32 batched path).
 __global__ void k_mask_multi_f32(float* __restrict__ U, int64_t T, int R, int n_adapters,
