@@ -543,6 +543,31 @@ def extra_rows(q, torch, S, dev, peaks, args):
                                           "tc_frac": fl / (med * 1e-6) / 1e12 / tc}
         del wl, X, ids, As, Bs, H, ws
 
+    # ---- many-adapter (segmented) forward: 4096^2 base, 1024 adapters of rank 16, T = 4096,
+    # ids uniform (about 4 tokens per adapter); adapters drawn on the device (268 MB > L2)
+    n_ad, r_ad, T_ad = 1024, 16, 4096
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    mc = S.make_multi_adapter(4096, 4096, 1, [1], seed=7)          # only W0 is used from it
+    wl = [q.nf4_quantize(torch.from_numpy(mc.W0).to(dev)) for _ in range(4)]
+    X = torch.randn((T_ad, 4096), generator=gen, device=dev).to(bf)
+    ids = torch.randint(0, n_ad, (T_ad,), generator=gen, device=dev, dtype=torch.int32)
+    As = [(torch.randn((r_ad, 4096), generator=gen, device=dev) / r_ad ** 0.5).to(bf) for _ in range(n_ad)]
+    Bs = [(torch.randn((4096, r_ad), generator=gen, device=dev) * 0.1).to(bf) for _ in range(n_ad)]
+    tab = q.AdapterTable(As, Bs, [2.0 * r_ad] * n_ad)
+    H = torch.empty((T_ad, 4096), dtype=bf, device=dev)
+    ws = torch.empty(q.workspace_bytes(q.OP_FWD_MULTI, q.BF16, T_ad, 4096, 4096, r_ad),
+                     dtype=torch.uint8, device=dev)
+    calls = [(lambda w=w: q.qlora_linear_fwd_multi(w, X, ids, tab, H=H, ws=ws)) for w in wl]
+    med, _ = _graph_time(torch, calls, reps=10)
+    fl = 2 * T_ad * 4096 * 4096 + 2 * T_ad * r_ad * (4096 + 4096)
+    byts = w_bytes(4096, 4096) + 2 * T_ad * 4096 * 3 + n_ad * r_ad * (4096 + 4096) * 2
+    t_roof = max(fl / (tc * 1e12), byts / (hbm * 1e9))
+    out["multi_1024x_r16_T4096"] = {"fwd_us": med, "tokens/s": T_ad / (med * 1e-6),
+                                    "tflops": fl / (med * 1e-6) / 1e12, "t_roof_us": t_roof * 1e6,
+                                    "roof_frac": t_roof / (med * 1e-6), "adapter_MB": n_ad * r_ad * 8192 * 2 / 1e6}
+    del wl, X, ids, As, Bs, tab, H, ws
+
     # ---- merge W_final = W^ + s B A on the 4096^2 shape, bf16 out
     c2_ = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
     d, k, r, alpha = c2_["d_out"], c2_["d_in"], c2_["r"], c2_["alpha"]

@@ -55,7 +55,8 @@ typedef enum {
 typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 
 typedef enum {
-    QLORA_OP_FWD = 0, QLORA_OP_BWD = 1, QLORA_OP_FWD_BATCHED = 2, QLORA_OP_MERGE = 3
+    QLORA_OP_FWD = 0, QLORA_OP_BWD = 1, QLORA_OP_FWD_BATCHED = 2, QLORA_OP_MERGE = 3,
+    QLORA_OP_FWD_MULTI = 4
 } qlora_op;
 
 /* Stored NF4 weight.  Block size 64 and group size 256 are fixed.
@@ -101,7 +102,8 @@ qlora_status nf4_dequantize(const qlora_nf4* w, void* W_out, qlora_dtype out_dty
                             cudaStream_t stream);
 
 /* Scratch bytes needed by an operation (host-only).  op is a qlora_op, dtype the call's dtype;
- * r_total is r for the single-adapter calls and the sum of ranks for QLORA_OP_FWD_BATCHED.
+ * r_total is r for the single-adapter calls, the sum of ranks for QLORA_OP_FWD_BATCHED and
+ * the largest rank for QLORA_OP_FWD_MULTI.
  * Returns 0 for an unsupported combination.                                                  */
 size_t qlora_workspace_bytes(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in,
                              int32_t r_total);
@@ -149,6 +151,32 @@ qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t
                                       const void* const* A, const void* const* B,
                                       const int32_t* r, const float* alpha, qlora_dtype dtype,
                                       void* H, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Multi-adapter forward for many adapters (bf16), the same result as qlora_linear_fwd_batched
+ * without its limits on the number and total rank of the adapters:
+ *   H[t] = X[t] W^T + s_i (X[t] A_i^T) B_i^T,  i = adapter_id[t].
+ * [CH] "Serving many adapters at once: the multi-tenant problem" (the shared x W once per
+ * batch, each request's correction by grouped kernels over adapters of different ranks);
+ * [UH] "6.2 Multi-Adapter Serving at Scale (S-LoRA & Punica)" (thousands of adapters over one
+ * base).  The base term is the fused NF4 GEMM without adapter steps, rounded to bf16 into H;
+ * the tokens are sorted by adapter on the device and each adapter's segment gets
+ * U = bf16(s_i X A_i^T) and H = bf16(H + U B_i^T), fp32 accumulation.
+ *   adapter_id  device int32 [T]
+ *   A_ptrs      DEVICE array of n_adapters device pointers, A_i bf16 [r_i, d_in], 16-byte
+ *               aligned (its rows then are too: d_in % 64 == 0 is already required)
+ *   B_ptrs      DEVICE array of n_adapters device pointers, B_i bf16 [d_out, r_i]
+ *   ranks       DEVICE int32 [n_adapters], 1 <= r_i <= r_max
+ *   scales      DEVICE float [n_adapters], s_i (alpha_i / r_i)
+ *   r_max       host: the largest rank, 1..128; ws >= qlora_workspace_bytes(QLORA_OP_FWD_MULTI,
+ *               QLORA_BF16, T, d_out, d_in, r_max)
+ * 1 <= n_adapters <= 65536.  An id outside [0, n_adapters), or an adapter whose rank is
+ * outside [1, r_max] or whose A_i is not 16-byte aligned, contributes no adapter term and sets
+ * QLORA_ERR_DEVICE in the device error word.                                                 */
+qlora_status qlora_linear_fwd_multi(const qlora_nf4* w, const void* X, int64_t T,
+                                    const int32_t* adapter_id, int32_t n_adapters,
+                                    const void* const* A_ptrs, const void* const* B_ptrs,
+                                    const int32_t* ranks, const float* scales, int32_t r_max,
+                                    void* H, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Size of the device scratch array behind qlora_linear_fwd_noalloc (bytes per GPU). */
 #define QLORA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

@@ -22,12 +22,13 @@ QLORA_OK = 0
 STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",
           3: "QLORA_ERR_CUDA", 4: "QLORA_ERR_TIMEOUT", 5: "QLORA_ERR_DEVICE"}
 F32, BF16 = 0, 1
-OP_FWD, OP_BWD, OP_FWD_BATCHED, OP_MERGE = 0, 1, 2, 3
+OP_FWD, OP_BWD, OP_FWD_BATCHED, OP_MERGE, OP_FWD_MULTI = 0, 1, 2, 3, 4
 
 # Every symbol include/qlora.h declares.
 EXPORTS = ["qlora_nf4_sizes", "qlora_nf4_levels", "nf4_quantize", "nf4_dequantize",
            "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "lora_merge",
-           "qlora_linear_fwd_batched", "qlora_linear_fwd_noalloc", "qlora_get_device_error",
+           "qlora_linear_fwd_batched", "qlora_linear_fwd_multi", "qlora_linear_fwd_noalloc",
+           "qlora_get_device_error",
            "qlora_selftest_wait_timeout", "qlora_set_gemm_events", "qlora_launch_count",
            "qlora_status_string"]
 
@@ -69,6 +70,8 @@ def load() -> ctypes.CDLL:
         "qlora_linear_fwd_batched": ([pnf4, vp, i64, vp, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                       ctypes.POINTER(i32), ctypes.POINTER(f32), ctypes.c_int, vp, vp, sz, vp],
                                      ctypes.c_int),
+        "qlora_linear_fwd_multi": ([pnf4, vp, i64, vp, i32, vp, vp, vp, vp, i32, vp, vp, sz, vp],
+                                   ctypes.c_int),
         "qlora_linear_fwd_noalloc": ([pnf4, vp, i64, vp, vp, i32, f32, ctypes.c_int, vp, vp, vp], ctypes.c_int),
         "qlora_get_device_error": ([vp], ctypes.c_int),
         "qlora_selftest_wait_timeout": ([ctypes.c_uint64, vp], ctypes.c_int),
@@ -256,6 +259,41 @@ def qlora_linear_fwd_batched(w: NF4Weight, X, adapter_id, As, Bs, alphas, H=None
     _check("qlora_linear_fwd_batched", load().qlora_linear_fwd_batched(
         ctypes.byref(c), _ptr(X), T, _ptr(adapter_id), n, Ap, Bp, rp, ap, dt, _ptr(H), _ptr(ws),
         ws.numel(), _stream(stream)))
+    return H
+
+
+class AdapterTable:
+    """Device-resident adapter table for qlora_linear_fwd_multi: pointer arrays, ranks and
+    scales built once from lists of bf16 tensors A_i [r_i, d_in], B_i [d_out, r_i]."""
+
+    def __init__(self, As, Bs, alphas):
+        torch = _torch()
+        _contig(*As, *Bs)
+        dev = As[0].device
+        self.As, self.Bs = list(As), list(Bs)        # keep the tensors alive
+        self.ranks_host = [int(a.shape[0]) for a in As]
+        self.n = len(As)
+        self.r_max = max(self.ranks_host)
+        self.A_ptrs = torch.tensor([a.data_ptr() for a in As], dtype=torch.int64, device=dev)
+        self.B_ptrs = torch.tensor([b.data_ptr() for b in Bs], dtype=torch.int64, device=dev)
+        self.ranks = torch.tensor(self.ranks_host, dtype=torch.int32, device=dev)
+        self.scales = torch.tensor([float(al) / r for al, r in zip(alphas, self.ranks_host)],
+                                   dtype=torch.float32, device=dev)
+
+
+def qlora_linear_fwd_multi(w: NF4Weight, X, adapter_id, table: AdapterTable, H=None, ws=None,
+                           stream=None):
+    torch = _torch()
+    _contig(X, adapter_id, H)
+    T = X.shape[0]
+    if H is None:
+        H = torch.empty((T, w.d_out), dtype=X.dtype, device=X.device)
+    ws = _ws(OP_FWD_MULTI, BF16, T, w.d_out, w.d_in, table.r_max, X.device, ws)
+    c = w._c()
+    _check("qlora_linear_fwd_multi", load().qlora_linear_fwd_multi(
+        ctypes.byref(c), _ptr(X), T, _ptr(adapter_id), table.n, _ptr(table.A_ptrs),
+        _ptr(table.B_ptrs), _ptr(table.ranks), _ptr(table.scales), table.r_max, _ptr(H),
+        _ptr(ws), ws.numel(), _stream(stream)))
     return H
 
 

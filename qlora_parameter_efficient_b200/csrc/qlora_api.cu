@@ -15,6 +15,7 @@
 #include "tc_gemm.cuh"
 #include "nf4_gemm2.cuh"
 #include "merge.cuh"
+#include "segmented.cuh"
 #include "qgemv.cuh"
 
 using namespace qlora;
@@ -213,6 +214,10 @@ struct Plan {
     size_t a_pad = 0, b_pad = 0, u_spad = 0, u_pad = 0, g_spad = 0, part = 0;
     size_t w32 = 0, uf = 0, gf = 0;
     size_t g2 = 0;         // fused-GEMM split-tail partials and tickets
+    // segmented multi-adapter forward
+    size_t seg_cnt = 0, seg_start = 0, seg_cursor = 0, seg_ntiles = 0, seg_tiles = 0, seg_perm = 0,
+           seg_u = 0;
+    int seg_ldu = 0, seg_max_tiles = 0;
     size_t total = 0;
 };
 
@@ -225,6 +230,21 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
         return o;
     };
     if (op == QLORA_OP_MERGE) return p;
+    if (op == QLORA_OP_FWD_MULTI) {
+        // base GEMM split tail, then the segmented adapter term (r = the largest rank)
+        p.g2 = take(g2_schedule(T, d_out, d_in).bytes());
+        p.seg_ldu = (r + 15) & ~15;
+        p.seg_cnt = take(static_cast<size_t>(kSegMaxAdapters) * 4);
+        p.seg_start = take(static_cast<size_t>(kSegMaxAdapters) * 4);
+        p.seg_cursor = take(static_cast<size_t>(kSegMaxAdapters) * 4);
+        p.seg_ntiles = take(4);
+        p.seg_max_tiles = static_cast<int>(cdiv(T, kSegTile) + std::min<int64_t>(T, kSegMaxAdapters));
+        p.seg_tiles = take(static_cast<size_t>(p.seg_max_tiles) * 16);
+        p.seg_perm = take(static_cast<size_t>(T) * 4);
+        p.seg_u = take(static_cast<size_t>(T) * p.seg_ldu * 2);
+        p.total = off;
+        return p;
+    }
     if (op == QLORA_OP_FWD && dtype == QLORA_BF16 && make_small_plan(T, d_out, d_in).ok) {
         p.small = true;
         p.s_us = take(static_cast<size_t>(T) * r * 4);
@@ -381,15 +401,20 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
     QL_TRY(tmap_bf16(&ta, act, T, K, K, 128));
     if (dx) QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 64, 64));
     else QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 32, 128));
-    QL_TRY(tmap_bf16(&tax, ext_a, T, RP, RP, 128));
-    if (dx) QL_TRY(tmap_bf16(&tbx, ext_b, ext_b_rank, d_in, d_in, 64));
-    else QL_TRY(tmap_bf16(&tbx, ext_b, d_out, ext_b_rank, ext_b_rank, 128));
+    if (RP > 0) {
+        QL_TRY(tmap_bf16(&tax, ext_a, T, RP, RP, 128));
+        if (dx) QL_TRY(tmap_bf16(&tbx, ext_b, ext_b_rank, d_in, d_in, 64));
+        else QL_TRY(tmap_bf16(&tbx, ext_b, d_out, ext_b_rank, ext_b_rank, 128));
+    } else {                 // no adapter steps: the maps are never read
+        tax = ta;
+        tbx = ta;
+    }
     Gemm2Args g{};
     g.M = static_cast<int>(T);
     g.N = static_cast<int>(N);
     g.k_steps = static_cast<int>(cdiv(K, 64));
     g.ext_steps = RP / 64;
-    g.ext_k16_last = static_cast<int>(std::min<int64_t>(4, cdiv(r_used - 64 * (g.ext_steps - 1), 16)));
+    g.ext_k16_last = RP > 0 ? static_cast<int>(std::min<int64_t>(4, cdiv(r_used - 64 * (g.ext_steps - 1), 16))) : 4;
     g.m_tiles = static_cast<int>(cdiv(T, 256));
     g.n_tiles = static_cast<int>(cdiv(N, 256));
     g.absmax_q = w->absmax_q;
@@ -648,7 +673,8 @@ qlora_status qlora_nf4_levels(float* out) {
 
 size_t qlora_workspace_bytes(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in,
                              int32_t r_total) {
-    if (op < QLORA_OP_FWD || op > QLORA_OP_MERGE) return 0;
+    if (op < QLORA_OP_FWD || op > QLORA_OP_FWD_MULTI) return 0;
+    if (op == QLORA_OP_FWD_MULTI && dtype != QLORA_BF16) return 0;
     if ((dtype != QLORA_BF16 && dtype != QLORA_F32) || T < 1 || d_out < 1 || d_in < 64 ||
         r_total < 1 || r_total > 128)
         return 0;
@@ -887,6 +913,65 @@ qlora_status lora_merge(const qlora_nf4* w, const void* A, const void* B, int32_
     if (adapter_dtype == QLORA_F32 && out_dtype == QLORA_F32)
         return run(k_merge<float, float>, static_cast<const float*>(A), static_cast<const float*>(B), static_cast<float*>(W_final));
     return QLORA_ERR_INVALID_ARG;
+}
+
+qlora_status qlora_linear_fwd_multi(const qlora_nf4* w, const void* X, int64_t T,
+                                    const int32_t* adapter_id, int32_t n_adapters,
+                                    const void* const* A_ptrs, const void* const* B_ptrs,
+                                    const int32_t* ranks, const float* scales, int32_t r_max,
+                                    void* H, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!A_ptrs || !B_ptrs || !ranks || !scales || !adapter_id) return QLORA_ERR_INVALID_ARG;
+    if (n_adapters < 1 || n_adapters > kSegMaxAdapters) return QLORA_ERR_UNSUPPORTED;
+    QL_TRY(check_layer(w, T, r_max, QLORA_BF16));
+    if (!aligned16(X) || !aligned16(H) || (reinterpret_cast<uintptr_t>(adapter_id) & 3u) ||
+        (reinterpret_cast<uintptr_t>(A_ptrs) & 7u) || (reinterpret_cast<uintptr_t>(B_ptrs) & 7u) ||
+        (reinterpret_cast<uintptr_t>(ranks) & 3u) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return QLORA_ERR_INVALID_ARG;
+    if (T > (1LL << 31) - 1) return QLORA_ERR_UNSUPPORTED;
+    const Plan p = make_plan(QLORA_OP_FWD_MULTI, QLORA_BF16, T, w->d_out, w->d_in, r_max);
+    QL_TRY(check_ws(ws, ws_bytes, p.total));
+    int* err = nullptr;
+    QL_TRY(err_word(&err));
+    SegArgs a{};
+    a.T = T;
+    a.n = n_adapters;
+    a.d_in = static_cast<int>(w->d_in);
+    a.d_out = static_cast<int>(w->d_out);
+    a.ldu = p.seg_ldu;
+    a.X = static_cast<const __nv_bfloat16*>(X);
+    a.H = static_cast<__nv_bfloat16*>(H);
+    a.ids = adapter_id;
+    a.A = reinterpret_cast<const __nv_bfloat16* const*>(A_ptrs);
+    a.B = reinterpret_cast<const __nv_bfloat16* const*>(B_ptrs);
+    a.ranks = ranks;
+    a.scales = scales;
+    a.cnt = at<int32_t>(ws, p.seg_cnt);
+    a.seg_start = at<int32_t>(ws, p.seg_start);
+    a.cursor = at<int32_t>(ws, p.seg_cursor);
+    a.n_tiles = at<int32_t>(ws, p.seg_ntiles);
+    a.tiles = at<int4>(ws, p.seg_tiles);
+    a.perm = at<int32_t>(ws, p.seg_perm);
+    a.U = at<__nv_bfloat16>(ws, p.seg_u);
+    a.err = err;
+    // sort and shrink, then the shared base term (H = bf16(X W^T)), then the corrections
+    if (cudaMemsetAsync(a.cnt, 0, static_cast<size_t>(n_adapters) * 4, stream) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    if (launch_pdl(k_seg_count, grid1d(T), dim3(256), 0, stream, a) != cudaSuccess) return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    if (launch_pdl(k_seg_plan, dim3(1), dim3(1024), 0, stream, a) != cudaSuccess) return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    if (launch_pdl(k_seg_scatter, grid1d(T), dim3(256), 0, stream, a) != cudaSuccess) return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    // persistent grids over the planned tiles: four resident CTAs of 128 threads per SM
+    const unsigned seg_grid = static_cast<unsigned>(std::min<int64_t>(p.seg_max_tiles, 4 * kSmsForSplit));
+    if (launch_pdl(k_seg_shrink, dim3(seg_grid), dim3(128), 0, stream, a) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    QL_TRY(nf4_gemm(false, w, X, T, nullptr, nullptr, 0, 0, 0, H, at<void>(ws, p.g2), err, stream));
+    if (launch_pdl(k_seg_expand, dim3(seg_grid), dim3(128), 0, stream, a) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
 }
 
 qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t T,

@@ -287,6 +287,78 @@ def test_batched_full_uniform_and_skewed(q):
         run_batched(q, mc, rows=rows)
 
 
+# ------------------------------------------------------------------ many-adapter (segmented) forward
+
+
+def run_multi(q, mc, rows=None):
+    import torch
+    w, oc = quantize_both(q, mc.W0)
+    Wh = oracle_weight(oc, mc.d_out, mc.d_in, "bf16")
+    tab = q.AdapterTable([dev(a, "bf16") for a in mc.As], [dev(b, "bf16") for b in mc.Bs], mc.alphas)
+    H = q.qlora_linear_fwd_multi(w, dev(mc.X, "bf16"), torch.from_numpy(mc.ids).cuda(), tab)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    sel = slice(None) if rows is None else rows
+    ref = O.lora_forward_batched(Wh, mc.X[sel], mc.ids[sel], mc.As, mc.Bs, mc.alphas, mc.ranks)
+    e = rel_fro(host(H)[sel], ref)
+    assert e <= TOL["bf16"], e
+    return H
+
+
+# mixed ranks 1..128 (odd ranks take the 16-bit B path, r > 64 two K tiles), ragged shapes
+def test_multi_mixed_ranks(q):
+    mc = S.make_multi_adapter(264, 320, 300, [1, 3, 8, 16, 33, 64, 100, 128, 7, 24], seed=11)
+    run_multi(q, mc)
+
+
+# a thousand adapters, about two tokens each (many partial tiles, some empty segments)
+def test_multi_many_adapters(q):
+    mc = S.make_multi_adapter(512, 512, 2048, [8, 16, 32, 64] * 250, seed=12)
+    run_multi(q, mc)
+
+
+# one adapter with most tokens (many full 16-token tiles of one segment)
+def test_multi_skewed(q):
+    mc = S.make_multi_adapter(384, 256, 1000, [16, 4, 64], split=[0.9, 0.05, 0.05], seed=13)
+    run_multi(q, mc)
+
+
+def test_multi_full_size_sampled_rows(q):
+    mc = S.make_multi_adapter(4096, 4096, 4096, [16] * 256, seed=14)
+    rows = np.sort(np.random.default_rng(2).choice(4096, 256, replace=False))
+    run_multi(q, mc, rows=rows)
+
+
+def test_multi_matches_single_adapter_path(q):
+    # one adapter for every token: the same layer as qlora_linear_fwd, within bf16 rounding
+    import torch
+    mc = S.make_multi_adapter(256, 384, 96, [16], seed=15)
+    w, _ = quantize_both(q, mc.W0)
+    X, A, B = dev(mc.X, "bf16"), dev(mc.As[0], "bf16"), dev(mc.Bs[0], "bf16")
+    H1, _ = q.qlora_linear_fwd(w, X, A, B, mc.alphas[0])
+    Hm = q.qlora_linear_fwd_multi(w, X, torch.from_numpy(mc.ids).cuda(), q.AdapterTable([A], [B], mc.alphas))
+    assert rel_fro(host(Hm), host(H1).astype(np.float64)) <= 4e-3
+
+
+def test_multi_bad_id_and_rank_report_device_error(q):
+    import torch
+    mc = S.make_multi_adapter(128, 128, 40, [4, 4], seed=16)
+    mc.ids[7] = 5
+    mc.ids[9] = -1
+    w, oc = quantize_both(q, mc.W0)
+    tab = q.AdapterTable([dev(a, "bf16") for a in mc.As], [dev(b, "bf16") for b in mc.Bs], mc.alphas)
+    H = q.qlora_linear_fwd_multi(w, dev(mc.X, "bf16"), torch.from_numpy(mc.ids).cuda(), tab)
+    assert q.get_device_error() == 5
+    assert q.get_device_error() == 0
+    ok = np.array([i for i in range(40) if i not in (7, 9)])
+    Wh = oracle_weight(oc, 128, 128, "bf16")
+    ref = O.lora_forward_batched(Wh, mc.X[ok], mc.ids[ok], mc.As, mc.Bs, mc.alphas, mc.ranks)
+    assert rel_fro(host(H)[ok], ref) <= TOL["bf16"]
+    # the bad tokens get the base term only
+    base = mc.X[[7, 9]].astype(np.float64) @ Wh.T
+    assert rel_fro(host(H)[[7, 9]], base) <= TOL["bf16"]
+
+
 def test_batched_bad_id_reports_device_error(q):
     import torch
     mc = S.make_multi_adapter(128, 128, 40, [4, 4], seed=6)
