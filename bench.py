@@ -188,6 +188,8 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     if args.only == "decode":
         return run_decode_only(args, q, qb, S, torch, dev)
+    if args.only == "multi":
+        return run_multi_only(args, q, qb, torch, dev)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -424,6 +426,49 @@ def run_decode_only(args, q, qb, S, torch, dev):
     return 0 if err == 0 else 1
 
 
+def make_multi_workload(q, torch, dev, n_ad=1024, r_ad=16, T=4096, seed=7, n_w=4):
+    """Many-adapter forward workload: 4096^2 NF4 base (n_w rotating copies), n_ad adapters of
+    rank r_ad drawn on the device, T tokens with uniform ids."""
+    bf = torch.bfloat16
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    W0 = torch.randn((4096, 4096), generator=gen, device=dev) * 0.02 ** 0.5
+    wl = [q.nf4_quantize(W0) for _ in range(n_w)]
+    del W0
+    X = torch.randn((T, 4096), generator=gen, device=dev).to(bf)
+    ids = torch.randint(0, n_ad, (T,), generator=gen, device=dev, dtype=torch.int32)
+    As = [(torch.randn((r_ad, 4096), generator=gen, device=dev) / r_ad ** 0.5).to(bf) for _ in range(n_ad)]
+    Bs = [(torch.randn((4096, r_ad), generator=gen, device=dev) * 0.1).to(bf) for _ in range(n_ad)]
+    tab = q.AdapterTable(As, Bs, [2.0 * r_ad] * n_ad)
+    H = torch.empty((T, 4096), dtype=bf, device=dev)
+    ws = torch.empty(q.workspace_bytes(q.OP_FWD_MULTI, q.BF16, T, 4096, 4096, r_ad),
+                     dtype=torch.uint8, device=dev)
+    return wl, X, ids, tab, H, ws
+
+
+def run_multi_only(args, q, qb, torch, dev):
+    """The many-adapter forward alone (4096^2, 1024 adapters of rank 16, 4096 tokens): W warm-up
+    and K timed eager calls over 4 rotating NF4 weights, for profiling its kernels."""
+    qb.build_library()
+    q.load()
+    wl, X, ids, tab, H, ws = make_multi_workload(q, torch, dev)
+    W = max(3, args.warmup)
+    for i in range(W):
+        q.qlora_linear_fwd_multi(wl[i % 4], X, ids, tab, H=H, ws=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        q.qlora_linear_fwd_multi(wl[i % 4], X, ids, tab, H=H, ws=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    err = q.get_device_error()
+    print(json.dumps({"only": "multi", "ms_per_call": e0.elapsed_time(e1) / args.steps,
+                      "device_error": err,
+                      "workload": "4096x4096 NF4 base, 1024 adapters r=16, T=4096 uniform ids"}), flush=True)
+    return 0 if err == 0 else 1
+
+
 def _graph_time(torch, calls, reps=20):
     """Per-call device time of `calls` (a list of zero-argument launches) captured in one CUDA
     graph and replayed `reps` times: (median, min) microseconds per call over 5 measurements."""
@@ -546,18 +591,7 @@ def extra_rows(q, torch, S, dev, peaks, args):
     # ---- many-adapter (segmented) forward: 4096^2 base, 1024 adapters of rank 16, T = 4096,
     # ids uniform (about 4 tokens per adapter); adapters drawn on the device (268 MB > L2)
     n_ad, r_ad, T_ad = 1024, 16, 4096
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(7)
-    mc = S.make_multi_adapter(4096, 4096, 1, [1], seed=7)          # only W0 is used from it
-    wl = [q.nf4_quantize(torch.from_numpy(mc.W0).to(dev)) for _ in range(4)]
-    X = torch.randn((T_ad, 4096), generator=gen, device=dev).to(bf)
-    ids = torch.randint(0, n_ad, (T_ad,), generator=gen, device=dev, dtype=torch.int32)
-    As = [(torch.randn((r_ad, 4096), generator=gen, device=dev) / r_ad ** 0.5).to(bf) for _ in range(n_ad)]
-    Bs = [(torch.randn((4096, r_ad), generator=gen, device=dev) * 0.1).to(bf) for _ in range(n_ad)]
-    tab = q.AdapterTable(As, Bs, [2.0 * r_ad] * n_ad)
-    H = torch.empty((T_ad, 4096), dtype=bf, device=dev)
-    ws = torch.empty(q.workspace_bytes(q.OP_FWD_MULTI, q.BF16, T_ad, 4096, 4096, r_ad),
-                     dtype=torch.uint8, device=dev)
+    wl, X, ids, tab, H, ws = make_multi_workload(q, torch, dev, n_ad, r_ad, T_ad)
     calls = [(lambda w=w: q.qlora_linear_fwd_multi(w, X, ids, tab, H=H, ws=ws)) for w in wl]
     med, _ = _graph_time(torch, calls, reps=10)
     fl = 2 * T_ad * 4096 * 4096 + 2 * T_ad * r_ad * (4096 + 4096)
@@ -566,7 +600,7 @@ def extra_rows(q, torch, S, dev, peaks, args):
     out["multi_1024x_r16_T4096"] = {"fwd_us": med, "tokens/s": T_ad / (med * 1e-6),
                                     "tflops": fl / (med * 1e-6) / 1e12, "t_roof_us": t_roof * 1e6,
                                     "roof_frac": t_roof / (med * 1e-6), "adapter_MB": n_ad * r_ad * 8192 * 2 / 1e6}
-    del wl, X, ids, As, Bs, tab, H, ws
+    del wl, X, ids, tab, H, ws
 
     # ---- merge W_final = W^ + s B A on the 4096^2 shape, bf16 out
     c2_ = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
@@ -599,9 +633,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--extra", action="store_true", help="also time the other hot-path rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--only", default="step", choices=["step", "fwd", "bwd", "decode"],
-                    help="time only the forward, only the backward, or the decode-size forward "
-                         "(11008x4096, r = 64, --tokens T) alone, for profiling one kernel")
+    ap.add_argument("--only", default="step", choices=["step", "fwd", "bwd", "decode", "multi"],
+                    help="time only the forward, only the backward, the decode-size forward "
+                         "(11008x4096, r = 64, --tokens T) or the many-adapter forward (4096^2, "
+                         "1024 adapters of rank 16) alone, for profiling its kernels")
     ap.add_argument("--tokens", type=int, default=1, help="tokens of the --only decode run")
     args = ap.parse_args()
     if args.impl == "reference":
