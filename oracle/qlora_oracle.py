@@ -31,6 +31,14 @@ What it computes, and where each step is defined:
 * Multi-adapter forward (shared x W0, per-request B_i A_i) -- "Large Language
   Model Fine-tuning and LoRA", section "Serving many adapters at once: the
   multi-tenant problem".
+* Adapter optimizer step: AdamW with an fp32 master copy, first moment m and
+  second moment v per trainable parameter -- Mathematical Foundations page,
+  section "The Memory Bottleneck of Full Parameter Fine-Tuning" (the AdamW
+  state list); gradient accumulation over micro-batches before one update --
+  "LoRA and QLoRA Fine-Tuning Under the Hood", section on gradient
+  accumulation (next to the FlashAttention-2 paragraph).  The pages name AdamW
+  but print no update rule; the oracle writes out the published decoupled
+  weight-decay rule (reading R23).
 
 Where the pages are silent or garbled the oracle takes the readings listed as
 R1..R19 in the design notes; each is named where it is applied.
@@ -294,6 +302,35 @@ def lora_forward_batched(W_hat, X, adapter_id, As, Bs, alphas, ranks):
         B = np.asarray(Bs[i], np.float64)
         H[t] += lora_scale(alphas[i], ranks[i]) * ((X[t] @ A.T) @ B.T)
     return H
+
+
+# ----------------------------------------------------------------------------
+# Adapter optimizer step (reading R23)
+# ----------------------------------------------------------------------------
+
+
+def adamw_step(w, g, m, v, step: int, lr: float, beta1: float, beta2: float,
+               eps: float, weight_decay: float, grad_scale: float = 1.0):
+    """One AdamW update of a trainable tensor (fp64), returning (w, m, v).
+
+    Decoupled weight decay (Loshchilov & Hutter's AdamW, the rule behind the
+    pages' "AdamW optimizer states"): the decay shrinks w directly, it is not
+    added to the gradient.  With step t >= 1 counted from 1 and the gradient
+    first multiplied by grad_scale (1 / micro-batches when accumulated):
+
+        g' = grad_scale * g
+        m  = beta1 m + (1 - beta1) g'
+        v  = beta2 v + (1 - beta2) g'^2
+        w  = w (1 - lr wd) - lr (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps)
+    """
+    w = np.asarray(w, np.float64)
+    g = np.asarray(g, np.float64) * grad_scale
+    m = beta1 * np.asarray(m, np.float64) + (1.0 - beta1) * g
+    v = beta2 * np.asarray(v, np.float64) + (1.0 - beta2) * g * g
+    m_hat = m / (1.0 - beta1 ** step)
+    v_hat = v / (1.0 - beta2 ** step)
+    w = w * (1.0 - lr * weight_decay) - lr * m_hat / (np.sqrt(v_hat) + eps)
+    return w, m, v
 
 
 # ----------------------------------------------------------------------------

@@ -295,6 +295,74 @@ def test_batched_matches_per_adapter():
         O.lora_forward_batched(W, X, np.full(T, 3), As, Bs, alphas, ranks)
 
 
+# ---------------------------------------------------------------- optimizer step (R23)
+
+ADAM = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
+
+
+def check_adamw_first_step(step_fn):
+    """From zero state the bias corrections make m_hat = g, v_hat = g^2 exactly:
+    w1 = w0 (1 - lr wd) - lr g / (|g| + eps)."""
+    rng = np.random.default_rng(21)
+    w0, g = rng.standard_normal(50), rng.standard_normal(50)
+    w1, m1, v1 = step_fn(w0, g, np.zeros(50), np.zeros(50), 1, **ADAM)
+    h = ADAM
+    ref = w0 * (1 - h["lr"] * h["weight_decay"]) - h["lr"] * g / (np.abs(g) + h["eps"])
+    return max(rel(w1, ref), rel(m1, (1 - h["beta1"]) * g), rel(v1, (1 - h["beta2"]) * g * g))
+
+
+def check_adamw_constant_gradient(step_fn):
+    """A constant gradient keeps m_hat = g and v_hat = g^2 at every step, so with no
+    decay each step moves w by exactly -lr g / (|g| + eps)."""
+    rng = np.random.default_rng(22)
+    w, g = rng.standard_normal(20), rng.standard_normal(20)
+    m, v = np.zeros(20), np.zeros(20)
+    h = dict(ADAM, weight_decay=0.0)
+    w0 = w.copy()
+    for t in range(1, 8):
+        w, m, v = step_fn(w, g, m, v, t, **h)
+    return rel(w, w0 - 7 * h["lr"] * g / (np.abs(g) + h["eps"]))
+
+
+def check_adamw_decay_only(step_fn):
+    """A zero gradient leaves m = v = 0 and only the decoupled decay: w_t = w0 (1 - lr wd)^t."""
+    w0 = np.linspace(-2, 2, 9)
+    w, m, v = w0.copy(), np.zeros(9), np.zeros(9)
+    for t in range(1, 6):
+        w, m, v = step_fn(w, np.zeros(9), m, v, t, **ADAM)
+    return rel(w, w0 * (1 - ADAM["lr"] * ADAM["weight_decay"]) ** 5)
+
+
+def test_adamw_first_step_closed_form():
+    assert check_adamw_first_step(O.adamw_step) < 1e-14
+
+
+def test_adamw_constant_gradient():
+    assert check_adamw_constant_gradient(O.adamw_step) < 1e-13
+
+
+def test_adamw_decay_only():
+    assert check_adamw_decay_only(O.adamw_step) < 1e-14
+
+
+def test_adamw_grad_scale_is_a_gradient_multiplier():
+    rng = np.random.default_rng(23)
+    w, g = rng.standard_normal(10), rng.standard_normal(10)
+    a = O.adamw_step(w, g, np.zeros(10), np.zeros(10), 3, grad_scale=0.25, **ADAM)
+    b = O.adamw_step(w, 0.25 * g, np.zeros(10), np.zeros(10), 3, **ADAM)
+    assert all(rel(x, y) < 1e-15 for x, y in zip(a, b))
+
+
+def test_gradient_accumulation_equals_full_batch():
+    """dA, dB are sums over tokens, so accumulating the micro-batches' gradients gives the
+    full batch's gradients (the pages' gradient accumulation before one update)."""
+    W, X, A, B, dH = small_layer(d=7, k=6, r=2, T=8)
+    full = O.lora_adapter_grads(X, dH, A, B, 4.0, 2)
+    parts = [O.lora_adapter_grads(X[i:i + 3], dH[i:i + 3], A, B, 4.0, 2) for i in (0, 3, 6)]
+    assert rel(sum(p[0] for p in parts), full[0]) < 1e-13
+    assert rel(sum(p[1] for p in parts), full[1]) < 1e-13
+
+
 # ---------------------------------------------------------------- mutants
 
 
@@ -328,6 +396,21 @@ def test_pins_catch_planted_mistakes():
     assert check_gradients_fd(O.lora_forward, bwd_dx_no_adapter) > 1e-3
     assert check_gradients_fd(O.lora_forward, bwd_transposed_W) > 1e-3
     assert check_merge(O.lora_forward, merge_noscale) > 1e-3
+
+    def adam_no_bias_correction(w, g, m, v, t, lr, beta1, beta2, eps, weight_decay, grad_scale=1.0):
+        m = beta1 * m + (1 - beta1) * g
+        v = beta2 * v + (1 - beta2) * g * g
+        return w * (1 - lr * weight_decay) - lr * m / (np.sqrt(v) + eps), m, v
+
+    def adam_coupled_decay(w, g, m, v, t, lr, beta1, beta2, eps, weight_decay, grad_scale=1.0):
+        return O.adamw_step(w, g + weight_decay * w, m, v, t, lr, beta1, beta2, eps, 0.0)
+
+    def adam_swapped_betas(w, g, m, v, t, lr, beta1, beta2, eps, weight_decay, grad_scale=1.0):
+        return O.adamw_step(w, g, m, v, t, lr, beta2, beta1, eps, weight_decay)
+
+    assert check_adamw_first_step(adam_no_bias_correction) > 1e-3
+    assert check_adamw_decay_only(adam_coupled_decay) > 1e-3
+    assert check_adamw_first_step(adam_swapped_betas) > 1e-3
 
     # quantizer mutants: swapped nibbles and a 255-level second stage
     L = O.nf4_levels()
