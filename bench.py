@@ -602,6 +602,25 @@ def extra_rows(q, torch, S, dev, peaks, args):
                                     "roof_frac": t_roof / (med * 1e-6), "adapter_MB": n_ad * r_ad * 8192 * 2 / 1e6}
     del wl, X, ids, tab, H, ws
 
+    # ---- AdamW step over the adapters of a 32-layer d = 4096 model with rank 16 on q, k, v, o:
+    # 32 * 4 * 16 * (4096 + 4096) = 16.8 M parameters, bf16 params + fp32 master, m, v, grad
+    # (30 bytes per parameter, 503 MB > L2)
+    n_p = 32 * 4 * 16 * 8192
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3)
+    master = torch.randn(n_p, generator=gen, device=dev)
+    param = master.to(bf)
+    grad = torch.randn(n_p, generator=gen, device=dev)
+    m_s = torch.zeros(n_p, device=dev)
+    v_s = torch.zeros(n_p, device=dev)
+    calls = [(lambda t=t: q.adamw_step(param, grad, m_s, v_s, t, 1e-4, weight_decay=0.01, master=master))
+             for t in range(1, 5)]
+    med, _ = _graph_time(torch, calls, reps=10)
+    byts = 30 * n_p
+    out["adamw_16.8M_params"] = {"us": med, "GB/s": byts / (med * 1e-6) / 1e9,
+                                 "hbm_frac": byts / (med * 1e-6) / 1e9 / hbm}
+    del master, param, grad, m_s, v_s
+
     # ---- merge W_final = W^ + s B A on the 4096^2 shape, bf16 out
     c2_ = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
     d, k, r, alpha = c2_["d_out"], c2_["d_in"], c2_["r"], c2_["alpha"]

@@ -130,6 +130,40 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
                               float* dA, float* dB, void* ws, size_t ws_bytes,
                               cudaStream_t stream);
 
+/* qlora_linear_bwd with flags.  QLORA_BWD_ACCUMULATE adds the call's dA, dB into the caller's
+ * buffers (dA += ..., dB += ...) instead of overwriting them: gradient accumulation over
+ * micro-batches before one optimizer update ([UH], the gradient-accumulation paragraph next to
+ * FlashAttention-2).  dX is always overwritten.  Unknown flag bits: QLORA_ERR_INVALID_ARG.    */
+#define QLORA_BWD_ACCUMULATE 1u
+qlora_status qlora_linear_bwd_ex(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                                 const void* A, const void* B, int32_t r, float alpha,
+                                 const void* U_saved, qlora_dtype dtype, void* dX,
+                                 float* dA, float* dB, void* ws, size_t ws_bytes,
+                                 uint32_t flags, cudaStream_t stream);
+
+/* One AdamW step of an adapter tensor of n elements (decoupled weight decay):
+ *   g' = grad_scale g;  m = beta1 m + (1 - beta1) g';  v = beta2 v + (1 - beta2) g'^2;
+ *   w  = w (1 - lr weight_decay) - lr (m / (1 - beta1^step)) / (sqrt(v / (1 - beta2^step)) + eps)
+ * in fp32, step counted from 1; grad_scale = 1 / micro-batches for accumulated gradients.
+ * [MF] "The Memory Bottleneck of Full Parameter Fine-Tuning" (AdamW state: fp32 master, m, v);
+ * the pages print no update rule, this is the published AdamW (reading R23).
+ *   param   bf16 (then master, fp32 [n], is the weight and param gets its RN-even copy) or
+ *           fp32 (updated in place; master must be NULL or equal to param)
+ *   grad, m, v  fp32 [n]; m, v updated in place.  Any of the fp32 arrays may be unified
+ *           memory (the "paged optimizer" state; see qlora_prefetch).
+ * 16-byte aligned arrays with n % 4 == 0 take the vector path.  No allocation; asynchronous.  */
+qlora_status qlora_adamw_step(void* param, qlora_dtype param_dtype, float* master,
+                              const float* grad, float* m, float* v, int64_t n, int32_t step,
+                              float lr, float beta1, float beta2, float eps, float weight_decay,
+                              float grad_scale, cudaStream_t stream);
+
+/* Page a caller-allocated unified-memory range (cudaMallocManaged) of optimizer state to the
+ * current device (to_device != 0) before a step, or back to host memory after it, so that the
+ * state occupies HBM only while it is used: [CH] "Paged optimizers", [MF] "3. Paged
+ * Optimizers", [L26] "Paged Optimizers" (optimizer state in unified memory, paged between GPU
+ * and CPU).  Asynchronous on `stream`; the library allocates nothing.                         */
+qlora_status qlora_prefetch(const void* ptr, size_t bytes, int32_t to_device, cudaStream_t stream);
+
 /* Merge: W_final = W + (alpha/r) B A, dense (not re-quantized), out_dtype fp32 or bf16;
  * W is the decoded weight in out_dtype's decode.  A, B are given in adapter_dtype.
  * [MF] "Production Serving and Multi-Tenant Routing", "1. Static Weight Merging";

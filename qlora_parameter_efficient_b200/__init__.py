@@ -27,6 +27,7 @@ OP_FWD, OP_BWD, OP_FWD_BATCHED, OP_MERGE, OP_FWD_MULTI = 0, 1, 2, 3, 4
 # Every symbol include/qlora.h declares.
 EXPORTS = ["qlora_nf4_sizes", "qlora_nf4_levels", "nf4_quantize", "nf4_dequantize",
            "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "lora_merge",
+           "qlora_linear_bwd_ex", "qlora_adamw_step", "qlora_prefetch",
            "qlora_linear_fwd_batched", "qlora_linear_fwd_multi", "qlora_linear_fwd_noalloc",
            "qlora_get_device_error",
            "qlora_selftest_wait_timeout", "qlora_set_gemm_events", "qlora_launch_count",
@@ -72,6 +73,11 @@ def load() -> ctypes.CDLL:
                                      ctypes.c_int),
         "qlora_linear_fwd_multi": ([pnf4, vp, i64, vp, i32, vp, vp, vp, vp, i32, vp, vp, sz, vp],
                                    ctypes.c_int),
+        "qlora_linear_bwd_ex": ([pnf4, vp, vp, i64, vp, vp, i32, f32, vp, ctypes.c_int, vp, vp, vp, vp, sz,
+                                 ctypes.c_uint32, vp], ctypes.c_int),
+        "qlora_adamw_step": ([vp, ctypes.c_int, vp, vp, vp, vp, i64, i32, f32, f32, f32, f32, f32, f32, vp],
+                             ctypes.c_int),
+        "qlora_prefetch": ([vp, sz, i32, vp], ctypes.c_int),
         "qlora_linear_fwd_noalloc": ([pnf4, vp, i64, vp, vp, i32, f32, ctypes.c_int, vp, vp, vp], ctypes.c_int),
         "qlora_get_device_error": ([vp], ctypes.c_int),
         "qlora_selftest_wait_timeout": ([ctypes.c_uint64, vp], ctypes.c_int),
@@ -205,9 +211,12 @@ def qlora_linear_fwd(w: NF4Weight, X, A, B, alpha, H=None, U_save=None, ws=None,
     return H, U_save
 
 
+BWD_ACCUMULATE = 1
+
+
 def qlora_linear_bwd(w: NF4Weight, X, dH, A, B, alpha, U_saved=None, dX=None, dA=None, dB=None,
-                     ws=None, stream=None, want_dx=True):
-    """Returns (dX, dA, dB); dA, dB fp32."""
+                     ws=None, stream=None, want_dx=True, accumulate=False):
+    """Returns (dX, dA, dB); dA, dB fp32.  accumulate=True adds into the given dA, dB."""
     torch = _torch()
     _contig(X, dH, A, B, U_saved, dX, dA, dB)
     T = X.shape[0]
@@ -221,10 +230,34 @@ def qlora_linear_bwd(w: NF4Weight, X, dH, A, B, alpha, U_saved=None, dX=None, dA
         dB = torch.empty((w.d_out, r), dtype=torch.float32, device=X.device)
     ws = _ws(OP_BWD, dt, T, w.d_out, w.d_in, r, X.device, ws)
     c = w._c()
-    _check("qlora_linear_bwd", load().qlora_linear_bwd(
-        ctypes.byref(c), _ptr(X), _ptr(dH), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(U_saved), dt,
-        _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream(stream)))
+    if accumulate:
+        _check("qlora_linear_bwd_ex", load().qlora_linear_bwd_ex(
+            ctypes.byref(c), _ptr(X), _ptr(dH), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(U_saved),
+            dt, _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), BWD_ACCUMULATE, _stream(stream)))
+    else:
+        _check("qlora_linear_bwd", load().qlora_linear_bwd(
+            ctypes.byref(c), _ptr(X), _ptr(dH), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(U_saved),
+            dt, _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream(stream)))
     return dX, dA, dB
+
+
+def adamw_step(param, grad, m, v, step, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0,
+               master=None, grad_scale=1.0, stream=None):
+    """One AdamW step in place: param (bf16 with an fp32 master, or fp32), grad, m, v fp32."""
+    torch = _torch()
+    _contig(param, grad, m, v, master)
+    n = param.numel()
+    _check("qlora_adamw_step", load().qlora_adamw_step(
+        _ptr(param), _dtype_code(param.dtype), _ptr(master), _ptr(grad), _ptr(m), _ptr(v), n,
+        int(step), float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+        float(grad_scale), _stream(stream)))
+    return param
+
+
+def prefetch(ptr: int, nbytes: int, to_device: bool, stream=None):
+    """Page a unified-memory range to the current device or back to the host."""
+    _check("qlora_prefetch", load().qlora_prefetch(ctypes.c_void_p(ptr), nbytes, 1 if to_device else 0,
+                                                   _stream(stream)))
 
 
 def lora_merge(w: NF4Weight, A, B, alpha, out_dtype, out=None, stream=None):

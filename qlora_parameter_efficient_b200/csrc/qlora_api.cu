@@ -16,6 +16,7 @@
 #include "nf4_gemm2.cuh"
 #include "merge.cuh"
 #include "segmented.cuh"
+#include "optim.cuh"
 #include "qgemv.cuh"
 
 using namespace qlora;
@@ -768,10 +769,13 @@ qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T, cons
                  static_cast<float*>(H), d_out);
 }
 
-qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
-                              const void* A, const void* B, int32_t r, float alpha,
-                              const void* U_saved, qlora_dtype dtype, void* dX, float* dA,
-                              float* dB, void* ws, size_t ws_bytes, cudaStream_t stream) {
+qlora_status qlora_linear_bwd_ex(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                                 const void* A, const void* B, int32_t r, float alpha,
+                                 const void* U_saved, qlora_dtype dtype, void* dX, float* dA,
+                                 float* dB, void* ws, size_t ws_bytes, uint32_t flags,
+                                 cudaStream_t stream) {
+    if (flags & ~static_cast<uint32_t>(QLORA_BWD_ACCUMULATE)) return QLORA_ERR_INVALID_ARG;
+    const int acc_grads = (flags & QLORA_BWD_ACCUMULATE) ? 1 : 0;
     QL_TRY(check_layer(w, T, r, dtype));
     if (!aligned16(X) || !aligned16(dH) || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
         !aligned16(dB) || !aligned16_or_null(dX) || !aligned16_or_null(U_saved))
@@ -832,7 +836,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
             QL_TRY(tmap_bf16(&tgm, g_spad, T, RP, RP, 64));
             QL_TRY(skinny_gemm(true, true, RP, r, txm, tgm, d_in, cdiv(T, kBK), p.split_da, part, err, stream));
             if (launch_pdl(k_finalize_dA, grid1d(static_cast<int64_t>(r) * d_in), dim3(256), 0,
-                           stream, part, p.split_da, d_in * RP, d_in, r, RP, dA) != cudaSuccess)
+                           stream, part, p.split_da, d_in * RP, d_in, r, RP, dA, acc_grads) != cudaSuccess)
                 return QLORA_ERR_CUDA;
             QL_LAUNCH_CHECK();
         }
@@ -843,7 +847,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
             QL_TRY(tmap_bf16(&tum, u_src, T, u_ld, u_ld, 64));
             QL_TRY(skinny_gemm(true, true, RP, r, thm, tum, d_out, cdiv(T, kBK), p.split_db, part, err, stream));
             if (launch_pdl(k_finalize_dB, grid1d(d_out * r), dim3(256), 0, stream, part, p.split_db,
-                           d_out * RP, d_out, r, RP, s, dB) != cudaSuccess)
+                           d_out * RP, d_out, r, RP, s, dB, acc_grads) != cudaSuccess)
                 return QLORA_ERR_CUDA;
             QL_LAUNCH_CHECK();
         }
@@ -869,8 +873,65 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
         QL_TRY(sgemm(stream, T, d_in, d_out, 1.f, dHf, d_out, false, w32, d_in, false, 0.f, dXf, d_in));
         QL_TRY(sgemm(stream, T, d_in, r, s, G, r, false, Af, d_in, false, 1.f, dXf, d_in));
     }
-    QL_TRY(sgemm(stream, r, d_in, T, s, G, r, true, Xf, d_in, false, 0.f, dA, d_in));
-    return sgemm(stream, d_out, r, T, s, dHf, d_out, true, Uc, r, false, 0.f, dB, r);
+    const float beta = acc_grads ? 1.f : 0.f;
+    QL_TRY(sgemm(stream, r, d_in, T, s, G, r, true, Xf, d_in, false, beta, dA, d_in));
+    return sgemm(stream, d_out, r, T, s, dHf, d_out, true, Uc, r, false, beta, dB, r);
+}
+
+qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                              const void* A, const void* B, int32_t r, float alpha,
+                              const void* U_saved, qlora_dtype dtype, void* dX, float* dA,
+                              float* dB, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    return qlora_linear_bwd_ex(w, X, dH, T, A, B, r, alpha, U_saved, dtype, dX, dA, dB, ws,
+                               ws_bytes, 0u, stream);
+}
+
+qlora_status qlora_adamw_step(void* param, qlora_dtype param_dtype, float* master,
+                              const float* grad, float* m, float* v, int64_t n, int32_t step,
+                              float lr, float beta1, float beta2, float eps, float weight_decay,
+                              float grad_scale, cudaStream_t stream) {
+    if (!param || !grad || !m || !v || n < 1 || step < 1) return QLORA_ERR_INVALID_ARG;
+    if (param_dtype == QLORA_BF16 && (!master || master == param)) return QLORA_ERR_INVALID_ARG;
+    if (param_dtype == QLORA_F32 && master && master != param) return QLORA_ERR_INVALID_ARG;
+    if (param_dtype != QLORA_BF16 && param_dtype != QLORA_F32) return QLORA_ERR_INVALID_ARG;
+    if (!(beta1 >= 0.f && beta1 < 1.f && beta2 >= 0.f && beta2 < 1.f)) return QLORA_ERR_INVALID_ARG;
+    AdamArgs a{};
+    a.n = n;
+    a.lr = lr;
+    a.beta1 = beta1;
+    a.beta2 = beta2;
+    a.eps = eps;
+    a.wd = weight_decay;
+    a.grad_scale = grad_scale;
+    a.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(beta1), step));
+    a.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(beta2), step));
+    const bool vec = n % 4 == 0 && aligned16(param) && aligned16(grad) && aligned16(m) &&
+                     aligned16(v) && (param_dtype == QLORA_F32 || aligned16(master)) &&
+                     (param_dtype == QLORA_F32 || (reinterpret_cast<uintptr_t>(param) & 7u) == 0);
+    const dim3 grid = grid1d(vec ? n / 4 : n);
+    cudaError_t e;
+    if (param_dtype == QLORA_BF16) {
+        auto* pb = static_cast<__nv_bfloat16*>(param);
+        e = vec ? launch_pdl(k_adamw<__nv_bfloat16, true>, grid, dim3(256), 0, stream, pb, master, grad, m, v, a)
+                : launch_pdl(k_adamw<__nv_bfloat16, false>, grid, dim3(256), 0, stream, pb, master, grad, m, v, a);
+    } else {
+        auto* pf = static_cast<float*>(param);
+        e = vec ? launch_pdl(k_adamw<float, true>, grid, dim3(256), 0, stream, pf, pf, grad, m, v, a)
+                : launch_pdl(k_adamw<float, false>, grid, dim3(256), 0, stream, pf, pf, grad, m, v, a);
+    }
+    if (e != cudaSuccess) return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+qlora_status qlora_prefetch(const void* ptr, size_t bytes, int32_t to_device, cudaStream_t stream) {
+    if (!ptr || bytes == 0) return QLORA_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+    cudaMemLocation loc{};
+    loc.type = to_device ? cudaMemLocationTypeDevice : cudaMemLocationTypeHost;
+    loc.id = to_device ? dev : 0;
+    return cudaMemPrefetchAsync(ptr, bytes, loc, 0, stream) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 qlora_status lora_merge(const qlora_nf4* w, const void* A, const void* B, int32_t r, float alpha,

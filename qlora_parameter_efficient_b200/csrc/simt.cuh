@@ -163,7 +163,7 @@ __global__ void k_finalize_multi(const float* __restrict__ P, int split, int64_t
 
 // dA[j, n] = sum_z P[z][n][j]  (the dA GEMM computes dA^T tiles), j < r.
 __global__ void k_finalize_dA(const float* __restrict__ P, int split, int64_t split_stride,
-                              int64_t d_in, int r, int RP, float* __restrict__ dA) {
+                              int64_t d_in, int r, int RP, float* __restrict__ dA, int accumulate) {
     griddep_enter();
     const int64_t n = static_cast<int64_t>(r) * d_in;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -171,13 +171,14 @@ __global__ void k_finalize_dA(const float* __restrict__ P, int split, int64_t sp
         const int64_t j = i / d_in, col = i % d_in;
         float acc = 0.f;
         for (int zz = 0; zz < split; ++zz) acc += P[zz * split_stride + col * RP + j];
-        dA[i] = acc;
+        dA[i] = accumulate ? dA[i] + acc : acc;
     }
 }
 
 // dB[i, j] = scale * sum_z P[z][i][j], j < r.
 __global__ void k_finalize_dB(const float* __restrict__ P, int split, int64_t split_stride,
-                              int64_t d_out, int r, int RP, float scale, float* __restrict__ dB) {
+                              int64_t d_out, int r, int RP, float scale, float* __restrict__ dB,
+                              int accumulate) {
     griddep_enter();
     const int64_t n = d_out * r;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -186,7 +187,7 @@ __global__ void k_finalize_dB(const float* __restrict__ P, int split, int64_t sp
         const int j = static_cast<int>(i % r);
         float acc = 0.f;
         for (int zz = 0; zz < split; ++zz) acc += P[zz * split_stride + row * RP + j];
-        dB[i] = scale * acc;
+        dB[i] = accumulate ? dB[i] + scale * acc : scale * acc;
     }
 }
 

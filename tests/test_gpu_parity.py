@@ -396,3 +396,143 @@ def test_launch_counter_moves(q):
     q.qlora_linear_fwd(w, dev(case.X, "bf16"), dev(case.A, "bf16"), dev(case.B, "bf16"), 8.0)
     torch.cuda.synchronize()
     assert q.launch_count() - n0 >= 3          # quantize, U pre-pass, weight stream
+
+
+# ------------------------------------------------------------------ training-step tail
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_bwd_accumulate_matches_full_batch(q, dtype):
+    """Two micro-batches with QLORA_BWD_ACCUMULATE give the full batch's dA, dB."""
+    import torch
+    case = S.make_layer(192, 256, 8, 16.0, 160, dtype=dtype, seed=31)
+    w, oc = quantize_both(q, case.W0)
+    X, A, B, dH = dev(case.X, dtype), dev(case.A, dtype), dev(case.B, dtype), dev(case.dH, dtype)
+    _, dA, dB = q.qlora_linear_bwd(w, X[:96], dH[:96], A, B, case.alpha, want_dx=False)
+    q.qlora_linear_bwd(w, X[96:], dH[96:], A, B, case.alpha, dA=dA, dB=dB, want_dx=False, accumulate=True)
+    _, dA_full, dB_full = q.qlora_linear_bwd(w, X, dH, A, B, case.alpha, want_dx=False)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    dAref, dBref = O.lora_adapter_grads(case.X, case.dH, case.A, case.B, case.alpha, case.r)
+    assert rel_fro(host(dA), dAref) <= TOL[dtype]
+    assert rel_fro(host(dB), dBref) <= TOL[dtype]
+    assert rel_fro(host(dA), host(dA_full).astype(np.float64)) <= 1e-5
+    assert rel_fro(host(dB), host(dB_full).astype(np.float64)) <= 1e-5
+
+
+# The API takes fp32 hyperparameters; the oracle gets the same (fp32-representable) values, since
+# 1 - beta2 magnifies the fp32 rounding of beta2 = 0.999 to ~1e-5 relative.
+HP = {k: float(np.float32(x)) for k, x in dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8,
+                                                 weight_decay=0.01).items()}
+
+
+def run_adam(q, n, param_dtype, steps=4, seed=41, grad_scale=0.5):
+    """`steps` AdamW steps on the GPU and in the oracle; returns the GPU state and the errors."""
+    import torch
+    rng = np.random.default_rng(seed)
+    w0 = rng.standard_normal(n).astype(np.float32)
+    grads = [rng.standard_normal(n).astype(np.float32) for _ in range(steps)]
+    mk = lambda a: torch.from_numpy(a).cuda()        # noqa: E731
+    m, v = mk(np.zeros(n, np.float32)), mk(np.zeros(n, np.float32))
+    if param_dtype == "bf16":
+        master = mk(w0.copy())
+        param = torch.from_numpy(w0).cuda().bfloat16()
+    else:
+        master, param = None, mk(w0.copy())
+    g = torch.empty(n, dtype=torch.float32, device="cuda")
+    wr, mr, vr = w0.astype(np.float64), np.zeros(n), np.zeros(n)
+    for t in range(1, steps + 1):
+        g.copy_(torch.from_numpy(grads[t - 1]))
+        q.adamw_step(param, g, m, v, t, master=master, grad_scale=grad_scale, **HP)
+        wr, mr, vr = O.adamw_step(wr, grads[t - 1], mr, vr, t, grad_scale=grad_scale, **HP)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    wg = host(master if master is not None else param)
+    err = (rel_fro(wg, wr), rel_fro(host(m), mr), rel_fro(host(v), vr))
+    return param, master, m, v, err
+
+
+@pytest.mark.parametrize("n", [4096, 1001])        # vector path and scalar path
+@pytest.mark.parametrize("param_dtype", ["bf16", "f32"])
+def test_adamw_matches_oracle(q, n, param_dtype):
+    import torch
+    param, master, m, v, err = run_adam(q, n, param_dtype)
+    assert max(err) <= 1e-6, err
+    if param_dtype == "bf16":
+        # the bf16 parameter is the RN-even copy of the fp32 master, bit for bit
+        assert torch.equal(param, master.bfloat16())
+
+
+def test_adamw_state_in_unified_memory(q):
+    """Optimizer state in cudaMallocManaged memory ("paged optimizers"), paged to the GPU
+    before each step and back to the host after: bit-identical to device-resident state."""
+    import ctypes, torch
+    rt = None
+    for name in ("/usr/local/cuda/lib64/libcudart.so", "/usr/local/cuda/lib64/libcudart.so.12", "libcudart.so.12"):
+        try:
+            rt = ctypes.CDLL(name)
+            break
+        except OSError:
+            continue
+    if rt is None:
+        pytest.skip("no libcudart to allocate unified memory with")
+    rt.cudaMallocManaged.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_size_t, ctypes.c_uint]
+    rt.cudaFree.argtypes = [ctypes.c_void_p]
+    bufs = []
+
+    def alloc(a):
+        p = ctypes.c_void_p()
+        assert rt.cudaMallocManaged(ctypes.byref(p), a.nbytes, 1) == 0
+        bufs.append(p)
+        arr = np.ctypeslib.as_array(ctypes.cast(p, ctypes.POINTER(ctypes.c_float)), shape=a.shape)
+        arr[...] = a
+        t = torch.from_numpy(arr)            # host view; the kernels take its address
+        return _ManagedTensor(t, p.value)
+
+    class _ManagedTensor:
+        """Float32 unified-memory array: a host view plus the address the kernels take."""
+
+        def __init__(self, t, addr):
+            self.t, self.addr = t, addr
+            self.dtype, self.shape = torch.float32, t.shape
+
+        def data_ptr(self):
+            return self.addr
+
+        def numel(self):
+            return self.t.numel()
+
+        def is_contiguous(self):
+            return True
+
+        def prefetch(self, to_device):
+            q.prefetch(self.addr, self.t.numel() * 4, to_device)
+
+    try:
+        n = 8192
+        rng = np.random.default_rng(42)
+        w0 = rng.standard_normal(n).astype(np.float32)
+        grads = [rng.standard_normal(n).astype(np.float32) for _ in range(3)]
+        mm, vm, wm = alloc(np.zeros(n, np.float32)), alloc(np.zeros(n, np.float32)), alloc(w0.copy())
+        md, vd, wd = (torch.zeros(n, device="cuda"), torch.zeros(n, device="cuda"),
+                      torch.from_numpy(w0.copy()).cuda())
+        pm, pd = torch.from_numpy(w0).cuda().bfloat16(), torch.from_numpy(w0).cuda().bfloat16()
+        g = torch.empty(n, dtype=torch.float32, device="cuda")
+        for t in range(1, 4):
+            g.copy_(torch.from_numpy(grads[t - 1]))
+            for s in (mm, vm, wm):
+                s.prefetch(True)
+            q.adamw_step(pm, g, mm, vm, t, master=wm, **HP)
+            for s in (mm, vm, wm):
+                s.prefetch(False)
+            q.adamw_step(pd, g, md, vd, t, master=wd, **HP)
+        torch.cuda.synchronize()
+        assert q.get_device_error() == 0
+        assert np.array_equal(mm.t.numpy(), md.cpu().numpy())
+        assert np.array_equal(vm.t.numpy(), vd.cpu().numpy())
+        assert np.array_equal(wm.t.numpy(), wd.cpu().numpy())
+        assert torch.equal(pm, pd)
+    finally:
+        torch.cuda.synchronize()
+        for p in bufs:
+            rt.cudaFree(p)
