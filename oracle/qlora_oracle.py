@@ -31,6 +31,12 @@ What it computes, and where each step is defined:
 * Multi-adapter forward (shared x W0, per-request B_i A_i) -- "Large Language
   Model Fine-tuning and LoRA", section "Serving many adapters at once: the
   multi-tenant problem".
+* DoRA forward -- "Large Language Model Fine-tuning and LoRA", section
+  "Choosing what to adapt" (a magnitude vector of size d_out trained directly,
+  the low-rank update applied to the direction); Mathematical Foundations
+  page, section "Advanced Variants: DoRA and LoRA+" (W = m (V + dW) / ||V + dW||).
+  Reading R24: one magnitude per output row, each row of W0 + s B A divided by
+  its Euclidean norm.
 * Adapter optimizer step: AdamW with an fp32 master copy, first moment m and
   second moment v per trainable parameter -- Mathematical Foundations page,
   section "The Memory Bottleneck of Full Parameter Fine-Tuning" (the AdamW
@@ -302,6 +308,32 @@ def lora_forward_batched(W_hat, X, adapter_id, As, Bs, alphas, ranks):
         B = np.asarray(Bs[i], np.float64)
         H[t] += lora_scale(alphas[i], ranks[i]) * ((X[t] @ A.T) @ B.T)
     return H
+
+
+# ----------------------------------------------------------------------------
+# DoRA (reading R24)
+# ----------------------------------------------------------------------------
+
+
+def dora_row_norms(W_hat, A, B, alpha, r):
+    """||W[j, :]||_2 of W = W_hat + s B A for every output row j (fp64)."""
+    W = np.asarray(W_hat, np.float64) + lora_scale(alpha, r) * (
+        np.asarray(B, np.float64) @ np.asarray(A, np.float64))
+    return np.sqrt(np.sum(W * W, axis=1))
+
+
+def dora_forward(W_hat, X, A, B, alpha, r, magnitude):
+    """H = X W'^T with W'[j, :] = m_j (W_hat + s B A)[j, :] / ||(W_hat + s B A)[j, :]||.
+
+    The decomposition puts the norm of every output row of the adapted weight into the
+    trained magnitude m (size d_out) and keeps only its direction; written as the plain
+    product with the full adapted weight.
+    """
+    W = np.asarray(W_hat, np.float64) + lora_scale(alpha, r) * (
+        np.asarray(B, np.float64) @ np.asarray(A, np.float64))
+    norms = np.sqrt(np.sum(W * W, axis=1))
+    Wd = (np.asarray(magnitude, np.float64) / norms)[:, None] * W
+    return np.asarray(X, np.float64) @ Wd.T
 
 
 # ----------------------------------------------------------------------------

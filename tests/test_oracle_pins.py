@@ -295,6 +295,44 @@ def test_batched_matches_per_adapter():
         O.lora_forward_batched(W, X, np.full(T, 3), As, Bs, alphas, ranks)
 
 
+# ---------------------------------------------------------------- DoRA (R24)
+
+
+def check_dora_brute(fwd):
+    """Loops over a tiny layer: W' = m_j W_j / ||W_j|| row by row, then h = W' x."""
+    W, X, A, B, dH = small_layer(d=5, k=4, r=2, T=3)
+    mag = np.array([0.5, 1.5, 2.0, 0.25, 1.0])
+    alpha, r = 3.0, 2
+    H = fwd(W, X, A, B, alpha, r, mag)
+    ref = np.zeros((3, 5))
+    for j in range(5):
+        row = [W[j, c] + (alpha / r) * sum(B[j, q] * A[q, c] for q in range(r)) for c in range(4)]
+        nrm = math.sqrt(sum(x * x for x in row))
+        for t in range(3):
+            ref[t, j] = sum(mag[j] * row[c] / nrm * X[t, c] for c in range(4))
+    return rel(H, ref)
+
+
+def test_dora_against_loops():
+    assert check_dora_brute(O.dora_forward) < 1e-13
+
+
+def test_dora_magnitude_equal_to_norms_is_lora():
+    """With m set to the row norms of W + sBA (DoRA's initialisation) the layer is LoRA."""
+    W, X, A, B, dH = small_layer(d=9, k=7, r=3, T=4)
+    mag = O.dora_row_norms(W, A, B, 6.0, 3)
+    assert rel(O.dora_forward(W, X, A, B, 6.0, 3, mag), O.lora_forward(W, X, A, B, 6.0, 3)) < 1e-13
+
+
+def test_dora_direction_is_scale_free():
+    """Scaling the adapted weight (W and B together) leaves the DoRA output unchanged."""
+    W, X, A, B, dH = small_layer(d=6, k=5, r=2, T=3)
+    mag = np.linspace(0.5, 2.0, 6)
+    h1 = O.dora_forward(W, X, A, B, 4.0, 2, mag)
+    h2 = O.dora_forward(3.5 * W, X, A, 3.5 * B, 4.0, 2, mag)
+    assert rel(h1, h2) < 1e-13
+
+
 # ---------------------------------------------------------------- optimizer step (R23)
 
 ADAM = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
@@ -411,6 +449,17 @@ def test_pins_catch_planted_mistakes():
     assert check_adamw_first_step(adam_no_bias_correction) > 1e-3
     assert check_adamw_decay_only(adam_coupled_decay) > 1e-3
     assert check_adamw_first_step(adam_swapped_betas) > 1e-3
+
+    def dora_no_adapter_in_norm(W, X, A, B, a, r, mag):
+        Wa = W + s(a, r) * (B @ A)
+        return X @ ((mag / np.sqrt(np.sum(W * W, axis=1)))[:, None] * Wa).T
+
+    def dora_column_norms(W, X, A, B, a, r, mag):
+        Wa = W + s(a, r) * (B @ A)
+        return X @ (mag[:, None] * Wa / np.sqrt(np.sum(Wa * Wa, axis=0))[None, :]).T
+
+    assert check_dora_brute(dora_no_adapter_in_norm) > 1e-3
+    assert check_dora_brute(dora_column_norms) > 1e-3
 
     # quantizer mutants: swapped nibbles and a 255-level second stage
     L = O.nf4_levels()
