@@ -602,6 +602,27 @@ def extra_rows(q, torch, S, dev, peaks, args):
                                     "roof_frac": t_roof / (med * 1e-6), "adapter_MB": n_ad * r_ad * 8192 * 2 / 1e6}
     del wl, X, ids, tab, H, ws
 
+    # ---- DoRA forward on the q_proj shape (4096^2, r = 16, T = 4096): row norms of W^ + sBA
+    # (recomputed every call) + the fused forward with the m / n column scale
+    c2d = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
+    case = S.make_layer(c2d["d_out"], c2d["d_in"], c2d["r"], c2d["alpha"], c2d["T"], dtype="bf16",
+                        seed=17, with_grad=False)
+    wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(4)]
+    X = torch.from_numpy(case.X).to(dev).to(bf)
+    A = torch.from_numpy(case.A).to(dev).to(bf)
+    B = torch.from_numpy(case.B).to(dev).to(bf)
+    mag = torch.ones(c2d["d_out"], dtype=torch.float32, device=dev)
+    H = torch.empty((c2d["T"], c2d["d_out"]), dtype=bf, device=dev)
+    ws = torch.empty(q.workspace_bytes(q.OP_DORA_FWD, q.BF16, c2d["T"], c2d["d_out"], c2d["d_in"], c2d["r"]),
+                     dtype=torch.uint8, device=dev)
+    calls = [(lambda w=w: q.qlora_dora_fwd(w, X, A, B, c2d["alpha"], mag, H=H, save_u=False, ws=ws))
+             for w in wl]
+    med, _ = _graph_time(torch, calls, reps=10)
+    fl = flops_fwd(c2d["T"], c2d["d_out"], c2d["d_in"], c2d["r"]) + 2 * c2d["d_out"] * c2d["r"] * c2d["d_in"]
+    out["dora_fwd_4096x4096_r16_T4096"] = {"fwd_us": med, "tflops": fl / (med * 1e-6) / 1e12,
+                                           "tc_frac": fl / (med * 1e-6) / 1e12 / tc}
+    del wl, X, A, B, mag, H, ws, case
+
     # ---- AdamW step over the adapters of a 32-layer d = 4096 model with rank 16 on q, k, v, o:
     # 32 * 4 * 16 * (4096 + 4096) = 16.8 M parameters, bf16 params + fp32 master, m, v, grad
     # (30 bytes per parameter, 503 MB > L2)

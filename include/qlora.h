@@ -56,7 +56,7 @@ typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 
 typedef enum {
     QLORA_OP_FWD = 0, QLORA_OP_BWD = 1, QLORA_OP_FWD_BATCHED = 2, QLORA_OP_MERGE = 3,
-    QLORA_OP_FWD_MULTI = 4
+    QLORA_OP_FWD_MULTI = 4, QLORA_OP_DORA_FWD = 5
 } qlora_op;
 
 /* Stored NF4 weight.  Block size 64 and group size 256 are fixed.
@@ -211,6 +211,27 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4* w, const void* X, int64_t T
                                     const void* const* A_ptrs, const void* const* B_ptrs,
                                     const int32_t* ranks, const float* scales, int32_t r_max,
                                     void* H, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* DoRA (bf16): one magnitude per output row, each row of the adapted weight W + s B A divided
+ * by its Euclidean norm ([CH] "Choosing what to adapt": a magnitude vector of size d_out trained
+ * directly, the low-rank update on the direction; [MF] "Advanced Variants: DoRA and LoRA+",
+ * W = m (V + dW) / ||V + dW||; reading R24).  With per-row norms n_j = ||(W^ + s B A)[j, :]||_2:
+ *   H[t, j] = (m_j / n_j) (X[t] W^T + s U[t] B^T)[j]        (a row of norm 0 gives 0)
+ * W^ is the bf16 decode.  magnitude: device fp32 [d_out].  The norms are recomputed every call
+ * (they depend on A, B) by the tensor-core merge tile in a row-norm mode, then the large-T
+ * fused forward applies m / n to each output column before rounding.  U_save as in
+ * qlora_linear_fwd.  ws >= qlora_workspace_bytes(QLORA_OP_DORA_FWD, QLORA_BF16, T, d_out,
+ * d_in, r).  Forward only.                                                                    */
+qlora_status qlora_dora_fwd(const qlora_nf4* w, const void* X, int64_t T, const void* A,
+                            const void* B, int32_t r, float alpha, const float* magnitude,
+                            void* H, void* U_save, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* The DoRA row norms n_j = ||(W^ + (alpha/r) B A)[j, :]||_2 (bf16 adapters, W^ the bf16 decode)
+ * into norms (device fp32 [d_out]); DoRA initialises the magnitude to them.  ws holds at least
+ * d_out * (d_in / 64) floats.                                                                 */
+qlora_status qlora_dora_row_norms(const qlora_nf4* w, const void* A, const void* B, int32_t r,
+                                  float alpha, float* norms, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream);
 
 /* Size of the device scratch array behind qlora_linear_fwd_noalloc (bytes per GPU). */
 #define QLORA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

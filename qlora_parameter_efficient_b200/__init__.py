@@ -22,12 +22,13 @@ QLORA_OK = 0
 STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",
           3: "QLORA_ERR_CUDA", 4: "QLORA_ERR_TIMEOUT", 5: "QLORA_ERR_DEVICE"}
 F32, BF16 = 0, 1
-OP_FWD, OP_BWD, OP_FWD_BATCHED, OP_MERGE, OP_FWD_MULTI = 0, 1, 2, 3, 4
+OP_FWD, OP_BWD, OP_FWD_BATCHED, OP_MERGE, OP_FWD_MULTI, OP_DORA_FWD = 0, 1, 2, 3, 4, 5
 
 # Every symbol include/qlora.h declares.
 EXPORTS = ["qlora_nf4_sizes", "qlora_nf4_levels", "nf4_quantize", "nf4_dequantize",
            "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "lora_merge",
-           "qlora_linear_bwd_ex", "qlora_adamw_step", "qlora_prefetch",
+           "qlora_linear_bwd_ex", "qlora_adamw_step", "qlora_prefetch", "qlora_dora_fwd",
+           "qlora_dora_row_norms",
            "qlora_linear_fwd_batched", "qlora_linear_fwd_multi", "qlora_linear_fwd_noalloc",
            "qlora_get_device_error",
            "qlora_selftest_wait_timeout", "qlora_set_gemm_events", "qlora_launch_count",
@@ -78,6 +79,8 @@ def load() -> ctypes.CDLL:
         "qlora_adamw_step": ([vp, ctypes.c_int, vp, vp, vp, vp, i64, i32, f32, f32, f32, f32, f32, f32, vp],
                              ctypes.c_int),
         "qlora_prefetch": ([vp, sz, i32, vp], ctypes.c_int),
+        "qlora_dora_fwd": ([pnf4, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_dora_row_norms": ([pnf4, vp, vp, i32, f32, vp, vp, sz, vp], ctypes.c_int),
         "qlora_linear_fwd_noalloc": ([pnf4, vp, i64, vp, vp, i32, f32, ctypes.c_int, vp, vp, vp], ctypes.c_int),
         "qlora_get_device_error": ([vp], ctypes.c_int),
         "qlora_selftest_wait_timeout": ([ctypes.c_uint64, vp], ctypes.c_int),
@@ -252,6 +255,40 @@ def adamw_step(param, grad, m, v, step, lr, beta1=0.9, beta2=0.999, eps=1e-8, we
         int(step), float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
         float(grad_scale), _stream(stream)))
     return param
+
+
+def dora_row_norms(w: NF4Weight, A, B, alpha, norms=None, ws=None, stream=None):
+    """n_j = ||(W^ + (alpha/r) B A)[j, :]||_2 for every output row (fp32 [d_out])."""
+    torch = _torch()
+    _contig(A, B, norms)
+    r = A.shape[0]
+    if norms is None:
+        norms = torch.empty(w.d_out, dtype=torch.float32, device=A.device)
+    if ws is None:
+        ws = torch.empty(w.d_out * (w.d_in // 64) * 4, dtype=torch.uint8, device=A.device)
+    _check("qlora_dora_row_norms", load().qlora_dora_row_norms(
+        ctypes.byref(w._c()), _ptr(A), _ptr(B), r, float(alpha), _ptr(norms), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return norms
+
+
+def qlora_dora_fwd(w: NF4Weight, X, A, B, alpha, magnitude, H=None, U_save=None, save_u=True,
+                   ws=None, stream=None):
+    """DoRA forward (bf16): H = (m / ||W^ + sBA||_rows) * (X W^T + s U B^T); returns (H, U)."""
+    torch = _torch()
+    _contig(X, A, B, magnitude, H, U_save)
+    T = X.shape[0]
+    r = A.shape[0]
+    if H is None:
+        H = torch.empty((T, w.d_out), dtype=X.dtype, device=X.device)
+    if U_save is None and save_u:
+        U_save = torch.empty((T, r), dtype=X.dtype, device=X.device)
+    ws = _ws(OP_DORA_FWD, BF16, T, w.d_out, w.d_in, r, X.device, ws)
+    c = w._c()
+    _check("qlora_dora_fwd", load().qlora_dora_fwd(
+        ctypes.byref(c), _ptr(X), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(magnitude), _ptr(H),
+        _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream)))
+    return H, U_save
 
 
 def prefetch(ptr: int, nbytes: int, to_device: bool, stream=None):

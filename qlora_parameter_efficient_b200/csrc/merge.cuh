@@ -39,14 +39,18 @@ struct MergeSmem {
     }
 };
 
-template <typename TOut>
+// NORM = true (DoRA): the tile's values are not stored; instead out_norm[row * (d_in / 64) +
+// tile column] receives the sum of squares of the row's 64 values in the tile (fp32, summed
+// in a fixed order), TOut giving the decode's rounding (bf16).
+template <typename TOut, bool NORM = false>
 __global__ void __launch_bounds__(kMergeThreads, 4) k_merge_tc(const uint8_t* __restrict__ codes,
                                                             const uint8_t* __restrict__ absmax_q,
                                                             const float* __restrict__ c2,
                                                             int64_t d_out, int64_t d_in,
                                                             const __nv_bfloat16* __restrict__ A,
                                                             const __nv_bfloat16* __restrict__ B,
-                                                            int r, float s, TOut* __restrict__ out) {
+                                                            int r, float s, TOut* __restrict__ out,
+                                                            float* __restrict__ out_norm = nullptr) {
     extern __shared__ __align__(16) uint8_t mtc_smem[];
     const int rp = (r + 15) & ~15;
     const int ldb = rp + 8;                      // bf16 elements per staged B row
@@ -143,6 +147,7 @@ __global__ void __launch_bounds__(kMergeThreads, 4) k_merge_tc(const uint8_t* __
 
     // epilogue: accumulator (row g [+8], columns 2t, 2t+1) of each fragment
     const int g = lane >> 2, t = lane & 3;
+    float sq[2][2] = {{0.f, 0.f}, {0.f, 0.f}};      // NORM: per (mi, h) row of the thread
 #pragma unroll
     for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll
@@ -159,6 +164,11 @@ __global__ void __launch_bounds__(kMergeThreads, 4) k_merge_tc(const uint8_t* __
                     w1 = __bfloat162float(__float2bfloat16_rn(w1));
                 }
                 const float v0 = w0 + s * acc[mi][ni][2 * h], v1 = w1 + s * acc[mi][ni][2 * h + 1];
+                if constexpr (NORM) {
+                    sq[mi][h] = fmaf(v0, v0, sq[mi][h]);
+                    sq[mi][h] = fmaf(v1, v1, sq[mi][h]);
+                    continue;
+                }
                 if constexpr (sizeof(TOut) == 2) {
                     *reinterpret_cast<__nv_bfloat162*>(sO + rr * kMergeLdo + cc) = __floats2bfloat162_rn(v0, v1);
                 } else {
@@ -166,6 +176,23 @@ __global__ void __launch_bounds__(kMergeThreads, 4) k_merge_tc(const uint8_t* __
                 }
             }
         }
+    }
+    if constexpr (NORM) {
+        // the 4 threads of a row (t = 0..3), then the 2 warps of a row group (32 columns each)
+        float* s_sq = reinterpret_cast<float*>(sO);                   // [128][2]
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float x = sq[mi][h];
+                x += __shfl_xor_sync(0xffffffffu, x, 1);
+                x += __shfl_xor_sync(0xffffffffu, x, 2);
+                if (t == 0) s_sq[(wr + 16 * mi + g + 8 * h) * 2 + (warp & 1)] = x;
+            }
+        __syncthreads();
+        if (tid < 128 && row0 + tid < d_out)
+            out_norm[(row0 + tid) * (d_in / 64) + blockIdx.x] = s_sq[tid * 2] + s_sq[tid * 2 + 1];
+        return;
     }
     __syncthreads();
     // whole rows of the tile, 16 bytes per thread per store
@@ -177,6 +204,21 @@ __global__ void __launch_bounds__(kMergeThreads, 4) k_merge_tc(const uint8_t* __
         if (gr < d_out)
             *reinterpret_cast<uint4*>(out + gr * d_in + gc) =
                 *reinterpret_cast<const uint4*>(sO + rr * kMergeLdo + v * kVec);
+    }
+}
+
+// DoRA column scale of the layer output: scale[j] = magnitude[j] / sqrt(sum_c partial[j][c])
+// (partials from k_merge_tc<., true>, summed in column order); magnitude == nullptr writes the
+// norms themselves.  A row of norm 0 has no direction: its scale is 0.
+__global__ void k_dora_scale(const float* __restrict__ partial, int64_t d_out, int n_cb,
+                             const float* __restrict__ magnitude, float* __restrict__ out) {
+    griddep_enter();
+    for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < d_out;
+         j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float acc = 0.f;
+        for (int c = 0; c < n_cb; ++c) acc += partial[j * n_cb + c];
+        const float nrm = sqrtf(acc);
+        out[j] = magnitude ? (nrm > 0.f ? magnitude[j] / nrm : 0.f) : nrm;
     }
 }
 

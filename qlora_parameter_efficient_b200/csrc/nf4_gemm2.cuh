@@ -127,6 +127,7 @@ struct Gemm2Args {
     int nf4_bpr;           // d_in / 64
     __nv_bfloat16* out;
     int64_t ld_out;
+    const float* col_scale;  // [N] factor applied to output column n before rounding, or NULL
     int split_tiles;       // trailing tiles split in two along K (0 = none)
     float* part;           // [split_tiles][2 ranks][4 warps][2 halves][2048 float4] fp32 partials
     int* cnt;              // [split_tiles][2 ranks][4 warps] tickets, zero at launch
@@ -413,6 +414,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
                 if (grow < args.M) {
                     const int gc = gc0 + c0;
                     __nv_bfloat16* o = args.out + grow * args.ld_out + gc;
+                    if (args.col_scale != nullptr) {
+                        // per-output-column factor (DoRA's m / ||W + sBA|| row norms)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (gc + e < args.N)
+                                r[e] = __float_as_uint(__uint_as_float(r[e]) * __ldg(args.col_scale + gc + e));
+                    }
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
                         if (gc + 8 * g < args.N) {

@@ -219,10 +219,12 @@ struct Plan {
     size_t seg_cnt = 0, seg_start = 0, seg_cursor = 0, seg_ntiles = 0, seg_tiles = 0, seg_perm = 0,
            seg_u = 0;
     int seg_ldu = 0, seg_max_tiles = 0;
+    size_t dora_part = 0, dora_scale = 0;   // DoRA row-norm partials and column scale
     size_t total = 0;
 };
 
 Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in, int r) {
+    // (QLORA_OP_DORA_FWD: the forward's workspace plus the DoRA row norms)
     Plan p;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -246,7 +248,9 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
         p.total = off;
         return p;
     }
-    if (op == QLORA_OP_FWD && dtype == QLORA_BF16 && make_small_plan(T, d_out, d_in).ok) {
+    const bool dora = op == QLORA_OP_DORA_FWD;
+    if (dora) op = QLORA_OP_FWD;          // the forward's plan, never the decode-size path
+    if (!dora && op == QLORA_OP_FWD && dtype == QLORA_BF16 && make_small_plan(T, d_out, d_in).ok) {
         p.small = true;
         p.s_us = take(static_cast<size_t>(T) * r * 4);
         p.total = off;
@@ -286,6 +290,10 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
             p.uf = take(static_cast<size_t>(T) * r * 4);
             if (op == QLORA_OP_BWD) p.gf = take(static_cast<size_t>(T) * r * 4);
         }
+    }
+    if (dora) {
+        p.dora_part = take(static_cast<size_t>(d_out) * (d_in / 64) * 4);
+        p.dora_scale = take(static_cast<size_t>(d_out) * 4);
     }
     p.total = off;
     return p;
@@ -394,7 +402,7 @@ qlora_status skinny_gemm(bool a_mn, bool b_mn, int RP, int n_valid, const CUtens
 // when the TMA zero-fills the rank padding out of bounds).
 qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, const void* ext_a,
                       const void* ext_b, int RP, int r_used, int ext_b_rank, void* out,
-                      void* g2ws, int* err, cudaStream_t st) {
+                      void* g2ws, int* err, cudaStream_t st, const float* col_scale = nullptr) {
     const int64_t d_out = w->d_out, d_in = w->d_in;
     CUtensorMap ta, tc, tax, tbx;
     const int64_t K = dx ? d_out : d_in;
@@ -411,6 +419,7 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
         tbx = ta;
     }
     Gemm2Args g{};
+    g.col_scale = col_scale;
     g.M = static_cast<int>(T);
     g.N = static_cast<int>(N);
     g.k_steps = static_cast<int>(cdiv(K, 64));
@@ -634,6 +643,63 @@ qlora_status compute_u_bf16(const void* X, int64_t T, int64_t d_in, const void* 
     return QLORA_OK;
 }
 
+// The large-T bf16 forward: U pre-pass, then the fused NF4 GEMM with the adapter K-extension;
+// col_scale (nullable) multiplies output column n before rounding (DoRA).
+qlora_status fwd_bf16_large(const qlora_nf4* w, const void* X, int64_t T, const void* A,
+                            const void* B, int32_t r, float s, void* H, void* U_save,
+                            const Plan& p, void* ws, int* err, cudaStream_t stream,
+                            const float* col_scale) {
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    {
+        const int RP = p.RP;
+        auto* a_pad = at<__nv_bfloat16>(ws, p.a_pad);
+        auto* b_pad = at<__nv_bfloat16>(ws, p.b_pad);
+        auto* u_spad = at<__nv_bfloat16>(ws, p.u_spad);
+        auto* part = at<float>(ws, p.part);
+        // With r a multiple of 8 every row of A, B is a whole number of 16-byte units, so the
+        // tensor maps address the caller's tensors and zero-fill the rank padding out of
+        // bounds; otherwise zero-padded copies are made.
+        const bool direct = r % 8 == 0;
+        const void* a_src = A;
+        const void* b_src = B;
+        int a_rows = r, b_ld = r;
+        if (!direct) {
+            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A), r, d_in, d_in, a_pad, RP, d_in, 0, d_in, stream));
+            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
+            a_src = a_pad;
+            b_src = b_pad;
+            a_rows = b_ld = RP;
+        }
+        QL_TRY(compute_u_bf16(X, T, d_in, a_src, a_rows, RP, r, s, p.split_u, part,
+                              static_cast<__nv_bfloat16*>(U_save), nullptr, u_spad, err, stream));
+        return nf4_gemm(false, w, X, T, u_spad, b_src, RP, r, b_ld, H, at<void>(ws, p.g2), err, stream,
+                        col_scale);
+    }
+}
+
+// DoRA: scale[j] = magnitude[j] / ||(W^ + s B A)[j, :]|| (or the norms when magnitude is NULL),
+// from the tensor-core merge tile in its row-norm mode and one reduction over the 64-column
+// tiles.
+qlora_status dora_scale(const qlora_nf4* w, const void* A, const void* B, int32_t r, float s,
+                        const float* magnitude, float* partial, float* out, cudaStream_t stream) {
+    using bf = __nv_bfloat16;
+    auto kern = k_merge_tc<bf, true>;
+    const int rp = (r + 15) & ~15;
+    const int tsmem = MergeSmem::bytes(rp, 2);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tsmem) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    dim3 tgrid(static_cast<unsigned>(w->d_in / 64), static_cast<unsigned>(cdiv(w->d_out, 128)));
+    kern<<<tgrid, kMergeThreads, tsmem, stream>>>(w->codes, w->absmax_q, w->c2, w->d_out, w->d_in,
+                                                   static_cast<const bf*>(A), static_cast<const bf*>(B),
+                                                   r, s, nullptr, partial);
+    QL_LAUNCH_CHECK();
+    if (launch_pdl(k_dora_scale, grid1d(w->d_out), dim3(256), 0, stream, partial, w->d_out,
+                   static_cast<int>(w->d_in / 64), magnitude, out) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
 }  // namespace
 
 // ======================================================================= C ABI
@@ -674,8 +740,8 @@ qlora_status qlora_nf4_levels(float* out) {
 
 size_t qlora_workspace_bytes(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in,
                              int32_t r_total) {
-    if (op < QLORA_OP_FWD || op > QLORA_OP_FWD_MULTI) return 0;
-    if (op == QLORA_OP_FWD_MULTI && dtype != QLORA_BF16) return 0;
+    if (op < QLORA_OP_FWD || op > QLORA_OP_DORA_FWD) return 0;
+    if ((op == QLORA_OP_FWD_MULTI || op == QLORA_OP_DORA_FWD) && dtype != QLORA_BF16) return 0;
     if ((dtype != QLORA_BF16 && dtype != QLORA_F32) || T < 1 || d_out < 1 || d_in < 64 ||
         r_total < 1 || r_total > 128)
         return 0;
@@ -734,30 +800,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T, cons
     const float s = alpha / static_cast<float>(r);
     if (p.small)
         return small_fwd(w, X, T, A, B, r, s, H, U_save, p, ws, err, stream);
-    if (dtype == QLORA_BF16) {
-        const int RP = p.RP;
-        auto* a_pad = at<__nv_bfloat16>(ws, p.a_pad);
-        auto* b_pad = at<__nv_bfloat16>(ws, p.b_pad);
-        auto* u_spad = at<__nv_bfloat16>(ws, p.u_spad);
-        auto* part = at<float>(ws, p.part);
-        // With r a multiple of 8 every row of A, B is a whole number of 16-byte units, so the
-        // tensor maps address the caller's tensors and zero-fill the rank padding out of
-        // bounds; otherwise zero-padded copies are made.
-        const bool direct = r % 8 == 0;
-        const void* a_src = A;
-        const void* b_src = B;
-        int a_rows = r, b_ld = r;
-        if (!direct) {
-            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A), r, d_in, d_in, a_pad, RP, d_in, 0, d_in, stream));
-            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
-            a_src = a_pad;
-            b_src = b_pad;
-            a_rows = b_ld = RP;
-        }
-        QL_TRY(compute_u_bf16(X, T, d_in, a_src, a_rows, RP, r, s, p.split_u, part,
-                              static_cast<__nv_bfloat16*>(U_save), nullptr, u_spad, err, stream));
-        return nf4_gemm(false, w, X, T, u_spad, b_src, RP, r, b_ld, H, at<void>(ws, p.g2), err, stream);
-    }
+    if (dtype == QLORA_BF16) return fwd_bf16_large(w, X, T, A, B, r, s, H, U_save, p, ws, err, stream, nullptr);
     // exact fp32 path
     float* w32 = at<float>(ws, p.w32);
     float* U = U_save ? static_cast<float*>(U_save) : at<float>(ws, p.uf);
@@ -767,6 +810,34 @@ qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T, cons
     QL_TRY(sgemm(stream, T, d_out, d_in, 1.f, Xf, d_in, false, w32, d_in, true, 0.f, static_cast<float*>(H), d_out));
     return sgemm(stream, T, d_out, r, s, U, r, false, static_cast<const float*>(B), r, true, 1.f,
                  static_cast<float*>(H), d_out);
+}
+
+qlora_status qlora_dora_row_norms(const qlora_nf4* w, const void* A, const void* B, int32_t r,
+                                  float alpha, float* norms, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream) {
+    QL_TRY(check_layer(w, 1, r, QLORA_BF16));
+    if (!aligned16(A) || !aligned16(B) || !norms) return QLORA_ERR_INVALID_ARG;
+    const size_t need = static_cast<size_t>(w->d_out) * (w->d_in / 64) * 4;
+    QL_TRY(check_ws(ws, ws_bytes, need));
+    return dora_scale(w, A, B, r, alpha / static_cast<float>(r), nullptr, static_cast<float*>(ws), norms,
+                      stream);
+}
+
+qlora_status qlora_dora_fwd(const qlora_nf4* w, const void* X, int64_t T, const void* A,
+                            const void* B, int32_t r, float alpha, const float* magnitude,
+                            void* H, void* U_save, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    QL_TRY(check_layer(w, T, r, QLORA_BF16));
+    if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) || !magnitude ||
+        !aligned16_or_null(U_save))
+        return QLORA_ERR_INVALID_ARG;
+    const Plan p = make_plan(QLORA_OP_DORA_FWD, QLORA_BF16, T, w->d_out, w->d_in, r);
+    QL_TRY(check_ws(ws, ws_bytes, p.total));
+    int* err = nullptr;
+    QL_TRY(err_word(&err));
+    const float s = alpha / static_cast<float>(r);
+    float* scale = at<float>(ws, p.dora_scale);
+    QL_TRY(dora_scale(w, A, B, r, s, magnitude, at<float>(ws, p.dora_part), scale, stream));
+    return fwd_bf16_large(w, X, T, A, B, r, s, H, U_save, p, ws, err, stream, scale);
 }
 
 qlora_status qlora_linear_bwd_ex(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
@@ -961,7 +1032,7 @@ qlora_status lora_merge(const qlora_nf4* w, const void* A, const void* B, int32_
         dim3 tgrid(static_cast<unsigned>(w->d_in / 64), static_cast<unsigned>(cdiv(w->d_out, 128)));
         kern<<<tgrid, kMergeThreads, tsmem, stream>>>(w->codes, w->absmax_q, w->c2, w->d_out, w->d_in,
                                                        static_cast<const bf*>(A), static_cast<const bf*>(B),
-                                                       r, s, o);
+                                                       r, s, o, nullptr);
         QL_LAUNCH_CHECK();
         return QLORA_OK;
     };

@@ -536,3 +536,57 @@ def test_adamw_state_in_unified_memory(q):
         torch.cuda.synchronize()
         for p in bufs:
             rt.cudaFree(p)
+
+
+# ------------------------------------------------------------------ DoRA (R24)
+
+
+@pytest.mark.parametrize("d_out,d_in,r", [(200, 192, 5), (264, 320, 16), (256, 1088, 128)])
+def test_dora_row_norms(q, d_out, d_in, r):
+    import torch
+    case = S.make_layer(d_out, d_in, r, 2.0 * r, 1, dtype="bf16", seed=d_out + r, with_grad=False)
+    w, oc = quantize_both(q, case.W0)
+    n = q.dora_row_norms(w, dev(case.A, "bf16"), dev(case.B, "bf16"), 2.0 * r)
+    torch.cuda.synchronize()
+    ref = O.dora_row_norms(oracle_weight(oc, d_out, d_in, "bf16"), case.A, case.B, 2.0 * r, r)
+    assert rel_fro(host(n), ref) <= 1e-5
+
+
+def run_dora(q, case, rows=None, seed=0):
+    import torch
+    w, oc = quantize_both(q, case.W0)
+    Wh = oracle_weight(oc, case.d_out, case.d_in, "bf16")
+    mag = np.random.default_rng(seed).uniform(0.5, 2.0, case.d_out).astype(np.float32)
+    H, U = q.qlora_dora_fwd(w, dev(case.X, "bf16"), dev(case.A, "bf16"), dev(case.B, "bf16"),
+                            case.alpha, torch.from_numpy(mag).cuda())
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    sel = slice(None) if rows is None else rows
+    ref = O.dora_forward(Wh, case.X[sel], case.A, case.B, case.alpha, case.r, mag)
+    assert rel_fro(host(H)[sel], ref) <= TOL["bf16"]
+    return w, H
+
+
+@pytest.mark.parametrize("d_out,d_in,r,T", [(256, 256, 8, 64), (200, 192, 5, 77), (520, 320, 16, 300),
+                                            (136, 256, 100, 3)])
+def test_dora_forward(q, d_out, d_in, r, T):
+    run_dora(q, S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_in + T, with_grad=False))
+
+
+def test_dora_forward_q_proj_sampled_rows(q):
+    case = S.make_layer(**S.CONFIGS["q_proj_4096x4096_r16_T4096"], seed=3, with_grad=False)
+    rows = np.sort(np.random.default_rng(5).choice(case.T, 256, replace=False))
+    run_dora(q, case, rows=rows)
+
+
+def test_dora_magnitude_at_norms_is_lora(q):
+    """DoRA's initialisation (m = the row norms) reproduces the LoRA layer."""
+    import torch
+    case = S.make_layer(384, 256, 16, 32.0, 96, dtype="bf16", seed=8, with_grad=False)
+    w, _ = quantize_both(q, case.W0)
+    X, A, B = dev(case.X, "bf16"), dev(case.A, "bf16"), dev(case.B, "bf16")
+    mag = q.dora_row_norms(w, A, B, case.alpha)
+    Hd, _ = q.qlora_dora_fwd(w, X, A, B, case.alpha, mag)
+    Hl, _ = q.qlora_linear_fwd(w, X, A, B, case.alpha)
+    torch.cuda.synchronize()
+    assert rel_fro(host(Hd), host(Hl).astype(np.float64)) <= 4e-3
