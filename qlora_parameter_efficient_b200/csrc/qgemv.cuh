@@ -503,10 +503,14 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 // so that they fit beside the stream kernel, which it overlaps through programmatic dependent
 // launch: warp w of CTA b computes adapter row j = 8b + w for the tokens two at a time, each
 // pass over a 4096-element chunk of K with all of its loads in flight at once.
+// u_spad (nullable): bf16(s U) [T, ldp] for a tensor-core K-extension (columns >= r are left
+// as they are: the caller zeroes them).
 __global__ void __launch_bounds__(256) k_small_u(const __nv_bfloat16* __restrict__ X, int T,
                                                  int d_in, const __nv_bfloat16* __restrict__ A,
                                                  int r, float s, float* __restrict__ us,
-                                                 __nv_bfloat16* __restrict__ u_save) {
+                                                 __nv_bfloat16* __restrict__ u_save,
+                                                 __nv_bfloat16* __restrict__ u_spad = nullptr,
+                                                 int ldp = 0) {
     griddep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int j = blockIdx.x * 8 + warp;
@@ -553,9 +557,11 @@ __global__ void __launch_bounds__(256) k_small_u(const __nv_bfloat16* __restrict
         if (lane == 0) {
             us[static_cast<int64_t>(t0) * r + j] = s * acc0;
             if (u_save) u_save[static_cast<int64_t>(t0) * r + j] = __float2bfloat16_rn(acc0);
+            if (u_spad) u_spad[static_cast<int64_t>(t0) * ldp + j] = __float2bfloat16_rn(s * acc0);
             if (two) {
                 us[static_cast<int64_t>(t0 + 1) * r + j] = s * acc1;
                 if (u_save) u_save[static_cast<int64_t>(t0 + 1) * r + j] = __float2bfloat16_rn(acc1);
+                if (u_spad) u_spad[static_cast<int64_t>(t0 + 1) * ldp + j] = __float2bfloat16_rn(s * acc1);
             }
         }
     }

@@ -31,6 +31,7 @@ constexpr int kMaxDevices = 64;
 constexpr int kSmsForSplit = 148;         // split-K is sized for a B200's 148 SMs
 constexpr uint64_t kWaitNs = 4000000000ull;
 constexpr int kTmaStages = 4;
+constexpr int kNf4Stages = 4;          // the mid-size NF4 GEMM: 4 x 56 KB stages
 
 std::atomic<uint64_t> g_launches{0};
 int* g_err_ptr[kMaxDevices] = {};
@@ -173,6 +174,26 @@ int pad_rank(int r) { return r <= 64 ? 64 : 128; }
 // Decode-size forward (bf16, T <= 16, d_in a multiple of 256): clusters of C CTAs own tiles of
 // M rows, the C ranks split K.  (C, M) is picked at launch by balanced cost.
 constexpr int kSmallT = 16;   // above this the large-T path is faster (measured)
+// Mid-size forward (bf16, 8 < T <= kMidT, or T <= 8 when the decode-size kernel does not
+// apply): split-K NF4 GEMM over all SMs with fp32 partials, then one finalize with the adapter.
+constexpr int64_t kMidT = 64;
+struct MidPlan {
+    bool ok = false;
+    int split = 1, n_tiles = 1;
+};
+MidPlan make_mid_plan(int64_t T, int64_t d_out, int64_t d_in) {
+    MidPlan mp;
+    if (T < 1 || T > kMidT) return mp;
+    mp.n_tiles = static_cast<int>(cdiv(d_out, 256));
+    const int64_t k_steps = d_in / 64;
+    int64_t s = std::max<int64_t>(1, kSmsForSplit / mp.n_tiles);   // one CTA per SM, one wave
+    s = std::min<int64_t>(s, std::max<int64_t>(1, k_steps / 2));
+    const int64_t per = cdiv(k_steps, s);
+    mp.split = static_cast<int>(cdiv(k_steps, per));                // no empty splits
+    mp.ok = true;
+    return mp;
+}
+
 struct SmallPlan {
     bool ok = false;
     int nt8 = 1, kt = 0;
@@ -182,6 +203,7 @@ SmallPlan make_small_plan(int64_t T, int64_t d_out, int64_t d_in) {
     (void)d_out;
     if (T < 1 || T > kSmallT) return sp;
     sp.nt8 = T <= 8 ? 1 : 2;
+    if (sp.nt8 == 2) return sp;          // 9..16 tokens: the mid-size path is faster
     sp.kt = static_cast<int>(d_in / 64);
     sp.ok = sp.kt % 4 == 0;
     return sp;
@@ -211,6 +233,9 @@ struct Plan {
     int RP = 0;
     bool small = false;
     size_t s_us = 0;
+    bool mid = false;
+    size_t mid_part = 0;
+    int mid_split = 1;
     int split_u = 1, split_g = 1, split_da = 1, split_db = 1;
     size_t a_pad = 0, b_pad = 0, u_spad = 0, u_pad = 0, g_spad = 0, part = 0;
     size_t w32 = 0, uf = 0, gf = 0;
@@ -255,6 +280,20 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
         p.s_us = take(static_cast<size_t>(T) * r * 4);
         p.total = off;
         return p;
+    }
+    if (!dora && op == QLORA_OP_FWD && dtype == QLORA_BF16) {
+        const MidPlan mp = make_mid_plan(T, d_out, d_in);
+        if (mp.ok) {
+            p.mid = true;
+            p.mid_split = mp.split;
+            p.RP = pad_rank(r);
+            p.s_us = take(static_cast<size_t>(T) * r * 4);
+            p.u_spad = take(static_cast<size_t>(T) * p.RP * 2);
+            p.b_pad = take(static_cast<size_t>(d_out) * p.RP * 2);
+            p.mid_part = take(static_cast<size_t>(mp.split) * T * d_out * 4);
+            p.total = off;
+            return p;
+        }
     }
     if (dtype == QLORA_BF16) {
         p.RP = pad_rank(r);
@@ -643,6 +682,59 @@ qlora_status compute_u_bf16(const void* X, int64_t T, int64_t d_in, const void* 
     return QLORA_OK;
 }
 
+// Mid-size forward: the U pre-pass (few CTAs) runs beside the split-K NF4 GEMM, which waits
+// for it only before exiting; the finalize then sums the partials and adds s U B^T.
+qlora_status mid_fwd(const qlora_nf4* w, const void* X, int64_t T, const void* A, const void* B,
+                     int r, float s, void* H, void* U_save, const Plan& p, void* ws, int* err,
+                     cudaStream_t st) {
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    const MidPlan mp = make_mid_plan(T, d_out, d_in);
+    const int RP = p.RP;
+    float* us = at<float>(ws, p.s_us);
+    float* part = at<float>(ws, p.mid_part);
+    auto* u_spad = at<__nv_bfloat16>(ws, p.u_spad);
+    // the adapter's B as the extension's B operand: the caller's B when its rows are whole
+    // 16-byte units (the map zero-fills the rank padding), else a zero-padded copy
+    const void* b_src = B;
+    int b_ld = r;
+    if (r % 8 != 0) {
+        auto* b_pad = at<__nv_bfloat16>(ws, p.b_pad);
+        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, st));
+        b_src = b_pad;
+        b_ld = RP;
+    }
+    if (cudaMemsetAsync(u_spad, 0, static_cast<size_t>(T) * RP * 2, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    k_small_u<<<static_cast<unsigned>(cdiv(r, 8)), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(X), static_cast<int>(T), static_cast<int>(d_in),
+        static_cast<const __nv_bfloat16*>(A), r, s, us, static_cast<__nv_bfloat16*>(U_save), u_spad, RP);
+    QL_LAUNCH_CHECK();
+    CUtensorMap ta, tc, tax, tbx;
+    QL_TRY(tmap_bf16(&ta, X, T, d_in, d_in, kBM));
+    QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 32, 256));
+    QL_TRY(tmap_bf16(&tax, u_spad, T, RP, RP, kBM));
+    QL_TRY(tmap_bf16(&tbx, b_src, d_out, b_ld, b_ld, 256));
+    GemmArgs g = base_args(static_cast<int>(T), static_cast<int>(d_out), static_cast<int>(d_in / 64), err);
+    g.ext_steps = RP / 64;              // s U B^T as extra K steps of the last split
+    g.ext_k16_last = static_cast<int>(std::min<int64_t>(4, cdiv(r - 64 * (g.ext_steps - 1), 16)));
+    g.split = mp.split;
+    g.absmax_q = w->absmax_q;
+    g.c2 = w->c2;
+    g.nf4_rows = static_cast<int>(d_out);
+    g.nf4_bpr = static_cast<int>(d_in / 64);
+    g.out = part;
+    g.ld_out = d_out;
+    g.split_stride = T * d_out;
+    g.late_wait = 1;    // the main steps read only X and W; the extension waits for k_small_u
+    dim3 grid(static_cast<unsigned>(mp.n_tiles), 1, static_cast<unsigned>(mp.split));
+    QL_TRY((launch_gemm<false, false, kBNf4, 256, kNf4Stages, true>(ta, tc, tax, tbx, g, grid, st, true)));
+    if (launch_pdl(k_finalize_mid, grid1d(T * d_out), dim3(256), 0, st, part, mp.split, T * d_out,
+                   static_cast<__nv_bfloat16*>(H)) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+
 // The large-T bf16 forward: U pre-pass, then the fused NF4 GEMM with the adapter K-extension;
 // col_scale (nullable) multiplies output column n before rounding (DoRA).
 qlora_status fwd_bf16_large(const qlora_nf4* w, const void* X, int64_t T, const void* A,
@@ -800,6 +892,8 @@ qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T, cons
     const float s = alpha / static_cast<float>(r);
     if (p.small)
         return small_fwd(w, X, T, A, B, r, s, H, U_save, p, ws, err, stream);
+    if (p.mid)
+        return mid_fwd(w, X, T, A, B, r, s, H, U_save, p, ws, err, stream);
     if (dtype == QLORA_BF16) return fwd_bf16_large(w, X, T, A, B, r, s, H, U_save, p, ws, err, stream, nullptr);
     // exact fp32 path
     float* w32 = at<float>(ws, p.w32);

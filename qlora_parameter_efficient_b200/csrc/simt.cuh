@@ -191,6 +191,19 @@ __global__ void k_finalize_dB(const float* __restrict__ P, int split, int64_t sp
     }
 }
 
+// Mid-size forward finalize: H = bf16(sum_z P[z]) over the split-K partials in z order (the
+// adapter term is already in the last split's partial).
+__global__ void k_finalize_mid(const float* __restrict__ P, int split, int64_t n_el,
+                               __nv_bfloat16* __restrict__ H) {
+    griddep_enter();
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_el;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float acc = 0.f;
+        for (int z = 0; z < split; ++z) acc += P[z * n_el + i];
+        H[i] = __float2bfloat16_rn(acc);
+    }
+}
+
 // Concatenated adapters of the multi-adapter forward, built in one pass:
 //   a_cat [RP, d_in]:  row j = row (j - off_i) of A_i for the adapter i holding column j, 0 for j >= R
 //   b_cat [d_out, RP]: column j = column (j - off_i) of B_i, 0 for j >= R

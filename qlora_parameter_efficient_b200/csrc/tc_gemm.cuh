@@ -44,7 +44,8 @@ struct GemmArgs {
     int k_steps;              // main-loop K steps of 64
     int ext_steps;            // K-extension steps of 64 (0: none)
     int ext_k16_last;         // K=16 MMAs issued in the last extension step (1..4)
-    int split;                // split-K over the main steps (grid.z); requires ext_steps == 0
+    int split;                // split-K over the main steps (grid.z); the extension steps are
+                              // taken by the last split only
     const uint8_t* absmax_q;  // NF4 operand
     const float* c2;
     int nf4_rows;             // d_out of the stored weight
@@ -52,6 +53,10 @@ struct GemmArgs {
     void* out;                // bf16 [M, ld_out] or fp32 partials [split][M][ld_out]
     int64_t ld_out;
     int64_t split_stride;     // elements between fp32 partials
+    // 1: the kernel reads nothing the previous kernel on the stream writes, so it lets the next
+    // kernel launch, starts at once, and waits for the previous one only before it exits (so a
+    // kernel after it still sees both finished).  0: it waits before its first global access.
+    int late_wait;
     int* err;
     uint64_t wait_ns;
 };
@@ -107,7 +112,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int k_begin = z * per;
     const int k_end = min(args.k_steps, k_begin + per);
     const int n_main = max(0, k_end - k_begin);
-    const int n_iters = n_main + args.ext_steps;
+    const int n_iters = n_main + (z == args.split - 1 ? args.ext_steps : 0);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -135,7 +140,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_acc = *tmem_slot;
-    griddep_enter();
+    if (args.late_wait) griddep_launch_dependents();
+    else griddep_enter();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -152,6 +158,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 uint8_t* a = sA + s * L::kABytes;
                 uint8_t* b = sB + s * L::kBBytes;
                 const bool main_step = it < n_main;
+                // late-wait launches: the extension operands come from the previous kernel
+                if (args.late_wait && it == n_main) griddep_wait();
                 const CUtensorMap* ma = main_step ? &tmA : &tmAx;
                 const int kx = main_step ? (k_begin + it) * kBK : (it - n_main) * kBK;
                 uint32_t bytes = L::kABytes;
@@ -353,6 +361,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem_acc, kTmemCols);
     }
+    if (args.late_wait) griddep_wait();
 }
 
 // Bounded-wait self-test: waits on a barrier that nothing arrives on.
