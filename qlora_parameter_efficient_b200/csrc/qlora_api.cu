@@ -1190,12 +1190,21 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4* w, const void* X, int64_t T
     QL_LAUNCH_CHECK();
     // persistent grids over the planned tiles: four resident CTAs of 128 threads per SM
     const unsigned seg_grid = static_cast<unsigned>(std::min<int64_t>(p.seg_max_tiles, 4 * kSmsForSplit));
-    if (launch_pdl(k_seg_shrink, dim3(seg_grid), dim3(128), 0, stream, a) != cudaSuccess)
-        return QLORA_ERR_CUDA;
+    // accumulators for the largest rank's n8 tiles (a rank above r_max is rejected on the device)
+    cudaError_t se;
+    if (r_max <= 16) se = launch_pdl(k_seg_shrink<2, 4>, dim3(seg_grid), dim3(128), 0, stream, a);
+    else if (r_max <= 32) se = launch_pdl(k_seg_shrink<4, 2>, dim3(seg_grid), dim3(128), 0, stream, a);
+    else if (r_max <= 64) se = launch_pdl(k_seg_shrink<8, 2>, dim3(seg_grid), dim3(128), 0, stream, a);
+    else se = launch_pdl(k_seg_shrink<16, 1>, dim3(seg_grid), dim3(128), 0, stream, a);
+    if (se != cudaSuccess) return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     QL_TRY(nf4_gemm(false, w, X, T, nullptr, nullptr, 0, 0, 0, H, at<void>(ws, p.g2), err, stream));
-    if (launch_pdl(k_seg_expand, dim3(seg_grid), dim3(128), 0, stream, a) != cudaSuccess)
-        return QLORA_ERR_CUDA;
+    cudaError_t ee;
+    if (r_max <= 16) ee = launch_pdl(k_seg_expand<1>, dim3(seg_grid), dim3(128), 0, stream, a);
+    else if (r_max <= 32) ee = launch_pdl(k_seg_expand<2>, dim3(seg_grid), dim3(128), 0, stream, a);
+    else if (r_max <= 64) ee = launch_pdl(k_seg_expand<4>, dim3(seg_grid), dim3(128), 0, stream, a);
+    else ee = launch_pdl(k_seg_expand<8>, dim3(seg_grid), dim3(128), 0, stream, a);
+    if (ee != cudaSuccess) return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     return QLORA_OK;
 }

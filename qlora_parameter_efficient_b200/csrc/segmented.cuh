@@ -149,7 +149,9 @@ __device__ __forceinline__ uint32_t ld_pair(const __nv_bfloat16* p, bool ok) {
 // its rows as two 16-byte vectors and uses words 2s and 2s+1 in step s.
 
 // One CTA (4 warps) per tile.  Warp w takes the 64-element K chunks w, w + 4, ...; the four
-// warps' sums are added in warp order.
+// warps' sums are added in warp order.  NT: n8 tiles of the largest rank (ranks up to 8 NT);
+// fewer accumulators let more K chunks' loads be in flight (UNR chunks per iteration).
+template <int NT, int UNR>
 __global__ void __launch_bounds__(128, 4) k_seg_shrink(SegArgs a) {
     griddep_enter();
     __shared__ float s_part[4][kSegTile][129];
@@ -168,13 +170,13 @@ __global__ void __launch_bounds__(128, 4) k_seg_shrink(SegArgs a) {
     const int tok_b = g + 8 < rows ? a.perm[start + g + 8] : -1;
     const __nv_bfloat16* xa = a.X + static_cast<int64_t>(tok_a < 0 ? 0 : tok_a) * a.d_in + 16 * t;
     const __nv_bfloat16* xb = a.X + static_cast<int64_t>(tok_b < 0 ? 0 : tok_b) * a.d_in + 16 * t;
-    float acc[16][4];
+    float acc[NT][4];
 #pragma unroll
-    for (int n = 0; n < 16; ++n)
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
     const uint4 z4 = make_uint4(0, 0, 0, 0);
-#pragma unroll 2
+#pragma unroll UNR
     for (int k0 = 64 * warp; k0 < a.d_in; k0 += 256) {
         uint4 x[4];
         x[0] = tok_a >= 0 ? __ldg(reinterpret_cast<const uint4*>(xa + k0)) : z4;
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(128, 4) k_seg_shrink(SegArgs a) {
         const uint32_t* wa = reinterpret_cast<const uint32_t*>(&x[0]);   // row g: 8 words
         const uint32_t* wb = reinterpret_cast<const uint32_t*>(&x[2]);   // row g + 8
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
+        for (int n = 0; n < NT; ++n) {
             if (n < nt8) {
                 const int j = 8 * n + g;                      // adapter row = output column
                 const __nv_bfloat16* arow = Ai + static_cast<int64_t>(j < r ? j : 0) * a.d_in + k0 + 16 * t;
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(128, 4) k_seg_shrink(SegArgs a) {
     }
     // accumulator (row g [+8], columns 8n + 2t, +1) -> shared, then summed over the warps
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
+    for (int n = 0; n < NT; ++n) {
         if (n < nt8) {
             s_part[warp][g][8 * n + 2 * t] = acc[n][0];
             s_part[warp][g][8 * n + 2 * t + 1] = acc[n][1];
@@ -240,6 +242,8 @@ __device__ __forceinline__ uint2 ld_quad(const __nv_bfloat16* row, int j, int va
 // slots of each 16-step mapped as in the shrink (thread-column t holds elements 4t .. 4t+3).
 // The tile's U fragments stay in registers for all its column blocks, and the H values of the
 // next block are loaded before the current block is stored.
+// KS: K steps of 16 of the largest rank (ranks up to 16 KS).
+template <int KS>
 __global__ void __launch_bounds__(128, 4) k_seg_expand(SegArgs a) {
     griddep_enter();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -254,10 +258,10 @@ __global__ void __launch_bounds__(128, 4) k_seg_expand(SegArgs a) {
         const bool ra = g < rows, rb = g + 8 < rows;
         const int tok_a = ra ? a.perm[start + g] : -1;
         const int tok_b = rb ? a.perm[start + g + 8] : -1;
-        // U fragments of the tile, all K steps (<= 8)
-        uint32_t uf[8][4];
+        // U fragments of the tile, all K steps (<= KS)
+        uint32_t uf[KS][4];
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
+        for (int ks = 0; ks < KS; ++ks) {
             uint2 qa = make_uint2(0, 0), qb = make_uint2(0, 0);
             if (ks < ksteps) {
                 if (ra) qa = __ldg(reinterpret_cast<const uint2*>(a.U + static_cast<int64_t>(start + g) * a.ldu + 16 * ks + 4 * t));
@@ -281,25 +285,38 @@ __global__ void __launch_bounds__(128, 4) k_seg_expand(SegArgs a) {
                 h[n][1] = (okc && rb) ? *reinterpret_cast<const uint32_t*>(hb + col) : 0u;
             }
         };
+        // B_i quads of one K step of a 64-column block (rows = output columns)
+        auto load_b = [&](int blk, int ks, uint2 (&bq)[8]) {
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                const int col = 64 * blk + 8 * n + g;
+                bq[n] = col < a.d_out ? ld_quad(Bi + static_cast<int64_t>(col) * r, 16 * ks + 4 * t, r, b_al8)
+                                      : make_uint2(0, 0);
+            }
+        };
         uint32_t h_cur[8][2], h_nxt[8][2];
-        if (warp < n_blocks) load_h(warp, h_cur);
+        uint2 b_cur[8], b_nxt[8];                          // K step 0 of this / the next block
+        if (warp < n_blocks) {
+            load_h(warp, h_cur);
+            load_b(warp, 0, b_cur);
+        }
         for (int blk = warp; blk < n_blocks; blk += 4) {
-            if (blk + 4 < n_blocks) load_h(blk + 4, h_nxt);
+            if (blk + 4 < n_blocks) {
+                load_h(blk + 4, h_nxt);
+                load_b(blk + 4, 0, b_nxt);
+            }
             float acc[8][4];
 #pragma unroll
             for (int n = 0; n < 8; ++n)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
+            for (int n = 0; n < 8; ++n) mma_bf16_16816(acc[n], uf[0], b_cur[n].x, b_cur[n].y, true);
+#pragma unroll
+            for (int ks = 1; ks < KS; ++ks) {
                 if (ks < ksteps) {
                     uint2 bq[8];
-#pragma unroll
-                    for (int n = 0; n < 8; ++n) {
-                        const int col = 64 * blk + 8 * n + g;      // output column = row of B_i
-                        bq[n] = col < a.d_out ? ld_quad(Bi + static_cast<int64_t>(col) * r, 16 * ks + 4 * t, r, b_al8)
-                                              : make_uint2(0, 0);
-                    }
+                    load_b(blk, ks, bq);
 #pragma unroll
                     for (int n = 0; n < 8; ++n) mma_bf16_16816(acc[n], uf[ks], bq[n].x, bq[n].y, true);
                 }
@@ -323,6 +340,7 @@ __global__ void __launch_bounds__(128, 4) k_seg_expand(SegArgs a) {
             for (int n = 0; n < 8; ++n) {
                 h_cur[n][0] = h_nxt[n][0];
                 h_cur[n][1] = h_nxt[n][1];
+                b_cur[n] = b_nxt[n];
             }
         }
     }
