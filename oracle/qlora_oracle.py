@@ -45,6 +45,13 @@ What it computes, and where each step is defined:
   accumulation (next to the FlashAttention-2 paragraph).  The pages name AdamW
   but print no update rule; the oracle writes out the published decoupled
   weight-decay rule (reading R23).
+* FP8 activations: E4M3 activations with a per-tensor scale, the decoded
+  weight rounded to E4M3 for the one FP8 contraction -- "LoRA and QLoRA
+  Fine-Tuning Under the Hood", section "1.3 Activation Memory Savings via
+  FlashAttention-2 & Activation Checkpointing" (FP8 formats E4M3 and E5M2 for
+  activations on Hopper and Blackwell).  The pages name the formats only; the
+  byte layout is the OCP 8-bit floating-point definition and the scaling,
+  rounding and operand choices are reading R25.
 
 Where the pages are silent or garbled the oracle takes the readings listed as
 R1..R19 in the design notes; each is named where it is applied.
@@ -363,6 +370,98 @@ def adamw_step(w, g, m, v, step: int, lr: float, beta1: float, beta2: float,
     v_hat = v / (1.0 - beta2 ** step)
     w = w * (1.0 - lr * weight_decay) - lr * m_hat / (np.sqrt(v_hat) + eps)
     return w, m, v
+
+
+# ----------------------------------------------------------------------------
+# FP8 activations (reading R25)
+# ----------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(code) -> np.ndarray:
+    """Value (fp64) of each E4M3 byte, the OCP 8-bit floating-point format the
+    pages name for activations: bit 7 sign, bits 6..3 exponent with bias 7,
+    bits 2..0 mantissa.  Exponent 0 holds the subnormals m/8 * 2^-6; the one
+    pattern S.1111.111 is NaN; there is no infinity (largest finite 448)."""
+    c = np.asarray(code, np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 15
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return sign * mag
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 byte of each finite fp32 value: the nearest representable value,
+    ties to the even code (mantissa lsb 0), magnitudes at or beyond 448
+    saturated to 448; the sign bit is the input's (so -0 and negatives that
+    round to zero give 0x80)."""
+    a = np.abs(np.asarray(x, np.float32).astype(np.float64))
+    neg = np.signbit(np.asarray(x, np.float32))
+    mags = e4m3_decode(np.arange(127, dtype=np.uint8))      # codes 0x00..0x7E, increasing
+    hi = np.minimum(np.searchsorted(mags, a, side="left"), 126)
+    lo = np.maximum(hi - 1, 0)
+    dlo = a - mags[lo]
+    dhi = mags[hi] - a
+    pick = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
+    pick = np.where(a >= E4M3_MAX, 126, pick)
+    return (pick.astype(np.uint8) | np.where(neg, 0x80, 0).astype(np.uint8)).astype(np.uint8)
+
+
+def fp8_pow2_scale(amax: float) -> float:
+    """Per-tensor scale sigma = 2^(8 - ceil(log2 amax)), so that amax * sigma
+    lies in (128, 256] below the E4M3 limit; 1 when amax is 0.  The exponent is
+    kept in [-126, 126] (an fp32 normal power of two)."""
+    if not amax > 0.0:
+        return 1.0
+    m, e = math.frexp(amax)                 # amax = m 2^e, 0.5 <= m < 1
+    c = e - 1 if m == 0.5 else e            # ceil(log2 amax)
+    return math.ldexp(1.0, min(max(8 - c, -126), 126))
+
+
+def fp8_quantize_act(X):
+    """(X8, sigma_x): X8 = E4M3(fl32(X * sigma_x)), sigma_x = fp8_pow2_scale(max|X|).
+    X is read as fp32 values (a bf16 activation is exact in fp32); X8 / sigma_x
+    stands for X."""
+    X32 = np.asarray(X, np.float32)
+    amax = float(np.max(np.abs(X32))) if X32.size else 0.0
+    sig = fp8_pow2_scale(amax)
+    return e4m3_encode((X32 * np.float32(sig)).astype(np.float32)), sig
+
+
+def fp8_weight_scale(c2) -> float:
+    """sigma_w of a double-quantized weight: every decoded weight is L * s_b with
+    |L| <= 1 and s_b <= c2 of its group (up to one fp32 rounding), so the
+    largest second-level constant bounds the tensor."""
+    c2 = np.asarray(c2, np.float32)
+    return fp8_pow2_scale(float(np.max(c2)) if c2.size else 0.0)
+
+
+def nf4_dequantize_e4m3(codes, absmax_q, c2, d_out: int, d_in: int, w_scale: float,
+                        levels: np.ndarray | None = None) -> np.ndarray:
+    """E4M3 bytes [d_out, d_in] of the decoded weight in sigma_w units:
+    E4M3(fl32(L[code] * s_b) * sigma_w) -- the fp32 decode of R11, scaled by an
+    exact power of two, rounded once to E4M3."""
+    w32 = nf4_dequantize(codes, absmax_q, c2, d_out, d_in, out="f32", levels=levels)
+    return e4m3_encode((w32 * np.float32(w_scale)).astype(np.float32))
+
+
+def lora_forward_fp8(X8, x_scale, W8, w_scale, A, B, alpha, r):
+    """Forward of the adapted layer with E4M3 activations and weights (fp64):
+
+        H = (X8 W8^T) / (sigma_x sigma_w) + s (X~ A^T) B^T,   X~ = X8 / sigma_x,
+
+    X8, W8 the E4M3 bytes (decoded here), the adapters A, B in their own dtype.
+    The base product is the one FP8 contraction; the low-rank branch reads the
+    same FP8 activation."""
+    Xv = e4m3_decode(X8)
+    Wv = e4m3_decode(W8)
+    Xt = Xv / float(x_scale)
+    A = np.asarray(A, np.float64)
+    B = np.asarray(B, np.float64)
+    return (Xv @ Wv.T) / (float(x_scale) * float(w_scale)) + lora_scale(alpha, r) * ((Xt @ A.T) @ B.T)
 
 
 # ----------------------------------------------------------------------------

@@ -401,6 +401,184 @@ def test_gradient_accumulation_equals_full_batch():
     assert rel(sum(p[1] for p in parts), full[1]) < 1e-13
 
 
+# ---------------------------------------------------------------- FP8 (R25)
+
+
+def brute_e4m3(x):
+    """Nearest finite E4M3 value by scanning all 254 finite codes; ties to the
+    even code; saturating at 448."""
+    vals = [(c, O.e4m3_decode(np.uint8(c)).item()) for c in range(256)
+            if (c & 0x7F) != 0x7F]
+    out = []
+    for v in np.asarray(x, np.float64).reshape(-1):
+        best = None
+        for c, cv in vals:
+            if (c & 0x80) != (0x80 if math.copysign(1.0, v) < 0 else 0):
+                continue
+            d = abs(v - cv)
+            if best is None or d < best[0] or (d == best[0] and c % 2 == 0):
+                best = (d, c)
+        out.append(best[1])
+    return np.array(out, np.uint8)
+
+
+def test_e4m3_format_constants():
+    # OCP 8-bit floating point, E4M3: largest finite 448, smallest normal 2^-6,
+    # smallest subnormal 2^-9, 1.0 = 0x38, one NaN pattern per sign, no infinity.
+    d = O.e4m3_decode
+    assert d(np.uint8(0x7E)) == 448.0 and d(np.uint8(0xFE)) == -448.0
+    assert d(np.uint8(0x08)) == 2.0 ** -6 and d(np.uint8(0x01)) == 2.0 ** -9
+    assert d(np.uint8(0x07)) == 7 * 2.0 ** -9
+    assert d(np.uint8(0x38)) == 1.0 and d(np.uint8(0x40)) == 2.0
+    assert np.isnan(d(np.uint8(0x7F))) and np.isnan(d(np.uint8(0xFF)))
+    pos = d(np.arange(127, dtype=np.uint8))
+    assert np.all(np.diff(pos) > 0)                        # codes 0..126 increase
+    assert np.sum(np.isfinite(d(np.arange(256, dtype=np.uint8)))) == 254
+
+
+def e4m3_probe_values():
+    rng = np.random.default_rng(11)
+    mags = np.exp2(rng.uniform(-12, 10, 3000))
+    x = mags * rng.choice([-1.0, 1.0], mags.size)
+    pos = O.e4m3_decode(np.arange(127, dtype=np.uint8))
+    mids = 0.5 * (pos[1:] + pos[:-1])                      # every tie
+    extra = np.array([0.0, -0.0, 448.0, 463.99, 464.0, 1e6, -1e6, 2.0 ** -10, -2.0 ** -10, 2.0 ** -11])
+    return np.concatenate([x, mids, -mids, extra]).astype(np.float32)
+
+
+def check_e4m3_encode(enc):
+    x = e4m3_probe_values()
+    return int(np.sum(enc(x) != brute_e4m3(x)))
+
+
+def test_e4m3_encode_against_brute_force():
+    assert check_e4m3_encode(O.e4m3_encode) == 0
+
+
+def test_e4m3_round_trip_and_error_bound():
+    c = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    assert np.array_equal(O.e4m3_encode(O.e4m3_decode(c).astype(np.float32)), c)
+    rng = np.random.default_rng(3)
+    x = (np.exp2(rng.uniform(-6, np.log2(448), 20000)) * rng.choice([-1, 1], 20000)).astype(np.float32)
+    err = np.abs(O.e4m3_decode(O.e4m3_encode(x)) - x.astype(np.float64))
+    assert np.all(err <= 2.0 ** -4 * np.abs(x))            # 3 mantissa bits: half an ulp
+    sub = (rng.uniform(-2.0 ** -6, 2.0 ** -6, 5000)).astype(np.float32)
+    assert np.all(np.abs(O.e4m3_decode(O.e4m3_encode(sub)) - sub) <= 2.0 ** -10)
+
+
+def check_pow2_scale(fn):
+    bad = 0
+    for amax in [4.0, 4.1, 0.06, 1e-3, 5.3, 255.0, 256.0, 300.0, 2.0 ** -20, 1e30]:
+        sig = fn(amax)
+        m, e = math.frexp(sig)
+        bad += (m != 0.5) or not (128.0 < amax * sig <= 256.0)
+    return bad + (fn(0.0) != 1.0)
+
+
+def test_fp8_scale_range():
+    assert check_pow2_scale(O.fp8_pow2_scale) == 0
+    assert O.fp8_pow2_scale(4.0) == 64.0 and O.fp8_pow2_scale(4.1) == 32.0
+
+
+def test_fp8_activation_quantizer():
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((37, 96)).astype(np.float32)
+    X8, sig = O.fp8_quantize_act(X)
+    assert X8.dtype == np.uint8 and X8.shape == X.shape
+    assert 128.0 < np.max(np.abs(X)) * sig <= 256.0
+    Xr = O.e4m3_decode(X8) / sig
+    big = np.abs(X) * sig >= 2.0 ** -6
+    assert np.all(np.abs(Xr - X)[big] <= 2.0 ** -4 * np.abs(X)[big])
+    assert np.all(np.abs(Xr - X)[~big] <= 2.0 ** -10 / sig)
+    # values already on the scaled E4M3 grid come back exactly
+    Xg = (O.e4m3_decode(X8) / sig).astype(np.float32)
+    X8g, sig_g = O.fp8_quantize_act(Xg)
+    assert sig_g == sig and np.array_equal(X8g, X8)
+    # an all-zero tensor: scale 1, all codes zero
+    Z8, zs = O.fp8_quantize_act(np.zeros((3, 64), np.float32))
+    assert zs == 1.0 and not Z8.any()
+
+
+def fp8_layer(T=5, d=7, k=128, r=3, seed=21):
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_normal((d, k)) * 0.02).astype(np.float32)
+    codes, q8, c2, c1 = O.nf4_quantize(W)
+    X = rng.standard_normal((T, k)).astype(np.float32)
+    A = rng.standard_normal((r, k)) / np.sqrt(r)
+    B = rng.standard_normal((d, r)) * 0.1
+    return W, codes, q8, c2, X, A, B
+
+
+def check_fp8_forward_loops(fwd):
+    W, codes, q8, c2, X, A, B = fp8_layer()
+    d, k = W.shape
+    T, r, alpha = X.shape[0], A.shape[0], 6.0
+    X8, sx = O.fp8_quantize_act(X)
+    sw = O.fp8_weight_scale(c2)
+    W8 = O.nf4_dequantize_e4m3(codes, q8, c2, d, k, sw)
+    H = fwd(X8, sx, W8, sw, A, B, alpha, r)
+    ref = np.zeros((T, d))
+    for t in range(T):
+        for i in range(d):
+            acc = 0.0
+            for j in range(k):
+                acc += O.e4m3_decode(X8[t, j]).item() * O.e4m3_decode(W8[i, j]).item()
+            acc /= sx * sw
+            for q in range(r):
+                u = 0.0
+                for j in range(k):
+                    u += A[q, j] * O.e4m3_decode(X8[t, j]).item() / sx
+                acc += (alpha / r) * B[i, q] * u
+            ref[t, i] = acc
+    return rel(H, ref)
+
+
+def check_fp8_forward_bound(fwd):
+    """The FP8 forward approximates the exact forward of the same layer: every
+    element within the E4M3 rounding bound (2^-4 relative per operand in the
+    normal range, 2^-10 / sigma absolute below it)."""
+    W, codes, q8, c2, X, A, B = fp8_layer(T=9, d=11, k=256, r=4, seed=2)
+    d, k = W.shape
+    X8, sx = O.fp8_quantize_act(X)
+    sw = O.fp8_weight_scale(c2)
+    W8 = O.nf4_dequantize_e4m3(codes, q8, c2, d, k, sw)
+    W32 = O.nf4_dequantize(codes, q8, c2, d, k, out="f32").astype(np.float64)
+    H = fwd(X8, sx, W8, sw, A, B, 8.0, 4)
+    exact = O.lora_forward(W32, X, A, B, 8.0, 4)
+    # x~ = x + e_x with |e_x| <= 2^-4 |x| + 2^-10 / sigma_x (likewise w), so
+    # |x~ w~ - x w| <= (2^-3 + 2^-8)|x||w| + (1 + 2^-4) 2^-10 (|x| / sigma_w + |w| / sigma_x)
+    #                  + 2^-20 / (sigma_x sigma_w)
+    aX = np.abs(X.astype(np.float64))
+    aW = np.abs(W32)
+    base = (2.0 ** -3 + 2.0 ** -8) * (aX @ aW.T) \
+        + (1 + 2.0 ** -4) * 2.0 ** -10 * (aX @ np.ones_like(aW).T / sw + np.ones_like(aX) @ aW.T / sx) \
+        + 2.0 ** -20 / (sx * sw) * k
+    lowrank = (8.0 / 4) * ((2.0 ** -10 / sx + 2.0 ** -4 * aX) @ np.abs(A).T) @ np.abs(B).T
+    return float(np.max(np.abs(H - exact) - (base + lowrank + 1e-12)))
+
+
+def test_fp8_forward_against_loops():
+    assert check_fp8_forward_loops(O.lora_forward_fp8) < 1e-12
+
+
+def test_fp8_forward_within_rounding_bound_of_exact():
+    assert check_fp8_forward_bound(O.lora_forward_fp8) <= 0.0
+
+
+def test_fp8_weight_decode():
+    W, codes, q8, c2, X, A, B = fp8_layer(d=9, k=192)
+    sw = O.fp8_weight_scale(c2)
+    W8 = O.nf4_dequantize_e4m3(codes, q8, c2, 9, 192, sw)
+    W32 = O.nf4_dequantize(codes, q8, c2, 9, 192, out="f32").astype(np.float64)
+    assert np.max(np.abs(W32)) * sw <= 256.0 * (1 + 2.0 ** -23)
+    Wr = O.e4m3_decode(W8) / sw
+    big = np.abs(W32) * sw >= 2.0 ** -6
+    assert np.all(np.abs(Wr - W32)[big] <= 2.0 ** -4 * np.abs(W32)[big])
+    # the zero level (code for |x| smallest) and the sign: W8 of -w is W8 of w with bit 7 flipped
+    assert np.array_equal(O.e4m3_encode(-(W32 * sw).astype(np.float32)) ^ W8,
+                          np.full_like(W8, 0x80))
+
+
 # ---------------------------------------------------------------- mutants
 
 
@@ -460,6 +638,49 @@ def test_pins_catch_planted_mistakes():
 
     assert check_dora_brute(dora_no_adapter_in_norm) > 1e-3
     assert check_dora_brute(dora_column_norms) > 1e-3
+
+    # FP8 mutants: ties away from zero, truncation, no saturation, a scale one power off,
+    # the weight scale dropped, the low-rank branch fed the scaled activation
+    def enc_ties_away(x):
+        a = np.abs(np.asarray(x, np.float32).astype(np.float64))
+        pos = O.e4m3_decode(np.arange(127, dtype=np.uint8))
+        hi = np.minimum(np.searchsorted(pos, a), 126)
+        lo = np.maximum(hi - 1, 0)
+        pick = np.where(a - pos[lo] < pos[hi] - a, lo, hi)
+        pick = np.where(a >= 448.0, 126, pick)
+        return (pick.astype(np.uint8) | np.where(np.signbit(np.asarray(x, np.float32)), 0x80, 0)).astype(np.uint8)
+
+    def enc_truncate(x):
+        a = np.abs(np.asarray(x, np.float32).astype(np.float64))
+        pos = O.e4m3_decode(np.arange(127, dtype=np.uint8))
+        pick = np.maximum(np.searchsorted(pos, a, side="right") - 1, 0)
+        return (pick.astype(np.uint8) | np.where(np.signbit(np.asarray(x, np.float32)), 0x80, 0)).astype(np.uint8)
+
+    def enc_no_saturation(x):
+        c = O.e4m3_encode(x)
+        a = np.abs(np.asarray(x, np.float32))
+        return np.where(a >= 464.0, c | 0x7F, c).astype(np.uint8)
+
+    assert check_e4m3_encode(enc_ties_away) > 0
+    assert check_e4m3_encode(enc_truncate) > 0
+    assert check_e4m3_encode(enc_no_saturation) > 0
+    assert check_pow2_scale(lambda a: 2.0 * O.fp8_pow2_scale(a)) > 0
+    assert check_pow2_scale(lambda a: 0.5 * O.fp8_pow2_scale(a)) > 0
+
+    def fwd8_no_wscale(X8, sx, W8, sw, A, B, a, r):
+        return O.lora_forward_fp8(X8, sx, W8, 1.0, A, B, a, r)
+
+    def fwd8_scaled_act_in_adapter(X8, sx, W8, sw, A, B, a, r):
+        return O.lora_forward_fp8(X8, sx, W8, sw, A, B, a, r) + s(a, r) * (
+            ((O.e4m3_decode(X8) - O.e4m3_decode(X8) / sx) @ np.asarray(A).T) @ np.asarray(B).T)
+
+    def fwd8_transposed(X8, sx, W8, sw, A, B, a, r):
+        H = O.lora_forward_fp8(X8, sx, W8, sw, A, B, a, r)
+        return H[::-1]
+
+    for m in (fwd8_no_wscale, fwd8_scaled_act_in_adapter, fwd8_transposed):
+        assert check_fp8_forward_bound(m) > 0.0
+    assert check_fp8_forward_loops(fwd8_no_wscale) > 1e-3
 
     # quantizer mutants: swapped nibbles and a 255-level second stage
     L = O.nf4_levels()
