@@ -190,6 +190,8 @@ def run_gpu(args):
         return run_decode_only(args, q, qb, S, torch, dev)
     if args.only == "multi":
         return run_multi_only(args, q, qb, torch, dev)
+    if args.only == "fp8":
+        return run_fp8_only(args, q, qb, S, torch, dev)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -469,6 +471,48 @@ def run_multi_only(args, q, qb, torch, dev):
     return 0 if err == 0 else 1
 
 
+def make_fp8_workload(q, S, torch, dev, n_weights=4, seed=19):
+    """The q_proj shape (4096^2, r = 16, T = 4096) with an E4M3 activation: n_weights NF4 copies
+    of one weight, their sigma_w, the bf16 and E4M3 activation, adapters, output, workspace."""
+    c = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
+    bf = torch.bfloat16
+    case = S.make_layer(c["d_out"], c["d_in"], c["r"], c["alpha"], c["T"], dtype="bf16", seed=seed,
+                        with_grad=False)
+    wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(n_weights)]
+    wsc = [q.fp8_weight_scale(w) for w in wl]
+    Xb = torch.from_numpy(case.X).to(dev).to(bf)
+    X8, xs = q.fp8_quantize(Xb)
+    A = torch.from_numpy(case.A).to(dev).to(bf)
+    B = torch.from_numpy(case.B).to(dev).to(bf)
+    H = torch.empty((c["T"], c["d_out"]), dtype=bf, device=dev)
+    ws = torch.empty(q.workspace_bytes(q.OP_FWD_FP8, q.BF16, c["T"], c["d_out"], c["d_in"], c["r"]),
+                     dtype=torch.uint8, device=dev)
+    return c, wl, wsc, Xb, X8, xs, A, B, H, ws
+
+
+def run_fp8_only(args, q, qb, S, torch, dev):
+    """The FP8 forward alone on the q_proj shape (4096^2, r = 16, T = 4096): W warm-up and K timed
+    eager calls over 4 rotating NF4 weights, for profiling its kernels."""
+    qb.build_library()
+    q.load()
+    c, wl, wsc, Xb, X8, xs, A, B, H, ws = make_fp8_workload(q, S, torch, dev)
+    W = max(3, args.warmup)
+    for i in range(W):
+        q.qlora_linear_fwd_fp8(wl[i % 4], X8, xs, wsc[i % 4], A, B, c["alpha"], H=H, ws=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        q.qlora_linear_fwd_fp8(wl[i % 4], X8, xs, wsc[i % 4], A, B, c["alpha"], H=H, ws=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    err = q.get_device_error()
+    print(json.dumps({"only": "fp8", "ms_per_call": e0.elapsed_time(e1) / args.steps,
+                      "device_error": err,
+                      "workload": "4096x4096 NF4, r=16, T=4096, E4M3 activation"}), flush=True)
+    return 0 if err == 0 else 1
+
+
 def _graph_time(torch, calls, reps=20):
     """Per-call device time of `calls` (a list of zero-argument launches) captured in one CUDA
     graph and replayed `reps` times: (median, min) microseconds per call over 5 measurements."""
@@ -623,6 +667,35 @@ def extra_rows(q, torch, S, dev, peaks, args):
                                            "tc_frac": fl / (med * 1e-6) / 1e12 / tc}
     del wl, X, A, B, mag, H, ws, case
 
+    # ---- FP8 forward on the q_proj shape (4096^2, r = 16, T = 4096): E4M3 activation, the weight
+    # decoded to E4M3 for kind::f8f6f4 tensor cores, the adapter term in bf16; the activation is
+    # quantized by its own (separately timed) call.  FP8 peak = measured bf16 x 2 (the dense
+    # fp8 : bf16 ratio of the part, 4.5 : 2.25 PFLOP/s).
+    c, wl, wsc, Xb, X8, xs, A, B, H, ws = make_fp8_workload(q, S, torch, dev)
+    calls = [(lambda w=w, sw=sw: q.qlora_linear_fwd_fp8(w, X8, xs, sw, A, B, c["alpha"], H=H, ws=ws))
+             for w, sw in zip(wl, wsc)]
+    med, _ = _graph_time(torch, calls, reps=10)
+    kev = []
+    for i in range(12):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        q.set_gemm_events(e0, e1)
+        q.qlora_linear_fwd_fp8(wl[i % 4], X8, xs, wsc[i % 4], A, B, c["alpha"], H=H, ws=ws)
+        q.set_gemm_events(None, None)
+        kev.append((e0, e1))
+    torch.cuda.synchronize()
+    kus = statistics.median(a.elapsed_time(b) * 1e3 for a, b in kev[4:])
+    qws = torch.empty(256, dtype=torch.uint8, device=dev)
+    qcalls = [(lambda: q.fp8_quantize(Xb, X8=X8, scale=xs, ws=qws))] * 4
+    qmed, _ = _graph_time(torch, qcalls, reps=10)
+    fl = flops_fwd(c["T"], c["d_out"], c["d_in"], c["r"])
+    tc8 = 2 * tc
+    qbytes = 3 * c["T"] * c["d_in"]
+    out["fp8_fwd_4096x4096_r16_T4096"] = {
+        "fwd_us": med, "tflops": fl / (med * 1e-6) / 1e12, "tc_frac_fp8": fl / (med * 1e-6) / 1e12 / tc8,
+        "gemm_us": kus, "gemm_tc_frac_fp8": fl / (kus * 1e-6) / 1e12 / tc8, "fp8_peak_tflops": tc8,
+        "quantize_us": qmed, "quantize_hbm_frac": qbytes / (qmed * 1e-6) / 1e9 / hbm}
+    del wl, wsc, Xb, X8, xs, A, B, H, ws, qws
+
     # ---- AdamW step over the adapters of a 32-layer d = 4096 model with rank 16 on q, k, v, o:
     # 32 * 4 * 16 * (4096 + 4096) = 16.8 M parameters, bf16 params + fp32 master, m, v, grad
     # (30 bytes per parameter, 503 MB > L2)
@@ -673,10 +746,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--extra", action="store_true", help="also time the other hot-path rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--only", default="step", choices=["step", "fwd", "bwd", "decode", "multi"],
+    ap.add_argument("--only", default="step", choices=["step", "fwd", "bwd", "decode", "multi", "fp8"],
                     help="time only the forward, only the backward, the decode-size forward "
                          "(11008x4096, r = 64, --tokens T) or the many-adapter forward (4096^2, "
-                         "1024 adapters of rank 16) alone, for profiling its kernels")
+                         "1024 adapters of rank 16) or the FP8 forward (4096^2, r = 16, T = 4096) "
+                         "alone, for profiling its kernels")
     ap.add_argument("--tokens", type=int, default=1, help="tokens of the --only decode run")
     args = ap.parse_args()
     if args.impl == "reference":

@@ -56,7 +56,7 @@ typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 
 typedef enum {
     QLORA_OP_FWD = 0, QLORA_OP_BWD = 1, QLORA_OP_FWD_BATCHED = 2, QLORA_OP_MERGE = 3,
-    QLORA_OP_FWD_MULTI = 4, QLORA_OP_DORA_FWD = 5
+    QLORA_OP_FWD_MULTI = 4, QLORA_OP_DORA_FWD = 5, QLORA_OP_FWD_FP8 = 6, QLORA_OP_FP8_QUANT = 7
 } qlora_op;
 
 /* Stored NF4 weight.  Block size 64 and group size 256 are fixed.
@@ -232,6 +232,36 @@ qlora_status qlora_dora_fwd(const qlora_nf4* w, const void* X, int64_t T, const 
 qlora_status qlora_dora_row_norms(const qlora_nf4* w, const void* A, const void* B, int32_t r,
                                   float alpha, float* norms, void* ws, size_t ws_bytes,
                                   cudaStream_t stream);
+
+/* ---- FP8 activations ------------------------------------------------------------------------
+ * [UH] "1.3 Activation Memory Savings via FlashAttention-2 & Activation Checkpointing": the
+ * FP8 formats E4M3 / E5M2, native on Blackwell, halve the activation bytes.  E4M3 is the OCP
+ * 8-bit float (sign, 4 exponent bits with bias 7, 3 mantissa bits; largest finite 448).  A
+ * tensor is held as bytes X8 with one per-tensor scale sigma (device fp32 scalar) such that
+ * X ~ E4M3value(X8) / sigma; sigma = 2^(8 - ceil(log2 max|X|)) (1 for an all-zero tensor).    */
+
+/* X8[n] = E4M3(fl32(X[i] * sigma)) (round to nearest even, saturating) and *scale = sigma, for
+ * a bf16 X of n >= 1 elements (device).  NaNs are ignored by the max.  Bit-exact.
+ * ws >= qlora_workspace_bytes(QLORA_OP_FP8_QUANT, QLORA_BF16, 1, 1, 64, 1) (256 bytes).      */
+qlora_status qlora_fp8_quantize(const void* X, int64_t n, uint8_t* X8, float* scale, void* ws,
+                                size_t ws_bytes, cudaStream_t stream);
+
+/* *w_scale (device fp32) = sigma_w = 2^(8 - ceil(log2 max c2)): every decoded weight
+ * L[code] * s_b has |L| <= 1 and s_b <= c2 of its group, so sigma_w * |w| <= 256.            */
+qlora_status qlora_fp8_weight_scale(const qlora_nf4* w, float* w_scale, cudaStream_t stream);
+
+/* Forward with the E4M3 activation X8[T, d_in] (scale *x_scale) and the weight decoded to E4M3
+ * inside the tensor-core GEMM (w8 = E4M3(fl32(L[code] * s_b) * sigma_w), sigma_w = *w_scale):
+ *   H = bf16( (X8 W8^T) / (sigma_x sigma_w) + s (X~ A^T) B^T ),   X~ = X8 / sigma_x,  s = alpha/r,
+ * the base product on kind::f8f6f4 tensor cores, the adapter term in bf16 (A, B bf16) added in
+ * the same fp32 accumulator.  x_scale and w_scale are device scalars from qlora_fp8_quantize /
+ * qlora_fp8_weight_scale (powers of two make every rescaling exact; other positive values are
+ * accepted).  ws >= qlora_workspace_bytes(QLORA_OP_FWD_FP8, QLORA_BF16, T, d_out, d_in, r).
+ * Forward only: no U is saved.                                                               */
+qlora_status qlora_linear_fwd_fp8(const qlora_nf4* w, const uint8_t* X8, int64_t T,
+                                  const float* x_scale, const float* w_scale, const void* A,
+                                  const void* B, int32_t r, float alpha, void* H, void* ws,
+                                  size_t ws_bytes, cudaStream_t stream);
 
 /* Size of the device scratch array behind qlora_linear_fwd_noalloc (bytes per GPU). */
 #define QLORA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

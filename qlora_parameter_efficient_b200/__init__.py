@@ -23,12 +23,14 @@ STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",
           3: "QLORA_ERR_CUDA", 4: "QLORA_ERR_TIMEOUT", 5: "QLORA_ERR_DEVICE"}
 F32, BF16 = 0, 1
 OP_FWD, OP_BWD, OP_FWD_BATCHED, OP_MERGE, OP_FWD_MULTI, OP_DORA_FWD = 0, 1, 2, 3, 4, 5
+OP_FWD_FP8, OP_FP8_QUANT = 6, 7
 
 # Every symbol include/qlora.h declares.
 EXPORTS = ["qlora_nf4_sizes", "qlora_nf4_levels", "nf4_quantize", "nf4_dequantize",
            "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "lora_merge",
            "qlora_linear_bwd_ex", "qlora_adamw_step", "qlora_prefetch", "qlora_dora_fwd",
-           "qlora_dora_row_norms",
+           "qlora_dora_row_norms", "qlora_fp8_quantize", "qlora_fp8_weight_scale",
+           "qlora_linear_fwd_fp8",
            "qlora_linear_fwd_batched", "qlora_linear_fwd_multi", "qlora_linear_fwd_noalloc",
            "qlora_get_device_error",
            "qlora_selftest_wait_timeout", "qlora_set_gemm_events", "qlora_launch_count",
@@ -81,6 +83,9 @@ def load() -> ctypes.CDLL:
         "qlora_prefetch": ([vp, sz, i32, vp], ctypes.c_int),
         "qlora_dora_fwd": ([pnf4, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "qlora_dora_row_norms": ([pnf4, vp, vp, i32, f32, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_fp8_quantize": ([vp, i64, vp, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_fp8_weight_scale": ([pnf4, vp, vp], ctypes.c_int),
+        "qlora_linear_fwd_fp8": ([pnf4, vp, i64, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp], ctypes.c_int),
         "qlora_linear_fwd_noalloc": ([pnf4, vp, i64, vp, vp, i32, f32, ctypes.c_int, vp, vp, vp], ctypes.c_int),
         "qlora_get_device_error": ([vp], ctypes.c_int),
         "qlora_selftest_wait_timeout": ([ctypes.c_uint64, vp], ctypes.c_int),
@@ -289,6 +294,52 @@ def qlora_dora_fwd(w: NF4Weight, X, A, B, alpha, magnitude, H=None, U_save=None,
         ctypes.byref(c), _ptr(X), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(magnitude), _ptr(H),
         _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream)))
     return H, U_save
+
+
+def fp8_quantize(X, X8=None, scale=None, ws=None, stream=None):
+    """E4M3 bytes of a bf16 tensor with its power-of-two scale: returns (X8 uint8, scale fp32[1]),
+    X ~ E4M3value(X8) / scale."""
+    torch = _torch()
+    _contig(X, X8)
+    if X.dtype != torch.bfloat16:
+        raise TypeError("fp8_quantize takes a bf16 tensor")
+    if X8 is None:
+        X8 = torch.empty(X.shape, dtype=torch.uint8, device=X.device)
+    if scale is None:
+        scale = torch.empty(1, dtype=torch.float32, device=X.device)
+    if ws is None:
+        ws = torch.empty(256, dtype=torch.uint8, device=X.device)
+    _check("qlora_fp8_quantize", load().qlora_fp8_quantize(
+        _ptr(X), X.numel(), _ptr(X8), _ptr(scale), _ptr(ws), ws.numel(), _stream(stream)))
+    return X8, scale
+
+
+def fp8_weight_scale(w: NF4Weight, out=None, stream=None):
+    """sigma_w (fp32[1], device) of a stored weight for the FP8 forward."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=w.codes.device)
+    _check("qlora_fp8_weight_scale", load().qlora_fp8_weight_scale(ctypes.byref(w._c()), _ptr(out),
+                                                                   _stream(stream)))
+    return out
+
+
+def qlora_linear_fwd_fp8(w: NF4Weight, X8, x_scale, w_scale, A, B, alpha, H=None, ws=None, stream=None):
+    """H = (X8 W8^T) / (sigma_x sigma_w) + (alpha/r) (X~ A^T) B^T with an E4M3 activation (bf16 H)."""
+    torch = _torch()
+    _contig(X8, A, B, H)
+    if X8.dtype != torch.uint8:
+        raise TypeError("X8 holds E4M3 bytes (uint8)")
+    T = X8.shape[0]
+    r = A.shape[0]
+    if H is None:
+        H = torch.empty((T, w.d_out), dtype=torch.bfloat16, device=X8.device)
+    ws = _ws(OP_FWD_FP8, BF16, T, w.d_out, w.d_in, r, X8.device, ws)
+    c = w._c()
+    _check("qlora_linear_fwd_fp8", load().qlora_linear_fwd_fp8(
+        ctypes.byref(c), _ptr(X8), T, _ptr(x_scale), _ptr(w_scale), _ptr(A), _ptr(B), r, float(alpha),
+        _ptr(H), _ptr(ws), ws.numel(), _stream(stream)))
+    return H
 
 
 def prefetch(ptr: int, nbytes: int, to_device: bool, stream=None):

@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqlora.so")
 SOURCES = ["qlora_api.cu", "noalloc.cu"]
-DEPS = ["qlora_api.cu", "noalloc.cu", "common.cuh", "nf4.cuh", "nf4_table.cuh", "tc_gemm.cuh", "nf4_gemm2.cuh", "qgemv.cuh", "simt.cuh"]
+DEPS = sorted(f for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh")))
 HEADER = os.path.join(os.path.dirname(HERE), "include", "qlora.h")
 
 NVCC_FLAGS = [

@@ -11,6 +11,8 @@
 //   decode:         s = fl32(fl32(q8 * c2) / 127), w = fl32(L[code] * s), bf16 = RN(w)
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "nf4_table.cuh"
 
@@ -72,6 +74,40 @@ __device__ __forceinline__ uint4 nf4_decode8(uint32_t q, const Nf4Planes& p) {
     out.z = prmt(lo_b, hi_b, 0x5140);
     out.w = prmt(lo_b, hi_b, 0x7362);
     return out;
+}
+
+// E4M3 decode for the FP8 GEMM.  The 8 positive magnitudes P[j] = E4M3(fl32(L[8+j] * s))
+// (round to nearest even, saturating at 448; s already carries the weight's power-of-two
+// scale) are bytes 0..7 of two registers; a code c < 8 decodes to P[7-c] with the sign bit set.
+struct Nf4Fp8Planes {
+    uint32_t lo, hi;
+};
+
+// Two fp32 values to two E4M3 bytes (a in the low byte).
+__device__ __forceinline__ uint32_t e4m3x2_bits(float a, float b) {
+    return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ Nf4Fp8Planes nf4_make_planes_e4m3(float s) {
+    const uint32_t p01 = e4m3x2_bits(__fmul_rn(c_nf4_levels[8], s), __fmul_rn(c_nf4_levels[9], s));
+    const uint32_t p23 = e4m3x2_bits(__fmul_rn(c_nf4_levels[10], s), __fmul_rn(c_nf4_levels[11], s));
+    const uint32_t p45 = e4m3x2_bits(__fmul_rn(c_nf4_levels[12], s), __fmul_rn(c_nf4_levels[13], s));
+    const uint32_t p67 = e4m3x2_bits(__fmul_rn(c_nf4_levels[14], s), __fmul_rn(c_nf4_levels[15], s));
+    return Nf4Fp8Planes{p01 | (p23 << 16), p45 | (p67 << 16)};
+}
+
+// Decode 8 packed codes (element e in nibble e) into 8 E4M3 bytes in element order.
+__device__ __forceinline__ uint2 nf4_decode8_e4m3(uint32_t q, const Nf4Fp8Planes& p) {
+    const uint32_t t = ~q & 0x88888888u;          // 8 in each nibble whose code is < 8
+    const uint32_t f = t - (t >> 3);              // -> 7 there, 0 elsewhere
+    const uint32_t m = (q ^ f) & 0x77777777u;     // magnitude index: c-8, or 7-c
+    uint32_t a = prmt(p.lo, p.hi, m);
+    uint32_t b = prmt(p.lo, p.hi, m >> 16);
+    // sign bytes (as in nf4_decode8): 0xFF where the element's code has bit 3 set
+    const uint32_t q4 = q << 4;
+    a |= ~prmt(q4, q, 0xD9C8) & 0x80808080u;
+    b |= ~prmt(q4, q, 0xFBEA) & 0x80808080u;
+    return make_uint2(a, b);
 }
 
 // ------------------------------------------------------------------ quantize

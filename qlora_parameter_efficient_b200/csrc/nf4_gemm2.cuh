@@ -2,6 +2,10 @@
 //
 //   forward (B_MN = false):  H[T, d_out]  = X[T, d_in]  W^T + sU[T, RP] B_pad[d_out, RP]^T
 //   dX      (B_MN = true):   dX[T, d_in]  = dH[T, d_out] W  + sG[T, RP] A_pad[RP, d_in]
+//   FP8 forward (FP8 = true): H = (X8 W8^T + U'[T, RP] B_pad^T) / (sigma_x sigma_w), X8 the
+//     E4M3 activation, W8 the weight decoded to E4M3 in sigma_w units, U' the adapter term
+//     already in those units; the main K steps are kind::f8f6f4 MMAs (K = 128 per step), the
+//     adapter steps stay kind::f16 bf16 MMAs into the same fp32 accumulator.
 //
 // A cluster of two CTAs (a "pair") computes 256 x 256 output tiles with 256x256x16 UMMA
 // instructions issued by the leader CTA.  Each CTA holds half of the A tile (128 token rows)
@@ -104,16 +108,48 @@ static_assert(kG2StagesA >= kG2StagesB, "B-slot reuse is gated through the A rin
 // group has already observed, so no parity wait can alias.
 static_assert(kG2StagesA % kG2DecGroups == 0, "A-ring depth must be a multiple of the groups");
 constexpr int kG2Threads = 32 * (6 + 4 * kG2DecGroups);
+// FP8: a K step is 128 E4M3 columns (the same 128-byte rows), its codes tile twice as large
+#ifndef QLORA_G2_FP8_STAGES_A
+#define QLORA_G2_FP8_STAGES_A 8
+#endif
+#ifndef QLORA_G2_FP8_STAGES_B
+#define QLORA_G2_FP8_STAGES_B 2
+#endif
+static_assert(QLORA_G2_FP8_STAGES_A >= QLORA_G2_FP8_STAGES_B, "B-slot reuse is gated through the A ring");
+static_assert(QLORA_G2_FP8_STAGES_A % kG2DecGroups == 0, "A-ring depth must be a multiple of the groups");
 
+template <bool FP8 = false>
 struct G2Smem {
-    static constexpr int kA = 128 * 64 * 2;       // this CTA's A half, one K step
-    static constexpr int kC = 128 * 64 / 2;       // NF4 codes of the B half
-    static constexpr int kB = 128 * 64 * 2;       // this CTA's decoded B half
+    static constexpr int SA = FP8 ? QLORA_G2_FP8_STAGES_A : kG2StagesA;
+    static constexpr int SB = FP8 ? QLORA_G2_FP8_STAGES_B : kG2StagesB;
+    static constexpr int kKStep = FP8 ? 128 : 64;  // K columns per step
+    static constexpr int kA = 128 * 128;          // this CTA's A half, one K step (128-byte rows)
+    static constexpr int kC = 128 * kKStep / 2;   // NF4 codes of the B half
+    static constexpr int kB = 128 * 128;          // this CTA's decoded B half
     static constexpr int kStageA = kA + kC;
     static constexpr int kBars = 512;
-    static constexpr int kTotal = 1024 + kG2StagesA * kStageA + kG2StagesB * kB + kBars;
+    static constexpr int kTotal = 1024 + SA * kStageA + SB * kB + kBars;
     static_assert(kTotal <= 232448, "shared memory budget");
 };
+
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B (K-major), fp32 D, dense.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N) {
+    return (1u << 4)                                  // D format fp32
+           | (0u << 7)                                // A format E4M3
+           | (0u << 10)                               // B format E4M3
+           | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
+__device__ __forceinline__ void umma_e4m3_ss_2sm(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 
 struct Gemm2Args {
     int M, N;              // output rows (tokens) and columns
@@ -131,6 +167,8 @@ struct Gemm2Args {
     int split_tiles;       // trailing tiles split in two along K (0 = none)
     float* part;           // [split_tiles][2 ranks][4 warps][2 halves][2048 float4] fp32 partials
     int* cnt;              // [split_tiles][2 ranks][4 warps] tickets, zero at launch
+    const float* x_scale;  // FP8: sigma_x (device scalar)
+    const float* w_scale;  // FP8: sigma_w (device scalar)
     int* err;
     uint64_t wait_ns;
 };
@@ -139,14 +177,15 @@ struct Gemm2Args {
 // consecutive lanes of one store are consecutive 16-byte words.
 __device__ __forceinline__ int g2_part_idx(int c, int g, int lane) { return (c * 8 + g) * 32 + lane; }
 
-template <bool B_MN>
+template <bool B_MN, bool FP8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
     k_nf4_gemm2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmC,
                 const __grid_constant__ CUtensorMap tmAx, const __grid_constant__ CUtensorMap tmBx,
                 const Gemm2Args args) {
-    using L = G2Smem;
-    constexpr int SA = kG2StagesA;
-    constexpr int SB = kG2StagesB;
+    static_assert(!(FP8 && B_MN), "the FP8 variant is the forward");
+    using L = G2Smem<FP8>;
+    constexpr int SA = L::SA;
+    constexpr int SB = L::SB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -268,7 +307,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
                 uint8_t* a = sA + s * L::kA;
                 uint8_t* c = sC + s * L::kC;
                 if (it < args.k_steps) {
-                    const int kx = it * 64;
+                    const int kx = it * L::kKStep;
                     mbar_arrive_expect_tx(&full[s], L::kA + L::kC);
                     tma_load_2d(a, &tmA, &full[s], kx, m0);
                     if (B_MN) tma_load_2d(c, &tmC, &full[s], n0 / 2, kx);
@@ -302,6 +341,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
         if (rank == 0 && lane == 0) {
             // ---------------------------------------------------------- MMA issuer (leader)
             const uint32_t idesc = make_idesc_bf16(256, 256, false, B_MN);
+            const uint32_t idesc8 = make_idesc_e4m3(256, 256);
             int git = 0;
             bool ok = true;
             for (int tc = 0; ok && tc < n_units; ++tc) {
@@ -327,11 +367,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
                     const uint32_t a = smem_u32(sA + s * L::kA);
                     const uint32_t b = smem_u32(sB + sb * L::kB);
                     const int nk = (it == iters_per_tile - 1 && it >= args.k_steps) ? args.ext_k16_last : 4;
-                    for (int k = 0; k < nk; ++k) {
-                        const uint64_t ad = make_sw128_desc(a + k * 32, 16, 1024);
-                        const uint64_t bd = B_MN ? make_sw128_desc(b + k * 2048, 8192, 1024)
-                                                 : make_sw128_desc(b + k * 32, 16, 1024);
-                        umma_bf16_ss_2sm(d_tmem, ad, bd, idesc, (it > it0 || k > 0) ? 1u : 0u);
+                    if (FP8 && it < args.k_steps) {
+                        // 4 x K = 32 E4M3 columns: 32 bytes of each 128-byte row per MMA
+                        for (int k = 0; k < 4; ++k)
+                            umma_e4m3_ss_2sm(d_tmem, make_sw128_desc(a + k * 32, 16, 1024),
+                                             make_sw128_desc(b + k * 32, 16, 1024), idesc8,
+                                             (it > it0 || k > 0) ? 1u : 0u);
+                    } else {
+                        for (int k = 0; k < nk; ++k) {
+                            const uint64_t ad = make_sw128_desc(a + k * 32, 16, 1024);
+                            const uint64_t bd = B_MN ? make_sw128_desc(b + k * 2048, 8192, 1024)
+                                                     : make_sw128_desc(b + k * 32, 16, 1024);
+                            umma_bf16_ss_2sm(d_tmem, ad, bd, idesc, (it > it0 || k > 0) ? 1u : 0u);
+                        }
                     }
                     umma_commit_2sm_both(&empty[s]);
                 }
@@ -355,6 +403,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
         // -------------------------------------------------------------- epilogue
         const int q = warp & 3;                    // TMEM lane quarter of this warp
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
+        // FP8: the accumulator holds sigma_x sigma_w H; both scales are powers of two
+        float out_scale = 1.f;
+        if constexpr (FP8) out_scale = __frcp_rn(__fmul_rn(__ldg(args.x_scale), __ldg(args.w_scale)));
         for (int tc = 0; tc < n_units; ++tc) {
             const bool is_half = tc >= n_full;
             const int tile = is_half ? half_tile : pair + tc * npairs;
@@ -414,6 +465,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
                 if (grow < args.M) {
                     const int gc = gc0 + c0;
                     __nv_bfloat16* o = args.out + grow * args.ld_out + gc;
+                    if constexpr (FP8) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * out_scale);
+                    }
                     if (args.col_scale != nullptr) {
                         // per-output-column factor (DoRA's m / ||W + sBA|| row norms)
 #pragma unroll
@@ -437,6 +492,104 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote_async_payload(acc_empty_leader + static_cast<uint32_t>(buf * 8));
+        }
+    } else if constexpr (FP8) {
+        // -------------------------------------------------------------- NF4 -> E4M3 decoders
+        // Thread j owns weight row j of this CTA's 128 and, per K step, that row's two
+        // consecutive 64-blocks: 128 E4M3 bytes, one whole 128-byte row of the swizzled tile.
+        const int grp = (warp - 6) >> 2;
+        const int j = ((warp - 6) & 3) * 32 + lane;
+        const float wsc = __ldg(args.w_scale);
+        struct Pre {
+            int nv;              // valid blocks of the step (0, 1 or 2)
+            uint32_t q8[2];
+            float c2[2];
+        };
+        auto fetch = [&](int git, Pre& pr) {
+            pr.nv = 0;
+            if (git >= total_iters) return;
+            int tile, it;
+            step_of(git, tile, it);
+            if (it >= args.k_steps) return;
+            const int64_t wrow = static_cast<int64_t>(tile / args.m_tiles) * 256 + rank * 128 + j;
+            const int64_t wblk = 2 * static_cast<int64_t>(it);
+            if (wrow >= args.nf4_rows || wblk >= args.nf4_bpr) return;
+            pr.nv = wblk + 1 < args.nf4_bpr ? 2 : 1;
+            const int64_t b0 = wrow * args.nf4_bpr + wblk;
+            for (int h = 0; h < pr.nv; ++h) {
+                pr.q8[h] = __ldg(args.absmax_q + b0 + h);
+                pr.c2[h] = __ldg(args.c2 + ((b0 + h) >> 8));
+            }
+        };
+        uint4 dec[8];
+        auto decode_into_regs = [&](int git, const Pre& pr) {
+            const uint8_t* src = sC + (git % SA) * L::kC + j * 64;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (h < pr.nv) {
+                    const Nf4Fp8Planes p = nf4_make_planes_e4m3(__fmul_rn(nf4_block_scale(pr.q8[h], pr.c2[h]), wsc));
+                    const uint4 qa = *reinterpret_cast<const uint4*>(src + 32 * h);
+                    const uint4 qb = *reinterpret_cast<const uint4*>(src + 32 * h + 16);
+                    const uint2 e0 = nf4_decode8_e4m3(qa.x, p), e1 = nf4_decode8_e4m3(qa.y, p);
+                    const uint2 e2 = nf4_decode8_e4m3(qa.z, p), e3 = nf4_decode8_e4m3(qa.w, p);
+                    const uint2 e4 = nf4_decode8_e4m3(qb.x, p), e5 = nf4_decode8_e4m3(qb.y, p);
+                    const uint2 e6 = nf4_decode8_e4m3(qb.z, p), e7 = nf4_decode8_e4m3(qb.w, p);
+                    dec[4 * h + 0] = make_uint4(e0.x, e0.y, e1.x, e1.y);
+                    dec[4 * h + 1] = make_uint4(e2.x, e2.y, e3.x, e3.y);
+                    dec[4 * h + 2] = make_uint4(e4.x, e4.y, e5.x, e5.y);
+                    dec[4 * h + 3] = make_uint4(e6.x, e6.y, e7.x, e7.y);
+                } else {
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) dec[4 * h + ch] = make_uint4(0, 0, 0, 0);
+                }
+            }
+        };
+        uint64_t* arrive_bar = rank == 0 ? ready : dec_done;
+        Pre nxt;
+        fetch(grp, nxt);
+        bool have = false;          // dec[] holds step `git` (decoded ahead)
+        for (int git = grp; git < total_iters; git += kG2DecGroups) {
+            const int s = git % SA;
+            int tile_unused, it;
+            step_of(git, tile_unused, it);
+            const bool main_step = it < args.k_steps;
+            if (!have) {
+                const Pre cur = nxt;
+                fetch(git + kG2DecGroups, nxt);
+                if (!mbar_wait_warp(&full[s], (git / SA) & 1, abort, args.wait_ns)) {
+                    fail();
+                    break;
+                }
+                if (main_step) decode_into_regs(git, cur);
+            }
+            if (main_step) {
+                if (!wait_slot_free_warp(git)) {
+                    fail();
+                    break;
+                }
+                uint8_t* dst_row = sB + (git % SB) * L::kB + j * 128;
+                const uint32_t sw = j & 7;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(dst_row + ((ch ^ sw) << 4)) = dec[ch];
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&arrive_bar[s]);
+            have = false;
+            const int gn = git + kG2DecGroups;
+            int tile_gn = 0, it_gn = 0;
+            if (gn < total_iters) step_of(gn, tile_gn, it_gn);
+            if (gn < total_iters && it_gn < args.k_steps) {
+                const Pre cur = nxt;
+                fetch(gn + kG2DecGroups, nxt);
+                if (!mbar_wait_warp(&full[gn % SA], (gn / SA) & 1, abort, args.wait_ns)) {
+                    fail();
+                    break;
+                }
+                decode_into_regs(gn, cur);
+                have = true;
+            }
         }
     } else {
         // -------------------------------------------------------------- NF4 decoders

@@ -17,6 +17,7 @@
 #include "merge.cuh"
 #include "segmented.cuh"
 #include "optim.cuh"
+#include "fp8.cuh"
 #include "qgemv.cuh"
 
 using namespace qlora;
@@ -158,6 +159,22 @@ qlora_status tmap_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t col
     return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// byte matrix [rows, cols] (row stride ld bytes), 128-byte swizzle, box = 128 bytes x box_rows:
+// an E4M3 operand tile in the UMMA K-major layout.
+qlora_status tmap_u8_sw128(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                           uint32_t box_rows) {
+    QL_TRY(get_encoder());
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 // ======================================================================= planning
 
 int choose_split(int64_t tiles, int64_t k_steps) {
@@ -216,12 +233,12 @@ struct G2Sched {
     size_t part_bytes = 0, cnt_bytes = 0;
     size_t bytes() const { return part_bytes + cnt_bytes; }
 };
-G2Sched g2_schedule(int64_t T, int64_t N, int64_t K) {
+G2Sched g2_schedule(int64_t T, int64_t N, int64_t K, int64_t k_step = 64) {
     G2Sched g;
     const int64_t tiles = cdiv(T, 256) * cdiv(N, 256);
     g.pairs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, kSmsForSplit / 2)));
     const int64_t rem = tiles % g.pairs;
-    if (tiles > g.pairs && rem > 0 && 2 * rem <= g.pairs && cdiv(K, 64) >= 2) {
+    if (tiles > g.pairs && rem > 0 && 2 * rem <= g.pairs && cdiv(K, k_step) >= 2) {
         g.split_tiles = static_cast<int>(rem);
         g.part_bytes = align256(static_cast<size_t>(rem) * 2 * 4 * 2 * 2048 * 16);
         g.cnt_bytes = align256(static_cast<size_t>(rem) * 2 * 4 * sizeof(int));
@@ -258,6 +275,18 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
         return o;
     };
     if (op == QLORA_OP_MERGE) return p;
+    if (op == QLORA_OP_FP8_QUANT) {
+        p.total = 256;      // the amax word
+        return p;
+    }
+    if (op == QLORA_OP_FWD_FP8) {
+        p.RP = pad_rank(r);
+        if (r % 8 != 0) p.b_pad = take(static_cast<size_t>(d_out) * p.RP * 2);
+        p.u_spad = take(static_cast<size_t>(T) * p.RP * 2);
+        p.g2 = take(g2_schedule(T, d_out, d_in, 128).bytes());
+        p.total = off;
+        return p;
+    }
     if (op == QLORA_OP_FWD_MULTI) {
         // base GEMM split tail, then the segmented adapter term (r = the largest rank)
         p.g2 = take(g2_schedule(T, d_out, d_in).bytes());
@@ -441,14 +470,25 @@ qlora_status skinny_gemm(bool a_mn, bool b_mn, int RP, int n_valid, const CUtens
 // when the TMA zero-fills the rank padding out of bounds).
 qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, const void* ext_a,
                       const void* ext_b, int RP, int r_used, int ext_b_rank, void* out,
-                      void* g2ws, int* err, cudaStream_t st, const float* col_scale = nullptr) {
+                      void* g2ws, int* err, cudaStream_t st, const float* col_scale = nullptr,
+                      const float* x_scale = nullptr, const float* w_scale = nullptr) {
+    // x_scale != NULL: the FP8 forward (act is the E4M3 activation, ext_a the adapter term in
+    // sigma_x sigma_w units)
+    const bool fp8 = x_scale != nullptr;
+    if (fp8 && dx) return QLORA_ERR_UNSUPPORTED;
     const int64_t d_out = w->d_out, d_in = w->d_in;
     CUtensorMap ta, tc, tax, tbx;
     const int64_t K = dx ? d_out : d_in;
     const int64_t N = dx ? d_in : d_out;
-    QL_TRY(tmap_bf16(&ta, act, T, K, K, 128));
-    if (dx) QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 64, 64));
-    else QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 32, 128));
+    const int64_t k_step = fp8 ? 128 : 64;
+    if (fp8) {
+        QL_TRY(tmap_u8_sw128(&ta, act, T, K, K, 128));
+        QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 64, 128));
+    } else {
+        QL_TRY(tmap_bf16(&ta, act, T, K, K, 128));
+        if (dx) QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 64, 64));
+        else QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 32, 128));
+    }
     if (RP > 0) {
         QL_TRY(tmap_bf16(&tax, ext_a, T, RP, RP, 128));
         if (dx) QL_TRY(tmap_bf16(&tbx, ext_b, ext_b_rank, d_in, d_in, 64));
@@ -459,9 +499,11 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
     }
     Gemm2Args g{};
     g.col_scale = col_scale;
+    g.x_scale = x_scale;
+    g.w_scale = w_scale;
     g.M = static_cast<int>(T);
     g.N = static_cast<int>(N);
-    g.k_steps = static_cast<int>(cdiv(K, 64));
+    g.k_steps = static_cast<int>(cdiv(K, k_step));
     g.ext_steps = RP / 64;
     g.ext_k16_last = RP > 0 ? static_cast<int>(std::min<int64_t>(4, cdiv(r_used - 64 * (g.ext_steps - 1), 16))) : 4;
     g.m_tiles = static_cast<int>(cdiv(T, 256));
@@ -474,7 +516,7 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
     g.ld_out = N;
     g.err = err;
     g.wait_ns = kWaitNs;
-    const G2Sched sch = g2_schedule(T, N, K);
+    const G2Sched sch = g2_schedule(T, N, K, k_step);
     const int pairs = sch.pairs;
     g.split_tiles = sch.split_tiles;
     if (sch.split_tiles > 0) {
@@ -482,22 +524,23 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
         g.part = static_cast<float*>(g2ws);
         g.cnt = reinterpret_cast<int*>(static_cast<uint8_t*>(g2ws) + sch.part_bytes);
     }
-    auto kern = dx ? k_nf4_gemm2<true> : k_nf4_gemm2<false>;
-    static std::atomic<uint64_t> configured[2] = {0, 0};
+    auto kern = fp8 ? k_nf4_gemm2<false, true> : dx ? k_nf4_gemm2<true> : k_nf4_gemm2<false>;
+    const int smem = fp8 ? G2Smem<true>::kTotal : G2Smem<false>::kTotal;
+    const int variant = fp8 ? 2 : dx ? 1 : 0;
+    static std::atomic<uint64_t> configured[3] = {0, 0, 0};
     int dev = 0;
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
-    if (!(configured[dx].load() & bit)) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G2Smem::kTotal) !=
-            cudaSuccess)
+    if (!(configured[variant].load() & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return QLORA_ERR_CUDA;
-        configured[dx].fetch_or(bit);
+        configured[variant].fetch_or(bit);
     }
     if (sch.split_tiles > 0 && cudaMemsetAsync(g.cnt, 0, sch.cnt_bytes, st) != cudaSuccess)
         return QLORA_ERR_CUDA;
     const bool ev = g_ev_start && g_ev_stop;
     if (ev) cudaEventRecord(g_ev_start, st);
-    if (launch_pdl(kern, dim3(2 * pairs), dim3(kG2Threads), G2Smem::kTotal, st, ta, tc, tax, tbx, g) !=
+    if (launch_pdl(kern, dim3(2 * pairs), dim3(kG2Threads), smem, st, ta, tc, tax, tbx, g) !=
         cudaSuccess)
         return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
@@ -832,8 +875,10 @@ qlora_status qlora_nf4_levels(float* out) {
 
 size_t qlora_workspace_bytes(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in,
                              int32_t r_total) {
-    if (op < QLORA_OP_FWD || op > QLORA_OP_DORA_FWD) return 0;
-    if ((op == QLORA_OP_FWD_MULTI || op == QLORA_OP_DORA_FWD) && dtype != QLORA_BF16) return 0;
+    if (op < QLORA_OP_FWD || op > QLORA_OP_FP8_QUANT) return 0;
+    if ((op == QLORA_OP_FWD_MULTI || op == QLORA_OP_DORA_FWD || op == QLORA_OP_FWD_FP8 ||
+         op == QLORA_OP_FP8_QUANT) && dtype != QLORA_BF16)
+        return 0;
     if ((dtype != QLORA_BF16 && dtype != QLORA_F32) || T < 1 || d_out < 1 || d_in < 64 ||
         r_total < 1 || r_total > 128)
         return 0;
@@ -932,6 +977,74 @@ qlora_status qlora_dora_fwd(const qlora_nf4* w, const void* X, int64_t T, const 
     float* scale = at<float>(ws, p.dora_scale);
     QL_TRY(dora_scale(w, A, B, r, s, magnitude, at<float>(ws, p.dora_part), scale, stream));
     return fwd_bf16_large(w, X, T, A, B, r, s, H, U_save, p, ws, err, stream, scale);
+}
+
+qlora_status qlora_fp8_quantize(const void* X, int64_t n, uint8_t* X8, float* scale, void* ws,
+                                size_t ws_bytes, cudaStream_t stream) {
+    if (!aligned16(X) || !aligned16(X8) || !scale) return QLORA_ERR_INVALID_ARG;
+    if (n < 1) return QLORA_ERR_UNSUPPORTED;
+    QL_TRY(check_ws(ws, ws_bytes, 256));
+    auto* amax = static_cast<unsigned*>(ws);
+    if (cudaMemsetAsync(amax, 0, 4, stream) != cudaSuccess) return QLORA_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(std::min<int64_t>(std::max<int64_t>(cdiv(n, 8 * 256), 1), 148 * 8)));
+    if (launch_pdl(k_fp8_amax, grid, dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(X), n, amax) !=
+        cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    if (launch_pdl(k_fp8_quant, grid, dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(X), n,
+                   static_cast<const unsigned*>(amax), X8, scale) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+qlora_status qlora_fp8_weight_scale(const qlora_nf4* w, float* w_scale, cudaStream_t stream) {
+    QL_TRY(check_nf4(w));
+    if (!w_scale) return QLORA_ERR_INVALID_ARG;
+    const int64_t groups = cdiv(w->d_out * w->d_in / 64, 256);
+    if (launch_pdl(k_fp8_wscale, dim3(1), dim3(256), 0, stream, w->c2, groups, w_scale) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd_fp8(const qlora_nf4* w, const uint8_t* X8, int64_t T,
+                                  const float* x_scale, const float* w_scale, const void* A,
+                                  const void* B, int32_t r, float alpha, void* H, void* ws,
+                                  size_t ws_bytes, cudaStream_t stream) {
+    QL_TRY(check_layer(w, T, r, QLORA_BF16));
+    if (!aligned16(X8) || !aligned16(A) || !aligned16(B) || !aligned16(H) || !x_scale || !w_scale)
+        return QLORA_ERR_INVALID_ARG;
+    const Plan p = make_plan(QLORA_OP_FWD_FP8, QLORA_BF16, T, w->d_out, w->d_in, r);
+    QL_TRY(check_ws(ws, ws_bytes, p.total));
+    int* err = nullptr;
+    QL_TRY(err_word(&err));
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    const float s = alpha / static_cast<float>(r);
+    const int RP = p.RP;
+    // B as the extension's B operand: the caller's B when its rows are whole 16-byte units
+    // (the map zero-fills the rank padding), else a zero-padded copy
+    const void* b_src = B;
+    int b_ld = r;
+    if (r % 8 != 0) {
+        auto* b_pad = at<__nv_bfloat16>(ws, p.b_pad);
+        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
+        b_src = b_pad;
+        b_ld = RP;
+    }
+    auto* u = at<__nv_bfloat16>(ws, p.u_spad);
+    const auto* Ab = static_cast<const __nv_bfloat16*>(A);
+    const dim3 ug(static_cast<unsigned>(cdiv(T, 16)));
+    const int di = static_cast<int>(d_in);
+    cudaError_t e;
+    if (r <= 16) e = launch_pdl(k_fp8_u<2>, ug, dim3(128), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
+    else if (r <= 32) e = launch_pdl(k_fp8_u<4>, ug, dim3(128), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
+    else if (r <= 64) e = launch_pdl(k_fp8_u<8>, ug, dim3(128), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
+    else e = launch_pdl(k_fp8_u<16>, ug, dim3(128), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
+    if (e != cudaSuccess) return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    return nf4_gemm(false, w, X8, T, u, b_src, RP, r, b_ld, H, at<void>(ws, p.g2), err, stream, nullptr,
+                    x_scale, w_scale);
 }
 
 qlora_status qlora_linear_bwd_ex(const qlora_nf4* w, const void* X, const void* dH, int64_t T,

@@ -590,3 +590,103 @@ def test_dora_magnitude_at_norms_is_lora(q):
     Hl, _ = q.qlora_linear_fwd(w, X, A, B, case.alpha)
     torch.cuda.synchronize()
     assert rel_fro(host(Hd), host(Hl).astype(np.float64)) <= 4e-3
+
+
+# ------------------------------------------------------------------ FP8 activations (R25)
+
+
+def fp8_probe_activation(n, seed):
+    """bf16 values whose scaled copies (amax 4 -> sigma 64) hit every E4M3 tie below 256, the
+    subnormal range and zeros, plus normal draws."""
+    rng = np.random.default_rng(seed)
+    x = S.round_to_bf16((rng.standard_normal(n) * 0.8).astype(np.float32))
+    x = np.clip(x, -3.875, 3.875)
+    pos = O.e4m3_decode(np.arange(127, dtype=np.uint8))
+    mids = 0.5 * (pos[1:] + pos[:-1])
+    mids = (mids[mids < 256.0] / 64.0).astype(np.float32)
+    probe = np.concatenate([mids, -mids, np.float32([0.0, 2.0 ** -20, -2.0 ** -17, 2.0 ** -110])])
+    m = min(n - 1, probe.size)
+    x[1:1 + m] = probe[:m]
+    x[0] = 4.0
+    assert np.array_equal(S.round_to_bf16(x), x)
+    return x
+
+
+@pytest.mark.parametrize("shape", [(12345,), (64, 4096), (3,), (7, 136)])
+def test_fp8_quantize_bit_exact(q, shape):
+    import torch
+    n = int(np.prod(shape))
+    X = fp8_probe_activation(n, seed=n).reshape(shape)
+    X8, sc = q.fp8_quantize(dev(X, "bf16"))
+    torch.cuda.synchronize()
+    ref8, sig = O.fp8_quantize_act(X)
+    assert float(sc.item()) == sig
+    assert np.array_equal(X8.cpu().numpy(), ref8)
+
+
+def test_fp8_quantize_zero_and_tiny_tensors(q):
+    import torch
+    for X in (np.zeros((5, 64), np.float32), np.full(9, 2.0 ** -100, np.float32)):
+        X8, sc = q.fp8_quantize(dev(X, "bf16"))
+        torch.cuda.synchronize()
+        ref8, sig = O.fp8_quantize_act(S.round_to_bf16(X))
+        assert float(sc.item()) == sig
+        assert np.array_equal(X8.cpu().numpy(), ref8)
+
+
+@pytest.mark.parametrize("d_out,d_in", [(200, 192), (4096, 4096)])
+def test_fp8_weight_scale(q, d_out, d_in):
+    import torch
+    rng = np.random.default_rng(d_in)
+    W = (rng.standard_normal((d_out, d_in)) * 0.141).astype(np.float32)
+    w, oc = quantize_both(q, W)
+    sw = q.fp8_weight_scale(w)
+    torch.cuda.synchronize()
+    assert float(sw.item()) == O.fp8_weight_scale(oc[2])
+
+
+def run_fp8(q, case, rows=None):
+    """FP8 forward on the oracle's E4M3 activation and scales (uploaded as inputs) against the
+    oracle's FP8 forward."""
+    import torch
+    w, oc = quantize_both(q, case.W0)
+    codes, q8, c2, _ = oc
+    X8, sx = O.fp8_quantize_act(case.X)
+    sw = O.fp8_weight_scale(c2)
+    W8 = O.nf4_dequantize_e4m3(codes, q8, c2, case.d_out, case.d_in, sw)
+    xs = torch.tensor([sx], dtype=torch.float32, device="cuda")
+    wsc = torch.tensor([sw], dtype=torch.float32, device="cuda")
+    H = q.qlora_linear_fwd_fp8(w, torch.from_numpy(X8).cuda(), xs, wsc, dev(case.A, "bf16"),
+                               dev(case.B, "bf16"), case.alpha)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    sel = slice(None) if rows is None else rows
+    ref = O.lora_forward_fp8(X8[sel], sx, W8, sw, case.A, case.B, case.alpha, case.r)
+    assert rel_fro(host(H)[sel], ref) <= TOL["bf16"]
+    return w, oc, H
+
+
+@pytest.mark.parametrize("d_out,d_in,r,T", [(256, 256, 8, 64), (200, 192, 5, 77), (520, 320, 16, 300),
+                                            (136, 256, 100, 3), (64, 128, 16, 1), (264, 1088, 64, 520)])
+def test_fp8_forward(q, d_out, d_in, r, T):
+    run_fp8(q, S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_out + T, with_grad=False))
+
+
+def test_fp8_forward_q_proj_sampled_rows(q):
+    case = S.make_layer(**S.CONFIGS["q_proj_4096x4096_r16_T4096"], seed=4, with_grad=False)
+    rows = np.sort(np.random.default_rng(6).choice(case.T, 256, replace=False))
+    run_fp8(q, case, rows=rows)
+
+
+def test_fp8_end_to_end_approximates_bf16_layer(q):
+    """Device quantizer -> FP8 forward stays within the E4M3 rounding of the exact layer."""
+    import torch
+    case = S.make_layer(384, 512, 16, 32.0, 200, dtype="bf16", seed=12, with_grad=False)
+    w, oc = quantize_both(q, case.W0)
+    X8, xs = q.fp8_quantize(dev(case.X, "bf16"))
+    H = q.qlora_linear_fwd_fp8(w, X8, xs, q.fp8_weight_scale(w), dev(case.A, "bf16"),
+                               dev(case.B, "bf16"), case.alpha)
+    torch.cuda.synchronize()
+    ref = O.lora_forward(oracle_weight(oc, 384, 512, "f32"), case.X, case.A, case.B, case.alpha, case.r)
+    e = rel_fro(host(H), ref)
+    assert 1e-3 < e < 0.06
