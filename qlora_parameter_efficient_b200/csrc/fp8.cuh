@@ -119,17 +119,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t v) {
 //   U'[t, j] = bf16(fl32(s * sigma_w) * sum_k X8v[t, k] A[j, k])   (j < r; zero for r <= j < ldu)
 // X8v the E4M3 values of X8 (X times sigma_x), so U' = sigma_x sigma_w bf16(s X A^T) up to the
 // activation's rounding: the adapter term in the units of the FP8 accumulator.  fp32
-// accumulation with mma.sync m16n8k16; the 4 warps split K in 64-wide chunks and their
+// accumulation with mma.sync m16n8k16; the WARPS warps split K in 64-wide chunks (each warp
+// issuing the loads of UNR chunks before their MMAs, to keep many loads in flight) and their
 // partials are summed in a fixed order.  Within a chunk, thread quad t owns the 16 consecutive
 // columns 16t..16t+15 of both operands (the same permutation of K for A and B leaves every dot
 // product unchanged), so each operand fragment is one contiguous load.
-template <int NT>
-__global__ void __launch_bounds__(128) k_fp8_u(const uint8_t* __restrict__ X8, int64_t T, int d_in,
-                                               const __nv_bfloat16* __restrict__ A, int r, float s,
-                                               const float* __restrict__ w_scale,
-                                               __nv_bfloat16* __restrict__ U, int ldu) {
+template <int NT, int WARPS, int UNR>
+__global__ void __launch_bounds__(32 * WARPS) k_fp8_u(const uint8_t* __restrict__ X8, int64_t T, int d_in,
+                                                      const __nv_bfloat16* __restrict__ A, int r, float s,
+                                                      const float* __restrict__ w_scale,
+                                                      __nv_bfloat16* __restrict__ U, int ldu) {
     griddep_enter();
-    __shared__ float s_part[4][16][NT * 8 + 1];
+    __shared__ float s_part[WARPS][16][NT * 8 + 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * 16;
     const int64_t ra = t0 + g, rb = t0 + g + 8;
@@ -141,32 +142,48 @@ __global__ void __launch_bounds__(128) k_fp8_u(const uint8_t* __restrict__ X8, i
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
     const uint4 z4 = make_uint4(0, 0, 0, 0);
-    for (int k0 = 64 * warp; k0 < d_in; k0 += 256) {
-        const uint4 qa = ra < T ? __ldg(reinterpret_cast<const uint4*>(xa + k0)) : z4;
-        const uint4 qb = rb < T ? __ldg(reinterpret_cast<const uint4*>(xb + k0)) : z4;
-        uint32_t fa[8], fb[8];
-        const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
+    constexpr int kStride = 64 * WARPS;
+    for (int kb = 64 * warp; kb < d_in; kb += kStride * UNR) {
+        uint4 qa[UNR], qb[UNR], b0[UNR][NT], b1[UNR][NT];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            fa[2 * k] = e4m3x2_to_bf16x2(wa[k]);
-            fa[2 * k + 1] = e4m3x2_to_bf16x2(wa[k] >> 16);
-            fb[2 * k] = e4m3x2_to_bf16x2(wb[k]);
-            fb[2 * k + 1] = e4m3x2_to_bf16x2(wb[k] >> 16);
+        for (int u = 0; u < UNR; ++u) {
+            const int k0 = kb + u * kStride;
+            const bool kin = k0 < d_in;
+            qa[u] = kin && ra < T ? __ldg(reinterpret_cast<const uint4*>(xa + k0)) : z4;
+            qb[u] = kin && rb < T ? __ldg(reinterpret_cast<const uint4*>(xb + k0)) : z4;
+#pragma unroll
+            for (int nn = 0; nn < NT; ++nn) {
+                const int n = 8 * nn + g;
+                b0[u][nn] = z4;
+                b1[u][nn] = z4;
+                if (kin && n < r) {
+                    const uint4* ap = reinterpret_cast<const uint4*>(A + static_cast<int64_t>(n) * d_in + k0 + 16 * t);
+                    b0[u][nn] = __ldg(ap);
+                    b1[u][nn] = __ldg(ap + 1);
+                }
+            }
         }
 #pragma unroll
-        for (int nn = 0; nn < NT; ++nn) {
-            const int n = 8 * nn + g;
-            uint4 b0 = z4, b1 = z4;
-            if (n < r) {
-                const uint4* ap = reinterpret_cast<const uint4*>(A + static_cast<int64_t>(n) * d_in + k0 + 16 * t);
-                b0 = __ldg(ap);
-                b1 = __ldg(ap + 1);
-            }
-            const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        for (int u = 0; u < UNR; ++u) {
+            uint32_t fa[8], fb[8];
+            const uint32_t wa[4] = {qa[u].x, qa[u].y, qa[u].z, qa[u].w};
+            const uint32_t wb[4] = {qb[u].x, qb[u].y, qb[u].z, qb[u].w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t a4[4] = {fa[2 * j], fb[2 * j], fa[2 * j + 1], fb[2 * j + 1]};
-                mma_bf16_16816(acc[nn], a4, bw[2 * j], bw[2 * j + 1], true);
+            for (int k = 0; k < 4; ++k) {
+                fa[2 * k] = e4m3x2_to_bf16x2(wa[k]);
+                fa[2 * k + 1] = e4m3x2_to_bf16x2(wa[k] >> 16);
+                fb[2 * k] = e4m3x2_to_bf16x2(wb[k]);
+                fb[2 * k + 1] = e4m3x2_to_bf16x2(wb[k] >> 16);
+            }
+#pragma unroll
+            for (int nn = 0; nn < NT; ++nn) {
+                const uint32_t bw[8] = {b0[u][nn].x, b0[u][nn].y, b0[u][nn].z, b0[u][nn].w,
+                                        b1[u][nn].x, b1[u][nn].y, b1[u][nn].z, b1[u][nn].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t a4[4] = {fa[2 * j], fb[2 * j], fa[2 * j + 1], fb[2 * j + 1]};
+                    mma_bf16_16816(acc[nn], a4, bw[2 * j], bw[2 * j + 1], true);
+                }
             }
         }
     }
@@ -184,9 +201,12 @@ __global__ void __launch_bounds__(128) k_fp8_u(const uint8_t* __restrict__ X8, i
         const int64_t tok = t0 + row;
         if (tok >= T) continue;
         float v = 0.f;
-        if (col < r)
-            v = __fmul_rn(fac, ((s_part[0][row][col] + s_part[1][row][col]) + s_part[2][row][col]) +
-                                   s_part[3][row][col]);
+        if (col < r) {
+            v = s_part[0][row][col];
+#pragma unroll
+            for (int w = 1; w < WARPS; ++w) v += s_part[w][row][col];
+            v = __fmul_rn(fac, v);
+        }
         U[tok * ldu + col] = __float2bfloat16_rn(v);
     }
 }

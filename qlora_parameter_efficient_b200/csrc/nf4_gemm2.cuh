@@ -108,7 +108,12 @@ static_assert(kG2StagesA >= kG2StagesB, "B-slot reuse is gated through the A rin
 // group has already observed, so no parity wait can alias.
 static_assert(kG2StagesA % kG2DecGroups == 0, "A-ring depth must be a multiple of the groups");
 constexpr int kG2Threads = 32 * (6 + 4 * kG2DecGroups);
-// FP8: a K step is 128 E4M3 columns (the same 128-byte rows), its codes tile twice as large
+// FP8: a K step is 128 E4M3 columns (the same 128-byte rows), its codes tile twice as large;
+// the deeper A ring (TMA latency) is paid for with a 2-slot decoded-B ring (measured best of
+// 1, 2 or 4 decoder groups and (8, 2), (6, 4), (4, 4) rings).
+#ifndef QLORA_G2_FP8_DEC_GROUPS
+#define QLORA_G2_FP8_DEC_GROUPS 4
+#endif
 #ifndef QLORA_G2_FP8_STAGES_A
 #define QLORA_G2_FP8_STAGES_A 8
 #endif
@@ -116,10 +121,13 @@ constexpr int kG2Threads = 32 * (6 + 4 * kG2DecGroups);
 #define QLORA_G2_FP8_STAGES_B 2
 #endif
 static_assert(QLORA_G2_FP8_STAGES_A >= QLORA_G2_FP8_STAGES_B, "B-slot reuse is gated through the A ring");
-static_assert(QLORA_G2_FP8_STAGES_A % kG2DecGroups == 0, "A-ring depth must be a multiple of the groups");
+static_assert(QLORA_G2_FP8_STAGES_A % QLORA_G2_FP8_DEC_GROUPS == 0,
+              "A-ring depth must be a multiple of the groups");
 
 template <bool FP8 = false>
 struct G2Smem {
+    static constexpr int kGroups = FP8 ? QLORA_G2_FP8_DEC_GROUPS : kG2DecGroups;
+    static constexpr int kThreads = 32 * (6 + 4 * kGroups);
     static constexpr int SA = FP8 ? QLORA_G2_FP8_STAGES_A : kG2StagesA;
     static constexpr int SB = FP8 ? QLORA_G2_FP8_STAGES_B : kG2StagesB;
     static constexpr int kKStep = FP8 ? 128 : 64;  // K columns per step
@@ -178,7 +186,7 @@ struct Gemm2Args {
 __device__ __forceinline__ int g2_part_idx(int c, int g, int lane) { return (c * 8 + g) * 32 + lane; }
 
 template <bool B_MN, bool FP8 = false>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThreads, 1)
     k_nf4_gemm2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmC,
                 const __grid_constant__ CUtensorMap tmAx, const __grid_constant__ CUtensorMap tmBx,
                 const Gemm2Args args) {
@@ -186,6 +194,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
     using L = G2Smem<FP8>;
     constexpr int SA = L::SA;
     constexpr int SB = L::SB;
+    constexpr int NG = L::kGroups;          // decoder groups of 4 warps
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -235,6 +244,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
         } else {
             tile = half_tile;
             ks = hb + (git - full_iters);
+        }
+    };
+
+    // Decoder cursor: (tile, K step) of the steps git = grp, grp + NG, ... of one decoder group,
+    // advanced incrementally (no integer division per step).
+    struct Cur {
+        int git, tile, it;
+    };
+    auto cur_at = [&](int git) {
+        Cur c;
+        c.git = git;
+        c.tile = 0;
+        c.it = 0;
+        if (git < total_iters) step_of(git, c.tile, c.it);
+        return c;
+    };
+    auto cur_next = [&](Cur& c) {
+        c.git += NG;
+        if (c.git >= full_iters) {
+            c.tile = half_tile;
+            c.it = hb + (c.git - full_iters);
+            return;
+        }
+        c.it += NG;
+        while (c.it >= iters_per_tile) {
+            c.it -= iters_per_tile;
+            c.tile += npairs;
         }
     };
 
@@ -505,14 +541,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             uint32_t q8[2];
             float c2[2];
         };
-        auto fetch = [&](int git, Pre& pr) {
+        int row_tile = -1;
+        int64_t wrow = 0;
+        Cur fc = cur_at(grp);                 // the next step to fetch scales for
+        auto fetch = [&](Pre& pr) {
             pr.nv = 0;
-            if (git >= total_iters) return;
-            int tile, it;
-            step_of(git, tile, it);
-            if (it >= args.k_steps) return;
-            const int64_t wrow = static_cast<int64_t>(tile / args.m_tiles) * 256 + rank * 128 + j;
-            const int64_t wblk = 2 * static_cast<int64_t>(it);
+            const Cur c = fc;
+            cur_next(fc);
+            if (c.git >= total_iters || c.it >= args.k_steps) return;
+            if (c.tile != row_tile) {
+                row_tile = c.tile;
+                wrow = static_cast<int64_t>(c.tile / args.m_tiles) * 256 + rank * 128 + j;
+            }
+            const int64_t wblk = 2 * static_cast<int64_t>(c.it);
             if (wrow >= args.nf4_rows || wblk >= args.nf4_bpr) return;
             pr.nv = wblk + 1 < args.nf4_bpr ? 2 : 1;
             const int64_t b0 = wrow * args.nf4_bpr + wblk;
@@ -546,16 +587,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
         };
         uint64_t* arrive_bar = rank == 0 ? ready : dec_done;
         Pre nxt;
-        fetch(grp, nxt);
+        fetch(nxt);
         bool have = false;          // dec[] holds step `git` (decoded ahead)
-        for (int git = grp; git < total_iters; git += kG2DecGroups) {
+        Cur mc = cur_at(grp);
+        for (int git = grp; git < total_iters; git += NG) {
             const int s = git % SA;
-            int tile_unused, it;
-            step_of(git, tile_unused, it);
-            const bool main_step = it < args.k_steps;
+            const bool main_step = mc.it < args.k_steps;
+            Cur nc = mc;
+            cur_next(nc);
             if (!have) {
                 const Pre cur = nxt;
-                fetch(git + kG2DecGroups, nxt);
+                fetch(nxt);
                 if (!mbar_wait_warp(&full[s], (git / SA) & 1, abort, args.wait_ns)) {
                     fail();
                     break;
@@ -577,12 +619,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&arrive_bar[s]);
             have = false;
-            const int gn = git + kG2DecGroups;
-            int tile_gn = 0, it_gn = 0;
-            if (gn < total_iters) step_of(gn, tile_gn, it_gn);
-            if (gn < total_iters && it_gn < args.k_steps) {
+            const int gn = git + NG;
+            if (gn < total_iters && nc.it < args.k_steps) {
                 const Pre cur = nxt;
-                fetch(gn + kG2DecGroups, nxt);
+                fetch(nxt);
                 if (!mbar_wait_warp(&full[gn % SA], (gn / SA) & 1, abort, args.wait_ns)) {
                     fail();
                     break;
@@ -590,6 +630,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
                 decode_into_regs(gn, cur);
                 have = true;
             }
+            mc = nc;
         }
     } else {
         // -------------------------------------------------------------- NF4 decoders
@@ -603,11 +644,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             row_in_tile = j;                // weight row within this CTA's 128
             blk_col_off = 0;
         }
-        auto block_at = [&](int git) -> int64_t {
-            int tile, it;
-            step_of(git, tile, it);
-            if (it >= args.k_steps) return -1;
-            const int n0 = (tile / args.m_tiles) * 256 + static_cast<int>(rank) * 128;
+        // block of the step at the fetch cursor (then advanced); -1 outside the weight
+        Cur fc = cur_at(grp);
+        int row_tile = -1, n0 = 0;
+        auto next_block = [&]() -> int64_t {
+            const Cur c = fc;
+            cur_next(fc);
+            if (c.git >= total_iters || c.it >= args.k_steps) return -1;
+            if (c.tile != row_tile) {
+                row_tile = c.tile;
+                n0 = (c.tile / args.m_tiles) * 256 + static_cast<int>(rank) * 128;
+            }
+            const int it = c.it;
             int64_t wrow, wblk;
             if (B_MN) {
                 wrow = static_cast<int64_t>(it) * 64 + row_in_tile;
@@ -644,7 +692,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
                 for (int ch = 0; ch < 8; ++ch) dec[ch] = make_uint4(0, 0, 0, 0);
             }
         };
-        int64_t blk_nxt = grp < total_iters ? block_at(grp) : -1;
+        int64_t blk_nxt = next_block();
         uint32_t q8_nxt = 0;
         float c2_nxt = 0.f;
         if (blk_nxt >= 0) {
@@ -652,18 +700,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             c2_nxt = __ldg(args.c2 + (blk_nxt >> 8));
         }
         bool have = false;          // dec[] holds step `git` (decoded ahead)
-        for (int git = grp; git < total_iters; git += kG2DecGroups) {
+        Cur mc = cur_at(grp);
+        for (int git = grp; git < total_iters; git += NG) {
             const int s = git % SA;
-            int tile_unused, it;
-            step_of(git, tile_unused, it);
-            const bool main_step = it < args.k_steps;
+            const bool main_step = mc.it < args.k_steps;
+            Cur nc = mc;
+            cur_next(nc);
             if (!have) {
                 // (first step, or after an adapter step) decode now
                 const int64_t blk = blk_nxt;
                 Nf4Planes p{};
                 if (blk >= 0) p = nf4_make_planes(nf4_block_scale(q8_nxt, c2_nxt));
-                const int gn = git + kG2DecGroups;
-                blk_nxt = gn < total_iters ? block_at(gn) : -1;
+                blk_nxt = next_block();
                 if (blk_nxt >= 0) {
                     q8_nxt = __ldg(args.absmax_q + blk_nxt);
                     c2_nxt = __ldg(args.c2 + (blk_nxt >> 8));
@@ -691,15 +739,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
             if (lane == 0) mbar_arrive(&arrive_bar[s]);
             // decode the next handled step ahead, as soon as its codes have landed
             have = false;
-            const int gn = git + kG2DecGroups;
-            int tile_gn = 0, it_gn = 0;
-            if (gn < total_iters) step_of(gn, tile_gn, it_gn);
-            if (gn < total_iters && it_gn < args.k_steps) {
+            const int gn = git + NG;
+            if (gn < total_iters && nc.it < args.k_steps) {
                 const int64_t blk = blk_nxt;
                 Nf4Planes p{};
                 if (blk >= 0) p = nf4_make_planes(nf4_block_scale(q8_nxt, c2_nxt));
-                const int g2 = gn + kG2DecGroups;
-                blk_nxt = g2 < total_iters ? block_at(g2) : -1;
+                blk_nxt = next_block();
                 if (blk_nxt >= 0) {
                     q8_nxt = __ldg(args.absmax_q + blk_nxt);
                     c2_nxt = __ldg(args.c2 + (blk_nxt >> 8));
@@ -711,6 +756,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
                 decode_into_regs(gn, blk, p);
                 have = true;
             }
+            mc = nc;
         }
     }
 

@@ -540,7 +540,8 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
         return QLORA_ERR_CUDA;
     const bool ev = g_ev_start && g_ev_stop;
     if (ev) cudaEventRecord(g_ev_start, st);
-    if (launch_pdl(kern, dim3(2 * pairs), dim3(kG2Threads), smem, st, ta, tc, tax, tbx, g) !=
+    const int threads = fp8 ? G2Smem<true>::kThreads : G2Smem<false>::kThreads;
+    if (launch_pdl(kern, dim3(2 * pairs), dim3(threads), smem, st, ta, tc, tax, tbx, g) !=
         cudaSuccess)
         return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
@@ -1037,10 +1038,10 @@ qlora_status qlora_linear_fwd_fp8(const qlora_nf4* w, const uint8_t* X8, int64_t
     const dim3 ug(static_cast<unsigned>(cdiv(T, 16)));
     const int di = static_cast<int>(d_in);
     cudaError_t e;
-    if (r <= 16) e = launch_pdl(k_fp8_u<2>, ug, dim3(128), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
-    else if (r <= 32) e = launch_pdl(k_fp8_u<4>, ug, dim3(128), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
-    else if (r <= 64) e = launch_pdl(k_fp8_u<8>, ug, dim3(128), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
-    else e = launch_pdl(k_fp8_u<16>, ug, dim3(128), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
+    if (r <= 16) e = launch_pdl(k_fp8_u<2, 8, 4>, ug, dim3(256), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
+    else if (r <= 32) e = launch_pdl(k_fp8_u<4, 8, 2>, ug, dim3(256), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
+    else if (r <= 64) e = launch_pdl(k_fp8_u<8, 8, 1>, ug, dim3(256), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
+    else e = launch_pdl(k_fp8_u<16, 4, 1>, ug, dim3(128), 0, stream, X8, T, di, Ab, r, s, w_scale, u, RP);
     if (e != cudaSuccess) return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     return nf4_gemm(false, w, X8, T, u, b_src, RP, r, b_ld, H, at<void>(ws, p.g2), err, stream, nullptr,
