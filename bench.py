@@ -678,6 +678,8 @@ def extra_rows(q, torch, S, dev, peaks, args):
     kev = []
     for i in range(12):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        e1.record()
         q.set_gemm_events(e0, e1)
         q.qlora_linear_fwd_fp8(wl[i % 4], X8, xs, wsc[i % 4], A, B, c["alpha"], H=H, ws=ws)
         q.set_gemm_events(None, None)
@@ -733,9 +735,9 @@ def extra_rows(q, torch, S, dev, peaks, args):
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one k_nf4_gemm2<0> launch at this workload,
 # from the ncu capture summarised in profiles/nf4_fused_gemm_q_proj_4096x4096_T4096.md
-# (43.73 MB read + 15.49 MB written; H is still partly in L2 when the kernel ends).  Set to
+# (43.27 MB read + 15.34 MB written; H is still partly in L2 when the kernel ends).  Set to
 # None whenever the kernel changes until it is captured again.
-GEMM_FWD_DRAM_BYTES = None
+GEMM_FWD_DRAM_BYTES = 43270400 + 15336960
 
 
 def main():
