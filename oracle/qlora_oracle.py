@@ -52,6 +52,10 @@ What it computes, and where each step is defined:
   activations on Hopper and Blackwell).  The pages name the formats only; the
   byte layout is the OCP 8-bit floating-point definition and the scaling,
   rounding and operand choices are reading R25.
+* FP8 backward: the E5M2 upstream gradient (same section's E5M2) and the
+  saved E4M3 activation in the three gradient equations of the Mathematical
+  Foundations page, section "Gradient Dynamics and Backpropagation Mechanics";
+  reading R26.
 
 Where the pages are silent or garbled the oracle takes the readings listed as
 R1..R19 in the design notes; each is named where it is applied.
@@ -448,6 +452,57 @@ def nf4_dequantize_e4m3(codes, absmax_q, c2, d_out: int, d_in: int, w_scale: flo
     return e4m3_encode((w32 * np.float32(w_scale)).astype(np.float32))
 
 
+E5M2_MAX = 57344.0
+
+
+def e5m2_decode(code) -> np.ndarray:
+    """Value (fp64) of each E5M2 byte, the OCP 8-bit float with the wider range
+    (the gradient format): bit 7 sign, bits 6..2 exponent with bias 15, bits
+    1..0 mantissa.  Exponent 0 holds the subnormals m/4 * 2^-14; exponent 31
+    is infinity (mantissa 0) or NaN.  Largest finite 57344."""
+    c = np.asarray(code, np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 2) & 31
+    m = (c & 3).astype(np.float64)
+    mag = np.where(e == 0, m / 4.0 * 2.0 ** -14, (1.0 + m / 4.0) * np.exp2(e - 15.0))
+    mag = np.where(e == 31, np.where(m == 0, np.inf, np.nan), mag)
+    return sign * mag
+
+
+def e5m2_encode(x) -> np.ndarray:
+    """E5M2 byte of each finite fp32 value: nearest finite value, ties to the
+    even code, magnitudes at or beyond 57344 saturated to 57344; sign bit the
+    input's."""
+    a = np.abs(np.asarray(x, np.float32).astype(np.float64))
+    neg = np.signbit(np.asarray(x, np.float32))
+    mags = e5m2_decode(np.arange(124, dtype=np.uint8))      # codes 0x00..0x7B, increasing
+    hi = np.minimum(np.searchsorted(mags, a, side="left"), 123)
+    lo = np.maximum(hi - 1, 0)
+    dlo = a - mags[lo]
+    dhi = mags[hi] - a
+    pick = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
+    pick = np.where(a >= E5M2_MAX, 123, pick)
+    return (pick.astype(np.uint8) | np.where(neg, 0x80, 0).astype(np.uint8)).astype(np.uint8)
+
+
+def fp8_pow2_scale_e5m2(amax: float) -> float:
+    """The gradient's scale sigma = 2^(15 - ceil(log2 amax)): amax * sigma in
+    (2^14, 2^15], below the E5M2 limit; 1 for amax = 0; exponent in [-126, 126]."""
+    if not amax > 0.0:
+        return 1.0
+    m, e = math.frexp(amax)
+    c = e - 1 if m == 0.5 else e
+    return math.ldexp(1.0, min(max(15 - c, -126), 126))
+
+
+def fp8_quantize_grad(dH):
+    """(dH8, sigma_g): dH8 = E5M2(fl32(dH * sigma_g)), sigma_g = fp8_pow2_scale_e5m2(max|dH|)."""
+    G32 = np.asarray(dH, np.float32)
+    amax = float(np.max(np.abs(G32))) if G32.size else 0.0
+    sig = fp8_pow2_scale_e5m2(amax)
+    return e5m2_encode((G32 * np.float32(sig)).astype(np.float32)), sig
+
+
 def lora_forward_fp8(X8, x_scale, W8, w_scale, A, B, alpha, r):
     """Forward of the adapted layer with E4M3 activations and weights (fp64):
 
@@ -462,6 +517,28 @@ def lora_forward_fp8(X8, x_scale, W8, w_scale, A, B, alpha, r):
     A = np.asarray(A, np.float64)
     B = np.asarray(B, np.float64)
     return (Xv @ Wv.T) / (float(x_scale) * float(w_scale)) + lora_scale(alpha, r) * ((Xt @ A.T) @ B.T)
+
+
+def lora_backward_fp8(X8, x_scale, dH8, g_scale, W8, w_scale, A, B, alpha, r):
+    """Backward of the adapted layer from the saved E4M3 activation and the E5M2
+    upstream gradient (fp64), returning (dX, dA, dB):
+
+        X~ = X8 / sigma_x,  dH~ = dH8 / sigma_g,  G = dH~ B,  U = X~ A^T
+        dX = (dH8 W8) / (sigma_g sigma_w) + s G A      (the FP8 contraction)
+        dA = s G^T X~,      dB = s dH~^T U
+
+    the page's three gradient equations with the stored FP8 tensors in place of
+    X and dH, and the E4M3 weight of the forward's FP8 contraction in dX."""
+    Xt = e4m3_decode(X8) / float(x_scale)
+    Gv = e5m2_decode(dH8)
+    dHt = Gv / float(g_scale)
+    Wv = e4m3_decode(W8)
+    A = np.asarray(A, np.float64)
+    B = np.asarray(B, np.float64)
+    s = lora_scale(alpha, r)
+    G = dHt @ B
+    dX = (Gv @ Wv) / (float(g_scale) * float(w_scale)) + s * (G @ A)
+    return dX, s * (G.T @ Xt), s * (dHt.T @ (Xt @ A.T))
 
 
 # ----------------------------------------------------------------------------

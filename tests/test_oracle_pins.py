@@ -579,6 +579,133 @@ def test_fp8_weight_decode():
                           np.full_like(W8, 0x80))
 
 
+# ---------------------------------------------------------------- FP8 backward (R26)
+
+
+def brute_e5m2(x):
+    vals = [(c, O.e5m2_decode(np.uint8(c)).item()) for c in range(256)
+            if ((c >> 2) & 31) != 31]
+    out = []
+    for v in np.asarray(x, np.float64).reshape(-1):
+        best = None
+        for c, cv in vals:
+            if (c & 0x80) != (0x80 if math.copysign(1.0, v) < 0 else 0):
+                continue
+            d = abs(v - cv)
+            if best is None or d < best[0] or (d == best[0] and c % 2 == 0):
+                best = (d, c)
+        out.append(best[1])
+    return np.array(out, np.uint8)
+
+
+def test_e5m2_format_constants():
+    # OCP 8-bit floating point, E5M2: largest finite 57344, smallest normal 2^-14, smallest
+    # subnormal 2^-16, 1.0 = 0x3C, infinity 0x7C, NaN 0x7D..0x7F.
+    d = O.e5m2_decode
+    assert d(np.uint8(0x7B)) == 57344.0 and d(np.uint8(0xFB)) == -57344.0
+    assert d(np.uint8(0x04)) == 2.0 ** -14 and d(np.uint8(0x01)) == 2.0 ** -16
+    assert d(np.uint8(0x3C)) == 1.0 and d(np.uint8(0x40)) == 2.0
+    assert np.isinf(d(np.uint8(0x7C))) and all(np.isnan(d(np.uint8(c))) for c in (0x7D, 0x7E, 0x7F))
+    pos = d(np.arange(124, dtype=np.uint8))
+    assert np.all(np.diff(pos) > 0)
+    assert np.sum(np.isfinite(d(np.arange(256, dtype=np.uint8)))) == 248
+
+
+def e5m2_probe_values():
+    rng = np.random.default_rng(13)
+    mags = np.exp2(rng.uniform(-18, 17, 2000))
+    x = mags * rng.choice([-1.0, 1.0], mags.size)
+    pos = O.e5m2_decode(np.arange(124, dtype=np.uint8))
+    mids = 0.5 * (pos[1:] + pos[:-1])
+    extra = np.array([0.0, -0.0, 57344.0, 61439.0, 61440.0, 1e9, -1e9, 2.0 ** -17, -2.0 ** -17])
+    return np.concatenate([x, mids, -mids, extra]).astype(np.float32)
+
+
+def check_e5m2_encode(enc):
+    x = e5m2_probe_values()
+    return int(np.sum(enc(x) != brute_e5m2(x)))
+
+
+def test_e5m2_encode_against_brute_force():
+    assert check_e5m2_encode(O.e5m2_encode) == 0
+
+
+def test_e5m2_round_trip_error_bound_and_scale():
+    c = np.array([c for c in range(256) if ((c >> 2) & 31) != 31], np.uint8)
+    assert np.array_equal(O.e5m2_encode(O.e5m2_decode(c).astype(np.float32)), c)
+    rng = np.random.default_rng(5)
+    x = (np.exp2(rng.uniform(-14, 15.8, 20000)) * rng.choice([-1, 1], 20000)).astype(np.float32)
+    err = np.abs(O.e5m2_decode(O.e5m2_encode(x)) - x.astype(np.float64))
+    assert np.all(err <= 2.0 ** -3 * np.abs(x))          # 2 mantissa bits: half an ulp
+    for amax in [1e-3, 0.7, 1.0, 3.0, 6e4, 2.0 ** -30]:
+        sig = O.fp8_pow2_scale_e5m2(amax)
+        assert math.frexp(sig)[0] == 0.5 and 2.0 ** 14 < amax * sig <= 2.0 ** 15
+    G = np.random.default_rng(2).standard_normal((9, 70)).astype(np.float32) * 1e-3
+    G8, sg = O.fp8_quantize_grad(G)
+    big = np.abs(G) * sg >= 2.0 ** -14
+    assert np.all(np.abs(O.e5m2_decode(G8) / sg - G)[big] <= 2.0 ** -3 * np.abs(G)[big])
+
+
+def fp8_bwd_case(T=4, d=6, k=128, r=2, seed=31):
+    W, codes, q8, c2, X, A, B = fp8_layer(T=T, d=d, k=k, r=r, seed=seed)
+    dH = (np.random.default_rng(seed + 1).standard_normal((T, d)) * 1e-2).astype(np.float32)
+    X8, sx = O.fp8_quantize_act(X)
+    G8, sg = O.fp8_quantize_grad(dH)
+    sw = O.fp8_weight_scale(c2)
+    W8 = O.nf4_dequantize_e4m3(codes, q8, c2, d, k, sw)
+    W32 = O.nf4_dequantize(codes, q8, c2, d, k, out="f32").astype(np.float64)
+    return X, dH, X8, sx, G8, sg, W8, sw, W32, A, B
+
+
+def check_fp8_backward_loops(bwd):
+    X, dH, X8, sx, G8, sg, W8, sw, W32, A, B = fp8_bwd_case()
+    T, k = X.shape
+    d, r = B.shape
+    alpha = 4.0
+    s = alpha / r
+    dX, dA, dB = bwd(X8, sx, G8, sg, W8, sw, A, B, alpha, r)
+    xv = lambda t, j: O.e4m3_decode(X8[t, j]).item() / sx
+    gv = lambda t, i: O.e5m2_decode(G8[t, i]).item() / sg
+    wv = lambda i, j: O.e4m3_decode(W8[i, j]).item() / sw
+    G = [[sum(gv(t, i) * B[i, q] for i in range(d)) for q in range(r)] for t in range(T)]
+    U = [[sum(xv(t, j) * A[q, j] for j in range(k)) for q in range(r)] for t in range(T)]
+    rdX = np.array([[sum(gv(t, i) * wv(i, j) for i in range(d)) + s * sum(G[t][q] * A[q, j] for q in range(r))
+                     for j in range(k)] for t in range(T)])
+    rdA = np.array([[s * sum(G[t][q] * xv(t, j) for t in range(T)) for j in range(k)] for q in range(r)])
+    rdB = np.array([[s * sum(gv(t, i) * U[t][q] for t in range(T)) for q in range(r)] for i in range(d)])
+    return max(rel(dX, rdX), rel(dA, rdA), rel(dB, rdB))
+
+
+def check_fp8_backward_bound(bwd):
+    """The FP8 backward against the exact backward of the same layer, elementwise within the
+    E4M3 / E5M2 rounding bounds (x~ = x + e_x, |e_x| <= 2^-4|x| + 2^-10/sigma_x; likewise
+    |e_g| <= 2^-3|g| + 2^-17/sigma_g and the weight)."""
+    X, dH, X8, sx, G8, sg, W8, sw, W32, A, B = fp8_bwd_case(T=7, d=9, k=192, r=3, seed=8)
+    alpha, r = 6.0, 3
+    s = alpha / r
+    dX, dA, dB = bwd(X8, sx, G8, sg, W8, sw, A, B, alpha, r)
+    eX, eA, eB = O.lora_backward(W32, X, dH, A, B, alpha, r)
+    aX, aG, aW = np.abs(X.astype(np.float64)), np.abs(dH.astype(np.float64)), np.abs(W32)
+    Ex = 2.0 ** -4 * aX + 2.0 ** -10 / sx
+    Eg = 2.0 ** -3 * aG + 2.0 ** -17 / sg
+    Ew = 2.0 ** -4 * aW + 2.0 ** -10 / sw
+    aA, aB = np.abs(A), np.abs(B)
+    bX = (aG + Eg) @ Ew + Eg @ aW + s * (Eg @ aB) @ aA
+    Gt = (aG + Eg) @ aB
+    bA = s * (Gt.T @ Ex + (Eg @ aB).T @ aX)
+    bB = s * ((aG + Eg).T @ (Ex @ aA.T) + Eg.T @ (aX @ aA.T))
+    return max(float(np.max(np.abs(dX - eX) - bX - 1e-12)), float(np.max(np.abs(dA - eA) - bA - 1e-12)),
+               float(np.max(np.abs(dB - eB) - bB - 1e-12)))
+
+
+def test_fp8_backward_against_loops():
+    assert check_fp8_backward_loops(O.lora_backward_fp8) < 1e-12
+
+
+def test_fp8_backward_within_rounding_bound_of_exact():
+    assert check_fp8_backward_bound(O.lora_backward_fp8) <= 0.0
+
+
 # ---------------------------------------------------------------- mutants
 
 
@@ -677,6 +804,34 @@ def test_pins_catch_planted_mistakes():
     def fwd8_transposed(X8, sx, W8, sw, A, B, a, r):
         H = O.lora_forward_fp8(X8, sx, W8, sw, A, B, a, r)
         return H[::-1]
+
+    def enc5_ties_away(x):
+        a = np.abs(np.asarray(x, np.float32).astype(np.float64))
+        pos = O.e5m2_decode(np.arange(124, dtype=np.uint8))
+        hi = np.minimum(np.searchsorted(pos, a), 123)
+        lo = np.maximum(hi - 1, 0)
+        pick = np.where(a - pos[lo] < pos[hi] - a, lo, hi)
+        pick = np.where(a >= 57344.0, 123, pick)
+        return (pick.astype(np.uint8) | np.where(np.signbit(np.asarray(x, np.float32)), 0x80, 0)).astype(np.uint8)
+
+    assert check_e5m2_encode(enc5_ties_away) > 0
+
+    def bwd8_no_gscale(X8, sx, G8, sg, W8, sw, A, B, a, r):
+        dX, dA, dB = O.lora_backward_fp8(X8, sx, G8, sg, W8, sw, A, B, a, r)
+        return dX * sg, dA, dB
+
+    def bwd8_scaled_x_in_dA(X8, sx, G8, sg, W8, sw, A, B, a, r):
+        dX, dA, dB = O.lora_backward_fp8(X8, sx, G8, sg, W8, sw, A, B, a, r)
+        return dX, dA * sx, dB
+
+    def bwd8_no_adapter_in_dX(X8, sx, G8, sg, W8, sw, A, B, a, r):
+        dX, dA, dB = O.lora_backward_fp8(X8, sx, G8, sg, W8, sw, A, B, a, r)
+        G = (O.e5m2_decode(G8) / sg) @ np.asarray(B)
+        return dX - s(a, r) * (G @ np.asarray(A)), dA, dB
+
+    for m in (bwd8_no_gscale, bwd8_scaled_x_in_dA, bwd8_no_adapter_in_dX):
+        assert check_fp8_backward_loops(m) > 1e-3
+        assert check_fp8_backward_bound(m) > 0.0
 
     for m in (fwd8_no_wscale, fwd8_scaled_act_in_adapter, fwd8_transposed):
         assert check_fp8_forward_bound(m) > 0.0
