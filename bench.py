@@ -190,7 +190,7 @@ def run_gpu(args):
         return run_decode_only(args, q, qb, S, torch, dev)
     if args.only == "multi":
         return run_multi_only(args, q, qb, torch, dev)
-    if args.only == "fp8":
+    if args.only in ("fp8", "fp8bwd"):
         return run_fp8_only(args, q, qb, S, torch, dev)
     if world > 1:
         import datetime
@@ -496,21 +496,45 @@ def run_fp8_only(args, q, qb, S, torch, dev):
     qb.build_library()
     q.load()
     c, wl, wsc, Xb, X8, xs, A, B, H, ws = make_fp8_workload(q, S, torch, dev)
+    if args.only == "fp8bwd":
+        G8, gs, dX, dA, dB, wsb = make_fp8_bwd_buffers(q, torch, dev, c)
+
+        def call(i):
+            q.qlora_linear_bwd_fp8(wl[i % 4], X8, xs, G8, gs, wsc[i % 4], A, B, c["alpha"], dX=dX, dA=dA,
+                                   dB=dB, ws=wsb)
+    else:
+        def call(i):
+            q.qlora_linear_fwd_fp8(wl[i % 4], X8, xs, wsc[i % 4], A, B, c["alpha"], H=H, ws=ws)
     W = max(3, args.warmup)
     for i in range(W):
-        q.qlora_linear_fwd_fp8(wl[i % 4], X8, xs, wsc[i % 4], A, B, c["alpha"], H=H, ws=ws)
+        call(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for i in range(args.steps):
-        q.qlora_linear_fwd_fp8(wl[i % 4], X8, xs, wsc[i % 4], A, B, c["alpha"], H=H, ws=ws)
+        call(i)
     e1.record()
     torch.cuda.synchronize()
     err = q.get_device_error()
-    print(json.dumps({"only": "fp8", "ms_per_call": e0.elapsed_time(e1) / args.steps,
+    print(json.dumps({"only": args.only, "ms_per_call": e0.elapsed_time(e1) / args.steps,
                       "device_error": err,
-                      "workload": "4096x4096 NF4, r=16, T=4096, E4M3 activation"}), flush=True)
+                      "workload": "4096x4096 NF4, r=16, T=4096, E4M3 activation"
+                                  + (", E5M2 gradient" if args.only == "fp8bwd" else "")}), flush=True)
     return 0 if err == 0 else 1
+
+
+def make_fp8_bwd_buffers(q, torch, dev, c, seed=23):
+    """E5M2 upstream gradient of the q_proj workload and the FP8 backward's outputs and workspace."""
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    dH = torch.randn((c["T"], c["d_out"]), generator=gen, device=dev).to(torch.bfloat16)
+    G8, gs = q.fp8_quantize_grad(dH)
+    dX = torch.empty((c["T"], c["d_in"]), dtype=torch.bfloat16, device=dev)
+    dA = torch.empty((c["r"], c["d_in"]), dtype=torch.float32, device=dev)
+    dB = torch.empty((c["d_out"], c["r"]), dtype=torch.float32, device=dev)
+    wsb = torch.empty(q.workspace_bytes(q.OP_BWD_FP8, q.BF16, c["T"], c["d_out"], c["d_in"], c["r"]),
+                      dtype=torch.uint8, device=dev)
+    return G8, gs, dX, dA, dB, wsb
 
 
 def _graph_time(torch, calls, reps=20):
@@ -692,11 +716,32 @@ def extra_rows(q, torch, S, dev, peaks, args):
     fl = flops_fwd(c["T"], c["d_out"], c["d_in"], c["r"])
     tc8 = 2 * tc
     qbytes = 3 * c["T"] * c["d_in"]
+    # the FP8 backward on the same workload (E5M2 gradient; dX on FP8 tensor cores, dA and dB
+    # from the E4M3 activation and E5M2 gradient dequantized to bf16)
+    G8, gs, dX, dA, dB, wsb = make_fp8_bwd_buffers(q, torch, dev, c)
+    bcalls = [(lambda w=w, sw=sw: q.qlora_linear_bwd_fp8(w, X8, xs, G8, gs, sw, A, B, c["alpha"], dX=dX, dA=dA,
+                                                         dB=dB, ws=wsb)) for w, sw in zip(wl, wsc)]
+    bmed, _ = _graph_time(torch, bcalls, reps=10)
+    kev = []
+    for i in range(12):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        e1.record()
+        q.set_gemm_events(e0, e1)
+        q.qlora_linear_bwd_fp8(wl[i % 4], X8, xs, G8, gs, wsc[i % 4], A, B, c["alpha"], dX=dX, dA=dA, dB=dB, ws=wsb)
+        q.set_gemm_events(None, None)
+        kev.append((e0, e1))
+    torch.cuda.synchronize()
+    bkus = statistics.median(a.elapsed_time(b) * 1e3 for a, b in kev[4:])
+    bfl = flops_bwd(c["T"], c["d_out"], c["d_in"], c["r"])
+    dxfl = 2 * c["T"] * c["d_out"] * c["d_in"] + 2 * c["T"] * c["r"] * c["d_in"]
     out["fp8_fwd_4096x4096_r16_T4096"] = {
         "fwd_us": med, "tflops": fl / (med * 1e-6) / 1e12, "tc_frac_fp8": fl / (med * 1e-6) / 1e12 / tc8,
         "gemm_us": kus, "gemm_tc_frac_fp8": fl / (kus * 1e-6) / 1e12 / tc8, "fp8_peak_tflops": tc8,
-        "quantize_us": qmed, "quantize_hbm_frac": qbytes / (qmed * 1e-6) / 1e9 / hbm}
-    del wl, wsc, Xb, X8, xs, A, B, H, ws, qws
+        "quantize_us": qmed, "quantize_hbm_frac": qbytes / (qmed * 1e-6) / 1e9 / hbm,
+        "bwd_us": bmed, "bwd_tflops": bfl / (bmed * 1e-6) / 1e12,
+        "dx_gemm_us": bkus, "dx_gemm_tc_frac_fp8": dxfl / (bkus * 1e-6) / 1e12 / tc8}
+    del wl, wsc, Xb, X8, xs, A, B, H, ws, qws, G8, gs, dX, dA, dB, wsb
 
     # ---- AdamW step over the adapters of a 32-layer d = 4096 model with rank 16 on q, k, v, o:
     # 32 * 4 * 16 * (4096 + 4096) = 16.8 M parameters, bf16 params + fp32 master, m, v, grad
@@ -748,11 +793,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--extra", action="store_true", help="also time the other hot-path rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--only", default="step", choices=["step", "fwd", "bwd", "decode", "multi", "fp8"],
+    ap.add_argument("--only", default="step", choices=["step", "fwd", "bwd", "decode", "multi", "fp8", "fp8bwd"],
                     help="time only the forward, only the backward, the decode-size forward "
                          "(11008x4096, r = 64, --tokens T) or the many-adapter forward (4096^2, "
-                         "1024 adapters of rank 16) or the FP8 forward (4096^2, r = 16, T = 4096) "
-                         "alone, for profiling its kernels")
+                         "1024 adapters of rank 16), the FP8 forward or the FP8 backward (4096^2, "
+                         "r = 16, T = 4096) alone, for profiling its kernels")
     ap.add_argument("--tokens", type=int, default=1, help="tokens of the --only decode run")
     args = ap.parse_args()
     if args.impl == "reference":

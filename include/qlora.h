@@ -56,7 +56,8 @@ typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 
 typedef enum {
     QLORA_OP_FWD = 0, QLORA_OP_BWD = 1, QLORA_OP_FWD_BATCHED = 2, QLORA_OP_MERGE = 3,
-    QLORA_OP_FWD_MULTI = 4, QLORA_OP_DORA_FWD = 5, QLORA_OP_FWD_FP8 = 6, QLORA_OP_FP8_QUANT = 7
+    QLORA_OP_FWD_MULTI = 4, QLORA_OP_DORA_FWD = 5, QLORA_OP_FWD_FP8 = 6, QLORA_OP_FP8_QUANT = 7,
+    QLORA_OP_BWD_FP8 = 8
 } qlora_op;
 
 /* Stored NF4 weight.  Block size 64 and group size 256 are fixed.
@@ -262,6 +263,31 @@ qlora_status qlora_linear_fwd_fp8(const qlora_nf4* w, const uint8_t* X8, int64_t
                                   const float* x_scale, const float* w_scale, const void* A,
                                   const void* B, int32_t r, float alpha, void* H, void* ws,
                                   size_t ws_bytes, cudaStream_t stream);
+
+/* dH8[n] = E5M2(fl32(dH[i] * sigma_g)) (round to nearest even, saturating at 57344) and
+ * *scale = sigma_g = 2^(15 - ceil(log2 max|dH|)), for the bf16 upstream gradient of n >= 1
+ * elements: the wider-range FP8 format of [UH] "1.3 ..." for gradients.  E5M2 is the OCP 8-bit
+ * float with 5 exponent bits (bias 15) and 2 mantissa bits.  Bit-exact.  ws as for
+ * qlora_fp8_quantize.                                                                          */
+qlora_status qlora_fp8_quantize_grad(const void* dH, int64_t n, uint8_t* dH8, float* scale, void* ws,
+                                     size_t ws_bytes, cudaStream_t stream);
+
+/* Backward from the saved E4M3 activation X8 (scale *x_scale) and the E5M2 upstream gradient
+ * dH8[T, d_out] (scale *g_scale), the three gradient equations of [MF] "Gradient Dynamics and
+ * Backpropagation Mechanics" with X~ = X8 / sigma_x and dH~ = dH8 / sigma_g in place of X, dH:
+ *   G = dH~ B,  dX = bf16( (dH8 W8) / (sigma_g sigma_w) + s G A ),  dA = s G^T X~,
+ *   dB = s dH~^T (X~ A^T),
+ * W8 the weight decoded to E4M3 as in qlora_linear_fwd_fp8.  dX's weight product runs on
+ * kind::f8f6f4 tensor cores (E5M2 x E4M3); G, U, dA, dB on bf16 tensor cores from X~, dH~
+ * (exact bf16 copies in the workspace).  dX bf16 (nullable: skipped), dA, dB fp32;
+ * QLORA_BWD_ACCUMULATE adds into dA, dB.  Needs d_out % 16 == 0 (the E5M2 rows are d_out bytes
+ * and are read by TMA), else QLORA_ERR_UNSUPPORTED with nothing launched.
+ * ws >= qlora_workspace_bytes(QLORA_OP_BWD_FP8, QLORA_BF16, T, d_out, d_in, r).              */
+qlora_status qlora_linear_bwd_fp8(const qlora_nf4* w, const uint8_t* X8, const float* x_scale,
+                                  const uint8_t* dH8, const float* g_scale, const float* w_scale,
+                                  int64_t T, const void* A, const void* B, int32_t r, float alpha,
+                                  void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                                  uint32_t flags, cudaStream_t stream);
 
 /* Size of the device scratch array behind qlora_linear_fwd_noalloc (bytes per GPU). */
 #define QLORA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

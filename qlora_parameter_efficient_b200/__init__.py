@@ -23,14 +23,14 @@ STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",
           3: "QLORA_ERR_CUDA", 4: "QLORA_ERR_TIMEOUT", 5: "QLORA_ERR_DEVICE"}
 F32, BF16 = 0, 1
 OP_FWD, OP_BWD, OP_FWD_BATCHED, OP_MERGE, OP_FWD_MULTI, OP_DORA_FWD = 0, 1, 2, 3, 4, 5
-OP_FWD_FP8, OP_FP8_QUANT = 6, 7
+OP_FWD_FP8, OP_FP8_QUANT, OP_BWD_FP8 = 6, 7, 8
 
 # Every symbol include/qlora.h declares.
 EXPORTS = ["qlora_nf4_sizes", "qlora_nf4_levels", "nf4_quantize", "nf4_dequantize",
            "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "lora_merge",
            "qlora_linear_bwd_ex", "qlora_adamw_step", "qlora_prefetch", "qlora_dora_fwd",
            "qlora_dora_row_norms", "qlora_fp8_quantize", "qlora_fp8_weight_scale",
-           "qlora_linear_fwd_fp8",
+           "qlora_linear_fwd_fp8", "qlora_fp8_quantize_grad", "qlora_linear_bwd_fp8",
            "qlora_linear_fwd_batched", "qlora_linear_fwd_multi", "qlora_linear_fwd_noalloc",
            "qlora_get_device_error",
            "qlora_selftest_wait_timeout", "qlora_set_gemm_events", "qlora_launch_count",
@@ -86,6 +86,9 @@ def load() -> ctypes.CDLL:
         "qlora_fp8_quantize": ([vp, i64, vp, vp, vp, sz, vp], ctypes.c_int),
         "qlora_fp8_weight_scale": ([pnf4, vp, vp], ctypes.c_int),
         "qlora_linear_fwd_fp8": ([pnf4, vp, i64, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_fp8_quantize_grad": ([vp, i64, vp, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_linear_bwd_fp8": ([pnf4, vp, vp, vp, vp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, sz,
+                                  ctypes.c_uint32, vp], ctypes.c_int),
         "qlora_linear_fwd_noalloc": ([pnf4, vp, i64, vp, vp, i32, f32, ctypes.c_int, vp, vp, vp], ctypes.c_int),
         "qlora_get_device_error": ([vp], ctypes.c_int),
         "qlora_selftest_wait_timeout": ([ctypes.c_uint64, vp], ctypes.c_int),
@@ -340,6 +343,45 @@ def qlora_linear_fwd_fp8(w: NF4Weight, X8, x_scale, w_scale, A, B, alpha, H=None
         ctypes.byref(c), _ptr(X8), T, _ptr(x_scale), _ptr(w_scale), _ptr(A), _ptr(B), r, float(alpha),
         _ptr(H), _ptr(ws), ws.numel(), _stream(stream)))
     return H
+
+
+def fp8_quantize_grad(dH, dH8=None, scale=None, ws=None, stream=None):
+    """E5M2 bytes of a bf16 gradient with its power-of-two scale: (dH8 uint8, scale fp32[1])."""
+    torch = _torch()
+    _contig(dH, dH8)
+    if dH.dtype != torch.bfloat16:
+        raise TypeError("fp8_quantize_grad takes a bf16 tensor")
+    if dH8 is None:
+        dH8 = torch.empty(dH.shape, dtype=torch.uint8, device=dH.device)
+    if scale is None:
+        scale = torch.empty(1, dtype=torch.float32, device=dH.device)
+    if ws is None:
+        ws = torch.empty(256, dtype=torch.uint8, device=dH.device)
+    _check("qlora_fp8_quantize_grad", load().qlora_fp8_quantize_grad(
+        _ptr(dH), dH.numel(), _ptr(dH8), _ptr(scale), _ptr(ws), ws.numel(), _stream(stream)))
+    return dH8, scale
+
+
+def qlora_linear_bwd_fp8(w: NF4Weight, X8, x_scale, dH8, g_scale, w_scale, A, B, alpha, dX=None,
+                         dA=None, dB=None, ws=None, accumulate=False, want_dx=True, stream=None):
+    """Backward from the E4M3 activation and the E5M2 gradient: returns (dX bf16, dA, dB fp32)."""
+    torch = _torch()
+    _contig(X8, dH8, A, B, dX, dA, dB)
+    T = X8.shape[0]
+    r = A.shape[0]
+    if dX is None and want_dx:
+        dX = torch.empty((T, w.d_in), dtype=torch.bfloat16, device=X8.device)
+    if dA is None:
+        dA = torch.zeros((r, w.d_in), dtype=torch.float32, device=X8.device)
+    if dB is None:
+        dB = torch.zeros((w.d_out, r), dtype=torch.float32, device=X8.device)
+    ws = _ws(OP_BWD_FP8, BF16, T, w.d_out, w.d_in, r, X8.device, ws)
+    c = w._c()
+    _check("qlora_linear_bwd_fp8", load().qlora_linear_bwd_fp8(
+        ctypes.byref(c), _ptr(X8), _ptr(x_scale), _ptr(dH8), _ptr(g_scale), _ptr(w_scale), T, _ptr(A),
+        _ptr(B), r, float(alpha), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(),
+        BWD_ACCUMULATE if accumulate else 0, _stream(stream)))
+    return dX, dA, dB
 
 
 def prefetch(ptr: int, nbytes: int, to_device: bool, stream=None):

@@ -8,7 +8,8 @@
 //   X8    = E4M3(fl32(x * sigma))         round to nearest even, saturating at 448
 // so amax * sigma lies in (128, 256] and X ~ X8 / sigma.  A power-of-two scale makes every
 // rescaling exact.  The weight's scale sigma_w comes from the largest second-level constant
-// (every decoded weight is L * s_b with |L| <= 1 and s_b <= c2 of its group).
+// (every decoded weight is L * s_b with |L| <= 1 and s_b <= c2 of its group).  The upstream
+// gradient of the backward takes E5M2 (range to 57344) with sigma = 2^(15 - ceil(log2 amax)).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -18,7 +19,8 @@
 
 namespace qlora {
 
-__device__ __forceinline__ float fp8_pow2_scale(float amax) {
+// 2^(top - ceil(log2 amax)); top = 8 (E4M3) or 15 (E5M2)
+__device__ __forceinline__ float fp8_pow2_scale(float amax, int top = 8) {
     if (!(amax > 0.f)) return 1.f;
     const uint32_t b = __float_as_uint(amax);
     const int e = static_cast<int>((b >> 23) & 255u);
@@ -30,7 +32,7 @@ __device__ __forceinline__ float fp8_pow2_scale(float amax) {
     } else {
         c = e - 127 + (m ? 1 : 0);
     }
-    const int k = min(max(8 - c, -126), 126);
+    const int k = min(max(top - c, -126), 126);
     return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
 }
 
@@ -70,12 +72,14 @@ __global__ void __launch_bounds__(256) k_fp8_amax(const __nv_bfloat16* __restric
     if (threadIdx.x == 0 && m > 0.f) atomicMax(amax_bits, __float_as_uint(m));
 }
 
-// X8 = E4M3(fl32(x * sigma)), sigma from the amax; block 0 stores sigma into *scale.
+// X8 = E4M3 (or E5M2) of fl32(x * sigma), sigma from the amax; block 0 stores sigma into *scale.
+template <bool E5M2>
 __global__ void __launch_bounds__(256) k_fp8_quant(const __nv_bfloat16* __restrict__ X, int64_t n,
                                                    const unsigned* __restrict__ amax_bits,
                                                    uint8_t* __restrict__ X8, float* __restrict__ scale) {
     griddep_enter();
-    const float sig = fp8_pow2_scale(__uint_as_float(*amax_bits));
+    constexpr __nv_fp8_interpretation_t kFmt = E5M2 ? __NV_E5M2 : __NV_E4M3;
+    const float sig = fp8_pow2_scale(__uint_as_float(*amax_bits), E5M2 ? 15 : 8);
     if (blockIdx.x == 0 && threadIdx.x == 0) *scale = sig;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     const int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -89,12 +93,57 @@ __global__ void __launch_bounds__(256) k_fp8_quant(const __nv_bfloat16* __restri
             b[k] = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
                 make_float2(__fmul_rn(__uint_as_float(w[k] << 16), sig),
                             __fmul_rn(__uint_as_float(w[k] & 0xFFFF0000u), sig)),
-                __NV_SATFINITE, __NV_E4M3));
+                __NV_SATFINITE, kFmt));
         reinterpret_cast<uint2*>(X8)[i] = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
     }
     for (int64_t i = n8 * 8 + i0; i < n; i += stride)
         X8[i] = static_cast<uint8_t>(
-            __nv_cvt_float_to_fp8(__fmul_rn(__bfloat162float(X[i]), sig), __NV_SATFINITE, __NV_E4M3));
+            __nv_cvt_float_to_fp8(__fmul_rn(__bfloat162float(X[i]), sig), __NV_SATFINITE, kFmt));
+}
+
+// dst = bf16(value(src) / sigma) for n FP8 bytes: exact (every E4M3 / E5M2 value times a power
+// of two is a bf16 value), the stored activation or gradient back in its own units.
+template <bool E5M2>
+__global__ void __launch_bounds__(256) k_fp8_dequant(const uint8_t* __restrict__ src, int64_t n,
+                                                     const float* __restrict__ scale,
+                                                     __nv_bfloat16* __restrict__ dst) {
+    griddep_enter();
+    constexpr __nv_fp8_interpretation_t kFmt = E5M2 ? __NV_E5M2 : __NV_E4M3;
+    const float inv = __frcp_rn(__ldg(scale));
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t n8 = n / 8;
+    for (int64_t i = i0; i < n8; i += stride) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(src) + i);
+        const uint32_t w[2] = {v.x, v.y};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                    static_cast<__nv_fp8x2_storage_t>((w[k] >> (16 * h)) & 0xFFFFu), kFmt);
+                const float2 f = __half22float2(__half2(hr));
+                o[2 * k + h] = pack_bf16x2(__fmul_rn(f.x, inv), __fmul_rn(f.y, inv));
+            }
+        }
+        reinterpret_cast<uint4*>(dst)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    for (int64_t i = n8 * 8 + i0; i < n; i += stride) {
+        const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(src[i]), kFmt);
+        dst[i] = __float2bfloat16_rn(__fmul_rn(__half2float(__half(hr)), inv));
+    }
+}
+
+// dst = bf16(src * a * b) for n bf16 values, a and b device scalars (powers of two: exact).
+__global__ void __launch_bounds__(256) k_scale2_bf16(const __nv_bfloat16* __restrict__ src, int64_t n,
+                                                     const float* __restrict__ a, const float* __restrict__ b,
+                                                     __nv_bfloat16* __restrict__ dst) {
+    griddep_enter();
+    const float f = __fmul_rn(__ldg(a), __ldg(b));
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        dst[i] = __float2bfloat16_rn(__fmul_rn(__bfloat162float(src[i]), f));
 }
 
 // sigma_w of a stored weight from its n second-level constants; one block of 256 threads.

@@ -6,6 +6,9 @@
 //     E4M3 activation, W8 the weight decoded to E4M3 in sigma_w units, U' the adapter term
 //     already in those units; the main K steps are kind::f8f6f4 MMAs (K = 128 per step), the
 //     adapter steps stay kind::f16 bf16 MMAs into the same fp32 accumulator.
+//   FP8 dX (FP8 = B_MN = true): dX = (dH8 W8 + G'[T, RP] A_pad) / (sigma_g sigma_w), dH8 the
+//     E5M2 gradient, W8 decoded MN-major (a K step is 128 weight rows x this CTA's 128 columns,
+//     one 128-byte swizzled row per weight row).
 //
 // A cluster of two CTAs (a "pair") computes 256 x 256 output tiles with 256x256x16 UMMA
 // instructions issued by the leader CTA.  Each CTA holds half of the A tile (128 token rows)
@@ -140,11 +143,13 @@ struct G2Smem {
     static_assert(kTotal <= 232448, "shared memory budget");
 };
 
-// Instruction descriptor for kind::f8f6f4 with E4M3 A and B (K-major), fp32 D, dense.
-__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N) {
+// Instruction descriptor for kind::f8f6f4, fp32 D, dense: A E4M3 (or E5M2), B E4M3 K-major
+// (or MN-major).
+__host__ __device__ constexpr uint32_t make_idesc_f8(int M, int N, bool a_e5m2, bool b_mn) {
     return (1u << 4)                                  // D format fp32
-           | (0u << 7)                                // A format E4M3
+           | (static_cast<uint32_t>(a_e5m2) << 7)     // A format: 0 E4M3, 1 E5M2
            | (0u << 10)                               // B format E4M3
+           | (static_cast<uint32_t>(b_mn) << 16)      // B major (0 = K)
            | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
@@ -190,7 +195,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThread
     k_nf4_gemm2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmC,
                 const __grid_constant__ CUtensorMap tmAx, const __grid_constant__ CUtensorMap tmBx,
                 const Gemm2Args args) {
-    static_assert(!(FP8 && B_MN), "the FP8 variant is the forward");
     using L = G2Smem<FP8>;
     constexpr int SA = L::SA;
     constexpr int SB = L::SB;
@@ -377,7 +381,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThread
         if (rank == 0 && lane == 0) {
             // ---------------------------------------------------------- MMA issuer (leader)
             const uint32_t idesc = make_idesc_bf16(256, 256, false, B_MN);
-            const uint32_t idesc8 = make_idesc_e4m3(256, 256);
+            const uint32_t idesc8 = make_idesc_f8(256, 256, B_MN, B_MN);
             int git = 0;
             bool ok = true;
             for (int tc = 0; ok && tc < n_units; ++tc) {
@@ -404,11 +408,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThread
                     const uint32_t b = smem_u32(sB + sb * L::kB);
                     const int nk = (it == iters_per_tile - 1 && it >= args.k_steps) ? args.ext_k16_last : 4;
                     if (FP8 && it < args.k_steps) {
-                        // 4 x K = 32 E4M3 columns: 32 bytes of each 128-byte row per MMA
+                        // 4 x K = 32 FP8 columns: 32 bytes of each 128-byte A row per MMA; B
+                        // K-major the same, B MN-major 32 rows of 128 bytes
                         for (int k = 0; k < 4; ++k)
                             umma_e4m3_ss_2sm(d_tmem, make_sw128_desc(a + k * 32, 16, 1024),
-                                             make_sw128_desc(b + k * 32, 16, 1024), idesc8,
-                                             (it > it0 || k > 0) ? 1u : 0u);
+                                             B_MN ? make_sw128_desc(b + k * 4096, 8192, 1024)
+                                                  : make_sw128_desc(b + k * 32, 16, 1024),
+                                             idesc8, (it > it0 || k > 0) ? 1u : 0u);
                     } else {
                         for (int k = 0; k < nk; ++k) {
                             const uint64_t ad = make_sw128_desc(a + k * 32, 16, 1024);
@@ -531,8 +537,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThread
         }
     } else if constexpr (FP8) {
         // -------------------------------------------------------------- NF4 -> E4M3 decoders
-        // Thread j owns weight row j of this CTA's 128 and, per K step, that row's two
+        // Forward: thread j owns weight row j of this CTA's 128 and, per K step, that row's two
         // consecutive 64-blocks: 128 E4M3 bytes, one whole 128-byte row of the swizzled tile.
+        // dX: thread j owns weight row j of the K step and this CTA's 128 columns of it (two
+        // 64-blocks): again one whole 128-byte row, now of the MN-major tile.
         const int grp = (warp - 6) >> 2;
         const int j = ((warp - 6) & 3) * 32 + lane;
         const float wsc = __ldg(args.w_scale);
@@ -542,7 +550,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThread
             float c2[2];
         };
         int row_tile = -1;
-        int64_t wrow = 0;
+        int64_t col0 = 0;                     // first of this CTA's 128 columns of the tile
         Cur fc = cur_at(grp);                 // the next step to fetch scales for
         auto fetch = [&](Pre& pr) {
             pr.nv = 0;
@@ -551,9 +559,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThread
             if (c.git >= total_iters || c.it >= args.k_steps) return;
             if (c.tile != row_tile) {
                 row_tile = c.tile;
-                wrow = static_cast<int64_t>(c.tile / args.m_tiles) * 256 + rank * 128 + j;
+                col0 = static_cast<int64_t>(c.tile / args.m_tiles) * 256 + rank * 128;
             }
-            const int64_t wblk = 2 * static_cast<int64_t>(c.it);
+            const int64_t wrow = B_MN ? static_cast<int64_t>(c.it) * 128 + j : col0 + j;
+            const int64_t wblk = B_MN ? col0 / 64 : 2 * static_cast<int64_t>(c.it);
             if (wrow >= args.nf4_rows || wblk >= args.nf4_bpr) return;
             pr.nv = wblk + 1 < args.nf4_bpr ? 2 : 1;
             const int64_t b0 = wrow * args.nf4_bpr + wblk;

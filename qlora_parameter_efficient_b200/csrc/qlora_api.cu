@@ -262,6 +262,7 @@ struct Plan {
            seg_u = 0;
     int seg_ldu = 0, seg_max_tiles = 0;
     size_t dora_part = 0, dora_scale = 0;   // DoRA row-norm partials and column scale
+    size_t f8_x = 0, f8_dh = 0, f8_g = 0;    // FP8 backward: bf16 X~, dH~ and sigma sigma_w s G
     size_t total = 0;
 };
 
@@ -277,6 +278,15 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
     if (op == QLORA_OP_MERGE) return p;
     if (op == QLORA_OP_FP8_QUANT) {
         p.total = 256;      // the amax word
+        return p;
+    }
+    if (op == QLORA_OP_BWD_FP8) {
+        p = make_plan(QLORA_OP_BWD, QLORA_BF16, T, d_out, d_in, r);
+        off = p.total;
+        p.f8_x = take(static_cast<size_t>(T) * d_in * 2);
+        p.f8_dh = take(static_cast<size_t>(T) * d_out * 2);
+        p.f8_g = take(static_cast<size_t>(T) * p.RP * 2);
+        p.total = off;
         return p;
     }
     if (op == QLORA_OP_FWD_FP8) {
@@ -472,10 +482,9 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
                       const void* ext_b, int RP, int r_used, int ext_b_rank, void* out,
                       void* g2ws, int* err, cudaStream_t st, const float* col_scale = nullptr,
                       const float* x_scale = nullptr, const float* w_scale = nullptr) {
-    // x_scale != NULL: the FP8 forward (act is the E4M3 activation, ext_a the adapter term in
-    // sigma_x sigma_w units)
+    // x_scale != NULL: the FP8 variant (act is the E4M3 activation or, for dX, the E5M2
+    // gradient; ext_a the adapter term in sigma sigma_w units; x_scale that tensor's sigma)
     const bool fp8 = x_scale != nullptr;
-    if (fp8 && dx) return QLORA_ERR_UNSUPPORTED;
     const int64_t d_out = w->d_out, d_in = w->d_in;
     CUtensorMap ta, tc, tax, tbx;
     const int64_t K = dx ? d_out : d_in;
@@ -524,10 +533,11 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
         g.part = static_cast<float*>(g2ws);
         g.cnt = reinterpret_cast<int*>(static_cast<uint8_t*>(g2ws) + sch.part_bytes);
     }
-    auto kern = fp8 ? k_nf4_gemm2<false, true> : dx ? k_nf4_gemm2<true> : k_nf4_gemm2<false>;
+    auto kern = fp8 ? (dx ? k_nf4_gemm2<true, true> : k_nf4_gemm2<false, true>)
+                    : (dx ? k_nf4_gemm2<true> : k_nf4_gemm2<false>);
     const int smem = fp8 ? G2Smem<true>::kTotal : G2Smem<false>::kTotal;
-    const int variant = fp8 ? 2 : dx ? 1 : 0;
-    static std::atomic<uint64_t> configured[3] = {0, 0, 0};
+    const int variant = (fp8 ? 2 : 0) + (dx ? 1 : 0);
+    static std::atomic<uint64_t> configured[4] = {0, 0, 0, 0};
     int dev = 0;
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
@@ -836,6 +846,101 @@ qlora_status dora_scale(const qlora_nf4* w, const void* A, const void* B, int32_
     return QLORA_OK;
 }
 
+// FP8 operands of the dX GEMM: the E5M2 gradient and its scale, the weight's scale, and the
+// workspace for sigma_g sigma_w bf16(s G).
+struct Fp8Dx {
+    const uint8_t* dH8;
+    const float* g_scale;
+    const float* w_scale;
+    __nv_bfloat16* g8;
+};
+
+// The bf16 backward: U (or U_saved), G = dH B, dX (bf16 GEMM, or the FP8 GEMM when f8 is set),
+// dA, dB by split-K tensor-core products and their finalizes.
+qlora_status bwd_bf16(const qlora_nf4* w, const void* X, const void* dH, int64_t T, const void* A,
+                      const void* B, int32_t r, float s, const void* U_saved, void* dX, float* dA,
+                      float* dB, const Plan& p, void* ws, int* err, int acc_grads, cudaStream_t stream,
+                      const Fp8Dx* f8) {
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    const int RP = p.RP;
+    auto* a_pad = at<__nv_bfloat16>(ws, p.a_pad);
+    auto* b_pad = at<__nv_bfloat16>(ws, p.b_pad);
+    auto* u_pad = at<__nv_bfloat16>(ws, p.u_pad);
+    auto* g_spad = at<__nv_bfloat16>(ws, p.g_spad);
+    auto* part = at<float>(ws, p.part);
+    // pad-free operands when r is a multiple of 8 (see the forward)
+    const bool direct = r % 8 == 0;
+    const void* a_src = A;
+    const void* b_src = B;
+    const void* u_src = u_pad;
+    int a_rows = r, b_ld = r, u_ld = RP;
+    if (!direct) {
+        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A), r, d_in, d_in, a_pad, RP, d_in, 0, d_in, stream));
+        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
+        a_src = a_pad;
+        b_src = b_pad;
+        a_rows = b_ld = RP;
+    }
+    if (U_saved && direct) {
+        u_src = U_saved;
+        u_ld = r;
+    } else if (U_saved) {
+        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(U_saved), T, r, r, u_pad, T, RP, 0, RP, stream));
+    } else {
+        QL_TRY(compute_u_bf16(X, T, d_in, a_src, a_rows, RP, r, s, p.split_u, part, nullptr,
+                              u_pad, nullptr, err, stream));
+    }
+    // G = dH B  ->  g_spad = bf16(s G)
+    {
+        CUtensorMap tdh, tbp;
+        QL_TRY(tmap_bf16(&tdh, dH, T, d_out, d_out, kBM));
+        QL_TRY(tmap_bf16(&tbp, b_src, d_out, b_ld, b_ld, 64));
+        QL_TRY(skinny_gemm(false, true, RP, r, tdh, tbp, T, cdiv(d_out, kBK), p.split_g, part, err, stream));
+        if (launch_pdl(k_finalize_rows<__nv_bfloat16>, grid1d(T * RP), dim3(256), 0, stream,
+                       part, p.split_g, T * RP, T, r, RP, s, nullptr, nullptr, g_spad) !=
+            cudaSuccess)
+            return QLORA_ERR_CUDA;
+        QL_LAUNCH_CHECK();
+    }
+    // dX = dH W^ + (sG) A
+    if (dX && !f8) QL_TRY(nf4_gemm(true, w, dH, T, g_spad, a_src, RP, r, a_rows, dX, at<void>(ws, p.g2), err, stream));
+    if (dX && f8) {
+        // FP8: the adapter operand in the accumulator's units (sigma_g sigma_w, powers of two),
+        // then the E5M2 x E4M3 GEMM with the epilogue factor 1 / (sigma_g sigma_w)
+        if (launch_pdl(k_scale2_bf16, grid1d(T * RP), dim3(256), 0, stream,
+                       static_cast<const __nv_bfloat16*>(g_spad), T * RP, f8->g_scale, f8->w_scale,
+                       f8->g8) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        QL_LAUNCH_CHECK();
+        QL_TRY(nf4_gemm(true, w, f8->dH8, T, f8->g8, a_src, RP, r, a_rows, dX, at<void>(ws, p.g2), err, stream,
+                        nullptr, f8->g_scale, f8->w_scale));
+    }
+    // dA^T[d_in, RP] = X^T (sG)
+    {
+        CUtensorMap txm, tgm;
+        QL_TRY(tmap_bf16(&txm, X, T, d_in, d_in, 64));
+        QL_TRY(tmap_bf16(&tgm, g_spad, T, RP, RP, 64));
+        QL_TRY(skinny_gemm(true, true, RP, r, txm, tgm, d_in, cdiv(T, kBK), p.split_da, part, err, stream));
+        if (launch_pdl(k_finalize_dA, grid1d(static_cast<int64_t>(r) * d_in), dim3(256), 0,
+                       stream, part, p.split_da, d_in * RP, d_in, r, RP, dA, acc_grads) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        QL_LAUNCH_CHECK();
+    }
+    // dB[d_out, RP] = s dH^T U
+    {
+        CUtensorMap thm, tum;
+        QL_TRY(tmap_bf16(&thm, dH, T, d_out, d_out, 64));
+        QL_TRY(tmap_bf16(&tum, u_src, T, u_ld, u_ld, 64));
+        QL_TRY(skinny_gemm(true, true, RP, r, thm, tum, d_out, cdiv(T, kBK), p.split_db, part, err, stream));
+        if (launch_pdl(k_finalize_dB, grid1d(d_out * r), dim3(256), 0, stream, part, p.split_db,
+                       d_out * RP, d_out, r, RP, s, dB, acc_grads) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        QL_LAUNCH_CHECK();
+    }
+    return QLORA_OK;
+    return QLORA_OK;
+}
+
 }  // namespace
 
 // ======================================================================= C ABI
@@ -876,9 +981,9 @@ qlora_status qlora_nf4_levels(float* out) {
 
 size_t qlora_workspace_bytes(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in,
                              int32_t r_total) {
-    if (op < QLORA_OP_FWD || op > QLORA_OP_FP8_QUANT) return 0;
+    if (op < QLORA_OP_FWD || op > QLORA_OP_BWD_FP8) return 0;
     if ((op == QLORA_OP_FWD_MULTI || op == QLORA_OP_DORA_FWD || op == QLORA_OP_FWD_FP8 ||
-         op == QLORA_OP_FP8_QUANT) && dtype != QLORA_BF16)
+         op == QLORA_OP_FP8_QUANT || op == QLORA_OP_BWD_FP8) && dtype != QLORA_BF16)
         return 0;
     if ((dtype != QLORA_BF16 && dtype != QLORA_F32) || T < 1 || d_out < 1 || d_in < 64 ||
         r_total < 1 || r_total > 128)
@@ -992,11 +1097,64 @@ qlora_status qlora_fp8_quantize(const void* X, int64_t n, uint8_t* X8, float* sc
         cudaSuccess)
         return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
-    if (launch_pdl(k_fp8_quant, grid, dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(X), n,
+    if (launch_pdl(k_fp8_quant<false>, grid, dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(X), n,
                    static_cast<const unsigned*>(amax), X8, scale) != cudaSuccess)
         return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     return QLORA_OK;
+}
+
+qlora_status qlora_fp8_quantize_grad(const void* dH, int64_t n, uint8_t* dH8, float* scale, void* ws,
+                                     size_t ws_bytes, cudaStream_t stream) {
+    if (!aligned16(dH) || !aligned16(dH8) || !scale) return QLORA_ERR_INVALID_ARG;
+    if (n < 1) return QLORA_ERR_UNSUPPORTED;
+    QL_TRY(check_ws(ws, ws_bytes, 256));
+    auto* amax = static_cast<unsigned*>(ws);
+    if (cudaMemsetAsync(amax, 0, 4, stream) != cudaSuccess) return QLORA_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(std::min<int64_t>(std::max<int64_t>(cdiv(n, 8 * 256), 1), 148 * 8)));
+    if (launch_pdl(k_fp8_amax, grid, dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(dH), n, amax) !=
+        cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    if (launch_pdl(k_fp8_quant<true>, grid, dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(dH), n,
+                   static_cast<const unsigned*>(amax), dH8, scale) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+qlora_status qlora_linear_bwd_fp8(const qlora_nf4* w, const uint8_t* X8, const float* x_scale,
+                                  const uint8_t* dH8, const float* g_scale, const float* w_scale,
+                                  int64_t T, const void* A, const void* B, int32_t r, float alpha,
+                                  void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                                  uint32_t flags, cudaStream_t stream) {
+    if (flags & ~static_cast<uint32_t>(QLORA_BWD_ACCUMULATE)) return QLORA_ERR_INVALID_ARG;
+    const int acc_grads = (flags & QLORA_BWD_ACCUMULATE) ? 1 : 0;
+    QL_TRY(check_layer(w, T, r, QLORA_BF16));
+    if (!aligned16(X8) || !aligned16(dH8) || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
+        !aligned16(dB) || !aligned16_or_null(dX) || !x_scale || !g_scale || !w_scale)
+        return QLORA_ERR_INVALID_ARG;
+    // the E5M2 gradient's rows are d_out bytes: a TMA row stride must be a multiple of 16
+    if (w->d_out % 16 != 0) return QLORA_ERR_UNSUPPORTED;
+    const Plan p = make_plan(QLORA_OP_BWD_FP8, QLORA_BF16, T, w->d_out, w->d_in, r);
+    QL_TRY(check_ws(ws, ws_bytes, p.total));
+    int* err = nullptr;
+    QL_TRY(err_word(&err));
+    const int64_t d_out = w->d_out, d_in = w->d_in;
+    // the stored FP8 tensors back in their own units (exact in bf16) for the skinny products
+    auto* xb = at<__nv_bfloat16>(ws, p.f8_x);
+    auto* hb = at<__nv_bfloat16>(ws, p.f8_dh);
+    if (launch_pdl(k_fp8_dequant<false>, grid1d(T * d_in / 8), dim3(256), 0, stream, X8, T * d_in, x_scale, xb) !=
+        cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    if (launch_pdl(k_fp8_dequant<true>, grid1d(T * d_out / 8), dim3(256), 0, stream, dH8, T * d_out, g_scale, hb) !=
+        cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    const Fp8Dx f8{dH8, g_scale, w_scale, at<__nv_bfloat16>(ws, p.f8_g)};
+    return bwd_bf16(w, xb, hb, T, A, B, r, alpha / static_cast<float>(r), nullptr, dX, dA, dB, p, ws, err,
+                    acc_grads, stream, &f8);
 }
 
 qlora_status qlora_fp8_weight_scale(const qlora_nf4* w, float* w_scale, cudaStream_t stream) {
@@ -1065,73 +1223,8 @@ qlora_status qlora_linear_bwd_ex(const qlora_nf4* w, const void* X, const void* 
     QL_TRY(err_word(&err));
     const int64_t d_out = w->d_out, d_in = w->d_in;
     const float s = alpha / static_cast<float>(r);
-    if (dtype == QLORA_BF16) {
-        const int RP = p.RP;
-        auto* a_pad = at<__nv_bfloat16>(ws, p.a_pad);
-        auto* b_pad = at<__nv_bfloat16>(ws, p.b_pad);
-        auto* u_pad = at<__nv_bfloat16>(ws, p.u_pad);
-        auto* g_spad = at<__nv_bfloat16>(ws, p.g_spad);
-        auto* part = at<float>(ws, p.part);
-        // pad-free operands when r is a multiple of 8 (see the forward)
-        const bool direct = r % 8 == 0;
-        const void* a_src = A;
-        const void* b_src = B;
-        const void* u_src = u_pad;
-        int a_rows = r, b_ld = r, u_ld = RP;
-        if (!direct) {
-            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(A), r, d_in, d_in, a_pad, RP, d_in, 0, d_in, stream));
-            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(B), d_out, r, r, b_pad, d_out, RP, 0, RP, stream));
-            a_src = a_pad;
-            b_src = b_pad;
-            a_rows = b_ld = RP;
-        }
-        if (U_saved && direct) {
-            u_src = U_saved;
-            u_ld = r;
-        } else if (U_saved) {
-            QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(U_saved), T, r, r, u_pad, T, RP, 0, RP, stream));
-        } else {
-            QL_TRY(compute_u_bf16(X, T, d_in, a_src, a_rows, RP, r, s, p.split_u, part, nullptr,
-                                  u_pad, nullptr, err, stream));
-        }
-        // G = dH B  ->  g_spad = bf16(s G)
-        {
-            CUtensorMap tdh, tbp;
-            QL_TRY(tmap_bf16(&tdh, dH, T, d_out, d_out, kBM));
-            QL_TRY(tmap_bf16(&tbp, b_src, d_out, b_ld, b_ld, 64));
-            QL_TRY(skinny_gemm(false, true, RP, r, tdh, tbp, T, cdiv(d_out, kBK), p.split_g, part, err, stream));
-            if (launch_pdl(k_finalize_rows<__nv_bfloat16>, grid1d(T * RP), dim3(256), 0, stream,
-                           part, p.split_g, T * RP, T, r, RP, s, nullptr, nullptr, g_spad) !=
-                cudaSuccess)
-                return QLORA_ERR_CUDA;
-            QL_LAUNCH_CHECK();
-        }
-        // dX = dH W^ + (sG) A
-        if (dX) QL_TRY(nf4_gemm(true, w, dH, T, g_spad, a_src, RP, r, a_rows, dX, at<void>(ws, p.g2), err, stream));
-        // dA^T[d_in, RP] = X^T (sG)
-        {
-            CUtensorMap txm, tgm;
-            QL_TRY(tmap_bf16(&txm, X, T, d_in, d_in, 64));
-            QL_TRY(tmap_bf16(&tgm, g_spad, T, RP, RP, 64));
-            QL_TRY(skinny_gemm(true, true, RP, r, txm, tgm, d_in, cdiv(T, kBK), p.split_da, part, err, stream));
-            if (launch_pdl(k_finalize_dA, grid1d(static_cast<int64_t>(r) * d_in), dim3(256), 0,
-                           stream, part, p.split_da, d_in * RP, d_in, r, RP, dA, acc_grads) != cudaSuccess)
-                return QLORA_ERR_CUDA;
-            QL_LAUNCH_CHECK();
-        }
-        // dB[d_out, RP] = s dH^T U
-        {
-            CUtensorMap thm, tum;
-            QL_TRY(tmap_bf16(&thm, dH, T, d_out, d_out, 64));
-            QL_TRY(tmap_bf16(&tum, u_src, T, u_ld, u_ld, 64));
-            QL_TRY(skinny_gemm(true, true, RP, r, thm, tum, d_out, cdiv(T, kBK), p.split_db, part, err, stream));
-            if (launch_pdl(k_finalize_dB, grid1d(d_out * r), dim3(256), 0, stream, part, p.split_db,
-                           d_out * RP, d_out, r, RP, s, dB, acc_grads) != cudaSuccess)
-                return QLORA_ERR_CUDA;
-            QL_LAUNCH_CHECK();
-        }
-        return QLORA_OK;
-    }
+    if (dtype == QLORA_BF16)
+        return bwd_bf16(w, X, dH, T, A, B, r, s, U_saved, dX, dA, dB, p, ws, err, acc_grads, stream, nullptr);
     // exact fp32 path
     const float* Xf = static_cast<const float*>(X);
     const float* dHf = static_cast<const float*>(dH);

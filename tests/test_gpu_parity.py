@@ -690,3 +690,98 @@ def test_fp8_end_to_end_approximates_bf16_layer(q):
     ref = O.lora_forward(oracle_weight(oc, 384, 512, "f32"), case.X, case.A, case.B, case.alpha, case.r)
     e = rel_fro(host(H), ref)
     assert 1e-3 < e < 0.06
+
+
+# ------------------------------------------------------------------ FP8 backward (R26)
+
+
+def fp8_probe_grad(n, seed):
+    """bf16 gradient values whose scaled copies (amax 1 -> sigma 2^15) hit every E5M2 tie
+    below 2^15, the subnormal range and zeros, plus small normal draws."""
+    rng = np.random.default_rng(seed)
+    x = S.round_to_bf16((rng.standard_normal(n) * 0.2).astype(np.float32))
+    x = np.clip(x, -0.96875, 0.96875)
+    pos = O.e5m2_decode(np.arange(124, dtype=np.uint8))
+    mids = 0.5 * (pos[1:] + pos[:-1])
+    mids = (mids[mids < 2.0 ** 15] / 2.0 ** 15).astype(np.float32)
+    probe = np.concatenate([mids, -mids, np.float32([0.0, 2.0 ** -40, -2.0 ** -33])])
+    m = min(n - 1, probe.size)
+    x[1:1 + m] = probe[:m]
+    x[0] = 1.0
+    assert np.array_equal(S.round_to_bf16(x), x)
+    return x
+
+
+@pytest.mark.parametrize("shape", [(9999,), (64, 4096), (2,)])
+def test_fp8_quantize_grad_bit_exact(q, shape):
+    import torch
+    n = int(np.prod(shape))
+    G = fp8_probe_grad(n, seed=n + 1).reshape(shape)
+    G8, sc = q.fp8_quantize_grad(dev(G, "bf16"))
+    torch.cuda.synchronize()
+    ref8, sig = O.fp8_quantize_grad(G)
+    assert float(sc.item()) == sig
+    assert np.array_equal(G8.cpu().numpy(), ref8)
+
+
+def run_fp8_bwd(q, case, rows=None):
+    """FP8 backward on the oracle's E4M3 activation, E5M2 gradient and scales (uploaded as
+    inputs) against the oracle's FP8 backward."""
+    import torch
+    w, oc = quantize_both(q, case.W0)
+    codes, q8, c2, _ = oc
+    X8, sx = O.fp8_quantize_act(case.X)
+    G8, sg = O.fp8_quantize_grad(case.dH)
+    sw = O.fp8_weight_scale(c2)
+    W8 = O.nf4_dequantize_e4m3(codes, q8, c2, case.d_out, case.d_in, sw)
+    t = lambda v: torch.tensor([v], dtype=torch.float32, device="cuda")
+    dX, dA, dB = q.qlora_linear_bwd_fp8(w, torch.from_numpy(X8).cuda(), t(sx), torch.from_numpy(G8).cuda(),
+                                        t(sg), t(sw), dev(case.A, "bf16"), dev(case.B, "bf16"), case.alpha)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    rdX, rdA, rdB = O.lora_backward_fp8(X8, sx, G8, sg, W8, sw, case.A, case.B, case.alpha, case.r)
+    sel = slice(None) if rows is None else rows
+    assert rel_fro(host(dX)[sel], rdX[sel]) <= TOL["bf16"]
+    assert rel_fro(host(dA), rdA) <= TOL["bf16"]
+    assert rel_fro(host(dB), rdB) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("d_out,d_in,r,T", [(256, 256, 8, 64), (208, 192, 5, 77), (528, 320, 16, 300),
+                                            (144, 256, 100, 3), (64, 128, 16, 1), (272, 1088, 64, 520)])
+def test_fp8_backward(q, d_out, d_in, r, T):
+    run_fp8_bwd(q, S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_in + r))
+
+
+def test_fp8_backward_q_proj_sampled_rows(q):
+    case = S.make_layer(**S.CONFIGS["q_proj_4096x4096_r16_T4096"], seed=9)
+    rows = np.sort(np.random.default_rng(7).choice(case.T, 256, replace=False))
+    run_fp8_bwd(q, case, rows=rows)
+
+
+def test_fp8_backward_accumulate(q):
+    """Two FP8 micro-batches with QLORA_BWD_ACCUMULATE add their dA, dB."""
+    import torch
+    case = S.make_layer(272, 320, 16, 32.0, 96, dtype="bf16", seed=14)
+    w, oc = quantize_both(q, case.W0)
+    ws_ = q.fp8_weight_scale(w)
+    A, B = dev(case.A, "bf16"), dev(case.B, "bf16")
+    X8, xs = q.fp8_quantize(dev(case.X, "bf16"))
+    G8, gs = q.fp8_quantize_grad(dev(case.dH, "bf16"))
+    _, dA1, dB1 = q.qlora_linear_bwd_fp8(w, X8, xs, G8, gs, ws_, A, B, case.alpha)
+    _, dA2, dB2 = q.qlora_linear_bwd_fp8(w, X8, xs, G8, gs, ws_, A, B, case.alpha, dA=dA1.clone(),
+                                         dB=dB1.clone(), accumulate=True, want_dx=False)
+    torch.cuda.synchronize()
+    assert torch.equal(dA2, 2 * dA1) and torch.equal(dB2, 2 * dB1)
+
+
+def test_fp8_backward_rejects_unaligned_gradient_rows(q):
+    """d_out % 16 != 0: the E5M2 rows cannot be read by TMA; refused on the host."""
+    import torch
+    case = S.make_layer(200, 192, 8, 16.0, 10, dtype="bf16", seed=1, with_grad=False)
+    w, _ = quantize_both(q, case.W0)
+    one = torch.ones(1, dtype=torch.float32, device="cuda")
+    X8 = torch.zeros((10, 192), dtype=torch.uint8, device="cuda")
+    G8 = torch.zeros((10, 200), dtype=torch.uint8, device="cuda")
+    with pytest.raises(q.QloraError) as e:
+        q.qlora_linear_bwd_fp8(w, X8, one, G8, one, one, dev(case.A, "bf16"), dev(case.B, "bf16"), 16.0)
+    assert e.value.code == 2
