@@ -151,8 +151,11 @@ __device__ __forceinline__ uint32_t ld_pair(const __nv_bfloat16* p, bool ok) {
 // One CTA (4 warps) per tile.  Warp w takes the 64-element K chunks w, w + 4, ...; the four
 // warps' sums are added in warp order.  NT: n8 tiles of the largest rank (ranks up to 8 NT);
 // fewer accumulators let more K chunks' loads be in flight (UNR chunks per iteration).
+#ifndef QLORA_SEG_SHRINK_MINB
+#define QLORA_SEG_SHRINK_MINB 3
+#endif
 template <int NT, int UNR>
-__global__ void __launch_bounds__(128, 4) k_seg_shrink(SegArgs a) {
+__global__ void __launch_bounds__(128, QLORA_SEG_SHRINK_MINB) k_seg_shrink(SegArgs a) {
     griddep_enter();
     __shared__ float s_part[4][kSegTile][129];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -176,28 +179,39 @@ __global__ void __launch_bounds__(128, 4) k_seg_shrink(SegArgs a) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
     const uint4 z4 = make_uint4(0, 0, 0, 0);
-#pragma unroll UNR
-    for (int k0 = 64 * warp; k0 < a.d_in; k0 += 256) {
-        uint4 x[4];
-        x[0] = tok_a >= 0 ? __ldg(reinterpret_cast<const uint4*>(xa + k0)) : z4;
-        x[1] = tok_a >= 0 ? __ldg(reinterpret_cast<const uint4*>(xa + k0 + 8)) : z4;
-        x[2] = tok_b >= 0 ? __ldg(reinterpret_cast<const uint4*>(xb + k0)) : z4;
-        x[3] = tok_b >= 0 ? __ldg(reinterpret_cast<const uint4*>(xb + k0 + 8)) : z4;
-        const uint32_t* wa = reinterpret_cast<const uint32_t*>(&x[0]);   // row g: 8 words
-        const uint32_t* wb = reinterpret_cast<const uint32_t*>(&x[2]);   // row g + 8
+    // UNR chunks of 64 columns per pass: every load of the pass is issued before its MMAs
+    for (int kb = 64 * warp; kb < a.d_in; kb += 256 * UNR) {
+        uint4 x[UNR][4], y[UNR][NT][2];
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            if (n < nt8) {
+        for (int u = 0; u < UNR; ++u) {
+            const int k0 = kb + 256 * u;
+            const bool kin = k0 < a.d_in;
+            x[u][0] = kin && tok_a >= 0 ? __ldg(reinterpret_cast<const uint4*>(xa + k0)) : z4;
+            x[u][1] = kin && tok_a >= 0 ? __ldg(reinterpret_cast<const uint4*>(xa + k0 + 8)) : z4;
+            x[u][2] = kin && tok_b >= 0 ? __ldg(reinterpret_cast<const uint4*>(xb + k0)) : z4;
+            x[u][3] = kin && tok_b >= 0 ? __ldg(reinterpret_cast<const uint4*>(xb + k0 + 8)) : z4;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
                 const int j = 8 * n + g;                      // adapter row = output column
-                const __nv_bfloat16* arow = Ai + static_cast<int64_t>(j < r ? j : 0) * a.d_in + k0 + 16 * t;
-                uint4 y[2];
-                y[0] = j < r ? __ldg(reinterpret_cast<const uint4*>(arow)) : z4;
-                y[1] = j < r ? __ldg(reinterpret_cast<const uint4*>(arow + 8)) : z4;
-                const uint32_t* wy = reinterpret_cast<const uint32_t*>(&y[0]);
+                const bool ok = kin && n < nt8 && j < r;
+                const __nv_bfloat16* arow = Ai + static_cast<int64_t>(ok ? j : 0) * a.d_in + (kin ? k0 : 0) + 16 * t;
+                y[u][n][0] = ok ? __ldg(reinterpret_cast<const uint4*>(arow)) : z4;
+                y[u][n][1] = ok ? __ldg(reinterpret_cast<const uint4*>(arow + 8)) : z4;
+            }
+        }
 #pragma unroll
-                for (int st = 0; st < 4; ++st) {
-                    const uint32_t af[4] = {wa[2 * st], wb[2 * st], wa[2 * st + 1], wb[2 * st + 1]};
-                    mma_bf16_16816(acc[n], af, wy[2 * st], wy[2 * st + 1], true);
+        for (int u = 0; u < UNR; ++u) {
+            const uint32_t* wa = reinterpret_cast<const uint32_t*>(&x[u][0]);   // row g: 8 words
+            const uint32_t* wb = reinterpret_cast<const uint32_t*>(&x[u][2]);   // row g + 8
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                if (n < nt8) {
+                    const uint32_t* wy = reinterpret_cast<const uint32_t*>(&y[u][n][0]);
+#pragma unroll
+                    for (int st = 0; st < 4; ++st) {
+                        const uint32_t af[4] = {wa[2 * st], wb[2 * st], wa[2 * st + 1], wb[2 * st + 1]};
+                        mma_bf16_16816(acc[n], af, wy[2 * st], wy[2 * st + 1], true);
+                    }
                 }
             }
         }
