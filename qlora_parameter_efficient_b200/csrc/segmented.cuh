@@ -254,11 +254,18 @@ __device__ __forceinline__ uint2 ld_quad(const __nv_bfloat16* row, int j, int va
 // Persistent over tiles; for a tile, warp w takes the 64-column blocks w, w + 4, ... of H as
 // eight n8 fragments each.  K = the adapter's rank rounded up to 16 (U is zero beyond r), the K
 // slots of each 16-step mapped as in the shrink (thread-column t holds elements 4t .. 4t+3).
-// The tile's U fragments stay in registers for all its column blocks, and the H values of the
-// next block are loaded before the current block is stored.
+// The tile's U fragments stay in registers for all its column blocks; each warp loads the H
+// values and first B quads of UNR blocks before multiplying and storing them.
 // KS: K steps of 16 of the largest rank (ranks up to 16 KS).
+#ifndef QLORA_SEG_EXPAND_UNR
+#define QLORA_SEG_EXPAND_UNR 2
+#endif
+#ifndef QLORA_SEG_EXPAND_MINB
+#define QLORA_SEG_EXPAND_MINB 4
+#endif
 template <int KS>
-__global__ void __launch_bounds__(128, 4) k_seg_expand(SegArgs a) {
+__global__ void __launch_bounds__(128, QLORA_SEG_EXPAND_MINB) k_seg_expand(SegArgs a) {
+    constexpr int UNR = QLORA_SEG_EXPAND_UNR;     // column blocks per pass of a warp
     griddep_enter();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int n_tiles = *a.n_tiles;
@@ -308,53 +315,54 @@ __global__ void __launch_bounds__(128, 4) k_seg_expand(SegArgs a) {
                                       : make_uint2(0, 0);
             }
         };
-        uint32_t h_cur[8][2], h_nxt[8][2];
-        uint2 b_cur[8], b_nxt[8];                          // K step 0 of this / the next block
-        if (warp < n_blocks) {
-            load_h(warp, h_cur);
-            load_b(warp, 0, b_cur);
-        }
-        for (int blk = warp; blk < n_blocks; blk += 4) {
-            if (blk + 4 < n_blocks) {
-                load_h(blk + 4, h_nxt);
-                load_b(blk + 4, 0, b_nxt);
-            }
-            float acc[8][4];
+        // warp w takes blocks w, w + 4, ...; UNR of them per pass, every H value and K step 0
+        // B quad of the pass loaded before its MMAs
+        for (int blk0 = warp; blk0 < n_blocks; blk0 += 4 * UNR) {
+            uint32_t hv[UNR][8][2];
+            uint2 bq0[UNR][8];
 #pragma unroll
-            for (int n = 0; n < 8; ++n)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
-#pragma unroll
-            for (int n = 0; n < 8; ++n) mma_bf16_16816(acc[n], uf[0], b_cur[n].x, b_cur[n].y, true);
-#pragma unroll
-            for (int ks = 1; ks < KS; ++ks) {
-                if (ks < ksteps) {
-                    uint2 bq[8];
-                    load_b(blk, ks, bq);
-#pragma unroll
-                    for (int n = 0; n < 8; ++n) mma_bf16_16816(acc[n], uf[ks], bq[n].x, bq[n].y, true);
+            for (int u = 0; u < UNR; ++u) {
+                const int blk = blk0 + 4 * u;
+                if (blk < n_blocks) {
+                    load_h(blk, hv[u]);
+                    load_b(blk, 0, bq0[u]);
                 }
             }
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const int col = 64 * blk + 8 * n + 2 * t;
-                if (col >= a.d_out) continue;
+            for (int u = 0; u < UNR; ++u) {
+                const int blk = blk0 + 4 * u;
+                if (blk >= n_blocks) break;
+                float acc[8][4];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int tok = hh ? tok_b : tok_a;
-                    if (tok < 0) continue;
-                    __nv_bfloat162 base;
-                    *reinterpret_cast<uint32_t*>(&base) = h_cur[n][hh];
-                    const float2 bf = __bfloat1622float2(base);
-                    *reinterpret_cast<__nv_bfloat162*>(a.H + static_cast<int64_t>(tok) * a.d_out + col) =
-                        __floats2bfloat162_rn(bf.x + acc[n][2 * hh], bf.y + acc[n][2 * hh + 1]);
+                for (int n = 0; n < 8; ++n)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+#pragma unroll
+                for (int n = 0; n < 8; ++n) mma_bf16_16816(acc[n], uf[0], bq0[u][n].x, bq0[u][n].y, true);
+#pragma unroll
+                for (int ks = 1; ks < KS; ++ks) {
+                    if (ks < ksteps) {
+                        uint2 bq[8];
+                        load_b(blk, ks, bq);
+#pragma unroll
+                        for (int n = 0; n < 8; ++n) mma_bf16_16816(acc[n], uf[ks], bq[n].x, bq[n].y, true);
+                    }
                 }
-            }
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                h_cur[n][0] = h_nxt[n][0];
-                h_cur[n][1] = h_nxt[n][1];
-                b_cur[n] = b_nxt[n];
+                for (int n = 0; n < 8; ++n) {
+                    const int col = 64 * blk + 8 * n + 2 * t;
+                    if (col >= a.d_out) continue;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int tok = hh ? tok_b : tok_a;
+                        if (tok < 0) continue;
+                        __nv_bfloat162 base;
+                        *reinterpret_cast<uint32_t*>(&base) = hv[u][n][hh];
+                        const float2 bf = __bfloat1622float2(base);
+                        *reinterpret_cast<__nv_bfloat162*>(a.H + static_cast<int64_t>(tok) * a.d_out + col) =
+                            __floats2bfloat162_rn(bf.x + acc[n][2 * hh], bf.y + acc[n][2 * hh + 1]);
+                    }
+                }
             }
         }
     }
