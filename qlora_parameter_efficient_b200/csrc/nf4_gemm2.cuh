@@ -111,17 +111,17 @@ static_assert(kG2StagesA >= kG2StagesB, "B-slot reuse is gated through the A rin
 // group has already observed, so no parity wait can alias.
 static_assert(kG2StagesA % kG2DecGroups == 0, "A-ring depth must be a multiple of the groups");
 constexpr int kG2Threads = 32 * (6 + 4 * kG2DecGroups);
-// FP8: a K step is 128 E4M3 columns (the same 128-byte rows), its codes tile twice as large;
-// the deeper A ring (TMA latency) is paid for with a 2-slot decoded-B ring (measured best of
-// 1, 2 or 4 decoder groups and (8, 2), (6, 4), (4, 4) rings).
+// FP8: a K step is 128 E4M3 columns (the same 128-byte rows), its codes tile twice as large,
+// so shared memory holds fewer stages: 3 decoder groups with 6 A stages and 3 decoded-B slots
+// (measured best of 1, 2, 3 or 4 groups with (8, 2), (6, 4), (6, 3), (6, 2), (4, 4) rings).
 #ifndef QLORA_G2_FP8_DEC_GROUPS
-#define QLORA_G2_FP8_DEC_GROUPS 4
+#define QLORA_G2_FP8_DEC_GROUPS 3
 #endif
 #ifndef QLORA_G2_FP8_STAGES_A
-#define QLORA_G2_FP8_STAGES_A 8
+#define QLORA_G2_FP8_STAGES_A 6
 #endif
 #ifndef QLORA_G2_FP8_STAGES_B
-#define QLORA_G2_FP8_STAGES_B 2
+#define QLORA_G2_FP8_STAGES_B 3
 #endif
 static_assert(QLORA_G2_FP8_STAGES_A >= QLORA_G2_FP8_STAGES_B, "B-slot reuse is gated through the A ring");
 static_assert(QLORA_G2_FP8_STAGES_A % QLORA_G2_FP8_DEC_GROUPS == 0,
