@@ -782,7 +782,7 @@ def extra_rows(q, torch, S, dev, peaks, args):
 # from the ncu capture summarised in profiles/nf4_fused_gemm_q_proj_4096x4096_T4096.md
 # (43.27 MB read + 15.34 MB written; H is still partly in L2 when the kernel ends).  Set to
 # None whenever the kernel changes until it is captured again.
-GEMM_FWD_DRAM_BYTES = 43270400 + 15336960
+GEMM_FWD_DRAM_BYTES = None
 
 
 def main():

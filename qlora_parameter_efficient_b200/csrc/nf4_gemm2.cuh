@@ -26,8 +26,8 @@
 //
 // Warp roles per CTA (6 + 4 x decoder groups warps):
 //   warp 0       TMA producer: this CTA's A half and NF4 code tile (or the K-extension
-//                adapter tiles) into an 8-stage ring, completing on the local full[s]; the
-//                decoded B halves live in a separate, shallower 4-slot ring (the adapter K
+//                adapter tiles) into a 6-stage ring, completing on the local full[s]; the
+//                decoded B halves live in a separate 6-slot ring (the adapter K
 //                step's B tile is loaded straight into its slot).
 //   warp 1       leader CTA only: issues the MMAs, commits stage release (empty[s]) and
 //                accumulator-ready (accf[b]) to both CTAs.
@@ -94,18 +94,21 @@ __device__ __forceinline__ void umma_commit_2sm_both(uint64_t* bar) {
 // ------------------------------------------------------------------ kernel
 
 #ifndef QLORA_G2_DEC_GROUPS
-#define QLORA_G2_DEC_GROUPS 4
+#define QLORA_G2_DEC_GROUPS 3
 #endif
 constexpr int kG2DecGroups = QLORA_G2_DEC_GROUPS;   // groups of 4 decoder warps
 #ifndef QLORA_G2_STAGES_A
-#define QLORA_G2_STAGES_A 8
+#define QLORA_G2_STAGES_A 6
 #endif
 #ifndef QLORA_G2_STAGES_B
-#define QLORA_G2_STAGES_B 4
+#define QLORA_G2_STAGES_B 6
 #endif
 constexpr int kG2StagesA = QLORA_G2_STAGES_A;   // A half + NF4 codes: covers the TMA latency
 constexpr int kG2StagesB = QLORA_G2_STAGES_B;   // decoded B half: covers the signalling latency
 static_assert(kG2StagesA >= kG2StagesB, "B-slot reuse is gated through the A ring");
+// (bf16: 3 groups with 6 A stages and 6 B slots measured best against 4 groups with (8, 4) and
+// 3 groups with (6, 5), (6, 4); a B slot freed SB - 1 MMA steps back gives the hand-off from
+// the decoders that much slack.)
 // Each decoder group waits on full[] of the steps it handles; with the ring depth a multiple
 // of the group count, the previous phase of every such barrier belongs to a step the same
 // group has already observed, so no parity wait can alias.
