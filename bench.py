@@ -780,9 +780,9 @@ def extra_rows(q, torch, S, dev, peaks, args):
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one k_nf4_gemm2<0> launch at this workload,
 # from the ncu capture summarised in profiles/nf4_fused_gemm_q_proj_4096x4096_T4096.md
-# (43.27 MB read + 15.34 MB written; H is still partly in L2 when the kernel ends).  Set to
+# (43.21 MB read + 15.32 MB written; H is still partly in L2 when the kernel ends).  Set to
 # None whenever the kernel changes until it is captured again.
-GEMM_FWD_DRAM_BYTES = None
+GEMM_FWD_DRAM_BYTES = 43208704 + 15316480
 
 
 def main():
