@@ -638,6 +638,38 @@ def extra_rows(q, torch, S, dev, peaks, args):
                                    "bwd_tc_frac": flops_bwd(T, d, k, r) / (bmed * 1e-6) / 1e12 / tc}
     del wl, X, dH, H, U, dX, dA, dB, ws
 
+    # ---- 70B-class projections at 16384 tokens (8192x8192 and 28672x8192, r = 16): forward and
+    # backward calls; inputs drawn on the device (W0 ~ N(0, 0.02), X, dH ~ N(0, 1), A ~ N(0, 1/r),
+    # B ~ N(0, 0.01)), 2 NF4 copies of the weight (> L2 with the activations)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    for name in ("proj70b_8192x8192_r16_T16384", "proj70b_28672x8192_r16_T16384"):
+        cc = S.CONFIGS[name]
+        d4, k4, r4, a4, T4 = cc["d_out"], cc["d_in"], cc["r"], cc["alpha"], cc["T"]
+        wl = [q.nf4_quantize(torch.randn((d4, k4), generator=gen, device=dev) * (0.02 ** 0.5)) for _ in range(2)]
+        X = torch.randn((T4, k4), generator=gen, device=dev).to(bf)
+        dH = torch.randn((T4, d4), generator=gen, device=dev).to(bf)
+        A = (torch.randn((r4, k4), generator=gen, device=dev) / r4 ** 0.5).to(bf)
+        B = (torch.randn((d4, r4), generator=gen, device=dev) * 0.1).to(bf)
+        H = torch.empty((T4, d4), dtype=bf, device=dev)
+        U = torch.empty((T4, r4), dtype=bf, device=dev)
+        dX = torch.empty((T4, k4), dtype=bf, device=dev)
+        dA = torch.empty((r4, k4), dtype=torch.float32, device=dev)
+        dB = torch.empty((d4, r4), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(q.workspace_bytes(q.OP_FWD, q.BF16, T4, d4, k4, r4),
+                             q.workspace_bytes(q.OP_BWD, q.BF16, T4, d4, k4, r4)), dtype=torch.uint8, device=dev)
+        fwd = [(lambda w=w: q.qlora_linear_fwd(w, X, A, B, a4, H=H, U_save=U, ws=ws)) for w in wl]
+        bwd = [(lambda w=w: q.qlora_linear_bwd(w, X, dH, A, B, a4, U_saved=U, dX=dX, dA=dA, dB=dB, ws=ws))
+               for w in wl]
+        fmed, _ = _graph_time(torch, fwd, reps=3)
+        bmed, _ = _graph_time(torch, bwd, reps=3)
+        out[name] = {"fwd_us": fmed, "bwd_us": bmed,
+                     "fwd_tflops": flops_fwd(T4, d4, k4, r4) / (fmed * 1e-6) / 1e12,
+                     "bwd_tflops": flops_bwd(T4, d4, k4, r4) / (bmed * 1e-6) / 1e12,
+                     "fwd_tc_frac": flops_fwd(T4, d4, k4, r4) / (fmed * 1e-6) / 1e12 / tc,
+                     "bwd_tc_frac": flops_bwd(T4, d4, k4, r4) / (bmed * 1e-6) / 1e12 / tc}
+        del wl, X, dH, A, B, H, U, dX, dA, dB, ws
+
     # ---- multi-adapter forward: 4096^2 base, 4 adapters r = 8, 16, 16, 64, T = 4096
     for split_name, split in (("uniform", None), ("skewed", [0.7, 0.1, 0.1, 0.1])):
         mc = S.make_multi_adapter(4096, 4096, 4096, [8, 16, 16, 64], split=split, dtype="bf16", seed=5)

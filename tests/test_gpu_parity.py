@@ -152,6 +152,46 @@ def test_q_proj_full_size_sampled_rows(q):
     run_layer(q, case, rows=rows)
 
 
+# The remaining full-size configurations: Llama-2-7B MLP up/gate (11008x4096, r = 64, 8192
+# tokens) and the 70B-class projections (8192x8192 and 28672x8192, r = 16, 2048 and 16384
+# tokens), forward and backward; H and dX on 256 sampled token rows, dA and dB in full.  The
+# oracle's quantization and decode of a shape are shared by its two token counts (the weight is
+# the first draw of the seed).
+FULL_CONFIGS = ["mlp_up_11008x4096_r64_T8192", "proj70b_8192x8192_r16_T2048", "proj70b_8192x8192_r16_T16384",
+                "proj70b_28672x8192_r16_T2048", "proj70b_28672x8192_r16_T16384"]
+_ORACLE_W = {}
+
+
+def oracle_weight_cached(case, seed):
+    key = (case.d_out, case.d_in, seed)
+    if key not in _ORACLE_W:
+        _ORACLE_W.clear()
+        oc = O.nf4_quantize(case.W0)
+        _ORACLE_W[key] = oracle_weight(oc, case.d_out, case.d_in, "bf16")
+    return _ORACLE_W[key]
+
+
+@pytest.mark.parametrize("name", FULL_CONFIGS)
+def test_config_full_size_sampled_rows(q, name):
+    import torch
+    case = S.make_layer(**S.CONFIGS[name], seed=0)
+    Wh = oracle_weight_cached(case, 0)
+    w = q.nf4_quantize(dev(case.W0))
+    X, A, B, dH = dev(case.X, "bf16"), dev(case.A, "bf16"), dev(case.B, "bf16"), dev(case.dH, "bf16")
+    H, U = q.qlora_linear_fwd(w, X, A, B, case.alpha)
+    dX, dA, dB = q.qlora_linear_bwd(w, X, dH, A, B, case.alpha, U_saved=U)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    rows = np.sort(np.random.default_rng(1).choice(case.T, 256, replace=False))
+    ridx = torch.from_numpy(rows).cuda()
+    Href = O.lora_forward(Wh, case.X[rows], case.A, case.B, case.alpha, case.r)
+    dXref, _, _ = O.lora_backward(Wh, case.X[rows], case.dH[rows], case.A, case.B, case.alpha, case.r)
+    dAref, dBref = O.lora_adapter_grads(case.X, case.dH, case.A, case.B, case.alpha, case.r)
+    err = {"H": rel_fro(host(H[ridx]), Href), "dX": rel_fro(host(dX[ridx]), dXref),
+           "dA": rel_fro(host(dA), dAref), "dB": rel_fro(host(dB), dBref)}
+    assert all(v <= TOL["bf16"] for v in err.values()), err
+
+
 # ------------------------------------------------------------------ decode-size forward
 
 
