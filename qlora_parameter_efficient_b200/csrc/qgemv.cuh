@@ -308,7 +308,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 #pragma unroll
             for (int j = 0; j < NBW; ++j) {
                 const int L = warp + 8 * j;
-                if (L >= nbk) break;
+                // (no early exit: past the rank's K range the X fragments are zero and the scale
+                // is 0, and every read stays inside the stage buffer and the scale table)
                 // stage layout [piece L/4][16 rows][128 B], 128-byte swizzle: block L of a row is
                 // 16-byte chunks 2(L%4), 2(L%4)+1, stored at chunk ^ (row & 7)
                 const uint8_t* piece = st + (L >> 2) * 2048;
@@ -328,7 +329,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
                     for (int n = 0; n < NT8; ++n)
                         mma_bf16_16816(tmp[n], A[k], xw[j][n][2 * k], xw[j][n][2 * k + 1], k > 0);
                 // q8 * c2 of rows ra_, rb_ from the tile's scale table
-                const float sa = tab_s[ra_ * sld + L], sb = tab_s[rb_ * sld + L];
+                const float sa = L < nbk ? tab_s[ra_ * sld + L] : 0.f;
+                const float sb = L < nbk ? tab_s[rb_ * sld + L] : 0.f;
 #pragma unroll
                 for (int n = 0; n < NT8; ++n) {
                     acc[n][0] = fmaf(sa, tmp[n][0], acc[n][0]);
