@@ -6,7 +6,10 @@
  * fp32 second-level constant per group.  The layer computes
  *     h = W0 x + (alpha/r) B (A x)
  * with W0 dequantized on the fly to bf16 inside the tensor-core GEMM, its backward pass, the
- * adapter merge, and a multi-adapter forward over one shared base.
+ * adapter merge, multi-adapter forwards over one shared base (a few adapters, or thousands of
+ * mixed-rank adapters), DoRA's forward, the adapter optimizer step (AdamW, gradient
+ * accumulation, paged state), and the forward and backward with FP8 (E4M3 / E5M2) activations
+ * and gradients on FP8 tensor cores.
  *
  * Sources of each definition (page title, then section):
  *  [MF]  "Low-Rank Adaptation (LoRA) and QLoRA: Mathematical Foundations, Intrinsic Rank
