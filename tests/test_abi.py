@@ -51,6 +51,12 @@ def test_workspace_sizes(L):
     for op in (q.OP_FWD, q.OP_BWD, q.OP_FWD_BATCHED):
         for dt in (q.BF16, q.F32):
             assert q.workspace_bytes(op, dt, 4096, 4096, 4096, 16) > 0
+    for op in (q.OP_FWD_MULTI, q.OP_DORA_FWD, q.OP_FWD_FP8, q.OP_BWD_FP8, q.OP_FP8_QUANT):
+        assert q.workspace_bytes(op, q.BF16, 4096, 4096, 4096, 16) > 0
+        assert q.workspace_bytes(op, q.F32, 4096, 4096, 4096, 16) == 0      # bf16 only
+    # the FP8 backward needs the bf16 backward's scratch plus the exact bf16 copies of X8, dH8
+    assert (q.workspace_bytes(q.OP_BWD_FP8, q.BF16, 4096, 4096, 4096, 16)
+            >= q.workspace_bytes(q.OP_BWD, q.BF16, 4096, 4096, 4096, 16) + 2 * 2 * 4096 * 4096)
     assert q.workspace_bytes(q.OP_MERGE, q.BF16, 1, 64, 64, 8) == 0
     assert q.workspace_bytes(q.OP_FWD, q.BF16, 1, 64, 64, 129) == 0
     assert q.workspace_bytes(9, q.BF16, 1, 64, 64, 8) == 0
@@ -77,3 +83,26 @@ def test_host_validation_rejects_before_launch(L):
     assert r == 1                                # bad dtype
     r = L.qlora_linear_fwd(ctypes.byref(nf4), 16, 1, 16, 16, 8, 16.0, q.BF16, 16, None, 256, 10, None)
     assert r == 1                                # workspace too small
+
+
+def test_fp8_host_validation_rejects_before_launch(L):
+    nf4 = q._NF4(16, 16, 16, 64, 64)
+    # forward: a missing scale, a misaligned E4M3 activation
+    r = L.qlora_linear_fwd_fp8(ctypes.byref(nf4), 16, 1, None, 16, 16, 16, 8, 16.0, 16, 256, 1 << 20, None)
+    assert r == 1
+    r = L.qlora_linear_fwd_fp8(ctypes.byref(nf4), 17, 1, 16, 16, 16, 16, 8, 16.0, 16, 256, 1 << 20, None)
+    assert r == 1
+    # backward: gradient rows of d_out bytes must be whole 16-byte units (d_out = 200)
+    nf4b = q._NF4(16, 16, 16, 200, 64)
+    r = L.qlora_linear_bwd_fp8(ctypes.byref(nf4b), 16, 16, 16, 16, 16, 1, 16, 16, 8, 16.0, 16, 16, 16,
+                               256, 1 << 20, 0, None)
+    assert r == 2
+    # unknown flag bits
+    r = L.qlora_linear_bwd_fp8(ctypes.byref(nf4), 16, 16, 16, 16, 16, 1, 16, 16, 8, 16.0, 16, 16, 16,
+                               256, 1 << 20, 4, None)
+    assert r == 1
+    # quantizers: empty input, misaligned input, missing weight-scale output
+    assert L.qlora_fp8_quantize(16, 0, 16, 16, 256, 256, None) == 2
+    assert L.qlora_fp8_quantize(18, 64, 16, 16, 256, 256, None) == 1
+    assert L.qlora_fp8_quantize_grad(16, 0, 16, 16, 256, 256, None) == 2
+    assert L.qlora_fp8_weight_scale(ctypes.byref(nf4), None, None) == 1
