@@ -113,7 +113,6 @@ static_assert(kG2StagesA >= kG2StagesB, "B-slot reuse is gated through the A rin
 // of the group count, the previous phase of every such barrier belongs to a step the same
 // group has already observed, so no parity wait can alias.
 static_assert(kG2StagesA % kG2DecGroups == 0, "A-ring depth must be a multiple of the groups");
-constexpr int kG2Threads = 32 * (6 + 4 * kG2DecGroups);
 // FP8: a K step is 128 E4M3 columns (the same 128-byte rows), its codes tile twice as large,
 // so shared memory holds fewer stages: 3 decoder groups with 6 A stages and 3 decoded-B slots
 // (measured best of 1, 2, 3 or 4 groups with (8, 2), (6, 4), (6, 3), (6, 2), (4, 4) rings).
