@@ -6,8 +6,13 @@ provides device memory and streams.  There is no CPU fallback: if the library
 is missing or a call fails, an exception is raised.
 
 Names follow the C ABI: ``nf4_quantize``, ``nf4_dequantize``,
-``qlora_linear_fwd``, ``qlora_linear_bwd``, ``lora_merge``,
-``qlora_linear_fwd_batched``.
+``qlora_linear_fwd``, ``qlora_linear_bwd`` (``accumulate=`` for gradient
+accumulation), ``lora_merge``, ``qlora_linear_fwd_batched`` (a few adapters),
+``qlora_linear_fwd_multi`` with an ``AdapterTable`` (thousands of mixed-rank
+adapters), ``qlora_dora_fwd`` / ``dora_row_norms``, ``adamw_step`` /
+``prefetch`` (optimizer step, unified-memory state), and the FP8 path:
+``fp8_quantize`` (E4M3 activation), ``fp8_quantize_grad`` (E5M2 gradient),
+``fp8_weight_scale``, ``qlora_linear_fwd_fp8``, ``qlora_linear_bwd_fp8``.
 """
 from __future__ import annotations
 
