@@ -21,7 +21,9 @@ import os
 from dataclasses import dataclass
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libqlora.so")
+# QLORA_LIB selects another build of the same library (e.g. libqlora_debug.so, whose kernels
+# check their index invariants); either way a missing file raises.
+LIB_PATH = os.environ.get("QLORA_LIB") or os.path.join(HERE, "libqlora.so")
 
 QLORA_OK = 0
 STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",

@@ -21,6 +21,24 @@ __device__ __forceinline__ void set_error(int* err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
 
+// Debug checks.  Built with -DQLORA_DEBUG=1 (`python -m qlora_parameter_efficient_b200.build
+// --debug` -> libqlora_debug.so) the kernels check the index invariants their loads and stores
+// rely on: a failed check records QLORA_ERR_DEVICE in the device error word and the access is
+// skipped (no assert, no trap).  Release builds compile every check to `true`.
+#ifndef QLORA_DEBUG
+#define QLORA_DEBUG 0
+#endif
+__device__ __forceinline__ bool dcheck(bool ok, int* err) {
+#if QLORA_DEBUG
+    if (!ok) set_error(err, kErrDevice);
+    return ok;
+#else
+    (void)ok;
+    (void)err;
+    return true;
+#endif
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -568,6 +568,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThread
             if (wrow >= args.nf4_rows || wblk >= args.nf4_bpr) return;
             pr.nv = wblk + 1 < args.nf4_bpr ? 2 : 1;
             const int64_t b0 = wrow * args.nf4_bpr + wblk;
+            if (!dcheck(b0 + pr.nv <= static_cast<int64_t>(args.nf4_rows) * args.nf4_bpr, args.err)) {
+                pr.nv = 0;
+                return;
+            }
             for (int h = 0; h < pr.nv; ++h) {
                 pr.q8[h] = __ldg(args.absmax_q + b0 + h);
                 pr.c2[h] = __ldg(args.c2 + ((b0 + h) >> 8));
@@ -676,7 +680,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThread
                 wblk = it;
             }
             if (wrow >= args.nf4_rows || wblk >= args.nf4_bpr) return -1;
-            return wrow * args.nf4_bpr + wblk;
+            const int64_t blk = wrow * args.nf4_bpr + wblk;
+            return dcheck(blk < static_cast<int64_t>(args.nf4_rows) * args.nf4_bpr, args.err) ? blk : -1;
         };
         uint64_t* arrive_bar = rank == 0 ? ready : dec_done;   // local arrive either way
         // Software pipeline per handled step: the step's 64 weights are decoded into registers

@@ -329,8 +329,9 @@ __global__ void __launch_bounds__(kGvThreads, 1)
                     for (int n = 0; n < NT8; ++n)
                         mma_bf16_16816(tmp[n], A[k], xw[j][n][2 * k], xw[j][n][2 * k + 1], k > 0);
                 // q8 * c2 of rows ra_, rb_ from the tile's scale table
-                const float sa = L < nbk ? tab_s[ra_ * sld + L] : 0.f;
-                const float sb = L < nbk ? tab_s[rb_ * sld + L] : 0.f;
+                const bool in_tab = L < nbk && dcheck(rb_ * sld + L < kGvTabS, args.err);
+                const float sa = in_tab ? tab_s[ra_ * sld + L] : 0.f;
+                const float sb = in_tab ? tab_s[rb_ * sld + L] : 0.f;
 #pragma unroll
                 for (int n = 0; n < NT8; ++n) {
                     acc[n][0] = fmaf(sa, tmp[n][0], acc[n][0]);

@@ -122,7 +122,8 @@ __global__ void k_seg_scatter(SegArgs a) {
          t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int id = a.ids[t];
         if (id < 0 || id >= a.n) continue;
-        a.perm[atomicAdd(a.cursor + id, 1)] = static_cast<int32_t>(t);
+        const int slot = atomicAdd(a.cursor + id, 1);
+        if (dcheck(slot >= 0 && slot < a.T, a.err)) a.perm[slot] = static_cast<int32_t>(t);
     }
 }
 
@@ -163,6 +164,8 @@ __global__ void __launch_bounds__(128, QLORA_SEG_SHRINK_MINB) k_seg_shrink(SegAr
     for (int b = blockIdx.x; b < n_tiles; b += gridDim.x) {
     const int4 tl = a.tiles[b];
     const int i = tl.x, start = tl.y, rows = tl.z, r = tl.w;
+    if (!dcheck(i >= 0 && i < a.n && start >= 0 && rows >= 1 && rows <= kSegTile && start + rows <= a.T, a.err))
+        continue;                     // (uniform over the CTA: every thread reads the same entry)
     const __nv_bfloat16* Ai = a.A[i];
     if (!seg_adapter_ok(a, r, Ai)) {
         if (threadIdx.x == 0) set_error(a.err, kErrDevice);
@@ -273,6 +276,9 @@ __global__ void __launch_bounds__(128, QLORA_SEG_EXPAND_MINB) k_seg_expand(SegAr
     for (int b = blockIdx.x; b < n_tiles; b += gridDim.x) {
         const int4 tl = a.tiles[b];
         const int i = tl.x, start = tl.y, rows = tl.z, r = tl.w;
+        if (!dcheck(i >= 0 && i < a.n && start >= 0 && rows >= 1 && rows <= kSegTile && start + rows <= a.T,
+                    a.err))
+            continue;
         if (!seg_adapter_ok(a, r, a.A[i])) continue;     // reported by k_seg_shrink
         const int ksteps = (r + 15) / 16;
         const __nv_bfloat16* Bi = a.B[i];

@@ -106,3 +106,13 @@ def test_fp8_host_validation_rejects_before_launch(L):
     assert L.qlora_fp8_quantize(18, 64, 16, 16, 256, 256, None) == 1
     assert L.qlora_fp8_quantize_grad(16, 0, 16, 16, 256, 256, None) == 2
     assert L.qlora_fp8_weight_scale(ctypes.byref(nf4), None, None) == 1
+
+
+def test_debug_build_compiles_and_exports_every_symbol(tmp_path):
+    """The QLORA_DEBUG=1 build (device-side index checks reporting QLORA_ERR_DEVICE) compiles for
+    sm_100a and exports the same C ABI."""
+    from qlora_parameter_efficient_b200 import build
+    lib = build.build_library(force=True, debug=True, out=str(tmp_path / "libqlora_debug.so"))
+    D = ctypes.CDLL(lib)
+    for n in declared_functions():
+        assert hasattr(D, n), n
