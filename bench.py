@@ -23,6 +23,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -50,6 +52,26 @@ def flops_fwd(T, d, k, r):
 
 def flops_bwd(T, d, k, r):
     return 2 * T * d * k + 4 * T * r * (d + k)
+
+
+def w_bytes(d, k):
+    """Stored NF4 weight: codes + uint8 absmax + fp32 second-level constants (0.5159 B/param)."""
+    return d * k * (0.5 + 1 / 64) + 4 * ((d * k // 64 + 255) // 256)
+
+
+def bytes_fwd(T, d, k, r):
+    """Forward call: W, X read, H written, A and B read, U saved (bf16)."""
+    return w_bytes(d, k) + 2 * T * k + 2 * T * d + 2 * r * (d + k) + 2 * T * r
+
+
+def bytes_bwd(T, d, k, r):
+    """Backward call: W, X, dH, U, A, B read; dX (bf16), dA and dB (fp32) written."""
+    return w_bytes(d, k) + 2 * T * k + 2 * T * d + 2 * T * k + 2 * T * r + 2 * r * (d + k) + 4 * r * (d + k)
+
+
+def t_roof(flops, byts, peaks):
+    """max(FLOPs at the measured burst bf16 tensor peak, bytes at the measured HBM peak), s."""
+    return max(flops / (peaks["bf16_tflops"] * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -129,14 +151,39 @@ def oracle_threads():
         return len(os.sched_getaffinity(0))
 
 
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(target_s=10.0):
+    """The oracle timed on this host: all of its BLAS threads on a sample sized for about
+    target_s seconds, and one thread on a smaller sample (tokens/s is per-token work, so the
+    rates compare)."""
     t_small = oracle_sample(256)
     n = int(min(cfg()["T"], max(256, 256 * target_s / max(t_small, 1e-3))))
     n = max(256, (n // 256) * 256)
     t = oracle_sample(n, seed=1)
-    return {"value": n / t, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{n} of {cfg()['T']} tokens of {WORKLOAD}: NF4 decode + fp64 fwd + bwd "
-                      f"({t:.1f} s)"}
+    out = {"value": n / t, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+           "cpu_model": cpu_model(),
+           "sample": f"{n} of {cfg()['T']} tokens of {WORKLOAD}: NF4 decode + fp64 fwd + bwd "
+                     f"({t:.1f} s)"}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            n1 = 128
+            t1 = oracle_sample(n1, seed=2)
+        out["value_1core"] = n1 / t1
+        out["sample_1core"] = f"{n1} tokens on 1 thread ({t1:.1f} s)"
+    except Exception as e:          # threadpoolctl missing: report the all-core figure only
+        out["value_1core"] = None
+        out["sample_1core"] = f"not measured: {type(e).__name__}"
+    return out
 
 
 def run_reference(args):
@@ -261,15 +308,18 @@ def run_gpu(args):
         return ms, launches, g_ms
 
     W = max(3, args.warmup)
+
+    def fn_fwd(i):
+        s = sets[i % NSETS]
+        q.qlora_linear_fwd(s["w"], s["X"], s["A"], s["B"], alpha, H=H, U_save=U, ws=ws)
+
+    def fn_bwd(i):
+        s = sets[i % NSETS]
+        q.qlora_linear_bwd(s["w"], s["X"], s["dH"], s["A"], s["B"], alpha, U_saved=U, dX=dX, dA=dA,
+                           dB=dB, ws=ws)
+
     if args.only != "step":
         # One part of the step alone (for profiling a single kernel on the same workload).
-        fn_fwd = lambda i: q.qlora_linear_fwd(sets[i % NSETS]["w"], sets[i % NSETS]["X"],  # noqa: E731
-                                              sets[i % NSETS]["A"], sets[i % NSETS]["B"], alpha,
-                                              H=H, U_save=U, ws=ws)
-        fn_bwd = lambda i: q.qlora_linear_bwd(sets[i % NSETS]["w"], sets[i % NSETS]["X"],  # noqa: E731
-                                              sets[i % NSETS]["dH"], sets[i % NSETS]["A"],
-                                              sets[i % NSETS]["B"], alpha, U_saved=U, dX=dX,
-                                              dA=dA, dB=dB, ws=ws)
         ms, launches, _ = timed(fn_fwd if args.only == "fwd" else fn_bwd, args.steps, W)
         if rank == 0:
             print(json.dumps({"only": args.only, "ms_per_call": ms / args.steps,
@@ -283,18 +333,10 @@ def run_gpu(args):
     # Dominant kernel: the fused NF4-decode GEMM of the forward (its last launch in each
     # step is the dX GEMM, the first the forward one; the hook records the latest launch,
     # so time the forward alone with the hook on).
-    _, _, g_ms = timed(lambda i: q.qlora_linear_fwd(sets[i % NSETS]["w"], sets[i % NSETS]["X"],
-                                                    sets[i % NSETS]["A"], sets[i % NSETS]["B"], alpha,
-                                                    H=H, U_save=U, ws=ws),
-                       args.steps, W, with_gemm_events=True)
+    _, _, g_ms = timed(fn_fwd, args.steps, W, with_gemm_events=True)
     # forward alone and backward alone (device time)
-    fwd_ms, _, _ = timed(lambda i: q.qlora_linear_fwd(sets[i % NSETS]["w"], sets[i % NSETS]["X"],
-                                                      sets[i % NSETS]["A"], sets[i % NSETS]["B"], alpha,
-                                                      H=H, U_save=U, ws=ws), args.steps, W)
-    bwd_ms, _, _ = timed(lambda i: q.qlora_linear_bwd(sets[i % NSETS]["w"], sets[i % NSETS]["X"],
-                                                      sets[i % NSETS]["dH"], sets[i % NSETS]["A"],
-                                                      sets[i % NSETS]["B"], alpha, U_saved=U, dX=dX,
-                                                      dA=dA, dB=dB, ws=ws), args.steps, W)
+    fwd_ms, _, _ = timed(fn_fwd, args.steps, W)
+    bwd_ms, _, _ = timed(fn_bwd, args.steps, W)
 
     # ------------------------------------------------------------------ end to end
     # Each step: pinned host X, dH -> device, fwd + bwd through the C ABI, dA, dB -> host.  The
@@ -349,23 +391,49 @@ def run_gpu(args):
     torch.cuda.synchronize()
     e2e_ms = dp.max_over_ranks(ee0.elapsed_time(ee1), device=dev)
 
-    extra = {}
-    if args.extra and rank == 0:
-        extra = extra_rows(q, torch, S, dev, peaks, args)
+    # CUDA-graph timing of the step, the forward and the backward (median and min per call over
+    # 5 replays of 20 captured calls on the rotating input sets); one GPU only (no NCCL capture)
+    graph = None
+    if world == 1:
+        gs = _graph_time(torch, [(lambda i=i: step(i)) for i in range(NSETS)], reps=5)
+        gf = _graph_time(torch, [(lambda i=i: fn_fwd(i)) for i in range(NSETS)], reps=5)
+        gb = _graph_time(torch, [(lambda i=i: fn_bwd(i)) for i in range(NSETS)], reps=5)
+        graph = {"step_us_median": gs[0], "step_us_min": gs[1], "fwd_us_median": gf[0],
+                 "fwd_us_min": gf[1], "bwd_us_median": gb[0], "bwd_us_min": gb[1],
+                 "calls_per_graph": 20}
+
+    rows = {}
+    if world == 1 and rank == 0 and not args.no_rows:
+        rows = extra_rows(q, torch, S, dev, peaks, args)
 
     toks = T * args.steps * world
     value = toks / (ms / 1e3)
     gemm_flops = 2 * T * d * k + 2 * T * r * d           # base GEMM + adapter K-extension
     g_avg = statistics.mean(g_ms) if g_ms else None
     achieved = gemm_flops / (g_avg / 1e3) / 1e12 if g_avg else None
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    # the fused GEMM is timed alone (each launch bracketed by events, a few ms of work at full
+    # clock): the measured burst bf16 peak applies; the sustained one is given beside it
+    peak = peaks["bf16_tflops"]
+    peak_sus = peaks.get("bf16_tflops_sustained")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": (achieved / peak) if achieved else None,
                 "traffic": GEMM_FWD_DRAM_BYTES, "traffic_unit": "bytes per launch",
                 "kernel": "k_nf4_gemm2<0> (fused NF4 decode + adapter K-extension, 2-SM tcgen05)",
-                "peak_source": f"{peak_src} bf16_tflops_sustained",
-                "kernel_ms": g_avg}
+                "peak_source": f"{peak_src} bf16_tflops (burst: the kernel is timed alone)",
+                "frac_of_sustained": (achieved / peak_sus) if (achieved and peak_sus) else None,
+                "kernel_ms": g_avg, "algorithmic_flops_per_launch": gemm_flops}
     step_flops = flops_fwd(T, d, k, r) + flops_bwd(T, d, k, r)
+    tr_f = t_roof(flops_fwd(T, d, k, r), bytes_fwd(T, d, k, r), peaks)
+    tr_b = t_roof(flops_bwd(T, d, k, r), bytes_bwd(T, d, k, r), peaks)
+    call_roof = {"t_roof_fwd_us": tr_f * 1e6, "t_roof_bwd_us": tr_b * 1e6,
+                 "fwd": tr_f / (fwd_ms / args.steps / 1e3), "bwd": tr_b / (bwd_ms / args.steps / 1e3),
+                 "step": (tr_f + tr_b) / (ms / args.steps / 1e3),
+                 "definition": "t_roof / t_measured, t_roof = max(FLOPs / bf16_tflops (burst), "
+                               "bytes / hbm_gbs); eager timing"}
+    if graph:
+        call_roof["fwd_graph"] = tr_f * 1e6 / graph["fwd_us_median"]
+        call_roof["bwd_graph"] = tr_b * 1e6 / graph["bwd_us_median"]
+        call_roof["step_graph"] = (tr_f + tr_b) * 1e6 / graph["step_us_median"]
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": W, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -376,14 +444,17 @@ def run_gpu(args):
         "tflops": step_flops * args.steps * world / (ms / 1e3) / 1e12,
         "fwd_ms": fwd_ms / args.steps, "bwd_ms": bwd_ms / args.steps,
         "roofline": roofline,
+        "call_roofline": call_roof,
         "e2e": {"value": toks / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(Xd[0].numel() * 2 + dHd[0].numel() * 2),
                 "d2h_bytes_per_step": int(dA.numel() * 4 + dB.numel() * 4)},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
-    if extra:
-        line["rows"] = extra
+    if graph:
+        line["graph"] = graph
+    if rows:
+        line["rows"] = rows
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:
@@ -566,252 +637,260 @@ def _graph_time(torch, calls, reps=20):
     return statistics.median(samples), min(samples)
 
 
+def _kernel_us(torch, q, calls, n_warm):
+    """Median device time of the library's main kernel over eager calls (events recorded by the
+    library right around that kernel's launch), after n_warm calls."""
+    kev = []
+    for fn in calls:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        e1.record()
+        q.set_gemm_events(e0, e1)
+        fn()
+        q.set_gemm_events(None, None)
+        kev.append((e0, e1))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) * 1e3 for a, b in kev[n_warm:])
+
+
 def extra_rows(q, torch, S, dev, peaks, args):
     """The other rows of the hot path, each timed on the device by CUDA-graph replay over
-    rotating weight copies whose working set exceeds the 126 MB L2 (not part of the headline)."""
+    rotating weight copies whose working set exceeds the 126 MB L2 (median and min per call).
+    Fractions: "roof_frac" = t_roof / t, t_roof = max(FLOPs at the measured burst bf16 peak,
+    algorithmic bytes at the measured HBM peak) -- the same definition as the headline's
+    call_roofline; "tc_frac" is against the burst peak and "tc_frac_sustained" against the
+    sustained one (calls that run for seconds settle near it under the power cap)."""
     out = {}
     bf = torch.bfloat16
     hbm = peaks["hbm_gbs"]
-    tc = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tc = peaks["bf16_tflops"]
+    tcs = peaks.get("bf16_tflops_sustained", tc)
 
-    def w_bytes(d, k):
-        return d * k * (0.5 + 1 / 64) + 4 * ((d * k // 64 + 255) // 256)
-
-    # ---- decode-size forward (T = 1, 4, 16) on the 11008 x 4096 MLP shape, r = 64
-    c3 = S.CONFIGS["mlp_up_11008x4096_r64_T8192"]
-    d, k, r, alpha = c3["d_out"], c3["d_in"], c3["r"], c3["alpha"]
-    NW = 8      # 8 x 23 MB of NF4 weights
-    base = S.make_layer(d, k, r, alpha, 16, dtype="bf16", seed=7, with_grad=False)
-    W0 = torch.from_numpy(base.W0).to(dev)
-    wl = [q.nf4_quantize(W0) for _ in range(NW)]
-    del W0
-    A = torch.from_numpy(base.A).to(dev).to(bf)
-    B = torch.from_numpy(base.B).to(dev).to(bf)
-    for T in (1, 4, 16):
-        X = torch.from_numpy(base.X[:T]).to(dev).to(bf)
-        H = torch.empty((T, d), dtype=bf, device=dev)
-        ws = torch.empty(q.workspace_bytes(q.OP_FWD, q.BF16, T, d, k, r), dtype=torch.uint8, device=dev)
-        calls = [(lambda w=w: q.qlora_linear_fwd(w, X, A, B, alpha, H=H, ws=ws, save_u=False)) for w in wl]
-        med, mn = _graph_time(torch, calls)
-        # the stream kernel alone (events around it; eager calls)
-        kev = []
-        for i in range(3 * NW):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            e1.record()
-            q.set_gemm_events(e0, e1)
-            q.qlora_linear_fwd(wl[i % NW], X, A, B, alpha, H=H, ws=ws, save_u=False)
-            q.set_gemm_events(None, None)
-            kev.append((e0, e1))
+    def guarded(name, fn):
+        try:
+            fn()
+        except Exception as e:          # one row failing must not lose the others
+            out[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
         torch.cuda.synchronize()
-        kus = statistics.median(a.elapsed_time(b) * 1e3 for a, b in kev[NW:])
-        byts = w_bytes(d, k) + 2 * T * (k + d) + 2 * r * (d + k)
-        out[f"decode_T{T}"] = {"call_us": med, "call_us_min": mn, "kernel_us": kus,
-                               "GB/s": byts / (med * 1e-6) / 1e9, "hbm_frac": byts / (med * 1e-6) / 1e9 / hbm,
-                               "kernel_hbm_frac": byts / (kus * 1e-6) / 1e9 / hbm,
-                               "bytes": byts, "hbm_peak_gbs": hbm}
-    del wl
+        torch.cuda.empty_cache()
 
-    # ---- large-T forward and backward on the same shape, T = 8192
-    T = c3["T"]
-    case = S.make_layer(d, k, r, alpha, T, dtype="bf16", seed=11)
-    wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(2)]
-    X = torch.from_numpy(case.X).to(dev).to(bf)
-    dH = torch.from_numpy(case.dH).to(dev).to(bf)
-    del case
-    H = torch.empty((T, d), dtype=bf, device=dev)
-    U = torch.empty((T, r), dtype=bf, device=dev)
-    dX = torch.empty((T, k), dtype=bf, device=dev)
-    dA = torch.empty((r, k), dtype=torch.float32, device=dev)
-    dB = torch.empty((d, r), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(q.workspace_bytes(q.OP_FWD, q.BF16, T, d, k, r),
-                         q.workspace_bytes(q.OP_BWD, q.BF16, T, d, k, r)), dtype=torch.uint8, device=dev)
-    fwd = [(lambda w=w: q.qlora_linear_fwd(w, X, A, B, alpha, H=H, U_save=U, ws=ws)) for w in wl]
-    bwd = [(lambda w=w: q.qlora_linear_bwd(w, X, dH, A, B, alpha, U_saved=U, dX=dX, dA=dA, dB=dB, ws=ws))
-           for w in wl]
-    fmed, _ = _graph_time(torch, fwd, reps=5)
-    bmed, _ = _graph_time(torch, bwd, reps=5)
-    out["mlp_11008x4096_T8192"] = {"fwd_us": fmed, "bwd_us": bmed,
-                                   "fwd_tflops": flops_fwd(T, d, k, r) / (fmed * 1e-6) / 1e12,
-                                   "bwd_tflops": flops_bwd(T, d, k, r) / (bmed * 1e-6) / 1e12,
-                                   "fwd_tc_frac": flops_fwd(T, d, k, r) / (fmed * 1e-6) / 1e12 / tc,
-                                   "bwd_tc_frac": flops_bwd(T, d, k, r) / (bmed * 1e-6) / 1e12 / tc}
-    del wl, X, dH, H, U, dX, dA, dB, ws
+    def fwd_bwd_row(name, d, k, r, alpha, T, wl, X, dH, A, B, reps):
+        H = torch.empty((T, d), dtype=bf, device=dev)
+        U = torch.empty((T, r), dtype=bf, device=dev)
+        dX = torch.empty((T, k), dtype=bf, device=dev)
+        dA = torch.empty((r, k), dtype=torch.float32, device=dev)
+        dB = torch.empty((d, r), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(q.workspace_bytes(q.OP_FWD, q.BF16, T, d, k, r),
+                             q.workspace_bytes(q.OP_BWD, q.BF16, T, d, k, r)), dtype=torch.uint8, device=dev)
+        fwd = [(lambda w=w: q.qlora_linear_fwd(w, X, A, B, alpha, H=H, U_save=U, ws=ws)) for w in wl]
+        bwd = [(lambda w=w: q.qlora_linear_bwd(w, X, dH, A, B, alpha, U_saved=U, dX=dX, dA=dA, dB=dB,
+                                               ws=ws)) for w in wl]
+        fmed, fmin = _graph_time(torch, fwd, reps=reps)
+        bmed, bmin = _graph_time(torch, bwd, reps=reps)
+        ff, fb = flops_fwd(T, d, k, r), flops_bwd(T, d, k, r)
+        trf, trb = t_roof(ff, bytes_fwd(T, d, k, r), peaks), t_roof(fb, bytes_bwd(T, d, k, r), peaks)
+        out[name] = {"fwd_us": fmed, "fwd_us_min": fmin, "bwd_us": bmed, "bwd_us_min": bmin,
+                     "fwd_tflops": ff / (fmed * 1e-6) / 1e12, "bwd_tflops": fb / (bmed * 1e-6) / 1e12,
+                     "t_roof_fwd_us": trf * 1e6, "t_roof_bwd_us": trb * 1e6,
+                     "fwd_roof_frac": trf / (fmed * 1e-6), "bwd_roof_frac": trb / (bmed * 1e-6),
+                     "fwd_tc_frac_sustained": ff / (fmed * 1e-6) / 1e12 / tcs,
+                     "bwd_tc_frac_sustained": fb / (bmed * 1e-6) / 1e12 / tcs}
 
-    # ---- 70B-class projections at 16384 tokens (8192x8192 and 28672x8192, r = 16): forward and
-    # backward calls; inputs drawn on the device (W0 ~ N(0, 0.02), X, dH ~ N(0, 1), A ~ N(0, 1/r),
-    # B ~ N(0, 0.01)), 2 NF4 copies of the weight (> L2 with the activations)
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(7)
-    for name in ("proj70b_8192x8192_r16_T16384", "proj70b_28672x8192_r16_T16384"):
-        cc = S.CONFIGS[name]
-        d4, k4, r4, a4, T4 = cc["d_out"], cc["d_in"], cc["r"], cc["alpha"], cc["T"]
-        wl = [q.nf4_quantize(torch.randn((d4, k4), generator=gen, device=dev) * (0.02 ** 0.5)) for _ in range(2)]
-        X = torch.randn((T4, k4), generator=gen, device=dev).to(bf)
-        dH = torch.randn((T4, d4), generator=gen, device=dev).to(bf)
-        A = (torch.randn((r4, k4), generator=gen, device=dev) / r4 ** 0.5).to(bf)
-        B = (torch.randn((d4, r4), generator=gen, device=dev) * 0.1).to(bf)
-        H = torch.empty((T4, d4), dtype=bf, device=dev)
-        U = torch.empty((T4, r4), dtype=bf, device=dev)
-        dX = torch.empty((T4, k4), dtype=bf, device=dev)
-        dA = torch.empty((r4, k4), dtype=torch.float32, device=dev)
-        dB = torch.empty((d4, r4), dtype=torch.float32, device=dev)
-        ws = torch.empty(max(q.workspace_bytes(q.OP_FWD, q.BF16, T4, d4, k4, r4),
-                             q.workspace_bytes(q.OP_BWD, q.BF16, T4, d4, k4, r4)), dtype=torch.uint8, device=dev)
-        fwd = [(lambda w=w: q.qlora_linear_fwd(w, X, A, B, a4, H=H, U_save=U, ws=ws)) for w in wl]
-        bwd = [(lambda w=w: q.qlora_linear_bwd(w, X, dH, A, B, a4, U_saved=U, dX=dX, dA=dA, dB=dB, ws=ws))
-               for w in wl]
-        fmed, _ = _graph_time(torch, fwd, reps=3)
-        bmed, _ = _graph_time(torch, bwd, reps=3)
-        out[name] = {"fwd_us": fmed, "bwd_us": bmed,
-                     "fwd_tflops": flops_fwd(T4, d4, k4, r4) / (fmed * 1e-6) / 1e12,
-                     "bwd_tflops": flops_bwd(T4, d4, k4, r4) / (bmed * 1e-6) / 1e12,
-                     "fwd_tc_frac": flops_fwd(T4, d4, k4, r4) / (fmed * 1e-6) / 1e12 / tc,
-                     "bwd_tc_frac": flops_bwd(T4, d4, k4, r4) / (bmed * 1e-6) / 1e12 / tc}
-        del wl, X, dH, A, B, H, U, dX, dA, dB, ws
+    # ---- decode-size forward (T = 1, 4, 16) on the 11008 x 4096 MLP shape, r = 64: an HBM
+    # stream of the 4-bit weight (8 rotating copies, 8 x 25 MB > 2 x L2)
+    def decode_rows():
+        c3 = S.CONFIGS["mlp_up_11008x4096_r64_T8192"]
+        d, k, r, alpha = c3["d_out"], c3["d_in"], c3["r"], c3["alpha"]
+        NW = 8
+        base = S.make_layer(d, k, r, alpha, 16, dtype="bf16", seed=7, with_grad=False)
+        W0 = torch.from_numpy(base.W0).to(dev)
+        wl = [q.nf4_quantize(W0) for _ in range(NW)]
+        del W0
+        A = torch.from_numpy(base.A).to(dev).to(bf)
+        B = torch.from_numpy(base.B).to(dev).to(bf)
+        for T in (1, 4, 16):
+            X = torch.from_numpy(base.X[:T]).to(dev).to(bf)
+            H = torch.empty((T, d), dtype=bf, device=dev)
+            ws = torch.empty(q.workspace_bytes(q.OP_FWD, q.BF16, T, d, k, r), dtype=torch.uint8, device=dev)
+            calls = [(lambda w=w: q.qlora_linear_fwd(w, X, A, B, alpha, H=H, ws=ws, save_u=False)) for w in wl]
+            med, mn = _graph_time(torch, calls)
+            kus = _kernel_us(torch, q, calls * 3, NW)
+            byts = w_bytes(d, k) + 2 * T * (k + d) + 2 * r * (d + k)
+            out[f"decode_11008x4096_r64_T{T}"] = {
+                "call_us": med, "call_us_min": min(mn, med), "kernel_us": kus,
+                "GB/s": byts / (med * 1e-6) / 1e9, "hbm_frac": byts / (med * 1e-6) / 1e9 / hbm,
+                "kernel_hbm_frac": byts / (kus * 1e-6) / 1e9 / hbm, "bytes": byts,
+                "t_roof_us": t_roof(flops_fwd(T, d, k, r), byts, peaks) * 1e6,
+                "hbm_peak_gbs": hbm, "device_error": q.get_device_error()}
 
-    # ---- multi-adapter forward: 4096^2 base, 4 adapters r = 8, 16, 16, 64, T = 4096
-    for split_name, split in (("uniform", None), ("skewed", [0.7, 0.1, 0.1, 0.1])):
-        mc = S.make_multi_adapter(4096, 4096, 4096, [8, 16, 16, 64], split=split, dtype="bf16", seed=5)
-        wl = [q.nf4_quantize(torch.from_numpy(mc.W0).to(dev)) for _ in range(4)]
-        X = torch.from_numpy(mc.X).to(dev).to(bf)
-        ids = torch.from_numpy(mc.ids).to(dev)
-        As = [torch.from_numpy(a).to(dev).to(bf) for a in mc.As]
-        Bs = [torch.from_numpy(b).to(dev).to(bf) for b in mc.Bs]
-        H = torch.empty((4096, 4096), dtype=bf, device=dev)
-        ws = torch.empty(q.workspace_bytes(q.OP_FWD_BATCHED, q.BF16, 4096, 4096, 4096, sum(mc.ranks)),
-                         dtype=torch.uint8, device=dev)
-        calls = [(lambda w=w: q.qlora_linear_fwd_batched(w, X, ids, As, Bs, mc.alphas, H=H, ws=ws)) for w in wl]
-        med, _ = _graph_time(torch, calls, reps=10)
-        fl = 2 * 4096 * 4096 * 4096 + sum(2 * 4096 * rr * (4096 + 4096) for rr in mc.ranks) // len(mc.ranks)
-        out[f"batched_4x_{split_name}"] = {"fwd_us": med, "tflops": fl / (med * 1e-6) / 1e12,
-                                          "tc_frac": fl / (med * 1e-6) / 1e12 / tc}
-        del wl, X, ids, As, Bs, H, ws
+    # ---- large-T forward and backward on the MLP shape, T = 8192
+    def mlp_row():
+        c3 = S.CONFIGS["mlp_up_11008x4096_r64_T8192"]
+        d, k, r, alpha, T = c3["d_out"], c3["d_in"], c3["r"], c3["alpha"], c3["T"]
+        case = S.make_layer(d, k, r, alpha, T, dtype="bf16", seed=11)
+        wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(2)]
+        X = torch.from_numpy(case.X).to(dev).to(bf)
+        dH = torch.from_numpy(case.dH).to(dev).to(bf)
+        A = torch.from_numpy(case.A).to(dev).to(bf)
+        B = torch.from_numpy(case.B).to(dev).to(bf)
+        del case
+        fwd_bwd_row("mlp_11008x4096_r64_T8192", d, k, r, alpha, T, wl, X, dH, A, B, reps=5)
+
+    # ---- 70B-class projections (8192x8192 and 28672x8192, r = 16) at 2048 and 16384 tokens;
+    # inputs drawn on the device (W0 ~ N(0, 0.02), X, dH ~ N(0, 1), A ~ N(0, 1/r), B ~ N(0, 0.01)),
+    # 2 NF4 copies of the weight
+    def proj70b_rows():
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(7)
+        for shape in ("8192x8192", "28672x8192"):
+            for T4 in (2048, 16384):
+                name = f"proj70b_{shape}_r16_T{T4}"
+                cc = S.CONFIGS[name]
+                d4, k4, r4, a4 = cc["d_out"], cc["d_in"], cc["r"], cc["alpha"]
+                wl = [q.nf4_quantize(torch.randn((d4, k4), generator=gen, device=dev) * (0.02 ** 0.5))
+                      for _ in range(2)]
+                X = torch.randn((T4, k4), generator=gen, device=dev).to(bf)
+                dH = torch.randn((T4, d4), generator=gen, device=dev).to(bf)
+                A = (torch.randn((r4, k4), generator=gen, device=dev) / r4 ** 0.5).to(bf)
+                B = (torch.randn((d4, r4), generator=gen, device=dev) * 0.1).to(bf)
+                fwd_bwd_row(name, d4, k4, r4, a4, T4, wl, X, dH, A, B, reps=3 if T4 > 4096 else 10)
+                del wl, X, dH, A, B
+                torch.cuda.empty_cache()
+
+    # ---- multi-adapter forward: 4096^2 base, 4 adapters r = 8, 16, 16, 64 (alpha = 2r), T = 4096
+    def batched_rows():
+        for split_name, split in (("uniform", None), ("skewed", [0.7, 0.1, 0.1, 0.1])):
+            mc = S.make_multi_adapter(4096, 4096, 4096, [8, 16, 16, 64], split=split, dtype="bf16", seed=5)
+            wl = [q.nf4_quantize(torch.from_numpy(mc.W0).to(dev)) for _ in range(4)]
+            X = torch.from_numpy(mc.X).to(dev).to(bf)
+            ids = torch.from_numpy(mc.ids).to(dev)
+            As = [torch.from_numpy(a).to(dev).to(bf) for a in mc.As]
+            Bs = [torch.from_numpy(b).to(dev).to(bf) for b in mc.Bs]
+            H = torch.empty((4096, 4096), dtype=bf, device=dev)
+            ws = torch.empty(q.workspace_bytes(q.OP_FWD_BATCHED, q.BF16, 4096, 4096, 4096, sum(mc.ranks)),
+                             dtype=torch.uint8, device=dev)
+            calls = [(lambda w=w: q.qlora_linear_fwd_batched(w, X, ids, As, Bs, mc.alphas, H=H, ws=ws))
+                     for w in wl]
+            med, mn = _graph_time(torch, calls, reps=10)
+            counts = np.bincount(mc.ids, minlength=len(mc.ranks))
+            fl = 2 * 4096 * 4096 * 4096 + sum(int(c) * 2 * rr * (4096 + 4096) for c, rr in zip(counts, mc.ranks))
+            byts = w_bytes(4096, 4096) + 2 * 4096 * 4096 * 2 + sum(2 * rr * 8192 for rr in mc.ranks)
+            tr = t_roof(fl, byts, peaks)
+            out[f"batched_4096x4096_4x_{split_name}_T4096"] = {
+                "fwd_us": med, "fwd_us_min": mn, "tflops": fl / (med * 1e-6) / 1e12,
+                "t_roof_us": tr * 1e6, "roof_frac": tr / (med * 1e-6), "device_error": q.get_device_error()}
+            del wl, X, ids, As, Bs, H, ws
 
     # ---- many-adapter (segmented) forward: 4096^2 base, 1024 adapters of rank 16, T = 4096,
     # ids uniform (about 4 tokens per adapter); adapters drawn on the device (268 MB > L2)
-    n_ad, r_ad, T_ad = 1024, 16, 4096
-    wl, X, ids, tab, H, ws = make_multi_workload(q, torch, dev, n_ad, r_ad, T_ad)
-    calls = [(lambda w=w: q.qlora_linear_fwd_multi(w, X, ids, tab, H=H, ws=ws)) for w in wl]
-    med, _ = _graph_time(torch, calls, reps=10)
-    fl = 2 * T_ad * 4096 * 4096 + 2 * T_ad * r_ad * (4096 + 4096)
-    byts = w_bytes(4096, 4096) + 2 * T_ad * 4096 * 3 + n_ad * r_ad * (4096 + 4096) * 2
-    t_roof = max(fl / (tc * 1e12), byts / (hbm * 1e9))
-    out["multi_1024x_r16_T4096"] = {"fwd_us": med, "tokens/s": T_ad / (med * 1e-6),
-                                    "tflops": fl / (med * 1e-6) / 1e12, "t_roof_us": t_roof * 1e6,
-                                    "roof_frac": t_roof / (med * 1e-6), "adapter_MB": n_ad * r_ad * 8192 * 2 / 1e6}
-    del wl, X, ids, tab, H, ws
+    def multi_row():
+        n_ad, r_ad, T_ad = 1024, 16, 4096
+        wl, X, ids, tab, H, ws = make_multi_workload(q, torch, dev, n_ad, r_ad, T_ad)
+        calls = [(lambda w=w: q.qlora_linear_fwd_multi(w, X, ids, tab, H=H, ws=ws)) for w in wl]
+        med, mn = _graph_time(torch, calls, reps=10)
+        fl = 2 * T_ad * 4096 * 4096 + 2 * T_ad * r_ad * (4096 + 4096)
+        byts = w_bytes(4096, 4096) + 2 * T_ad * 4096 * 3 + n_ad * r_ad * (4096 + 4096) * 2
+        tr = t_roof(fl, byts, peaks)
+        out["multi_4096x4096_1024xr16_T4096"] = {
+            "fwd_us": med, "fwd_us_min": mn, "tokens/s": T_ad / (med * 1e-6),
+            "tflops": fl / (med * 1e-6) / 1e12, "t_roof_us": tr * 1e6, "roof_frac": tr / (med * 1e-6),
+            "adapter_MB": n_ad * r_ad * 8192 * 2 / 1e6, "device_error": q.get_device_error()}
 
     # ---- DoRA forward on the q_proj shape (4096^2, r = 16, T = 4096): row norms of W^ + sBA
     # (recomputed every call) + the fused forward with the m / n column scale
-    c2d = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
-    case = S.make_layer(c2d["d_out"], c2d["d_in"], c2d["r"], c2d["alpha"], c2d["T"], dtype="bf16",
-                        seed=17, with_grad=False)
-    wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(4)]
-    X = torch.from_numpy(case.X).to(dev).to(bf)
-    A = torch.from_numpy(case.A).to(dev).to(bf)
-    B = torch.from_numpy(case.B).to(dev).to(bf)
-    mag = torch.ones(c2d["d_out"], dtype=torch.float32, device=dev)
-    H = torch.empty((c2d["T"], c2d["d_out"]), dtype=bf, device=dev)
-    ws = torch.empty(q.workspace_bytes(q.OP_DORA_FWD, q.BF16, c2d["T"], c2d["d_out"], c2d["d_in"], c2d["r"]),
-                     dtype=torch.uint8, device=dev)
-    calls = [(lambda w=w: q.qlora_dora_fwd(w, X, A, B, c2d["alpha"], mag, H=H, save_u=False, ws=ws))
-             for w in wl]
-    med, _ = _graph_time(torch, calls, reps=10)
-    fl = flops_fwd(c2d["T"], c2d["d_out"], c2d["d_in"], c2d["r"]) + 2 * c2d["d_out"] * c2d["r"] * c2d["d_in"]
-    out["dora_fwd_4096x4096_r16_T4096"] = {"fwd_us": med, "tflops": fl / (med * 1e-6) / 1e12,
-                                           "tc_frac": fl / (med * 1e-6) / 1e12 / tc}
-    del wl, X, A, B, mag, H, ws, case
+    def dora_row():
+        c2d = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
+        d, k, r, al, T = c2d["d_out"], c2d["d_in"], c2d["r"], c2d["alpha"], c2d["T"]
+        case = S.make_layer(d, k, r, al, T, dtype="bf16", seed=17, with_grad=False)
+        wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(4)]
+        X = torch.from_numpy(case.X).to(dev).to(bf)
+        A = torch.from_numpy(case.A).to(dev).to(bf)
+        B = torch.from_numpy(case.B).to(dev).to(bf)
+        mag = torch.ones(d, dtype=torch.float32, device=dev)
+        H = torch.empty((T, d), dtype=bf, device=dev)
+        ws = torch.empty(q.workspace_bytes(q.OP_DORA_FWD, q.BF16, T, d, k, r), dtype=torch.uint8, device=dev)
+        calls = [(lambda w=w: q.qlora_dora_fwd(w, X, A, B, al, mag, H=H, save_u=False, ws=ws)) for w in wl]
+        med, mn = _graph_time(torch, calls, reps=10)
+        fl = flops_fwd(T, d, k, r) + 2 * d * r * k
+        tr = t_roof(fl, bytes_fwd(T, d, k, r), peaks)
+        out["dora_fwd_4096x4096_r16_T4096"] = {"fwd_us": med, "fwd_us_min": mn,
+                                               "tflops": fl / (med * 1e-6) / 1e12, "t_roof_us": tr * 1e6,
+                                               "roof_frac": tr / (med * 1e-6)}
 
-    # ---- FP8 forward on the q_proj shape (4096^2, r = 16, T = 4096): E4M3 activation, the weight
-    # decoded to E4M3 for kind::f8f6f4 tensor cores, the adapter term in bf16; the activation is
-    # quantized by its own (separately timed) call.  FP8 peak = measured bf16 x 2 (the dense
-    # fp8 : bf16 ratio of the part, 4.5 : 2.25 PFLOP/s).
-    c, wl, wsc, Xb, X8, xs, A, B, H, ws = make_fp8_workload(q, S, torch, dev)
-    calls = [(lambda w=w, sw=sw: q.qlora_linear_fwd_fp8(w, X8, xs, sw, A, B, c["alpha"], H=H, ws=ws))
-             for w, sw in zip(wl, wsc)]
-    med, _ = _graph_time(torch, calls, reps=10)
-    kev = []
-    for i in range(12):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        e1.record()
-        q.set_gemm_events(e0, e1)
-        q.qlora_linear_fwd_fp8(wl[i % 4], X8, xs, wsc[i % 4], A, B, c["alpha"], H=H, ws=ws)
-        q.set_gemm_events(None, None)
-        kev.append((e0, e1))
-    torch.cuda.synchronize()
-    kus = statistics.median(a.elapsed_time(b) * 1e3 for a, b in kev[4:])
-    qws = torch.empty(256, dtype=torch.uint8, device=dev)
-    qcalls = [(lambda: q.fp8_quantize(Xb, X8=X8, scale=xs, ws=qws))] * 4
-    qmed, _ = _graph_time(torch, qcalls, reps=10)
-    fl = flops_fwd(c["T"], c["d_out"], c["d_in"], c["r"])
-    tc8 = 2 * tc
-    qbytes = 3 * c["T"] * c["d_in"]
-    # the FP8 backward on the same workload (E5M2 gradient; dX on FP8 tensor cores, dA and dB
-    # from the E4M3 activation and E5M2 gradient dequantized to bf16)
-    G8, gs, dX, dA, dB, wsb = make_fp8_bwd_buffers(q, torch, dev, c)
-    bcalls = [(lambda w=w, sw=sw: q.qlora_linear_bwd_fp8(w, X8, xs, G8, gs, sw, A, B, c["alpha"], dX=dX, dA=dA,
-                                                         dB=dB, ws=wsb)) for w, sw in zip(wl, wsc)]
-    bmed, _ = _graph_time(torch, bcalls, reps=10)
-    kev = []
-    for i in range(12):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        e1.record()
-        q.set_gemm_events(e0, e1)
-        q.qlora_linear_bwd_fp8(wl[i % 4], X8, xs, G8, gs, wsc[i % 4], A, B, c["alpha"], dX=dX, dA=dA, dB=dB, ws=wsb)
-        q.set_gemm_events(None, None)
-        kev.append((e0, e1))
-    torch.cuda.synchronize()
-    bkus = statistics.median(a.elapsed_time(b) * 1e3 for a, b in kev[4:])
-    bfl = flops_bwd(c["T"], c["d_out"], c["d_in"], c["r"])
-    dxfl = 2 * c["T"] * c["d_out"] * c["d_in"] + 2 * c["T"] * c["r"] * c["d_in"]
-    out["fp8_fwd_4096x4096_r16_T4096"] = {
-        "fwd_us": med, "tflops": fl / (med * 1e-6) / 1e12, "tc_frac_fp8": fl / (med * 1e-6) / 1e12 / tc8,
-        "gemm_us": kus, "gemm_tc_frac_fp8": fl / (kus * 1e-6) / 1e12 / tc8, "fp8_peak_tflops": tc8,
-        "quantize_us": qmed, "quantize_hbm_frac": qbytes / (qmed * 1e-6) / 1e9 / hbm,
-        "bwd_us": bmed, "bwd_tflops": bfl / (bmed * 1e-6) / 1e12,
-        "dx_gemm_us": bkus, "dx_gemm_tc_frac_fp8": dxfl / (bkus * 1e-6) / 1e12 / tc8}
-    del wl, wsc, Xb, X8, xs, A, B, H, ws, qws, G8, gs, dX, dA, dB, wsb
+    # ---- FP8 forward and backward on the q_proj shape (4096^2, r = 16, T = 4096): E4M3
+    # activation, E5M2 gradient, the weight decoded to E4M3 for kind::f8f6f4 tensor cores, the
+    # adapter term in bf16.  FP8 peak = measured burst bf16 x 2 (the part's dense fp8 : bf16
+    # ratio, 4.5 : 2.25 PFLOP/s).
+    def fp8_row():
+        c, wl, wsc, Xb, X8, xs, A, B, H, ws = make_fp8_workload(q, S, torch, dev)
+        calls = [(lambda w=w, sw=sw: q.qlora_linear_fwd_fp8(w, X8, xs, sw, A, B, c["alpha"], H=H, ws=ws))
+                 for w, sw in zip(wl, wsc)]
+        med, mn = _graph_time(torch, calls, reps=10)
+        kus = _kernel_us(torch, q, calls * 3, 4)
+        qws = torch.empty(256, dtype=torch.uint8, device=dev)
+        qcalls = [(lambda: q.fp8_quantize(Xb, X8=X8, scale=xs, ws=qws))] * 4
+        qmed, _ = _graph_time(torch, qcalls, reps=10)
+        T, d, k, r = c["T"], c["d_out"], c["d_in"], c["r"]
+        fl = flops_fwd(T, d, k, r)
+        tc8 = 2 * tc
+        G8, gs, dX, dA, dB, wsb = make_fp8_bwd_buffers(q, torch, dev, c)
+        bcalls = [(lambda w=w, sw=sw: q.qlora_linear_bwd_fp8(w, X8, xs, G8, gs, sw, A, B, c["alpha"], dX=dX,
+                                                             dA=dA, dB=dB, ws=wsb)) for w, sw in zip(wl, wsc)]
+        bmed, bmn = _graph_time(torch, bcalls, reps=10)
+        bkus = _kernel_us(torch, q, bcalls * 3, 4)
+        bfl = flops_bwd(T, d, k, r)
+        dxfl = 2 * T * d * k + 2 * T * r * k
+        out["fp8_4096x4096_r16_T4096"] = {
+            "fwd_us": med, "fwd_us_min": mn, "tflops": fl / (med * 1e-6) / 1e12,
+            "tc_frac_fp8": fl / (med * 1e-6) / 1e12 / tc8, "gemm_us": kus,
+            "gemm_tc_frac_fp8": fl / (kus * 1e-6) / 1e12 / tc8, "fp8_peak_tflops": tc8,
+            "quantize_us": qmed, "quantize_hbm_frac": 3 * T * k / (qmed * 1e-6) / 1e9 / hbm,
+            "bwd_us": bmed, "bwd_us_min": bmn, "bwd_tflops": bfl / (bmed * 1e-6) / 1e12,
+            "dx_gemm_us": bkus, "dx_gemm_tc_frac_fp8": dxfl / (bkus * 1e-6) / 1e12 / tc8}
 
     # ---- AdamW step over the adapters of a 32-layer d = 4096 model with rank 16 on q, k, v, o:
     # 32 * 4 * 16 * (4096 + 4096) = 16.8 M parameters, bf16 params + fp32 master, m, v, grad
     # (30 bytes per parameter, 503 MB > L2)
-    n_p = 32 * 4 * 16 * 8192
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(3)
-    master = torch.randn(n_p, generator=gen, device=dev)
-    param = master.to(bf)
-    grad = torch.randn(n_p, generator=gen, device=dev)
-    m_s = torch.zeros(n_p, device=dev)
-    v_s = torch.zeros(n_p, device=dev)
-    calls = [(lambda t=t: q.adamw_step(param, grad, m_s, v_s, t, 1e-4, weight_decay=0.01, master=master))
-             for t in range(1, 5)]
-    med, _ = _graph_time(torch, calls, reps=10)
-    byts = 30 * n_p
-    out["adamw_16.8M_params"] = {"us": med, "GB/s": byts / (med * 1e-6) / 1e9,
-                                 "hbm_frac": byts / (med * 1e-6) / 1e9 / hbm}
-    del master, param, grad, m_s, v_s
+    def adamw_row():
+        n_p = 32 * 4 * 16 * 8192
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(3)
+        master = torch.randn(n_p, generator=gen, device=dev)
+        param = master.to(bf)
+        grad = torch.randn(n_p, generator=gen, device=dev)
+        m_s = torch.zeros(n_p, device=dev)
+        v_s = torch.zeros(n_p, device=dev)
+        calls = [(lambda t=t: q.adamw_step(param, grad, m_s, v_s, t, 1e-4, weight_decay=0.01, master=master))
+                 for t in range(1, 5)]
+        med, mn = _graph_time(torch, calls, reps=10)
+        byts = 30 * n_p
+        out["adamw_16.8M_params"] = {"us": med, "us_min": mn, "GB/s": byts / (med * 1e-6) / 1e9,
+                                     "hbm_frac": byts / (med * 1e-6) / 1e9 / hbm}
 
     # ---- merge W_final = W^ + s B A on the 4096^2 shape, bf16 out
-    c2_ = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
-    d, k, r, alpha = c2_["d_out"], c2_["d_in"], c2_["r"], c2_["alpha"]
-    case = S.make_layer(d, k, r, alpha, 1, dtype="bf16", seed=13, with_grad=False)
-    wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(8)]
-    A = torch.from_numpy(case.A).to(dev).to(bf)
-    B = torch.from_numpy(case.B).to(dev).to(bf)
-    outs = [torch.empty((d, k), dtype=bf, device=dev) for _ in range(8)]
-    calls = [(lambda w=w, o=o: q.lora_merge(w, A, B, alpha, bf, out=o)) for w, o in zip(wl, outs)]
-    med, _ = _graph_time(torch, calls, reps=10)
-    byts = w_bytes(d, k) + 2 * d * k + 2 * r * (d + k)
-    out["merge_4096x4096_bf16"] = {"us": med, "GB/s": byts / (med * 1e-6) / 1e9,
-                                   "hbm_frac": byts / (med * 1e-6) / 1e9 / hbm}
+    def merge_row():
+        c2_ = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
+        d, k, r, alpha = c2_["d_out"], c2_["d_in"], c2_["r"], c2_["alpha"]
+        case = S.make_layer(d, k, r, alpha, 1, dtype="bf16", seed=13, with_grad=False)
+        wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(8)]
+        A = torch.from_numpy(case.A).to(dev).to(bf)
+        B = torch.from_numpy(case.B).to(dev).to(bf)
+        outs = [torch.empty((d, k), dtype=bf, device=dev) for _ in range(8)]
+        calls = [(lambda w=w, o=o: q.lora_merge(w, A, B, alpha, bf, out=o)) for w, o in zip(wl, outs)]
+        med, mn = _graph_time(torch, calls, reps=10)
+        byts = w_bytes(d, k) + 2 * d * k + 2 * r * (d + k)
+        out["merge_4096x4096_r16_bf16"] = {"us": med, "us_min": mn, "GB/s": byts / (med * 1e-6) / 1e9,
+                                           "hbm_frac": byts / (med * 1e-6) / 1e9 / hbm}
+
+    for name, fn in (("decode", decode_rows), ("mlp", mlp_row), ("proj70b", proj70b_rows),
+                     ("batched", batched_rows), ("multi", multi_row), ("dora", dora_row),
+                     ("fp8", fp8_row), ("adamw", adamw_row), ("merge", merge_row)):
+        guarded(name, fn)
     return out
 
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one k_nf4_gemm2<0> launch at this workload,
-# from the ncu capture summarised in profiles/nf4_fused_gemm_q_proj_4096x4096_T4096.md
+# from an ncu capture of the forward call on the q_proj shape
 # (43.21 MB read + 15.32 MB written; H is still partly in L2 when the kernel ends).  Set to
 # None whenever the kernel changes until it is captured again.
 GEMM_FWD_DRAM_BYTES = 43208704 + 15316480
@@ -823,7 +902,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--extra", action="store_true", help="also time the other hot-path rows")
+    ap.add_argument("--no-rows", action="store_true",
+                    help="skip the other hot-path rows (decode-size sweep, 7B MLP, 70B-class, "
+                         "multi-adapter, DoRA, FP8, AdamW, merge) that a 1-GPU run reports")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--only", default="step", choices=["step", "fwd", "bwd", "decode", "multi", "fp8", "fp8bwd"],
                     help="time only the forward, only the backward, the decode-size forward "

@@ -34,6 +34,10 @@
  *    device error word that the next qlora_get_device_error() returns and clears.
  *  - Workspace: calls that take (ws, ws_bytes) need at least qlora_workspace_bytes(...) bytes
  *    of device scratch, 256-byte aligned; contents need not be initialised and are clobbered.
+ *  - The device error word's address is looked up again on every call made outside stream
+ *    capture (so a context re-created after cudaDeviceReset is followed) and cached per device
+ *    for calls made while the stream is captured: the first call on a device must precede any
+ *    capture.
  */
 #ifndef QLORA_H_
 #define QLORA_H_
@@ -204,7 +208,8 @@ qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t
  *               aligned (its rows then are too: d_in % 64 == 0 is already required)
  *   B_ptrs      DEVICE array of n_adapters device pointers, B_i bf16 [d_out, r_i]
  *   ranks       DEVICE int32 [n_adapters], 1 <= r_i <= r_max
- *   scales      DEVICE float [n_adapters], s_i (alpha_i / r_i)
+ *   alphas      DEVICE float [n_adapters], alpha_i; the library forms s_i = alpha_i / r_i
+ *               (IEEE fp32 division on the device, the same value the single-adapter calls use)
  *   r_max       host: the largest rank, 1..128; ws >= qlora_workspace_bytes(QLORA_OP_FWD_MULTI,
  *               QLORA_BF16, T, d_out, d_in, r_max)
  * 1 <= n_adapters <= 65536.  An id outside [0, n_adapters), or an adapter whose rank is
@@ -213,7 +218,7 @@ qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t
 qlora_status qlora_linear_fwd_multi(const qlora_nf4* w, const void* X, int64_t T,
                                     const int32_t* adapter_id, int32_t n_adapters,
                                     const void* const* A_ptrs, const void* const* B_ptrs,
-                                    const int32_t* ranks, const float* scales, int32_t r_max,
+                                    const int32_t* ranks, const float* alphas, int32_t r_max,
                                     void* H, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* DoRA (bf16): one magnitude per output row, each row of the adapted weight W + s B A divided
@@ -303,9 +308,13 @@ qlora_status qlora_linear_bwd_fp8(const qlora_nf4* w, const uint8_t* X8, const f
  * the computation and the other arguments are exactly those of qlora_linear_fwd.
  *   - QLORA_ERR_UNSUPPORTED, with nothing launched, when qlora_workspace_bytes(QLORA_OP_FWD,
  *     dtype, T, d_out, d_in, r) exceeds QLORA_NOALLOC_SCRATCH_BYTES.
- *   - All calls share the array; calls whose work overlaps on the GPU race on it.
- *   - The first call on a device looks up the array's device address; make it before any
- *     stream capture.                                                                        */
+ *   - Other errors are those of qlora_linear_fwd for the same arguments.
+ *   - All calls share the array, which keeps the previous call's contents (the forward's
+ *     kernels write every scratch byte before they read it); calls whose work overlaps on the
+ *     GPU (two streams, two host threads) race on it.
+ *   - The array's device address is looked up on every call made outside stream capture;
+ *     during a capture the address from the last such call on the device is used, so the first
+ *     call on a device must come before any stream capture.                                  */
 qlora_status qlora_linear_fwd_noalloc(const qlora_nf4* w, const void* X, int64_t T,
                                       const void* A, const void* B, int32_t r, float alpha,
                                       qlora_dtype dtype, void* H, void* U_save,

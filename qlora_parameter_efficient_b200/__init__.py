@@ -434,7 +434,8 @@ def qlora_linear_fwd_batched(w: NF4Weight, X, adapter_id, As, Bs, alphas, H=None
 
 class AdapterTable:
     """Device-resident adapter table for qlora_linear_fwd_multi: pointer arrays, ranks and
-    scales built once from lists of bf16 tensors A_i [r_i, d_in], B_i [d_out, r_i]."""
+    alphas uploaded once from lists of bf16 tensors A_i [r_i, d_in], B_i [d_out, r_i] (the
+    library forms alpha_i / r_i itself)."""
 
     def __init__(self, As, Bs, alphas):
         torch = _torch()
@@ -447,8 +448,7 @@ class AdapterTable:
         self.A_ptrs = torch.tensor([a.data_ptr() for a in As], dtype=torch.int64, device=dev)
         self.B_ptrs = torch.tensor([b.data_ptr() for b in Bs], dtype=torch.int64, device=dev)
         self.ranks = torch.tensor(self.ranks_host, dtype=torch.int32, device=dev)
-        self.scales = torch.tensor([float(al) / r for al, r in zip(alphas, self.ranks_host)],
-                                   dtype=torch.float32, device=dev)
+        self.alphas = torch.tensor([float(al) for al in alphas], dtype=torch.float32, device=dev)
 
 
 def qlora_linear_fwd_multi(w: NF4Weight, X, adapter_id, table: AdapterTable, H=None, ws=None,
@@ -462,7 +462,7 @@ def qlora_linear_fwd_multi(w: NF4Weight, X, adapter_id, table: AdapterTable, H=N
     c = w._c()
     _check("qlora_linear_fwd_multi", load().qlora_linear_fwd_multi(
         ctypes.byref(c), _ptr(X), T, _ptr(adapter_id), table.n, _ptr(table.A_ptrs),
-        _ptr(table.B_ptrs), _ptr(table.ranks), _ptr(table.scales), table.r_max, _ptr(H),
+        _ptr(table.B_ptrs), _ptr(table.ranks), _ptr(table.alphas), table.r_max, _ptr(H),
         _ptr(ws), ws.numel(), _stream(stream)))
     return H
 

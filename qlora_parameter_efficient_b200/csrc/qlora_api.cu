@@ -73,18 +73,32 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
-qlora_status err_word(int** out) {
+// The device address of a __device__ variable on the current device.  Looked up again on
+// every call made outside stream capture (a context torn down by cudaDeviceReset and re-created
+// may place the module's variables elsewhere), and taken from the per-device cache while the
+// stream is being captured, where the lookup may not be allowed; the first call on a device must
+// therefore come before any capture.
+qlora_status symbol_address(const void* symbol, void** cache, cudaStream_t stream, void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
-    if (!g_err_ptr[dev]) {
-        std::lock_guard<std::mutex> lk(g_mu);
-        if (!g_err_ptr[dev]) {
-            void* p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_qlora_error) != cudaSuccess) return QLORA_ERR_CUDA;
-            g_err_ptr[dev] = static_cast<int*>(p);
-        }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    const bool capturing = cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone;
+    if (capturing) cudaGetLastError();   // a refused query leaves no sticky error behind
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!capturing || !cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess || !p) return QLORA_ERR_CUDA;
+        cache[dev] = p;
     }
-    *out = g_err_ptr[dev];
+    *out = cache[dev];
+    return QLORA_OK;
+}
+
+qlora_status err_word(int** out, cudaStream_t stream) {
+    void* p = nullptr;
+    QL_TRY(symbol_address(reinterpret_cast<const void*>(&g_qlora_error), reinterpret_cast<void**>(g_err_ptr),
+                          stream, &p));
+    *out = static_cast<int*>(p);
     return QLORA_OK;
 }
 
@@ -1028,17 +1042,26 @@ qlora_status nf4_dequantize(const qlora_nf4* w, void* W_out, qlora_dtype out_dty
     return QLORA_ERR_INVALID_ARG;
 }
 
-qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T, const void* A,
-                              const void* B, int32_t r, float alpha, qlora_dtype dtype, void* H,
-                              void* U_save, void* ws, size_t ws_bytes, cudaStream_t stream) {
+// Argument checks of qlora_linear_fwd (everything but the workspace), shared with
+// qlora_linear_fwd_noalloc so that both return the same status for the same arguments.
+__attribute__((visibility("hidden"))) qlora_status qlora_fwd_check_args(
+    const qlora_nf4* w, const void* X, int64_t T, const void* A, const void* B, int32_t r,
+    qlora_dtype dtype, const void* H, const void* U_save) {
     QL_TRY(check_layer(w, T, r, dtype));
     if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) ||
         !aligned16_or_null(U_save))
         return QLORA_ERR_INVALID_ARG;
+    return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd(const qlora_nf4* w, const void* X, int64_t T, const void* A,
+                              const void* B, int32_t r, float alpha, qlora_dtype dtype, void* H,
+                              void* U_save, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    QL_TRY(qlora_fwd_check_args(w, X, T, A, B, r, dtype, H, U_save));
     const Plan p = make_plan(QLORA_OP_FWD, dtype, T, w->d_out, w->d_in, r);
     QL_TRY(check_ws(ws, ws_bytes, p.total));
     int* err = nullptr;
-    QL_TRY(err_word(&err));
+    QL_TRY(err_word(&err, stream));
     const int64_t d_out = w->d_out, d_in = w->d_in;
     const float s = alpha / static_cast<float>(r);
     if (p.small)
@@ -1078,7 +1101,7 @@ qlora_status qlora_dora_fwd(const qlora_nf4* w, const void* X, int64_t T, const 
     const Plan p = make_plan(QLORA_OP_DORA_FWD, QLORA_BF16, T, w->d_out, w->d_in, r);
     QL_TRY(check_ws(ws, ws_bytes, p.total));
     int* err = nullptr;
-    QL_TRY(err_word(&err));
+    QL_TRY(err_word(&err, stream));
     const float s = alpha / static_cast<float>(r);
     float* scale = at<float>(ws, p.dora_scale);
     QL_TRY(dora_scale(w, A, B, r, s, magnitude, at<float>(ws, p.dora_part), scale, stream));
@@ -1139,7 +1162,7 @@ qlora_status qlora_linear_bwd_fp8(const qlora_nf4* w, const uint8_t* X8, const f
     const Plan p = make_plan(QLORA_OP_BWD_FP8, QLORA_BF16, T, w->d_out, w->d_in, r);
     QL_TRY(check_ws(ws, ws_bytes, p.total));
     int* err = nullptr;
-    QL_TRY(err_word(&err));
+    QL_TRY(err_word(&err, stream));
     const int64_t d_out = w->d_out, d_in = w->d_in;
     // the stored FP8 tensors back in their own units (exact in bf16) for the skinny products
     auto* xb = at<__nv_bfloat16>(ws, p.f8_x);
@@ -1177,7 +1200,7 @@ qlora_status qlora_linear_fwd_fp8(const qlora_nf4* w, const uint8_t* X8, int64_t
     const Plan p = make_plan(QLORA_OP_FWD_FP8, QLORA_BF16, T, w->d_out, w->d_in, r);
     QL_TRY(check_ws(ws, ws_bytes, p.total));
     int* err = nullptr;
-    QL_TRY(err_word(&err));
+    QL_TRY(err_word(&err, stream));
     const int64_t d_out = w->d_out, d_in = w->d_in;
     const float s = alpha / static_cast<float>(r);
     const int RP = p.RP;
@@ -1220,7 +1243,7 @@ qlora_status qlora_linear_bwd_ex(const qlora_nf4* w, const void* X, const void* 
     const Plan p = make_plan(QLORA_OP_BWD, dtype, T, w->d_out, w->d_in, r);
     QL_TRY(check_ws(ws, ws_bytes, p.total));
     int* err = nullptr;
-    QL_TRY(err_word(&err));
+    QL_TRY(err_word(&err, stream));
     const int64_t d_out = w->d_out, d_in = w->d_in;
     const float s = alpha / static_cast<float>(r);
     if (dtype == QLORA_BF16)
@@ -1351,20 +1374,20 @@ qlora_status lora_merge(const qlora_nf4* w, const void* A, const void* B, int32_
 qlora_status qlora_linear_fwd_multi(const qlora_nf4* w, const void* X, int64_t T,
                                     const int32_t* adapter_id, int32_t n_adapters,
                                     const void* const* A_ptrs, const void* const* B_ptrs,
-                                    const int32_t* ranks, const float* scales, int32_t r_max,
+                                    const int32_t* ranks, const float* alphas, int32_t r_max,
                                     void* H, void* ws, size_t ws_bytes, cudaStream_t stream) {
-    if (!A_ptrs || !B_ptrs || !ranks || !scales || !adapter_id) return QLORA_ERR_INVALID_ARG;
+    if (!A_ptrs || !B_ptrs || !ranks || !alphas || !adapter_id) return QLORA_ERR_INVALID_ARG;
     if (n_adapters < 1 || n_adapters > kSegMaxAdapters) return QLORA_ERR_UNSUPPORTED;
     QL_TRY(check_layer(w, T, r_max, QLORA_BF16));
     if (!aligned16(X) || !aligned16(H) || (reinterpret_cast<uintptr_t>(adapter_id) & 3u) ||
         (reinterpret_cast<uintptr_t>(A_ptrs) & 7u) || (reinterpret_cast<uintptr_t>(B_ptrs) & 7u) ||
-        (reinterpret_cast<uintptr_t>(ranks) & 3u) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        (reinterpret_cast<uintptr_t>(ranks) & 3u) || (reinterpret_cast<uintptr_t>(alphas) & 3u))
         return QLORA_ERR_INVALID_ARG;
     if (T > (1LL << 31) - 1) return QLORA_ERR_UNSUPPORTED;
     const Plan p = make_plan(QLORA_OP_FWD_MULTI, QLORA_BF16, T, w->d_out, w->d_in, r_max);
     QL_TRY(check_ws(ws, ws_bytes, p.total));
     int* err = nullptr;
-    QL_TRY(err_word(&err));
+    QL_TRY(err_word(&err, stream));
     SegArgs a{};
     a.T = T;
     a.n = n_adapters;
@@ -1377,7 +1400,7 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4* w, const void* X, int64_t T
     a.A = reinterpret_cast<const __nv_bfloat16* const*>(A_ptrs);
     a.B = reinterpret_cast<const __nv_bfloat16* const*>(B_ptrs);
     a.ranks = ranks;
-    a.scales = scales;
+    a.alphas = alphas;
     a.cnt = at<int32_t>(ws, p.seg_cnt);
     a.seg_start = at<int32_t>(ws, p.seg_start);
     a.cursor = at<int32_t>(ws, p.seg_cursor);
@@ -1434,7 +1457,7 @@ qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t
     const Plan p = make_plan(QLORA_OP_FWD_BATCHED, dtype, T, w->d_out, w->d_in, R);
     QL_TRY(check_ws(ws, ws_bytes, p.total));
     int* err = nullptr;
-    QL_TRY(err_word(&err));
+    QL_TRY(err_word(&err, stream));
     const int64_t d_out = w->d_out, d_in = w->d_in;
     SegTable seg;
     for (int j = 0; j < 128; ++j) seg.seg_of[j] = -1;
@@ -1506,7 +1529,7 @@ qlora_status qlora_linear_fwd_batched(const qlora_nf4* w, const void* X, int64_t
 
 qlora_status qlora_get_device_error(cudaStream_t stream) {
     int* err = nullptr;
-    QL_TRY(err_word(&err));
+    QL_TRY(err_word(&err, stream));
     if (cudaStreamSynchronize(stream) != cudaSuccess) return QLORA_ERR_CUDA;
     int v = 0;
     if (cudaMemcpy(&v, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return QLORA_ERR_CUDA;
@@ -1520,7 +1543,7 @@ qlora_status qlora_get_device_error(cudaStream_t stream) {
 
 qlora_status qlora_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
     int* err = nullptr;
-    QL_TRY(err_word(&err));
+    QL_TRY(err_word(&err, stream));
     k_wait_timeout_selftest<<<1, 32, 0, stream>>>(err, limit_ns);
     QL_LAUNCH_CHECK();
     return QLORA_OK;

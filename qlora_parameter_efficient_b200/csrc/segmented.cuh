@@ -42,7 +42,7 @@ struct SegArgs {
     const __nv_bfloat16* const* A;    // [n] -> A_i [r_i, d_in]
     const __nv_bfloat16* const* B;    // [n] -> B_i [d_out, r_i]
     const int32_t* ranks;             // [n]
-    const float* scales;              // [n]
+    const float* alphas;              // [n] alpha_i; s_i = alpha_i / r_i is formed here
     int32_t* cnt;                     // [n] zero at launch of k_seg_count
     int32_t* seg_start;               // [n]
     int32_t* cursor;                  // [n]
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(128, QLORA_SEG_SHRINK_MINB) k_seg_shrink(SegAr
         }
     }
     __syncthreads();
-    const float s = a.scales[i];
+    const float s = __fdiv_rn(a.alphas[i], static_cast<float>(r));   // alpha_i / r_i
     const int rp = (r + 15) & ~15;
     for (int e = threadIdx.x; e < kSegTile * rp; e += blockDim.x) {
         const int row = e / rp, j = e % rp;

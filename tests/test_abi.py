@@ -116,3 +116,19 @@ def test_debug_build_compiles_and_exports_every_symbol(tmp_path):
     D = ctypes.CDLL(lib)
     for n in declared_functions():
         assert hasattr(D, n), n
+
+
+def test_noalloc_host_validation_matches_workspace_forward(L):
+    # The no-allocation forward checks its arguments exactly as qlora_linear_fwd does and
+    # returns the same status, before any CUDA call (nothing here reaches a device).
+    cases = [
+        (q._NF4(16, 16, 16, 64, 100), 16, 8, q.BF16),     # d_in not a multiple of 64
+        (q._NF4(16, 16, 16, 64, 64), 16, 200, q.BF16),    # r > 128
+        (q._NF4(16, 16, 16, 64, 64), 17, 8, q.BF16),      # misaligned X
+        (q._NF4(16, 16, 16, 64, 64), 16, 8, 7),           # unknown dtype
+        (q._NF4(16, 17, 16, 64, 64), 16, 8, q.BF16),      # misaligned absmax bytes
+    ]
+    for nf4, x_ptr, r, dt in cases:
+        ref = L.qlora_linear_fwd(ctypes.byref(nf4), x_ptr, 1, 16, 16, r, 16.0, dt, 16, None, 256, 1 << 20, None)
+        got = L.qlora_linear_fwd_noalloc(ctypes.byref(nf4), x_ptr, 1, 16, 16, r, 16.0, dt, 16, None, None)
+        assert ref != 0 and got == ref, (r, dt, ref, got)

@@ -6,6 +6,8 @@ Small cases span several 128x256 tiles with ragged tails in T, d_out, d_in and r
 full-size Llama-2-7B q_proj case is checked on sampled token rows (H, dX) and in full
 (dA, dB, decode).
 """
+import os
+
 import numpy as np
 import pytest
 
@@ -507,15 +509,25 @@ def test_adamw_state_in_unified_memory(q):
     """Optimizer state in cudaMallocManaged memory ("paged optimizers"), paged to the GPU
     before each step and back to the host after: bit-identical to device-resident state."""
     import ctypes, torch
+    import ctypes.util
+    torch.zeros(1, device="cuda")           # torch's CUDA runtime is loaded from here on
+    # the CUDA runtime this process already has mapped (torch's), else the loader's choice
+    names = []
+    with open("/proc/self/maps") as f:
+        for line in f:
+            path = line.split()[-1]
+            if "libcudart" in os.path.basename(path) and path not in names:
+                names.append(path)
+    names += [n for n in (ctypes.util.find_library("cudart"), "libcudart.so.12", "libcudart.so") if n]
     rt = None
-    for name in ("/usr/local/cuda/lib64/libcudart.so", "/usr/local/cuda/lib64/libcudart.so.12", "libcudart.so.12"):
+    for name in names:
         try:
             rt = ctypes.CDLL(name)
             break
         except OSError:
             continue
     if rt is None:
-        pytest.skip("no libcudart to allocate unified memory with")
+        pytest.skip("no CUDA runtime library to allocate unified memory with")
     rt.cudaMallocManaged.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_size_t, ctypes.c_uint]
     rt.cudaFree.argtypes = [ctypes.c_void_p]
     bufs = []
