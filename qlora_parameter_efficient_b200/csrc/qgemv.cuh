@@ -13,31 +13,33 @@
 // the output.  Identical in exact arithmetic; the level is rounded to bf16 before the scale
 // instead of after (relative 2^-9 per weight, averaging out in the sum).
 //
-// Why warp-level mma.sync and not tcgen05 here: one tcgen05.mma of M = 128, K = 16 occupies
-// the SM's tensor core for ~130-190 cycles whatever N is (measured on B200 with N = 16..256),
-// i.e. at most ~16 weights per cycle when the weights are the M x K operand -- well below the
-// stream rate.  mma.sync m16n8k16 (~900 MAC per SM cycle measured) takes its operands from
-// registers, so the codes decode (byte-permute arithmetic on the symmetric level table) straight
-// into A fragments.
+// Decode by table look-up.  A code byte holds two consecutive weights, and with the scale
+// factored out the pair's two bf16 levels depend on the byte alone: a 256-entry table of bf16x2
+// words turns a byte into an mma A register with one shared-memory load.  The table is
+// replicated per lane (entry e, lane l at byte e * 256 + 4 l), so the 32 loads of a warp hit 32
+// different banks whatever the bytes are, and the table starts on a 64 KB boundary of the
+// shared window: the load address of byte i of a code word is then a single byte permute of the
+// word and a per-lane constant (table address | 4 lane).  Two instructions per two weights, one of them on
+// the memory pipe, against ~4.5 integer instructions per two weights for arithmetic decoding.
 //
-// K order inside a block.  The dot product over a block's 64 K is order-free, so K is permuted
-// consistently in A and X: in k16 step j, mma K positions {2c, 2c+1, 2c+8, 2c+9} (thread c of
-// a quad) are block elements 16c + 4j + {0, 1, 2, 3}.  A thread's 8 code bytes 8c..8c+7 of a row
-// then supply its A registers of all four steps, and its X fragment is the 16 consecutive
-// elements 16c..16c+15 of the token's row.
-//
-// Work split.  The rows are cut into tiles of M rows (a multiple of 16, chosen per shape so
-// that the tiles fill the SMs); a cluster of C CTAs (C = 1, 2, 4 or 8) owns a contiguous range
-// of tiles and CTA rank p owns K blocks [kb_lo, kb_hi) of every row.  Warp w owns the blocks
-// kb_lo + w + 8j: their X fragments are loaded once into registers and stay there.  A stage is
-// 16 consecutive rows x the rank's K range -- 16 contiguous runs, one 3-D TMA box (pieces of 128
-// bytes, 128-byte swizzle, so the fragment reads are bank-conflict free); the warps take turns
-// issuing the refills.  Across the M/16 stages of a tile each warp accumulates q8 c2 x partial
-// in fp32 registers; the tile's absmax bytes and c2 values come in once per tile by cp.async.
-// At the end of a tile warp w sums 16-row group w over the 8 warps in warp order, the ranks' sums
-// meet in rank 0's shared memory over DSMEM, and rank 0 sums them in rank order, applies 1/127,
-// adds the adapter term (a few mma steps) and writes H.  No global partials, atomics or
+// Work split.  Rows come in tiles of 16; a cluster of C CTAs (C = 1, 2, 4 or 8) owns a
+// contiguous range of tiles and its 16 warps x C ranks split K: warp w of rank p owns the KB
+// consecutive 64-blocks starting at (16 p + w) KB (KB = 4 for up to 8 tokens, 2 for up to 16).
+// The warp's X fragments stay in registers for the whole kernel; per tile it streams the codes
+// of its 16 rows x KB blocks straight from global memory into registers (8 bytes of a row per
+// thread, the k order inside a block permuted consistently in the codes and X so that those 8
+// bytes are the thread's A registers of the block's four k16 steps), one tile ahead, with the
+// tile two ahead prefetched into L2.  Each warp writes its tile partial to shared memory; warp
+// (tile mod 16) sums the 16 partials in warp order, the ranks' sums meet in rank 0 over DSMEM
+// (rank order), and rank 0 applies 1/127, adds the adapter term with a few mma steps over bf16
+// s U (from the pre-pass) and the tile's B rows, and writes H.  Partial-sum buffers are double
+// buffered so that the warps run on while a tile is finalised.  No global partials, atomics or
 // semaphores: the sums are deterministic and the tail is on-chip.
+//
+// Why warp-level mma.sync and not tcgen05 here: one tcgen05.mma of M = 128, K = 16 occupies the
+// SM's tensor core for ~130-190 cycles whatever N is (measured on B200 with N = 16..256), i.e. at
+// most ~16 weights per cycle when the weights are the M x K operand, well below the stream rate;
+// mma.sync takes its A operand from registers, where the table look-up leaves it.
 #pragma once
 
 #include "common.cuh"
@@ -45,379 +47,399 @@
 
 namespace qlora {
 
-constexpr int kGvWarps = 8;
-constexpr int kGvThreads = 32 * kGvWarps;
-constexpr int kGvUsMax = 16 * 128; // s*U staging (bf16): T <= 16 tokens x r <= 128
-constexpr int kGvTabS = 6144;      // a tile's block scales: M x (kb_hi - kb_lo + 1) <= this
-constexpr int kGvRawC2 = 320;      // a tile's c2 groups: M x kt / 256 + 2 <= this
-constexpr int kGvBrowMax = 8192;  // a tile's adapter rows: M x (r + 8) bf16 <= this
+constexpr int kLvWarps = 16;                 // compute warps
+constexpr int kLvTableBytes = 256 * 128;     // 256 entries x 32 lanes x 4 bytes
+constexpr int kLvMaxRanks = 8;
+constexpr int kLvRpMax = 128;                // adapter rank padded to 16
+constexpr int kLvSuLd = kLvRpMax + 8;        // row stride (bf16) of s U and of staged B rows
 
 template <int NT8>
-struct GvCfg {
-    static constexpr int NT = 8 * NT8;                 // token tile
-    static constexpr int NBW = 8 / NT8;                // blocks per warp (X fragments in registers)
-    static constexpr int kMaxBlk = 8 * NBW;            // blocks of a CTA's K range
-    static constexpr int MW = NT8 == 1 ? 8 : 6;        // max 16-row groups per tile
-    static constexpr int kStage = 16 * kMaxBlk * 32;   // 16 rows x the K range (<= 32 KB)
-    static constexpr int S = NT8 == 1 ? 3 : 4;
-    static constexpr int kMaxRanks = NT8 == 1 ? 4 : 8;  // cluster size limit
-    static constexpr int kSlot = 32 * MW * NT8 * 16;   // one warp's partials of a tile
-    static constexpr int kTree = 8 * kSlot;            // every warp's partials
-    static constexpr int kRing = kMaxRanks * kSlot;    // rank 0: one CTA sum per rank
-    static constexpr int kStageOff = 0;
-    static constexpr int kTreeOff = kStageOff + S * kStage;
-    static constexpr int kRingOff = kTreeOff + kTree;
-    static constexpr int kUsOff = kRingOff + kRing;
-    static constexpr int kTabOff = kUsOff + kGvUsMax * 2;   // the tile's scales [M][nbk + 1] fp32
-    static constexpr int kBrowOff = kTabOff + kGvTabS * 4;  // the tile's B rows [M][r + 8] bf16
-    static constexpr int kRawOff = kBrowOff + kGvBrowMax * 2;   // [2] absmax bytes, then c2
-    static constexpr int kRawBuf = kGvTabS + kGvRawC2 * 4;
-    static constexpr int kBarOff = kRawOff + 2 * kRawBuf;
-    static constexpr int kSmem = kBarOff + 256 + 1024;   // barriers + alignment slack
+struct LvCfg {
+    static constexpr int KB = NT8 == 1 ? 4 : 2;                      // 64-blocks per warp
+    static constexpr int NBUF = NT8 == 1 ? 4 : 3;                    // tile partial buffers
+    static constexpr int S = NT8 == 1 ? 3 : 4;                       // code slices in flight per warp
+    static constexpr int kThreads = 32 * (kLvWarps + NBUF);          // + one finaliser per buffer
+    static constexpr int kMaxRanks = NT8 == 1 ? 8 : 4;
+    static constexpr int kRowBytes = KB * 32;                         // a warp's bytes of a row
+    static constexpr int kSlice = 16 * kRowBytes;                     // a warp's bytes of a tile
+    static constexpr int kTableOff = 0;
+    static constexpr int kCodesOff = kTableOff + kLvTableBytes;      // [warp][stage] slices
+    static constexpr int kPartOff = kCodesOff + kLvWarps * S * kSlice;   // [buf][warp][n][lane] float4
+    static constexpr int kRingOff = kPartOff + NBUF * kLvWarps * NT8 * 512;     // [buf][rank][n][lane] float4
+    static constexpr int kSuOff = kRingOff + NBUF * kMaxRanks * NT8 * 512;      // bf16 s U [16][kLvSuLd]
+    static constexpr int kSbOff = kSuOff + 16 * kLvSuLd * 2;         // bf16 B rows [NBUF][16][kLvSuLd]
+    static constexpr int kBarOff = kSbOff + NBUF * 16 * kLvSuLd * 2;
+    static constexpr int kSmem = kBarOff + 256;
     static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
-// 4-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros without reading.
-__device__ __forceinline__ void cp_async_4(void* dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)),
+struct LvArgs {
+    int T;                   // tokens (1..8 NT8)
+    int d_out, d_in, kt;     // kt = d_in / 64 (a multiple of 4)
+    int tiles;               // ceil(d_out / 16)
+    int C;                   // CTAs per cluster (K ranks)
+    int clusters;            // grid / C
+    int r, rp;               // adapter rank and its padding to 16
+    const uint8_t* codes;
+    const uint8_t* absmax_q;
+    const float* c2;
+    const __nv_bfloat16* X;       // [T][d_in]
+    const __nv_bfloat16* us_pad;  // [16][kLvSuLd] bf16(s U), zero beyond T and r (pre-pass)
+    const __nv_bfloat16* B;       // [d_out][r]
+    __nv_bfloat16* H;             // [T][d_out]
+    int* err;
+    uint64_t wait_ns;
+    uint32_t lv16[8];        // the 16 levels rounded to bf16, two per word (level 2i low)
+};
+
+// A load from the byte table or from a warp's own code slice: both are read-only while read (the
+// table after a barrier, a slice between its cp.async wait and the warp's next refill), so the
+// load is a pure function of its address and the compiler may batch and hoist it.
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
                  "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes)
                  : "memory");
 }
-// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros without reading.
-__device__ __forceinline__ void cp_async_16(void* dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),
-                 "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
-                 "r"(bytes)
-                 : "memory");
-}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float4 v) {
     asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x),
                  "f"(v.y), "f"(v.z), "f"(v.w)
                  : "memory");
 }
 
-
-struct GvArgs {
-    int T;                   // tokens (1..NT)
-    int d_out, d_in, kt;     // kt = d_in / 64 blocks per row (a multiple of 4)
-    int M;                   // rows per tile (multiple of 16, <= MMAX)
-    int tiles;               // ceil(d_out / M)
-    int C;                   // CTAs per cluster (K ranks)
-    int clusters;            // grid / C
-    int pieces;              // 128-byte pieces per row in a stage box: ceil(kt / 4 / C)
-    const __nv_bfloat16* X;  // [T][d_in]
-    const uint8_t* absmax_q;
-    const float* c2;
-    const float* us;         // [T][r]  s * U in fp32, from the pre-pass
-    const __nv_bfloat16* B;  // [d_out][r]
-    int r;
-    int b_vec;               // r % 8 == 0 (B rows are 16-byte aligned)
-    __nv_bfloat16* H;        // [T][d_out]
-    int* err;
-    uint64_t wait_ns;
-};
-
 template <int NT8>
-__global__ void __launch_bounds__(kGvThreads, 1)
-    k_qgemv(const __grid_constant__ CUtensorMap tmC, const GvArgs args) {
-    using Cf = GvCfg<NT8>;
-    constexpr int S = Cf::S, MW = Cf::MW, NT = Cf::NT, NBW = Cf::NBW;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
-    uint8_t* stages = smem + Cf::kStageOff;
-    float4* part = reinterpret_cast<float4*>(smem + Cf::kTreeOff);           // [8 warps][MW][NT8][32]
-    float4* ring = reinterpret_cast<float4*>(smem + Cf::kRingOff);           // [ranks][MW][NT8][32]
-    __nv_bfloat16* s_us = reinterpret_cast<__nv_bfloat16*>(smem + Cf::kUsOff);   // [NT][rp]
-    float* tab_s = reinterpret_cast<float*>(smem + Cf::kTabOff);             // [M][nbk + 1]
-    __nv_bfloat16* s_b = reinterpret_cast<__nv_bfloat16*>(smem + Cf::kBrowOff);  // [M][r + 8]
-    uint8_t* raw = smem + Cf::kRawOff;        // [2][absmax bytes [M][nbk] | c2 groups], by tile parity
+__global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
+    using Cf = LvCfg<NT8>;
+    constexpr int KB = Cf::KB, NBUF = Cf::NBUF, MR = Cf::kMaxRanks, S = Cf::S;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint32_t* table = reinterpret_cast<uint32_t*>(smem + Cf::kTableOff);
+    float4* part = reinterpret_cast<float4*>(smem + Cf::kPartOff);
+    float4* ring = reinterpret_cast<float4*>(smem + Cf::kRingOff);
+    __nv_bfloat16* s_us = reinterpret_cast<__nv_bfloat16*>(smem + Cf::kSuOff);
+    __nv_bfloat16* s_b = reinterpret_cast<__nv_bfloat16*>(smem + Cf::kSbOff);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::kBarOff);
-    uint64_t* full = bars;                     // [S] the stage's code box landed
-    uint64_t* empty = full + S;                // [S] all warps done with the stage
-    uint64_t* csync_bar = empty + S;           // the 8 warps meet
-    uint64_t* ring_full = csync_bar + 1;       // rank 0: every rank's sum of the tile is in
-    uint64_t* ring_free = ring_full + 1;       // every rank: rank 0 has consumed the ring
-    volatile int* abort = reinterpret_cast<volatile int*>(ring_free + 1);
+    uint64_t* full = bars;                  // [NBUF] the 16 warps' partials of a tile are in
+    uint64_t* freeb = bars + NBUF;          // [NBUF] the finaliser has read them
+    uint64_t* ring_full = bars + 2 * NBUF;  // [NBUF] rank 0: the other ranks' sums are in
+    uint64_t* ring_free = bars + 3 * NBUF;  // [NBUF] rank p: rank 0 has read this rank's sum
+    uint64_t* us_bar = bars + 4 * NBUF;     // rank 0: s U is staged
+    volatile int* abort = reinterpret_cast<volatile int*>(bars + 4 * NBUF + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, c = lane & 3;          // mma fragment coordinates
-    const int C = args.C;
-    const int rank = static_cast<int>(blockIdx.x) % C;      // cluster dims (C, 1, 1)
+    const int g = lane >> 2, q = lane & 3;
+    const int C = a.C;
+    const int rank = static_cast<int>(blockIdx.x) % C;
     const int cl = static_cast<int>(blockIdx.x) / C;
-    const int t_lo = static_cast<int>((static_cast<int64_t>(cl) * args.tiles) / args.clusters);
-    const int t_hi = static_cast<int>((static_cast<int64_t>(cl + 1) * args.tiles) / args.clusters);
-    const int q4 = args.kt / 4;
-    const int kb_lo = 4 * ((rank * q4) / C), kb_hi = 4 * (((rank + 1) * q4) / C);
-    const int nbk = kb_hi - kb_lo;
-    const int M = args.M, mw = M / 16;
-    const int n_units = (t_hi - t_lo) * mw;          // (tile, 16-row group) sequence
-
-    auto fail = [&]() {
-        set_error(args.err, kErrTimeout);
-        *abort = 1;
-    };
-    // ---- stage issue (one warp in turn, lane 0): 16 full rows of the rank's K range as one box
-    auto issue = [&](int u) {
-        if (lane != 0) return;
-        const int s = u % S;
-        const int row0 = (t_lo + u / mw) * M + (u % mw) * 16;
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(16 * 128 * args.pieces));
-        tma_load_3d(stages + s * Cf::kStage, &tmC, &full[s], 0, row0, kb_lo / 4);
-    };
+    const int t_lo = static_cast<int>((static_cast<int64_t>(cl) * a.tiles) / a.clusters);
+    const int t_hi = static_cast<int>((static_cast<int64_t>(cl + 1) * a.tiles) / a.clusters);
+    const int ntl = t_hi - t_lo;
+    const int64_t row_bytes = a.d_in / 2;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kGvWarps);
+        for (int i = 0; i < NBUF; ++i) {
+            mbar_init(&full[i], kLvWarps);
+            mbar_init(&freeb[i], 1);
+            mbar_init(&ring_full[i], C > 1 ? C - 1 : 1);
+            mbar_init(&ring_free[i], 1);
         }
-        mbar_init(csync_bar, kGvWarps);
-        mbar_init(ring_full, 32 * mw * C);
-        mbar_init(ring_free, 1);
+        mbar_init(us_bar, 1);
         *abort = 0;
-        fence_mbar_init();
-        tma_prefetch_desc(&tmC);
-        for (int u = 0; u < S - 1 && u < n_units; ++u) issue(u);
+        if (C > 1) fence_mbar_init();       // other CTAs of the cluster arrive on these
     }
-    const Nf4Planes planes = nf4_make_planes(1.0f);
-    // X fragments of this warp's blocks, held for the whole kernel: token 8n + g, elements
-    // 16c .. 16c + 15 of block kb_lo + warp + 8j
-    uint32_t xw[NBW][NT8][8];
+
+    const bool compute = warp < kLvWarps;
+    const int kb0 = (rank * kLvWarps + warp) * KB;          // this warp's first 64-block
+    const bool k_ok = compute && kb0 < a.kt;                // kt % 4 == 0: all KB blocks or none
+    // ---- compute warps: the warp's slice of tile li (16 rows x KB blocks) into its ring stage
+    // li % S, a row's 16-byte chunk c at chunk c ^ swz(row) (so that the fragment reads of 8 rows
+    // fall in different banks); rows past d_out are zero-filled
+    const uint32_t slices = smem_u32(smem + Cf::kCodesOff) + warp * S * Cf::kSlice;
+    auto swz = [](int row) { return KB == 4 ? (row & 7) : ((row >> 1) & 3); };
+    const uint8_t* const w0 = a.codes + static_cast<int64_t>(t_lo) * 16 * row_bytes + kb0 * 32;
+    auto issue_slice = [&](int li) {
+        if (k_ok && li < ntl) {
+            const uint32_t dst = slices + (li % S) * Cf::kSlice;
+            constexpr int kChunks = 16 * 2 * KB;            // 16-byte chunks of a slice
 #pragma unroll
-    for (int j = 0; j < NBW; ++j) {
-        const int L = warp + 8 * j;
-#pragma unroll
-        for (int n = 0; n < NT8; ++n) {
-            const int t = 8 * n + g;
-            uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
-            if (L < nbk && t < args.T) {
-                const uint4* src = reinterpret_cast<const uint4*>(args.X + static_cast<int64_t>(t) * args.d_in + (kb_lo + L) * 64 + 16 * c);
-                x0 = __ldg(src);
-                x1 = __ldg(src + 1);
+            for (int i = 0; i < kChunks / 32; ++i) {
+                const int idx = lane + 32 * i, row = idx / (2 * KB), c = idx % (2 * KB);
+                const bool ok = (t_lo + li) * 16 + row < a.d_out;
+                cp_async16(dst + row * Cf::kRowBytes + ((c ^ swz(row)) << 4),
+                           ok ? static_cast<const void*>(w0 + (static_cast<int64_t>(li) * 16 + row) * row_bytes + 16 * c)
+                              : static_cast<const void*>(a.codes),
+                           ok ? 16u : 0u);
             }
-            xw[j][n][0] = x0.x; xw[j][n][1] = x0.y; xw[j][n][2] = x0.z; xw[j][n][3] = x0.w;
-            xw[j][n][4] = x1.x; xw[j][n][5] = x1.y; xw[j][n][6] = x1.z; xw[j][n][7] = x1.w;
+        }
+        cp_async_commit();
+    };
+    // the tile's absmax bytes of rows g, g + 8 and each row's second-level constant (a warp's
+    // KB blocks never straddle a group of 256 blocks: kt and kb0 are multiples of KB)
+    struct Scales {
+        uint32_t qa, qb;
+        float c2a, c2b;
+    };
+    const int64_t ia0 = static_cast<int64_t>(t_lo * 16 + g) * a.kt + kb0;
+    auto load_scales = [&](int li, Scales& R) {
+        const int ra = (t_lo + li) * 16 + g, rb = ra + 8;
+        const bool va = k_ok && li < ntl && ra < a.d_out, vb = k_ok && li < ntl && rb < a.d_out;
+        const int64_t ia = ia0 + static_cast<int64_t>(li) * 16 * a.kt, ib = ia + 8 * static_cast<int64_t>(a.kt);
+        if constexpr (KB == 4) {
+            R.qa = va ? __ldg(reinterpret_cast<const uint32_t*>(a.absmax_q + ia)) : 0u;
+            R.qb = vb ? __ldg(reinterpret_cast<const uint32_t*>(a.absmax_q + ib)) : 0u;
+        } else {
+            R.qa = va ? static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(a.absmax_q + ia))) : 0u;
+            R.qb = vb ? static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(a.absmax_q + ib))) : 0u;
+        }
+        R.c2a = va ? __ldg(a.c2 + (ia >> 8)) : 0.f;
+        R.c2b = vb ? __ldg(a.c2 + (ib >> 8)) : 0.f;
+    };
+
+    Scales sc_cur;
+    uint32_t xw[KB][NT8][8];
+    if (compute) {
+        for (int st = 0; st < S - 1; ++st) issue_slice(st);
+        load_scales(0, sc_cur);
+        // X fragments of this warp's blocks, held for the whole kernel: token 8n + g, elements
+        // 16q .. 16q + 15 of block kb0 + b
+#pragma unroll
+        for (int b = 0; b < KB; ++b) {
+#pragma unroll
+            for (int n = 0; n < NT8; ++n) {
+                const int t = 8 * n + g;
+                uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
+                if (k_ok && t < a.T) {
+                    const uint4* src = reinterpret_cast<const uint4*>(a.X + static_cast<int64_t>(t) * a.d_in + (kb0 + b) * 64 + 16 * q);
+                    x0 = __ldg(src);
+                    x1 = __ldg(src + 1);
+                }
+                xw[b][n][0] = x0.x; xw[b][n][1] = x0.y; xw[b][n][2] = x0.z; xw[b][n][3] = x0.w;
+                xw[b][n][4] = x1.x; xw[b][n][5] = x1.y; xw[b][n][6] = x1.z; xw[b][n][7] = x1.w;
+            }
+        }
+        // the byte table: entry e = (high code << 4) | low code -> bf16x2 (L[low], L[high]), the
+        // same word for every lane; warp w writes entries w, w + 16, ...
+        const uint32_t pair = a.lv16[(lane & 15) >> 1];
+        const uint32_t lv = (lane & 1) ? (pair >> 16) : (pair & 0xFFFFu);   // bf16 of L[lane & 15]
+#pragma unroll 4
+        for (int e = warp; e < 256; e += kLvWarps) {
+            const uint32_t lo = __shfl_sync(0xffffffffu, lv, e & 15);
+            const uint32_t hi = __shfl_sync(0xffffffffu, lv, e >> 4);
+            table[e * 32 + lane] = lo | (hi << 16);
         }
     }
-    // barriers initialised (and visible cluster-wide) before any remote arrive or store
+    // barriers initialised (and visible cluster-wide) and the table written before use
     if (C > 1) cluster_barrier();
     else __syncthreads();
 
-    uint32_t phase = 0;
-    // bounded meeting point of the 8 warps (no hardware barrier that a warp leaving on a timeout
-    // could strand the others at)
-    auto csync = [&]() -> bool {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(csync_bar);
-        const bool ok = mbar_spin(csync_bar, phase & 1, abort, args.wait_ns);
-        ++phase;
-        return ok;
-    };
-
-    // the raw tables of a tile: absmax bytes [M][nbk] and its c2 groups, by all threads, into the
-    // buffer of the tile's parity
-    auto prefetch_tables = [&](int tile) {
-        const int row0 = tile * M;
-        uint8_t* rabs = raw + ((tile - t_lo) & 1) * Cf::kRawBuf;
-        float* rc2 = reinterpret_cast<float*>(rabs + kGvTabS);
-        const int wpr = nbk / 4;
-        for (int wi = threadIdx.x; wi < M * wpr; wi += kGvThreads) {
-            const int rr = wi / wpr, q = wi % wpr;
-            const bool ok = row0 + rr < args.d_out;
-            cp_async_4(rabs + rr * nbk + 4 * q,
-                       args.absmax_q + (ok ? static_cast<int64_t>(row0 + rr) * args.kt + kb_lo + 4 * q : 0),
-                       ok ? 4u : 0u);
-        }
-        const int64_t rlast = min(row0 + M, args.d_out) - 1;
-        const int64_t g_first = (static_cast<int64_t>(row0) * args.kt + kb_lo) >> 8;
-        const int n_c2 = static_cast<int>(((rlast * args.kt + kb_hi - 1) >> 8) - g_first + 1);
-        for (int e = threadIdx.x; e < n_c2; e += kGvThreads) cp_async_4(rc2 + e, args.c2 + g_first + e, 4u);
-    };
-    if (t_lo < t_hi) prefetch_tables(t_lo);
-    int last_issued = -1;       // latest stage this warp issued (beyond the initial ones)
-    bool ok_all = true;
-    int tiles_done = 0;
-
-    for (int tile = t_lo; tile < t_hi && ok_all; ++tile) {
-        const int row0 = tile * M;
-        // ---- the tile's block scales q8 * c2 [M][nbk + 1] from its raw tables (prefetched during
-        // the previous tile), then the next tile's raw tables and (rank 0) this tile's adapter
-        // rows go out; the previous tile's readers are past its end-of-tile meetings
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        if (!csync()) {
-            fail();
-            break;
-        }
-        const int sld = nbk + 1;                  // padded row: the 8 rows a warp reads hit 8 banks
-        {
-            const uint8_t* rabs = raw + ((tile - t_lo) & 1) * Cf::kRawBuf;
-            const float* rc2 = reinterpret_cast<const float*>(rabs + kGvTabS);
-            const int64_t g_first = (static_cast<int64_t>(row0) * args.kt + kb_lo) >> 8;
-            for (int e = threadIdx.x; e < M * nbk; e += kGvThreads) {
-                const int rr = e / nbk, L = e % nbk;
-                const int64_t blk = static_cast<int64_t>(row0 + rr) * args.kt + kb_lo + L;
-                tab_s[rr * sld + L] = row0 + rr < args.d_out
-                    ? static_cast<float>(rabs[e]) * rc2[(blk >> 8) - g_first] : 0.f;
-            }
-        }
-        if (!csync()) {
-            fail();
-            break;
-        }
-        if (rank == 0 && args.b_vec) {
-            const int cpr = args.r / 8;           // 16-byte pieces per row
-            for (int e = threadIdx.x; e < M * cpr; e += kGvThreads) {
-                const int rr = e / cpr, q = e % cpr;
-                const bool ok = row0 + rr < args.d_out;
-                cp_async_16(s_b + rr * (args.r + 8) + 8 * q,
-                            args.B + (ok ? static_cast<int64_t>(row0 + rr) * args.r + 8 * q : 0), ok ? 16u : 0u);
-            }
-        }
-        if (tile + 1 < t_hi) prefetch_tables(tile + 1);
-        // ---- the tile's 16-row groups, one stage each (a runtime loop: its body is emitted once)
-#pragma unroll 1
-        for (int m = 0; m < mw; ++m) {
-            const int u = (tile - t_lo) * mw + m;
-            const int s = u % S;
-            if (warp == u % kGvWarps && u + S - 1 < n_units) {
-                // refill the slot of stage u - 1 with stage u + S - 1 once every warp has left it
-                // (the warps take this duty in turn)
-                const int nxt = u + S - 1;
-                if (!mbar_wait_warp(&empty[nxt % S], ((nxt / S) & 1) ^ 1, abort, args.wait_ns)) {
-                    ok_all = false;
-                    break;
-                }
-                issue(nxt);
-                last_issued = nxt;
-            }
-            if (!mbar_wait_warp(&full[s], (u / S) & 1, abort, args.wait_ns)) {
-                ok_all = false;
-                break;
-            }
-            const uint8_t* st = stages + s * Cf::kStage;
-            const int ra_ = 16 * m + g, rb_ = ra_ + 8;          // rows within the tile
+    if (compute) {
+        // ================================================================ compute warps
+        const uint32_t lb = smem_u32(table) + (static_cast<uint32_t>(lane) << 2);
+        // table address of byte i of a code word: entry (byte << 7) + this lane's word
+        auto tab = [&](uint32_t w, uint32_t i) -> uint32_t { return lb + (prmt(w, 0u, 0x4440u | i) << 7); };
+        // the warp's part of tile li (its slice in stage li % S, its scales in R); false on a
+        // failed wait
+        auto process = [&](int li, const Scales& R) -> bool {
+            const int buf = li % NBUF;
+            const uint32_t slc = slices + (li % S) * Cf::kSlice;
             float acc[NT8][4];
 #pragma unroll
             for (int n = 0; n < NT8; ++n)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
 #pragma unroll
-            for (int j = 0; j < NBW; ++j) {
-                const int L = warp + 8 * j;
-                // (no early exit: past the rank's K range the X fragments are zero and the scale
-                // is 0, and every read stays inside the stage buffer and the scale table)
-                // stage layout [piece L/4][16 rows][128 B], 128-byte swizzle: block L of a row is
-                // 16-byte chunks 2(L%4), 2(L%4)+1, stored at chunk ^ (row & 7)
-                const uint8_t* piece = st + (L >> 2) * 2048;
-                const int chunk = ((((L & 3) * 2 + (c >> 1)) ^ g) << 4) + (c & 1) * 8;
-                const uint2 ca = *reinterpret_cast<const uint2*>(piece + g * 128 + chunk);
-                const uint2 cb = *reinterpret_cast<const uint2*>(piece + (g + 8) * 128 + chunk);
-                const uint4 a0 = nf4_decode8(ca.x, planes), a1 = nf4_decode8(ca.y, planes);
-                const uint4 b0 = nf4_decode8(cb.x, planes), b1 = nf4_decode8(cb.y, planes);
-                // A registers per k16 step: {row g: byte 2k, row g+8: byte 2k, row g: byte 2k+1,
-                // row g+8: byte 2k+1} of the thread's 8 bytes
-                const uint32_t A[4][4] = {{a0.x, b0.x, a0.y, b0.y}, {a0.z, b0.z, a0.w, b0.w},
-                                          {a1.x, b1.x, a1.y, b1.y}, {a1.z, b1.z, a1.w, b1.w}};
+            for (int b = 0; b < KB; ++b) {
+                // the thread's 8 code bytes of block b in rows g and g + 8: logical chunk
+                // 2b + q / 2, half q % 2
+                const int c = 2 * b + (q >> 1);
+                const uint2 ca = lds_v2(slc + g * Cf::kRowBytes + ((c ^ swz(g)) << 4) + ((q & 1) << 3));
+                const uint2 cb = lds_v2(slc + (g + 8) * Cf::kRowBytes + ((c ^ swz(g + 8)) << 4) + ((q & 1) << 3));
                 float tmp[NT8][4];
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
+                for (int s = 0; s < 4; ++s) {
+                    // A registers of k16 step s: bytes 2s (slots 2q, 2q+1) and 2s + 1 (slots
+                    // 2q+8, 2q+9) of the thread's 8 code bytes, rows g and g + 8
+                    const uint32_t wa = (s < 2) ? ca.x : ca.y;
+                    const uint32_t wb = (s < 2) ? cb.x : cb.y;
+                    const uint32_t i0 = 2 * (s & 1), i1 = i0 + 1;
+                    const uint32_t A[4] = {lds_u32(tab(wa, i0)), lds_u32(tab(wb, i0)), lds_u32(tab(wa, i1)),
+                                           lds_u32(tab(wb, i1))};
 #pragma unroll
                     for (int n = 0; n < NT8; ++n)
-                        mma_bf16_16816(tmp[n], A[k], xw[j][n][2 * k], xw[j][n][2 * k + 1], k > 0);
-                // q8 * c2 of rows ra_, rb_ from the tile's scale table
-                const bool in_tab = L < nbk && dcheck(rb_ * sld + L < kGvTabS, args.err);
-                const float sa = in_tab ? tab_s[ra_ * sld + L] : 0.f;
-                const float sb = in_tab ? tab_s[rb_ * sld + L] : 0.f;
+                        mma_bf16_16816(tmp[n], A, xw[b][n][2 * s], xw[b][n][2 * s + 1], s > 0);
+                }
+                // the unscaled block partial times the block's absmax byte; c2 multiplies the sum
+                const float qa = static_cast<float>((R.qa >> (8 * b)) & 0xFFu);
+                const float qb = static_cast<float>((R.qb >> (8 * b)) & 0xFFu);
 #pragma unroll
                 for (int n = 0; n < NT8; ++n) {
-                    acc[n][0] = fmaf(sa, tmp[n][0], acc[n][0]);
-                    acc[n][1] = fmaf(sa, tmp[n][1], acc[n][1]);
-                    acc[n][2] = fmaf(sb, tmp[n][2], acc[n][2]);
-                    acc[n][3] = fmaf(sb, tmp[n][3], acc[n][3]);
+                    acc[n][0] = fmaf(qa, tmp[n][0], acc[n][0]);
+                    acc[n][1] = fmaf(qa, tmp[n][1], acc[n][1]);
+                    acc[n][2] = fmaf(qb, tmp[n][2], acc[n][2]);
+                    acc[n][3] = fmaf(qb, tmp[n][3], acc[n][3]);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-            // the warp's partial of this 16-row group
+            // the warp's partial into this tile's buffer, free once the finaliser has read the
+            // tile NBUF back (1/127 is applied to the output)
+            if (li >= NBUF && !mbar_wait_warp(&freeb[buf], ((li / NBUF) - 1) & 1, abort, a.wait_ns)) {
+                set_error(a.err, kErrTimeout);
+                *abort = 1;
+                return false;
+            }
 #pragma unroll
             for (int n = 0; n < NT8; ++n)
-                part[((warp * MW + m) * NT8 + n) * 32 + lane] = make_float4(acc[n][0], acc[n][1], acc[n][2], acc[n][3]);
+                part[((buf * kLvWarps + warp) * NT8 + n) * 32 + lane] =
+                    make_float4(R.c2a * acc[n][0], R.c2a * acc[n][1], R.c2b * acc[n][2], R.c2b * acc[n][3]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[buf]);
+            return !*abort;
+        };
+        // per tile: refill the stage of the previous tile with the slice S - 1 ahead, wait for this
+        // tile's slice (the warp's own copies), then compute; scales ping-pong one tile ahead
+        Scales sc_nxt;
+        for (int li = 0; li < ntl; li += 2) {
+            __syncwarp();
+            issue_slice(li + S - 1);
+            load_scales(li + 1, sc_nxt);
+            cp_async_wait<S - 1>();
+            __syncwarp();
+            if (!process(li, sc_cur) || li + 1 >= ntl) break;
+            __syncwarp();
+            issue_slice(li + S);
+            load_scales(li + 2, sc_cur);
+            cp_async_wait<S - 1>();
+            __syncwarp();
+            if (!process(li + 1, sc_nxt)) break;
         }
-        if (!ok_all) {
-            fail();
-            break;
-        }
-
-        asm volatile("cp.async.wait_all;" ::: "memory");   // this tile's adapter rows
-        if (tiles_done == 0 && rank == 0) {
-            // s*U from the pre-pass as bf16 [NT][rp] (zero beyond T and r), once per CTA; the
-            // pre-pass has long finished by the end of the first tile
-            const int rp = (args.r + 15) & ~15;
+        cp_async_wait<0>();     // no copy in flight into the shared memory of an exiting CTA
+    } else {
+        // ================================================================ finaliser warps
+        // Finaliser f takes the tiles of buffer f (tile li -> warp 16 + li % NBUF): it sums the 16
+        // partials in warp order, sends the sum to rank 0 or (rank 0) adds the other ranks' sums in
+        // rank order, applies 1/127, adds the adapter term and writes H.  Each keeps the adapter
+        // rows of its next tile in flight (cp.async into its own s_b buffer).
+        const int f = warp - kLvWarps;
+        // (rank 0) s U from the pre-pass, staged by finaliser 0 once it has finished
+        if (rank == 0 && f == 0) {
             griddep_wait();
-            for (int e = threadIdx.x; e < NT * rp; e += kGvThreads) {
-                const int t = e / rp, jj = e % rp;
-                s_us[e] = __float2bfloat16_rn(t < args.T && jj < args.r ? args.us[t * args.r + jj] : 0.f);
-            }
+            const uint32_t dst = smem_u32(s_us);
+            for (int i = lane; i < 16 * kLvSuLd / 8; i += 32) cp_async16(dst + 16 * i, a.us_pad + 8 * i, 16u);
+            cp_async_commit();
+            cp_async_wait<0>();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(us_bar);
         }
-        // ---- end of the tile: warp w sums group w over the 8 warps in warp order and sends it to
-        // rank 0 (its own ring when C == 1)
-        if (!csync()) {
-            fail();
-            break;
-        }
-        if (warp < mw) {
-            float4 sum[NT8];
-#pragma unroll
-            for (int n = 0; n < NT8; ++n) {
-                sum[n] = part[(warp * NT8 + n) * 32 + lane];
-#pragma unroll
-                for (int w = 1; w < kGvWarps; ++w) {
-                    const float4 v = part[((w * MW + warp) * NT8 + n) * 32 + lane];
-                    sum[n].x += v.x;
-                    sum[n].y += v.y;
-                    sum[n].z += v.z;
-                    sum[n].w += v.w;
+        // the adapter rows of tile li into this finaliser's s_b buffer (one cp.async group; rows
+        // whose r bf16 are not whole 16-byte units are read at use instead)
+        const bool b_vec = (a.r % 8) == 0;
+        const int cpr = a.r / 8;                            // 16-byte pieces of a B row
+        __nv_bfloat16* const sbf = s_b + f * 16 * kLvSuLd;
+        auto stage_b = [&](int li) {
+            if (rank == 0 && b_vec && li < ntl) {
+                const int row0 = (t_lo + li) * 16;
+                for (int rr = 0; rr < 16; ++rr) {
+                    if (lane < cpr && row0 + rr < a.d_out)
+                        cp_async16(smem_u32(sbf + rr * kLvSuLd + 8 * lane),
+                                   a.B + static_cast<int64_t>(row0 + rr) * a.r + 8 * lane, 16u);
                 }
             }
-            if (tiles_done > 0 && !mbar_wait_warp(ring_free, (tiles_done - 1) & 1, abort, args.wait_ns)) {
-                fail();
+            cp_async_commit();
+        };
+        // B fragment e of k16 step kk for tile li: rows g (+8 for odd e), columns 16 kk + 2q (+8)
+        auto b_frag = [&](int li, int kk, int e) -> uint32_t {
+            const int rr = g + 8 * (e & 1), col = 16 * kk + 2 * q + 8 * (e >> 1);
+            const int row = (t_lo + li) * 16 + rr;
+            if (row >= a.d_out || col >= a.r) return 0u;
+            if (b_vec) return *reinterpret_cast<const uint32_t*>(sbf + rr * kLvSuLd + col);
+            const __nv_bfloat16* p = a.B + static_cast<int64_t>(row) * a.r + col;
+            const uint32_t lo = __ldg(reinterpret_cast<const unsigned short*>(p));
+            const uint32_t hi = col + 1 < a.r ? __ldg(reinterpret_cast<const unsigned short*>(p + 1)) : 0u;
+            return lo | (hi << 16);
+        };
+        stage_b(f);
+        bool us_ready = false;
+        for (int li = f; li < ntl; li += NBUF) {
+            const int buf = f;                              // li % NBUF
+            // ---- the 16 partials of the tile in warp order
+            if (!mbar_wait_warp(&full[buf], (li / NBUF) & 1, abort, a.wait_ns)) {
+                set_error(a.err, kErrTimeout);
+                *abort = 1;
                 break;
             }
-            const uint32_t dst = mapa_shared(smem_u32(ring + rank * (Cf::kSlot / 16) + (warp * NT8) * 32 + lane), 0);
-#pragma unroll
-            for (int n = 0; n < NT8; ++n) st_cluster_v4(dst + n * 32 * 16, sum[n]);
-            mbar_arrive_remote(mapa_shared(smem_u32(ring_full), 0));   // release.cluster
-        }
-        ++tiles_done;
-        if (rank != 0) continue;
-
-        // ---- rank 0: finalize the tile -- ranks in order, 1/127, adapter term, H.  Warp w
-        // takes m16 tiles w, w + 8, ...
-        if (!mbar_wait_cluster(ring_full, (tiles_done - 1) & 1, abort, args.wait_ns)) {
-            fail();
-            break;
-        }
-        const int rp = (args.r + 15) & ~15;          // adapter rank padded to the mma K
-        for (int m = warp; m < mw; m += kGvWarps) {
             float4 tot[NT8];
 #pragma unroll
-            for (int n = 0; n < NT8; ++n) tot[n] = ring[(m * NT8 + n) * 32 + lane];
-            for (int rr = 1; rr < C; ++rr) {
+            for (int n = 0; n < NT8; ++n) {
+                tot[n] = part[((buf * kLvWarps) * NT8 + n) * 32 + lane];
 #pragma unroll
-                for (int n = 0; n < NT8; ++n) {
-                    const float4 v = ring[rr * (Cf::kSlot / 16) + (m * NT8 + n) * 32 + lane];
+                for (int w = 1; w < kLvWarps; ++w) {
+                    const float4 v = part[((buf * kLvWarps + w) * NT8 + n) * 32 + lane];
                     tot[n].x += v.x;
                     tot[n].y += v.y;
                     tot[n].z += v.z;
                     tot[n].w += v.w;
                 }
             }
-            const int rbase = row0 + 16 * m;
-            // this thread's outputs: rows rbase + g, rbase + g + 8; tokens 8n + 2c, 8n + 2c + 1
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&freeb[buf]);
+            if (C > 1) {
+                if (rank != 0) {
+                    // this rank's sum to rank 0 (its ring slot is free once rank 0 has read the
+                    // sum of the tile NBUF back)
+                    if (li >= NBUF && !mbar_wait_warp(&ring_free[buf], ((li / NBUF) - 1) & 1, abort, a.wait_ns)) {
+                        set_error(a.err, kErrTimeout);
+                        *abort = 1;
+                        break;
+                    }
+#pragma unroll
+                    for (int n = 0; n < NT8; ++n)
+                        st_cluster_v4(mapa_shared(smem_u32(ring + ((buf * MR + rank) * NT8 + n) * 32 + lane), 0), tot[n]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&ring_full[buf]), 0));
+                    continue;
+                }
+                bool got = mbar_try_wait_acq_cluster(smem_u32(&ring_full[buf]), (li / NBUF) & 1);
+                if (!got) got = mbar_wait_cluster(&ring_full[buf], (li / NBUF) & 1, abort, a.wait_ns);
+                if (__shfl_sync(0xffffffffu, got ? 1u : 0u, 0) == 0u) {
+                    set_error(a.err, kErrTimeout);
+                    *abort = 1;
+                    break;
+                }
+                for (int p = 1; p < C; ++p) {
+#pragma unroll
+                    for (int n = 0; n < NT8; ++n) {
+                        const float4 v = ring[((buf * MR + p) * NT8 + n) * 32 + lane];
+                        tot[n].x += v.x;
+                        tot[n].y += v.y;
+                        tot[n].z += v.z;
+                        tot[n].w += v.w;
+                    }
+                }
+                __syncwarp();
+                // every rank's slot of this buffer is free again (its last use needs none)
+                if (lane >= 1 && lane < C && li + NBUF < ntl)
+                    mbar_arrive_remote(mapa_shared(smem_u32(&ring_free[buf]), static_cast<uint32_t>(lane)));
+            }
+            // ---- rank 0: 1/127, the adapter term (B rows times bf16 s U on the tensor cores,
+            // fp32 accumulation), H
+            if (!us_ready) {
+                if (!mbar_wait_warp(us_bar, 0, abort, a.wait_ns)) {
+                    set_error(a.err, kErrTimeout);
+                    *abort = 1;
+                    break;
+                }
+                us_ready = true;
+            }
             float out[2][NT8][2];
 #pragma unroll
             for (int n = 0; n < NT8; ++n) {
@@ -426,78 +448,175 @@ __global__ void __launch_bounds__(kGvThreads, 1)
                 out[1][n][0] = __fdiv_rn(tot[n].z, 127.0f);
                 out[1][n][1] = __fdiv_rn(tot[n].w, 127.0f);
             }
-            if (args.b_vec) {
-                // adapter term on the tensor cores: [16 rows x rp] B rows times [rp x NT]
-                // (s U)^T, fp32 accumulation
-                float adp[NT8][4];
-                for (int k0 = 0; k0 < rp; k0 += 16) {
-                    uint32_t a[4];
+            float adp[NT8][4];
 #pragma unroll
-                    for (int q2 = 0; q2 < 4; ++q2) {
-                        const int rr = 16 * m + g + 8 * (q2 & 1);     // row within the tile
-                        const int col = k0 + 2 * c + 8 * (q2 >> 1);
-                        a[q2] = col < args.r ? *reinterpret_cast<const uint32_t*>(s_b + rr * (args.r + 8) + col) : 0u;
-                    }
+            for (int n = 0; n < NT8; ++n)
 #pragma unroll
-                    for (int n = 0; n < NT8; ++n) {
-                        const __nv_bfloat16* ub = s_us + (8 * n + g) * rp + k0 + 2 * c;
-                        mma_bf16_16816(adp[n], a, *reinterpret_cast<const uint32_t*>(ub),
-                                       *reinterpret_cast<const uint32_t*>(ub + 8), k0 > 0);
-                    }
-                }
+                for (int e = 0; e < 4; ++e) adp[n][e] = 0.f;
+            cp_async_wait<0>();                             // this tile's B rows
+            __syncwarp();
+#pragma unroll
+            for (int kk = 0; kk < kLvRpMax / 16; ++kk) {
+                if (16 * kk >= a.rp) break;
+                const uint32_t af[4] = {b_frag(li, kk, 0), b_frag(li, kk, 1), b_frag(li, kk, 2), b_frag(li, kk, 3)};
 #pragma unroll
                 for (int n = 0; n < NT8; ++n) {
-                    out[0][n][0] += adp[n][0];
-                    out[0][n][1] += adp[n][1];
-                    out[1][n][0] += adp[n][2];
-                    out[1][n][1] += adp[n][3];
-                }
-            } else {
-                // r % 8 != 0: scalar adapter term
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int64_t grow = rbase + g + 8 * h;
-                    if (grow >= args.d_out) continue;
-                    const __nv_bfloat16* brow = args.B + grow * args.r;
-                    for (int j = 0; j < args.r; ++j) {
-                        const float bj = __bfloat162float(brow[j]);
-#pragma unroll
-                        for (int n = 0; n < NT8; ++n)
-#pragma unroll
-                            for (int e2 = 0; e2 < 2; ++e2)
-                                out[h][n][e2] = fmaf(__bfloat162float(s_us[(8 * n + 2 * c + e2) * rp + j]), bj, out[h][n][e2]);
-                    }
+                    const __nv_bfloat16* ub = s_us + (8 * n + g) * kLvSuLd + 16 * kk + 2 * q;
+                    mma_bf16_16816(adp[n], af, *reinterpret_cast<const uint32_t*>(ub),
+                                   *reinterpret_cast<const uint32_t*>(ub + 8), true);
                 }
             }
+            __syncwarp();
+            stage_b(li + NBUF);                             // this finaliser's next tile
+            const int ra = (t_lo + li) * 16 + g, rb = ra + 8;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const int64_t grow = rbase + g + 8 * h;
-                if (grow >= args.d_out) continue;
+                const int row = h ? rb : ra;
+                if (row >= a.d_out) continue;
 #pragma unroll
                 for (int n = 0; n < NT8; ++n)
 #pragma unroll
-                    for (int e2 = 0; e2 < 2; ++e2) {
-                        const int t = 8 * n + 2 * c + e2;
-                        if (t < args.T) args.H[static_cast<int64_t>(t) * args.d_out + grow] = __float2bfloat16_rn(out[h][n][e2]);
+                    for (int e = 0; e < 2; ++e) {
+                        const int t = 8 * n + 2 * q + e;
+                        if (t < a.T)
+                            a.H[static_cast<int64_t>(t) * a.d_out + row] =
+                                __float2bfloat16_rn(out[h][n][e] + adp[n][2 * h + e]);
                     }
             }
         }
-        // everyone is done with the ring: release it to every rank (the last tile needs none)
-        if (!csync()) {
-            fail();
-            break;
-        }
-        if (warp == 0 && lane < C && tile + 1 < t_hi)
-            mbar_arrive_remote(mapa_shared(smem_u32(ring_free), static_cast<uint32_t>(lane)));
+        cp_async_wait<0>();
     }
-    if (lane == 0 && *abort) {
-        // leave no copy in flight into shared memory of an exiting CTA: the stages this warp
-        // issued (thread 0 also the initial ones) are waited for, each bounded
-        if (warp == 0)
-            for (int i = 0; i < min(S - 1, n_units); ++i)
-                mbar_wait(&full[i % S], (i / S) & 1, nullptr, args.wait_ns);
-        if (last_issued >= 0)
-            mbar_wait(&full[last_issued % S], (last_issued / S) & 1, nullptr, args.wait_ns);
+    // a rank's shared memory is the target of the others' remote stores and arrives: no CTA of a
+    // cluster leaves before all are done (every wait above is bounded, so all arrive here)
+    if (C > 1) cluster_barrier();
+}
+
+// Pre-pass of the decode-size forward: U = X A^T on the tensor cores.  A cluster of KS CTAs owns
+// 16 adapter rows and splits K; warp w of rank p takes every 8th 64-block of the rank's share (the
+// same in-block k order as the stream kernel, at most 4 blocks per warp so that its loads are in
+// flight together); the warps' and then the ranks' partials are summed in order in rank 0, which
+// writes bf16(s U) into the padded [16][kLvSuLd] layout the stream kernel stages (zero beyond T
+// and r) and U (the call dtype, unscaled) for the backward.  It takes a few SMs of its own (the
+// stream kernel's grid leaves them free) and is launched with programmatic dependent launch: it
+// waits for the previous kernel, then lets the stream kernel start, whose finaliser reads its
+// output once it has finished.
+constexpr int kLuWarps = 8;
+struct LuArgs {
+    const __nv_bfloat16* X;
+    int T, d_in, kt;
+    const __nv_bfloat16* A;
+    int r;
+    float s;
+    int KS;                         // CTAs per cluster
+    __nv_bfloat16* us_pad;          // [16][kLvSuLd]
+    __nv_bfloat16* u_save;          // nullable [T][r]
+};
+
+__global__ void __launch_bounds__(32 * kLuWarps) k_lora_u_tc(const LuArgs a) {
+    griddep_wait();
+    griddep_launch_dependents();
+    __shared__ float4 red[kLuWarps][2][32];       // the warps' partials
+    __shared__ float4 rsum[kLvMaxRanks][2][32];   // rank 0: the ranks' sums
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int KS = a.KS;
+    const int rank = static_cast<int>(blockIdx.x) % KS;
+    const int j0 = (static_cast<int>(blockIdx.x) / KS) * 16;
+    const int lo = (rank * a.kt) / KS, hi = ((rank + 1) * a.kt) / KS;
+    const int ja = j0 + g, jb = ja + 8;
+    float acc[2][4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+    const int nt8 = a.T > 8 ? 2 : 1;
+    // at most 4 blocks per warp (the launch sizes KS for it): all of their loads in flight at once
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int blk = lo + warp + i * kLuWarps;
+        if (blk >= hi) break;
+        uint32_t ra[8], rb[8], xf[2][8];
+        auto ld8 = [&](uint32_t (&dst)[8], const __nv_bfloat16* src, bool ok) {
+            uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+            if (ok) {
+                v0 = __ldg(reinterpret_cast<const uint4*>(src));
+                v1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+            }
+            dst[0] = v0.x; dst[1] = v0.y; dst[2] = v0.z; dst[3] = v0.w;
+            dst[4] = v1.x; dst[5] = v1.y; dst[6] = v1.z; dst[7] = v1.w;
+        };
+        const int64_t col = static_cast<int64_t>(blk) * 64 + 16 * q;
+        ld8(ra, a.A + static_cast<int64_t>(ja) * a.d_in + col, ja < a.r);
+        ld8(rb, a.A + static_cast<int64_t>(jb) * a.d_in + col, jb < a.r);
+        ld8(xf[0], a.X + static_cast<int64_t>(g) * a.d_in + col, g < a.T);
+        ld8(xf[1], a.X + static_cast<int64_t>(8 + g) * a.d_in + col, nt8 > 1 && 8 + g < a.T);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const uint32_t af[4] = {ra[2 * s], rb[2 * s], ra[2 * s + 1], rb[2 * s + 1]};
+            mma_bf16_16816(acc[0], af, xf[0][2 * s], xf[0][2 * s + 1], true);
+            if (nt8 > 1) mma_bf16_16816(acc[1], af, xf[1][2 * s], xf[1][2 * s + 1], true);
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < 2; ++n) red[warp][n][lane] = make_float4(acc[n][0], acc[n][1], acc[n][2], acc[n][3]);
+    __syncthreads();
+    if (warp == 0) {
+        float4 tot[2];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+            tot[n] = red[0][n][lane];
+            for (int w = 1; w < kLuWarps; ++w) {
+                tot[n].x += red[w][n][lane].x;
+                tot[n].y += red[w][n][lane].y;
+                tot[n].z += red[w][n][lane].z;
+                tot[n].w += red[w][n][lane].w;
+            }
+        }
+        if (KS > 1) {
+            const uint32_t dst = mapa_shared(smem_u32(&rsum[rank][0][lane]), 0);
+#pragma unroll
+            for (int n = 0; n < 2; ++n) st_cluster_v4(dst + n * 32 * 16, tot[n]);
+        } else {
+#pragma unroll
+            for (int n = 0; n < 2; ++n) rsum[0][n][lane] = tot[n];
+        }
+    }
+    if (KS > 1) cluster_barrier();
+    else __syncthreads();
+    if (rank != 0 || warp != 0) return;
+    float4 tot[2];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+        tot[n] = rsum[0][n][lane];
+        for (int p = 1; p < KS; ++p) {
+            tot[n].x += rsum[p][n][lane].x;
+            tot[n].y += rsum[p][n][lane].y;
+            tot[n].z += rsum[p][n][lane].z;
+            tot[n].w += rsum[p][n][lane].w;
+        }
+    }
+    // thread (g, q) holds U[t][j] for j = ja, jb and t = 8n + 2q + e
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+        const float v[2][2] = {{tot[n].x, tot[n].y}, {tot[n].z, tot[n].w}};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int j = h ? jb : ja;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int t = 8 * n + 2 * q + e;
+                const bool valid = t < a.T && j < a.r;
+                a.us_pad[t * kLvSuLd + j] = __float2bfloat16_rn(valid ? a.s * v[h][e] : 0.f);
+                if (valid && a.u_save) a.u_save[static_cast<int64_t>(t) * a.r + j] = __float2bfloat16_rn(v[h][e]);
+            }
+        }
+    }
+    // the padding columns past the last group (one group writes them)
+    if (j0 == 0) {
+        const int rp = (a.r + 15) & ~15;
+        for (int i = lane; i < 16 * (kLvSuLd - rp); i += 32) {
+            const int t = i / (kLvSuLd - rp), j = rp + i % (kLvSuLd - rp);
+            a.us_pad[t * kLvSuLd + j] = __float2bfloat16_rn(0.f);
+        }
     }
 }
 

@@ -120,30 +120,17 @@ bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15
 bool aligned16_or_null(const void* p) { return !p || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// bf16 bits of a finite fp32 value, round to nearest even (the NF4 levels, on the host)
+inline uint32_t bf16_bits(float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+}
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // ======================================================================= TMA descriptors
 
-// 3-D tensor map over a row-major matrix viewed as [dim2 = column blocks][dim1 = rows]
-// [dim0 = inner bytes of a block]: one box brings box2 consecutive column blocks of box1 rows,
-// laid out block-major in shared memory.  elem = element size, inner = elements per block.
-qlora_status tmap_blocks(CUtensorMap* m, CUtensorMapDataType dt, uint32_t elem, const void* base,
-                         int64_t rows, int64_t row_bytes, uint32_t inner, uint32_t box1,
-                         uint32_t box2, CUtensorMapSwizzle sw) {
-    QL_TRY(get_encoder());
-    const int64_t blocks = row_bytes / (static_cast<int64_t>(inner) * elem);
-    cuuint64_t dims[3] = {inner, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(blocks)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(inner) * elem};
-    cuuint32_t box[3] = {inner, box1, box2};
-    cuuint32_t es[3] = {1, 1, 1};
-    CUresult r = g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? QLORA_OK : QLORA_ERR_CUDA;
-}
-
-// bf16 matrix [rows, cols] (cols contiguous, row stride ld elements), 128-byte swizzle,
-// box = 64 columns x box_rows rows.
 qlora_status tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
                        uint32_t box_rows) {
     QL_TRY(get_encoder());
@@ -227,16 +214,21 @@ MidPlan make_mid_plan(int64_t T, int64_t d_out, int64_t d_in) {
 
 struct SmallPlan {
     bool ok = false;
-    int nt8 = 1, kt = 0;
+    int nt8 = 1, kt = 0, C = 1, ks = 1;
 };
+// Decode-size forward: 16 warps x C ranks split K in slices of KB 64-blocks (4 for up to 8
+// tokens, 2 for up to 16); d_in a multiple of 256 and at most 8 ranks.
 SmallPlan make_small_plan(int64_t T, int64_t d_out, int64_t d_in) {
     SmallPlan sp;
     (void)d_out;
     if (T < 1 || T > kSmallT) return sp;
     sp.nt8 = T <= 8 ? 1 : 2;
-    if (sp.nt8 == 2) return sp;          // 9..16 tokens: the mid-size path is faster
     sp.kt = static_cast<int>(d_in / 64);
-    sp.ok = sp.kt % 4 == 0;
+    const int kb = sp.nt8 == 1 ? 4 : 2;
+    sp.C = static_cast<int>(cdiv(sp.kt, kLvWarps * kb));
+    // U pre-pass: K ranks per cluster, at most 4 blocks for each of a CTA's warps
+    sp.ks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kLvMaxRanks, cdiv(sp.kt, 4 * kLuWarps))));
+    sp.ok = sp.kt % 4 == 0 && sp.C <= (sp.nt8 == 1 ? LvCfg<1>::kMaxRanks : LvCfg<2>::kMaxRanks);
     return sp;
 }
 
@@ -330,7 +322,7 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
     if (dora) op = QLORA_OP_FWD;          // the forward's plan, never the decode-size path
     if (!dora && op == QLORA_OP_FWD && dtype == QLORA_BF16 && make_small_plan(T, d_out, d_in).ok) {
         p.small = true;
-        p.s_us = take(static_cast<size_t>(T) * r * 4);
+        p.s_us = take(static_cast<size_t>(16) * kLvSuLd * 2);   // bf16 s U, padded
         p.total = off;
         return p;
     }
@@ -573,27 +565,19 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
     return QLORA_OK;
 }
 
-// The stream kernel leaves 8 SMs to the U pre-pass (which takes ceil(r / 8) <= 16 CTAs), so the
-// two run side by side.
-constexpr int kGvStreamSms = kSmsForSplit - 8;
-
-// Decode-size forward: the U pre-pass overlapped with the weight stream through programmatic
-// dependent launch; the stream kernel runs as clusters of C CTAs over tiles of M rows.
+// Decode-size forward: the tensor-core U pre-pass (a few clusters of 128-thread CTAs that fit
+// beside the stream kernel's CTAs) and the stream kernel, both launched with programmatic
+// dependent launch so that the stream starts while U is computed.
 template <int NT8>
-qlora_status launch_qgemv(const qlora_nf4* w, const void* X, int64_t T, GvArgs g, cudaStream_t st) {
-    (void)X;
-    (void)T;
-    auto kern = k_qgemv<NT8>;
-    constexpr int smem = GvCfg<NT8>::kSmem;
+qlora_status launch_qgemv(LvArgs g, int ks, const LuArgs& u, cudaStream_t st) {
     int dev = 0;
     cudaGetDevice(&dev);
-    // per device and cluster size 1, 2, 4, 8: clusters that fit at once (0 = not queried,
-    // -1 = none)
-    static std::atomic<int> fit[64][4];
     static std::atomic<uint64_t> configured{0};
+    static std::atomic<int> fit[64][kLvMaxRanks + 1];   // clusters of C CTAs that fit at once
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load() & bit)) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        if (cudaFuncSetAttribute(k_qgemv_lut<NT8>, cudaFuncAttributeMaxDynamicSharedMemorySize, LvCfg<NT8>::kSmem) !=
+            cudaSuccess)
             return QLORA_ERR_CUDA;
         configured.fetch_or(bit);
     }
@@ -604,71 +588,44 @@ qlora_status launch_qgemv(const qlora_nf4* w, const void* X, int64_t T, GvArgs g
     attr[1].val.clusterDim.y = 1;
     attr[1].val.clusterDim.z = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kGvThreads);
-    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-    cfg.stream = st;
     cfg.attrs = attr;
-    const int64_t d_out = g.d_out, q4 = g.kt / 4;
-    int64_t best_cost = -1;
-    int best_C = 0, best_M = 0, best_clusters = 0;
-    for (int e = 0; e < 4; ++e) {
-        const int C = 1 << e;
-        if (C > q4 || C > GvCfg<NT8>::kMaxRanks) break;
-        if (4 * cdiv(q4, C) > GvCfg<NT8>::kMaxBlk) continue;
-        int n = fit[dev & 63][e].load();
-        if (n == 0) {
-            if (C == 1) {
-                n = kGvStreamSms;
-            } else {
-                attr[1].val.clusterDim.x = static_cast<unsigned>(C);
-                cfg.gridDim = dim3(static_cast<unsigned>(C * (kSmsForSplit / C)));
-                cfg.numAttrs = 2;
-                int m = 0;
-                if (cudaOccupancyMaxActiveClusters(&m, kern, &cfg) != cudaSuccess) {
-                    cudaGetLastError();
-                    m = 0;
-                }
-                n = std::min(m, kGvStreamSms / C);
+    cfg.stream = st;
+    // the U pre-pass
+    attr[1].val.clusterDim.x = static_cast<unsigned>(ks);
+    const int pre_ctas = static_cast<int>(cdiv(u.r, 16) * ks);
+    cfg.gridDim = dim3(static_cast<unsigned>(pre_ctas));
+    cfg.blockDim = dim3(32 * kLuWarps);
+    cfg.dynamicSmemBytes = 0;
+    cfg.numAttrs = ks > 1 ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, k_lora_u_tc, u) != cudaSuccess) return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    // the stream kernel
+    const int C = g.C;
+    int n = fit[dev & 63][C].load();
+    cfg.blockDim = dim3(LvCfg<NT8>::kThreads);
+    cfg.dynamicSmemBytes = LvCfg<NT8>::kSmem;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(C);
+    cfg.numAttrs = C > 1 ? 2 : 1;
+    // the stream kernel's CTAs take the SMs the pre-pass leaves (so that none waits for it)
+    const int sms = std::max(C, kSmsForSplit - pre_ctas);
+    if (n == 0) {
+        n = kSmsForSplit / C;
+        if (C > 1) {
+            cfg.gridDim = dim3(static_cast<unsigned>(C * (kSmsForSplit / C)));
+            int m = 0;
+            if (cudaOccupancyMaxActiveClusters(&m, k_qgemv_lut<NT8>, &cfg) != cudaSuccess) {
+                cudaGetLastError();
+                m = 0;
             }
-            if (n <= 0) n = -1;
-            fit[dev & 63][e].store(n);
+            n = std::min(n, std::max(m, 1));
         }
-        if (n < 0) continue;
-        const int64_t nbk = 4 * cdiv(q4, C);
-        for (int M = 16; M <= 16 * GvCfg<NT8>::MW && M * (nbk + 1) <= kGvTabS &&
-                        M * g.kt / 256 + 2 <= kGvRawC2 &&
-                        (!g.b_vec || M * (g.r + 8) <= kGvBrowMax); M += 16) {
-            const int64_t tiles = cdiv(d_out, M);
-            const int64_t clusters = std::min<int64_t>(n, tiles);
-            const int64_t tpc = cdiv(tiles, clusters);
-            // busiest cluster: its rows x its K range, plus a fixed cost per tile end
-            const int64_t cost = tpc * (M * nbk + 1024) + (C > 1 ? 512 : 0);
-            if (best_cost < 0 || cost < best_cost) {
-                best_cost = cost;
-                best_C = C;
-                best_M = M;
-                best_clusters = static_cast<int>(clusters);
-            }
-        }
+        fit[dev & 63][C].store(n);
     }
-    if (best_C == 0) return QLORA_ERR_UNSUPPORTED;
-    g.C = best_C;
-    g.M = best_M;
-    g.tiles = static_cast<int>(cdiv(d_out, best_M));
-    g.clusters = best_clusters;
-    g.pieces = static_cast<int>(cdiv(q4, best_C));
-    CUtensorMap tc;
-    QL_TRY(tmap_blocks(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, w->d_out, w->d_in / 2, 128, 16,
-                       static_cast<uint32_t>(g.pieces), CU_TENSOR_MAP_SWIZZLE_128B));
-    cfg.gridDim = dim3(static_cast<unsigned>(best_C * best_clusters));
-    cfg.numAttrs = 1;
-    if (best_C > 1) {
-        attr[1].val.clusterDim.x = static_cast<unsigned>(best_C);
-        cfg.numAttrs = 2;
-    }
+    g.clusters = static_cast<int>(std::min<int64_t>(std::min(n, sms / C), g.tiles));
+    cfg.gridDim = dim3(static_cast<unsigned>(C * g.clusters));
     const bool ev = g_ev_start && g_ev_stop;
     if (ev) cudaEventRecord(g_ev_start, st);
-    if (cudaLaunchKernelEx(&cfg, kern, tc, g) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, k_qgemv_lut<NT8>, g) != cudaSuccess) return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     if (ev) cudaEventRecord(g_ev_stop, st);
     return QLORA_OK;
@@ -680,28 +637,42 @@ qlora_status small_fwd(const qlora_nf4* w, const void* X, int64_t T, const void*
     const int64_t d_out = w->d_out, d_in = w->d_in;
     const SmallPlan sp = make_small_plan(T, d_out, d_in);
     if (!sp.ok) return QLORA_ERR_UNSUPPORTED;
-    float* us = at<float>(ws, p.s_us);
-    k_small_u<<<static_cast<unsigned>(cdiv(r, 8)), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(X), static_cast<int>(T), static_cast<int>(d_in),
-        static_cast<const __nv_bfloat16*>(A), r, s, us, static_cast<__nv_bfloat16*>(U_save));
-    QL_LAUNCH_CHECK();
-    GvArgs g{};
+    auto* us_pad = at<__nv_bfloat16>(ws, p.s_us);
+    LuArgs u{};
+    u.X = static_cast<const __nv_bfloat16*>(X);
+    u.T = static_cast<int>(T);
+    u.d_in = static_cast<int>(d_in);
+    u.kt = sp.kt;
+    u.A = static_cast<const __nv_bfloat16*>(A);
+    u.r = r;
+    u.s = s;
+    u.KS = sp.ks;
+    u.us_pad = us_pad;
+    u.u_save = static_cast<__nv_bfloat16*>(U_save);
+    LvArgs g{};
     g.T = static_cast<int>(T);
     g.d_out = static_cast<int>(d_out);
     g.d_in = static_cast<int>(d_in);
     g.kt = sp.kt;
-    g.X = static_cast<const __nv_bfloat16*>(X);
+    g.tiles = static_cast<int>(cdiv(d_out, 16));
+    g.C = sp.C;
+    g.r = r;
+    g.rp = (r + 15) & ~15;
+    g.codes = w->codes;
     g.absmax_q = w->absmax_q;
     g.c2 = w->c2;
-    g.us = us;
+    g.X = static_cast<const __nv_bfloat16*>(X);
+    g.us_pad = us_pad;
     g.B = static_cast<const __nv_bfloat16*>(B);
-    g.r = r;
-    g.b_vec = (r % 8 == 0) ? 1 : 0;    // B is 16-byte aligned (checked by the caller)
     g.H = static_cast<__nv_bfloat16*>(H);
     g.err = err;
     g.wait_ns = kWaitNs;
-    if (sp.nt8 == 1) return launch_qgemv<1>(w, X, T, g, st);
-    return launch_qgemv<2>(w, X, T, g, st);
+    {
+        static const float lv[16] = QLORA_NF4_LEVELS;
+        for (int i = 0; i < 8; ++i) g.lv16[i] = bf16_bits(lv[2 * i]) | (bf16_bits(lv[2 * i + 1]) << 16);
+    }
+    if (sp.nt8 == 1) return launch_qgemv<1>(g, sp.ks, u, st);
+    return launch_qgemv<2>(g, sp.ks, u, st);
 }
 
 qlora_status sgemm(cudaStream_t st, int64_t M, int64_t N, int64_t K, float alpha, const float* A,

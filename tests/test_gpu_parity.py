@@ -194,6 +194,25 @@ def test_config_full_size_sampled_rows(q, name):
     assert all(v <= TOL["bf16"] for v in err.values()), err
 
 
+@pytest.mark.parametrize("T", [3, 12])
+def test_decode_size_70b_shape(q, T):
+    # The 28672 x 8192 projection at decode sizes: 3 tokens (two ranks split K, 74 clusters of
+    # 24-25 tiles, the tile sums kept for the end phase) and 12 tokens (four ranks, 37 clusters of
+    # 48-49 tiles: more than the end phase keeps, so every finaliser finishes its tile at once).
+    # Runs right after the full-size cases so that the oracle's decode of the weight is shared.
+    import torch
+    case = S.make_layer(**S.CONFIGS["proj70b_28672x8192_r16_T2048"], seed=0)
+    Wh = oracle_weight_cached(case, 0)
+    w = q.nf4_quantize(dev(case.W0))
+    X, A, B = dev(case.X[:T], "bf16"), dev(case.A, "bf16"), dev(case.B, "bf16")
+    H, U = q.qlora_linear_fwd(w, X, A, B, case.alpha)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    ref = O.lora_forward(Wh, case.X[:T], case.A, case.B, case.alpha, case.r)
+    assert rel_fro(host(H), ref) <= TOL["bf16"]
+    assert rel_fro(host(U), case.X[:T].astype(np.float64) @ case.A.astype(np.float64).T) <= TOL["bf16"]
+
+
 # ------------------------------------------------------------------ decode-size forward
 
 
@@ -205,8 +224,12 @@ def test_config_full_size_sampled_rows(q, name):
     (2048, 1024, 128, 32),   # 32-token tile
     (264, 4352, 33, 3),      # 68 blocks per row: K split over a cluster, uneven ranks; r % 8 != 0
     (2056, 1024, 16, 24),    # 32-token tile, ragged rows
-    (4096, 4096, 16, 1),     # q_proj shape: K split over a cluster
+    (4096, 4096, 16, 1),     # q_proj shape
     (4096, 4096, 16, 8),
+    (4096, 4096, 16, 12),    # 9..16 tokens: two ranks split K
+    (1032, 11008, 1, 2),     # 172 blocks per row: three ranks, the last one partly idle; r = 1
+    (4104, 8192, 100, 13),   # four ranks; r even but not a multiple of 8
+    (528, 2048, 128, 9),     # the largest rank
 ])
 def test_decode_size_forward(q, d_out, d_in, r, T):
     import torch
