@@ -48,7 +48,7 @@
 namespace qlora {
 
 constexpr int kLvWarps = 16;                 // compute warps
-constexpr int kLvTableBytes = 256 * 128;     // 256 entries x 32 lanes x 4 bytes
+constexpr int kLvTableBytes = 0x10000;       // 256 entries x 256 bytes (lanes' words in the low half)
 constexpr int kLvMaxRanks = 8;
 constexpr int kLvRpMax = 128;                // adapter rank padded to 16
 constexpr int kLvSuLd = kLvRpMax + 8;        // row stride (bf16) of s U and of staged B rows
@@ -56,20 +56,28 @@ constexpr int kLvSuLd = kLvRpMax + 8;        // row stride (bf16) of s U and of 
 template <int NT8>
 struct LvCfg {
     static constexpr int KB = NT8 == 1 ? 4 : 2;                      // 64-blocks per warp
-    static constexpr int NBUF = NT8 == 1 ? 4 : 3;                    // tile partial buffers
-    static constexpr int S = NT8 == 1 ? 3 : 4;                       // code slices in flight per warp
+    static constexpr int NBUF = 3;                                   // tile partial buffers
+    static constexpr int S = 3;                                      // code slices in flight per warp
     static constexpr int kThreads = 32 * (kLvWarps + NBUF);          // + one finaliser per buffer
     static constexpr int kMaxRanks = NT8 == 1 ? 8 : 4;
     static constexpr int kRowBytes = KB * 32;                         // a warp's bytes of a row
     static constexpr int kSlice = 16 * kRowBytes;                     // a warp's bytes of a tile
-    static constexpr int kTableOff = 0;
-    static constexpr int kCodesOff = kTableOff + kLvTableBytes;      // [warp][stage] slices
-    static constexpr int kPartOff = kCodesOff + kLvWarps * S * kSlice;   // [buf][warp][n][lane] float4
-    static constexpr int kRingOff = kPartOff + NBUF * kLvWarps * NT8 * 512;     // [buf][rank][n][lane] float4
-    static constexpr int kSuOff = kRingOff + NBUF * kMaxRanks * NT8 * 512;      // bf16 s U [16][kLvSuLd]
-    static constexpr int kSbOff = kSuOff + 16 * kLvSuLd * 2;         // bf16 B rows [NBUF][16][kLvSuLd]
-    static constexpr int kBarOff = kSbOff + NBUF * 16 * kLvSuLd * 2;
-    static constexpr int kSmem = kBarOff + 256;
+    static constexpr int kCodes = kLvWarps * S * kSlice;              // [warp][stage] slices
+    static constexpr int kPart = NBUF * kLvWarps * NT8 * 512;         // [buf][warp][n][lane] float4
+    static constexpr int kRing = NBUF * kMaxRanks * NT8 * 512;        // [buf][rank][n][lane] float4
+    static constexpr int kSu = 16 * kLvSuLd * 2;                      // bf16 s U [16][kLvSuLd]
+    static constexpr int kSb = NBUF * 16 * kLvSuLd * 2;               // bf16 B rows [NBUF][16][kLvSuLd]
+    // The table sits on the first 64 KB boundary of the shared window above the buffers placed
+    // below it (at most 62 KB of them: the window starts within the first KB); the others follow
+    // it.  Up to 8 tokens the tile partials live in the unused upper halves of the table entries
+    // (128-byte pieces, a quarter warp's float4 each) and the code slices follow the table; for
+    // 9..16 tokens the code slices go below the table and the partials after it.
+    static constexpr bool kPartInTable = NT8 == 1;
+    static_assert(!kPartInTable || NBUF * kLvWarps * NT8 * 4 <= 256, "partials must fit in the table");
+    static constexpr int kBelow = kPartInTable ? kRing + kSu + kSb + 256 : kCodes + kSu + 256;
+    static constexpr int kAbove = kPartInTable ? kCodes : kPart + kRing + kSb;
+    static_assert(kBelow <= 62 * 1024, "buffers below the table");
+    static constexpr int kSmem = 64 * 1024 + kLvTableBytes + kAbove;    // window start .. end
     static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
@@ -124,12 +132,39 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
     using Cf = LvCfg<NT8>;
     constexpr int KB = Cf::KB, NBUF = Cf::NBUF, MR = Cf::kMaxRanks, S = Cf::S;
     extern __shared__ __align__(1024) uint8_t smem[];
-    uint32_t* table = reinterpret_cast<uint32_t*>(smem + Cf::kTableOff);
-    float4* part = reinterpret_cast<float4*>(smem + Cf::kPartOff);
-    float4* ring = reinterpret_cast<float4*>(smem + Cf::kRingOff);
-    __nv_bfloat16* s_us = reinterpret_cast<__nv_bfloat16*>(smem + Cf::kSuOff);
-    __nv_bfloat16* s_b = reinterpret_cast<__nv_bfloat16*>(smem + Cf::kSbOff);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::kBarOff);
+    // the table on the first 64 KB boundary above the buffers placed below it: the table address
+    // of a code byte is then a single byte permute (table address bits 16+, byte, 4 lane)
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t tab_addr = (sbase + Cf::kBelow + 0xFFFFu) & ~0xFFFFu;
+    if (tab_addr + kLvTableBytes + Cf::kAbove > sbase + Cf::kSmem) {
+        if (threadIdx.x == 0) set_error(a.err, kErrDevice);
+        // still meet the other ranks at both cluster barriers (theirs time out on the missing
+        // partials and reach the last one)
+        if (a.C > 1) {
+            cluster_barrier();
+            cluster_barrier();
+        }
+        return;
+    }
+    uint8_t* const below = smem;
+    uint8_t* const above = smem + (tab_addr - sbase) + kLvTableBytes;
+    uint32_t* table = reinterpret_cast<uint32_t*>(smem + (tab_addr - sbase));
+    uint8_t* const codes_sm = Cf::kPartInTable ? above : below;
+    float4* const part_lin = reinterpret_cast<float4*>(above);             // (9..16 tokens)
+    float4* const ring = reinterpret_cast<float4*>(Cf::kPartInTable ? below : above + Cf::kPart);
+    __nv_bfloat16* s_us = reinterpret_cast<__nv_bfloat16*>(Cf::kPartInTable ? below + Cf::kRing : below + Cf::kCodes);
+    __nv_bfloat16* s_b = reinterpret_cast<__nv_bfloat16*>(Cf::kPartInTable ? below + Cf::kRing + Cf::kSu
+                                                                            : above + Cf::kPart + Cf::kRing);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(Cf::kPartInTable ? below + Cf::kRing + Cf::kSu + Cf::kSb
+                                                                   : below + Cf::kCodes + Cf::kSu);
+    // the float4 of lane ln for (buffer, warp, n) of the tile partials
+    auto part_at = [&](int buf, int w, int n, int ln) -> float4* {
+        const int idx = (buf * kLvWarps + w) * NT8 + n;
+        if constexpr (Cf::kPartInTable)
+            return reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(table) + (idx * 4 + (ln >> 3)) * 256 + 128) + (ln & 7);
+        else
+            return part_lin + idx * 32 + ln;
+    };
     uint64_t* full = bars;                  // [NBUF] the 16 warps' partials of a tile are in
     uint64_t* freeb = bars + NBUF;          // [NBUF] the finaliser has read them
     uint64_t* ring_full = bars + 2 * NBUF;  // [NBUF] rank 0: the other ranks' sums are in
@@ -165,7 +200,7 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
     // ---- compute warps: the warp's slice of tile li (16 rows x KB blocks) into its ring stage
     // li % S, a row's 16-byte chunk c at chunk c ^ swz(row) (so that the fragment reads of 8 rows
     // fall in different banks); rows past d_out are zero-filled
-    const uint32_t slices = smem_u32(smem + Cf::kCodesOff) + warp * S * Cf::kSlice;
+    const uint32_t slices = smem_u32(codes_sm) + warp * S * Cf::kSlice;
     auto swz = [](int row) { return KB == 4 ? (row & 7) : ((row >> 1) & 3); };
     const uint8_t* const w0 = a.codes + static_cast<int64_t>(t_lo) * 16 * row_bytes + kb0 * 32;
     auto issue_slice = [&](int li) {
@@ -210,6 +245,14 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
     uint32_t xw[KB][NT8][8];
     if (compute) {
         for (int st = 0; st < S - 1; ++st) issue_slice(st);
+        // the byte table: entry e = (high code << 4) | low code -> bf16x2 (L[low], L[high]), the
+        // same word in every lane's slot; warp w writes the entries of low code w
+        {
+            const uint32_t lo = (a.lv16[warp >> 1] >> (16 * (warp & 1))) & 0xFFFFu;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                table[(16 * j + warp) * 64 + lane] = lo | (a.lv16[j >> 1] >> (16 * (j & 1)) << 16);
+        }
         load_scales(0, sc_cur);
         // X fragments of this warp's blocks, held for the whole kernel: token 8n + g, elements
         // 16q .. 16q + 15 of block kb0 + b
@@ -228,16 +271,6 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
                 xw[b][n][4] = x1.x; xw[b][n][5] = x1.y; xw[b][n][6] = x1.z; xw[b][n][7] = x1.w;
             }
         }
-        // the byte table: entry e = (high code << 4) | low code -> bf16x2 (L[low], L[high]), the
-        // same word for every lane; warp w writes entries w, w + 16, ...
-        const uint32_t pair = a.lv16[(lane & 15) >> 1];
-        const uint32_t lv = (lane & 1) ? (pair >> 16) : (pair & 0xFFFFu);   // bf16 of L[lane & 15]
-#pragma unroll 4
-        for (int e = warp; e < 256; e += kLvWarps) {
-            const uint32_t lo = __shfl_sync(0xffffffffu, lv, e & 15);
-            const uint32_t hi = __shfl_sync(0xffffffffu, lv, e >> 4);
-            table[e * 32 + lane] = lo | (hi << 16);
-        }
     }
     // barriers initialised (and visible cluster-wide) and the table written before use
     if (C > 1) cluster_barrier();
@@ -245,9 +278,10 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
 
     if (compute) {
         // ================================================================ compute warps
-        const uint32_t lb = smem_u32(table) + (static_cast<uint32_t>(lane) << 2);
-        // table address of byte i of a code word: entry (byte << 7) + this lane's word
-        auto tab = [&](uint32_t w, uint32_t i) -> uint32_t { return lb + (prmt(w, 0u, 0x4440u | i) << 7); };
+        const uint32_t lb = tab_addr | (static_cast<uint32_t>(lane) << 2);
+        // table address of byte i of a code word: bits 16+ and the lane's word from lb, the byte as
+        // bits 8..15 (entry stride 256 bytes)
+        auto tab = [&](uint32_t w, uint32_t i) -> uint32_t { return prmt(w, lb, 0x7604u | (i << 4)); };
         // the warp's part of tile li (its slice in stage li % S, its scales in R); false on a
         // failed wait
         auto process = [&](int li, const Scales& R) -> bool {
@@ -258,20 +292,24 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
             for (int n = 0; n < NT8; ++n)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+            // the thread's 8 code bytes of each block in rows g and g + 8 (logical chunk 2b + q / 2,
+            // half q % 2), all loaded before the look-ups
+            uint2 ca[KB], cb[KB];
 #pragma unroll
             for (int b = 0; b < KB; ++b) {
-                // the thread's 8 code bytes of block b in rows g and g + 8: logical chunk
-                // 2b + q / 2, half q % 2
                 const int c = 2 * b + (q >> 1);
-                const uint2 ca = lds_v2(slc + g * Cf::kRowBytes + ((c ^ swz(g)) << 4) + ((q & 1) << 3));
-                const uint2 cb = lds_v2(slc + (g + 8) * Cf::kRowBytes + ((c ^ swz(g + 8)) << 4) + ((q & 1) << 3));
+                ca[b] = lds_v2(slc + g * Cf::kRowBytes + ((c ^ swz(g)) << 4) + ((q & 1) << 3));
+                cb[b] = lds_v2(slc + (g + 8) * Cf::kRowBytes + ((c ^ swz(g + 8)) << 4) + ((q & 1) << 3));
+            }
+#pragma unroll
+            for (int b = 0; b < KB; ++b) {
                 float tmp[NT8][4];
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
                     // A registers of k16 step s: bytes 2s (slots 2q, 2q+1) and 2s + 1 (slots
                     // 2q+8, 2q+9) of the thread's 8 code bytes, rows g and g + 8
-                    const uint32_t wa = (s < 2) ? ca.x : ca.y;
-                    const uint32_t wb = (s < 2) ? cb.x : cb.y;
+                    const uint32_t wa = (s < 2) ? ca[b].x : ca[b].y;
+                    const uint32_t wb = (s < 2) ? cb[b].x : cb[b].y;
                     const uint32_t i0 = 2 * (s & 1), i1 = i0 + 1;
                     const uint32_t A[4] = {lds_u32(tab(wa, i0)), lds_u32(tab(wb, i0)), lds_u32(tab(wa, i1)),
                                            lds_u32(tab(wb, i1))};
@@ -299,7 +337,7 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
             }
 #pragma unroll
             for (int n = 0; n < NT8; ++n)
-                part[((buf * kLvWarps + warp) * NT8 + n) * 32 + lane] =
+                *part_at(buf, warp, n, lane) =
                     make_float4(R.c2a * acc[n][0], R.c2a * acc[n][1], R.c2b * acc[n][2], R.c2b * acc[n][3]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[buf]);
@@ -380,10 +418,10 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
             float4 tot[NT8];
 #pragma unroll
             for (int n = 0; n < NT8; ++n) {
-                tot[n] = part[((buf * kLvWarps) * NT8 + n) * 32 + lane];
+                tot[n] = *part_at(buf, 0, n, lane);
 #pragma unroll
                 for (int w = 1; w < kLvWarps; ++w) {
-                    const float4 v = part[((buf * kLvWarps + w) * NT8 + n) * 32 + lane];
+                    const float4 v = *part_at(buf, w, n, lane);
                     tot[n].x += v.x;
                     tot[n].y += v.y;
                     tot[n].z += v.z;
