@@ -347,6 +347,35 @@ def dora_forward(W_hat, X, A, B, alpha, r, magnitude):
     return np.asarray(X, np.float64) @ Wd.T
 
 
+def dora_backward(W_hat, X, dH, A, B, alpha, r, magnitude):
+    """(dX, dA, dB, dm) of the DoRA forward above for the upstream gradient dH[T, d_out].
+
+    With V = W_hat + s B A, n_j = ||V[j, :]||, c_j = m_j / n_j and Z = X V^T (so H = Z diag(c)),
+    the chain rule through every factor, the norm included:
+      dZ = dH diag(c)
+      dc_j = sum_t dH[t, j] Z[t, j],   dm_j = dc_j / n_j,   dn_j = -dc_j m_j / n_j^2
+      dX = dZ V;   dV = dZ^T X + diag(dn / n) V   (dn_j V[j, :] / n_j is the norm's gradient)
+      dA = s B^T dV,   dB = s dV A^T             (V depends on A, B through s B A only)
+    A row with n_j = 0 contributes nothing (its output is 0 and its direction undefined).
+    """
+    W_hat, X, dH, A, B = (np.asarray(t, np.float64) for t in (W_hat, X, dH, A, B))
+    m = np.asarray(magnitude, np.float64)
+    s = lora_scale(alpha, r)
+    V = W_hat + s * (B @ A)
+    n = np.sqrt(np.sum(V * V, axis=1))
+    ok = n > 0
+    safe = np.where(ok, n, 1.0)
+    c = np.where(ok, m / safe, 0.0)
+    Z = X @ V.T
+    dZ = dH * c[None, :]
+    dc = np.sum(dH * Z, axis=0)
+    dm = np.where(ok, dc / safe, 0.0)
+    dn = np.where(ok, -dc * m / (safe * safe), 0.0)
+    dX = dZ @ V
+    dV = dZ.T @ X + (np.where(ok, dn / safe, 0.0))[:, None] * V
+    return dX, s * (B.T @ dV), s * (dV @ A.T), dm
+
+
 # ----------------------------------------------------------------------------
 # Adapter optimizer step (reading R23)
 # ----------------------------------------------------------------------------

@@ -370,6 +370,48 @@ def test_dora_direction_is_scale_free():
     assert rel(h1, h2) < 1e-13
 
 
+def check_dora_gradients_fd(bwd):
+    """Largest relative gap between bwd's (dX, dA, dB, dm) and central finite differences of
+    L = <dH, H> through the DoRA forward (nonlinear in A, B, m through the row norm: the
+    difference quotient is exact to O(h^2); h = 1e-5 in fp64)."""
+    W, X, A, B, dH = small_layer(d=5, k=6, r=2, T=3, seed=11)
+    mag = np.array([0.7, 1.3, 2.0, 0.4, 1.1])
+    alpha, r = 3.0, 2
+    got = bwd(W, X, dH, A, B, alpha, r, mag)
+    h = 1e-5
+
+    def loss(X_, A_, B_, m_):
+        return float(np.sum(dH * O.dora_forward(W, X_, A_, B_, alpha, r, m_)))
+
+    refs = []
+    for which, base in enumerate((X, A, B, mag)):
+        g = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            args_p = [X.copy(), A.copy(), B.copy(), mag.copy()]
+            args_m = [X.copy(), A.copy(), B.copy(), mag.copy()]
+            args_p[which][idx] += h
+            args_m[which][idx] -= h
+            g[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        refs.append(g)
+    return max(rel(gv, rv) for gv, rv in zip(got, refs))
+
+
+def test_dora_backward_against_finite_differences():
+    assert check_dora_gradients_fd(O.dora_backward) < 1e-8
+
+
+def test_dora_backward_reduces_to_lora_at_initialisation():
+    # m = the row norms makes the forward LoRA's; the gradients of X, A, B then differ from
+    # LoRA's only by the norm's term, and dm is the per-row <dH, Z> / n
+    W, X, A, B, dH = small_layer(d=7, k=5, r=2, T=4, seed=12)
+    n = O.dora_row_norms(W, A, B, 4.0, 2)
+    dX, dA, dB, dm = O.dora_backward(W, X, dH, A, B, 4.0, 2, n)
+    dXl, _, _ = O.lora_backward(W, X, dH, A, B, 4.0, 2)
+    assert rel(dX, dXl) < 1e-13
+    Z = O.lora_forward(W, X, A, B, 4.0, 2)
+    assert rel(dm, np.sum(dH * Z, axis=0) / n) < 1e-13
+
+
 # ---------------------------------------------------------------- optimizer step (R23)
 
 ADAM = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
@@ -802,6 +844,21 @@ def test_pins_catch_planted_mistakes():
 
     assert check_dora_brute(dora_no_adapter_in_norm) > 1e-3
     assert check_dora_brute(dora_column_norms) > 1e-3
+
+    def dora_bwd_detached_norm(W, X, dH, A, B, a, r, mag):
+        # the norm treated as a constant: its term dropped from dA, dB
+        dX, dA, dB, dm = O.dora_backward(W, X, dH, A, B, a, r, mag)
+        V = W + s(a, r) * (B @ A)
+        n = np.sqrt(np.sum(V * V, axis=1))
+        dZ = dH * (mag / n)[None, :]
+        return dX, s(a, r) * (B.T @ (dZ.T @ X)), s(a, r) * ((dZ.T @ X) @ A.T), dm
+
+    def dora_bwd_unscaled_dX(W, X, dH, A, B, a, r, mag):
+        dX, dA, dB, dm = O.dora_backward(W, X, dH, A, B, a, r, mag)
+        return dH @ (W + s(a, r) * (B @ A)), dA, dB, dm
+
+    assert check_dora_gradients_fd(dora_bwd_detached_norm) > 1e-3
+    assert check_dora_gradients_fd(dora_bwd_unscaled_dX) > 1e-3
 
     # FP8 mutants: ties away from zero, truncation, no saturation, a scale one power off,
     # the weight scale dropped, the low-rank branch fed the scaled activation
