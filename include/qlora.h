@@ -64,7 +64,7 @@ typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 typedef enum {
     QLORA_OP_FWD = 0, QLORA_OP_BWD = 1, QLORA_OP_FWD_BATCHED = 2, QLORA_OP_MERGE = 3,
     QLORA_OP_FWD_MULTI = 4, QLORA_OP_DORA_FWD = 5, QLORA_OP_FWD_FP8 = 6, QLORA_OP_FP8_QUANT = 7,
-    QLORA_OP_BWD_FP8 = 8
+    QLORA_OP_BWD_FP8 = 8, QLORA_OP_DORA_BWD = 9
 } qlora_op;
 
 /* Stored NF4 weight.  Block size 64 and group size 256 are fixed.
@@ -230,10 +230,29 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4* w, const void* X, int64_t T
  * (they depend on A, B) by the tensor-core merge tile in a row-norm mode, then the large-T
  * fused forward applies m / n to each output column before rounding.  U_save as in
  * qlora_linear_fwd.  ws >= qlora_workspace_bytes(QLORA_OP_DORA_FWD, QLORA_BF16, T, d_out,
- * d_in, r).  Forward only.                                                                    */
+ * d_in, r).  The backward is qlora_dora_bwd.                                                  */
 qlora_status qlora_dora_fwd(const qlora_nf4* w, const void* X, int64_t T, const void* A,
                             const void* B, int32_t r, float alpha, const float* magnitude,
                             void* H, void* U_save, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* DoRA backward (bf16): the gradients of the DoRA forward above for the upstream gradient dH,
+ * by the chain rule through every factor of H = Z diag(c), Z = X V^T, V = W^ + s B A,
+ * c_j = m_j / n_j, n_j = ||V[j, :]||_2 -- the norm included (the pages give the forward only;
+ * the derivative of the Euclidean norm is V[j, :] / n_j):
+ *   dZ = dH diag(c),  dc_j = sum_t dH[t, j] Z[t, j],  dm_j = dc_j / n_j,  e_j = -dc_j m_j / n_j^3
+ *   dX = dZ V,  dA = s B^T (dZ^T X + diag(e) V),  dB = s (dZ^T X + diag(e) V) A^T
+ * A row of norm 0 contributes nothing.  The library recomputes n and Z (a large-T forward), runs
+ * the LoRA backward on dZ and adds the norm's term through two passes over the weight with the
+ * adapter rows as tokens (A W^T and B^T diag(e) W^ on the fused NF4 GEMM) and r x r products.
+ * [CH] "Choosing what to adapt: targets and rank"; [MF] "Advanced Variants: DoRA and LoRA+";
+ * [MF] "Gradient Dynamics and Backpropagation Mechanics" (the LoRA part).
+ *   X [T, d_in], dH [T, d_out], A, B bf16; magnitude fp32 [d_out]; dX (nullable) bf16 [T, d_in];
+ *   dA fp32 [r, d_in], dB fp32 [d_out, r], dm fp32 [d_out], all overwritten.
+ *   ws >= qlora_workspace_bytes(QLORA_OP_DORA_BWD, QLORA_BF16, T, d_out, d_in, r).            */
+qlora_status qlora_dora_bwd(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                            const void* A, const void* B, int32_t r, float alpha,
+                            const float* magnitude, void* dX, float* dA, float* dB, float* dm,
+                            void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* The DoRA row norms n_j = ||(W^ + (alpha/r) B A)[j, :]||_2 (bf16 adapters, W^ the bf16 decode)
  * into norms (device fp32 [d_out]); DoRA initialises the magnitude to them.  ws holds at least

@@ -30,13 +30,13 @@ STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",
           3: "QLORA_ERR_CUDA", 4: "QLORA_ERR_TIMEOUT", 5: "QLORA_ERR_DEVICE"}
 F32, BF16 = 0, 1
 OP_FWD, OP_BWD, OP_FWD_BATCHED, OP_MERGE, OP_FWD_MULTI, OP_DORA_FWD = 0, 1, 2, 3, 4, 5
-OP_FWD_FP8, OP_FP8_QUANT, OP_BWD_FP8 = 6, 7, 8
+OP_FWD_FP8, OP_FP8_QUANT, OP_BWD_FP8, OP_DORA_BWD = 6, 7, 8, 9
 
 # Every symbol include/qlora.h declares.
 EXPORTS = ["qlora_nf4_sizes", "qlora_nf4_levels", "nf4_quantize", "nf4_dequantize",
            "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "lora_merge",
            "qlora_linear_bwd_ex", "qlora_adamw_step", "qlora_prefetch", "qlora_dora_fwd",
-           "qlora_dora_row_norms", "qlora_fp8_quantize", "qlora_fp8_weight_scale",
+           "qlora_dora_bwd", "qlora_dora_row_norms", "qlora_fp8_quantize", "qlora_fp8_weight_scale",
            "qlora_linear_fwd_fp8", "qlora_fp8_quantize_grad", "qlora_linear_bwd_fp8",
            "qlora_linear_fwd_batched", "qlora_linear_fwd_multi", "qlora_linear_fwd_noalloc",
            "qlora_get_device_error",
@@ -90,6 +90,7 @@ def load() -> ctypes.CDLL:
         "qlora_prefetch": ([vp, sz, i32, vp], ctypes.c_int),
         "qlora_dora_fwd": ([pnf4, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "qlora_dora_row_norms": ([pnf4, vp, vp, i32, f32, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_dora_bwd": ([pnf4, vp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "qlora_fp8_quantize": ([vp, i64, vp, vp, vp, sz, vp], ctypes.c_int),
         "qlora_fp8_weight_scale": ([pnf4, vp, vp], ctypes.c_int),
         "qlora_linear_fwd_fp8": ([pnf4, vp, i64, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp], ctypes.c_int),
@@ -304,6 +305,30 @@ def qlora_dora_fwd(w: NF4Weight, X, A, B, alpha, magnitude, H=None, U_save=None,
         ctypes.byref(c), _ptr(X), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(magnitude), _ptr(H),
         _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream)))
     return H, U_save
+
+
+def qlora_dora_bwd(w: NF4Weight, X, dH, A, B, alpha, magnitude, dX=None, dA=None, dB=None, dm=None,
+                   want_dx=True, ws=None, stream=None):
+    """DoRA backward (bf16), the chain rule through the row norm: returns (dX, dA, dB, dm)."""
+    torch = _torch()
+    _contig(X, dH, A, B, magnitude, dX, dA, dB, dm)
+    T = X.shape[0]
+    r = A.shape[0]
+    dev = X.device
+    if dX is None and want_dx:
+        dX = torch.empty((T, w.d_in), dtype=X.dtype, device=dev)
+    if dA is None:
+        dA = torch.empty((r, w.d_in), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((w.d_out, r), dtype=torch.float32, device=dev)
+    if dm is None:
+        dm = torch.empty((w.d_out,), dtype=torch.float32, device=dev)
+    ws = _ws(OP_DORA_BWD, BF16, T, w.d_out, w.d_in, r, dev, ws)
+    c = w._c()
+    _check("qlora_dora_bwd", load().qlora_dora_bwd(
+        ctypes.byref(c), _ptr(X), _ptr(dH), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(magnitude),
+        _ptr(dX), _ptr(dA), _ptr(dB), _ptr(dm), _ptr(ws), ws.numel(), _stream(stream)))
+    return dX, dA, dB, dm
 
 
 def fp8_quantize(X, X8=None, scale=None, ws=None, stream=None):

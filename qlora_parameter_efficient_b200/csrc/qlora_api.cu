@@ -19,6 +19,7 @@
 #include "optim.cuh"
 #include "fp8.cuh"
 #include "qgemv.cuh"
+#include "dora.cuh"
 
 using namespace qlora;
 
@@ -381,6 +382,41 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
     }
     p.total = off;
     return p;
+}
+
+// DoRA backward workspace: one region shared in turn by the large-T forward (the pre-scale
+// output Z), the LoRA backward of dZ and the two weight passes with the adapter rows as tokens,
+// then the DoRA buffers.
+struct DoraBwdLayout {
+    size_t shared = 0, merge_part = 0, norms = 0, e = 0, colpart = 0, z = 0, u = 0, dz = 0, ge = 0,
+           pm = 0, qm = 0, aat = 0, beb = 0, total = 0;
+};
+DoraBwdLayout dora_bwd_layout(int64_t T, int64_t d, int64_t k, int r) {
+    DoraBwdLayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    const size_t shared = std::max({make_plan(QLORA_OP_DORA_FWD, QLORA_BF16, T, d, k, r).total,
+                                    make_plan(QLORA_OP_BWD, QLORA_BF16, T, d, k, r).total,
+                                    g2_schedule(r, d, k).bytes(), g2_schedule(r, k, d).bytes()});
+    L.shared = take(shared);
+    L.merge_part = take(static_cast<size_t>(d) * (k / 64) * 4);
+    L.norms = take(static_cast<size_t>(d) * 4);
+    L.e = take(static_cast<size_t>(d) * 4);
+    L.colpart = take(static_cast<size_t>(kDoraChunks) * d * 4);
+    L.z = take(static_cast<size_t>(T) * d * 2);
+    L.u = take(static_cast<size_t>(T) * r * 2);
+    L.dz = take(static_cast<size_t>(T) * d * 2);
+    L.ge = take(static_cast<size_t>(r) * d * 2);
+    L.pm = take(static_cast<size_t>(r) * d * 2);
+    L.qm = take(static_cast<size_t>(r) * k * 2);
+    L.aat = take(static_cast<size_t>(r) * r * 4);
+    L.beb = take(static_cast<size_t>(r) * r * 4);
+    L.total = off;
+    return L;
 }
 
 template <typename P>
@@ -966,13 +1002,15 @@ qlora_status qlora_nf4_levels(float* out) {
 
 size_t qlora_workspace_bytes(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in,
                              int32_t r_total) {
-    if (op < QLORA_OP_FWD || op > QLORA_OP_BWD_FP8) return 0;
+    if (op < QLORA_OP_FWD || op > QLORA_OP_DORA_BWD) return 0;
     if ((op == QLORA_OP_FWD_MULTI || op == QLORA_OP_DORA_FWD || op == QLORA_OP_FWD_FP8 ||
-         op == QLORA_OP_FP8_QUANT || op == QLORA_OP_BWD_FP8) && dtype != QLORA_BF16)
+         op == QLORA_OP_FP8_QUANT || op == QLORA_OP_BWD_FP8 || op == QLORA_OP_DORA_BWD) &&
+        dtype != QLORA_BF16)
         return 0;
     if ((dtype != QLORA_BF16 && dtype != QLORA_F32) || T < 1 || d_out < 1 || d_in < 64 ||
         r_total < 1 || r_total > 128)
         return 0;
+    if (op == QLORA_OP_DORA_BWD) return dora_bwd_layout(T, d_out, d_in, r_total).total;
     return make_plan(op, dtype, T, d_out, d_in, r_total).total;
 }
 
@@ -1077,6 +1115,77 @@ qlora_status qlora_dora_fwd(const qlora_nf4* w, const void* X, int64_t T, const 
     float* scale = at<float>(ws, p.dora_scale);
     QL_TRY(dora_scale(w, A, B, r, s, magnitude, at<float>(ws, p.dora_part), scale, stream));
     return fwd_bf16_large(w, X, T, A, B, r, s, H, U_save, p, ws, err, stream, scale);
+}
+
+qlora_status qlora_dora_bwd(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                            const void* A, const void* B, int32_t r, float alpha,
+                            const float* magnitude, void* dX, float* dA, float* dB, float* dm,
+                            void* ws, size_t ws_bytes, cudaStream_t stream) {
+    QL_TRY(check_layer(w, T, r, QLORA_BF16));
+    if (!aligned16(X) || !aligned16(dH) || !aligned16(A) || !aligned16(B) || !magnitude ||
+        !aligned16(dA) || !aligned16(dB) || !dm || !aligned16_or_null(dX))
+        return QLORA_ERR_INVALID_ARG;
+    const int64_t d = w->d_out, k = w->d_in;
+    const DoraBwdLayout L = dora_bwd_layout(T, d, k, r);
+    QL_TRY(check_ws(ws, ws_bytes, L.total));
+    int* err = nullptr;
+    QL_TRY(err_word(&err, stream));
+    using bf = __nv_bfloat16;
+    const float s = alpha / static_cast<float>(r);
+    void* shared = at<void>(ws, L.shared);
+    float* norms = at<float>(ws, L.norms);
+    float* e = at<float>(ws, L.e);
+    float* colpart = at<float>(ws, L.colpart);
+    bf* Z = at<bf>(ws, L.z);
+    bf* U = at<bf>(ws, L.u);
+    bf* dZ = at<bf>(ws, L.dz);
+    bf* ge = at<bf>(ws, L.ge);
+    bf* pm = at<bf>(ws, L.pm);
+    bf* qm = at<bf>(ws, L.qm);
+    float* aat = at<float>(ws, L.aat);
+    float* beb = at<float>(ws, L.beb);
+    // n_j = ||(W^ + s B A)[j, :]|| and the pre-scale output Z = X V^T (with U for the backward)
+    QL_TRY(dora_scale(w, A, B, r, s, nullptr, at<float>(ws, L.merge_part), norms, stream));
+    const Plan pf = make_plan(QLORA_OP_DORA_FWD, QLORA_BF16, T, d, k, r);
+    QL_TRY(fwd_bf16_large(w, X, T, A, B, r, s, Z, U, pf, shared, err, stream, nullptr));
+    // dZ = dH diag(m / n), dc_j = sum_t dH[t, j] Z[t, j], dm = dc / n, e = -dc m / n^3
+    const dim3 cgrid(static_cast<unsigned>(cdiv(d / 2, 256)), static_cast<unsigned>(kDoraChunks));
+    if (launch_pdl(k_dora_colred, cgrid, dim3(256), 0, stream, static_cast<const bf*>(dH),
+                   static_cast<const bf*>(Z), magnitude, static_cast<const float*>(norms), T, d, dZ,
+                   colpart) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    if (launch_pdl(k_dora_coef, grid1d(d), dim3(256), 0, stream, static_cast<const float*>(colpart),
+                   kDoraChunks, d, magnitude, static_cast<const float*>(norms), dm, e) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    // the LoRA backward of dZ: dX = dZ V, dA and dB without the norm's term
+    const Plan pb = make_plan(QLORA_OP_BWD, QLORA_BF16, T, d, k, r);
+    QL_TRY(bwd_bf16(w, X, dZ, T, A, B, r, s, U, dX, dA, dB, pb, shared, err, 0, stream, nullptr));
+    // the norm's term: P = A W^T and Q = (B^T diag(e)) W^ by the fused NF4 GEMM with the r
+    // adapter rows as tokens, then the r x r Gram products and the two updates
+    if (launch_pdl(k_dora_ge, grid1d(r * d), dim3(256), 0, stream, static_cast<const bf*>(B),
+                   static_cast<const float*>(e), static_cast<int>(r), d, ge) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    QL_TRY(nf4_gemm(false, w, A, r, nullptr, nullptr, 0, 0, 0, pm, shared, err, stream));
+    QL_TRY(nf4_gemm(true, w, ge, r, nullptr, nullptr, 0, 0, 0, qm, shared, err, stream));
+    if (launch_pdl(k_dora_gram, dim3(static_cast<unsigned>(r * r), 2), dim3(256), 0, stream,
+                   static_cast<const bf*>(A), static_cast<const bf*>(B), static_cast<const float*>(e),
+                   static_cast<int>(r), d, k, aat, beb) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    if (launch_pdl(k_dora_add_db, grid1d(d * r), dim3(256), 0, stream, static_cast<const bf*>(pm),
+                   static_cast<const bf*>(B), static_cast<const float*>(aat), static_cast<const float*>(e),
+                   static_cast<int>(r), d, s, dB) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    if (launch_pdl(k_dora_add_da, grid1d(r * k), dim3(256), 0, stream, static_cast<const bf*>(qm),
+                   static_cast<const bf*>(A), static_cast<const float*>(beb), static_cast<int>(r), k, s,
+                   dA) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
 }
 
 qlora_status qlora_fp8_quantize(const void* X, int64_t n, uint8_t* X8, float* scale, void* ws,

@@ -51,7 +51,7 @@ def test_workspace_sizes(L):
     for op in (q.OP_FWD, q.OP_BWD, q.OP_FWD_BATCHED):
         for dt in (q.BF16, q.F32):
             assert q.workspace_bytes(op, dt, 4096, 4096, 4096, 16) > 0
-    for op in (q.OP_FWD_MULTI, q.OP_DORA_FWD, q.OP_FWD_FP8, q.OP_BWD_FP8, q.OP_FP8_QUANT):
+    for op in (q.OP_FWD_MULTI, q.OP_DORA_FWD, q.OP_FWD_FP8, q.OP_BWD_FP8, q.OP_FP8_QUANT, q.OP_DORA_BWD):
         assert q.workspace_bytes(op, q.BF16, 4096, 4096, 4096, 16) > 0
         assert q.workspace_bytes(op, q.F32, 4096, 4096, 4096, 16) == 0      # bf16 only
     # the FP8 backward needs the bf16 backward's scratch plus the exact bf16 copies of X8, dH8
@@ -59,7 +59,10 @@ def test_workspace_sizes(L):
             >= q.workspace_bytes(q.OP_BWD, q.BF16, 4096, 4096, 4096, 16) + 2 * 2 * 4096 * 4096)
     assert q.workspace_bytes(q.OP_MERGE, q.BF16, 1, 64, 64, 8) == 0
     assert q.workspace_bytes(q.OP_FWD, q.BF16, 1, 64, 64, 129) == 0
-    assert q.workspace_bytes(9, q.BF16, 1, 64, 64, 8) == 0
+    # the DoRA backward holds the pre-scale output Z and dZ besides the LoRA backward's scratch
+    assert (q.workspace_bytes(q.OP_DORA_BWD, q.BF16, 4096, 4096, 4096, 16)
+            >= q.workspace_bytes(q.OP_BWD, q.BF16, 4096, 4096, 4096, 16) + 2 * 2 * 4096 * 4096)
+    assert q.workspace_bytes(10, q.BF16, 1, 64, 64, 8) == 0
 
 
 def test_status_strings(L):

@@ -667,6 +667,36 @@ def test_dora_magnitude_at_norms_is_lora(q):
     assert rel_fro(host(Hd), host(Hl).astype(np.float64)) <= 4e-3
 
 
+def run_dora_bwd(q, case, rows=None, seed=0):
+    """DoRA backward through the C ABI against the oracle's exact chain rule: dA, dB, dm in full,
+    dX on the given token rows (all by default)."""
+    import torch
+    w, oc = quantize_both(q, case.W0)
+    Wh = oracle_weight(oc, case.d_out, case.d_in, "bf16")
+    mag = np.random.default_rng(seed).uniform(0.5, 2.0, case.d_out).astype(np.float32)
+    dX, dA, dB, dm = q.qlora_dora_bwd(w, dev(case.X, "bf16"), dev(case.dH, "bf16"), dev(case.A, "bf16"),
+                                      dev(case.B, "bf16"), case.alpha, torch.from_numpy(mag).cuda())
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    rX, rA, rB, rm = O.dora_backward(Wh, case.X, case.dH, case.A, case.B, case.alpha, case.r, mag)
+    sel = slice(None) if rows is None else rows
+    err = {"dX": rel_fro(host(dX)[sel], rX[sel]), "dA": rel_fro(host(dA), rA), "dB": rel_fro(host(dB), rB),
+           "dm": rel_fro(host(dm), rm)}
+    assert all(v <= TOL["bf16"] for v in err.values()), err
+
+
+@pytest.mark.parametrize("d_out,d_in,r,T", [(256, 256, 8, 64), (200, 192, 5, 77), (520, 320, 16, 300),
+                                            (136, 256, 100, 3)])
+def test_dora_backward(q, d_out, d_in, r, T):
+    run_dora_bwd(q, S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_out + T))
+
+
+def test_dora_backward_q_proj_sampled_rows(q):
+    case = S.make_layer(**S.CONFIGS["q_proj_4096x4096_r16_T4096"], seed=4)
+    rows = np.sort(np.random.default_rng(6).choice(case.T, 256, replace=False))
+    run_dora_bwd(q, case, rows=rows)
+
+
 # ------------------------------------------------------------------ FP8 activations (R25)
 
 
