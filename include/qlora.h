@@ -25,8 +25,10 @@
  *    the library never allocates or frees device memory and never synchronises the host,
  *    except qlora_get_device_error().  All work is enqueued on the given stream.
  *  - Alignment: device pointers must be 16-byte aligned, else QLORA_ERR_INVALID_ARG.
- *  - Shapes: d_in % 64 == 0 (a block never straddles rows), d_out % 8 == 0, T >= 1,
- *    1 <= r <= 128; otherwise QLORA_ERR_UNSUPPORTED.  Ragged tiles in T, d_out, d_in are handled.
+ *  - Shapes: d_in % 64 == 0 (a block never straddles rows), d_out >= 1 (any value: ragged last
+ *    rows are masked, and a backward whose dH rows are not whole 16-byte units copies dH into
+ *    padded rows first), T >= 1, 1 <= r <= 128; otherwise QLORA_ERR_UNSUPPORTED.  The FP8
+ *    backward alone needs d_out % 16 == 0 (its E5M2 gradient rows are read by a tensor map).
  *  - dtype: QLORA_BF16 or QLORA_F32 sets X, H, dH, dX, A and B.  dA and dB are always fp32 and
  *    are overwritten (not accumulated).  The fp32 path is exact fp32 arithmetic (no TF32).
  *  - Errors found on the host return at once and nothing is launched.  Errors found on the

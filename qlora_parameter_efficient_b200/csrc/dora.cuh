@@ -29,20 +29,34 @@ __global__ void __launch_bounds__(256) k_dora_colred(const __nv_bfloat16* __rest
     griddep_enter();
     const int64_t j = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
     if (j >= d) return;
+    const bool two = j + 1 < d;
+    const bool pairs = (d & 1) == 0;                  // rows of whole bf16 pairs (4-byte aligned)
     const int64_t t0 = (T * blockIdx.y) / gridDim.y, t1 = (T * (blockIdx.y + 1)) / gridDim.y;
-    const float n0 = norms[j], n1 = norms[j + 1];
-    const float c0 = n0 > 0.f ? magnitude[j] / n0 : 0.f, c1 = n1 > 0.f ? magnitude[j + 1] / n1 : 0.f;
+    const float n0 = norms[j], n1 = two ? norms[j + 1] : 0.f;
+    const float c0 = n0 > 0.f ? magnitude[j] / n0 : 0.f;
+    const float c1 = n1 > 0.f ? magnitude[j + 1] / n1 : 0.f;
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll 4
     for (int64_t t = t0; t < t1; ++t) {
-        const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dH + t * d + j));
-        const float2 z = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Z + t * d + j));
-        a0 = fmaf(g.x, z.x, a0);
-        a1 = fmaf(g.y, z.y, a1);
-        *reinterpret_cast<__nv_bfloat162*>(dZ + t * d + j) = __floats2bfloat162_rn(g.x * c0, g.y * c1);
+        float2 gv, zv;
+        if (pairs) {
+            gv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dH + t * d + j));
+            zv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Z + t * d + j));
+        } else {
+            gv = make_float2(__bfloat162float(dH[t * d + j]), two ? __bfloat162float(dH[t * d + j + 1]) : 0.f);
+            zv = make_float2(__bfloat162float(Z[t * d + j]), two ? __bfloat162float(Z[t * d + j + 1]) : 0.f);
+        }
+        a0 = fmaf(gv.x, zv.x, a0);
+        a1 = fmaf(gv.y, zv.y, a1);
+        if (pairs) {
+            *reinterpret_cast<__nv_bfloat162*>(dZ + t * d + j) = __floats2bfloat162_rn(gv.x * c0, gv.y * c1);
+        } else {
+            dZ[t * d + j] = __float2bfloat16_rn(gv.x * c0);
+            if (two) dZ[t * d + j + 1] = __float2bfloat16_rn(gv.y * c1);
+        }
     }
     part[blockIdx.y * d + j] = a0;
-    part[blockIdx.y * d + j + 1] = a1;
+    if (two) part[blockIdx.y * d + j + 1] = a1;
 }
 
 // dc (chunks in order), dm = dc / n and e = -dc m / n^3 (0 for a row of norm 0)
@@ -60,14 +74,16 @@ __global__ void k_dora_coef(const float* __restrict__ part, int chunks, int64_t 
     }
 }
 
-// Ge[i][j] = bf16(B[j][i] e_j): the rows B^T diag(e) that the dX-form GEMM multiplies by W^
+// Ge[i][j] = bf16(B[j][i] e_j): the rows B^T diag(e) that the dX-form GEMM multiplies by W^ (row
+// stride ld >= d, a multiple of 8 so that the GEMM's tensor map can read it; columns past d are
+// zero)
 __global__ void k_dora_ge(const __nv_bfloat16* __restrict__ B, const float* __restrict__ e, int r,
-                          int64_t d, __nv_bfloat16* __restrict__ ge) {
+                          int64_t d, int64_t ld, __nv_bfloat16* __restrict__ ge) {
     griddep_enter();
-    for (int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; x < r * d;
+    for (int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; x < r * ld;
          x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t i = x / d, j = x % d;
-        ge[x] = __float2bfloat16_rn(__bfloat162float(B[j * r + i]) * e[j]);
+        const int64_t i = x / ld, j = x % ld;
+        ge[x] = __float2bfloat16_rn(j < d ? __bfloat162float(B[j * r + i]) * e[j] : 0.f);
     }
 }
 

@@ -509,6 +509,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThread
                 if (grow < args.M) {
                     const int gc = gc0 + c0;
                     __nv_bfloat16* o = args.out + grow * args.ld_out + gc;
+                    const bool vec_rows = (args.ld_out & 7) == 0;      // every row 16-byte aligned
                     if constexpr (FP8) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * out_scale);
@@ -522,13 +523,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G2Smem<FP8>::kThread
                     }
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
-                        if (gc + 8 * g < args.N) {
+                        if (gc + 8 * g + 8 <= args.N && vec_rows) {
                             uint4 v;
                             v.x = pack_bf16x2(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
                             v.y = pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
                             v.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
                             v.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
                             *reinterpret_cast<uint4*>(o + 8 * g) = v;
+                        } else {
+                            // a ragged last column block, or rows that are not whole 16-byte units
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                if (gc + 8 * g + e < args.N) o[8 * g + e] = __float2bfloat16_rn(__uint_as_float(r[8 * g + e]));
                         }
                     }
                 }

@@ -270,6 +270,7 @@ struct Plan {
     int seg_ldu = 0, seg_max_tiles = 0;
     size_t dora_part = 0, dora_scale = 0;   // DoRA row-norm partials and column scale
     size_t f8_x = 0, f8_dh = 0, f8_g = 0;    // FP8 backward: bf16 X~, dH~ and sigma sigma_w s G
+    size_t dh_pad = 0;     // bf16 backward, d_out not a multiple of 8: dH with 16-byte rows
     size_t total = 0;
 };
 
@@ -357,6 +358,7 @@ Plan make_plan(int op, qlora_dtype dtype, int64_t T, int64_t d_out, int64_t d_in
             p.split_g = choose_split(mt, cdiv(d_out, kBK));
             p.split_da = choose_split(cdiv(d_in, kBM), cdiv(T, kBK));
             p.split_db = choose_split(cdiv(d_out, kBM), cdiv(T, kBK));
+            if (d_out % 8 != 0) p.dh_pad = take(static_cast<size_t>(T) * (d_out + 7) / 8 * 8 * 2);
             part = std::max(part, static_cast<size_t>(p.split_g) * T * RP * 4);
             part = std::max(part, static_cast<size_t>(p.split_da) * d_in * RP * 4);
             part = std::max(part, static_cast<size_t>(p.split_db) * d_out * RP * 4);
@@ -410,7 +412,7 @@ DoraBwdLayout dora_bwd_layout(int64_t T, int64_t d, int64_t k, int r) {
     L.z = take(static_cast<size_t>(T) * d * 2);
     L.u = take(static_cast<size_t>(T) * r * 2);
     L.dz = take(static_cast<size_t>(T) * d * 2);
-    L.ge = take(static_cast<size_t>(r) * d * 2);
+    L.ge = take(static_cast<size_t>(r) * ((d + 7) / 8 * 8) * 2);
     L.pm = take(static_cast<size_t>(r) * d * 2);
     L.qm = take(static_cast<size_t>(r) * k * 2);
     L.aat = take(static_cast<size_t>(r) * r * 4);
@@ -433,7 +435,7 @@ dim3 grid1d(int64_t n) {
 qlora_status check_nf4(const qlora_nf4* w) {
     if (!w || !aligned16(w->codes) || !aligned16(w->absmax_q) || !aligned16(w->c2))
         return QLORA_ERR_INVALID_ARG;
-    if (w->d_out < 1 || w->d_in < 64 || w->d_in % 64 || w->d_out % 8) return QLORA_ERR_UNSUPPORTED;
+    if (w->d_out < 1 || w->d_in < 64 || w->d_in % 64) return QLORA_ERR_UNSUPPORTED;
     if (w->d_out > (1 << 30) || w->d_in > (1 << 30)) return QLORA_ERR_UNSUPPORTED;
     return QLORA_OK;
 }
@@ -523,7 +525,8 @@ qlora_status skinny_gemm(bool a_mn, bool b_mn, int RP, int n_valid, const CUtens
 qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, const void* ext_a,
                       const void* ext_b, int RP, int r_used, int ext_b_rank, void* out,
                       void* g2ws, int* err, cudaStream_t st, const float* col_scale = nullptr,
-                      const float* x_scale = nullptr, const float* w_scale = nullptr) {
+                      const float* x_scale = nullptr, const float* w_scale = nullptr,
+                      int64_t act_ld = 0) {
     // x_scale != NULL: the FP8 variant (act is the E4M3 activation or, for dX, the E5M2
     // gradient; ext_a the adapter term in sigma sigma_w units; x_scale that tensor's sigma)
     const bool fp8 = x_scale != nullptr;
@@ -536,7 +539,7 @@ qlora_status nf4_gemm(bool dx, const qlora_nf4* w, const void* act, int64_t T, c
         QL_TRY(tmap_u8_sw128(&ta, act, T, K, K, 128));
         QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 64, 128));
     } else {
-        QL_TRY(tmap_bf16(&ta, act, T, K, K, 128));
+        QL_TRY(tmap_bf16(&ta, act, T, K, act_ld > 0 ? act_ld : K, 128));
         if (dx) QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 64, 64));
         else QL_TRY(tmap_u8(&tc, w->codes, d_out, d_in / 2, d_in / 2, 32, 128));
     }
@@ -911,10 +914,19 @@ qlora_status bwd_bf16(const qlora_nf4* w, const void* X, const void* dH, int64_t
         QL_TRY(compute_u_bf16(X, T, d_in, a_src, a_rows, RP, r, s, p.split_u, part, nullptr,
                               u_pad, nullptr, err, stream));
     }
+    // Rows of d_out bf16 that are not whole 16-byte units cannot be read by a tensor map: such a
+    // dH is copied into rows of d_out rounded up to 8 (the maps still stop at column d_out).
+    int64_t dh_ld = d_out;
+    if (d_out % 8 != 0 && !f8) {
+        dh_ld = (d_out + 7) / 8 * 8;
+        auto* dh_pad = at<__nv_bfloat16>(ws, p.dh_pad);
+        QL_TRY(pad_bf16(static_cast<const __nv_bfloat16*>(dH), T, d_out, d_out, dh_pad, T, dh_ld, 0, dh_ld, stream));
+        dH = dh_pad;
+    }
     // G = dH B  ->  g_spad = bf16(s G)
     {
         CUtensorMap tdh, tbp;
-        QL_TRY(tmap_bf16(&tdh, dH, T, d_out, d_out, kBM));
+        QL_TRY(tmap_bf16(&tdh, dH, T, d_out, dh_ld, kBM));
         QL_TRY(tmap_bf16(&tbp, b_src, d_out, b_ld, b_ld, 64));
         QL_TRY(skinny_gemm(false, true, RP, r, tdh, tbp, T, cdiv(d_out, kBK), p.split_g, part, err, stream));
         if (launch_pdl(k_finalize_rows<__nv_bfloat16>, grid1d(T * RP), dim3(256), 0, stream,
@@ -924,7 +936,9 @@ qlora_status bwd_bf16(const qlora_nf4* w, const void* X, const void* dH, int64_t
         QL_LAUNCH_CHECK();
     }
     // dX = dH W^ + (sG) A
-    if (dX && !f8) QL_TRY(nf4_gemm(true, w, dH, T, g_spad, a_src, RP, r, a_rows, dX, at<void>(ws, p.g2), err, stream));
+    if (dX && !f8)
+        QL_TRY(nf4_gemm(true, w, dH, T, g_spad, a_src, RP, r, a_rows, dX, at<void>(ws, p.g2), err, stream,
+                        nullptr, nullptr, nullptr, dh_ld));
     if (dX && f8) {
         // FP8: the adapter operand in the accumulator's units (sigma_g sigma_w, powers of two),
         // then the E5M2 x E4M3 GEMM with the epilogue factor 1 / (sigma_g sigma_w)
@@ -950,7 +964,7 @@ qlora_status bwd_bf16(const qlora_nf4* w, const void* X, const void* dH, int64_t
     // dB[d_out, RP] = s dH^T U
     {
         CUtensorMap thm, tum;
-        QL_TRY(tmap_bf16(&thm, dH, T, d_out, d_out, 64));
+        QL_TRY(tmap_bf16(&thm, dH, T, d_out, dh_ld, 64));
         QL_TRY(tmap_bf16(&tum, u_src, T, u_ld, u_ld, 64));
         QL_TRY(skinny_gemm(true, true, RP, r, thm, tum, d_out, cdiv(T, kBK), p.split_db, part, err, stream));
         if (launch_pdl(k_finalize_dB, grid1d(d_out * r), dim3(256), 0, stream, part, p.split_db,
@@ -1164,12 +1178,14 @@ qlora_status qlora_dora_bwd(const qlora_nf4* w, const void* X, const void* dH, i
     QL_TRY(bwd_bf16(w, X, dZ, T, A, B, r, s, U, dX, dA, dB, pb, shared, err, 0, stream, nullptr));
     // the norm's term: P = A W^T and Q = (B^T diag(e)) W^ by the fused NF4 GEMM with the r
     // adapter rows as tokens, then the r x r Gram products and the two updates
-    if (launch_pdl(k_dora_ge, grid1d(r * d), dim3(256), 0, stream, static_cast<const bf*>(B),
-                   static_cast<const float*>(e), static_cast<int>(r), d, ge) != cudaSuccess)
+    const int64_t ge_ld = (d + 7) / 8 * 8;
+    if (launch_pdl(k_dora_ge, grid1d(r * ge_ld), dim3(256), 0, stream, static_cast<const bf*>(B),
+                   static_cast<const float*>(e), static_cast<int>(r), d, ge_ld, ge) != cudaSuccess)
         return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     QL_TRY(nf4_gemm(false, w, A, r, nullptr, nullptr, 0, 0, 0, pm, shared, err, stream));
-    QL_TRY(nf4_gemm(true, w, ge, r, nullptr, nullptr, 0, 0, 0, qm, shared, err, stream));
+    QL_TRY(nf4_gemm(true, w, ge, r, nullptr, nullptr, 0, 0, 0, qm, shared, err, stream, nullptr, nullptr,
+                    nullptr, ge_ld));
     if (launch_pdl(k_dora_gram, dim3(static_cast<unsigned>(r * r), 2), dim3(256), 0, stream,
                    static_cast<const bf*>(A), static_cast<const bf*>(B), static_cast<const float*>(e),
                    static_cast<int>(r), d, k, aat, beb) != cudaSuccess)

@@ -308,8 +308,15 @@ __global__ void __launch_bounds__(128, QLORA_SEG_EXPAND_MINB) k_seg_expand(SegAr
             for (int n = 0; n < 8; ++n) {
                 const int col = 64 * blk + 8 * n + 2 * t;
                 const bool okc = col < a.d_out;
-                h[n][0] = (okc && ra) ? *reinterpret_cast<const uint32_t*>(ha + col) : 0u;
-                h[n][1] = (okc && rb) ? *reinterpret_cast<const uint32_t*>(hb + col) : 0u;
+                // two adjacent bf16 of a row (read one by one when rows have an odd length)
+                auto pair = [&](const __nv_bfloat16* row) -> uint32_t {
+                    if (!(a.d_out & 1)) return *reinterpret_cast<const uint32_t*>(row + col);
+                    const uint32_t lo = *reinterpret_cast<const unsigned short*>(row + col);
+                    const uint32_t hi = col + 1 < a.d_out ? *reinterpret_cast<const unsigned short*>(row + col + 1) : 0u;
+                    return lo | (hi << 16);
+                };
+                h[n][0] = (okc && ra) ? pair(ha) : 0u;
+                h[n][1] = (okc && rb) ? pair(hb) : 0u;
             }
         };
         // B_i quads of one K step of a 64-column block (rows = output columns)
@@ -365,8 +372,14 @@ __global__ void __launch_bounds__(128, QLORA_SEG_EXPAND_MINB) k_seg_expand(SegAr
                         __nv_bfloat162 base;
                         *reinterpret_cast<uint32_t*>(&base) = hv[u][n][hh];
                         const float2 bf = __bfloat1622float2(base);
-                        *reinterpret_cast<__nv_bfloat162*>(a.H + static_cast<int64_t>(tok) * a.d_out + col) =
-                            __floats2bfloat162_rn(bf.x + acc[n][2 * hh], bf.y + acc[n][2 * hh + 1]);
+                        __nv_bfloat16* dst = a.H + static_cast<int64_t>(tok) * a.d_out + col;
+                        if (!(a.d_out & 1)) {
+                            *reinterpret_cast<__nv_bfloat162*>(dst) =
+                                __floats2bfloat162_rn(bf.x + acc[n][2 * hh], bf.y + acc[n][2 * hh + 1]);
+                        } else {
+                            dst[0] = __float2bfloat16_rn(bf.x + acc[n][2 * hh]);
+                            if (col + 1 < a.d_out) dst[1] = __float2bfloat16_rn(bf.y + acc[n][2 * hh + 1]);
+                        }
                     }
                 }
             }

@@ -330,23 +330,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (OUT_F32) {
                         float* o = reinterpret_cast<float*>(args.out) + z * args.split_stride +
                                    grow * args.ld_out + gc;
+                        // 16-byte stores where the row and the block are whole, else one by one
+                        const bool vec = (args.ld_out & 3) == 0 && (args.split_stride & 3) == 0;
 #pragma unroll
-                        for (int g = 0; g < 8; ++g)
-                            if (gc + 4 * g < args.N)
+                        for (int g = 0; g < 8; ++g) {
+                            if (vec && gc + 4 * g + 4 <= args.N) {
                                 *reinterpret_cast<uint4*>(o + 4 * g) =
                                     make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    if (gc + 4 * g + e < args.N) o[4 * g + e] = __uint_as_float(r[4 * g + e]);
+                            }
+                        }
                     } else {
                         __nv_bfloat16* o =
                             reinterpret_cast<__nv_bfloat16*>(args.out) + grow * args.ld_out + gc;
+                        const bool vec = (args.ld_out & 7) == 0;
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
-                            if (gc + 8 * g < args.N) {
+                            if (vec && gc + 8 * g + 8 <= args.N) {
                                 uint4 v;
                                 v.x = pack_bf16x2(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
                                 v.y = pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
                                 v.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
                                 v.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
                                 *reinterpret_cast<uint4*>(o + 8 * g) = v;
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    if (gc + 8 * g + e < args.N) o[8 * g + e] = __float2bfloat16_rn(__uint_as_float(r[8 * g + e]));
                             }
                         }
                     }

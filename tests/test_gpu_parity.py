@@ -137,6 +137,18 @@ def test_layer_bf16_split_tail(q, d_out, d_in, r, T):
     run_layer(q, case)
 
 
+# d_out that is not a multiple of 8: the output rows are not whole 16-byte units (the GEMM
+# epilogues store element by element) and the backward copies dH into padded rows for its tensor
+# maps.  Token counts take the large-T route (300, 1030), the mid-size split-K route (40) and the
+# decode-size stream (1, 5, 12).
+@pytest.mark.parametrize("d_out,d_in,r,T", [(100, 256, 16, 300), (203, 320, 5, 1030), (203, 512, 8, 40),
+                                            (100, 512, 16, 1), (203, 1024, 33, 5), (1001, 4096, 64, 12),
+                                            (77, 192, 3, 130)])
+def test_layer_bf16_ragged_d_out(q, d_out, d_in, r, T):
+    case = S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_out + T)
+    run_layer(q, case)
+
+
 @pytest.mark.parametrize("d_out,d_in,r,T", [(256, 256, 8, 64), (200, 192, 5, 77), (64, 128, 3, 1)])
 def test_layer_f32(q, d_out, d_in, r, T):
     case = S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="f32", seed=3)
@@ -345,6 +357,11 @@ def test_batched_small(q, dtype):
     run_batched(q, mc)
 
 
+def test_batched_ragged_d_out(q):
+    mc = S.make_multi_adapter(203, 320, 150, [3, 8, 20], dtype="bf16", seed=18)
+    run_batched(q, mc)
+
+
 def test_batched_full_uniform_and_skewed(q):
     for split in (None, [0.7, 0.1, 0.1, 0.1]):
         mc = S.make_multi_adapter(4096, 4096, 4096, [8, 16, 16, 64], split=split, seed=0)
@@ -373,6 +390,13 @@ def run_multi(q, mc, rows=None):
 # mixed ranks 1..128 (odd ranks take the 16-bit B path, r > 64 two K tiles), ragged shapes
 def test_multi_mixed_ranks(q):
     mc = S.make_multi_adapter(264, 320, 300, [1, 3, 8, 16, 33, 64, 100, 128, 7, 24], seed=11)
+    run_multi(q, mc)
+
+
+# odd and non-multiple-of-8 output widths: rows of H are not whole bf16 pairs / 16-byte units
+@pytest.mark.parametrize("d_out", [203, 100])
+def test_multi_ragged_d_out(q, d_out):
+    mc = S.make_multi_adapter(d_out, 256, 150, [5, 16, 64], seed=17 + d_out)
     run_multi(q, mc)
 
 
@@ -643,7 +667,7 @@ def run_dora(q, case, rows=None, seed=0):
 
 
 @pytest.mark.parametrize("d_out,d_in,r,T", [(256, 256, 8, 64), (200, 192, 5, 77), (520, 320, 16, 300),
-                                            (136, 256, 100, 3)])
+                                            (136, 256, 100, 3), (203, 256, 8, 90)])
 def test_dora_forward(q, d_out, d_in, r, T):
     run_dora(q, S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_in + T, with_grad=False))
 
@@ -686,7 +710,7 @@ def run_dora_bwd(q, case, rows=None, seed=0):
 
 
 @pytest.mark.parametrize("d_out,d_in,r,T", [(256, 256, 8, 64), (200, 192, 5, 77), (520, 320, 16, 300),
-                                            (136, 256, 100, 3)])
+                                            (136, 256, 100, 3), (203, 256, 8, 90)])
 def test_dora_backward(q, d_out, d_in, r, T):
     run_dora_bwd(q, S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_out + T))
 
