@@ -127,6 +127,28 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float4 v) {
                  : "memory");
 }
 
+// Bounded wait for a finaliser: polls the barrier with a short sleep between tries, so that a
+// finaliser waiting for its next tile takes few issue slots from the compute warps of its
+// scheduler.  Gives up (false) on *abort or after limit_ns, like mbar_wait_warp.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit_ns) {
+    const uint32_t addr = smem_u32(bar);
+    uint32_t ok = mbar_test_wait(addr, parity) ? 1u : 0u;
+    if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        const uint64_t t0 = globaltimer_ns();
+        while (true) {
+            __nanosleep(128);
+            if (mbar_test_wait(addr, parity)) {
+                ok = 1u;
+                break;
+            }
+            if (*abort || globaltimer_ns() - t0 > limit_ns) break;
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    return ok != 0u;
+}
+
 template <int NT8>
 __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
     using Cf = LvCfg<NT8>;
@@ -368,16 +390,6 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
         // rank order, applies 1/127, adds the adapter term and writes H.  Each keeps the adapter
         // rows of its next tile in flight (cp.async into its own s_b buffer).
         const int f = warp - kLvWarps;
-        // (rank 0) s U from the pre-pass, staged by finaliser 0 once it has finished
-        if (rank == 0 && f == 0) {
-            griddep_wait();
-            const uint32_t dst = smem_u32(s_us);
-            for (int i = lane; i < 16 * kLvSuLd / 8; i += 32) cp_async16(dst + 16 * i, a.us_pad + 8 * i, 16u);
-            cp_async_commit();
-            cp_async_wait<0>();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(us_bar);
-        }
         // the adapter rows of tile li into this finaliser's s_b buffer (one cp.async group; rows
         // whose r bf16 are not whole 16-byte units are read at use instead)
         const bool b_vec = (a.r % 8) == 0;
@@ -410,7 +422,7 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
         for (int li = f; li < ntl; li += NBUF) {
             const int buf = f;                              // li % NBUF
             // ---- the 16 partials of the tile in warp order
-            if (!mbar_wait_warp(&full[buf], (li / NBUF) & 1, abort, a.wait_ns)) {
+            if (!mbar_wait_idle(&full[buf], (li / NBUF) & 1, abort, a.wait_ns)) {
                 set_error(a.err, kErrTimeout);
                 *abort = 1;
                 break;
@@ -470,8 +482,19 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
             }
             // ---- rank 0: 1/127, the adapter term (B rows times bf16 s U on the tensor cores,
             // fp32 accumulation), H
+            // s U from the pre-pass, staged by finaliser 0 once its first tile is summed (the
+            // sums never wait for the pre-pass)
             if (!us_ready) {
-                if (!mbar_wait_warp(us_bar, 0, abort, a.wait_ns)) {
+                if (f == 0) {
+                    griddep_wait();
+                    cp_async_wait<0>();                     // this tile's B rows (group order)
+                    const uint32_t dst = smem_u32(s_us);
+                    for (int i = lane; i < 16 * kLvSuLd / 8; i += 32) cp_async16(dst + 16 * i, a.us_pad + 8 * i, 16u);
+                    cp_async_commit();
+                    cp_async_wait<0>();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(us_bar);
+                } else if (!mbar_wait_warp(us_bar, 0, abort, a.wait_ns)) {
                     set_error(a.err, kErrTimeout);
                     *abort = 1;
                     break;
