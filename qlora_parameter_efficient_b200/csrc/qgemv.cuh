@@ -25,16 +25,17 @@
 // Work split.  Rows come in tiles of 16; a cluster of C CTAs (C = 1, 2, 4 or 8) owns a
 // contiguous range of tiles and its 16 warps x C ranks split K: warp w of rank p owns the KB
 // consecutive 64-blocks starting at (16 p + w) KB (KB = 4 for up to 8 tokens, 2 for up to 16).
-// The warp's X fragments stay in registers for the whole kernel; per tile it streams the codes
-// of its 16 rows x KB blocks straight from global memory into registers (8 bytes of a row per
-// thread, the k order inside a block permuted consistently in the codes and X so that those 8
-// bytes are the thread's A registers of the block's four k16 steps), one tile ahead, with the
-// tile two ahead prefetched into L2.  Each warp writes its tile partial to shared memory; warp
-// (tile mod 16) sums the 16 partials in warp order, the ranks' sums meet in rank 0 over DSMEM
-// (rank order), and rank 0 applies 1/127, adds the adapter term with a few mma steps over bf16
-// s U (from the pre-pass) and the tile's B rows, and writes H.  Partial-sum buffers are double
-// buffered so that the warps run on while a tile is finalised.  No global partials, atomics or
-// semaphores: the sums are deterministic and the tail is on-chip.
+// The warp's X fragments stay in registers for the whole kernel; the codes of its 16 rows x KB
+// blocks of a tile (a "slice") come through its own ring of S slices in shared memory, filled by
+// 16-byte cp.async S - 1 tiles ahead of use (XOR-swizzled 16-byte chunks, so that the fragment
+// reads of 8 rows fall in different banks).  A thread reads 8 bytes of a row per block, the k
+// order inside a block permuted consistently in the codes and X so that those 8 bytes are the
+// thread's A registers of the block's four k16 steps.  Each warp writes its tile partial to one
+// of NBUF shared buffers; a dedicated finaliser warp per buffer sums the 16 partials in warp
+// order, the ranks' sums meet in rank 0 over DSMEM (rank order), and rank 0 applies 1/127, adds
+// the adapter term with a few mma steps over bf16 s U (from the pre-pass) and the tile's B rows,
+// and writes H, while the compute warps run on into the next tiles.  No global partials,
+// atomics or semaphores: the sums are deterministic and the tail is on-chip.
 //
 // Why warp-level mma.sync and not tcgen05 here: one tcgen05.mma of M = 128, K = 16 occupies the
 // SM's tensor core for ~130-190 cycles whatever N is (measured on B200 with N = 16..256), i.e. at
@@ -232,7 +233,7 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
 #pragma unroll
             for (int i = 0; i < kChunks / 32; ++i) {
                 const int idx = lane + 32 * i, row = idx / (2 * KB), c = idx % (2 * KB);
-                const bool ok = (t_lo + li) * 16 + row < a.d_out;
+                const bool ok = (t_lo + li) * 16 + row < a.d_out && dcheck(kb0 + KB <= a.kt, a.err);
                 cp_async16(dst + row * Cf::kRowBytes + ((c ^ swz(row)) << 4),
                            ok ? static_cast<const void*>(w0 + (static_cast<int64_t>(li) * 16 + row) * row_bytes + 16 * c)
                               : static_cast<const void*>(a.codes),
@@ -451,6 +452,7 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
                         *abort = 1;
                         break;
                     }
+                    if (!dcheck(rank < MR, a.err)) break;
 #pragma unroll
                     for (int n = 0; n < NT8; ++n)
                         st_cluster_v4(mapa_shared(smem_u32(ring + ((buf * MR + rank) * NT8 + n) * 32 + lane), 0), tot[n]);
