@@ -266,18 +266,29 @@ def run_gpu(args):
     H = torch.empty((T, d), dtype=bf, device=dev)
     U = torch.empty((T, r), dtype=bf, device=dev)
     dX = torch.empty((T, k), dtype=bf, device=dev)
-    dA = torch.empty((r, k), dtype=torch.float32, device=dev)
-    dB = torch.empty((d, r), dtype=torch.float32, device=dev)
+    # dA and dB in one flat buffer: one all-reduce per step when the data-parallel ranks sum them
+    grads = torch.empty(r * k + d * r, dtype=torch.float32, device=dev)
+    dA = grads[: r * k].view(r, k)
+    dB = grads[r * k:].view(d, r)
     ws = torch.empty(max(q.workspace_bytes(q.OP_FWD, q.BF16, T, d, k, r),
                          q.workspace_bytes(q.OP_BWD, q.BF16, T, d, k, r)), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    def backward(w, X_, dH_, A_, B_):
+        if world == 1:
+            q.qlora_linear_bwd(w, X_, dH_, A_, B_, alpha, U_saved=U, dX=dX, dA=dA, dB=dB, ws=ws)
+            return
+        # dA, dB first, then their sum over ranks on NCCL's stream beside the dX GEMM
+        dp.backward_overlapped(
+            lambda: q.qlora_linear_bwd(w, X_, dH_, A_, B_, alpha, U_saved=U, dA=dA, dB=dB, ws=ws,
+                                       phase="grads"),
+            lambda: q.qlora_linear_bwd(w, X_, dH_, A_, B_, alpha, U_saved=U, dX=dX, ws=ws, phase="dx"),
+            grads)
+
     def step(i):
         s = sets[i % NSETS]
         q.qlora_linear_fwd(s["w"], s["X"], s["A"], s["B"], alpha, H=H, U_save=U, ws=ws)
-        q.qlora_linear_bwd(s["w"], s["X"], s["dH"], s["A"], s["B"], alpha, U_saved=U, dX=dX, dA=dA,
-                           dB=dB, ws=ws)
-        dp.allreduce_adapter_grads(dA, dB)
+        backward(s["w"], s["X"], s["dH"], s["A"], s["B"])
 
     def timed(fn, K, W, with_gemm_events=False):
         for i in range(W):
@@ -372,10 +383,8 @@ def run_gpu(args):
             stream.wait_event(ev_in[bi])
             s = sets[i % NSETS]
             q.qlora_linear_fwd(s["w"], Xd[bi], s["A"], s["B"], alpha, H=H, U_save=U, ws=ws)
-            q.qlora_linear_bwd(s["w"], Xd[bi], dHd[bi], s["A"], s["B"], alpha, U_saved=U, dX=dX,
-                               dA=dA, dB=dB, ws=ws)
+            backward(s["w"], Xd[bi], dHd[bi], s["A"], s["B"])
             ev_free[bi].record(stream)
-            dp.allreduce_adapter_grads(dA, dB)
             hdA.copy_(dA, non_blocking=True)
             hdB.copy_(dB, non_blocking=True)
 

@@ -145,6 +145,16 @@ qlora_status qlora_linear_bwd(const qlora_nf4* w, const void* X, const void* dH,
  * micro-batches before one optimizer update ([UH], the gradient-accumulation paragraph next to
  * FlashAttention-2).  dX is always overwritten.  Unknown flag bits: QLORA_ERR_INVALID_ARG.    */
 #define QLORA_BWD_ACCUMULATE 1u
+/* The backward in two calls, so that a data-parallel caller can reduce dA and dB over ranks
+ * while dX is computed ([MF] "Gradient Dynamics and Backpropagation Mechanics": dA and dB are
+ * sums over tokens, dX is per token).  QLORA_BWD_GRADS_ONLY computes G, dA and dB (dX is
+ * ignored and may be NULL) and leaves bf16(s G) in the workspace; QLORA_BWD_DX_FROM_WS then
+ * computes dX only (dA, dB ignored, may be NULL; dX required), reading that bf16(s G) from the
+ * same workspace, which the caller must not have reused in between, with the same w, dH, T, A,
+ * B, r, alpha and dtype.  The pair gives results identical to one call.  Both bits together:
+ * QLORA_ERR_INVALID_ARG. */
+#define QLORA_BWD_GRADS_ONLY 2u
+#define QLORA_BWD_DX_FROM_WS 4u
 qlora_status qlora_linear_bwd_ex(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
                                  const void* A, const void* B, int32_t r, float alpha,
                                  const void* U_saved, qlora_dtype dtype, void* dX,

@@ -231,28 +231,39 @@ def qlora_linear_fwd(w: NF4Weight, X, A, B, alpha, H=None, U_save=None, ws=None,
 
 
 BWD_ACCUMULATE = 1
+BWD_GRADS_ONLY = 2
+BWD_DX_FROM_WS = 4
+_BWD_PHASES = {"all": 0, "grads": BWD_GRADS_ONLY, "dx": BWD_DX_FROM_WS}
 
 
 def qlora_linear_bwd(w: NF4Weight, X, dH, A, B, alpha, U_saved=None, dX=None, dA=None, dB=None,
-                     ws=None, stream=None, want_dx=True, accumulate=False):
-    """Returns (dX, dA, dB); dA, dB fp32.  accumulate=True adds into the given dA, dB."""
+                     ws=None, stream=None, want_dx=True, accumulate=False, phase="all"):
+    """Returns (dX, dA, dB); dA, dB fp32.  accumulate=True adds into the given dA, dB.
+
+    phase="grads" computes dA and dB only and leaves bf16(s G) in ws; phase="dx" then computes
+    dX only from that ws (pass the same ws and operands); phase="all" does both in one call."""
     torch = _torch()
     _contig(X, dH, A, B, U_saved, dX, dA, dB)
+    if phase not in _BWD_PHASES:
+        raise ValueError(f"phase must be one of {sorted(_BWD_PHASES)}")
+    if phase == "dx" and ws is None:
+        raise ValueError('phase="dx" reads the workspace of the preceding phase="grads" call')
     T = X.shape[0]
     r = A.shape[0]
     dt = _dtype_code(X.dtype)
-    if dX is None and want_dx:
+    if dX is None and want_dx and phase != "grads":
         dX = torch.empty((T, w.d_in), dtype=X.dtype, device=X.device)
-    if dA is None:
+    if dA is None and phase != "dx":
         dA = torch.empty((r, w.d_in), dtype=torch.float32, device=X.device)
-    if dB is None:
+    if dB is None and phase != "dx":
         dB = torch.empty((w.d_out, r), dtype=torch.float32, device=X.device)
     ws = _ws(OP_BWD, dt, T, w.d_out, w.d_in, r, X.device, ws)
     c = w._c()
-    if accumulate:
+    flags = _BWD_PHASES[phase] | (BWD_ACCUMULATE if accumulate else 0)
+    if flags:
         _check("qlora_linear_bwd_ex", load().qlora_linear_bwd_ex(
             ctypes.byref(c), _ptr(X), _ptr(dH), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(U_saved),
-            dt, _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), BWD_ACCUMULATE, _stream(stream)))
+            dt, _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), flags, _stream(stream)))
     else:
         _check("qlora_linear_bwd", load().qlora_linear_bwd(
             ctypes.byref(c), _ptr(X), _ptr(dH), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(U_saved),

@@ -881,10 +881,13 @@ struct Fp8Dx {
 
 // The bf16 backward: U (or U_saved), G = dH B, dX (bf16 GEMM, or the FP8 GEMM when f8 is set),
 // dA, dB by split-K tensor-core products and their finalizes.
+// phase: kBwdAll (G, dX, dA, dB), kBwdGrads (G, dA, dB; bf16(sG) stays in the workspace) or
+// kBwdDx (dX only, from the bf16(sG) a kBwdGrads call left in the same workspace).
+enum BwdPhase { kBwdAll = 0, kBwdGrads = 1, kBwdDx = 2 };
 qlora_status bwd_bf16(const qlora_nf4* w, const void* X, const void* dH, int64_t T, const void* A,
                       const void* B, int32_t r, float s, const void* U_saved, void* dX, float* dA,
                       float* dB, const Plan& p, void* ws, int* err, int acc_grads, cudaStream_t stream,
-                      const Fp8Dx* f8) {
+                      const Fp8Dx* f8, BwdPhase phase = kBwdAll) {
     const int64_t d_out = w->d_out, d_in = w->d_in;
     const int RP = p.RP;
     auto* a_pad = at<__nv_bfloat16>(ws, p.a_pad);
@@ -905,7 +908,9 @@ qlora_status bwd_bf16(const qlora_nf4* w, const void* X, const void* dH, int64_t
         b_src = b_pad;
         a_rows = b_ld = RP;
     }
-    if (U_saved && direct) {
+    if (phase == kBwdDx) {
+        // U is not needed for dX
+    } else if (U_saved && direct) {
         u_src = U_saved;
         u_ld = r;
     } else if (U_saved) {
@@ -924,7 +929,7 @@ qlora_status bwd_bf16(const qlora_nf4* w, const void* X, const void* dH, int64_t
         dH = dh_pad;
     }
     // G = dH B  ->  g_spad = bf16(s G)
-    {
+    if (phase != kBwdDx) {
         CUtensorMap tdh, tbp;
         QL_TRY(tmap_bf16(&tdh, dH, T, d_out, dh_ld, kBM));
         QL_TRY(tmap_bf16(&tbp, b_src, d_out, b_ld, b_ld, 64));
@@ -936,6 +941,7 @@ qlora_status bwd_bf16(const qlora_nf4* w, const void* X, const void* dH, int64_t
         QL_LAUNCH_CHECK();
     }
     // dX = dH W^ + (sG) A
+    if (phase == kBwdGrads) dX = nullptr;
     if (dX && !f8)
         QL_TRY(nf4_gemm(true, w, dH, T, g_spad, a_src, RP, r, a_rows, dX, at<void>(ws, p.g2), err, stream,
                         nullptr, nullptr, nullptr, dh_ld));
@@ -950,6 +956,7 @@ qlora_status bwd_bf16(const qlora_nf4* w, const void* X, const void* dH, int64_t
         QL_TRY(nf4_gemm(true, w, f8->dH8, T, f8->g8, a_src, RP, r, a_rows, dX, at<void>(ws, p.g2), err, stream,
                         nullptr, f8->g_scale, f8->w_scale));
     }
+    if (phase == kBwdDx) return QLORA_OK;
     // dA^T[d_in, RP] = X^T (sG)
     {
         CUtensorMap txm, tgm;
@@ -972,7 +979,6 @@ qlora_status bwd_bf16(const qlora_nf4* w, const void* X, const void* dH, int64_t
             return QLORA_ERR_CUDA;
         QL_LAUNCH_CHECK();
     }
-    return QLORA_OK;
     return QLORA_OK;
 }
 
@@ -1330,12 +1336,19 @@ qlora_status qlora_linear_bwd_ex(const qlora_nf4* w, const void* X, const void* 
                                  const void* U_saved, qlora_dtype dtype, void* dX, float* dA,
                                  float* dB, void* ws, size_t ws_bytes, uint32_t flags,
                                  cudaStream_t stream) {
-    if (flags & ~static_cast<uint32_t>(QLORA_BWD_ACCUMULATE)) return QLORA_ERR_INVALID_ARG;
+    constexpr uint32_t kKnown = QLORA_BWD_ACCUMULATE | QLORA_BWD_GRADS_ONLY | QLORA_BWD_DX_FROM_WS;
+    if (flags & ~kKnown) return QLORA_ERR_INVALID_ARG;
+    const bool grads_only = (flags & QLORA_BWD_GRADS_ONLY) != 0;
+    const bool dx_only = (flags & QLORA_BWD_DX_FROM_WS) != 0;
+    if (grads_only && dx_only) return QLORA_ERR_INVALID_ARG;
     const int acc_grads = (flags & QLORA_BWD_ACCUMULATE) ? 1 : 0;
     QL_TRY(check_layer(w, T, r, dtype));
-    if (!aligned16(X) || !aligned16(dH) || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
-        !aligned16(dB) || !aligned16_or_null(dX) || !aligned16_or_null(U_saved))
+    if (!aligned16(X) || !aligned16(dH) || !aligned16(A) || !aligned16(B) || !aligned16_or_null(dX) ||
+        !aligned16_or_null(U_saved))
         return QLORA_ERR_INVALID_ARG;
+    if (dx_only ? dX == nullptr : (!aligned16(dA) || !aligned16(dB))) return QLORA_ERR_INVALID_ARG;
+    if (grads_only) dX = nullptr;
+    const BwdPhase phase = grads_only ? kBwdGrads : dx_only ? kBwdDx : kBwdAll;
     const Plan p = make_plan(QLORA_OP_BWD, dtype, T, w->d_out, w->d_in, r);
     QL_TRY(check_ws(ws, ws_bytes, p.total));
     int* err = nullptr;
@@ -1343,7 +1356,8 @@ qlora_status qlora_linear_bwd_ex(const qlora_nf4* w, const void* X, const void* 
     const int64_t d_out = w->d_out, d_in = w->d_in;
     const float s = alpha / static_cast<float>(r);
     if (dtype == QLORA_BF16)
-        return bwd_bf16(w, X, dH, T, A, B, r, s, U_saved, dX, dA, dB, p, ws, err, acc_grads, stream, nullptr);
+        return bwd_bf16(w, X, dH, T, A, B, r, s, U_saved, dX, dA, dB, p, ws, err, acc_grads, stream, nullptr,
+                        phase);
     // exact fp32 path
     const float* Xf = static_cast<const float*>(X);
     const float* dHf = static_cast<const float*>(dH);
@@ -1352,18 +1366,19 @@ qlora_status qlora_linear_bwd_ex(const qlora_nf4* w, const void* X, const void* 
     float* w32 = at<float>(ws, p.w32);
     float* U = at<float>(ws, p.uf);
     float* G = at<float>(ws, p.gf);
-    QL_TRY(dequant_f32(w, w32, stream));
+    if (phase != kBwdGrads) QL_TRY(dequant_f32(w, w32, stream));
     const float* Uc = static_cast<const float*>(U_saved);
-    if (!Uc) {
+    if (!Uc && phase != kBwdDx) {
         QL_TRY(sgemm(stream, T, r, d_in, 1.f, Xf, d_in, false, Af, d_in, true, 0.f, U, r));
         Uc = U;
     }
-    QL_TRY(sgemm(stream, T, r, d_out, 1.f, dHf, d_out, false, Bf, r, false, 0.f, G, r));
+    if (phase != kBwdDx) QL_TRY(sgemm(stream, T, r, d_out, 1.f, dHf, d_out, false, Bf, r, false, 0.f, G, r));
     if (dX) {
         float* dXf = static_cast<float*>(dX);
         QL_TRY(sgemm(stream, T, d_in, d_out, 1.f, dHf, d_out, false, w32, d_in, false, 0.f, dXf, d_in));
         QL_TRY(sgemm(stream, T, d_in, r, s, G, r, false, Af, d_in, false, 1.f, dXf, d_in));
     }
+    if (phase == kBwdDx) return QLORA_OK;
     const float beta = acc_grads ? 1.f : 0.f;
     QL_TRY(sgemm(stream, r, d_in, T, s, G, r, true, Xf, d_in, false, beta, dA, d_in));
     return sgemm(stream, d_out, r, T, s, dHf, d_out, true, Uc, r, false, beta, dB, r);
@@ -1526,10 +1541,15 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4* w, const void* X, int64_t T
     QL_LAUNCH_CHECK();
     QL_TRY(nf4_gemm(false, w, X, T, nullptr, nullptr, 0, 0, 0, H, at<void>(ws, p.g2), err, stream));
     cudaError_t ee;
-    if (r_max <= 16) ee = launch_pdl(k_seg_expand<1>, dim3(seg_grid), dim3(128), 0, stream, a);
-    else if (r_max <= 32) ee = launch_pdl(k_seg_expand<2>, dim3(seg_grid), dim3(128), 0, stream, a);
-    else if (r_max <= 64) ee = launch_pdl(k_seg_expand<4>, dim3(seg_grid), dim3(128), 0, stream, a);
-    else ee = launch_pdl(k_seg_expand<8>, dim3(seg_grid), dim3(128), 0, stream, a);
+    const bool odd = (w->d_out & 1) != 0;
+    if (r_max <= 16)
+        ee = launch_pdl(odd ? k_seg_expand<1, true> : k_seg_expand<1, false>, dim3(seg_grid), dim3(128), 0, stream, a);
+    else if (r_max <= 32)
+        ee = launch_pdl(odd ? k_seg_expand<2, true> : k_seg_expand<2, false>, dim3(seg_grid), dim3(128), 0, stream, a);
+    else if (r_max <= 64)
+        ee = launch_pdl(odd ? k_seg_expand<4, true> : k_seg_expand<4, false>, dim3(seg_grid), dim3(128), 0, stream, a);
+    else
+        ee = launch_pdl(odd ? k_seg_expand<8, true> : k_seg_expand<8, false>, dim3(seg_grid), dim3(128), 0, stream, a);
     if (ee != cudaSuccess) return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     return QLORA_OK;

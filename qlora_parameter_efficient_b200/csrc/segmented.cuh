@@ -266,7 +266,9 @@ __device__ __forceinline__ uint2 ld_quad(const __nv_bfloat16* row, int j, int va
 #ifndef QLORA_SEG_EXPAND_MINB
 #define QLORA_SEG_EXPAND_MINB 4
 #endif
-template <int KS>
+// ODD: d_out is odd, so H's rows are not whole bf16 pairs and are read and written element by
+// element (a separate instance keeps the common even case free of the per-element branches).
+template <int KS, bool ODD>
 __global__ void __launch_bounds__(128, QLORA_SEG_EXPAND_MINB) k_seg_expand(SegArgs a) {
     constexpr int UNR = QLORA_SEG_EXPAND_UNR;     // column blocks per pass of a warp
     griddep_enter();
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(128, QLORA_SEG_EXPAND_MINB) k_seg_expand(SegAr
                 const bool okc = col < a.d_out;
                 // two adjacent bf16 of a row (read one by one when rows have an odd length)
                 auto pair = [&](const __nv_bfloat16* row) -> uint32_t {
-                    if (!(a.d_out & 1)) return *reinterpret_cast<const uint32_t*>(row + col);
+                    if constexpr (!ODD) return *reinterpret_cast<const uint32_t*>(row + col);
                     const uint32_t lo = *reinterpret_cast<const unsigned short*>(row + col);
                     const uint32_t hi = col + 1 < a.d_out ? *reinterpret_cast<const unsigned short*>(row + col + 1) : 0u;
                     return lo | (hi << 16);
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(128, QLORA_SEG_EXPAND_MINB) k_seg_expand(SegAr
                         *reinterpret_cast<uint32_t*>(&base) = hv[u][n][hh];
                         const float2 bf = __bfloat1622float2(base);
                         __nv_bfloat16* dst = a.H + static_cast<int64_t>(tok) * a.d_out + col;
-                        if (!(a.d_out & 1)) {
+                        if constexpr (!ODD) {
                             *reinterpret_cast<__nv_bfloat162*>(dst) =
                                 __floats2bfloat162_rn(bf.x + acc[n][2 * hh], bf.y + acc[n][2 * hh + 1]);
                         } else {

@@ -27,6 +27,25 @@ def allreduce_adapter_grads(dA, dB):
     return dA, dB
 
 
+def backward_overlapped(grads_fn, dx_fn, grads):
+    """The backward with the sum of the adapter gradients over ranks overlapping dX.
+
+    grads_fn() enqueues dA and dB (the library's grads-only phase), which live in the one flat
+    tensor `grads`; the all-reduce of `grads` is then started without waiting, dx_fn() enqueues
+    dX (the library's dX-only phase) meanwhile, and the caller's stream is made to wait for the
+    sum before returning.  With NCCL the reduction runs on NCCL's own stream after the gradient
+    kernels and beside the dX GEMM; every rank issues the same single collective."""
+    import torch.distributed as dist
+    grads_fn()
+    work = None
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        work = dist.all_reduce(grads, async_op=True)
+    dx_fn()
+    if work is not None:
+        work.wait()
+    return grads
+
+
 def max_over_ranks(value: float, device=None) -> float:
     """Largest value over ranks (timings are reported as the slowest rank's)."""
     import torch

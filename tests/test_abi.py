@@ -88,6 +88,21 @@ def test_host_validation_rejects_before_launch(L):
     assert r == 1                                # workspace too small
 
 
+def test_split_backward_flags_validated_before_launch(L):
+    # the grads-only / dX-from-workspace phases of qlora_linear_bwd_ex
+    nf4 = q._NF4(16, 16, 16, 64, 64)
+
+    def bwd(flags, dX=16, dA=16, dB=16):
+        return L.qlora_linear_bwd_ex(ctypes.byref(nf4), 16, 16, 8, 16, 16, 8, 16.0, None, q.BF16,
+                                     dX, dA, dB, 256, 1 << 20, flags, None)
+    assert bwd(q.BWD_GRADS_ONLY | q.BWD_DX_FROM_WS) == 1      # both phases at once
+    assert bwd(8) == 1                                         # unknown bit
+    assert bwd(q.BWD_DX_FROM_WS, dX=None) == 1                 # dX phase without dX
+    assert bwd(q.BWD_GRADS_ONLY, dA=None) == 1                 # grads phase without dA
+    assert bwd(q.BWD_GRADS_ONLY | q.BWD_ACCUMULATE, dB=17) == 1
+    assert bwd(0, dX=None, dA=None) == 1                       # one-call backward needs dA, dB
+
+
 def test_fp8_host_validation_rejects_before_launch(L):
     nf4 = q._NF4(16, 16, 16, 64, 64)
     # forward: a missing scale, a misaligned E4M3 activation

@@ -66,3 +66,46 @@ def test_world2_allreduce_equals_full_batch():
         assert np.allclose(gB, dB, rtol=1e-12, atol=1e-12)
         assert slow == 2.0
     assert out[0][3] == (0, 19) and out[1][3] == (19, 37)
+
+
+def _overlap_worker(rank, world, port, out):
+    import torch
+    import torch.distributed as dist
+
+    from qlora_parameter_efficient_b200 import dp
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        order = []
+        grads = torch.zeros(6, dtype=torch.float64)
+        dX = torch.zeros(3, dtype=torch.float64)
+
+        def grads_fn():
+            order.append("grads")
+            grads.copy_(torch.arange(6, dtype=torch.float64) + 10 * rank)
+
+        def dx_fn():
+            order.append("dx")
+            dX.fill_(rank + 1)
+
+        dp.backward_overlapped(grads_fn, dx_fn, grads)
+        out[rank] = (grads.numpy().copy(), dX.numpy().copy(), order)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_world2_overlapped_backward_sums_grads_and_keeps_dx_local():
+    # dA and dB (one flat tensor) are summed over ranks; dX stays per rank; the gradient phase
+    # is enqueued before the dX phase, which runs while the reduction is in flight
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_overlap_worker, args=(2, port, out), nprocs=2, join=True)
+    want = 2 * np.arange(6, dtype=np.float64) + 10
+    for rank in range(2):
+        g, dx, order = out[rank]
+        assert np.array_equal(g, want)
+        assert np.array_equal(dx, np.full(3, rank + 1.0))
+        assert list(order) == ["grads", "dx"]

@@ -509,6 +509,31 @@ def test_bwd_accumulate_matches_full_batch(q, dtype):
     assert rel_fro(host(dB), host(dB_full).astype(np.float64)) <= 1e-5
 
 
+@pytest.mark.parametrize("dtype,d_out,d_in,r,T", [("bf16", 192, 256, 8, 160), ("bf16", 203, 512, 5, 77),
+                                                  ("bf16", 4096, 4096, 16, 512), ("f32", 192, 256, 8, 160)])
+def test_split_backward_equals_one_call(q, dtype, d_out, d_in, r, T):
+    """The grads-only phase then the dX-from-workspace phase give exactly the one-call results,
+    and both match the oracle."""
+    import torch
+    case = S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype=dtype, seed=37)
+    w, oc = quantize_both(q, case.W0)
+    X, A, B, dH = dev(case.X, dtype), dev(case.A, dtype), dev(case.B, dtype), dev(case.dH, dtype)
+    dX1, dA1, dB1 = q.qlora_linear_bwd(w, X, dH, A, B, case.alpha)
+    ws = torch.empty(q.workspace_bytes(q.OP_BWD, q.BF16 if dtype == "bf16" else q.F32, T, d_out, d_in, r),
+                     dtype=torch.uint8, device="cuda")
+    _, dA2, dB2 = q.qlora_linear_bwd(w, X, dH, A, B, case.alpha, ws=ws, phase="grads")
+    dX2, dA_none, dB_none = q.qlora_linear_bwd(w, X, dH, A, B, case.alpha, ws=ws, phase="dx")
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    assert dA_none is None and dB_none is None
+    assert torch.equal(dX1, dX2) and torch.equal(dA1, dA2) and torch.equal(dB1, dB2)
+    dXref, dAref, dBref = O.lora_backward(oracle_weight(oc, d_out, d_in, dtype), case.X, case.dH, case.A,
+                                          case.B, case.alpha, case.r)
+    assert rel_fro(host(dX2), dXref) <= TOL[dtype]
+    assert rel_fro(host(dA2), dAref) <= TOL[dtype]
+    assert rel_fro(host(dB2), dBref) <= TOL[dtype]
+
+
 # The API takes fp32 hyperparameters; the oracle gets the same (fp32-representable) values, since
 # 1 - beta2 magnifies the fp32 rounding of beta2 = 0.999 to ~1e-5 relative.
 HP = {k: float(np.float32(x)) for k, x in dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8,
