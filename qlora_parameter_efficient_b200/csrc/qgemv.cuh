@@ -30,7 +30,11 @@
 // 16-byte cp.async S - 1 tiles ahead of use (XOR-swizzled 16-byte chunks, so that the fragment
 // reads of 8 rows fall in different banks).  A thread reads 8 bytes of a row per block, the k
 // order inside a block permuted consistently in the codes and X so that those 8 bytes are the
-// thread's A registers of the block's four k16 steps.  Each warp writes its tile partial to one
+// thread's A registers of the block's four k16 steps.  Up to 8 tokens the slice's block scales
+// (16 absmax words and 16 c2 values) ride in the same copy group, one 4-byte cp.async per lane,
+// and are read from shared memory; for 9..16 tokens (half the weights per warp and tile, more
+// registers in use) each warp loads them into registers a tile ahead, which measured faster
+// there (21.9 against 20.9 us at 16 tokens; 12.4 against 13.3 us at 1 token the other way).  Each warp writes its tile partial to one
 // of NBUF shared buffers; a dedicated finaliser warp per buffer sums the 16 partials in warp
 // order, the ranks' sums meet in rank 0 over DSMEM (rank order), and rank 0 applies 1/127, adds
 // the adapter term with a few mma steps over bf16 s U (from the pre-pass) and the tile's B rows,
@@ -68,6 +72,8 @@ struct LvCfg {
     static constexpr int kRing = NBUF * kMaxRanks * NT8 * 512;        // [buf][rank][n][lane] float4
     static constexpr int kSu = 16 * kLvSuLd * 2;                      // bf16 s U [16][kLvSuLd]
     static constexpr int kSb = NBUF * 16 * kLvSuLd * 2;               // bf16 B rows [NBUF][16][kLvSuLd]
+    static constexpr bool kSmemScales = NT8 == 1;                    // scales through the copy ring
+    static constexpr int kScl = kSmemScales ? kLvWarps * S * 32 * 4 : 0;   // [warp][stage] absmax words, c2
     // The table sits on the first 64 KB boundary of the shared window above the buffers placed
     // below it (at most 62 KB of them: the window starts within the first KB); the others follow
     // it.  Up to 8 tokens the tile partials live in the unused upper halves of the table entries
@@ -75,7 +81,7 @@ struct LvCfg {
     // 9..16 tokens the code slices go below the table and the partials after it.
     static constexpr bool kPartInTable = NT8 == 1;
     static_assert(!kPartInTable || NBUF * kLvWarps * NT8 * 4 <= 256, "partials must fit in the table");
-    static constexpr int kBelow = kPartInTable ? kRing + kSu + kSb + 256 : kCodes + kSu + 256;
+    static constexpr int kBelow = kPartInTable ? kRing + kSu + kSb + kScl + 256 : kCodes + kSu + kScl + 256;
     static constexpr int kAbove = kPartInTable ? kCodes : kPart + kRing + kSb;
     static_assert(kBelow <= 62 * 1024, "buffers below the table");
     static constexpr int kSmem = 64 * 1024 + kLvTableBytes + kAbove;    // window start .. end
@@ -116,6 +122,12 @@ __device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
 }
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes)
+                 : "memory");
+}
+// 4-byte copy (src_bytes 0: zero fill), through L1
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst),
                  "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes)
                  : "memory");
 }
@@ -178,8 +190,9 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
     __nv_bfloat16* s_us = reinterpret_cast<__nv_bfloat16*>(Cf::kPartInTable ? below + Cf::kRing : below + Cf::kCodes);
     __nv_bfloat16* s_b = reinterpret_cast<__nv_bfloat16*>(Cf::kPartInTable ? below + Cf::kRing + Cf::kSu
                                                                             : above + Cf::kPart + Cf::kRing);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(Cf::kPartInTable ? below + Cf::kRing + Cf::kSu + Cf::kSb
-                                                                   : below + Cf::kCodes + Cf::kSu);
+    uint32_t* scl = reinterpret_cast<uint32_t*>(Cf::kPartInTable ? below + Cf::kRing + Cf::kSu + Cf::kSb
+                                                                  : below + Cf::kCodes + Cf::kSu);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scl) + Cf::kScl);
     // the float4 of lane ln for (buffer, warp, n) of the tile partials
     auto part_at = [&](int buf, int w, int n, int ln) -> float4* {
         const int idx = (buf * kLvWarps + w) * NT8 + n;
@@ -226,8 +239,24 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
     const uint32_t slices = smem_u32(codes_sm) + warp * S * Cf::kSlice;
     auto swz = [](int row) { return KB == 4 ? (row & 7) : ((row >> 1) & 3); };
     const uint8_t* const w0 = a.codes + static_cast<int64_t>(t_lo) * 16 * row_bytes + kb0 * 32;
+    // the slice's block scales: lane l < 16 copies the absmax word of row l (the aligned 4 bytes
+    // holding its KB bytes), lane 16 + l the second-level constant of row l (KB blocks never
+    // straddle a group of 256 blocks: kt and kb0 are multiples of KB)
+    const uint32_t scl_w = smem_u32(scl) + warp * S * 128;
+    const int rr = lane & 15;
+    const int64_t i_row = static_cast<int64_t>(t_lo * 16 + rr) * a.kt + kb0;   // absmax index, tile 0
+    const uint8_t* const q_src0 = a.absmax_q + (i_row & ~static_cast<int64_t>(3));
+    const int64_t tile_q = 16 * static_cast<int64_t>(a.kt);                 // absmax bytes per tile
     auto issue_slice = [&](int li) {
         if (k_ok && li < ntl) {
+            if constexpr (Cf::kSmemScales) {
+                const bool ok = (t_lo + li) * 16 + rr < a.d_out;
+                const int64_t iq = static_cast<int64_t>(li) * tile_q;
+                const void* src = lane < 16 ? static_cast<const void*>(q_src0 + iq)
+                                            : static_cast<const void*>(a.c2 + ((i_row + iq) >> 8));
+                cp_async4(scl_w + ((li % S) * 32 + lane) * 4, ok ? src : static_cast<const void*>(a.c2),
+                          ok ? 4u : 0u);
+            }
             const uint32_t dst = slices + (li % S) * Cf::kSlice;
             constexpr int kChunks = 16 * 2 * KB;            // 16-byte chunks of a slice
 #pragma unroll
@@ -242,7 +271,9 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
         }
         cp_async_commit();
     };
-    // the tile's absmax bytes of rows g, g + 8 and each row's second-level constant (a warp's
+    // the absmax word of a row holds its KB bytes at this shift (KB = 2: kb0 may be 2 mod 4)
+    const int q_shift = (kb0 & 3) * 8;
+    // (9..16 tokens) the tile's absmax bytes of rows g, g + 8 and each row's second-level constant (a warp's
     // KB blocks never straddle a group of 256 blocks: kt and kb0 are multiples of KB)
     struct Scales {
         uint32_t qa, qb;
@@ -264,7 +295,9 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
         R.c2b = vb ? __ldg(a.c2 + (ib >> 8)) : 0.f;
     };
 
+
     Scales sc_cur;
+    if constexpr (Cf::kSmemScales) sc_cur = Scales{};
     uint32_t xw[KB][NT8][8];
     if (compute) {
         for (int st = 0; st < S - 1; ++st) issue_slice(st);
@@ -276,7 +309,7 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
             for (int j = 0; j < 16; ++j)
                 table[(16 * j + warp) * 64 + lane] = lo | (a.lv16[j >> 1] >> (16 * (j & 1)) << 16);
         }
-        load_scales(0, sc_cur);
+        if constexpr (!Cf::kSmemScales) load_scales(0, sc_cur);
         // X fragments of this warp's blocks, held for the whole kernel: token 8n + g, elements
         // 16q .. 16q + 15 of block kb0 + b
 #pragma unroll
@@ -305,11 +338,21 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
         // table address of byte i of a code word: bits 16+ and the lane's word from lb, the byte as
         // bits 8..15 (entry stride 256 bytes)
         auto tab = [&](uint32_t w, uint32_t i) -> uint32_t { return prmt(w, lb, 0x7604u | (i << 4)); };
-        // the warp's part of tile li (its slice in stage li % S, its scales in R); false on a
-        // failed wait
+        // the warp's part of tile li (its slice in stage li % S; its scales there too, or in R);
+        // false on a failed wait
         auto process = [&](int li, const Scales& R) -> bool {
             const int buf = li % NBUF;
-            const uint32_t slc = slices + (li % S) * Cf::kSlice;
+            const int st = li % S;
+            const uint32_t slc = slices + st * Cf::kSlice;
+            uint32_t qa_w = R.qa, qb_w = R.qb;
+            float c2a = R.c2a, c2b = R.c2b;
+            if constexpr (Cf::kSmemScales) {
+                // (a warp past its rank's K range copies no scales: it contributes zeros)
+                qa_w = k_ok ? lds_u32(scl_w + (st * 32 + g) * 4) >> q_shift : 0u;
+                qb_w = k_ok ? lds_u32(scl_w + (st * 32 + g + 8) * 4) >> q_shift : 0u;
+                c2a = k_ok ? __uint_as_float(lds_u32(scl_w + (st * 32 + 16 + g) * 4)) : 0.f;
+                c2b = k_ok ? __uint_as_float(lds_u32(scl_w + (st * 32 + 24 + g) * 4)) : 0.f;
+            }
             float acc[NT8][4];
 #pragma unroll
             for (int n = 0; n < NT8; ++n)
@@ -341,8 +384,8 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
                         mma_bf16_16816(tmp[n], A, xw[b][n][2 * s], xw[b][n][2 * s + 1], s > 0);
                 }
                 // the unscaled block partial times the block's absmax byte; c2 multiplies the sum
-                const float qa = static_cast<float>((R.qa >> (8 * b)) & 0xFFu);
-                const float qb = static_cast<float>((R.qb >> (8 * b)) & 0xFFu);
+                const float qa = static_cast<float>((qa_w >> (8 * b)) & 0xFFu);
+                const float qb = static_cast<float>((qb_w >> (8 * b)) & 0xFFu);
 #pragma unroll
                 for (int n = 0; n < NT8; ++n) {
                     acc[n][0] = fmaf(qa, tmp[n][0], acc[n][0]);
@@ -361,27 +404,38 @@ __global__ void __maxnreg__(96) k_qgemv_lut(const __grid_constant__ LvArgs a) {
 #pragma unroll
             for (int n = 0; n < NT8; ++n)
                 *part_at(buf, warp, n, lane) =
-                    make_float4(R.c2a * acc[n][0], R.c2a * acc[n][1], R.c2b * acc[n][2], R.c2b * acc[n][3]);
+                    make_float4(c2a * acc[n][0], c2a * acc[n][1], c2b * acc[n][2], c2b * acc[n][3]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[buf]);
             return !*abort;
         };
         // per tile: refill the stage of the previous tile with the slice S - 1 ahead, wait for this
-        // tile's slice (the warp's own copies), then compute; scales ping-pong one tile ahead
-        Scales sc_nxt;
-        for (int li = 0; li < ntl; li += 2) {
-            __syncwarp();
-            issue_slice(li + S - 1);
-            load_scales(li + 1, sc_nxt);
-            cp_async_wait<S - 1>();
-            __syncwarp();
-            if (!process(li, sc_cur) || li + 1 >= ntl) break;
-            __syncwarp();
-            issue_slice(li + S);
-            load_scales(li + 2, sc_cur);
-            cp_async_wait<S - 1>();
-            __syncwarp();
-            if (!process(li + 1, sc_nxt)) break;
+        // tile's slice (and scales: the warp's own copies), then compute
+        if constexpr (Cf::kSmemScales) {
+            for (int li = 0; li < ntl; ++li) {
+                __syncwarp();
+                issue_slice(li + S - 1);
+                cp_async_wait<S - 1>();
+                __syncwarp();
+                if (!process(li, sc_cur)) break;
+            }
+        } else {
+            // scales ping-pong one tile ahead in registers
+            Scales sc_nxt;
+            for (int li = 0; li < ntl; li += 2) {
+                __syncwarp();
+                issue_slice(li + S - 1);
+                load_scales(li + 1, sc_nxt);
+                cp_async_wait<S - 1>();
+                __syncwarp();
+                if (!process(li, sc_cur) || li + 1 >= ntl) break;
+                __syncwarp();
+                issue_slice(li + S);
+                load_scales(li + 2, sc_cur);
+                cp_async_wait<S - 1>();
+                __syncwarp();
+                if (!process(li + 1, sc_nxt)) break;
+            }
         }
         cp_async_wait<0>();     // no copy in flight into the shared memory of an exiting CTA
     } else {
