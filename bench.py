@@ -810,11 +810,13 @@ def extra_rows(q, torch, S, dev, peaks, args):
     def dora_row():
         c2d = S.CONFIGS["q_proj_4096x4096_r16_T4096"]
         d, k, r, al, T = c2d["d_out"], c2d["d_in"], c2d["r"], c2d["alpha"], c2d["T"]
-        case = S.make_layer(d, k, r, al, T, dtype="bf16", seed=17, with_grad=False)
+        case = S.make_layer(d, k, r, al, T, dtype="bf16", seed=17, with_grad=True)
         wl = [q.nf4_quantize(torch.from_numpy(case.W0).to(dev)) for _ in range(4)]
         X = torch.from_numpy(case.X).to(dev).to(bf)
+        dH = torch.from_numpy(case.dH).to(dev).to(bf)
         A = torch.from_numpy(case.A).to(dev).to(bf)
         B = torch.from_numpy(case.B).to(dev).to(bf)
+        del case
         mag = torch.ones(d, dtype=torch.float32, device=dev)
         H = torch.empty((T, d), dtype=bf, device=dev)
         ws = torch.empty(q.workspace_bytes(q.OP_DORA_FWD, q.BF16, T, d, k, r), dtype=torch.uint8, device=dev)
@@ -822,9 +824,39 @@ def extra_rows(q, torch, S, dev, peaks, args):
         med, mn = _graph_time(torch, calls, reps=10)
         fl = flops_fwd(T, d, k, r) + 2 * d * r * k
         tr = t_roof(fl, bytes_fwd(T, d, k, r), peaks)
-        out["dora_fwd_4096x4096_r16_T4096"] = {"fwd_us": med, "fwd_us_min": mn,
-                                               "tflops": fl / (med * 1e-6) / 1e12, "t_roof_us": tr * 1e6,
-                                               "roof_frac": tr / (med * 1e-6)}
+        row = {"fwd_us": med, "fwd_us_min": mn, "tflops": fl / (med * 1e-6) / 1e12, "t_roof_us": tr * 1e6,
+               "roof_frac": tr / (med * 1e-6)}
+        # the backward (exact chain rule through the row norm): algorithmic work = the LoRA
+        # backward + the norms (2dkr) + the norm's two weight products A W^T and (B^T e) W^
+        # (4dkr); the call also recomputes the pre-scale output Z (not counted)
+        del H, ws
+        dX = torch.empty((T, k), dtype=bf, device=dev)
+        dA = torch.empty((r, k), dtype=torch.float32, device=dev)
+        dB = torch.empty((d, r), dtype=torch.float32, device=dev)
+        dm = torch.empty((d,), dtype=torch.float32, device=dev)
+        wsb = torch.empty(q.workspace_bytes(q.OP_DORA_BWD, q.BF16, T, d, k, r), dtype=torch.uint8, device=dev)
+        bcalls = [(lambda w=w: q.qlora_dora_bwd(w, X, dH, A, B, al, mag, dX=dX, dA=dA, dB=dB, dm=dm, ws=wsb))
+                  for w in wl]
+        # eager launches between CUDA events (this call is not captured into a graph here)
+        for c_ in bcalls:
+            c_()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(3):
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0.record()
+            for c_ in bcalls:
+                c_()
+            b1.record()
+            torch.cuda.synchronize()
+            times.append(b0.elapsed_time(b1) * 1e3 / len(bcalls))
+        bmed, bmn = sorted(times)[1], min(times)
+        bfl = flops_bwd(T, d, k, r) + 6 * d * k * r
+        btr = t_roof(bfl, bytes_bwd(T, d, k, r), peaks)
+        row.update({"bwd_us": bmed, "bwd_us_min": bmn, "bwd_tflops": bfl / (bmed * 1e-6) / 1e12,
+                    "t_roof_bwd_us": btr * 1e6, "bwd_roof_frac": btr / (bmed * 1e-6),
+                    "device_error": q.get_device_error()})
+        out["dora_4096x4096_r16_T4096"] = row
 
     # ---- FP8 forward and backward on the q_proj shape (4096^2, r = 16, T = 4096): E4M3
     # activation, E5M2 gradient, the weight decoded to E4M3 for kind::f8f6f4 tensor cores, the

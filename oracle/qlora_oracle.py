@@ -57,8 +57,9 @@ What it computes, and where each step is defined:
   Foundations page, section "Gradient Dynamics and Backpropagation Mechanics";
   reading R26.
 
-Where the pages are silent or garbled the oracle takes the readings listed as
-R1..R19 in the design notes; each is named where it is applied.
+Where the pages are silent or garbled the oracle takes a reading (numbered R1,
+R2, ...); each is cited by its number, with the choice it makes, where it is
+applied.
 
 Parity unpinned: the absolute NF4 code values and the double-quantization
 rounding order are conventions (R1, R5, R8, R10, R11) -- no page prints a

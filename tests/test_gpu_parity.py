@@ -939,3 +939,51 @@ def test_fp8_backward_rejects_unaligned_gradient_rows(q):
     with pytest.raises(q.QloraError) as e:
         q.qlora_linear_bwd_fp8(w, X8, one, G8, one, one, dev(case.A, "bf16"), dev(case.B, "bf16"), 16.0)
     assert e.value.code == 2
+
+
+# ------------------------------------------------------------------ row-sharded (tensor-parallel) layer
+
+
+@pytest.mark.parametrize("d_out,d_in,r,T", [(600, 512, 16, 300), (600, 512, 16, 5), (1000, 1024, 8, 40)])
+def test_row_shards_through_the_library(q, d_out, d_in, r, T):
+    """Two row shards of W0 and B (the tensor-parallel split of tp.row_shard), each run through the
+    library's own forward and backward on this GPU, combined as the ranks' exchanges would (H
+    columns gathered, dX and dA partials summed, dB rows kept): equal to the unsharded layer
+    within bf16 rounding, and each shard's quantization is the same rows of the whole one."""
+    import torch
+    from qlora_parameter_efficient_b200 import tp
+    case = S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_out + r)
+    W0 = dev(case.W0)
+    X, A, B, dH = dev(case.X, "bf16"), dev(case.A, "bf16"), dev(case.B, "bf16"), dev(case.dH, "bf16")
+    full = q.nf4_quantize(W0)
+    H_f, U_f = q.qlora_linear_fwd(full, X, A, B, case.alpha)
+    dX_f, dA_f, dB_f = q.qlora_linear_bwd(full, X, dH, A, B, case.alpha, U_saved=U_f)
+    world = 2
+    Hs, dBs = [], []
+    dX = torch.zeros((T, d_in), dtype=torch.float32, device="cuda")
+    dA = torch.zeros((r, d_in), dtype=torch.float32, device="cuda")
+    bpr = d_in // 64
+    for p in range(world):
+        b, e = tp.row_shard(d_out, d_in, world, p)
+        w = q.nf4_quantize(W0[b:e].contiguous())
+        assert torch.equal(w.codes.reshape(-1), full.codes.reshape(-1)[b * d_in // 2:e * d_in // 2])
+        assert torch.equal(w.absmax_q, full.absmax_q[b * bpr:e * bpr])
+        assert torch.equal(w.c2, full.c2[b * bpr // 256:b * bpr // 256 + w.c2.numel()])
+        Bp = B[b:e].contiguous()
+        H_p, U_p = q.qlora_linear_fwd(w, X, A, Bp, case.alpha)
+        dX_p, dA_p, dB_p = q.qlora_linear_bwd(w, X, dH[:, b:e].contiguous(), A, Bp, case.alpha, U_saved=U_p)
+        Hs.append(H_p)
+        dX += dX_p.float()
+        dA += dA_p
+        dBs.append(dB_p)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    H = torch.cat(Hs, dim=1)
+    dB = torch.cat(dBs, dim=0)
+    assert rel_fro(host(H), host(H_f)) <= 5e-3
+    assert rel_fro(host(dX), host(dX_f)) <= 5e-3
+    assert rel_fro(host(dA), host(dA_f)) <= 5e-3
+    assert rel_fro(host(dB), host(dB_f)) <= 5e-3
+    Wh = O.nf4_dequantize(*O.nf4_quantize(case.W0)[:3], d_out, d_in, out="bf16").astype(np.float64)
+    Href = O.lora_forward(Wh, case.X, case.A, case.B, case.alpha, r)
+    assert rel_fro(host(H), Href) <= TOL["bf16"]
