@@ -854,7 +854,31 @@ def extra_rows(q, torch, S, dev, peaks, args):
         bfl = flops_bwd(T, d, k, r) + 6 * d * k * r
         btr = t_roof(bfl, bytes_bwd(T, d, k, r), peaks)
         row.update({"bwd_us": bmed, "bwd_us_min": bmn, "bwd_tflops": bfl / (bmed * 1e-6) / 1e12,
-                    "t_roof_bwd_us": btr * 1e6, "bwd_roof_frac": btr / (bmed * 1e-6),
+                    "t_roof_bwd_us": btr * 1e6, "bwd_roof_frac": btr / (bmed * 1e-6)})
+        # training form: the forward keeps Z, U and the norms (qlora_dora_fwd_save) and the backward
+        # reuses them; one weight's saved tensors serve every timed call (the same arithmetic)
+        H2 = torch.empty((T, d), dtype=bf, device=dev)
+        wsf = torch.empty(q.workspace_bytes(q.OP_DORA_FWD, q.BF16, T, d, k, r), dtype=torch.uint8, device=dev)
+        fcalls = [(lambda w=w: q.qlora_dora_fwd_save(w, X, A, B, al, mag, H=H2, ws=wsf)) for w in wl]
+        fmed, _ = _graph_time(torch, fcalls, reps=10)
+        _, saved = q.qlora_dora_fwd_save(wl[0], X, A, B, al, mag, H=H2, ws=wsf)
+        del wsf
+        scalls = [(lambda w=w: q.qlora_dora_bwd(w, X, dH, A, B, al, mag, dX=dX, dA=dA, dB=dB, dm=dm, ws=wsb,
+                                                saved=saved)) for w in wl]
+        for c_ in scalls:
+            c_()
+        torch.cuda.synchronize()
+        stimes = []
+        for _ in range(3):
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0.record()
+            for c_ in scalls:
+                c_()
+            b1.record()
+            torch.cuda.synchronize()
+            stimes.append(b0.elapsed_time(b1) * 1e3 / len(scalls))
+        smed = sorted(stimes)[1]
+        row.update({"fwd_save_us": fmed, "bwd_saved_us": smed, "bwd_saved_roof_frac": btr / (smed * 1e-6),
                     "device_error": q.get_device_error()})
         out["dora_4096x4096_r16_T4096"] = row
 

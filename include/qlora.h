@@ -266,6 +266,29 @@ qlora_status qlora_dora_bwd(const qlora_nf4* w, const void* X, const void* dH, i
                             const float* magnitude, void* dX, float* dA, float* dB, float* dm,
                             void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* DoRA forward for training: the layer of qlora_dora_fwd that also keeps what its backward needs,
+ * so that qlora_dora_bwd_saved does not recompute it.  It writes the row norms n (norms_save,
+ * device fp32 [d_out]), the pre-scale output Z = X W^T + s U B^T (Z_save, bf16 [T, d_out], from
+ * the large-T kernels whatever T), U (U_save, bf16 [T, r], required) and
+ * H[t, j] = bf16(Z[t, j] (m_j / n_j)) (0 where n_j = 0) -- Z rounded to bf16 before the scale,
+ * where qlora_dora_fwd scales the fp32 accumulator (one bf16 rounding more: a relative 2^-9).
+ * Same sources, readings and ws size as qlora_dora_fwd.                                        */
+qlora_status qlora_dora_fwd_save(const qlora_nf4* w, const void* X, int64_t T, const void* A,
+                                 const void* B, int32_t r, float alpha, const float* magnitude,
+                                 void* H, void* Z_save, void* U_save, float* norms_save, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream);
+
+/* qlora_dora_bwd from the Z, U and norms that qlora_dora_fwd_save wrote for the same w, X, A, B,
+ * alpha (the caller keeps them unchanged in between): the same results as qlora_dora_bwd bit
+ * for bit (which recomputes exactly these three), without the norm pass and the forward.
+ * Z_saved bf16 [T, d_out], U_saved bf16 [T, r], norms_saved fp32 [d_out]; the rest as in
+ * qlora_dora_bwd, the same ws size.                                                           */
+qlora_status qlora_dora_bwd_saved(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                                  const void* A, const void* B, int32_t r, float alpha,
+                                  const float* magnitude, const void* Z_saved, const void* U_saved,
+                                  const float* norms_saved, void* dX, float* dA, float* dB, float* dm,
+                                  void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* The DoRA row norms n_j = ||(W^ + (alpha/r) B A)[j, :]||_2 (bf16 adapters, W^ the bf16 decode)
  * into norms (device fp32 [d_out]); DoRA initialises the magnitude to them.  ws holds at least
  * d_out * (d_in / 64) floats.                                                                 */

@@ -9,7 +9,8 @@ Names follow the C ABI: ``nf4_quantize``, ``nf4_dequantize``,
 ``qlora_linear_fwd``, ``qlora_linear_bwd`` (``accumulate=`` for gradient
 accumulation), ``lora_merge``, ``qlora_linear_fwd_batched`` (a few adapters),
 ``qlora_linear_fwd_multi`` with an ``AdapterTable`` (thousands of mixed-rank
-adapters), ``qlora_dora_fwd`` / ``dora_row_norms``, ``adamw_step`` /
+adapters), ``qlora_dora_fwd`` / ``qlora_dora_bwd`` / ``dora_row_norms`` (and
+``qlora_dora_fwd_save`` whose saved tensors ``qlora_dora_bwd(saved=...)`` reuses), ``adamw_step`` /
 ``prefetch`` (optimizer step, unified-memory state), and the FP8 path:
 ``fp8_quantize`` (E4M3 activation), ``fp8_quantize_grad`` (E5M2 gradient),
 ``fp8_weight_scale``, ``qlora_linear_fwd_fp8``, ``qlora_linear_bwd_fp8``.
@@ -36,7 +37,7 @@ OP_FWD_FP8, OP_FP8_QUANT, OP_BWD_FP8, OP_DORA_BWD = 6, 7, 8, 9
 EXPORTS = ["qlora_nf4_sizes", "qlora_nf4_levels", "nf4_quantize", "nf4_dequantize",
            "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "lora_merge",
            "qlora_linear_bwd_ex", "qlora_adamw_step", "qlora_prefetch", "qlora_dora_fwd",
-           "qlora_dora_bwd", "qlora_dora_row_norms", "qlora_fp8_quantize", "qlora_fp8_weight_scale",
+           "qlora_dora_bwd", "qlora_dora_fwd_save", "qlora_dora_bwd_saved", "qlora_dora_row_norms", "qlora_fp8_quantize", "qlora_fp8_weight_scale",
            "qlora_linear_fwd_fp8", "qlora_fp8_quantize_grad", "qlora_linear_bwd_fp8",
            "qlora_linear_fwd_batched", "qlora_linear_fwd_multi", "qlora_linear_fwd_noalloc",
            "qlora_get_device_error",
@@ -91,6 +92,9 @@ def load() -> ctypes.CDLL:
         "qlora_dora_fwd": ([pnf4, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "qlora_dora_row_norms": ([pnf4, vp, vp, i32, f32, vp, vp, sz, vp], ctypes.c_int),
         "qlora_dora_bwd": ([pnf4, vp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_dora_fwd_save": ([pnf4, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_dora_bwd_saved": ([pnf4, vp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+                                 ctypes.c_int),
         "qlora_fp8_quantize": ([vp, i64, vp, vp, vp, sz, vp], ctypes.c_int),
         "qlora_fp8_weight_scale": ([pnf4, vp, vp], ctypes.c_int),
         "qlora_linear_fwd_fp8": ([pnf4, vp, i64, vp, vp, vp, vp, i32, f32, vp, vp, sz, vp], ctypes.c_int),
@@ -318,11 +322,39 @@ def qlora_dora_fwd(w: NF4Weight, X, A, B, alpha, magnitude, H=None, U_save=None,
     return H, U_save
 
 
+def qlora_dora_fwd_save(w: NF4Weight, X, A, B, alpha, magnitude, H=None, Z=None, U=None, norms=None,
+                        ws=None, stream=None):
+    """DoRA forward that keeps what the backward needs: returns (H, saved) with saved = (Z, U,
+    norms), the pre-scale output, U and the row norms, for qlora_dora_bwd(..., saved=saved)."""
+    torch = _torch()
+    _contig(X, A, B, magnitude, H, Z, U, norms)
+    T = X.shape[0]
+    r = A.shape[0]
+    dev = X.device
+    if H is None:
+        H = torch.empty((T, w.d_out), dtype=X.dtype, device=dev)
+    if Z is None:
+        Z = torch.empty((T, w.d_out), dtype=X.dtype, device=dev)
+    if U is None:
+        U = torch.empty((T, r), dtype=X.dtype, device=dev)
+    if norms is None:
+        norms = torch.empty((w.d_out,), dtype=torch.float32, device=dev)
+    ws = _ws(OP_DORA_FWD, BF16, T, w.d_out, w.d_in, r, dev, ws)
+    c = w._c()
+    _check("qlora_dora_fwd_save", load().qlora_dora_fwd_save(
+        ctypes.byref(c), _ptr(X), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(magnitude), _ptr(H),
+        _ptr(Z), _ptr(U), _ptr(norms), _ptr(ws), ws.numel(), _stream(stream)))
+    return H, (Z, U, norms)
+
+
 def qlora_dora_bwd(w: NF4Weight, X, dH, A, B, alpha, magnitude, dX=None, dA=None, dB=None, dm=None,
-                   want_dx=True, ws=None, stream=None):
-    """DoRA backward (bf16), the chain rule through the row norm: returns (dX, dA, dB, dm)."""
+                   want_dx=True, ws=None, stream=None, saved=None):
+    """DoRA backward (bf16), the chain rule through the row norm: returns (dX, dA, dB, dm).
+    saved: the (Z, U, norms) of qlora_dora_fwd_save for the same operands (else recomputed)."""
     torch = _torch()
     _contig(X, dH, A, B, magnitude, dX, dA, dB, dm)
+    if saved is not None:
+        _contig(*saved)
     T = X.shape[0]
     r = A.shape[0]
     dev = X.device
@@ -336,9 +368,16 @@ def qlora_dora_bwd(w: NF4Weight, X, dH, A, B, alpha, magnitude, dX=None, dA=None
         dm = torch.empty((w.d_out,), dtype=torch.float32, device=dev)
     ws = _ws(OP_DORA_BWD, BF16, T, w.d_out, w.d_in, r, dev, ws)
     c = w._c()
-    _check("qlora_dora_bwd", load().qlora_dora_bwd(
-        ctypes.byref(c), _ptr(X), _ptr(dH), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(magnitude),
-        _ptr(dX), _ptr(dA), _ptr(dB), _ptr(dm), _ptr(ws), ws.numel(), _stream(stream)))
+    if saved is None:
+        _check("qlora_dora_bwd", load().qlora_dora_bwd(
+            ctypes.byref(c), _ptr(X), _ptr(dH), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(magnitude),
+            _ptr(dX), _ptr(dA), _ptr(dB), _ptr(dm), _ptr(ws), ws.numel(), _stream(stream)))
+    else:
+        Z, U, norms = saved
+        _check("qlora_dora_bwd_saved", load().qlora_dora_bwd_saved(
+            ctypes.byref(c), _ptr(X), _ptr(dH), T, _ptr(A), _ptr(B), r, float(alpha), _ptr(magnitude),
+            _ptr(Z), _ptr(U), _ptr(norms), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(dm), _ptr(ws), ws.numel(),
+            _stream(stream)))
     return dX, dA, dB, dm
 
 

@@ -146,4 +146,38 @@ __global__ void k_dora_add_da(const __nv_bfloat16* __restrict__ Q, const __nv_bf
     }
 }
 
+// H[t, j] = bf16(Z[t, j] c_j), c_j = m_j / n_j (0 where n_j = 0): the DoRA output from the saved
+// pre-scale output.  Eight elements per thread when rows are whole 16-byte units, else one.
+__global__ void k_dora_apply(const __nv_bfloat16* __restrict__ Z, const float* __restrict__ magnitude,
+                             const float* __restrict__ norms, int64_t T, int64_t d,
+                             __nv_bfloat16* __restrict__ H) {
+    griddep_enter();
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    auto coef = [&](int64_t j) {
+        const float n = norms[j];
+        return n > 0.f ? magnitude[j] / n : 0.f;
+    };
+    if ((d & 7) == 0) {
+        const int64_t n8 = T * d / 8;
+        for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
+            const int64_t j0 = (i * 8) % d;
+            const uint4 z = reinterpret_cast<const uint4*>(Z)[i];
+            const uint32_t zw[4] = {z.x, z.y, z.z, z.w};
+            uint32_t hw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 v;
+                *reinterpret_cast<uint32_t*>(&v) = zw[e];
+                const float2 f = __bfloat1622float2(v);
+                const __nv_bfloat162 h = __floats2bfloat162_rn(f.x * coef(j0 + 2 * e), f.y * coef(j0 + 2 * e + 1));
+                hw[e] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            reinterpret_cast<uint4*>(H)[i] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        }
+    } else {
+        for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < T * d; i += stride)
+            H[i] = __float2bfloat16_rn(__bfloat162float(Z[i]) * coef(i % d));
+    }
+}
+
 }  // namespace qlora

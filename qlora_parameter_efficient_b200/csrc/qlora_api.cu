@@ -1137,13 +1137,44 @@ qlora_status qlora_dora_fwd(const qlora_nf4* w, const void* X, int64_t T, const 
     return fwd_bf16_large(w, X, T, A, B, r, s, H, U_save, p, ws, err, stream, scale);
 }
 
-qlora_status qlora_dora_bwd(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
-                            const void* A, const void* B, int32_t r, float alpha,
-                            const float* magnitude, void* dX, float* dA, float* dB, float* dm,
-                            void* ws, size_t ws_bytes, cudaStream_t stream) {
+qlora_status qlora_dora_fwd_save(const qlora_nf4* w, const void* X, int64_t T, const void* A,
+                                 const void* B, int32_t r, float alpha, const float* magnitude,
+                                 void* H, void* Z_save, void* U_save, float* norms_save, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream) {
+    QL_TRY(check_layer(w, T, r, QLORA_BF16));
+    if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(H) || !magnitude ||
+        !aligned16(Z_save) || !aligned16(U_save) || !norms_save)
+        return QLORA_ERR_INVALID_ARG;
+    const Plan p = make_plan(QLORA_OP_DORA_FWD, QLORA_BF16, T, w->d_out, w->d_in, r);
+    QL_TRY(check_ws(ws, ws_bytes, p.total));
+    int* err = nullptr;
+    QL_TRY(err_word(&err, stream));
+    const float s = alpha / static_cast<float>(r);
+    // n (the merge tile's row-norm mode), Z and U (the plain large-T forward), then H = Z c
+    QL_TRY(dora_scale(w, A, B, r, s, nullptr, at<float>(ws, p.dora_part), norms_save, stream));
+    QL_TRY(fwd_bf16_large(w, X, T, A, B, r, s, Z_save, U_save, p, ws, err, stream, nullptr));
+    const int64_t n = (w->d_out % 8 == 0) ? T * w->d_out / 8 : T * w->d_out;
+    if (launch_pdl(k_dora_apply, grid1d(n), dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(Z_save),
+                   magnitude, static_cast<const float*>(norms_save), T, w->d_out,
+                   static_cast<__nv_bfloat16*>(H)) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    QL_LAUNCH_CHECK();
+    return QLORA_OK;
+}
+
+// The DoRA backward; Zs, Us, ns: the pre-scale output, U and the row norms saved by the forward,
+// or all null (recomputed here).
+qlora_status dora_bwd_impl(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                           const void* A, const void* B, int32_t r, float alpha,
+                           const float* magnitude, const void* Zs, const void* Us, const float* ns,
+                           void* dX, float* dA, float* dB, float* dm, void* ws, size_t ws_bytes,
+                           cudaStream_t stream) {
     QL_TRY(check_layer(w, T, r, QLORA_BF16));
     if (!aligned16(X) || !aligned16(dH) || !aligned16(A) || !aligned16(B) || !magnitude ||
         !aligned16(dA) || !aligned16(dB) || !dm || !aligned16_or_null(dX))
+        return QLORA_ERR_INVALID_ARG;
+    const bool saved = Zs != nullptr;
+    if (saved ? (!aligned16(Zs) || !aligned16(Us) || !ns) : (Us != nullptr || ns != nullptr))
         return QLORA_ERR_INVALID_ARG;
     const int64_t d = w->d_out, k = w->d_in;
     const DoraBwdLayout L = dora_bwd_layout(T, d, k, r);
@@ -1153,21 +1184,25 @@ qlora_status qlora_dora_bwd(const qlora_nf4* w, const void* X, const void* dH, i
     using bf = __nv_bfloat16;
     const float s = alpha / static_cast<float>(r);
     void* shared = at<void>(ws, L.shared);
-    float* norms = at<float>(ws, L.norms);
+    const float* norms = saved ? ns : at<float>(ws, L.norms);
     float* e = at<float>(ws, L.e);
     float* colpart = at<float>(ws, L.colpart);
-    bf* Z = at<bf>(ws, L.z);
-    bf* U = at<bf>(ws, L.u);
+    const bf* Z = saved ? static_cast<const bf*>(Zs) : at<bf>(ws, L.z);
+    const bf* U = saved ? static_cast<const bf*>(Us) : at<bf>(ws, L.u);
     bf* dZ = at<bf>(ws, L.dz);
     bf* ge = at<bf>(ws, L.ge);
     bf* pm = at<bf>(ws, L.pm);
     bf* qm = at<bf>(ws, L.qm);
     float* aat = at<float>(ws, L.aat);
     float* beb = at<float>(ws, L.beb);
-    // n_j = ||(W^ + s B A)[j, :]|| and the pre-scale output Z = X V^T (with U for the backward)
-    QL_TRY(dora_scale(w, A, B, r, s, nullptr, at<float>(ws, L.merge_part), norms, stream));
-    const Plan pf = make_plan(QLORA_OP_DORA_FWD, QLORA_BF16, T, d, k, r);
-    QL_TRY(fwd_bf16_large(w, X, T, A, B, r, s, Z, U, pf, shared, err, stream, nullptr));
+    // n_j = ||(W^ + s B A)[j, :]|| and the pre-scale output Z = X V^T (with U for the backward),
+    // unless the forward saved them
+    if (!saved) {
+        QL_TRY(dora_scale(w, A, B, r, s, nullptr, at<float>(ws, L.merge_part), at<float>(ws, L.norms), stream));
+        const Plan pf = make_plan(QLORA_OP_DORA_FWD, QLORA_BF16, T, d, k, r);
+        QL_TRY(fwd_bf16_large(w, X, T, A, B, r, s, at<bf>(ws, L.z), at<bf>(ws, L.u), pf, shared, err, stream,
+                              nullptr));
+    }
     // dZ = dH diag(m / n), dc_j = sum_t dH[t, j] Z[t, j], dm = dc / n, e = -dc m / n^3
     const dim3 cgrid(static_cast<unsigned>(cdiv(d / 2, 256)), static_cast<unsigned>(kDoraChunks));
     if (launch_pdl(k_dora_colred, cgrid, dim3(256), 0, stream, static_cast<const bf*>(dH),
@@ -1208,6 +1243,24 @@ qlora_status qlora_dora_bwd(const qlora_nf4* w, const void* X, const void* dH, i
         return QLORA_ERR_CUDA;
     QL_LAUNCH_CHECK();
     return QLORA_OK;
+}
+
+qlora_status qlora_dora_bwd(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                            const void* A, const void* B, int32_t r, float alpha,
+                            const float* magnitude, void* dX, float* dA, float* dB, float* dm,
+                            void* ws, size_t ws_bytes, cudaStream_t stream) {
+    return dora_bwd_impl(w, X, dH, T, A, B, r, alpha, magnitude, nullptr, nullptr, nullptr, dX, dA, dB,
+                         dm, ws, ws_bytes, stream);
+}
+
+qlora_status qlora_dora_bwd_saved(const qlora_nf4* w, const void* X, const void* dH, int64_t T,
+                                  const void* A, const void* B, int32_t r, float alpha,
+                                  const float* magnitude, const void* Z_saved, const void* U_saved,
+                                  const float* norms_saved, void* dX, float* dA, float* dB, float* dm,
+                                  void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!Z_saved || !U_saved || !norms_saved) return QLORA_ERR_INVALID_ARG;
+    return dora_bwd_impl(w, X, dH, T, A, B, r, alpha, magnitude, Z_saved, U_saved, norms_saved, dX, dA,
+                         dB, dm, ws, ws_bytes, stream);
 }
 
 qlora_status qlora_fp8_quantize(const void* X, int64_t n, uint8_t* X8, float* scale, void* ws,

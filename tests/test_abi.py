@@ -103,6 +103,20 @@ def test_split_backward_flags_validated_before_launch(L):
     assert bwd(0, dX=None, dA=None) == 1                       # one-call backward needs dA, dB
 
 
+def test_dora_save_entries_validate_before_launch(L):
+    nf4 = q._NF4(16, 16, 16, 64, 64)
+    # forward with saving: the norms output and Z are required
+    assert L.qlora_dora_fwd_save(ctypes.byref(nf4), 16, 8, 16, 16, 8, 16.0, 16, 16, 16, 16, None,
+                                 256, 1 << 20, None) == 1
+    assert L.qlora_dora_fwd_save(ctypes.byref(nf4), 16, 8, 16, 16, 8, 16.0, 16, 16, None, 16, 16,
+                                 256, 1 << 20, None) == 1
+    # backward from saved tensors: all three are required, and must be aligned
+    assert L.qlora_dora_bwd_saved(ctypes.byref(nf4), 16, 16, 8, 16, 16, 8, 16.0, 16, None, 16, 16,
+                                  16, 16, 16, 16, 256, 1 << 20, None) == 1
+    assert L.qlora_dora_bwd_saved(ctypes.byref(nf4), 16, 16, 8, 16, 16, 8, 16.0, 16, 17, 16, 16,
+                                  16, 16, 16, 16, 256, 1 << 20, None) == 1
+
+
 def test_fp8_host_validation_rejects_before_launch(L):
     nf4 = q._NF4(16, 16, 16, 64, 64)
     # forward: a missing scale, a misaligned E4M3 activation

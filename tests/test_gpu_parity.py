@@ -740,6 +740,40 @@ def test_dora_backward(q, d_out, d_in, r, T):
     run_dora_bwd(q, S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_out + T))
 
 
+@pytest.mark.parametrize("d_out,d_in,r,T", [(203, 320, 5, 37), (256, 512, 16, 300), (4096, 4096, 16, 512)])
+def test_dora_saved_forward_and_backward(q, d_out, d_in, r, T):
+    """qlora_dora_fwd_save keeps Z (the LoRA forward, on the large-T kernels whatever T), U and the
+    row norms (bit for bit the dora_row_norms result); its H matches the oracle and the
+    fused-epilogue forward; the backward from those saved tensors is bit-identical to the
+    backward that recomputes them."""
+    import torch
+    case = S.make_layer(d_out, d_in, r, 2.0 * r, T, dtype="bf16", seed=d_out + r + T)
+    w, oc = quantize_both(q, case.W0)
+    Wh = oracle_weight(oc, d_out, d_in, "bf16")
+    X, A, B, dH = dev(case.X, "bf16"), dev(case.A, "bf16"), dev(case.B, "bf16"), dev(case.dH, "bf16")
+    mag_np = np.random.default_rng(d_out).uniform(0.5, 2.0, d_out).astype(np.float32)
+    mag = torch.from_numpy(mag_np).cuda()
+    H1, _ = q.qlora_dora_fwd(w, X, A, B, case.alpha, mag)
+    H2, saved = q.qlora_dora_fwd_save(w, X, A, B, case.alpha, mag)
+    Z, U, norms = saved
+    Zl, Ul = q.qlora_linear_fwd(w, X, A, B, case.alpha)
+    nl = q.dora_row_norms(w, A, B, case.alpha)
+    g1 = q.qlora_dora_bwd(w, X, dH, A, B, case.alpha, mag)
+    g2 = q.qlora_dora_bwd(w, X, dH, A, B, case.alpha, mag, saved=saved)
+    torch.cuda.synchronize()
+    assert q.get_device_error() == 0
+    assert torch.equal(norms, nl)
+    # (for T <= 64 qlora_linear_fwd takes the decode-size or mid-size route: same values, other
+    # summation orders)
+    assert rel_fro(host(Z), host(Zl).astype(np.float64)) <= 4e-3
+    assert rel_fro(host(U), host(Ul).astype(np.float64)) <= 4e-3
+    assert rel_fro(host(Z), O.lora_forward(Wh, case.X, case.A, case.B, case.alpha, r)) <= TOL["bf16"]
+    assert rel_fro(host(H2), host(H1).astype(np.float64)) <= 4e-3
+    assert rel_fro(host(H2), O.dora_forward(Wh, case.X, case.A, case.B, case.alpha, r, mag_np)) <= TOL["bf16"]
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
+
+
 def test_dora_backward_q_proj_sampled_rows(q):
     case = S.make_layer(**S.CONFIGS["q_proj_4096x4096_r16_T4096"], seed=4)
     rows = np.sort(np.random.default_rng(6).choice(case.T, 256, replace=False))
