@@ -253,7 +253,8 @@ qlora_status qlora_dora_fwd(const qlora_nf4* w, const void* X, int64_t T, const 
  * the derivative of the Euclidean norm is V[j, :] / n_j):
  *   dZ = dH diag(c),  dc_j = sum_t dH[t, j] Z[t, j],  dm_j = dc_j / n_j,  e_j = -dc_j m_j / n_j^3
  *   dX = dZ V,  dA = s B^T (dZ^T X + diag(e) V),  dB = s (dZ^T X + diag(e) V) A^T
- * A row of norm 0 contributes nothing.  The library recomputes n and Z (a large-T forward), runs
+ * A row of norm 0 contributes nothing.  The library recomputes n and Z (a large-T forward;
+ * qlora_dora_bwd_saved takes them from qlora_dora_fwd_save instead), runs
  * the LoRA backward on dZ and adds the norm's term through two passes over the weight with the
  * adapter rows as tokens (A W^T and B^T diag(e) W^ on the fused NF4 GEMM) and r x r products.
  * [CH] "Choosing what to adapt: targets and rank"; [MF] "Advanced Variants: DoRA and LoRA+";
