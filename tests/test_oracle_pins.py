@@ -947,3 +947,52 @@ def test_pins_catch_planted_mistakes():
     assert check_round_trip(quantize_swapped_nibbles) > 0
     assert check_double_quant(quantize_255) > 0
     assert check_round_trip(quantize_255) > 0
+
+# ------------------------------------------------------------------ helpers of the level table and the encoder
+
+
+def test_normal_cdf_matches_library_routine():
+    """Phi against scipy's ndtr (an independent implementation of the standard normal CDF) over
+    the range the level table uses, and its exact symmetry Phi(-x) = 1 - Phi(x)."""
+    from scipy.special import ndtr
+    xs = np.linspace(-4.0, 4.0, 801)
+    got = np.array([O.normal_cdf(float(x)) for x in xs])
+    assert np.max(np.abs(got - ndtr(xs))) <= 1e-15
+    assert np.max(np.abs(got + got[::-1] - 1.0)) <= 1e-15
+    assert O.normal_cdf(0.0) == 0.5
+
+
+def test_midpoints_separate_the_levels():
+    """The 15 decision thresholds lie strictly between neighbouring levels and each is within one
+    fp32 ulp of the exact midpoint."""
+    L = O.nf4_levels()
+    m = O.nf4_midpoints(L)
+    assert m.shape == (15,) and m.dtype == np.float32
+    assert np.all(L[:-1] < m) and np.all(m < L[1:])
+    exact = (L[:-1].astype(np.float64) + L[1:].astype(np.float64)) / 2.0
+    assert np.all(np.abs(m.astype(np.float64) - exact) <= np.spacing(np.abs(m)).astype(np.float64))
+
+
+def test_codes_of_normalised_are_nearest_levels_by_brute_force():
+    """The threshold encoder against an exhaustive nearest-level search: on a dense grid of [-1, 1]
+    plus every threshold and its fp32 neighbours, the code is the index of the nearest level,
+    and a value exactly on a threshold takes the upper level (the stated tie rule)."""
+    L = O.nf4_levels()
+    m = O.nf4_midpoints(L)
+    grid = np.linspace(-1.0, 1.0, 20001, dtype=np.float32)
+    near = np.concatenate([m, np.nextafter(m, np.float32(-2)), np.nextafter(m, np.float32(2))])
+    xs = np.concatenate([grid, near]).astype(np.float32)
+    got = O.nf4_codes_of_normalised(xs, m)
+    dist = np.abs(xs[:, None].astype(np.float64) - L[None, :].astype(np.float64))
+    best = np.argmin(dist, axis=1)
+    # where the two nearest fp64 distances are too close to order (x a few ulps from a
+    # threshold), decide with exact rational arithmetic
+    from fractions import Fraction
+    srt = np.sort(dist, axis=1)
+    for i in np.nonzero(srt[:, 1] - srt[:, 0] < 1e-12)[0]:
+        x = Fraction(float(xs[i]))
+        best[i] = min(range(16), key=lambda j: (abs(x - Fraction(float(L[j]))), j))
+    off = ~np.isin(xs, m)                      # away from a threshold: the unique nearest level
+    assert np.array_equal(got[off], best[off].astype(np.uint8))
+    on = np.searchsorted(m, m)                 # exactly on threshold i: the upper level i + 1
+    assert np.array_equal(O.nf4_codes_of_normalised(m, m), (on + 1).astype(np.uint8))
