@@ -1,5 +1,6 @@
 // dora.cuh -- the DoRA backward's element-wise and small kernels (the two weight passes reuse the
-// fused NF4 GEMM with the adapter rows as tokens, the rest of the backward is the LoRA one).
+// fused NF4 GEMM with the adapter rows as tokens, the rest of the backward is the LoRA one), and
+// the scale pass of the forward that keeps the pre-scale output Z for the backward.
 //
 // DoRA with one magnitude per output row ("Large Language Model Fine-tuning and LoRA", section
 // "Choosing what to adapt: targets and rank"; "Low-Rank Adaptation (LoRA) and QLoRA:
