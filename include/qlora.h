@@ -7,7 +7,7 @@
  *     h = W0 x + (alpha/r) B (A x)
  * with W0 dequantized on the fly to bf16 inside the tensor-core GEMM, its backward pass, the
  * adapter merge, multi-adapter forwards over one shared base (a few adapters, or thousands of
- * mixed-rank adapters), DoRA's forward, the adapter optimizer step (AdamW, gradient
+ * mixed-rank adapters), DoRA's forward and backward, the adapter optimizer step (AdamW, gradient
  * accumulation, paged state), and the forward and backward with FP8 (E4M3 / E5M2) activations
  * and gradients on FP8 tensor cores.
  *
