@@ -272,7 +272,8 @@ qlora_status qlora_dora_bwd(const qlora_nf4* w, const void* X, const void* dH, i
  * device fp32 [d_out]), the pre-scale output Z = X W^T + s U B^T (Z_save, bf16 [T, d_out], from
  * the large-T kernels whatever T), U (U_save, bf16 [T, r], required) and
  * H[t, j] = bf16(Z[t, j] (m_j / n_j)) (0 where n_j = 0) -- Z rounded to bf16 before the scale,
- * where qlora_dora_fwd scales the fp32 accumulator (one bf16 rounding more: a relative 2^-9).
+ * where qlora_dora_fwd scales the fp32 accumulator (one bf16 rounding more: a relative 2^-9;
+ * reading R28).
  * Same sources, readings and ws size as qlora_dora_fwd.                                        */
 qlora_status qlora_dora_fwd_save(const qlora_nf4* w, const void* X, int64_t T, const void* A,
                                  const void* B, int32_t r, float alpha, const float* magnitude,
